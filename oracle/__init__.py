@@ -1,0 +1,132 @@
+"""CPU float64 oracle for the SSD layer scan -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / reference legs may
+import this package.  It wraps ``ssd_oracle.c`` (the token-by-token recurrence, see that file for
+the definition and its sources) through ctypes and never touches the CUDA library.
+
+Parity status: pinned.  ``tests/test_oracle_pins.py`` checks it against the explicit
+semiseparable matrix form on tiny inputs, a hand-worked example, closed forms for N = P = 1, the
+low-rank property of off-diagonal blocks, and invariances (dt = 0 padding, split/resume,
+linearity).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssd_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libssd_oracle.so")
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no fused multiply-add) if the library is missing or stale."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-std=c11", "-shared",
+                    "-fPIC", _SRC, "-o", tmp, "-lm"], check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.oracle_ssd_scan.restype = ctypes.c_int
+        lib.oracle_ssd_scan.argtypes = [_I64] * 6 + [_D] * 6 + [_D, _D, _D, _D, _I64, _I64,
+                                                                 ctypes.POINTER(_I64), _I64]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_num_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_D)
+
+
+def ssd_scan(x, dt, A, B, C, D, init=None, every: int = 0,
+             bh: Optional[Sequence[int]] = None):
+    """Token-by-token SSD recurrence in float64.
+
+    x (b, L, H, P), dt (b, L, H), A (H,), B/C (b, L, G, N), D (H,), init (b, H, P, N) or None.
+    Returns (y (b, L, H, P), final_state (b, H, P, N), boundary) where boundary holds the state
+    after every ``every``-th token, shape (b, H, L // every, P, N), or None when every == 0.
+    With ``bh`` only the listed flattened b*H + h pairs are computed (others stay zero).
+    """
+    x, dt, A, B, C, D, init = map(_f64, (x, dt, A, B, C, D, init))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    assert dt.shape == (b, L, H) and A.shape == (H,) and D.shape == (H,)
+    assert B.shape == (b, L, G, N) and C.shape == (b, L, G, N)
+    assert init is None or init.shape == (b, H, P, N)
+    y = np.zeros((b, L, H, P))
+    final = np.zeros((b, H, P, N))
+    nb = L // every if every > 0 else 0
+    boundary = np.zeros((b, H, nb, P, N)) if every > 0 else None
+    idx = None if bh is None else np.ascontiguousarray(bh, dtype=np.int64)
+    rc = _load().oracle_ssd_scan(
+        b, L, H, P, N, G, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init),
+        _ptr(y), _ptr(final), _ptr(boundary), every, nb,
+        None if idx is None else idx.ctypes.data_as(ctypes.POINTER(_I64)),
+        0 if idx is None else len(idx))
+    if rc != 0:
+        raise RuntimeError("oracle_ssd_scan rejected its arguments")
+    return y, final, boundary
+
+
+def ssd_scan_pairs(inp, pairs: Sequence[Tuple[int, int]], every: int = 0,
+                   seqlen: Optional[int] = None):
+    """Recurrence for selected (batch, head) pairs of a full-size input draw.
+
+    The selected pairs are gathered (pure re-indexing, no arithmetic) into one batch whose
+    "heads" are the pairs, each with its own group, so only those slices are widened to float64.
+    Returns y (n, L, P), final (n, P, N) and the boundary states (n, nb, P, N) or None.
+    """
+    H = inp.A.shape[0]
+    G = inp.B.shape[2]
+    L = inp.x.shape[1] if seqlen is None else seqlen
+    bs = np.array([p[0] for p in pairs], dtype=np.int64)
+    hs = np.array([p[1] for p in pairs], dtype=np.int64)
+    gs = hs // (H // G)
+    x = np.stack([inp.x[b, :L, h] for b, h in pairs], 1)
+    dt = np.stack([inp.dt[b, :L, h] for b, h in pairs], 1)
+    Bv = np.stack([inp.B[b, :L, g] for b, g in zip(bs, gs)], 1)
+    Cv = np.stack([inp.C[b, :L, g] for b, g in zip(bs, gs)], 1)
+    init = None
+    if inp.init is not None:
+        init = np.stack([inp.init[b, h] for b, h in pairs], 0)[None]
+    y, final, boundary = ssd_scan(x[None], dt[None], inp.A[hs], Bv[None], Cv[None], inp.D[hs],
+                                  init, every=every)
+    y = np.moveaxis(y[0], 1, 0)                      # (n, L, P)
+    return y, final[0], (None if boundary is None else boundary[0])
+
+
+def ssd_state_update(state, x, dt, A, B, C, D):
+    """One decode step: the recurrence over a single token, state (b, H, P, N) updated and returned.
+
+    x (b, H, P), dt (b, H), B/C (b, G, N).  Returns (y (b, H, P), new_state).
+    """
+    x = np.asarray(x)
+    y, final, _ = ssd_scan(x[:, None], np.asarray(dt)[:, None], A, np.asarray(B)[:, None],
+                           np.asarray(C)[:, None], D, init=state)
+    return y[:, 0], final

@@ -1,0 +1,259 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix, not against itself.
+
+Each test states the passage or the mathematical fact it relies on.  Together they are chosen so
+that a plausible slip in the oracle -- a dropped D term, the readout taken before the update,
+a wrong decay sign, B and C swapped, p and n transposed, heads mapped to the wrong group, dt
+missing from the input term -- fails at least one of them.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from mamba_ssd_layer_scan_b200 import configs, inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand_case(seed, b=2, L=29, H=4, G=2, P=3, N=5, init=True):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((b, L, H, P))
+    dt = rng.uniform(0.01, 0.5, (b, L, H))
+    A = -rng.uniform(0.1, 3.0, H)
+    B = rng.standard_normal((b, L, G, N))
+    C = rng.standard_normal((b, L, G, N))
+    D = rng.standard_normal(H)
+    h0 = rng.standard_normal((b, H, P, N)) if init else None
+    return x, dt, A, B, C, D, h0
+
+
+def _matrix_form(x, dt, A, B, C, D, h0):
+    """Brute force from the dual (matrix) form: y = M x + D x + C_t (prod a_j) h0, with
+    M[t, i] = C_t . B_i * dt_i * prod_{j=i+1..t} a_j and a_j = exp(dt_j A_h)
+    (eightmm.github.io "Mamba-2", Matrix Mixer View; mohakchugh.is-a.dev "Mamba-2", The Duality).
+    Products are formed term by term, as written, not through a cumulative sum."""
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    y = np.zeros_like(x)
+    final = np.zeros((b, H, P, N))
+    for bi in range(b):
+        for h in range(H):
+            g = h // (H // G)
+            a = np.exp(dt[bi, :, h] * A[h])
+            M = np.zeros((L, L))
+            for t in range(L):
+                for i in range(t + 1):
+                    M[t, i] = C[bi, t, g] @ B[bi, i, g] * dt[bi, i, h] * np.prod(a[i + 1:t + 1])
+            y[bi, :, h] = M @ x[bi, :, h] + D[h] * x[bi, :, h]
+            for i in range(L):
+                final[bi, h] += np.prod(a[i + 1:]) * dt[bi, i, h] * np.outer(x[bi, i, h], B[bi, i, g])
+            if h0 is not None:
+                for t in range(L):
+                    y[bi, t, h] += np.prod(a[:t + 1]) * (h0[bi, h] @ C[bi, t, g])
+                final[bi, h] += np.prod(a) * h0[bi, h]
+    return y, final
+
+
+def _rel(a, b):
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+@pytest.mark.parametrize("init", [False, True])
+def test_recurrence_equals_semiseparable_matrix(seed, init):
+    case = _rand_case(seed, init=init)
+    y, final, _ = oracle.ssd_scan(*case)
+    y_ref, final_ref = _matrix_form(*case)
+    assert _rel(y, y_ref) < 1e-12
+    assert _rel(final, final_ref) < 1e-12
+
+
+def test_group_mapping_contiguous():
+    """Heads split into G contiguous groups (h // (H/G)); a case with G = H/2 and B, C that differ
+    per group must match the matrix form, and not the one with an interleaved mapping."""
+    x, dt, A, B, C, D, h0 = _rand_case(7, b=1, L=9, H=4, G=2, P=2, N=3)
+    y, _, _ = oracle.ssd_scan(x, dt, A, B, C, D, h0)
+    y_ref, _ = _matrix_form(x, dt, A, B, C, D, h0)
+    assert _rel(y, y_ref) < 1e-12
+    # swap groups of heads 1 and 2 (an interleaved h % G mapping would read these)
+    Bs, Cs = B.copy(), C.copy()
+    Bs[:, :, [0, 1]] = B[:, :, [1, 0]]
+    Cs[:, :, [0, 1]] = C[:, :, [1, 0]]
+    y_wrong, _ = _matrix_form(x, dt, A, Bs, Cs, D, h0)
+    assert _rel(y[:, :, 1], y_wrong[:, :, 1]) > 1e-3
+
+
+def test_hand_worked_example():
+    d = json.load(open(os.path.join(GOLDEN, "worked_example_p2_n2.json")))
+    A = np.array(d["A_over_ln2"]) * np.log(2.0)
+    y, final, _ = oracle.ssd_scan(np.array(d["x"]), np.array(d["dt"]), A, np.array(d["B"]),
+                                  np.array(d["C"]), np.array(d["D"]))
+    np.testing.assert_allclose(y, np.array(d["y"]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(final, np.array(d["final_state"]), rtol=0, atol=1e-12)
+
+
+def _scalar(x, dt, A, B, C, D, h0=None):
+    """N = P = 1, one head: 1-D sequences in, 1-D y out."""
+    L = len(x)
+    y, final, _ = oracle.ssd_scan(np.reshape(x, (1, L, 1, 1)), np.reshape(dt, (1, L, 1)),
+                                  np.array([A]), np.reshape(B, (1, L, 1, 1)),
+                                  np.reshape(C, (1, L, 1, 1)), np.array([D]),
+                                  None if h0 is None else np.full((1, 1, 1, 1), h0))
+    return y.reshape(L), final.reshape(())
+
+
+def test_closed_form_constant_input_geometric_series():
+    """dt, B, C, x constant (B = C = x = 1), h0 = 0: h_t = dt (1 - a^{t+1}) / (1 - a), a geometric
+    series, so y_t = dt (1 - a^{t+1}) / (1 - a) + D."""
+    L, dt, A, D = 50, 0.07, -1.3, 0.4
+    a = np.exp(dt * A)
+    y, _ = _scalar(np.ones(L), np.full(L, dt), A, np.ones(L), np.ones(L), D)
+    t = np.arange(L)
+    np.testing.assert_allclose(y, dt * (1 - a ** (t + 1)) / (1 - a) + D, rtol=1e-13)
+
+
+def test_closed_form_no_decay_is_prefix_sum():
+    """A = 0 makes every a_t = 1: the state is the running sum of dt B x, y_t = C_t sum_{i<=t}
+    dt_i B_i x_i + D x_t."""
+    rng = np.random.default_rng(3)
+    L = 40
+    x, dt, B, C = rng.standard_normal(L), rng.uniform(0, 1, L), rng.standard_normal(L), \
+        rng.standard_normal(L)
+    y, final = _scalar(x, dt, 0.0, B, C, 0.25)
+    np.testing.assert_allclose(y, C * np.cumsum(dt * B * x) + 0.25 * x, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(final, np.sum(dt * B * x), rtol=1e-12)
+
+
+def test_closed_form_free_decay_of_initial_state():
+    """x = 0, h0 != 0: nothing enters, h_t = h0 exp(A sum_{j<=t} dt_j), y_t = C_t h_t."""
+    rng = np.random.default_rng(4)
+    L, A, h0 = 60, -2.0, 1.7
+    dt, C = rng.uniform(0, 0.2, L), rng.standard_normal(L)
+    y, final = _scalar(np.zeros(L), dt, A, rng.standard_normal(L), C, 0.9, h0=h0)
+    decay = np.exp(A * np.cumsum(dt))
+    np.testing.assert_allclose(y, C * h0 * decay, rtol=1e-12)
+    np.testing.assert_allclose(final, h0 * decay[-1], rtol=1e-12)
+
+
+def test_zero_dt_token_leaves_state_unchanged():
+    """dt = 0 gives a = exp(0) = 1 and no input: the state passes through untouched, and y at that
+    token is C_t h_{t-1} + D x_t."""
+    rng = np.random.default_rng(5)
+    L = 12
+    x, dt, B, C = (rng.standard_normal(L), rng.uniform(0.01, 0.3, L), rng.standard_normal(L),
+                   rng.standard_normal(L))
+    dt[6] = 0.0
+    _, h5 = _scalar(x[:6], dt[:6], -1.1, B[:6], C[:6], 0.3)
+    _, h6 = _scalar(x[:7], dt[:7], -1.1, B[:7], C[:7], 0.3)
+    y, _ = _scalar(x[:7], dt[:7], -1.1, B[:7], C[:7], 0.3)
+    assert h6 == h5
+    np.testing.assert_allclose(y[6], C[6] * h5 + 0.3 * x[6], rtol=1e-14)
+
+
+def test_off_diagonal_blocks_have_rank_at_most_N():
+    """Every lower-triangular submatrix M[k:, :k] of the SSD matrix has rank <= N, the state size
+    (mohakchugh.is-a.dev "Mamba-2", The Duality; eightmm.github.io, Structured Semiseparable
+    Matrices).  M is read off the oracle column by column (x = unit vectors, D = 0, h0 = 0); its
+    singular values past the N-th vanish while the N-th does not."""
+    rng = np.random.default_rng(6)
+    L, N = 24, 3
+    dt = rng.uniform(0.05, 0.4, (1, L, 1))
+    A = np.array([-0.8])
+    B = rng.standard_normal((1, L, 1, N))
+    C = rng.standard_normal((1, L, 1, N))
+    M = np.zeros((L, L))
+    for i in range(L):
+        e = np.zeros((1, L, 1, 1))
+        e[0, i, 0, 0] = 1.0
+        y, _, _ = oracle.ssd_scan(e, dt, A, B, C, np.zeros(1))
+        M[:, i] = y[0, :, 0, 0]
+    assert np.all(np.triu(M, 1) == 0.0)                 # causal
+    for k in (6, 12, 18):
+        s = np.linalg.svd(M[k:, :k], compute_uv=False)
+        assert s[N] / s[0] < 1e-10
+        assert s[N - 1] / s[0] > 1e-6
+
+
+def test_split_resume_equals_single_call():
+    """The state is the whole memory of the past (ql.gl, Recurrent state): running the first part,
+    then the rest from its final state, equals one call."""
+    x, dt, A, B, C, D, h0 = _rand_case(8, L=31)
+    y, final, _ = oracle.ssd_scan(x, dt, A, B, C, D, h0)
+    y1, f1, _ = oracle.ssd_scan(x[:, :13], dt[:, :13], A, B[:, :13], C[:, :13], D, h0)
+    y2, f2, _ = oracle.ssd_scan(x[:, 13:], dt[:, 13:], A, B[:, 13:], C[:, 13:], D, f1)
+    np.testing.assert_allclose(np.concatenate([y1, y2], 1), y, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(f2, final, rtol=1e-13, atol=1e-13)
+
+
+def test_linear_in_input_and_initial_state():
+    x, dt, A, B, C, D, h0 = _rand_case(9)
+    x2, _, _, _, _, _, h2 = _rand_case(10)
+    ya, fa, _ = oracle.ssd_scan(x, dt, A, B, C, D, h0)
+    yb, fb, _ = oracle.ssd_scan(x2, dt, A, B, C, D, h2)
+    yc, fc, _ = oracle.ssd_scan(2 * x - 3 * x2, dt, A, B, C, D, 2 * h0 - 3 * h2)
+    np.testing.assert_allclose(yc, 2 * ya - 3 * yb, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(fc, 2 * fa - 3 * fb, rtol=1e-12, atol=1e-12)
+
+
+def test_causal():
+    x, dt, A, B, C, D, h0 = _rand_case(11)
+    y, _, _ = oracle.ssd_scan(x, dt, A, B, C, D, h0)
+    x2, B2 = x.copy(), B.copy()
+    x2[:, 20:] += 1.0
+    B2[:, 20:] *= -2.0
+    y2, _, _ = oracle.ssd_scan(x2, dt, A, B2, C, D, h0)
+    np.testing.assert_array_equal(y2[:, :20], y[:, :20])
+
+
+def test_boundary_states_match_prefix_finals():
+    x, dt, A, B, C, D, h0 = _rand_case(12, L=30)
+    _, _, bnd = oracle.ssd_scan(x, dt, A, B, C, D, h0, every=8)
+    assert bnd.shape == (2, 4, 3, 3, 5)
+    for k in range(3):
+        _, f, _ = oracle.ssd_scan(x[:, :8 * (k + 1)], dt[:, :8 * (k + 1)], A, B[:, :8 * (k + 1)],
+                                  C[:, :8 * (k + 1)], D, h0)
+        np.testing.assert_array_equal(bnd[:, :, k], f)
+
+
+def test_decode_steps_equal_scan():
+    """Running the recurrence one token per call (the O(1)-per-token decode of crackai.dev
+    "Transformers are SSMs", Why It Matters) equals the scan over the same sequence."""
+    x, dt, A, B, C, D, h0 = _rand_case(13, L=10)
+    y, final, _ = oracle.ssd_scan(x, dt, A, B, C, D, h0)
+    st = h0.copy()
+    for t in range(10):
+        yt, st = oracle.ssd_state_update(st, x[:, t], dt[:, t], A, B[:, t], C[:, t], D)
+        np.testing.assert_allclose(yt, y[:, t], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(st, final, rtol=1e-13, atol=1e-13)
+
+
+def test_selected_pairs_match_full_scan():
+    w = configs.SSD_F32_SMALL.with_(batch=2, seqlen=40, nheads=4, ngroups=2, headdim=4, dstate=8,
+                                    init_state=True)
+    inp = inputs.make_inputs(w)
+    y, final, bnd = oracle.ssd_scan(inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, inp.init, every=16)
+    pairs = [(1, 3), (0, 0), (1, 1)]
+    ys, fs, bs = oracle.ssd_scan_pairs(inp, pairs, every=16)
+    for j, (b, h) in enumerate(pairs):
+        np.testing.assert_array_equal(ys[j], y[b, :, h])
+        np.testing.assert_array_equal(fs[j], final[b, h])
+        np.testing.assert_array_equal(bs[j], bnd[b, h])
+
+
+def test_bf16_rounding_matches_torch():
+    import torch
+    rng = np.random.default_rng(14)
+    a = (rng.standard_normal(100000) * np.exp(rng.uniform(-20, 20, 100000))).astype(np.float32)
+    ours = inputs.round_bf16(a)
+    ref = torch.from_numpy(a).to(torch.bfloat16).to(torch.float32).numpy()
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_input_recipe_ranges():
+    inp = inputs.make_inputs(configs.SSD_370M.with_(seqlen=256))
+    assert inp.dt.min() >= 1e-3 and inp.dt.max() <= 0.1
+    assert np.all(inp.A < 0) and np.all(inp.A >= -16.0) and np.all(inp.A <= -1.0)
+    np.testing.assert_array_equal(inputs.round_bf16(inp.x), inp.x)
+    assert abs(inp.B.std() * np.sqrt(128) - 1.0) < 0.05
