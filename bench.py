@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""Benchmark of the SSD layer scan on B200: one JSON line on rank 0.
+
+Workload (one "step"): the chunked scan forward of a 2.7B-scale Mamba-2 layer -- batch 4,
+4096 tokens, 80 heads of headdim 64, state 128, 1 group, chunk 256, bf16 x/B/C with fp32
+accumulation, final states returned -- i.e. all four kernels of the chunked path (dA cumsum,
+chunk state, state passing, chunk scan).  The recurrent decode update (batch 128, 80 heads,
+64 x 128 fp32 state, one token per call) is timed in the same run and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on the launching
+stream, with a 256 MB buffer written between steps (outside the events) to flush L2; inputs
+already resident in HBM.  Per-kernel times come from events the library records between its
+kernels (ssd_chunk_scan_fwd_staged).  Under torchrun each rank runs its own replica (weak
+scaling, no data-path collective) and the time is the max over ranks.  --impl reference times
+the float64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mamba_ssd_layer_scan_b200 import configs, inputs  # noqa: E402
+
+KERNELS = ("chunk_cumsum", "chunk_state", "state_passing", "chunk_scan")
+KERNEL_SOURCES = {
+    "chunk_cumsum": ["chunk_cumsum.cu"],
+    "chunk_state": ["chunk_tc.cu", "sm100.cuh"],
+    "state_passing": ["state_passing.cu"],
+    "chunk_scan": ["chunk_tc.cu", "sm100.cuh"],
+    "state_update": ["state_update.cu"],
+}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ work model
+def work_model(w):
+    """Algorithmic bytes and flops per launch of each kernel, and for the whole step.
+
+    Bytes are what each kernel must move at minimum given its inputs and outputs (element size
+    e for x/B/C/y, 4 for fp32); flops count the dense Q x Q intra-chunk product as the method
+    materialises it, plus the chunk-state and off-chunk products (2NP each per token-head) and
+    C B^T once per group (2QN per token-group)."""
+    b, L, H, P, N, G, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
+    c = -(-L // Q)
+    e = 2 if w.dtype == "bf16" else 4
+    x = b * L * H * P * e
+    bc = b * L * G * N * e
+    dt = b * L * H * 4
+    cs = b * c * H * Q * 4
+    st = b * c * H * P * N
+    fin = b * H * P * N * 4
+    init = fin if w.init_state else 0
+    k = {
+        "chunk_cumsum": {"bytes": dt + cs, "flops": 0},
+        "chunk_state": {"bytes": x + bc + dt + cs + st * 4, "flops": 2 * b * L * H * P * N},
+        "state_passing": {"bytes": st * 4 + st * 2 + fin + init, "flops": 0},
+        "chunk_scan": {"bytes": x + 2 * bc + dt + cs + st * 2 + x,
+                       "flops": b * L * H * (2 * Q * P + 2 * N * P) + b * L * G * 2 * Q * N,
+                       "flops_causal": b * L * H * ((Q + 1) * P + 2 * N * P)
+                       + b * L * G * (Q + 1) * N},
+    }
+    total = {"bytes": x + 2 * bc + dt + x + fin + init,
+             "flops": b * L * H * (2 * Q * P + 4 * N * P) + b * L * G * 2 * Q * N,
+             "flops_causal": b * L * H * ((Q + 1) * P + 4 * N * P) + b * L * G * (Q + 1) * N}
+    return k, total
+
+
+def decode_bytes(w):
+    e = 2 if w.dtype == "bf16" else 4
+    b, H, P, N, G = w.batch, w.nheads, w.headdim, w.dstate, w.ngroups
+    return 2 * b * H * P * N * 4 + 2 * b * H * P * e + 2 * b * G * N * e + b * H * 4
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(kernel):
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(ROOT, "mamba_ssd_layer_scan_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload):
+    """dram bytes per launch from the committed ncu summary, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(workload, {}).get(kernel)
+    if not d or d.get("source_sha") != source_hash(kernel):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples of one GPU while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, nvml_index):
+        self.idx = nvml_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def nvml_index(torch, dev):
+    try:
+        return torch.cuda._get_nvml_device_index(dev)
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            try:
+                return int(vis.split(",")[dev])
+            except ValueError:
+                pass
+        return dev
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def time_oracle(w, inp, target_s, max_pairs=None):
+    """Run the float64 oracle on (batch, head) slices of the full sequence until about
+    target_s seconds have passed; returns (tokens/s scaled to whole-layer tokens, sample text,
+    threads)."""
+    import oracle
+    threads = oracle.num_threads()
+    pairs_all = [(b, h) for b in range(w.batch) for h in range(w.nheads)]
+    rng = np.random.default_rng(0)
+    order = rng.permutation(len(pairs_all))
+    done, t0 = 0, time.perf_counter()
+    while done == 0 or (time.perf_counter() - t0 < target_s and done < len(pairs_all)):
+        batch = [pairs_all[i] for i in order[done:done + threads]]
+        if max_pairs is not None:
+            batch = batch[:max(0, max_pairs - done)]
+            if not batch:
+                break
+        oracle.ssd_scan_pairs(inp, batch)
+        done += len(batch)
+    el = time.perf_counter() - t0
+    tokens = done * w.seqlen / w.nheads
+    sample = (f"{done} of {w.batch * w.nheads} (batch, head) slices over the full "
+              f"{w.seqlen}-token sequence, float64 recurrence; tokens/s = slices * L / H / s")
+    return tokens / el, sample, threads, el
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inp = inputs.make_inputs(w)
+    import oracle
+    threads = oracle.num_threads()
+    # one step = one bounded sample: `threads` slices (about 1-3 s of host work)
+    steps = []
+    for i in range(args.warmup + args.steps):
+        v, sample, thr, el = time_oracle(w, inp, target_s=0.0, max_pairs=threads)
+        if i >= args.warmup:
+            steps.append((v, el))
+    value = len(steps) / sum(1.0 / v for v, _ in steps)   # tokens over total time
+    ms = 1e3 * statistics.mean(el for _, el in steps)
+    line = {
+        "impl": "reference", "metric": "ssd_chunk_scan_fwd_tokens_per_s", "value": value,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
+                   "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups,
+                   "chunk": w.chunk, "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                         "sample": f"per step: {thr} (batch, head) slices over the full "
+                                   f"{w.seqlen}-token sequence, float64 recurrence; "
+                                   "tokens/s = slices * L / H / s"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=None)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = configs.SSD_2P7B
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    from mamba_ssd_layer_scan_b200 import ssd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    # ---- inputs for the scan (same seeded draw on every rank: weak-scaling replicas)
+    inp = inputs.make_inputs(w)
+    xdt = torch.bfloat16
+    host = {k: torch.from_numpy(np.ascontiguousarray(v)) for k, v in
+            dict(x=inp.x, dt=inp.dt, A=inp.A, B=inp.B, C=inp.C, D=inp.D).items()}
+    host["x"], host["B"], host["C"] = (host[k].to(xdt) for k in ("x", "B", "C"))
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    t = {k: v.to(dev) for k, v in host.items()}
+    shape = ssd.make_shape(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                           ssd.SSD_BF16)
+    ws = ssd.new_workspace(shape, w.chunk, dev)
+    y = torch.empty_like(t["x"])
+    final = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
+                        device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def fwd(events=None):
+        ssd.chunk_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], w.chunk, y=y,
+                           final_state=final, workspace=ws, stage_events=events)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for row in ev:            # create the underlying CUDA events before handing them over
+        for e in row:
+            e.record(stream)
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        fwd()
+    torch.cuda.synchronize()
+    assert ssd.workspace_status(ws) == ssd.SSD_OK, "in-kernel timeout during warm-up"
+
+    sampler = ClockSampler(nvml_index(torch, local)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        t_pre = time.perf_counter()
+        while time.perf_counter() - t_pre < 0.6:      # load the GPU while sampling starts
+            fwd()
+        torch.cuda.synchronize()
+
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(K):
+        flush.fill_(1.0)
+        fwd(ev[i])
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop() if sampler else None
+    assert ssd.workspace_status(ws) == ssd.SSD_OK, "in-kernel timeout during timing"
+
+    step_ms = [ev[i][0].elapsed_time(ev[i][4]) for i in range(K)]
+    kern_ms = {name: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)]
+               for j, name in enumerate(KERNELS)}
+    total_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / K
+    tokens_per_step = w.batch * w.seqlen
+    value = world * tokens_per_step * K / (total_ms / 1e3)
+
+    # ---- end to end through the C ABI with host buffers: H2D of inputs, scan, D2H of y + final
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    f_host = torch.empty(final.shape, dtype=final.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = y_host.numel() * y_host.element_size() + f_host.numel() * f_host.element_size()
+    K_e2e = max(3, min(K, 20))
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    for i in range(K_e2e + 2):
+        if i == 2:
+            barrier()
+            torch.cuda.synchronize()
+            e_start.record(stream)
+        for k, v in pinned.items():
+            t[k].copy_(v, non_blocking=True)
+        fwd()
+        y_host.copy_(y, non_blocking=True)
+        f_host.copy_(final, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end) / K_e2e
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = world * tokens_per_step / (e2e_ms / 1e3)
+
+    # ---- decode update at batch 128, 80 heads, 64 x 128 fp32 state
+    wd = configs.SSD_DECODE
+    gen = torch.Generator(device=dev).manual_seed(wd.seed)
+    state = 0.1 * torch.randn((wd.batch, wd.nheads, wd.headdim, wd.dstate), device=dev,
+                              generator=gen)
+    xd = torch.randn((wd.batch, wd.nheads, wd.headdim), device=dev, generator=gen).to(xdt)
+    dtd = torch.nn.functional.softplus(
+        torch.randn((wd.batch, wd.nheads), device=dev, generator=gen) - 4).clamp(1e-3, 0.1)
+    Bd = (torch.randn((wd.batch, wd.ngroups, wd.dstate), device=dev, generator=gen)
+          / wd.dstate ** 0.5).to(xdt)
+    Cd = (torch.randn((wd.batch, wd.ngroups, wd.dstate), device=dev, generator=gen)
+          / wd.dstate ** 0.5).to(xdt)
+    yd = torch.empty_like(xd)
+    Kd = args.decode_steps or max(20, K)
+    for _ in range(5):
+        ssd.state_update(state, xd, dtd, t["A"], Bd, Cd, t["D"], y=yd)
+    d0 = torch.cuda.Event(enable_timing=True)
+    d1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    d0.record(stream)
+    for _ in range(Kd):
+        ssd.state_update(state, xd, dtd, t["A"], Bd, Cd, t["D"], y=yd)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    dec_ms = d0.elapsed_time(d1) / Kd
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    # ---- rooflines
+    peaks, peak_src = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tc_peak = peaks["bf16_tflops"]
+    kmodel, total = work_model(w)
+    kernels = {}
+    for name in KERNELS:
+        ms = statistics.mean(kern_ms[name])
+        m = kmodel[name]
+        gbs = m["bytes"] / (ms / 1e3) / 1e9
+        tfs = m["flops"] / (ms / 1e3) / 1e12
+        t_hbm = m["bytes"] / (hbm * 1e9)
+        t_tc = m["flops"] / (tc_peak * 1e12)
+        kernels[name] = {"ms": ms, "share": ms / ms_per_step, "gbs": gbs,
+                         "frac_hbm": gbs / hbm, "tflops": tfs, "frac_tensor": tfs / tc_peak,
+                         "bound": "tensor" if t_tc > t_hbm else "hbm",
+                         "alg_bytes": m["bytes"], "alg_flops": m["flops"]}
+    dom = max(KERNELS, key=lambda n: kernels[n]["ms"])
+    kd = kernels[dom]
+    if kd["bound"] == "tensor":
+        roof = {"bound": "tensor", "achieved": kd["tflops"], "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": kd["tflops"] / tc_peak}
+    else:
+        roof = {"bound": "hbm", "achieved": kd["gbs"], "peak": hbm, "unit": "GB/s",
+                "frac": kd["gbs"] / hbm}
+    roof.update({"kernel": dom, "traffic": profiled_traffic(dom, w.name),
+                 "alg_bytes_per_launch": kd["alg_bytes"], "alg_flops_per_launch": kd["alg_flops"],
+                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured"
+                 else "fallback"})
+    tc_ms = kernels["chunk_state"]["ms"] + kernels["chunk_scan"]["ms"]
+    tc_flops = kmodel["chunk_state"]["flops"] + kmodel["chunk_scan"]["flops"]
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, sample, thr, el = time_oracle(w, inp, target_s=15.0)
+        cpu = {"value": v, "unit": "tokens/s", "cores": thr, "kind": "oracle", "sample": sample,
+               "seconds": el}
+
+    dbytes = decode_bytes(wd)
+    line = {
+        "metric": "ssd_chunk_scan_fwd_tokens_per_s", "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
+                   "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups,
+                   "chunk": w.chunk, "final_state": True,
+                   "l2": "256 MB buffer written between timed steps (outside the events)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "tensor_core_kernels": {"tflops": tc_flops / (tc_ms / 1e3) / 1e12,
+                                "frac_of_bf16_peak": tc_flops / (tc_ms / 1e3) / 1e12 / tc_peak,
+                                "ms": tc_ms, "flops": tc_flops},
+        "step_totals": {"alg_bytes": total["bytes"], "alg_flops": total["flops"],
+                        "alg_flops_causal": total["flops_causal"],
+                        "gbs_compulsory": total["bytes"] / (ms_per_step / 1e3) / 1e9,
+                        "tflops_dense": total["flops"] / (ms_per_step / 1e3) / 1e12},
+        "kernels": kernels,
+        "decode": {"workload": wd.name, "metric": "ssd_state_update_GBps", "value":
+                   dbytes / (dec_ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": dec_ms,
+                   "frac_hbm": dbytes / (dec_ms / 1e3) / 1e9 / hbm, "bytes_per_step": dbytes,
+                   "tokens_per_s": wd.batch / (dec_ms / 1e3), "steps": Kd},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "cpu_baseline": cpu,
+        "clocks": clocks,
+        "gpu_launches": 4 * K,
+        "wall_s_timed_region": wall,
+        "peaks": {"hbm_gbs": hbm, "bf16_tflops": tc_peak, "source": peak_src},
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

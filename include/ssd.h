@@ -1,0 +1,153 @@
+/*
+ * ssd.h -- C ABI of the B200 (sm_100a) Mamba-2 SSD sequence mixer.
+ *
+ * The operation (per batch b, head h; g = h / (H/G) is the head's group of B/C):
+ *
+ *     a_t    = exp(dt_t * A_h)
+ *     h_t    = a_t * h_{t-1} + dt_t * x_t (outer) B_t      state P x N, h_{-1} = init or 0
+ *     y_t    = h_t C_t + D_h * x_t
+ *
+ * This is the selective SSM recurrence with a scalar-times-identity transition per head
+ * (ql.gl "Why Does Mamba-2 Resemble the Transformer?", The Problem; chipfoundryservices.com
+ * "hybrid attention-SSM", third paragraph), with A-bar = exp(dt A) and the D skip term
+ * (mohakchugh.is-a.dev "Mamba-2", State Space Models: The Core Abstraction), and the input
+ * scaled by dt as the same page's Multi-Head SSM block feeds it.
+ *
+ * Layouts (row-major, innermost last; all tensors dense and contiguous):
+ *     x, y        (batch, seqlen, nheads, headdim)    element type `dtype`
+ *     dt          (batch, seqlen, nheads)             float32, already positive (post-softplus)
+ *     A, D        (nheads)                            float32
+ *     B, C        (batch, seqlen, ngroups, dstate)    element type `dtype`
+ *     state, init_state, final_state
+ *                 (batch, nheads, headdim, dstate)    float32, dstate fastest
+ *
+ * Ownership: every pointer is a device pointer owned by the caller; the library allocates no
+ * device or host memory in these calls and keeps no state across calls except a thread-local
+ * error string.  Scratch space for the chunked scan is passed in by the caller (`workspace`).
+ * All pointers to x, y, B, C, states and the workspace must be 16-byte aligned.
+ *
+ * Errors: functions return an ssd_status and never abort or throw.  Calls are asynchronous on
+ * `stream` (a cudaStream_t passed as void*; NULL is the legacy default stream): the status
+ * covers argument validation and launch errors only; faults inside a kernel surface at the
+ * caller's next synchronisation.  ssd_last_error() describes the last non-OK status of the
+ * calling thread.
+ */
+#ifndef SSD_B200_SSD_H
+#define SSD_B200_SSD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer, short workspace */
+    SSD_ERR_UNSUPPORTED = 2,   /* a size outside the ranges listed below */
+    SSD_ERR_CUDA = 3,          /* a CUDA call or kernel launch failed */
+    SSD_ERR_TIMEOUT = 4        /* a bounded in-kernel wait gave up (see ssd_workspace_status) */
+} ssd_status;
+
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+
+/* Problem sizes.  seqlen is ignored by ssd_state_update (one token per call). */
+typedef struct {
+    int64_t batch;     /* >= 0 */
+    int64_t seqlen;    /* >= 0 */
+    int64_t nheads;    /* H >= 1 */
+    int64_t headdim;   /* P: 1..128 */
+    int64_t dstate;    /* N: multiple of 32 in 32..256, headdim * dstate <= 16384 */
+    int64_t ngroups;   /* G >= 1, nheads % ngroups == 0 */
+    int32_t dtype;     /* ssd_dtype of x, B, C and y */
+} ssd_shape;
+
+/*
+ * Bytes of workspace ssd_chunk_scan_fwd needs for this shape and chunk size (0 when the
+ * arguments are invalid; the call then also fails with the reason).  The workspace holds the
+ * per-chunk cumulative log-decays, the per-chunk states and a device status word.
+ */
+size_t ssd_chunk_scan_workspace_size(const ssd_shape *shape, int chunk_size);
+
+/*
+ * Chunked (block-decomposed) SSD scan over a whole sequence: y for every token and, when
+ * final_state is non-NULL, the state after the last token.
+ *
+ * The sequence is cut into chunks of chunk_size tokens (the last one may be partial); within a
+ * chunk the output is the masked quadratic form (C B^T o L) (dt x) computed as dense matrix
+ * products on tensor cores, and across chunks a P x N state is carried by the linear
+ * recurrence (mohakchugh.is-a.dev "Mamba-2", Block Decomposition and The Tensor Core
+ * Connection; ql.gl, The Core of SSD).  The result equals the token-by-token recurrence above
+ * up to rounding, for any chunk_size.
+ *
+ *   chunk_size     Q in {16, 32, 64, 128, 256}.  bf16 with headdim 64, dstate 128 and
+ *                  Q in {128, 256} runs the tensor-core (tcgen05) kernels; every other
+ *                  supported shape runs the CUDA-core kernels in float32.
+ *   init_state     nullable: NULL means a zero initial state.
+ *   final_state    nullable: NULL means not written.  May alias init_state.
+ *   y              must not alias any input.
+ *   workspace      at least ssd_chunk_scan_workspace_size() bytes, 256-byte aligned; its
+ *                  contents on entry do not matter and on exit are unspecified.
+ *
+ * Concurrent calls must use distinct workspaces.  batch == 0 or seqlen == 0 is valid: y is
+ * empty and final_state is set to init_state (or zeros).
+ */
+ssd_status ssd_chunk_scan_fwd(const ssd_shape *shape, const void *x, const float *dt,
+                              const float *A, const void *B, const void *C, const float *D,
+                              int chunk_size, const float *init_state, void *y,
+                              float *final_state, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/*
+ * Same as ssd_chunk_scan_fwd, and additionally records caller-created CUDA events on `stream`
+ * around its kernels so that each stage can be timed on the device:
+ *     stage_events[0]  before the dA cumsum kernel
+ *     stage_events[1]  after it (before the chunk-state kernel)
+ *     stage_events[2]  after the chunk-state kernel (before state passing)
+ *     stage_events[3]  after state passing (before the chunk-scan kernel)
+ *     stage_events[4]  after the chunk-scan kernel
+ * stage_events points to 5 cudaEvent_t values (passed as void*); NULL behaves exactly like
+ * ssd_chunk_scan_fwd.  The events are only recorded, never created, waited on or destroyed.
+ */
+ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, const float *dt,
+                                     const float *A, const void *B, const void *C,
+                                     const float *D, int chunk_size, const float *init_state,
+                                     void *y, float *final_state, void *workspace,
+                                     size_t workspace_bytes, void *stream,
+                                     void *const *stage_events);
+
+/*
+ * One recurrent (decode) step for one new token per sequence, O(1) in the length of the past
+ * (crackai.dev "Transformers are SSMs", Why It Matters; mohakchugh.is-a.dev "Mamba-2", Why
+ * This Matters for Hardware, linear mode):
+ *     state <- exp(dt A) * state + dt * x (outer) B,     y = state C + D x
+ *
+ *   state  (batch, nheads, headdim, dstate) float32, updated in place.
+ *   x, y   (batch, nheads, headdim)         element type `dtype`
+ *   dt     (batch, nheads) float32;  B, C (batch, ngroups, dstate) element type `dtype`.
+ *   y must not alias state or the inputs.
+ */
+ssd_status ssd_state_update(const ssd_shape *shape, float *state, const void *x,
+                            const float *dt, const float *A, const void *B, const void *C,
+                            const float *D, void *y, void *stream);
+
+/*
+ * Synchronises `stream` and reads the device status word the last ssd_chunk_scan_fwd call on
+ * this workspace left behind: SSD_OK, or SSD_ERR_TIMEOUT when an in-kernel wait on a
+ * shared-memory barrier exceeded its bound and the kernel returned early (its outputs are
+ * then incomplete).  Returns SSD_ERR_CUDA if the synchronisation itself reports an error.
+ */
+ssd_status ssd_workspace_status(const void *workspace, size_t workspace_bytes, void *stream);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+const char *ssd_last_error(void);
+
+/* Library version string. */
+const char *ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_B200_SSD_H */

@@ -1,0 +1,72 @@
+// Shared device helpers and the internal launch interface of the SSD kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+using bf16 = __nv_bfloat16;
+
+// Element access for the two storage types of x, B, C and y.
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Workspace regions of one ssd_chunk_scan_fwd call (byte offsets from the workspace base).
+struct WsLayout {
+    size_t status;      // 256 bytes: device status word (nonzero after an in-kernel timeout)
+    size_t cs;          // float [b][c][H][Q]: chunk-local inclusive cumsum of dt*A
+    size_t states;      // float [b][c][H][P][N]: per-chunk state, then (in place) state entering
+    size_t hin_bf16;    // bf16  [b][c][H][P][N]: state entering each chunk (tensor-core path)
+    size_t total;
+};
+
+// ---- launchers (each returns the launch's cudaError_t) ----
+// Also zeroes *status (nullable) so each scan starts with a clean status word.
+cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, int *status,
+                                int64_t batch, int64_t seqlen, int nheads, int Q,
+                                int64_t nchunks, cudaStream_t st);
+
+cudaError_t launch_chunk_state_simt(bool is_bf16, const void *x, const float *dt,
+                                    const void *B, const float *cs, float *states,
+                                    int64_t batch, int64_t seqlen, int H, int G, int P, int N,
+                                    int Q, int64_t nchunks, cudaStream_t st);
+
+// Carries the state across chunks: states[k] (chunk-local contribution) is replaced in place by
+// the state entering chunk k (float32), or that state is written to hin_bf16 when non-null.
+cudaError_t launch_state_passing(float *states, const float *cs, const float *init,
+                                 float *final_state, bf16 *hin_bf16, int64_t batch, int H,
+                                 int P, int N, int Q, int64_t nchunks, cudaStream_t st);
+
+cudaError_t launch_chunk_scan_simt(bool is_bf16, const void *x, const float *dt,
+                                   const void *B, const void *C, const float *cs,
+                                   const float *hin, const float *D, void *y, int64_t batch,
+                                   int64_t seqlen, int H, int G, int P, int N, int Q,
+                                   int64_t nchunks, cudaStream_t st);
+
+cudaError_t launch_state_update(bool is_bf16, float *state, const void *x, const float *dt,
+                                const float *A, const void *B, const void *C, const float *D,
+                                void *y, int64_t batch, int H, int G, int P, int N,
+                                cudaStream_t st);
+
+cudaError_t launch_fill_final(const float *init, float *final_state, int64_t n,
+                              cudaStream_t st);
+
+// Tensor-core (tcgen05 + TMA) path: bf16, P = 64, N = 128, Q in {128, 256}.
+bool tc_supported(bool is_bf16, int P, int N, int Q);
+cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dt, const bf16 *B,
+                                  const float *cs, float *states, int *status, int64_t batch,
+                                  int64_t seqlen, int H, int G, int Q, int64_t nchunks,
+                                  cudaStream_t st, const char **why);
+cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dt, const bf16 *B, const bf16 *C,
+                                 const float *cs, const bf16 *hin, const float *D, bf16 *y,
+                                 int *status, int64_t batch, int64_t seqlen, int H, int G,
+                                 int Q, int64_t nchunks, cudaStream_t st, const char **why);
+
+}  // namespace ssd

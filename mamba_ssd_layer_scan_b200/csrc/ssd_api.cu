@@ -1,0 +1,247 @@
+// C ABI entry points (include/ssd.h): argument validation, workspace carving, kernel dispatch.
+//
+// ssd_chunk_scan_fwd enqueues, on the caller's stream and in this order:
+//   1. dA cumsum            chunk-local prefix sums of dt*A            (chunk_cumsum.cu)
+//   2. chunk state          each chunk's own contribution to its end state (chunk_tc.cu /
+//                           chunk_simt.cu)
+//   3. state passing        the recurrence across chunks               (state_passing.cu)
+//   4. chunk scan           within-chunk quadratic form + off-chunk term (chunk_tc.cu /
+//                           chunk_simt.cu)
+// following the block decomposition of mohakchugh.is-a.dev "Mamba-2" (Block Decomposition:
+// quadratic form inside a chunk, linear recurrence across chunks).  Nothing is allocated and
+// nothing synchronises; errors are reported through the returned status.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/ssd.h"
+#include "common.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+ssd_status fail(ssd_status s, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+ssd_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(SSD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+cudaError_t record(void *const *events, int i, cudaStream_t st)
+{
+    return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) : cudaSuccess;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
+
+ssd_status check_shape(const ssd_shape *s, bool need_seq)
+{
+    if (!s) return fail(SSD_ERR_INVALID_ARG, "shape is NULL");
+    if (s->batch < 0 || (need_seq && s->seqlen < 0))
+        return fail(SSD_ERR_INVALID_ARG, "batch and seqlen must be >= 0");
+    if (s->nheads < 1 || s->ngroups < 1 || s->nheads % s->ngroups != 0)
+        return fail(SSD_ERR_INVALID_ARG, "need nheads >= 1, ngroups >= 1, nheads %% ngroups == 0 "
+                    "(got %lld, %lld)", (long long)s->nheads, (long long)s->ngroups);
+    if (s->dtype != SSD_F32 && s->dtype != SSD_BF16)
+        return fail(SSD_ERR_INVALID_ARG, "dtype must be SSD_F32 or SSD_BF16");
+    if (s->headdim < 1 || s->headdim > 128)
+        return fail(SSD_ERR_UNSUPPORTED, "headdim must be in 1..128 (got %lld)",
+                    (long long)s->headdim);
+    if (s->dstate < 32 || s->dstate > 256 || s->dstate % 32 != 0)
+        return fail(SSD_ERR_UNSUPPORTED, "dstate must be a multiple of 32 in 32..256 (got %lld)",
+                    (long long)s->dstate);
+    if (s->headdim * s->dstate > 16384)
+        return fail(SSD_ERR_UNSUPPORTED, "headdim * dstate must be <= 16384");
+    if (s->nheads > 65535 || s->batch > 65535)
+        return fail(SSD_ERR_UNSUPPORTED, "batch and nheads must be <= 65535");
+    return SSD_OK;
+}
+
+bool valid_chunk(int q) { return q == 16 || q == 32 || q == 64 || q == 128 || q == 256; }
+
+ssd::WsLayout layout(const ssd_shape *s, int Q)
+{
+    const int64_t nchunks = (s->seqlen + Q - 1) / Q;
+    const size_t rows = (size_t)s->batch * nchunks * s->nheads;
+    ssd::WsLayout w;
+    w.status = 0;
+    w.cs = 256;
+    w.states = w.cs + round256(rows * Q * sizeof(float));
+    w.hin_bf16 = w.states + round256(rows * s->headdim * s->dstate * sizeof(float));
+    const bool tc = ssd::tc_supported(s->dtype == SSD_BF16, (int)s->headdim, (int)s->dstate, Q);
+    w.total = w.hin_bf16 + (tc ? round256(rows * s->headdim * s->dstate * sizeof(uint16_t)) : 0);
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ssd_last_error(void) { return g_err; }
+
+const char *ssd_version(void) { return "ssd-b200 0.1 (sm_100a)"; }
+
+size_t ssd_chunk_scan_workspace_size(const ssd_shape *shape, int chunk_size)
+{
+    if (check_shape(shape, true) != SSD_OK) return 0;
+    if (!valid_chunk(chunk_size)) {
+        fail(SSD_ERR_UNSUPPORTED, "chunk_size must be 16, 32, 64, 128 or 256 (got %d)",
+             chunk_size);
+        return 0;
+    }
+    return layout(shape, chunk_size).total;
+}
+
+ssd_status ssd_chunk_scan_fwd(const ssd_shape *shape, const void *x, const float *dt,
+                              const float *A, const void *B, const void *C, const float *D,
+                              int chunk_size, const float *init_state, void *y,
+                              float *final_state, void *workspace, size_t workspace_bytes,
+                              void *stream)
+{
+    return ssd_chunk_scan_fwd_staged(shape, x, dt, A, B, C, D, chunk_size, init_state, y,
+                                     final_state, workspace, workspace_bytes, stream, nullptr);
+}
+
+ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, const float *dt,
+                                     const float *A, const void *B, const void *C,
+                                     const float *D, int chunk_size, const float *init_state,
+                                     void *y, float *final_state, void *workspace,
+                                     size_t workspace_bytes, void *stream,
+                                     void *const *stage_events)
+{
+    ssd_status st = check_shape(shape, true);
+    if (st != SSD_OK) return st;
+    if (!valid_chunk(chunk_size))
+        return fail(SSD_ERR_UNSUPPORTED, "chunk_size must be 16, 32, 64, 128 or 256 (got %d)",
+                    chunk_size);
+    const ssd_shape s = *shape;
+    const int H = (int)s.nheads, G = (int)s.ngroups, P = (int)s.headdim, N = (int)s.dstate;
+    const int Q = chunk_size;
+    const bool bf = s.dtype == SSD_BF16;
+    cudaStream_t cs_stream = static_cast<cudaStream_t>(stream);
+    const int64_t PNtot = s.batch * s.nheads * s.headdim * s.dstate;
+
+    if (final_state && !aligned16(final_state))
+        return fail(SSD_ERR_INVALID_ARG, "final_state must be 16-byte aligned");
+    if (init_state && !aligned16(init_state))
+        return fail(SSD_ERR_INVALID_ARG, "init_state must be 16-byte aligned");
+    if (s.batch == 0) return SSD_OK;
+    if (s.seqlen == 0) {
+        if (final_state) {
+            cudaError_t e = ssd::launch_fill_final(init_state, final_state, PNtot, cs_stream);
+            if (e != cudaSuccess) return cuda_fail(e, "fill final state");
+        }
+        return SSD_OK;
+    }
+    if (!x || !dt || !A || !B || !C || !D || !y || !workspace)
+        return fail(SSD_ERR_INVALID_ARG, "x, dt, A, B, C, D, y and workspace must be non-NULL");
+    if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(y))
+        return fail(SSD_ERR_INVALID_ARG, "x, B, C and y must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(SSD_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const int64_t nchunks = (s.seqlen + Q - 1) / Q;
+    if (s.batch * nchunks * s.nheads * ((Q + 31) / 32) > 0x7fffffffLL)
+        return fail(SSD_ERR_UNSUPPORTED, "problem too large for one launch grid");
+    const ssd::WsLayout wl = layout(&s, Q);
+    if (workspace_bytes < wl.total)
+        return fail(SSD_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu",
+                    wl.total, workspace_bytes);
+
+    char *ws = static_cast<char *>(workspace);
+    int *status = reinterpret_cast<int *>(ws + wl.status);
+    float *cs = reinterpret_cast<float *>(ws + wl.cs);
+    float *states = reinterpret_cast<float *>(ws + wl.states);
+    cudaError_t e = record(stage_events, 0, cs_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "record stage event");
+    e = ssd::launch_chunk_cumsum(dt, A, cs, status, s.batch, s.seqlen, H, Q, nchunks, cs_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "dA cumsum launch");
+    if ((e = record(stage_events, 1, cs_stream)) != cudaSuccess)
+        return cuda_fail(e, "record stage event");
+
+    if (ssd::tc_supported(bf, P, N, Q)) {
+        const char *why = "";
+        ssd::bf16 *hin = reinterpret_cast<ssd::bf16 *>(ws + wl.hin_bf16);
+        e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dt, (const ssd::bf16 *)B, cs,
+                                       states, status, s.batch, s.seqlen, H, G, Q, nchunks,
+                                       cs_stream, &why);
+        if (e != cudaSuccess) return cuda_fail(e, why);
+        if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess)
+            return cuda_fail(e, "record stage event");
+        e = ssd::launch_state_passing(states, cs, init_state, final_state, hin, s.batch, H, P,
+                                      N, Q, nchunks, cs_stream);
+        if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
+        if ((e = record(stage_events, 3, cs_stream)) != cudaSuccess)
+            return cuda_fail(e, "record stage event");
+        e = ssd::launch_chunk_scan_tc((const ssd::bf16 *)x, dt, (const ssd::bf16 *)B,
+                                      (const ssd::bf16 *)C, cs, hin, D, (ssd::bf16 *)y, status,
+                                      s.batch, s.seqlen, H, G, Q, nchunks, cs_stream, &why);
+        if (e != cudaSuccess) return cuda_fail(e, why);
+        if ((e = record(stage_events, 4, cs_stream)) != cudaSuccess)
+            return cuda_fail(e, "record stage event");
+        return SSD_OK;
+    }
+
+    e = ssd::launch_chunk_state_simt(bf, x, dt, B, cs, states, s.batch, s.seqlen, H, G, P, N, Q,
+                                     nchunks, cs_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk state launch");
+    if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess)
+        return cuda_fail(e, "record stage event");
+    e = ssd::launch_state_passing(states, cs, init_state, final_state, nullptr, s.batch, H, P, N,
+                                  Q, nchunks, cs_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
+    if ((e = record(stage_events, 3, cs_stream)) != cudaSuccess)
+        return cuda_fail(e, "record stage event");
+    e = ssd::launch_chunk_scan_simt(bf, x, dt, B, C, cs, states, D, y, s.batch, s.seqlen, H, G,
+                                    P, N, Q, nchunks, cs_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk scan launch");
+    if ((e = record(stage_events, 4, cs_stream)) != cudaSuccess)
+        return cuda_fail(e, "record stage event");
+    return SSD_OK;
+}
+
+ssd_status ssd_state_update(const ssd_shape *shape, float *state, const void *x,
+                            const float *dt, const float *A, const void *B, const void *C,
+                            const float *D, void *y, void *stream)
+{
+    ssd_status st = check_shape(shape, false);
+    if (st != SSD_OK) return st;
+    const ssd_shape s = *shape;
+    if (s.batch == 0) return SSD_OK;
+    if (!state || !x || !dt || !A || !B || !C || !D || !y)
+        return fail(SSD_ERR_INVALID_ARG, "state, x, dt, A, B, C, D and y must be non-NULL");
+    if (!aligned16(state) || !aligned16(B) || !aligned16(C))
+        return fail(SSD_ERR_INVALID_ARG, "state, B and C must be 16-byte aligned");
+    cudaError_t e = ssd::launch_state_update(s.dtype == SSD_BF16, state, x, dt, A, B, C, D, y,
+                                             s.batch, (int)s.nheads, (int)s.ngroups,
+                                             (int)s.headdim, (int)s.dstate,
+                                             static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "state update launch");
+    return SSD_OK;
+}
+
+ssd_status ssd_workspace_status(const void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!workspace || workspace_bytes < sizeof(int))
+        return fail(SSD_ERR_INVALID_ARG, "workspace is NULL or too small");
+    int word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost,
+                                    static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "read workspace status");
+    if (word != 0)
+        return fail(SSD_ERR_TIMEOUT, "an in-kernel barrier wait exceeded its bound (code %d)",
+                    word);
+    return SSD_OK;
+}
+
+}  // extern "C"

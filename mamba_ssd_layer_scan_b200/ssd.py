@@ -1,0 +1,198 @@
+"""Thin Python binding over the C ABI in ``include/ssd.h`` (argument marshalling only).
+
+Every computation runs in ``libssd_b200.so``'s CUDA kernels; torch is used for device memory,
+streams and dtypes.  There is no fallback: if the shared library is missing or was built
+without the CUDA kernels, loading it raises.
+
+    y, final = chunk_scan_fwd(x, dt, A, B, C, D, chunk_size=256, init_state=None)
+    y = state_update(state, x, dt, A, B, C, D)          # state updated in place
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libssd_b200.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "ssd.h")
+
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(5)
+SSD_F32, SSD_BF16 = 0, 1
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"ssd status {status}: {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64),
+                ("dtype", ctypes.c_int32)]
+
+
+_lib = None
+_vp = ctypes.c_void_p
+
+
+def declared_functions():
+    """Names of the functions ``include/ssd.h`` declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssd_[a-z0-9_]+)\s*\(", text)))
+
+
+def lib():
+    """Load the shared library (raises if it is missing: there is no fallback path)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m mamba_ssd_layer_scan_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.ssd_chunk_scan_workspace_size.restype = ctypes.c_size_t
+    L.ssd_chunk_scan_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int]
+    L.ssd_chunk_scan_fwd.restype = ctypes.c_int
+    L.ssd_chunk_scan_fwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
+                                     ctypes.c_int, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    L.ssd_chunk_scan_fwd_staged.restype = ctypes.c_int
+    L.ssd_chunk_scan_fwd_staged.argtypes = L.ssd_chunk_scan_fwd.argtypes + [
+        ctypes.POINTER(ctypes.c_void_p)]
+    L.ssd_state_update.restype = ctypes.c_int
+    L.ssd_state_update.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _vp, _vp]
+    L.ssd_workspace_status.restype = ctypes.c_int
+    L.ssd_workspace_status.argtypes = [_vp, ctypes.c_size_t, _vp]
+    L.ssd_last_error.restype = ctypes.c_char_p
+    L.ssd_last_error.argtypes = []
+    L.ssd_version.restype = ctypes.c_char_p
+    L.ssd_version.argtypes = []
+    _lib = L
+    return L
+
+
+def last_error() -> str:
+    return lib().ssd_last_error().decode()
+
+
+def _check(status: int):
+    if status != SSD_OK:
+        raise SSDError(status, last_error())
+
+
+def make_shape(batch, seqlen, nheads, headdim, dstate, ngroups, dtype) -> Shape:
+    return Shape(batch, seqlen, nheads, headdim, dstate, ngroups, dtype)
+
+
+def workspace_size(shape: Shape, chunk_size: int) -> int:
+    n = lib().ssd_chunk_scan_workspace_size(ctypes.byref(shape), chunk_size)
+    if n == 0:
+        raise SSDError(SSD_ERR_INVALID_ARG, last_error())
+    return n
+
+
+# ---------------------------------------------------------------- torch marshalling
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return SSD_F32
+    if t.dtype == torch.bfloat16:
+        return SSD_BF16
+    raise TypeError(f"x must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream) -> Optional[int]:
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _require(t, name, dtype=None, device=None):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def new_workspace(shape: Shape, chunk_size: int, device):
+    """A device buffer of ssd_chunk_scan_workspace_size bytes (256-byte aligned by torch)."""
+    torch = _torch()
+    return torch.empty(workspace_size(shape, chunk_size), dtype=torch.uint8, device=device)
+
+
+def chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int = 256, init_state=None,
+                   return_final_state: bool = True, y=None, final_state=None, workspace=None,
+                   stream=None, stage_events=None):
+    """Chunked SSD scan.  x (b, L, H, P), dt (b, L, H) f32, A/D (H,) f32, B/C (b, L, G, N),
+    init_state (b, H, P, N) f32 or None.  Returns (y, final_state or None).
+
+    stage_events: optional list of 5 recorded-once torch.cuda.Event objects, recorded on the
+    stream around the four kernels (see ssd_chunk_scan_fwd_staged)."""
+    torch = _torch()
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = x.device
+    code = _dtype_code(x)
+    for t, n in ((x, "x"), (B, "B"), (C, "C")):
+        _require(t, n, x.dtype, dev)
+    for t, n in ((dt, "dt"), (A, "A"), (D, "D")):
+        _require(t, n, torch.float32, dev)
+    if init_state is not None:
+        _require(init_state, "init_state", torch.float32, dev)
+    shape = make_shape(b, L, H, P, N, G, code)
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(shape, chunk_size, dev)
+    args = (ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+            chunk_size, _ptr(init_state), _ptr(y), _ptr(final_state), _ptr(workspace),
+            workspace.numel(), _stream_handle(stream))
+    if stage_events is None:
+        _check(lib().ssd_chunk_scan_fwd(*args))
+    else:
+        handles = (ctypes.c_void_p * 5)(*[ev.cuda_event for ev in stage_events])
+        _check(lib().ssd_chunk_scan_fwd_staged(*args, handles))
+    return y, final_state
+
+
+def state_update(state, x, dt, A, B, C, D, y=None, stream=None):
+    """One decode step.  state (b, H, P, N) f32 (in place), x (b, H, P), dt (b, H) f32,
+    B/C (b, G, N).  Returns y (b, H, P)."""
+    torch = _torch()
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    dev = x.device
+    code = _dtype_code(x)
+    for t, n in ((x, "x"), (B, "B"), (C, "C")):
+        _require(t, n, x.dtype, dev)
+    for t, n in ((state, "state"), (dt, "dt"), (A, "A"), (D, "D")):
+        _require(t, n, torch.float32, dev)
+    shape = make_shape(b, 1, H, P, N, G, code)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(lib().ssd_state_update(ctypes.byref(shape), _ptr(state), _ptr(x), _ptr(dt), _ptr(A),
+                                  _ptr(B), _ptr(C), _ptr(D), _ptr(y), _stream_handle(stream)))
+    return y
+
+
+def workspace_status(workspace, stream=None) -> int:
+    """Synchronise and return the status word the last scan on ``workspace`` left (0 = OK)."""
+    return lib().ssd_workspace_status(_ptr(workspace), workspace.numel(), _stream_handle(stream))

@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every function the
+header declares, sizes its workspace, and rejects bad arguments before touching the device."""
+import ctypes
+import subprocess
+
+import pytest
+
+from mamba_ssd_layer_scan_b200 import build, ssd
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ssd.lib()
+
+
+def test_exports_every_declared_function(L):
+    declared = ssd.declared_functions()
+    assert {"ssd_chunk_scan_fwd", "ssd_state_update", "ssd_chunk_scan_workspace_size",
+            "ssd_last_error"} <= set(declared)
+    out = subprocess.run(["nm", "-D", "--defined-only", ssd.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared:
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_version(L):
+    assert b"sm_100a" in L.ssd_version()
+
+
+def _shape(**kw):
+    d = dict(batch=4, seqlen=4096, nheads=80, headdim=64, dstate=128, ngroups=1,
+             dtype=ssd.SSD_BF16)
+    d.update(kw)
+    return ssd.make_shape(**d)
+
+
+def test_workspace_size_layout():
+    b, L_, H, P, N, Q = 4, 4096, 80, 64, 128, 256
+    c = L_ // Q
+    ws = ssd.workspace_size(_shape(), Q)
+    # status word + cs (f32) + chunk states (f32) + bf16 entering states (tensor-core path)
+    expect = 256 + b * c * H * Q * 4 + b * c * H * P * N * 4 + b * c * H * P * N * 2
+    assert ws == expect
+    # float32 inputs run the CUDA-core path, which keeps the entering state in place (no bf16 copy)
+    ws32 = ssd.workspace_size(_shape(dtype=ssd.SSD_F32), Q)
+    assert ws32 == 256 + b * c * H * Q * 4 + b * c * H * P * N * 4
+    # a ragged length rounds the chunk count up
+    assert ssd.workspace_size(_shape(seqlen=4097), Q) > ws
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ngroups=3), ssd.SSD_ERR_INVALID_ARG),
+    (dict(nheads=0), ssd.SSD_ERR_INVALID_ARG),
+    (dict(batch=-1), ssd.SSD_ERR_INVALID_ARG),
+    (dict(dtype=7), ssd.SSD_ERR_INVALID_ARG),
+    (dict(headdim=129), ssd.SSD_ERR_UNSUPPORTED),
+    (dict(dstate=48), ssd.SSD_ERR_UNSUPPORTED),
+    (dict(headdim=128, dstate=256), ssd.SSD_ERR_UNSUPPORTED),
+])
+def test_bad_shapes_rejected(L, kw, code):
+    sh = _shape(**kw)
+    fake = ctypes.c_void_p(1 << 20)
+    rc = L.ssd_chunk_scan_fwd(ctypes.byref(sh), fake, fake, fake, fake, fake, fake, 256, None,
+                              fake, None, fake, 1 << 40, None)
+    assert rc == code
+    assert ssd.last_error()
+    assert L.ssd_chunk_scan_workspace_size(ctypes.byref(sh), 256) == 0
+
+
+def test_bad_chunk_and_pointers_rejected(L):
+    sh = _shape()
+    ok = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    big = 1 << 40
+    rc = L.ssd_chunk_scan_fwd(ctypes.byref(sh), ok, ok, ok, ok, ok, ok, 100, None, ok, None, ok,
+                              big, None)
+    assert rc == ssd.SSD_ERR_UNSUPPORTED and "chunk_size" in ssd.last_error()
+    rc = L.ssd_chunk_scan_fwd(ctypes.byref(sh), None, ok, ok, ok, ok, ok, 256, None, ok, None,
+                              ok, big, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "NULL" in ssd.last_error()
+    rc = L.ssd_chunk_scan_fwd(ctypes.byref(sh), mis, ok, ok, ok, ok, ok, 256, None, ok, None, ok,
+                              big, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "aligned" in ssd.last_error()
+    rc = L.ssd_chunk_scan_fwd(ctypes.byref(sh), ok, ok, ok, ok, ok, ok, 256, None, ok, None,
+                              ctypes.c_void_p((1 << 20) + 16), big, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "256-byte" in ssd.last_error()
+    rc = L.ssd_chunk_scan_fwd(ctypes.byref(sh), ok, ok, ok, ok, ok, ok, 256, None, ok, None, ok,
+                              1024, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "workspace too small" in ssd.last_error()
+    rc = L.ssd_chunk_scan_fwd(None, ok, ok, ok, ok, ok, ok, 256, None, ok, None, ok, big, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op(L):
+    sh = _shape(batch=0)
+    assert L.ssd_chunk_scan_fwd(ctypes.byref(sh), None, None, None, None, None, None, 256, None,
+                                None, None, None, 0, None) == ssd.SSD_OK
+    assert L.ssd_state_update(ctypes.byref(sh), None, None, None, None, None, None, None, None,
+                              None) == ssd.SSD_OK
+
+
+def test_state_update_rejects_bad_args(L):
+    ok = ctypes.c_void_p(1 << 20)
+    sh = _shape(batch=128)
+    rc = L.ssd_state_update(ctypes.byref(sh), None, ok, ok, ok, ok, ok, ok, ok, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG
+    rc = L.ssd_state_update(ctypes.byref(sh), ctypes.c_void_p((1 << 20) + 4), ok, ok, ok, ok, ok,
+                            ok, ok, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG
+    sh = _shape(batch=128, dstate=100)
+    rc = L.ssd_state_update(ctypes.byref(sh), ok, ok, ok, ok, ok, ok, ok, ok, None)
+    assert rc == ssd.SSD_ERR_UNSUPPORTED
+
+
+def test_product_path_has_no_cpu_fallback(tmp_path, monkeypatch):
+    """With the shared library absent, the binding raises instead of computing anything."""
+    monkeypatch.setattr(ssd, "_lib", None)
+    monkeypatch.setattr(ssd, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        ssd.lib()
