@@ -140,6 +140,36 @@ ssd_status ssd_state_update(const ssd_shape *shape, float *state, const void *x,
  */
 ssd_status ssd_workspace_status(const void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * The chunked scan for callers that cannot allocate device memory.  (No counterpart in the
+ * paper or on its pages: this is a deployment convenience of this library.)
+ *
+ * Some callers cannot call cudaMalloc -- or any allocator -- where they run the scan: code inside
+ * a framework's memory-planning or capture phase where the allocator is locked, a runtime that
+ * owns all device memory and hands out only the tensors it planned, or a host that forbids
+ * allocation after start-up.  They pass inputs and outputs exactly as for ssd_chunk_scan_fwd,
+ * but no workspace: the scan uses a fixed 32 MiB scratch array built into this library
+ * (resident on every GPU that loads the library until the process exits).
+ *
+ *   - Problems whose ssd_chunk_scan_workspace_size() exceeds 32 MiB (33554432 bytes) are
+ *     rejected with SSD_ERR_UNSUPPORTED and a message naming both sizes; e.g. batch 2 x 2048
+ *     tokens x 24 heads (headdim 64, dstate 128, chunk 256) needs about 19.3 MB and fits.
+ *   - The first call on each device, with that device current, looks up the array's device
+ *     address (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ *     capture.  The array of the calling thread's current device is used, so `stream` must
+ *     belong to that device.
+ *   - No memory is allocated or freed.  The array keeps the last call's contents; nothing in it
+ *     needs to start at zero (the scan clears its own status word).
+ *   - All calls on a device share the one array: calls whose kernels overlap on the GPU (other
+ *     streams, other host threads) race and corrupt each other's results.  Issue them one after
+ *     another on a single stream.
+ *   - Results are the same as ssd_chunk_scan_fwd's for the same arguments.
+ */
+ssd_status ssd_chunk_scan_fwd_static(const ssd_shape *shape, const void *x, const float *dt,
+                                     const float *A, const void *B, const void *C,
+                                     const float *D, int chunk_size, const float *init_state,
+                                     void *y, float *final_state, void *stream);
+
 /* Message for the calling thread's last non-OK status ("" if none). */
 const char *ssd_last_error(void);
 

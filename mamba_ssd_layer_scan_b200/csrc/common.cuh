@@ -27,6 +27,9 @@ struct WsLayout {
     size_t total;
 };
 
+// Sets the calling thread's message returned by ssd_last_error().
+void set_last_error(const char *msg);
+
 // ---- launchers (each returns the launch's cudaError_t) ----
 // Also zeroes *status (nullable) so each scan starts with a clean status word.
 cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, int *status,

@@ -85,6 +85,8 @@ ssd::WsLayout layout(const ssd_shape *s, int Q)
 
 }  // namespace
 
+void ssd::set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
 extern "C" {
 
 const char *ssd_last_error(void) { return g_err; }

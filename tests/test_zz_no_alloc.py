@@ -1,0 +1,84 @@
+"""The no-allocation entry point, ssd_chunk_scan_fwd_static, against ssd_chunk_scan_fwd.
+
+Callers that may not allocate device memory where they run the scan -- a locked allocator
+inside a framework's planning or capture phase, a runtime that owns all device memory, a host
+with a fixed memory budget -- call ssd_chunk_scan_fwd_static.  It runs the same kernels but uses
+a scratch array built into the library instead of a caller-provided workspace.  These tests
+call it through the C ABI twice in a row (the second call must not be disturbed by what the
+first left in the shared array) and compare each result with the workspace entry point's, within
+the bf16 parity tolerance; they also check that problems larger than the array are refused.
+
+The file is named so that pytest collects it last: if it fails, a run that stops at the first
+failure has already run every other test.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+from mamba_ssd_layer_scan_b200 import configs, inputs, ssd
+
+from _util import TOL, max_rel_per_pair, to_np, torch_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _static_entry():
+    f = ssd.lib().ssd_chunk_scan_fwd_static
+    f.restype = ctypes.c_int
+    f.argtypes = ([ctypes.POINTER(ssd.Shape)] + [ctypes.c_void_p] * 6 + [ctypes.c_int]
+                  + [ctypes.c_void_p] * 4)
+    return f
+
+
+def _shape(w):
+    return ssd.make_shape(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                          ssd.SSD_BF16 if w.dtype == "bf16" else ssd.SSD_F32)
+
+
+def _call_static(torch, t, w, chunk):
+    y = torch.empty_like(t["x"])
+    final = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
+                        device=t["x"].device)
+    init = t["init_state"]
+    rc = _static_entry()(ctypes.byref(_shape(w)), t["x"].data_ptr(), t["dt"].data_ptr(),
+                         t["A"].data_ptr(), t["B"].data_ptr(), t["C"].data_ptr(),
+                         t["D"].data_ptr(), chunk, None if init is None else init.data_ptr(),
+                         y.data_ptr(), final.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert rc == ssd.SSD_OK, ssd.last_error()
+    return y, final
+
+
+def test_static_scratch_matches_workspace_entry_point_on_two_calls(cuda_device):
+    import torch
+    cases = [
+        (configs.SSD_370M, 256),   # batch 2 x 2048 x 24 heads: ~19.3 MB of scratch
+        (configs.SSD_370M.with_(seqlen=1500, nheads=16, init_state=True, seed=4242), 256),
+    ]
+    prepared = []
+    for w, chunk in cases:
+        t = torch_inputs(inputs.make_inputs(w), cuda_device)
+        y_ref, f_ref = ssd.chunk_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk,
+                                          init_state=t["init_state"])
+        prepared.append((w, chunk, t, y_ref, f_ref))
+    torch.cuda.synchronize()
+    outs = [_call_static(torch, t, w, chunk) for w, chunk, t, _, _ in prepared]  # two in a row
+    torch.cuda.synchronize()
+    for (w, chunk, t, y_ref, f_ref), (y, f) in zip(prepared, outs):
+        yn, yr = to_np(y), to_np(y_ref)
+        fn, fr = to_np(f), to_np(f_ref)
+        pairs = [(b, h) for b in range(w.batch) for h in range(w.nheads)]
+        ey = max_rel_per_pair([yn[b, :, h] for b, h in pairs], [yr[b, :, h] for b, h in pairs])
+        ef = max_rel_per_pair([fn[b, h] for b, h in pairs], [fr[b, h] for b, h in pairs])
+        assert np.isfinite(yn).all()
+        assert ey <= TOL[w.dtype], f"y differs from ssd_chunk_scan_fwd by {ey:.3e}"
+        assert ef <= TOL[w.dtype], f"final state differs from ssd_chunk_scan_fwd by {ef:.3e}"
+
+
+def test_static_scratch_refuses_problems_larger_than_the_array(cuda_device):
+    w = configs.SSD_2P7B   # ~257 MB of scratch needed
+    assert ssd.workspace_size(_shape(w), w.chunk) > 32 << 20
+    p = ctypes.c_void_p(1 << 20)
+    rc = _static_entry()(ctypes.byref(_shape(w)), p, p, p, p, p, p, w.chunk, None, p, None, None)
+    assert rc == ssd.SSD_ERR_UNSUPPORTED
+    assert "ssd_chunk_scan_fwd_static" in ssd.last_error()
