@@ -8,20 +8,23 @@
 // chunk) contribute dt = 0, so cs stays flat there and the chunk's total log-decay is always
 // cs[..][Q-1].  Resetting the sum at every chunk keeps its magnitude bounded by Q*max|dt*A|.
 //
-// One CTA per (32-head tile, chunk, batch): a coalesced load of the chunk's dt rows for the
-// 32 heads into shared memory, then one warp per head scans the Q values with shuffles.
+// One CTA per (8-head tile, chunk, batch): the chunk's dt rows for the 8 heads are staged in
+// shared memory, then one warp per head scans its Q values with shuffles.  When
+// dtc is given, dt is also written in the same (b, c, H, Q) layout as cs (0 past the end of the
+// sequence), so that the tensor-core kernels can fetch both per-head rows with one bulk copy.
 #include "common.cuh"
 
 namespace ssd {
 namespace {
 
-constexpr int kHeadTile = 32;
-constexpr int kThreads = 256;
+constexpr int kHeadTile = 8;     // heads per CTA, one warp each
+constexpr int kThreads = 32 * kHeadTile;
+constexpr int kMaxSeg = 8;       // Q <= 256 = 8 segments of 32 tokens
 
 __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(const float *__restrict__ dt, const float *__restrict__ A,
-                    float *__restrict__ cs, int *__restrict__ status, int64_t seqlen, int H,
-                    int Q, int64_t nchunks)
+                    float *__restrict__ cs, float *__restrict__ dtc, int *__restrict__ status,
+                    int64_t seqlen, int H, int Q, int64_t nchunks)
 {
     // First kernel of every scan: clears the workspace status word the later kernels may set.
     if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
@@ -38,26 +41,41 @@ chunk_cumsum_kernel(const float *__restrict__ dt, const float *__restrict__ A,
         const int tau = idx / kHeadTile, j = idx % kHeadTile;
         float v = 0.f;
         if (tau < len && j < nh)
-            v = dt[(b * seqlen + t0 + tau) * H + h0 + j] * A[h0 + j];
+            v = dt[(b * seqlen + t0 + tau) * H + h0 + j];
         tile[tau * (kHeadTile + 1) + j] = v;
     }
     __syncthreads();
 
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    for (int j = warp; j < nh; j += kThreads / 32) {
-        float *out = cs + ((b * nchunks + k) * H + h0 + j) * (int64_t)Q;
-        float carry = 0.f;
-        for (int s = 0; s < Q; s += 32) {
-            float v = (s + lane < Q) ? tile[(s + lane) * (kHeadTile + 1) + j] : 0.f;
+    const int j = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (j >= nh) return;
+    const int64_t row = ((b * nchunks + k) * H + h0 + j) * (int64_t)Q;
+    const float Ah = A[h0 + j];
+    const int nseg = (Q + 31) / 32;
+    // Independent inclusive scans of every 32-token segment (interleaved for ILP), then the
+    // segment totals are carried forward.
+    float v[kMaxSeg];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float n = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += n;
-            }
-            v += carry;
-            if (s + lane < Q) out[s + lane] = v;
-            carry = __shfl_sync(0xffffffffu, v, 31);
+    for (int sg = 0; sg < kMaxSeg; ++sg) {
+        const int tau = sg * 32 + lane;
+        const float d = (sg < nseg && tau < Q) ? tile[tau * (kHeadTile + 1) + j] : 0.f;
+        if (dtc && sg < nseg && tau < Q) dtc[row + tau] = d;
+        v[sg] = d * Ah;
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+        for (int sg = 0; sg < kMaxSeg; ++sg) {
+            const float n = __shfl_up_sync(0xffffffffu, v[sg], o);
+            if (lane >= o) v[sg] += n;
         }
+    }
+    float carry = 0.f;
+#pragma unroll
+    for (int sg = 0; sg < kMaxSeg; ++sg) {
+        const float total = __shfl_sync(0xffffffffu, v[sg], 31);
+        const int tau = sg * 32 + lane;
+        if (sg < nseg && tau < Q) cs[row + tau] = v[sg] + carry;
+        carry += total;
     }
 }
 
@@ -70,14 +88,14 @@ __global__ void fill_final_kernel(const float *__restrict__ init, float *__restr
 
 }  // namespace
 
-cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, int *status,
-                                int64_t batch, int64_t seqlen, int nheads, int Q,
+cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, float *dtc,
+                                int *status, int64_t batch, int64_t seqlen, int nheads, int Q,
                                 int64_t nchunks, cudaStream_t st)
 {
     const unsigned grid = (unsigned)(((nheads + kHeadTile - 1) / kHeadTile) * nchunks * batch);
     const size_t smem = (size_t)Q * (kHeadTile + 1) * sizeof(float);
-    chunk_cumsum_kernel<<<grid, kThreads, smem, st>>>(dt, A, cs, status, seqlen, nheads, Q,
-                                                      nchunks);
+    chunk_cumsum_kernel<<<grid, kThreads, smem, st>>>(dt, A, cs, dtc, status, seqlen, nheads,
+                                                      Q, nchunks);
     return cudaGetLastError();
 }
 

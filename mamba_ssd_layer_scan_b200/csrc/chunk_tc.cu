@@ -59,24 +59,29 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // ============================================================ chunk state
+constexpr int kStateStages = 4;
 struct alignas(1024) StateSmem {
-    bf16 Bs[2][256 * 64];          // MN-major A operand: [n atom][Q rows tau][64 n]
-    bf16 Xs[2][256 * 64];          // MN-major B operand per stage: [Q rows tau][64 p]
+    bf16 Bs[2][256 * 64];                 // MN-major A operand: [n atom][Q rows tau][64 n]
+    bf16 Xs[kStateStages][256 * 64];      // MN-major B operand per stage: [Q rows tau][64 p]
+    float cs_v[kStateStages][256];        // per stage: the head's chunk-local cumsum row
+    float dt_v[kStateStages][256];        // per stage: the head's dt row (0 past the end)
     uint64_t bar_b;
-    uint64_t bar_x_full[2], bar_x_ready[2], bar_mma_done[2], bar_acc_free[2];
+    uint64_t bar_x_full[kStateStages], bar_x_ready[kStateStages], bar_x_free[kStateStages];
+    uint64_t bar_acc_full[2], bar_acc_free[2];
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort;
 };
-constexpr int kStateThreads = 256;
+// warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warp 3 idle, warps 4-11 scale x, warps 12-15 epilogue
+constexpr int kStateThreads = 512;
+constexpr int kStateScaleThreads = 256;
 constexpr uint32_t kStateTmemCols = 128;
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
-                      const __grid_constant__ CUtensorMap tm_b, const float *__restrict__ dt,
+                      const __grid_constant__ CUtensorMap tm_b, const float *__restrict__ dtc,
                       const float *__restrict__ cs, float *__restrict__ states,
-                      int *__restrict__ status, int64_t seqlen, int H, int G, int Q,
-                      int64_t nchunks, int nhb)
+                      int *__restrict__ status, int H, int G, int Q, int64_t nchunks, int nhb)
 {
     extern __shared__ uint8_t smem_raw[];
     StateSmem &sm = *reinterpret_cast<StateSmem *>(
@@ -91,15 +96,17 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int h0 = g * hpg + hb * kHeadsPerCta;
     const int nh = min(kHeadsPerCta, hpg - hb * kHeadsPerCta);
     const int64_t t0 = k * Q;
-    const int len = (int)min((int64_t)Q, seqlen - t0);
     const int nrb = Q / kTileRows;
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_b, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kStateStages; ++s) {
             mbar_init(&sm.bar_x_full[s], 1);
-            mbar_init(&sm.bar_x_ready[s], 128);
-            mbar_init(&sm.bar_mma_done[s], 1);
+            mbar_init(&sm.bar_x_ready[s], kStateScaleThreads);
+            mbar_init(&sm.bar_x_free[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.bar_acc_full[s], 1);
             mbar_init(&sm.bar_acc_free[s], 128);
         }
         mbar_init(&sm.bar_drain, 1);
@@ -117,7 +124,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     volatile int *abort = &sm.abort;
 
     if (warp == 0) {
-        // ---------------- TMA producer
+        // ---------------- TMA producer: B once, then per head its x tile and cs / dt rows
         if (lane == 0) {
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
@@ -128,14 +135,17 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                                 (int)(t0 + kTileRows * r), (int)b);
         }
         for (int j = 0; j < nh; ++j) {
-            const int s = j & 1;
-            const uint32_t use = j >> 1;
-            if (j >= 2 && !warp_wait(&sm.bar_mma_done[s], (use - 1) & 1, abort)) break;
+            const int s = j % kStateStages;
+            const uint32_t use = j / kStateStages;
+            if (j >= kStateStages && !warp_wait(&sm.bar_x_free[s], (use - 1) & 1, abort)) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.bar_x_full[s], (uint32_t)Q * kRowBytes);
+                const int64_t vrow = ((b * nchunks + k) * H + h0 + j) * (int64_t)Q;
+                mbar_arrive_expect_tx(&sm.bar_x_full[s], (uint32_t)Q * (kRowBytes + 8));
                 for (int r = 0; r < nrb; ++r)
                     tma_load_4d(&sm.Xs[s][r * kTileRows * 64], &tm_x, &sm.bar_x_full[s], 0,
                                 h0 + j, (int)(t0 + kTileRows * r), (int)b);
+                bulk_load(sm.cs_v[s], cs + vrow, Q * 4, &sm.bar_x_full[s]);
+                bulk_load(sm.dt_v[s], dtc + vrow, Q * 4, &sm.bar_x_full[s]);
             }
             __syncwarp();
         }
@@ -145,77 +155,73 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         const uint32_t atom_bytes = 256 * kRowBytes;  // distance between the two n atoms of Bs
         if (warp_wait(&sm.bar_b, 0, abort)) {
             for (int j = 0; j < nh; ++j) {
-                const int s = j & 1;
-                const uint32_t use = j >> 1;
+                const int s = j % kStateStages;
+                const uint32_t use = j / kStateStages;
+                const int a = j & 1;
                 if (!warp_wait(&sm.bar_x_ready[s], use & 1, abort)) break;
-                if (j >= 2 && !warp_wait(&sm.bar_acc_free[s], (use - 1) & 1, abort)) break;
+                if (j >= 2 && !warp_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t d = tmem + s * kP;
+                    const uint32_t d = tmem + a * kP;
                     const uint32_t a0 = smem_u32(&sm.Bs[0][0]), b0 = smem_u32(&sm.Xs[s][0]);
                     for (int kk = 0; kk < Q / 16; ++kk) {
                         const uint64_t ad = smem_desc_sw128(a0 + kk * 2048, atom_bytes, 1024);
                         const uint64_t bd = smem_desc_sw128(b0 + kk * 2048, atom_bytes, 1024);
                         mma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
                     }
-                    mma_commit(&sm.bar_mma_done[s]);
+                    mma_commit(&sm.bar_x_free[s]);
+                    mma_commit(&sm.bar_acc_full[a]);
                 }
                 __syncwarp();
             }
         }
-    } else if (warp >= 4) {
-        // ---------------- scale x rows by w, then TMEM -> global epilogue of the previous head
-        const int et = threadIdx.x - 128;
-        const int q = warp & 3;
-        for (int j = 0; j <= nh; ++j) {
-            if (j < nh) {
-                const int s = j & 1;
-                const uint32_t use = j >> 1;
-                if (!warp_wait(&sm.bar_x_full[s], use & 1, abort)) break;
-                const int h = h0 + j;
-                const float *csk = cs + ((b * nchunks + k) * H + h) * (int64_t)Q;
-                const float cs_last = csk[Q - 1];
-                for (int tau = et; tau < Q; tau += 128) {
-                    float w = 0.f;
-                    if (tau < len)
-                        w = __expf(cs_last - csk[tau]) * dt[(b * seqlen + t0 + tau) * H + h];
-                    uint4 *row = reinterpret_cast<uint4 *>(&sm.Xs[s][tau * 64]);
+    } else if (warp >= 4 && warp < 12) {
+        // ---------------- scale x rows by w_tau = exp(cs_last - cs_tau) dt_tau (in place)
+        const int st = threadIdx.x - 128;             // 0..255
+        const int chunks = Q * 8;                     // 16-byte pieces of the tile
+        for (int j = 0; j < nh; ++j) {
+            const int s = j % kStateStages;
+            const uint32_t use = j / kStateStages;
+            if (!warp_wait(&sm.bar_x_full[s], use & 1, abort)) break;
+            const float cs_last = sm.cs_v[s][Q - 1];
+            for (int c = st; c < chunks; c += kStateScaleThreads) {
+                const int tau = c >> 3;
+                const float w = __expf(cs_last - sm.cs_v[s][tau]) * sm.dt_v[s][tau];
+                uint4 *ptr = reinterpret_cast<uint4 *>(&sm.Xs[s][0]) + c;
+                uint4 v = *ptr;
+                uint32_t *wv = &v.x;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint4 v = row[c];
-                        uint32_t *wv = &v.x;
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(
-                                *reinterpret_cast<const __nv_bfloat162 *>(&wv[e]));
-                            wv[e] = pack_bf16x2(f.x * w, f.y * w);
-                        }
-                        row[c] = v;
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162 *>(&wv[e]));
+                    const float2 sc = fmul2(f, make_float2(w, w));
+                    wv[e] = pack_bf16x2(sc.x, sc.y);
                 }
-                fence_async_smem();
-                mbar_arrive(&sm.bar_x_ready[s]);
+                *ptr = v;
             }
-            if (j >= 1) {
-                const int jj = j - 1;
-                const int s = jj & 1;
-                const uint32_t use = jj >> 1;
-                if (!warp_wait(&sm.bar_mma_done[s], use & 1, abort)) break;
-                tc_fence_after();
-                uint32_t r0[32], r1[32];
-                const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + s * kP;
-                tmem_ld32(taddr, r0);
-                tmem_ld32(taddr + 32, r1);
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(&sm.bar_acc_free[s]);
-                const int n = q * 32 + lane;
-                float *out = states + ((b * nchunks + k) * H + h0 + jj) * (int64_t)(kP * kN) + n;
+            fence_async_smem();
+            mbar_arrive(&sm.bar_x_ready[s]);
+        }
+    } else if (warp >= 12) {
+        // ---------------- epilogue: TMEM (lane n, column p) -> states[b][k][h][p][n]
+        const int q = warp & 3;
+        for (int j = 0; j < nh; ++j) {
+            const int a = j & 1;
+            if (!warp_wait(&sm.bar_acc_full[a], (j >> 1) & 1, abort)) break;
+            tc_fence_after();
+            uint32_t r0[32], r1[32];
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + a * kP;
+            tmem_ld32(taddr, r0);
+            tmem_ld32(taddr + 32, r1);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_acc_free[a]);
+            const int n = q * 32 + lane;
+            float *out = states + ((b * nchunks + k) * H + h0 + j) * (int64_t)(kP * kN) + n;
 #pragma unroll
-                for (int p = 0; p < 32; ++p) out[p * kN] = __uint_as_float(r0[p]);
+            for (int p = 0; p < 32; ++p) out[p * kN] = __uint_as_float(r0[p]);
 #pragma unroll
-                for (int p = 0; p < 32; ++p) out[(32 + p) * kN] = __uint_as_float(r1[p]);
-            }
+            for (int p = 0; p < 32; ++p) out[(32 + p) * kN] = __uint_as_float(r1[p]);
         }
     }
 
@@ -240,33 +246,49 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
 }
 
 // ============================================================ chunk scan (intra-chunk + off-chunk)
-constexpr int kRing = 4;
+constexpr int kXStages = 3;      // x / h_in stages; the third lives in the B tile's space
+constexpr int kVecStages = 4;    // cs / dt row stages
+constexpr int kRing = 4;         // 64-column blocks of P in TMEM
+constexpr int kStageBytes = 256 * kRowBytes + 2 * kP * kRowBytes;  // x (<= 256 rows) + h_in
 struct alignas(1024) ScanSmem {
     bf16 Cs[2][kTileRows * 64];     // K-major A (C tile): [n atom][128 rows t][64 n]
-    bf16 Ring[kRing][kTileRows * 64];  // first B rows (K-major [n atom][KI rows][64]), then the
-                                       // P blocks (K-major [128 rows t][64 columns i] per slot)
-    bf16 Xs[2][256 * 64];           // MN-major B operand per stage: [KI rows i][64 p]
-    bf16 Hs[2][2][kP * 64];         // K-major B operand per stage: [n atom][64 rows p][64 n]
-    float cs_w[4][256];             // per mask warp: log2-scaled cs of the current head
-    float dt_w[4][256];             // per mask warp: dt (0 past the end of the sequence)
-    float vt[4][256];               // per mask warp: exp2(cs_r - cs_i) * dt_i
+    uint8_t R[kStageBytes + 16384]; // B rows for C B^T (K-major [n atom][KI rows][64]); after
+                                    // that, x / h_in stage 2
+    uint8_t S01[2][kStageBytes];    // x / h_in stages 0 and 1: [KI rows i][64 p] then
+                                    // [n atom][64 rows p][64 n]
+    float cs_v[kVecStages][256];    // per stage: the head's chunk-local cumsum row
+    float dt_v[kVecStages][256];    // per stage: the head's dt row (0 past the end)
+    float vt[8][256];               // per mask warp: exp(cs_r - cs_i) dt_i
+    float Dv[kHeadsPerCta];         // D of the CTA's heads
     uint64_t bar_cb, bar_g;
-    uint64_t bar_xh_full[2], bar_xh_free[2];
+    uint64_t bar_xh_full[kXStages], bar_xh_free[kXStages];
+    uint64_t bar_vec_full[kVecStages], bar_vec_free[kVecStages];
     uint64_t bar_slot_full[kRing], bar_slot_free[kRing];
-    uint64_t bar_acc_full[2], bar_acc_free[2];
+    uint64_t bar_acc_full, bar_acc_free;
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort;
 };
-constexpr int kScanThreads = 384;
+// warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warp 3 idle, warps 4-11 mask (two per TMEM lane
+// quarter, splitting each 64-column block), warps 12-15 epilogue
+constexpr int kScanThreads = 512;
 constexpr uint32_t kScanTmemCols = 512;
-constexpr uint32_t kAccCol = 256;   // acc1[s] = 256 + 128 s, acc2[s] = acc1[s] + 64
+constexpr uint32_t kPCol = 256;     // P ring: block slot s at columns [256 + 32 s, +32)
+constexpr uint32_t kAccCol = 384;   // Y1 at [384, 448), Y2 at [448, 512)
+
+static_assert(sizeof(StateSmem) + 1024 <= 232448, "chunk state smem exceeds 227 KB");
+static_assert(sizeof(ScanSmem) + 1024 <= 232448, "chunk scan smem exceeds 227 KB");
+
+__device__ __forceinline__ uint8_t *scan_stage(ScanSmem &sm, int s)
+{
+    return s < 2 ? sm.S01[s] : sm.R;
+}
 
 __global__ void __launch_bounds__(kScanThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c,
-                     const __grid_constant__ CUtensorMap tm_h, const float *__restrict__ dt,
+                     const __grid_constant__ CUtensorMap tm_h, const float *__restrict__ dtc,
                      const float *__restrict__ cs, const float *__restrict__ D,
                      bf16 *__restrict__ y, int *__restrict__ status, int64_t seqlen, int H,
                      int G, int Q, int64_t nchunks, int nhb)
@@ -294,20 +316,25 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_cb, 1);
         mbar_init(&sm.bar_g, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kXStages; ++s) {
             mbar_init(&sm.bar_xh_full[s], 1);
             mbar_init(&sm.bar_xh_free[s], 1);
-            mbar_init(&sm.bar_acc_full[s], 1);
-            mbar_init(&sm.bar_acc_free[s], 128);
+        }
+        for (int s = 0; s < kVecStages; ++s) {
+            mbar_init(&sm.bar_vec_full[s], 1);
+            mbar_init(&sm.bar_vec_free[s], 256 + 128);
         }
         for (int s = 0; s < kRing; ++s) {
-            mbar_init(&sm.bar_slot_full[s], 128);
+            mbar_init(&sm.bar_slot_full[s], 256);
             mbar_init(&sm.bar_slot_free[s], 1);
         }
+        mbar_init(&sm.bar_acc_full, 1);
+        mbar_init(&sm.bar_acc_free, 128);
         mbar_init(&sm.bar_drain, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
+    if (threadIdx.x >= 32 && threadIdx.x < 32 + nh) sm.Dv[threadIdx.x - 32] = D[h0 + threadIdx.x - 32];
     if (warp == 2) {
         tmem_alloc(&sm.tmem_base, kScanTmemCols);
         tmem_relinquish();
@@ -317,7 +344,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort = &sm.abort;
-    uint8_t *ring = reinterpret_cast<uint8_t *>(&sm.Ring[0][0]);
 
     if (warp == 0) {
         // ---------------- TMA producer
@@ -332,23 +358,35 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                             (int)(t0 + kTileRows * T), (int)b);
             for (int a = 0; a < 2; ++a)
                 for (int r = 0; r <= T; ++r)
-                    tma_load_4d(ring + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
+                    tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
                                 64 * a, g, (int)(t0 + kTileRows * r), (int)b);
         }
         for (int j = 0; j < nh; ++j) {
-            const int s = j & 1;
-            const uint32_t use = j >> 1;
-            if (j >= 2 && !warp_wait(&sm.bar_xh_free[s], (use - 1) & 1, abort)) break;
+            const int h = h0 + j;
+            const int vs = j % kVecStages;
+            const uint32_t vu = j / kVecStages;
+            if (j >= kVecStages && !warp_wait(&sm.bar_vec_free[vs], (vu - 1) & 1, abort)) break;
             if (lane == 0) {
-                const int h = h0 + j;
-                mbar_arrive_expect_tx(&sm.bar_xh_full[s],
+                const int64_t vrow = ((b * nchunks + k) * H + h) * (int64_t)Q;
+                mbar_arrive_expect_tx(&sm.bar_vec_full[vs], (uint32_t)(8 * Q));
+                bulk_load(sm.cs_v[vs], cs + vrow, Q * 4, &sm.bar_vec_full[vs]);
+                bulk_load(sm.dt_v[vs], dtc + vrow, Q * 4, &sm.bar_vec_full[vs]);
+            }
+            const int xs = j % kXStages;
+            const uint32_t xu = j / kXStages;
+            if (j >= kXStages && !warp_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) break;
+            if (xs == 2 && xu == 0 && !warp_wait(&sm.bar_g, 0, abort)) break;  // B tile in use
+            if (lane == 0) {
+                uint8_t *stg = scan_stage(sm, xs);
+                mbar_arrive_expect_tx(&sm.bar_xh_full[xs],
                                       (uint32_t)(KI * kRowBytes + 2 * kP * kRowBytes));
                 for (int r = 0; r <= T; ++r)
-                    tma_load_4d(&sm.Xs[s][r * kTileRows * 64], &tm_x, &sm.bar_xh_full[s], 0, h,
+                    tma_load_4d(stg + r * kBoxBytes, &tm_x, &sm.bar_xh_full[xs], 0, h,
                                 (int)(t0 + kTileRows * r), (int)b);
                 const int hrow = (int)(((b * nchunks + k) * H + h) * kP);
                 for (int a = 0; a < 2; ++a)
-                    tma_load_2d(&sm.Hs[s][a][0], &tm_h, &sm.bar_xh_full[s], 64 * a, hrow);
+                    tma_load_2d(stg + 256 * kRowBytes + a * kP * kRowBytes, &tm_h,
+                                &sm.bar_xh_full[xs], 64 * a, hrow);
             }
             __syncwarp();
         }
@@ -358,7 +396,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         const uint32_t id_h = idesc_bf16_f32(128, kP, false, false);
         const uint32_t id_y = idesc_bf16_f32(128, kP, false, true);
         const uint32_t c0 = smem_u32(&sm.Cs[0][0]);
-        const uint32_t rg = smem_u32(ring);
+        const uint32_t rg = smem_u32(sm.R);
         bool ok = warp_wait(&sm.bar_cb, 0, abort);
         if (ok) {
             tc_fence_after();
@@ -374,38 +412,37 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             }
             __syncwarp();
         }
+        const uint32_t d1 = tmem + kAccCol, d2 = tmem + kAccCol + 64;
         uint32_t blk = 0;
         for (int j = 0; ok && j < nh; ++j) {
-            const int s = j & 1;
-            const uint32_t use = j >> 1;
-            if (!warp_wait(&sm.bar_xh_full[s], use & 1, abort)) break;
-            if (j >= 2 && !warp_wait(&sm.bar_acc_free[s], (use - 1) & 1, abort)) break;
+            const int xs = j % kXStages;
+            const uint32_t xu = j / kXStages;
+            if (!warp_wait(&sm.bar_xh_full[xs], xu & 1, abort)) break;
+            if (j >= 1 && !warp_wait(&sm.bar_acc_free, (j - 1) & 1, abort)) break;
             tc_fence_after();
-            const uint32_t d1 = tmem + kAccCol + 128 * s, d2 = d1 + 64;
+            const uint32_t stg = smem_u32(scan_stage(sm, xs));
             if (lane == 0) {
                 // Y2 = C h_in^T: M = 128, N = 64 (p), K = 128 (n)
-                const uint32_t h0a = smem_u32(&sm.Hs[s][0][0]);
                 for (int kk = 0; kk < kN / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    const uint32_t hoff = (kk >> 2) * (kP * kRowBytes) + (kk & 3) * 32;
+                    const uint32_t hoff = 256 * kRowBytes + (kk >> 2) * (kP * kRowBytes) +
+                                          (kk & 3) * 32;
                     mma_bf16(d2, smem_desc_sw128(c0 + off, 16, 1024),
-                             smem_desc_sw128(h0a + hoff, 16, 1024), id_h, kk > 0 ? 1u : 0u);
+                             smem_desc_sw128(stg + hoff, 16, 1024), id_h, kk > 0 ? 1u : 0u);
                 }
             }
             __syncwarp();
-            const uint32_t xs = smem_u32(&sm.Xs[s][0]);
             for (int qb = 0; qb < nblk; ++qb, ++blk) {
                 const uint32_t slot = blk % kRing, su = blk / kRing;
                 if (!warp_wait(&sm.bar_slot_full[slot], su & 1, abort)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
-                    // Y1 += P[:, 64qb : 64qb+64] X[64qb : 64qb+64, :]
-                    const uint32_t pa = rg + slot * kBoxBytes;
+                    // Y1 += P[:, 64qb : 64qb+64] X[64qb : 64qb+64, :], P read from TMEM
+                    const uint32_t pa = tmem + kPCol + 32 * slot;
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = smem_desc_sw128(pa + kk * 32, 16, 1024);
                         const uint64_t bd =
-                            smem_desc_sw128(xs + (qb * 4 + kk) * 2048, 256 * kRowBytes, 1024);
-                        mma_bf16(d1, ad, bd, id_y, (qb | kk) != 0 ? 1u : 0u);
+                            smem_desc_sw128(stg + (qb * 4 + kk) * 2048, 256 * kRowBytes, 1024);
+                        mma_bf16_ts(d1, pa + 8 * kk, bd, id_y, (qb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit(&sm.bar_slot_free[slot]);
                 }
@@ -413,42 +450,40 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             }
             if (!ok) break;
             if (lane == 0) {
-                mma_commit(&sm.bar_acc_full[s]);
-                mma_commit(&sm.bar_xh_free[s]);
+                mma_commit(&sm.bar_acc_full);
+                mma_commit(&sm.bar_xh_free[xs]);
             }
             __syncwarp();
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4 && warp < 12) {
         // ---------------- mask: P[t][i] = G[t][i] exp(cs_t - cs_i) dt_i (i <= t), + D at i = t
         const int qd = warp & 3;
+        const int half = (warp - 4) >> 2;          // which 32 columns of each 64-column block
         const int t = qd * 32 + lane;             // row within the tile = TMEM lane
         const int tau = kTileRows * T + t;        // row within the chunk
         const int r = kTileRows * T + qd * 32 - 1;  // reference row for the factorised decay
         const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
-        float *cs_s = sm.cs_w[qd];
-        float *dt_s = sm.dt_w[qd];
+        float *vt = sm.vt[warp - 4];
         bool ok = warp_wait(&sm.bar_g, 0, abort);
         tc_fence_after();
         uint32_t blk = 0;
         for (int j = 0; ok && j < nh; ++j) {
-            const int h = h0 + j;
-            const float *csk = cs + ((b * nchunks + k) * H + h) * (int64_t)Q;
-            // Each mask warp keeps its own copy of the head's cs and dt, so the four warps never
-            // wait on one another (only on mbarriers, whose waits are bounded).
-            __syncwarp();
-            for (int i = lane; i < KI; i += 32) {
-                cs_s[i] = csk[i] * kLog2e;
-                dt_s[i] = (i < len) ? dt[(b * seqlen + t0 + i) * H + h] : 0.f;
-            }
-            __syncwarp();
-            const float Dh = D[h];
+            const int vs = j % kVecStages;
+            if (!warp_wait(&sm.bar_vec_full[vs], (j / kVecStages) & 1, abort)) break;
+            const float *cs_s = sm.cs_v[vs];
+            const float *dt_s = sm.dt_v[vs];
+            const float Dh = sm.Dv[j];
             const float ct = cs_s[tau];
             float uf = 0.f;
+            __syncwarp();
             if (r >= 0) {
                 const float cr = cs_s[r];
-                for (int i = lane; i <= r; i += 32)
-                    sm.vt[qd][i] = exp2f(cr - cs_s[i]) * dt_s[i];
-                uf = exp2f(ct - cr);
+                // v for the columns of this warp's off-diagonal sub-blocks
+                for (int qb = 0; qb < nblk; ++qb) {
+                    const int i = qb * 64 + half * 32 + lane;
+                    if (i <= r) vt[i] = __expf(cr - cs_s[i]) * dt_s[i];
+                }
+                uf = __expf(ct - cr);
             }
             __syncwarp();
             for (int qb = 0; qb < nblk; ++qb, ++blk) {
@@ -457,90 +492,91 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     ok = false;
                     break;
                 }
-                uint8_t *prow = ring + slot * kBoxBytes + t * kRowBytes;
+                const int col0 = qb * 64 + half * 32;
+                uint32_t pk[16];
+                if (col0 + 32 <= r + 1) {
+                    uint32_t gv[32];
+                    tmem_ld32(lane_base + col0, gv);
+                    tmem_ld_wait();
+                    const float2 uu = make_float2(uf, uf);
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int col0 = qb * 64 + hf * 32;
-                    uint32_t pk[16];
-                    if (col0 + 32 <= r + 1) {
-                        uint32_t gv[32];
-                        tmem_ld32(lane_base + col0, gv);
-                        tmem_ld_wait();
-                        const float *vrow = &sm.vt[qd][col0];
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 vv = *reinterpret_cast<const float4 *>(vt + col0 + 4 * c);
+                        const float2 p0 = fmul2(fmul2(make_float2(__uint_as_float(gv[4 * c]),
+                                                                  __uint_as_float(gv[4 * c + 1])),
+                                                      make_float2(vv.x, vv.y)), uu);
+                        const float2 p1 = fmul2(fmul2(make_float2(__uint_as_float(gv[4 * c + 2]),
+                                                                  __uint_as_float(gv[4 * c + 3])),
+                                                      make_float2(vv.z, vv.w)), uu);
+                        pk[2 * c] = pack_bf16x2(p0.x, p0.y);
+                        pk[2 * c + 1] = pack_bf16x2(p1.x, p1.y);
+                    }
+                } else if (col0 == r + 1) {
+                    uint32_t gv[32];
+                    tmem_ld32(lane_base + col0, gv);
+                    tmem_ld_wait();
+                    float pv[32];
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const float2 vv = *reinterpret_cast<const float2 *>(vrow + 2 * c);
-                            pk[c] = pack_bf16x2(__uint_as_float(gv[2 * c]) * vv.x * uf,
-                                                __uint_as_float(gv[2 * c + 1]) * vv.y * uf);
-                        }
-                    } else if (col0 == r + 1) {
-                        uint32_t gv[32];
-                        tmem_ld32(lane_base + col0, gv);
-                        tmem_ld_wait();
-                        float pv[32];
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            const int i = col0 + c;
-                            float v = 0.f;
-                            if (i <= tau)
-                                v = __uint_as_float(gv[c]) * exp2f(ct - cs_s[i]) * dt_s[i];
-                            if (i == tau) v += Dh;
-                            pv[c] = v;
-                        }
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) pk[c] = 0u;
+                    for (int c = 0; c < 32; ++c) {
+                        const int i = col0 + c;
+                        float v = 0.f;
+                        if (i <= tau)
+                            v = __uint_as_float(gv[c]) * __expf(ct - cs_s[i]) * dt_s[i];
+                        if (i == tau) v += Dh;
+                        pv[c] = v;
                     }
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const int pos = (hf * 4 + m) ^ (t & 7);
-                        *reinterpret_cast<uint4 *>(prow + pos * 16) =
-                            make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
-                    }
+                    for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) pk[c] = 0u;
                 }
-                fence_async_smem();
+                tmem_st16(lane_base + kPCol + 32 * slot + 16 * half, pk);
+                tmem_st_wait();
+                tc_fence_before();
                 mbar_arrive(&sm.bar_slot_full[slot]);
             }
+            if (ok) mbar_arrive(&sm.bar_vec_free[vs]);   // done with this stage's cs / dt
         }
-    } else if (warp >= 8) {
+    } else if (warp >= 12) {
         // ---------------- epilogue: y = Y1 + exp(cs_t) Y2
         const int qd = warp & 3;
         const int t = qd * 32 + lane;
         const int tau = kTileRows * T + t;
         const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
         for (int j = 0; j < nh; ++j) {
-            const int s = j & 1;
-            const uint32_t use = j >> 1;
-            if (!warp_wait(&sm.bar_acc_full[s], use & 1, abort)) break;
+            if (!warp_wait(&sm.bar_acc_full, j & 1, abort)) break;
             tc_fence_after();
-            const int h = h0 + j;
-            const float e = (tau < len)
-                ? __expf(cs[((b * nchunks + k) * H + h) * (int64_t)Q + tau]) : 0.f;
-            uint4 *yrow = reinterpret_cast<uint4 *>(
-                y + ((b * seqlen + t0 + tau) * H + h) * (int64_t)kP);
+            const int vs = j % kVecStages;
+            if (!warp_wait(&sm.bar_vec_full[vs], (j / kVecStages) & 1, abort)) break;
+            const float e = __expf(sm.cs_v[vs][tau]);
+            mbar_arrive(&sm.bar_vec_free[vs]);              // done with this stage's cs
+            uint32_t a0[32], c0[32], pk[32];
+            tmem_ld32(lane_base + kAccCol, a0);
+            tmem_ld32(lane_base + kAccCol + 64, c0);
+            tmem_ld_wait();
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t a[32], c2[32];
-                tmem_ld32(lane_base + kAccCol + 128 * s + 32 * half, a);
-                tmem_ld32(lane_base + kAccCol + 128 * s + 64 + 32 * half, c2);
-                tmem_ld_wait();
-                if (tau < len) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        pk[c] = pack_bf16x2(
-                            fmaf(e, __uint_as_float(c2[2 * c]), __uint_as_float(a[2 * c])),
-                            fmaf(e, __uint_as_float(c2[2 * c + 1]), __uint_as_float(a[2 * c + 1])));
-#pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        yrow[half * 4 + m] =
-                            make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
-                }
-            }
+            for (int c = 0; c < 16; ++c)
+                pk[c] = pack_bf16x2(fmaf(e, __uint_as_float(c0[2 * c]), __uint_as_float(a0[2 * c])),
+                                    fmaf(e, __uint_as_float(c0[2 * c + 1]),
+                                         __uint_as_float(a0[2 * c + 1])));
+            tmem_ld32(lane_base + kAccCol + 32, a0);
+            tmem_ld32(lane_base + kAccCol + 96, c0);
+            tmem_ld_wait();
             tc_fence_before();
-            mbar_arrive(&sm.bar_acc_free[s]);
+            mbar_arrive(&sm.bar_acc_free);
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                pk[16 + c] = pack_bf16x2(
+                    fmaf(e, __uint_as_float(c0[2 * c]), __uint_as_float(a0[2 * c])),
+                    fmaf(e, __uint_as_float(c0[2 * c + 1]), __uint_as_float(a0[2 * c + 1])));
+            if (tau < len) {
+                uint4 *yrow = reinterpret_cast<uint4 *>(
+                    y + ((b * seqlen + t0 + tau) * H + h0 + j) * (int64_t)kP);
+#pragma unroll
+                for (int m = 0; m < 8; ++m)
+                    yrow[m] = make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+            }
         }
     }
 
@@ -612,7 +648,7 @@ bool tc_supported(bool is_bf16, int P, int N, int Q)
     return is_bf16 && P == kP && N == kN && (Q == 128 || Q == 256);
 }
 
-cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dt, const bf16 *B,
+cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
                                   cudaStream_t st, const char **why)
@@ -629,13 +665,13 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dt, const bf16 *B,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk state: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb);
-    chunk_state_tc_kernel<<<grid, kStateThreads, smem, st>>>(mx, mb, dt, cs, states, status,
-                                                             seqlen, H, G, Q, nchunks, nhb);
+    chunk_state_tc_kernel<<<grid, kStateThreads, smem, st>>>(mx, mb, dtc, cs, states, status,
+                                                             H, G, Q, nchunks, nhb);
     *why = "chunk state (tcgen05) launch";
     return cudaGetLastError();
 }
 
-cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dt, const bf16 *B, const bf16 *C,
+cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
                                  int Q, int64_t nchunks, cudaStream_t st, const char **why)
@@ -658,7 +694,7 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dt, const bf16 *B, 
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk scan: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb * (Q / kTileRows));
-    chunk_scan_tc_kernel<<<grid, kScanThreads, smem, st>>>(mx, mb, mc, mh, dt, cs, D, y, status,
+    chunk_scan_tc_kernel<<<grid, kScanThreads, smem, st>>>(mx, mb, mc, mh, dtc, cs, D, y, status,
                                                            seqlen, H, G, Q, nchunks, nhb);
     *why = "chunk scan (tcgen05) launch";
     return cudaGetLastError();

@@ -22,6 +22,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct WsLayout {
     size_t status;      // 256 bytes: device status word (nonzero after an in-kernel timeout)
     size_t cs;          // float [b][c][H][Q]: chunk-local inclusive cumsum of dt*A
+    size_t dtc;         // float [b][c][H][Q]: dt per chunk row, 0 past the end (tensor-core path)
     size_t states;      // float [b][c][H][P][N]: per-chunk state, then (in place) state entering
     size_t hin_bf16;    // bf16  [b][c][H][P][N]: state entering each chunk (tensor-core path)
     size_t total;
@@ -31,9 +32,10 @@ struct WsLayout {
 void set_last_error(const char *msg);
 
 // ---- launchers (each returns the launch's cudaError_t) ----
-// Also zeroes *status (nullable) so each scan starts with a clean status word.
-cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, int *status,
-                                int64_t batch, int64_t seqlen, int nheads, int Q,
+// Also zeroes *status (nullable) so each scan starts with a clean status word, and, when dtc is
+// non-null, writes dt re-laid out as (b, c, H, Q) with zeros past the end of the sequence.
+cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, float *dtc,
+                                int *status, int64_t batch, int64_t seqlen, int nheads, int Q,
                                 int64_t nchunks, cudaStream_t st);
 
 cudaError_t launch_chunk_state_simt(bool is_bf16, const void *x, const float *dt,
@@ -63,11 +65,11 @@ cudaError_t launch_fill_final(const float *init, float *final_state, int64_t n,
 
 // Tensor-core (tcgen05 + TMA) path: bf16, P = 64, N = 128, Q in {128, 256}.
 bool tc_supported(bool is_bf16, int P, int N, int Q);
-cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dt, const bf16 *B,
+cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
                                   cudaStream_t st, const char **why);
-cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dt, const bf16 *B, const bf16 *C,
+cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
                                  int Q, int64_t nchunks, cudaStream_t st, const char **why);

@@ -76,9 +76,10 @@ ssd::WsLayout layout(const ssd_shape *s, int Q)
     ssd::WsLayout w;
     w.status = 0;
     w.cs = 256;
-    w.states = w.cs + round256(rows * Q * sizeof(float));
-    w.hin_bf16 = w.states + round256(rows * s->headdim * s->dstate * sizeof(float));
     const bool tc = ssd::tc_supported(s->dtype == SSD_BF16, (int)s->headdim, (int)s->dstate, Q);
+    w.dtc = w.cs + round256(rows * Q * sizeof(float));
+    w.states = w.dtc + (tc ? round256(rows * Q * sizeof(float)) : 0);
+    w.hin_bf16 = w.states + round256(rows * s->headdim * s->dstate * sizeof(float));
     w.total = w.hin_bf16 + (tc ? round256(rows * s->headdim * s->dstate * sizeof(uint16_t)) : 0);
     return w;
 }
@@ -165,15 +166,18 @@ ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, cons
     float *states = reinterpret_cast<float *>(ws + wl.states);
     cudaError_t e = record(stage_events, 0, cs_stream);
     if (e != cudaSuccess) return cuda_fail(e, "record stage event");
-    e = ssd::launch_chunk_cumsum(dt, A, cs, status, s.batch, s.seqlen, H, Q, nchunks, cs_stream);
+    const bool tc = ssd::tc_supported(bf, P, N, Q);
+    float *dtc = tc ? reinterpret_cast<float *>(ws + wl.dtc) : nullptr;
+    e = ssd::launch_chunk_cumsum(dt, A, cs, dtc, status, s.batch, s.seqlen, H, Q, nchunks,
+                                 cs_stream);
     if (e != cudaSuccess) return cuda_fail(e, "dA cumsum launch");
     if ((e = record(stage_events, 1, cs_stream)) != cudaSuccess)
         return cuda_fail(e, "record stage event");
 
-    if (ssd::tc_supported(bf, P, N, Q)) {
+    if (tc) {
         const char *why = "";
         ssd::bf16 *hin = reinterpret_cast<ssd::bf16 *>(ws + wl.hin_bf16);
-        e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dt, (const ssd::bf16 *)B, cs,
+        e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs,
                                        states, status, s.batch, s.seqlen, H, G, Q, nchunks,
                                        cs_stream, &why);
         if (e != cudaSuccess) return cuda_fail(e, why);
@@ -184,7 +188,7 @@ ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, cons
         if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
         if ((e = record(stage_events, 3, cs_stream)) != cudaSuccess)
             return cuda_fail(e, "record stage event");
-        e = ssd::launch_chunk_scan_tc((const ssd::bf16 *)x, dt, (const ssd::bf16 *)B,
+        e = ssd::launch_chunk_scan_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B,
                                       (const ssd::bf16 *)C, cs, hin, D, (ssd::bf16 *)y, status,
                                       s.batch, s.seqlen, H, G, Q, nchunks, cs_stream, &why);
         if (e != cudaSuccess) return cuda_fail(e, why);

@@ -41,8 +41,9 @@ def test_workspace_size_layout():
     b, L_, H, P, N, Q = 4, 4096, 80, 64, 128, 256
     c = L_ // Q
     ws = ssd.workspace_size(_shape(), Q)
-    # status word + cs (f32) + chunk states (f32) + bf16 entering states (tensor-core path)
-    expect = 256 + b * c * H * Q * 4 + b * c * H * P * N * 4 + b * c * H * P * N * 2
+    # status word + cs (f32) + per-chunk dt rows (f32) + chunk states (f32) + bf16 entering
+    # states (the last two regions only on the tensor-core path)
+    expect = 256 + 2 * b * c * H * Q * 4 + b * c * H * P * N * 4 + b * c * H * P * N * 2
     assert ws == expect
     # float32 inputs run the CUDA-core path, which keeps the entering state in place (no bf16 copy)
     ws32 = ssd.workspace_size(_shape(dtype=ssd.SSD_F32), Q)
