@@ -9,28 +9,25 @@
 // block matrix multiplications).  Two kernels:
 //
 // chunk_state_tc_kernel   S_k^T = B_k^T (w o X_k),  w_tau = exp(cs_last - cs_tau) dt_tau
-//     One CTA per (batch, chunk, group, block of heads).  The chunk's B rows are loaded once and
-//     shared by the heads of the block; per head, the x tile is TMA-loaded, scaled row by row
-//     by w (CUDA cores, in shared memory), and one M=128 (n) x N=64 (p) x K=Q MMA chain
-//     accumulates S^T in TMEM, double-buffered so that head j+1's MMAs run under head j's
-//     TMEM -> global epilogue.
+//     One CTA per (batch, chunk, group, block of 8 heads).  The chunk's B rows are loaded once
+//     and shared by the heads of the block; per head, the x tile and the head's cs / dt rows
+//     arrive by TMA (4 stages), 8 warps scale the x rows by w in shared memory, one
+//     M=128 (n) x N=64 (p) x K=Q MMA chain accumulates S^T in TMEM (double-buffered), and 4
+//     epilogue warps move it to global memory while the next head's MMAs run.
 //
 // chunk_scan_tc_kernel    y = (C B^T o L o dt + diag(D)) X  +  exp(cs) o (C h_in^T)
-//     One CTA per (batch, chunk, 128-row tile of the chunk, group, block of heads).  G = C B^T
-//     (128 x KI, KI = 128 * (tile + 1) causal columns) is computed once per CTA into TMEM and
-//     shared by the heads (all heads of a group see the same B, C).  Per head the mask warps
-//     read G from TMEM, apply the decay exp(cs_t - cs_i) dt_i (and D on the diagonal), round to
-//     bf16 and write 64-column blocks of the K-major A operand into a 4-slot shared-memory ring
-//     that the MMA thread consumes as it fills; the off-chunk term C h_in^T is a second TMEM
-//     accumulator; the epilogue warps combine both as y = Y1 + exp(cs_t) Y2 and store bf16.
-//     The decay is factorised to keep the exponentials off the inner loop: for columns i at or
-//     before r (the row just above the warp's 32-row slice), exp(cs_t - cs_i) = exp(cs_t - cs_r)
-//     * exp(cs_r - cs_i), both factors <= 1 (cs is non-increasing), so each element costs two
-//     multiplies; only the 32 x 32 diagonal block evaluates exp per element.
+//     One CTA per (batch, chunk, 128-row tile of the chunk, group, block of 8 heads).  C B^T is
+//     computed once per CTA and shared by the heads (all heads of a group see the same B, C).
+//     The diagonal 128 x 128 block of the masked matrix is built per head by 8 worker warps from
+//     TMEM and written back to TMEM as bf16 (a ring of 64-column blocks), where the MMAs read it
+//     as their A operand; for the second tile of a 256-token chunk the off-diagonal block is
+//     rank-1 in its decay and runs as a plain product with C B_off^T converted to bf16 once
+//     (see the section comment below).  The decay is factorised so that no element needs an
+//     exponential of its own.  The same worker warps then run the previous head's epilogue.
 //
 // Roles (warp-specialised; every wait is on an mbarrier and bounded, see sm100.cuh):
-//   state kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-7 scale + epilogue
-//   scan  kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-7 mask, warps 8-11 epilogue
+//   state kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-11 scale, 12-15 epilogue
+//   scan  kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-11 mask + epilogue
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -246,35 +243,50 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
 }
 
 // ============================================================ chunk scan (intra-chunk + off-chunk)
-constexpr int kXStages = 3;      // x / h_in stages; the third lives in the B tile's space
+//
+// Tile T of a chunk holds rows [128 T, 128 T + 128).  Its output splits into
+//   - the diagonal 128 x 128 block (source columns of the same tile): P = C B^T o L o dt (+ D on
+//     the diagonal), built elementwise by the mask warps and multiplied by x from TMEM;
+//   - for T = 1, the off-diagonal block (source columns [0, 128)): every source precedes every
+//     target, so with the reference row r = 127, exp(cs_t - cs_i) = u_t v_i, u_t = exp(cs_t -
+//     cs_127), v_i = exp(cs_127 - cs_i) (both <= 1), and the block's contribution is
+//     diag(u) (C B_off^T) diag(v dt) X_off: C B_off^T is converted to bf16 once per CTA and
+//     shared by all heads, X_off is scaled row-wise per head, and u is applied in the epilogue;
+//   - the off-chunk term exp(cs_t) C h_in^T = u_t C (exp(cs_127) h_in)^T, which (scaled h_in)
+//     accumulates into the same TMEM accumulator as the off-diagonal block.
+// So y = Y_diag + f_t Y_A with f_t = exp(cs_t) (T = 0) or u_t (T = 1).
+constexpr int kXStagesMax = 3;   // x / h_in stages (T = 0: 3, the third in the B tile's space;
+                                 // T = 1: 2, that space holds the bf16 off-diagonal block)
 constexpr int kVecStages = 4;    // cs / dt row stages
-constexpr int kRing = 4;         // 64-column blocks of P in TMEM
+constexpr int kRing = 4;         // 64-column blocks of P in TMEM (two heads)
 constexpr int kStageBytes = 256 * kRowBytes + 2 * kP * kRowBytes;  // x (<= 256 rows) + h_in
+constexpr int kHOff = 256 * kRowBytes;                              // h_in inside a stage
 struct alignas(1024) ScanSmem {
     bf16 Cs[2][kTileRows * 64];     // K-major A (C tile): [n atom][128 rows t][64 n]
     uint8_t R[kStageBytes + 16384]; // B rows for C B^T (K-major [n atom][KI rows][64]); after
-                                    // that, x / h_in stage 2
+                                    // that, T = 0: x / h_in stage 2; T = 1: bf16 C B_off^T
+                                    // (K-major [i atom][128 rows t][64 i])
     uint8_t S01[2][kStageBytes];    // x / h_in stages 0 and 1: [KI rows i][64 p] then
                                     // [n atom][64 rows p][64 n]
     float cs_v[kVecStages][256];    // per stage: the head's chunk-local cumsum row
     float dt_v[kVecStages][256];    // per stage: the head's dt row (0 past the end)
-    float vt[8][256];               // per mask warp: exp(cs_r - cs_i) dt_i
+    float vt[8][128];               // per mask warp: exp(cs_r - cs_i) dt_i over the tile
     float Dv[kHeadsPerCta];         // D of the CTA's heads
-    uint64_t bar_cb, bar_g;
-    uint64_t bar_xh_full[kXStages], bar_xh_free[kXStages];
+    uint64_t bar_cb, bar_g, bar_goff;
+    uint64_t bar_xh_full[kXStagesMax], bar_xh_free[kXStagesMax], bar_xv_ready[kXStagesMax];
     uint64_t bar_vec_full[kVecStages], bar_vec_free[kVecStages];
     uint64_t bar_slot_full[kRing], bar_slot_free[kRing];
-    uint64_t bar_acc_full, bar_acc_free;
+    uint64_t bar_acc_full[2], bar_acc_free[2];
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort;
 };
-// warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warp 3 idle, warps 4-11 mask (two per TMEM lane
-// quarter, splitting each 64-column block), warps 12-15 epilogue
-constexpr int kScanThreads = 512;
+// warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warp 3 idle, warps 4-11 workers: two per TMEM lane
+// quarter, each owning one 32-column half of every 64-column block; per head they build their
+// half of P (mask) and then run the epilogue of the previous head for their half of y
+constexpr int kScanThreads = 384;
 constexpr uint32_t kScanTmemCols = 512;
-constexpr uint32_t kPCol = 256;     // P ring: block slot s at columns [256 + 32 s, +32)
-constexpr uint32_t kAccCol = 384;   // Y1 at [384, 448), Y2 at [448, 512)
+constexpr uint32_t kAccCol = 256;   // accumulator buffer a: Y_diag at 256 + 128 a, Y_A at +64
 
 static_assert(sizeof(StateSmem) + 1024 <= 232448, "chunk state smem exceeds 227 KB");
 static_assert(sizeof(ScanSmem) + 1024 <= 232448, "chunk scan smem exceeds 227 KB");
@@ -282,6 +294,31 @@ static_assert(sizeof(ScanSmem) + 1024 <= 232448, "chunk scan smem exceeds 227 KB
 __device__ __forceinline__ uint8_t *scan_stage(ScanSmem &sm, int s)
 {
     return s < 2 ? sm.S01[s] : sm.R;
+}
+
+// Scale the 16-byte pieces [first, first + count * stride) of a bf16 smem tile in place; the
+// factor of piece c is f(c).  Works on any swizzled layout whose rows are whole 128-byte lines.
+template <int kCount, typename F>
+__device__ __forceinline__ void scale_pieces(uint8_t *base, int first, int stride, F f)
+{
+    float wf[kCount];
+#pragma unroll
+    for (int m = 0; m < kCount; ++m) wf[m] = f(first + m * stride);   // independent: overlap
+#pragma unroll
+    for (int m = 0; m < kCount; ++m) {
+        const int c = first + m * stride;
+        const float w = wf[m];
+        uint4 *ptr = reinterpret_cast<uint4 *>(base) + c;
+        uint4 v = *ptr;
+        uint32_t *wv = &v.x;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wv[e]));
+            const float2 sc = fmul2(x, make_float2(w, w));
+            wv[e] = pack_bf16x2(sc.x, sc.y);
+        }
+        *ptr = v;
+    }
 }
 
 __global__ void __launch_bounds__(kScanThreads, 1)
@@ -311,25 +348,32 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int len = (int)min((int64_t)Q, seqlen - t0);
     if (T * kTileRows >= len) return;  // tile entirely past the end of the sequence
     const int KI = kTileRows * (T + 1);  // causal source columns of this tile
-    const int nblk = KI / 64;
+    const int nst = T ? 2 : 3;           // x / h_in stages
+    const uint32_t gdiag = T ? 128u : 0u;  // TMEM column of the diagonal block of C B^T
+    const uint32_t pcol = T ? 0u : 128u;   // TMEM columns of the P ring (T = 1: over C B_off^T)
+    const int xdiag = kTileRows * T;       // first x row of the diagonal block
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_cb, 1);
         mbar_init(&sm.bar_g, 1);
-        for (int s = 0; s < kXStages; ++s) {
+        mbar_init(&sm.bar_goff, 256);
+        for (int s = 0; s < kXStagesMax; ++s) {
             mbar_init(&sm.bar_xh_full[s], 1);
             mbar_init(&sm.bar_xh_free[s], 1);
+            mbar_init(&sm.bar_xv_ready[s], 256);
         }
         for (int s = 0; s < kVecStages; ++s) {
             mbar_init(&sm.bar_vec_full[s], 1);
-            mbar_init(&sm.bar_vec_free[s], 256 + 128);
+            mbar_init(&sm.bar_vec_free[s], 256);
         }
         for (int s = 0; s < kRing; ++s) {
             mbar_init(&sm.bar_slot_full[s], 256);
             mbar_init(&sm.bar_slot_free[s], 1);
         }
-        mbar_init(&sm.bar_acc_full, 1);
-        mbar_init(&sm.bar_acc_free, 128);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&sm.bar_acc_full[a], 1);
+            mbar_init(&sm.bar_acc_free[a], 256);
+        }
         mbar_init(&sm.bar_drain, 1);
         sm.abort = 0;
         fence_mbar_init();
@@ -372,9 +416,9 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 bulk_load(sm.cs_v[vs], cs + vrow, Q * 4, &sm.bar_vec_full[vs]);
                 bulk_load(sm.dt_v[vs], dtc + vrow, Q * 4, &sm.bar_vec_full[vs]);
             }
-            const int xs = j % kXStages;
-            const uint32_t xu = j / kXStages;
-            if (j >= kXStages && !warp_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) break;
+            const int xs = j % nst;
+            const uint32_t xu = j / nst;
+            if (j >= nst && !warp_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) break;
             if (xs == 2 && xu == 0 && !warp_wait(&sm.bar_g, 0, abort)) break;  // B tile in use
             if (lane == 0) {
                 uint8_t *stg = scan_stage(sm, xs);
@@ -385,16 +429,16 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                                 (int)(t0 + kTileRows * r), (int)b);
                 const int hrow = (int)(((b * nchunks + k) * H + h) * kP);
                 for (int a = 0; a < 2; ++a)
-                    tma_load_2d(stg + 256 * kRowBytes + a * kP * kRowBytes, &tm_h,
-                                &sm.bar_xh_full[xs], 64 * a, hrow);
+                    tma_load_2d(stg + kHOff + a * kP * kRowBytes, &tm_h, &sm.bar_xh_full[xs],
+                                64 * a, hrow);
             }
             __syncwarp();
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer
         const uint32_t id_g = idesc_bf16_f32(128, KI, false, false);
-        const uint32_t id_h = idesc_bf16_f32(128, kP, false, false);
-        const uint32_t id_y = idesc_bf16_f32(128, kP, false, true);
+        const uint32_t id_kk = idesc_bf16_f32(128, kP, false, false);   // K-major A and B
+        const uint32_t id_kmn = idesc_bf16_f32(128, kP, false, true);   // B (x) MN-major
         const uint32_t c0 = smem_u32(&sm.Cs[0][0]);
         const uint32_t rg = smem_u32(sm.R);
         bool ok = warp_wait(&sm.bar_cb, 0, abort);
@@ -412,37 +456,51 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             }
             __syncwarp();
         }
-        const uint32_t d1 = tmem + kAccCol, d2 = tmem + kAccCol + 64;
+        if (ok && T) ok = warp_wait(&sm.bar_goff, 0, abort);   // bf16 C B_off^T in smem
         uint32_t blk = 0;
         for (int j = 0; ok && j < nh; ++j) {
-            const int xs = j % kXStages;
-            const uint32_t xu = j / kXStages;
+            const int xs = j % nst;
+            const uint32_t xu = j / nst;
+            const int a = j & 1;
             if (!warp_wait(&sm.bar_xh_full[xs], xu & 1, abort)) break;
-            if (j >= 1 && !warp_wait(&sm.bar_acc_free, (j - 1) & 1, abort)) break;
+            if (T && !warp_wait(&sm.bar_xv_ready[xs], xu & 1, abort)) break;
+            if (j >= 2 && !warp_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
             tc_fence_after();
             const uint32_t stg = smem_u32(scan_stage(sm, xs));
+            const uint32_t dD = tmem + kAccCol + 128 * a, dA = dD + 64;
             if (lane == 0) {
-                // Y2 = C h_in^T: M = 128, N = 64 (p), K = 128 (n)
+                uint32_t acc = 0;
+                if (T) {
+                    // Y_A = (C B_off^T) (v dt o X_off): A = bf16 block in R, K = 128 (i)
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t aoff = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                        mma_bf16(dA, smem_desc_sw128(rg + aoff, 16, 1024),
+                                 smem_desc_sw128(stg + kk * 2048, 256 * kRowBytes, 1024), id_kmn,
+                                 acc);
+                        acc = 1;
+                    }
+                }
+                // Y_A (+)= C h^T: K = 128 (n); h = h_in (T = 0) or exp(cs_127) h_in (T = 1)
                 for (int kk = 0; kk < kN / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    const uint32_t hoff = 256 * kRowBytes + (kk >> 2) * (kP * kRowBytes) +
-                                          (kk & 3) * 32;
-                    mma_bf16(d2, smem_desc_sw128(c0 + off, 16, 1024),
-                             smem_desc_sw128(stg + hoff, 16, 1024), id_h, kk > 0 ? 1u : 0u);
+                    const uint32_t hoff = kHOff + (kk >> 2) * (kP * kRowBytes) + (kk & 3) * 32;
+                    mma_bf16(dA, smem_desc_sw128(c0 + off, 16, 1024),
+                             smem_desc_sw128(stg + hoff, 16, 1024), id_kk, acc);
+                    acc = 1;
                 }
             }
             __syncwarp();
-            for (int qb = 0; qb < nblk; ++qb, ++blk) {
+            for (int qb = 0; qb < 2; ++qb, ++blk) {
                 const uint32_t slot = blk % kRing, su = blk / kRing;
                 if (!warp_wait(&sm.bar_slot_full[slot], su & 1, abort)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
-                    // Y1 += P[:, 64qb : 64qb+64] X[64qb : 64qb+64, :], P read from TMEM
-                    const uint32_t pa = tmem + kPCol + 32 * slot;
+                    // Y_diag += P[:, 64qb : +64] X[xdiag + 64qb : +64, :], P read from TMEM
+                    const uint32_t pa = tmem + pcol + 32 * slot;
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bd =
-                            smem_desc_sw128(stg + (qb * 4 + kk) * 2048, 256 * kRowBytes, 1024);
-                        mma_bf16_ts(d1, pa + 8 * kk, bd, id_y, (qb | kk) != 0 ? 1u : 0u);
+                        const uint64_t bd = smem_desc_sw128(
+                            stg + (xdiag / 16 + qb * 4 + kk) * 2048, 256 * kRowBytes, 1024);
+                        mma_bf16_ts(dD, pa + 8 * kk, bd, id_kmn, (qb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit(&sm.bar_slot_free[slot]);
                 }
@@ -450,132 +508,176 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             }
             if (!ok) break;
             if (lane == 0) {
-                mma_commit(&sm.bar_acc_full);
+                mma_commit(&sm.bar_acc_full[a]);
                 mma_commit(&sm.bar_xh_free[xs]);
             }
             __syncwarp();
         }
-    } else if (warp >= 4 && warp < 12) {
-        // ---------------- mask: P[t][i] = G[t][i] exp(cs_t - cs_i) dt_i (i <= t), + D at i = t
+    } else if (warp >= 4) {
+        // ---------------- workers: mask of head j (for T = 1 after scaling x_off and h_in),
+        // then the epilogue y = Y_diag + f_t Y_A of head j - 1, each for this warp's half
+        const int mt = threadIdx.x - 128;          // 0..255
         const int qd = warp & 3;
         const int half = (warp - 4) >> 2;          // which 32 columns of each 64-column block
         const int t = qd * 32 + lane;             // row within the tile = TMEM lane
         const int tau = kTileRows * T + t;        // row within the chunk
-        const int r = kTileRows * T + qd * 32 - 1;  // reference row for the factorised decay
+        const int r = kTileRows * T + qd * 32 - 1;  // last row above this warp's 32-row slice
         const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
         float *vt = sm.vt[warp - 4];
         bool ok = warp_wait(&sm.bar_g, 0, abort);
         tc_fence_after();
-        uint32_t blk = 0;
-        for (int j = 0; ok && j < nh; ++j) {
-            const int vs = j % kVecStages;
-            if (!warp_wait(&sm.bar_vec_full[vs], (j / kVecStages) & 1, abort)) break;
-            const float *cs_s = sm.cs_v[vs];
-            const float *dt_s = sm.dt_v[vs];
-            const float Dh = sm.Dv[j];
-            const float ct = cs_s[tau];
-            float uf = 0.f;
-            __syncwarp();
-            if (r >= 0) {
-                const float cr = cs_s[r];
-                // v for the columns of this warp's off-diagonal sub-blocks
-                for (int qb = 0; qb < nblk; ++qb) {
-                    const int i = qb * 64 + half * 32 + lane;
-                    if (i <= r) vt[i] = __expf(cr - cs_s[i]) * dt_s[i];
-                }
-                uf = __expf(ct - cr);
-            }
-            __syncwarp();
-            for (int qb = 0; qb < nblk; ++qb, ++blk) {
-                const uint32_t slot = blk % kRing, su = blk / kRing;
-                if (su >= 1 && !warp_wait(&sm.bar_slot_free[slot], (su - 1) & 1, abort)) {
-                    ok = false;
-                    break;
-                }
-                const int col0 = qb * 64 + half * 32;
-                uint32_t pk[16];
-                if (col0 + 32 <= r + 1) {
-                    uint32_t gv[32];
-                    tmem_ld32(lane_base + col0, gv);
-                    tmem_ld_wait();
-                    const float2 uu = make_float2(uf, uf);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const float4 vv = *reinterpret_cast<const float4 *>(vt + col0 + 4 * c);
-                        const float2 p0 = fmul2(fmul2(make_float2(__uint_as_float(gv[4 * c]),
-                                                                  __uint_as_float(gv[4 * c + 1])),
-                                                      make_float2(vv.x, vv.y)), uu);
-                        const float2 p1 = fmul2(fmul2(make_float2(__uint_as_float(gv[4 * c + 2]),
-                                                                  __uint_as_float(gv[4 * c + 3])),
-                                                      make_float2(vv.z, vv.w)), uu);
-                        pk[2 * c] = pack_bf16x2(p0.x, p0.y);
-                        pk[2 * c + 1] = pack_bf16x2(p1.x, p1.y);
-                    }
-                } else if (col0 == r + 1) {
-                    uint32_t gv[32];
-                    tmem_ld32(lane_base + col0, gv);
-                    tmem_ld_wait();
-                    float pv[32];
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int i = col0 + c;
-                        float v = 0.f;
-                        if (i <= tau)
-                            v = __uint_as_float(gv[c]) * __expf(ct - cs_s[i]) * dt_s[i];
-                        if (i == tau) v += Dh;
-                        pv[c] = v;
-                    }
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) pk[c] = 0u;
-                }
-                tmem_st16(lane_base + kPCol + 32 * slot + 16 * half, pk);
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&sm.bar_slot_full[slot]);
-            }
-            if (ok) mbar_arrive(&sm.bar_vec_free[vs]);   // done with this stage's cs / dt
-        }
-    } else if (warp >= 12) {
-        // ---------------- epilogue: y = Y1 + exp(cs_t) Y2
-        const int qd = warp & 3;
-        const int t = qd * 32 + lane;
-        const int tau = kTileRows * T + t;
-        const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
-        for (int j = 0; j < nh; ++j) {
-            if (!warp_wait(&sm.bar_acc_full, j & 1, abort)) break;
-            tc_fence_after();
-            const int vs = j % kVecStages;
-            if (!warp_wait(&sm.bar_vec_full[vs], (j / kVecStages) & 1, abort)) break;
-            const float e = __expf(sm.cs_v[vs][tau]);
-            mbar_arrive(&sm.bar_vec_free[vs]);              // done with this stage's cs
-            uint32_t a0[32], c0[32], pk[32];
-            tmem_ld32(lane_base + kAccCol, a0);
-            tmem_ld32(lane_base + kAccCol + 64, c0);
+        if (ok && T) {
+            // C B_off^T (TMEM columns [0, 128)) -> bf16, K-major swizzled tile in R; this warp
+            // converts its 32 rows x 64 columns [64 half, 64 half + 64)
+            uint8_t *dst = sm.R + half * kBoxBytes + t * kRowBytes;
+            uint32_t gv[64];
+            tmem_ld32(lane_base + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(gv));
+            tmem_ld32(lane_base + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(gv + 32));
             tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-                pk[c] = pack_bf16x2(fmaf(e, __uint_as_float(c0[2 * c]), __uint_as_float(a0[2 * c])),
-                                    fmaf(e, __uint_as_float(c0[2 * c + 1]),
-                                         __uint_as_float(a0[2 * c + 1])));
-            tmem_ld32(lane_base + kAccCol + 32, a0);
-            tmem_ld32(lane_base + kAccCol + 96, c0);
-            tmem_ld_wait();
+            for (int m = 0; m < 8; ++m) {
+                const int pos = m ^ (t & 7);
+                *reinterpret_cast<uint4 *>(dst + pos * 16) = make_uint4(
+                    pack_bf16x2(__uint_as_float(gv[8 * m]), __uint_as_float(gv[8 * m + 1])),
+                    pack_bf16x2(__uint_as_float(gv[8 * m + 2]), __uint_as_float(gv[8 * m + 3])),
+                    pack_bf16x2(__uint_as_float(gv[8 * m + 4]), __uint_as_float(gv[8 * m + 5])),
+                    pack_bf16x2(__uint_as_float(gv[8 * m + 6]), __uint_as_float(gv[8 * m + 7])));
+            }
+            fence_async_smem();
             tc_fence_before();
-            mbar_arrive(&sm.bar_acc_free);
+            mbar_arrive(&sm.bar_goff);
+            // the P ring reuses these TMEM columns: wait until every warp has read them
+            ok = warp_wait(&sm.bar_goff, 0, abort);
+            tc_fence_after();
+        }
+        uint32_t blk = 0;
+        for (int j = 0; ok && j <= nh; ++j) {
+            if (j < nh) {
+                const int vs = j % kVecStages;
+                if (!warp_wait(&sm.bar_vec_full[vs], (j / kVecStages) & 1, abort)) break;
+                const float *cs_s = sm.cs_v[vs];
+                const float *dt_s = sm.dt_v[vs];
+                // this warp's two 32-column sub-blocks of the diagonal block: sbl = 2 qb + half
+                const int sb0 = half, sb1 = 2 + half;
+                uint32_t g0[32], g1[32];
+                if (sb0 <= qd) tmem_ld32(lane_base + gdiag + 32 * sb0, g0);
+                if (sb1 <= qd) tmem_ld32(lane_base + gdiag + 32 * sb1, g1);
+                if (T) {
+                    // x rows [0, 128) *= exp(cs_127 - cs_i) dt_i; h_in *= exp(cs_127)
+                    const int xs = j % nst;
+                    if (!warp_wait(&sm.bar_xh_full[xs], (j / nst) & 1, abort)) break;
+                    uint8_t *stg = scan_stage(sm, xs);
+                    const float c127 = cs_s[127];
+                    scale_pieces<4>(stg, mt, 256, [&](int c) {
+                        const int i = c >> 3;
+                        return __expf(c127 - cs_s[i]) * dt_s[i];
+                    });
+                    const float sh = __expf(c127);
+                    scale_pieces<4>(stg + kHOff, mt, 256, [&](int) { return sh; });
+                    fence_async_smem();
+                    mbar_arrive(&sm.bar_xv_ready[xs]);
+                }
+                const float Dh = sm.Dv[j];
+                const float ct = cs_s[tau];
+                // Column factors over this warp's sub-blocks (local column lc = 32 sbl + lane):
+                // below the 32 x 32 diagonal sub-block (sbl < qd) relative to row r, both
+                // factors <= 1; inside it (sbl == qd) relative to m = r + 1, the slice's first
+                // row: exp(cs_m - cs_i) <= exp(32 max|dt A|) and exp(cs_t - cs_m) <= 1, so
+                // neither over- nor underflows, and no element needs an exponential of its own.
+                const float cm = cs_s[r + 1];
+                const float um = __expf(ct - cm);
+                __syncwarp();
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-                pk[16 + c] = pack_bf16x2(
-                    fmaf(e, __uint_as_float(c0[2 * c]), __uint_as_float(a0[2 * c])),
-                    fmaf(e, __uint_as_float(c0[2 * c + 1]), __uint_as_float(a0[2 * c + 1])));
-            if (tau < len) {
-                uint4 *yrow = reinterpret_cast<uint4 *>(
-                    y + ((b * seqlen + t0 + tau) * H + h0 + j) * (int64_t)kP);
+                for (int qb = 0; qb < 2; ++qb) {
+                    const int sbl = qb * 2 + half;
+                    const int lc = sbl * 32 + lane;
+                    const int i = kTileRows * T + lc;
+                    if (sbl < qd) vt[lc] = __expf(cs_s[r] - cs_s[i]) * dt_s[i];
+                    else if (sbl == qd) vt[lc] = __expf(cm - cs_s[i]) * dt_s[i];
+                }
+                const float uf = qd > 0 ? __expf(ct - cs_s[r]) : 0.f;
+                __syncwarp();
+                tmem_ld_wait();
 #pragma unroll
-                for (int m = 0; m < 8; ++m)
-                    yrow[m] = make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+                for (int qb = 0; qb < 2; ++qb, ++blk) {
+                    const uint32_t slot = blk % kRing, su = blk / kRing;
+                    const int sbl = qb * 2 + half;
+                    const int lc0 = 32 * sbl;
+                    const uint32_t *gv = qb ? g1 : g0;
+                    uint32_t pk[16];
+                    if (sbl < qd) {
+                        const float2 uu = make_float2(uf, uf);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const float4 vv = *reinterpret_cast<const float4 *>(vt + lc0 + 4 * c);
+                            const float2 p0 = fmul2(
+                                fmul2(make_float2(__uint_as_float(gv[4 * c]),
+                                                  __uint_as_float(gv[4 * c + 1])),
+                                      make_float2(vv.x, vv.y)), uu);
+                            const float2 p1 = fmul2(
+                                fmul2(make_float2(__uint_as_float(gv[4 * c + 2]),
+                                                  __uint_as_float(gv[4 * c + 3])),
+                                      make_float2(vv.z, vv.w)), uu);
+                            pk[2 * c] = pack_bf16x2(p0.x, p0.y);
+                            pk[2 * c + 1] = pack_bf16x2(p1.x, p1.y);
+                        }
+                    } else if (sbl == qd) {
+                        // causal 32 x 32 block: column c <= lane kept, + D at c = lane
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const float2 ww = *reinterpret_cast<const float2 *>(vt + lc0 + 2 * c);
+                            float p0 = __uint_as_float(gv[2 * c]) * ww.x * um;
+                            float p1 = __uint_as_float(gv[2 * c + 1]) * ww.y * um;
+                            p0 = (2 * c <= lane) ? p0 : 0.f;
+                            p1 = (2 * c + 1 <= lane) ? p1 : 0.f;
+                            p0 += (2 * c == lane) ? Dh : 0.f;
+                            p1 += (2 * c + 1 == lane) ? Dh : 0.f;
+                            pk[c] = pack_bf16x2(p0, p1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) pk[c] = 0u;
+                    }
+                    if (su >= 1 && !warp_wait(&sm.bar_slot_free[slot], (su - 1) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tmem_st16(lane_base + pcol + 32 * slot + 16 * half, pk);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(&sm.bar_slot_full[slot]);
+                }
+                if (!ok) break;
+            }
+            if (j >= 1) {
+                // epilogue of head jj = j - 1 for output columns [32 half, 32 half + 32)
+                const int jj = j - 1;
+                const int a = jj & 1;
+                const int vs = jj % kVecStages;
+                if (!warp_wait(&sm.bar_acc_full[a], (jj >> 1) & 1, abort)) break;
+                tc_fence_after();
+                const uint32_t col = lane_base + kAccCol + 128 * a + 32 * half;
+                uint32_t d0[32], a0[32];
+                tmem_ld32(col, d0);
+                tmem_ld32(col + 64, a0);
+                const float f = __expf(sm.cs_v[vs][tau] - (T ? sm.cs_v[vs][127] : 0.f));
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&sm.bar_acc_free[a]);
+                mbar_arrive(&sm.bar_vec_free[vs]);   // done with this head's cs / dt
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    pk[c] = pack_bf16x2(
+                        fmaf(f, __uint_as_float(a0[2 * c]), __uint_as_float(d0[2 * c])),
+                        fmaf(f, __uint_as_float(a0[2 * c + 1]), __uint_as_float(d0[2 * c + 1])));
+                if (tau < len) {
+                    uint4 *yrow = reinterpret_cast<uint4 *>(
+                        y + ((b * seqlen + t0 + tau) * H + h0 + jj) * (int64_t)kP + 32 * half);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        yrow[m] = make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+                }
             }
         }
     }
