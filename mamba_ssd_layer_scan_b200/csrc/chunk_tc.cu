@@ -26,7 +26,8 @@
 //     exponential of its own.  The same worker warps then run the previous head's epilogue.
 //
 // Roles (warp-specialised; every wait is on an mbarrier and bounded, see sm100.cuh):
-//   state kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-11 scale, 12-15 epilogue
+//   state kernel: warp 0 TMA, warps 1 and 3 MMA (alternate heads), warp 2 TMEM owner,
+//                 warps 4-11 scale, 12-15 epilogue
 //   scan  kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-11 mask + epilogue
 #include <cudaTypedefs.h>
 
@@ -69,7 +70,8 @@ struct alignas(1024) StateSmem {
     uint32_t tmem_base;
     int abort;
 };
-// warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warp 3 idle, warps 4-11 scale x, warps 12-15 epilogue
+// warp 0 TMA, warps 1 and 3 MMA (alternate heads), warp 2 TMEM owner, warps 4-11 scale x,
+// warps 12-15 epilogue
 constexpr int kStateThreads = 512;
 constexpr int kStateScaleThreads = 256;
 constexpr uint32_t kStateTmemCols = 128;
@@ -106,7 +108,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_init(&sm.bar_acc_full[s], 1);
             mbar_init(&sm.bar_acc_free[s], 128);
         }
-        mbar_init(&sm.bar_drain, 1);
+        mbar_init(&sm.bar_drain, 2);
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -146,12 +148,15 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             }
             __syncwarp();
         }
-    } else if (warp == 1) {
-        // ---------------- MMA issuer: D[n][p] += sum_tau B[tau][n] * Xw[tau][p]
+    } else if (warp == 1 || warp == 3) {
+        // ---------------- MMA issuers: D[n][p] += sum_tau B[tau][n] * Xw[tau][p].  A single
+        // issuing thread waits ~100+ cycles per tcgen05.mma, so two warps issue alternate heads
+        // (each into its own accumulator buffer) to keep the tensor core busy.
+        const int par = warp == 1 ? 0 : 1;
         const uint32_t idesc = idesc_bf16_f32(128, kP, true, true);
         const uint32_t atom_bytes = 256 * kRowBytes;  // distance between the two n atoms of Bs
         if (warp_wait(&sm.bar_b, 0, abort)) {
-            for (int j = 0; j < nh; ++j) {
+            for (int j = par; j < nh; j += 2) {
                 const int s = j % kStateStages;
                 const uint32_t use = j / kStateStages;
                 const int a = j & 1;
@@ -225,7 +230,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     __syncthreads();
     if (sm.abort) {
         // Let this CTA's own MMAs and TMA copies finish before TMEM and smem are released.
-        if (warp == 1 && lane == 0) {
+        if ((warp == 1 || warp == 3) && lane == 0) {
             mma_commit(&sm.bar_drain);
             mbar_wait_drain(&sm.bar_drain, 0);
         }
@@ -457,7 +462,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             __syncwarp();
         }
         if (ok && T) ok = warp_wait(&sm.bar_goff, 0, abort);   // bf16 C B_off^T in smem
-        uint32_t blk = 0;
         for (int j = 0; ok && j < nh; ++j) {
             const int xs = j % nst;
             const uint32_t xu = j / nst;
@@ -490,7 +494,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 }
             }
             __syncwarp();
-            for (int qb = 0; qb < 2; ++qb, ++blk) {
+            for (int qb = 0; qb < 2; ++qb) {
+                const uint32_t blk = 2 * j + qb;           // P blocks are numbered per head
                 const uint32_t slot = blk % kRing, su = blk / kRing;
                 if (!warp_wait(&sm.bar_slot_full[slot], su & 1, abort)) { ok = false; break; }
                 tc_fence_after();
