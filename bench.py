@@ -102,13 +102,14 @@ def source_hash(kernel):
 
 def profiled_traffic(kernel, workload):
     """dram bytes per launch from the committed ncu summary, if taken on the current source."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get(workload, {}).get(kernel)
-    if not d or d.get("source_sha") != source_hash(kernel):
-        return None
-    return d.get("dram_bytes_per_launch")
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 4 and not line.startswith("#") and f[0] == workload and f[1] == kernel:
+            return int(f[2]) if f[3] == source_hash(kernel) else None
+    return None
 
 
 class ClockSampler:
