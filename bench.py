@@ -176,6 +176,23 @@ def nvml_index(torch, dev):
         return dev
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The maximum of `value` over all ranks of the default process group (the value itself when
+    there is no group).  Timing of a multi-GPU step is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def scaled_throughput(units_per_rank: float, world: int, seconds: float) -> float:
+    """Whole-job throughput: every rank processed `units_per_rank` in (max-over-ranks) `seconds`."""
+    return world * units_per_rank / seconds
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 def time_oracle(w, inp, target_s, max_pairs=None):
     """Run the float64 oracle on (batch, head) slices of the full sequence until about
@@ -327,14 +344,10 @@ def main():
     step_ms = [ev[i][0].elapsed_time(ev[i][4]) for i in range(K)]
     kern_ms = {name: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)]
                for j, name in enumerate(KERNELS)}
-    total_ms = sum(step_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / K
     tokens_per_step = w.batch * w.seqlen
-    value = world * tokens_per_step * K / (total_ms / 1e3)
+    value = scaled_throughput(tokens_per_step * K, world, total_ms / 1e3)
 
     # ---- end to end through the C ABI with host buffers: H2D of inputs, scan, D2H of y + final
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
@@ -357,12 +370,8 @@ def main():
     e_end.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e_start.elapsed_time(e_end) / K_e2e
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = world * tokens_per_step / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / K_e2e, dev)
+    e2e_value = scaled_throughput(tokens_per_step, world, e2e_ms / 1e3)
 
     # ---- decode update at batch 128, 80 heads, 64 x 128 fp32 state
     wd = configs.SSD_DECODE

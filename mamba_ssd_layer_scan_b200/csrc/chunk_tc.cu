@@ -9,14 +9,14 @@
 // block matrix multiplications).  Two kernels:
 //
 // chunk_state_tc_kernel   S_k^T = B_k^T (w o X_k),  w_tau = exp(cs_last - cs_tau) dt_tau
-//     One CTA per (batch, chunk, group, block of 8 heads).  The chunk's B rows are loaded once
+//     One CTA per (batch, chunk, group, block of heads).  The chunk's B rows are loaded once
 //     and shared by the heads of the block; per head, the x tile and the head's cs / dt rows
 //     arrive by TMA (4 stages), 8 warps scale the x rows by w in shared memory, one
 //     M=128 (n) x N=64 (p) x K=Q MMA chain accumulates S^T in TMEM (double-buffered), and 4
 //     epilogue warps move it to global memory while the next head's MMAs run.
 //
 // chunk_scan_tc_kernel    y = (C B^T o L o dt + diag(D)) X  +  exp(cs) o (C h_in^T)
-//     One CTA per (batch, chunk, 128-row tile of the chunk, group, block of 8 heads).  C B^T is
+//     One CTA per (batch, chunk, 128-row tile of the chunk, group, block of heads).  C B^T is
 //     computed once per CTA and shared by the heads (all heads of a group see the same B, C).
 //     The diagonal 128 x 128 block of the masked matrix is built per head by 8 worker warps from
 //     TMEM and written back to TMEM as bf16 (a ring of 64-column blocks), where the MMAs read it
@@ -31,6 +31,8 @@
 //   scan  kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-11 mask + epilogue
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "common.cuh"
@@ -43,7 +45,7 @@ using namespace sm100;
 
 constexpr int kP = 64;
 constexpr int kN = 128;
-constexpr int kHeadsPerCta = 8;
+constexpr int kMaxHeadsPerCta = 128;   // heads one CTA walks through (chosen per launch)
 constexpr int kRowBytes = 128;                  // one swizzled smem row: 64 bf16
 constexpr int kTileRows = 128;                  // rows of one TMA box / one MMA M tile
 constexpr int kBoxBytes = kTileRows * kRowBytes;  // 16 KB
@@ -80,7 +82,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                       const __grid_constant__ CUtensorMap tm_b, const float *__restrict__ dtc,
                       const float *__restrict__ cs, float *__restrict__ states,
-                      int *__restrict__ status, int H, int G, int Q, int64_t nchunks, int nhb)
+                      int *__restrict__ status, int H, int G, int Q, int64_t nchunks, int nhb,
+                      int hpc)
 {
     extern __shared__ uint8_t smem_raw[];
     StateSmem &sm = *reinterpret_cast<StateSmem *>(
@@ -92,8 +95,8 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int g = (int)(u % G); u /= G;
     const int64_t k = u % nchunks, b = u / nchunks;
     const int hpg = H / G;
-    const int h0 = g * hpg + hb * kHeadsPerCta;
-    const int nh = min(kHeadsPerCta, hpg - hb * kHeadsPerCta);
+    const int h0 = g * hpg + hb * hpc;
+    const int nh = min(hpc, hpg - hb * hpc);
     const int64_t t0 = k * Q;
     const int nrb = Q / kTileRows;
 
@@ -276,7 +279,7 @@ struct alignas(1024) ScanSmem {
     float cs_v[kVecStages][256];    // per stage: the head's chunk-local cumsum row
     float dt_v[kVecStages][256];    // per stage: the head's dt row (0 past the end)
     float vt[8][128];               // per mask warp: exp(cs_r - cs_i) dt_i over the tile
-    float Dv[kHeadsPerCta];         // D of the CTA's heads
+    float Dv[kMaxHeadsPerCta];      // D of the CTA's heads
     uint64_t bar_cb, bar_g, bar_goff;
     uint64_t bar_xh_full[kXStagesMax], bar_xh_free[kXStagesMax], bar_xv_ready[kXStagesMax];
     uint64_t bar_vec_full[kVecStages], bar_vec_free[kVecStages];
@@ -333,7 +336,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_h, const float *__restrict__ dtc,
                      const float *__restrict__ cs, const float *__restrict__ D,
                      bf16 *__restrict__ y, int *__restrict__ status, int64_t seqlen, int H,
-                     int G, int Q, int64_t nchunks, int nhb)
+                     int G, int Q, int64_t nchunks, int nhb, int hpc)
 {
     extern __shared__ uint8_t smem_raw[];
     ScanSmem &sm = *reinterpret_cast<ScanSmem *>(
@@ -347,8 +350,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int g = (int)(u % G); u /= G;
     const int64_t k = u % nchunks, b = u / nchunks;
     const int hpg = H / G;
-    const int h0 = g * hpg + hb * kHeadsPerCta;
-    const int nh = min(kHeadsPerCta, hpg - hb * kHeadsPerCta);
+    const int h0 = g * hpg + hb * hpc;
+    const int nh = min(hpc, hpg - hb * hpc);
     const int64_t t0 = k * Q;
     const int len = (int)min((int64_t)Q, seqlen - t0);
     if (T * kTileRows >= len) return;  // tile entirely past the end of the sequence
@@ -383,7 +386,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         sm.abort = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x >= 32 && threadIdx.x < 32 + nh) sm.Dv[threadIdx.x - 32] = D[h0 + threadIdx.x - 32];
+    for (int i = threadIdx.x; i < nh; i += blockDim.x) sm.Dv[i] = D[h0 + i];
     if (warp == 2) {
         tmem_alloc(&sm.tmem_base, kScanTmemCols);
         tmem_relinquish();
@@ -748,6 +751,29 @@ bool make_seq_map(CUtensorMap *m, const void *ptr, int64_t batch, int64_t seqlen
     return make_map(m, ptr, 4, dims, strides, box);
 }
 
+// Heads per CTA.  Every CTA pays a fixed ramp-up (its B / C tiles, C B^T, the first TMA round
+// trips) and drain, which only a long run of heads amortises, while too few CTAs leave SMs idle.
+// Pick the count that minimises waves x (ramp + heads x per-head time), with the waves counted
+// over the SMs of the device.
+int heads_per_cta(int64_t groups_work, int hpg, double ramp_us, double head_us)
+{
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int best = 1;
+    double best_t = 1e30;
+    for (int hpc = 1; hpc <= std::min(hpg, kMaxHeadsPerCta); ++hpc) {
+        const int nhb = (hpg + hpc - 1) / hpc;
+        if (hpc > 1 && (hpg + hpc - 2) / (hpc - 1) == nhb) continue;   // same split, fewer heads
+        const double ctas = (double)groups_work * nhb;
+        const double waves = std::ceil(ctas / sms);
+        const double t = waves * (ramp_us + hpc * head_us);
+        if (t < best_t - 1e-9) { best_t = t; best = hpc; }
+    }
+    return best;
+}
+
 }  // namespace
 
 bool tc_supported(bool is_bf16, int P, int N, int Q)
@@ -766,14 +792,15 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
         return cudaErrorInvalidValue;
     }
     const int hpg = H / G;
-    const int nhb = (hpg + kHeadsPerCta - 1) / kHeadsPerCta;
+    const int hpc = heads_per_cta(batch * nchunks * G, hpg, 4.0, 2.0);
+    const int nhb = (hpg + hpc - 1) / hpc;
     const size_t smem = sizeof(StateSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(chunk_state_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk state: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb);
     chunk_state_tc_kernel<<<grid, kStateThreads, smem, st>>>(mx, mb, dtc, cs, states, status,
-                                                             H, G, Q, nchunks, nhb);
+                                                             H, G, Q, nchunks, nhb, hpc);
     *why = "chunk state (tcgen05) launch";
     return cudaGetLastError();
 }
@@ -795,14 +822,15 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
         return cudaErrorInvalidValue;
     }
     const int hpg = H / G;
-    const int nhb = (hpg + kHeadsPerCta - 1) / kHeadsPerCta;
+    const int hpc = heads_per_cta(batch * nchunks * G * (Q / kTileRows), hpg, 5.0, 2.0);
+    const int nhb = (hpg + hpc - 1) / hpc;
     const size_t smem = sizeof(ScanSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(chunk_scan_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk scan: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb * (Q / kTileRows));
     chunk_scan_tc_kernel<<<grid, kScanThreads, smem, st>>>(mx, mb, mc, mh, dtc, cs, D, y, status,
-                                                           seqlen, H, G, Q, nchunks, nhb);
+                                                           seqlen, H, G, Q, nchunks, nhb, hpc);
     *why = "chunk scan (tcgen05) launch";
     return cudaGetLastError();
 }
