@@ -822,7 +822,9 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
         return cudaErrorInvalidValue;
     }
     const int hpg = H / G;
-    const int hpc = heads_per_cta(batch * nchunks * G * (Q / kTileRows), hpg, 5.0, 2.0);
+    // The scan's per-head cost (mask, three MMA chains, epilogue) dominates its per-CTA ramp, and
+    // its two tiles differ in cost, so many small CTAs balance better than one CTA per group.
+    const int hpc = std::min(hpg, 8);
     const int nhb = (hpg + hpc - 1) / hpc;
     const size_t smem = sizeof(ScanSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(chunk_scan_tc_kernel,
