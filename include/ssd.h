@@ -92,6 +92,10 @@ size_t ssd_chunk_scan_workspace_size(const ssd_shape *shape, int chunk_size);
  *
  * Concurrent calls must use distinct workspaces.  batch == 0 or seqlen == 0 is valid: y is
  * empty and final_state is set to init_state (or zeros).
+ *
+ * On the tensor-core path the per-chunk states and the carry across chunks run as two kernels
+ * by default; setting the environment variable SSD_STATE_PASSING=fused runs them as one kernel
+ * that walks the chunks in order (=split forces the two kernels).  Both give the same result.
  */
 ssd_status ssd_chunk_scan_fwd(const ssd_shape *shape, const void *x, const float *dt,
                               const float *A, const void *B, const void *C, const float *D,

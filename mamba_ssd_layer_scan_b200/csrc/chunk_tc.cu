@@ -126,7 +126,8 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     volatile int *abort = &sm.abort;
 
     if (warp == 0) {
-        // ---------------- TMA producer: B once, then per head its x tile and cs / dt rows
+        // ---------------- TMA producer (lane 0 alone): B once, then per head its x tile and
+        // cs / dt rows
         if (lane == 0) {
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
@@ -135,12 +136,11 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 for (int r = 0; r < nrb; ++r)
                     tma_load_4d(&sm.Bs[a][r * kTileRows * 64], &tm_b, &sm.bar_b, 64 * a, g,
                                 (int)(t0 + kTileRows * r), (int)b);
-        }
-        for (int j = 0; j < nh; ++j) {
-            const int s = j % kStateStages;
-            const uint32_t use = j / kStateStages;
-            if (j >= kStateStages && !warp_wait(&sm.bar_x_free[s], (use - 1) & 1, abort)) break;
-            if (lane == 0) {
+            for (int j = 0; j < nh; ++j) {
+                const int s = j % kStateStages;
+                const uint32_t use = j / kStateStages;
+                if (j >= kStateStages && !mbar_wait(&sm.bar_x_free[s], (use - 1) & 1, abort))
+                    break;
                 const int64_t vrow = ((b * nchunks + k) * H + h0 + j) * (int64_t)Q;
                 mbar_arrive_expect_tx(&sm.bar_x_full[s], (uint32_t)Q * (kRowBytes + 8));
                 for (int r = 0; r < nrb; ++r)
@@ -149,35 +149,32 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 bulk_load(sm.cs_v[s], cs + vrow, Q * 4, &sm.bar_x_full[s]);
                 bulk_load(sm.dt_v[s], dtc + vrow, Q * 4, &sm.bar_x_full[s]);
             }
-            __syncwarp();
         }
     } else if (warp == 1 || warp == 3) {
-        // ---------------- MMA issuers: D[n][p] += sum_tau B[tau][n] * Xw[tau][p].  A single
-        // issuing thread waits ~100+ cycles per tcgen05.mma, so two warps issue alternate heads
-        // (each into its own accumulator buffer) to keep the tensor core busy.
+        // ---------------- MMA issuers: D[n][p] += sum_tau B[tau][n] * Xw[tau][p].  Two warps
+        // issue alternate heads (each into its own accumulator buffer).  In each, lane 0 alone
+        // runs the whole loop, waits included: a lane that issued tcgen05.mma and then rejoins
+        // its warp stalls for the MMAs' issue latency (hundreds of cycles) at every rejoin.
         const int par = warp == 1 ? 0 : 1;
         const uint32_t idesc = idesc_bf16_f32(128, kP, true, true);
         const uint32_t atom_bytes = 256 * kRowBytes;  // distance between the two n atoms of Bs
-        if (warp_wait(&sm.bar_b, 0, abort)) {
+        if (lane == 0 && mbar_wait(&sm.bar_b, 0, abort)) {
             for (int j = par; j < nh; j += 2) {
                 const int s = j % kStateStages;
                 const uint32_t use = j / kStateStages;
                 const int a = j & 1;
-                if (!warp_wait(&sm.bar_x_ready[s], use & 1, abort)) break;
-                if (j >= 2 && !warp_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
+                if (!mbar_wait(&sm.bar_x_ready[s], use & 1, abort)) break;
+                if (j >= 2 && !mbar_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
                 tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t d = tmem + a * kP;
-                    const uint32_t a0 = smem_u32(&sm.Bs[0][0]), b0 = smem_u32(&sm.Xs[s][0]);
-                    for (int kk = 0; kk < Q / 16; ++kk) {
-                        const uint64_t ad = smem_desc_sw128(a0 + kk * 2048, atom_bytes, 1024);
-                        const uint64_t bd = smem_desc_sw128(b0 + kk * 2048, atom_bytes, 1024);
-                        mma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&sm.bar_x_free[s]);
-                    mma_commit(&sm.bar_acc_full[a]);
+                const uint32_t d = tmem + a * kP;
+                const uint32_t a0 = smem_u32(&sm.Bs[0][0]), b0 = smem_u32(&sm.Xs[s][0]);
+                for (int kk = 0; kk < Q / 16; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(a0 + kk * 2048, atom_bytes, 1024);
+                    const uint64_t bd = smem_desc_sw128(b0 + kk * 2048, atom_bytes, 1024);
+                    mma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
                 }
-                __syncwarp();
+                mma_commit(&sm.bar_x_free[s]);
+                mma_commit(&sm.bar_acc_full[a]);
             }
         }
     } else if (warp >= 4 && warp < 12) {
@@ -247,6 +244,261 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     if (warp == 2) {
         tc_fence_after();
         tmem_dealloc(tmem, kStateTmemCols);
+    }
+}
+
+// ============================================================ chunk state + state passing, fused
+//
+// One CTA per (batch, group, block of up to 3 heads) walks the chunks in order and carries the
+// recurrence across them itself (mohakchugh.is-a.dev "Mamba-2", Block Decomposition: across
+// blocks the state is propagated sequentially):
+//
+//     S_k     = B_k^T (w o X_k)              (tensor cores, TMEM)
+//     h_in[k] = h;   h <- exp(cs_k[Q-1]) h + S_k      (h in TMEM, fp32)
+//
+// so the float32 chunk states never go to HBM.  Each chunk is consumed in 128-row halves
+// through a 2-stage ring (the half's B rows, shared by the heads, and each head's x rows).
+// Three MMA issuer warps (one per head) keep three accumulation chains in flight; 8 epilogue
+// warps own the state: per chunk they store h (bf16) as the state entering the chunk and fold
+// S into it; after the last chunk they store it (float32) as the final state.
+constexpr int kFusedHeads = 3;
+struct alignas(1024) FusedSmem {
+    bf16 Bs[2][2][kTileRows * 64];                  // per stage: MN-major A, [n atom][128 tau][64 n]
+    bf16 Xs[2][kFusedHeads][kTileRows * 64];        // per stage and head: MN-major B [128 tau][64 p]
+    float cs_v[2][kFusedHeads][256];                // per chunk slot and head: cs row
+    float dt_v[2][kFusedHeads][256];                // per chunk slot and head: dt row
+    uint64_t bar_full[2], bar_ready[2], bar_free[2];
+    uint64_t bar_vec_full[2], bar_vec_free[2];
+    uint64_t bar_acc_full[kFusedHeads], bar_acc_free[kFusedHeads];
+    uint64_t bar_drain;
+    uint32_t tmem_base;
+    int abort;
+};
+// warp 0 TMA, warps 1-3 MMA (warp 1 + j issues head j; warp 2 also owns TMEM), warps 4-11 scale
+// x, warps 12-19 state epilogue (two per TMEM lane quarter, 32 columns p each)
+constexpr int kFusedThreads = 640;
+constexpr uint32_t kFusedTmemCols = 512;   // S of head j at 64 j, h of head j at 256 + 64 j
+static_assert(sizeof(FusedSmem) + 1024 <= 232448, "fused state smem exceeds 227 KB");
+
+__global__ void __launch_bounds__(kFusedThreads, 1)
+chunk_state_pass_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
+                           const __grid_constant__ CUtensorMap tm_b,
+                           const float *__restrict__ dtc, const float *__restrict__ cs,
+                           const float *__restrict__ init, float *__restrict__ final_state,
+                           bf16 *__restrict__ hin, int *__restrict__ status, int H, int G, int Q,
+                           int64_t nchunks, int nhb)
+{
+    extern __shared__ uint8_t smem_raw[];
+    FusedSmem &sm = *reinterpret_cast<FusedSmem *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    int64_t u = blockIdx.x;
+    const int hb = (int)(u % nhb); u /= nhb;
+    const int g = (int)(u % G); u /= G;
+    const int64_t b = u;
+    const int hpg = H / G;
+    const int h0 = g * hpg + hb * kFusedHeads;
+    const int nh = min(kFusedHeads, hpg - hb * kFusedHeads);
+    const int nrb = Q / kTileRows;               // 128-row halves per chunk
+    const int64_t nunits = nchunks * nrb;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.bar_full[s], 1);
+            mbar_init(&sm.bar_ready[s], 256);
+            mbar_init(&sm.bar_free[s], nh);
+            mbar_init(&sm.bar_vec_full[s], 1);
+            mbar_init(&sm.bar_vec_free[s], 256 + 256);
+        }
+        for (int j = 0; j < kFusedHeads; ++j) {
+            mbar_init(&sm.bar_acc_full[j], 1);
+            mbar_init(&sm.bar_acc_free[j], 256);
+        }
+        mbar_init(&sm.bar_drain, kFusedHeads);
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(&sm.tmem_base, kFusedTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort = &sm.abort;
+
+    if (warp == 0) {
+        // ---------------- TMA producer (lane 0 alone)
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_x);
+            tma_prefetch_desc(&tm_b);
+            for (int64_t un = 0; un < nunits; ++un) {
+                const int64_t k = un / nrb;
+                const int r = (int)(un % nrb);
+                if (r == 0) {
+                    const int vs = (int)(k & 1);
+                    if (k >= 2 &&
+                        !mbar_wait(&sm.bar_vec_free[vs], (uint32_t)((k >> 1) - 1) & 1, abort))
+                        break;
+                    mbar_arrive_expect_tx(&sm.bar_vec_full[vs], (uint32_t)(8 * Q * nh));
+                    for (int j = 0; j < nh; ++j) {
+                        const int64_t vrow = ((b * nchunks + k) * H + h0 + j) * (int64_t)Q;
+                        bulk_load(sm.cs_v[vs][j], cs + vrow, Q * 4, &sm.bar_vec_full[vs]);
+                        bulk_load(sm.dt_v[vs][j], dtc + vrow, Q * 4, &sm.bar_vec_full[vs]);
+                    }
+                }
+                const int s = (int)(un & 1);
+                if (un >= 2 && !mbar_wait(&sm.bar_free[s], (uint32_t)((un >> 1) - 1) & 1, abort))
+                    break;
+                const int row = (int)(k * Q + kTileRows * r);
+                mbar_arrive_expect_tx(&sm.bar_full[s], (uint32_t)((2 + nh) * kBoxBytes));
+                for (int a = 0; a < 2; ++a)
+                    tma_load_4d(&sm.Bs[s][a][0], &tm_b, &sm.bar_full[s], 64 * a, g, row, (int)b);
+                for (int j = 0; j < nh; ++j)
+                    tma_load_4d(&sm.Xs[s][j][0], &tm_x, &sm.bar_full[s], 0, h0 + j, row, (int)b);
+            }
+        }
+    } else if (warp >= 1 && warp <= 3) {
+        // ---------------- MMA issuer for head j = warp - 1: S_j (+)= B^T (w o X_j); lane 0
+        // alone runs the loop (see the chunk state kernel)
+        const int j = warp - 1;
+        if (j < nh && lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, kP, true, true);
+            const uint32_t d = tmem + 64 * j;
+            for (int64_t un = 0; un < nunits; ++un) {
+                const int64_t k = un / nrb;
+                const int r = (int)(un % nrb);
+                const int s = (int)(un & 1);
+                if (!mbar_wait(&sm.bar_ready[s], (uint32_t)(un >> 1) & 1, abort)) break;
+                if (r == 0 && k >= 1 &&
+                    !mbar_wait(&sm.bar_acc_free[j], (uint32_t)(k - 1) & 1, abort))
+                    break;
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(&sm.Bs[s][0][0]);
+                const uint32_t b0 = smem_u32(&sm.Xs[s][j][0]);
+                for (int kk = 0; kk < kTileRows / 16; ++kk)
+                    mma_bf16(d, smem_desc_sw128(a0 + kk * 2048, kBoxBytes, 1024),
+                             smem_desc_sw128(b0 + kk * 2048, kBoxBytes, 1024), idesc,
+                             (r > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&sm.bar_free[s]);
+                if (r == nrb - 1) mma_commit(&sm.bar_acc_full[j]);
+            }
+        }
+    } else if (warp >= 4 && warp < 12) {
+        // ---------------- scale x rows of every head by w_tau = exp(cs_last - cs_tau) dt_tau
+        const int st = threadIdx.x - 128;             // 0..255
+        for (int64_t un = 0; un < nunits; ++un) {
+            const int64_t k = un / nrb;
+            const int r = (int)(un % nrb);
+            const int s = (int)(un & 1);
+            const int vs = (int)(k & 1);
+            if (!warp_wait(&sm.bar_full[s], (uint32_t)(un >> 1) & 1, abort)) break;
+            if (!warp_wait(&sm.bar_vec_full[vs], (uint32_t)(k >> 1) & 1, abort)) break;
+            for (int c = st; c < nh * kTileRows * 8; c += 256) {
+                const int j = c / (kTileRows * 8);
+                const int pc = c % (kTileRows * 8);
+                const int tau = kTileRows * r + (pc >> 3);
+                const float w = __expf(sm.cs_v[vs][j][Q - 1] - sm.cs_v[vs][j][tau]) *
+                                sm.dt_v[vs][j][tau];
+                uint4 *ptr = reinterpret_cast<uint4 *>(&sm.Xs[s][j][0]) + pc;
+                uint4 v = *ptr;
+                uint32_t *wv = &v.x;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162 *>(&wv[e]));
+                    const float2 sc = fmul2(f, make_float2(w, w));
+                    wv[e] = pack_bf16x2(sc.x, sc.y);
+                }
+                *ptr = v;
+            }
+            fence_async_smem();
+            mbar_arrive(&sm.bar_ready[s]);
+            if (r == nrb - 1) mbar_arrive(&sm.bar_vec_free[vs]);
+        }
+    } else {
+        // ---------------- state epilogue: lane n (TMEM lane), columns p in [32 half, +32)
+        const int qd = warp & 3;
+        const int half = (warp - 12) >> 2;
+        const int n = qd * 32 + lane;
+        const int p0 = 32 * half;
+        const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
+        // initial state (caller layout [p][n]) -> TMEM h
+        for (int j = 0; j < nh; ++j) {
+            uint32_t hv[16];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const int p = p0 + 16 * hh + c;
+                    hv[c] = __float_as_uint(
+                        init ? init[((b * H + h0 + j) * kP + p) * (int64_t)kN + n] : 0.f);
+                }
+                tmem_st16(lane_base + 256 + 64 * j + p0 + 16 * hh, hv);
+            }
+        }
+        tmem_st_wait();
+        bool ok = true;
+        for (int64_t k = 0; ok && k < nchunks; ++k) {
+            const int vs = (int)(k & 1);
+            if (!warp_wait(&sm.bar_vec_full[vs], (uint32_t)(k >> 1) & 1, abort)) break;
+            for (int j = 0; j < nh; ++j) {
+                if (!warp_wait(&sm.bar_acc_full[j], (uint32_t)k & 1, abort)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t sv[32], hv[32];
+                tmem_ld32(lane_base + 64 * j + p0, sv);
+                tmem_ld32(lane_base + 256 + 64 * j + p0, hv);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&sm.bar_acc_free[j]);
+                const float a = __expf(sm.cs_v[vs][j][Q - 1]);
+                // the state entering chunk k, bf16, [p][n]: 64 contiguous bytes per warp store
+                bf16 *out = hin + (((b * nchunks + k) * H + h0 + j) * kP + p0) * (int64_t)kN + n;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) out[c * kN] = __float2bfloat16_rn(__uint_as_float(hv[c]));
+                uint32_t nv[16];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        nv[c] = __float_as_uint(fmaf(a, __uint_as_float(hv[16 * hh + c]),
+                                                     __uint_as_float(sv[16 * hh + c])));
+                    tmem_st16(lane_base + 256 + 64 * j + p0 + 16 * hh, nv);
+                }
+                tmem_st_wait();
+            }
+            if (ok) mbar_arrive(&sm.bar_vec_free[vs]);
+        }
+        if (ok && final_state) {
+            for (int j = 0; j < nh; ++j) {
+                uint32_t hv[32];
+                tmem_ld32(lane_base + 256 + 64 * j + p0, hv);
+                tmem_ld_wait();
+                float *fo = final_state + ((b * H + h0 + j) * kP + p0) * (int64_t)kN + n;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) fo[c * kN] = __uint_as_float(hv[c]);
+            }
+        }
+    }
+
+    __syncthreads();
+    if (sm.abort) {
+        if (warp >= 1 && warp <= 3 && lane == 0) {
+            mma_commit(&sm.bar_drain);
+            mbar_wait_drain(&sm.bar_drain, 0);
+        }
+        if (threadIdx.x == 0) {
+            drain_sleep();
+            atomicOr(status, 4);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kFusedTmemCols);
     }
 }
 
@@ -413,113 +665,97 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
                                 64 * a, g, (int)(t0 + kTileRows * r), (int)b);
         }
-        for (int j = 0; j < nh; ++j) {
+        for (int j = 0; lane == 0 && j < nh; ++j) {   // lane 0 alone runs the loop
             const int h = h0 + j;
             const int vs = j % kVecStages;
             const uint32_t vu = j / kVecStages;
-            if (j >= kVecStages && !warp_wait(&sm.bar_vec_free[vs], (vu - 1) & 1, abort)) break;
-            if (lane == 0) {
-                const int64_t vrow = ((b * nchunks + k) * H + h) * (int64_t)Q;
-                mbar_arrive_expect_tx(&sm.bar_vec_full[vs], (uint32_t)(8 * Q));
-                bulk_load(sm.cs_v[vs], cs + vrow, Q * 4, &sm.bar_vec_full[vs]);
-                bulk_load(sm.dt_v[vs], dtc + vrow, Q * 4, &sm.bar_vec_full[vs]);
-            }
+            if (j >= kVecStages && !mbar_wait(&sm.bar_vec_free[vs], (vu - 1) & 1, abort)) break;
+            const int64_t vrow = ((b * nchunks + k) * H + h) * (int64_t)Q;
+            mbar_arrive_expect_tx(&sm.bar_vec_full[vs], (uint32_t)(8 * Q));
+            bulk_load(sm.cs_v[vs], cs + vrow, Q * 4, &sm.bar_vec_full[vs]);
+            bulk_load(sm.dt_v[vs], dtc + vrow, Q * 4, &sm.bar_vec_full[vs]);
             const int xs = j % nst;
             const uint32_t xu = j / nst;
-            if (j >= nst && !warp_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) break;
-            if (xs == 2 && xu == 0 && !warp_wait(&sm.bar_g, 0, abort)) break;  // B tile in use
-            if (lane == 0) {
-                uint8_t *stg = scan_stage(sm, xs);
-                mbar_arrive_expect_tx(&sm.bar_xh_full[xs],
-                                      (uint32_t)(KI * kRowBytes + 2 * kP * kRowBytes));
-                for (int r = 0; r <= T; ++r)
-                    tma_load_4d(stg + r * kBoxBytes, &tm_x, &sm.bar_xh_full[xs], 0, h,
-                                (int)(t0 + kTileRows * r), (int)b);
-                const int hrow = (int)(((b * nchunks + k) * H + h) * kP);
-                for (int a = 0; a < 2; ++a)
-                    tma_load_2d(stg + kHOff + a * kP * kRowBytes, &tm_h, &sm.bar_xh_full[xs],
-                                64 * a, hrow);
-            }
-            __syncwarp();
+            if (j >= nst && !mbar_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) break;
+            if (xs == 2 && xu == 0 && !mbar_wait(&sm.bar_g, 0, abort)) break;  // B tile in use
+            uint8_t *stg = scan_stage(sm, xs);
+            mbar_arrive_expect_tx(&sm.bar_xh_full[xs],
+                                  (uint32_t)(KI * kRowBytes + 2 * kP * kRowBytes));
+            for (int r = 0; r <= T; ++r)
+                tma_load_4d(stg + r * kBoxBytes, &tm_x, &sm.bar_xh_full[xs], 0, h,
+                            (int)(t0 + kTileRows * r), (int)b);
+            const int hrow = (int)(((b * nchunks + k) * H + h) * kP);
+            for (int a = 0; a < 2; ++a)
+                tma_load_2d(stg + kHOff + a * kP * kRowBytes, &tm_h, &sm.bar_xh_full[xs],
+                            64 * a, hrow);
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer (lane 0 alone runs the loop: a lane that issued
+        // tcgen05.mma and then rejoins its warp stalls for the MMAs' issue latency)
         const uint32_t id_g = idesc_bf16_f32(128, KI, false, false);
         const uint32_t id_kk = idesc_bf16_f32(128, kP, false, false);   // K-major A and B
         const uint32_t id_kmn = idesc_bf16_f32(128, kP, false, true);   // B (x) MN-major
         const uint32_t c0 = smem_u32(&sm.Cs[0][0]);
         const uint32_t rg = smem_u32(sm.R);
-        bool ok = warp_wait(&sm.bar_cb, 0, abort);
+        bool ok = lane == 0 && mbar_wait(&sm.bar_cb, 0, abort);
         if (ok) {
             tc_fence_after();
-            if (lane == 0) {
-                // G = C B^T: M = 128 rows t, N = KI columns i, K = 128 (n)
-                for (int kk = 0; kk < kN / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    const uint32_t boff = (kk >> 2) * KI * kRowBytes + (kk & 3) * 32;
-                    mma_bf16(tmem, smem_desc_sw128(c0 + off, 16, 1024),
-                             smem_desc_sw128(rg + boff, 16, 1024), id_g, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(&sm.bar_g);
+            // G = C B^T: M = 128 rows t, N = KI columns i, K = 128 (n)
+            for (int kk = 0; kk < kN / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                const uint32_t boff = (kk >> 2) * KI * kRowBytes + (kk & 3) * 32;
+                mma_bf16(tmem, smem_desc_sw128(c0 + off, 16, 1024),
+                         smem_desc_sw128(rg + boff, 16, 1024), id_g, kk > 0 ? 1u : 0u);
             }
-            __syncwarp();
+            mma_commit(&sm.bar_g);
         }
-        if (ok && T) ok = warp_wait(&sm.bar_goff, 0, abort);   // bf16 C B_off^T in smem
+        if (ok && T) ok = mbar_wait(&sm.bar_goff, 0, abort);   // bf16 C B_off^T in smem
         for (int j = 0; ok && j < nh; ++j) {
             const int xs = j % nst;
             const uint32_t xu = j / nst;
             const int a = j & 1;
-            if (!warp_wait(&sm.bar_xh_full[xs], xu & 1, abort)) break;
-            if (T && !warp_wait(&sm.bar_xv_ready[xs], xu & 1, abort)) break;
-            if (j >= 2 && !warp_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
+            if (!mbar_wait(&sm.bar_xh_full[xs], xu & 1, abort)) break;
+            if (T && !mbar_wait(&sm.bar_xv_ready[xs], xu & 1, abort)) break;
+            if (j >= 2 && !mbar_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
             tc_fence_after();
             const uint32_t stg = smem_u32(scan_stage(sm, xs));
             const uint32_t dD = tmem + kAccCol + 128 * a, dA = dD + 64;
-            if (lane == 0) {
-                uint32_t acc = 0;
-                if (T) {
-                    // Y_A = (C B_off^T) (v dt o X_off): A = bf16 block in R, K = 128 (i)
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t aoff = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                        mma_bf16(dA, smem_desc_sw128(rg + aoff, 16, 1024),
-                                 smem_desc_sw128(stg + kk * 2048, 256 * kRowBytes, 1024), id_kmn,
-                                 acc);
-                        acc = 1;
-                    }
-                }
-                // Y_A (+)= C h^T: K = 128 (n); h = h_in (T = 0) or exp(cs_127) h_in (T = 1)
-                for (int kk = 0; kk < kN / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    const uint32_t hoff = kHOff + (kk >> 2) * (kP * kRowBytes) + (kk & 3) * 32;
-                    mma_bf16(dA, smem_desc_sw128(c0 + off, 16, 1024),
-                             smem_desc_sw128(stg + hoff, 16, 1024), id_kk, acc);
+            uint32_t acc = 0;
+            if (T) {
+                // Y_A = (C B_off^T) (v dt o X_off): A = bf16 block in R, K = 128 (i)
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t aoff = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                    mma_bf16(dA, smem_desc_sw128(rg + aoff, 16, 1024),
+                             smem_desc_sw128(stg + kk * 2048, 256 * kRowBytes, 1024), id_kmn,
+                             acc);
                     acc = 1;
                 }
             }
-            __syncwarp();
+            // Y_A (+)= C h^T: K = 128 (n); h = h_in (T = 0) or exp(cs_127) h_in (T = 1)
+            for (int kk = 0; kk < kN / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                const uint32_t hoff = kHOff + (kk >> 2) * (kP * kRowBytes) + (kk & 3) * 32;
+                mma_bf16(dA, smem_desc_sw128(c0 + off, 16, 1024),
+                         smem_desc_sw128(stg + hoff, 16, 1024), id_kk, acc);
+                acc = 1;
+            }
             for (int qb = 0; qb < 2; ++qb) {
                 const uint32_t blk = 2 * j + qb;           // P blocks are numbered per head
                 const uint32_t slot = blk % kRing, su = blk / kRing;
-                if (!warp_wait(&sm.bar_slot_full[slot], su & 1, abort)) { ok = false; break; }
+                if (!mbar_wait(&sm.bar_slot_full[slot], su & 1, abort)) { ok = false; break; }
                 tc_fence_after();
-                if (lane == 0) {
-                    // Y_diag += P[:, 64qb : +64] X[xdiag + 64qb : +64, :], P read from TMEM
-                    const uint32_t pa = tmem + pcol + 32 * slot;
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bd = smem_desc_sw128(
-                            stg + (xdiag / 16 + qb * 4 + kk) * 2048, 256 * kRowBytes, 1024);
-                        mma_bf16_ts(dD, pa + 8 * kk, bd, id_kmn, (qb | kk) != 0 ? 1u : 0u);
-                    }
-                    mma_commit(&sm.bar_slot_free[slot]);
+                // Y_diag += P[:, 64qb : +64] X[xdiag + 64qb : +64, :], P read from TMEM
+                const uint32_t pa = tmem + pcol + 32 * slot;
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bd = smem_desc_sw128(
+                        stg + (xdiag / 16 + qb * 4 + kk) * 2048, 256 * kRowBytes, 1024);
+                    mma_bf16_ts(dD, pa + 8 * kk, bd, id_kmn, (qb | kk) != 0 ? 1u : 0u);
                 }
-                __syncwarp();
+                mma_commit(&sm.bar_slot_free[slot]);
             }
             if (!ok) break;
-            if (lane == 0) {
-                mma_commit(&sm.bar_acc_full[a]);
-                mma_commit(&sm.bar_xh_free[xs]);
-            }
-            __syncwarp();
+            mma_commit(&sm.bar_acc_full[a]);
+            mma_commit(&sm.bar_xh_free[xs]);
         }
     } else if (warp >= 4) {
         // ---------------- workers: mask of head j (for T = 1 after scaling x_off and h_in),
@@ -802,6 +1038,36 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
     chunk_state_tc_kernel<<<grid, kStateThreads, smem, st>>>(mx, mb, dtc, cs, states, status,
                                                              H, G, Q, nchunks, nhb, hpc);
     *why = "chunk state (tcgen05) launch";
+    return cudaGetLastError();
+}
+
+// The fused chunk state + state passing kernel walks the chunks of a (batch, group, 3 heads)
+// block in order, one CTA per block, so it needs about one block per SM to keep the GPU busy; at
+// the shapes measured so far (b 4 x H 80, b 2 x H 24, b 1 x H 32 with 8 groups) the two-kernel
+// path was faster, so the fused form is used only on request.
+bool fused_state_pass_ok(int64_t, int, int) { return false; }
+
+cudaError_t launch_chunk_state_pass_tc(const bf16 *x, const float *dtc, const bf16 *B,
+                                       const float *cs, const float *init, float *final_state,
+                                       bf16 *hin, int *status, int64_t batch, int64_t seqlen,
+                                       int H, int G, int Q, int64_t nchunks, cudaStream_t st,
+                                       const char **why)
+{
+    CUtensorMap mx, mb;
+    if (!make_seq_map(&mx, x, batch, seqlen, H, kP) || !make_seq_map(&mb, B, batch, seqlen, G, kN)) {
+        *why = "fused chunk state: cuTensorMapEncodeTiled failed";
+        return cudaErrorInvalidValue;
+    }
+    const int hpg = H / G;
+    const int nhb = (hpg + kFusedHeads - 1) / kFusedHeads;
+    const size_t smem = sizeof(FusedSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(chunk_state_pass_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) { *why = "fused chunk state: set smem attribute"; return e; }
+    const unsigned grid = (unsigned)(batch * G * nhb);
+    chunk_state_pass_tc_kernel<<<grid, kFusedThreads, smem, st>>>(
+        mx, mb, dtc, cs, init, final_state, hin, status, H, G, Q, nchunks, nhb);
+    *why = "fused chunk state (tcgen05) launch";
     return cudaGetLastError();
 }
 

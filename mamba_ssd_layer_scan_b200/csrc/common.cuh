@@ -69,6 +69,14 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
                                   cudaStream_t st, const char **why);
+// Chunk state and state passing in one kernel (chunks walked in order per block of heads):
+// writes the bf16 entering states and the float32 final state; no float32 chunk states.
+bool fused_state_pass_ok(int64_t batch, int H, int G);
+cudaError_t launch_chunk_state_pass_tc(const bf16 *x, const float *dtc, const bf16 *B,
+                                       const float *cs, const float *init, float *final_state,
+                                       bf16 *hin, int *status, int64_t batch, int64_t seqlen,
+                                       int H, int G, int Q, int64_t nchunks, cudaStream_t st,
+                                       const char **why);
 cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,

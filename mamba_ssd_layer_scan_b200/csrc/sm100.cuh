@@ -76,21 +76,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may stay suspended (issuing nothing) until the phase
+// completes or about `suspend_ns` nanoseconds have passed.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t suspend_ns)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns) : "memory");
+    return ok != 0;
+}
+
+constexpr uint32_t kSuspendNs = 1000000;   // longest single suspension inside a bounded wait
+
 // Wait for the phase of `bar` with the given parity to complete.  Gives up -- setting *abort --
 // after kWaitLimitNs, or as soon as another thread of the CTA has set *abort.  Returns false
-// when it gave up.
+// when it gave up.  Between checks the thread sleeps in the barrier instead of spinning, so
+// waiting warps leave the issue slots to the warps that work.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
-            if (*abort) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
-                *abort = 1;
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            return false;
         }
     }
 }
@@ -100,7 +114,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 __device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity)
 {
     const unsigned long long t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity))
+    while (!mbar_try_wait_sleep(bar, parity, kSuspendNs))
         if (globaltimer() - t0 > kWaitLimitNs) return;
 }
 

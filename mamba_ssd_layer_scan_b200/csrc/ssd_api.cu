@@ -12,6 +12,7 @@
 // nothing synchronises; errors are reported through the returned status.
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "../../include/ssd.h"
@@ -65,6 +66,18 @@ ssd_status check_shape(const ssd_shape *s, bool need_seq)
     if (s->nheads > 65535 || s->batch > 65535)
         return fail(SSD_ERR_UNSUPPORTED, "batch and nheads must be <= 65535");
     return SSD_OK;
+}
+
+// Tensor-core path: chunk state and state passing run either as one fused kernel or as two
+// kernels; ssd::fused_state_pass_ok picks the form, and the environment variable
+// SSD_STATE_PASSING=fused|split forces one (both compute the same result; the switch exists to
+// test and time each).
+bool use_fused_state_pass(int64_t batch, int H, int G)
+{
+    const char *f = getenv("SSD_STATE_PASSING");
+    if (f && strcmp(f, "fused") == 0) return true;
+    if (f && strcmp(f, "split") == 0) return false;
+    return ssd::fused_state_pass_ok(batch, H, G);
 }
 
 bool valid_chunk(int q) { return q == 16 || q == 32 || q == 64 || q == 128 || q == 256; }
@@ -177,17 +190,29 @@ ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, cons
     if (tc) {
         const char *why = "";
         ssd::bf16 *hin = reinterpret_cast<ssd::bf16 *>(ws + wl.hin_bf16);
-        e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs,
-                                       states, status, s.batch, s.seqlen, H, G, Q, nchunks,
-                                       cs_stream, &why);
-        if (e != cudaSuccess) return cuda_fail(e, why);
-        if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess)
-            return cuda_fail(e, "record stage event");
-        e = ssd::launch_state_passing(states, cs, init_state, final_state, hin, s.batch, H, P,
-                                      N, Q, nchunks, cs_stream);
-        if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
-        if ((e = record(stage_events, 3, cs_stream)) != cudaSuccess)
-            return cuda_fail(e, "record stage event");
+        if (use_fused_state_pass(s.batch, H, G)) {
+            // chunk state and state passing in one launch; the passing stage is then empty
+            e = ssd::launch_chunk_state_pass_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B,
+                                                cs, init_state, final_state, hin, status,
+                                                s.batch, s.seqlen, H, G, Q, nchunks, cs_stream,
+                                                &why);
+            if (e != cudaSuccess) return cuda_fail(e, why);
+            if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess ||
+                (e = record(stage_events, 3, cs_stream)) != cudaSuccess)
+                return cuda_fail(e, "record stage event");
+        } else {
+            e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs,
+                                           states, status, s.batch, s.seqlen, H, G, Q, nchunks,
+                                           cs_stream, &why);
+            if (e != cudaSuccess) return cuda_fail(e, why);
+            if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess)
+                return cuda_fail(e, "record stage event");
+            e = ssd::launch_state_passing(states, cs, init_state, final_state, hin, s.batch, H,
+                                          P, N, Q, nchunks, cs_stream);
+            if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
+            if ((e = record(stage_events, 3, cs_stream)) != cudaSuccess)
+                return cuda_fail(e, "record stage event");
+        }
         e = ssd::launch_chunk_scan_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B,
                                       (const ssd::bf16 *)C, cs, hin, D, (ssd::bf16 *)y, status,
                                       s.batch, s.seqlen, H, G, Q, nchunks, cs_stream, &why);

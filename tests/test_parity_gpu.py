@@ -100,15 +100,35 @@ def test_small_full_parity(cuda_device, name, w, chunk):
     check_against_oracle(inp, y, final)
 
 
-# ------------------------------------------------------------------ full-size workloads
-FULL = [("ssd_370m", configs.SSD_370M, None),
-        ("ssd_2p7b", configs.SSD_2P7B, 24),
-        ("ssd_long", configs.SSD_LONG, 8)]
+# The tensor-core path carries states across chunks either in one fused kernel (chunk state and
+# state passing together, chosen when it fills the GPU) or in two kernels; force each in turn.
+TC_SMALL = [s for s in SMALL if s[0].startswith("bf16_tc")]
 
 
-@pytest.mark.parametrize("name,w,npairs", FULL, ids=[f[0] for f in FULL])
-def test_full_size_parity(cuda_device, name, w, npairs):
+@pytest.mark.parametrize("form", ["fused", "split"])
+@pytest.mark.parametrize("name,w,chunk", TC_SMALL, ids=[s[0] for s in TC_SMALL])
+def test_small_parity_each_state_passing_form(cuda_device, monkeypatch, form, name, w, chunk):
     import torch
+    monkeypatch.setenv("SSD_STATE_PASSING", form)
+    inp = inputs.make_inputs(w.with_(init_state=True, seed=w.seed + 17))
+    t = torch_inputs(inp, cuda_device)
+    y, final = run_fwd(torch, t, inp.w, chunk, cuda_device)
+    check_against_oracle(inp, y, final)
+
+
+# ------------------------------------------------------------------ full-size workloads
+FULL = [("ssd_370m", configs.SSD_370M, None, None),
+        ("ssd_2p7b", configs.SSD_2P7B, 24, None),
+        ("ssd_2p7b_split", configs.SSD_2P7B, 12, "split"),
+        ("ssd_long", configs.SSD_LONG, 8, None),
+        ("ssd_long_fused", configs.SSD_LONG, 4, "fused")]
+
+
+@pytest.mark.parametrize("name,w,npairs,form", FULL, ids=[f[0] for f in FULL])
+def test_full_size_parity(cuda_device, monkeypatch, name, w, npairs, form):
+    import torch
+    if form:
+        monkeypatch.setenv("SSD_STATE_PASSING", form)
     inp = inputs.make_inputs(w)
     t = torch_inputs(inp, cuda_device)
     y, final = run_fwd(torch, t, w, w.chunk, cuda_device, guards=False)
