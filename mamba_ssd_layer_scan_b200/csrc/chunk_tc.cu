@@ -28,7 +28,7 @@
 // Roles (warp-specialised; every wait is on an mbarrier and bounded, see sm100.cuh):
 //   state kernel: warp 0 TMA, warps 1 and 3 MMA (alternate heads), warp 2 TMEM owner,
 //                 warps 4-11 scale, 12-15 epilogue
-//   scan  kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-11 mask + epilogue
+//   scan  kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-19 mask + epilogue
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -530,7 +530,7 @@ struct alignas(1024) ScanSmem {
                                     // [n atom][64 rows p][64 n]
     float cs_v[kVecStages][256];    // per stage: the head's chunk-local cumsum row
     float dt_v[kVecStages][256];    // per stage: the head's dt row (0 past the end)
-    float vt[8][128];               // per mask warp: exp(cs_r - cs_i) dt_i over the tile
+    float vt[16][32];               // per worker warp: column factors of its two slices
     float Dv[kMaxHeadsPerCta];      // D of the CTA's heads
     uint64_t bar_cb, bar_g, bar_goff;
     uint64_t bar_xh_full[kXStagesMax], bar_xh_free[kXStagesMax], bar_xv_ready[kXStagesMax];
@@ -541,10 +541,11 @@ struct alignas(1024) ScanSmem {
     uint32_t tmem_base;
     int abort;
 };
-// warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warp 3 idle, warps 4-11 workers: two per TMEM lane
-// quarter, each owning one 32-column half of every 64-column block; per head they build their
-// half of P (mask) and then run the epilogue of the previous head for their half of y
-constexpr int kScanThreads = 384;
+// warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warp 3 idle, warps 4-19 workers: four per TMEM
+// lane quarter, each owning a 16-column slice of every 64-column block; per head they build
+// their slice of P (mask) and then run the epilogue of the previous head for their slice of y
+constexpr int kScanWorkers = 512;
+constexpr int kScanThreads = 128 + kScanWorkers;
 constexpr uint32_t kScanTmemCols = 512;
 constexpr uint32_t kAccCol = 256;   // accumulator buffer a: Y_diag at 256 + 128 a, Y_A at +64
 
@@ -616,23 +617,23 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_cb, 1);
         mbar_init(&sm.bar_g, 1);
-        mbar_init(&sm.bar_goff, 256);
+        mbar_init(&sm.bar_goff, kScanWorkers);
         for (int s = 0; s < kXStagesMax; ++s) {
             mbar_init(&sm.bar_xh_full[s], 1);
             mbar_init(&sm.bar_xh_free[s], 1);
-            mbar_init(&sm.bar_xv_ready[s], 256);
+            mbar_init(&sm.bar_xv_ready[s], kScanWorkers);
         }
         for (int s = 0; s < kVecStages; ++s) {
             mbar_init(&sm.bar_vec_full[s], 1);
-            mbar_init(&sm.bar_vec_free[s], 256);
+            mbar_init(&sm.bar_vec_free[s], kScanWorkers);
         }
         for (int s = 0; s < kRing; ++s) {
-            mbar_init(&sm.bar_slot_full[s], 256);
+            mbar_init(&sm.bar_slot_full[s], kScanWorkers);
             mbar_init(&sm.bar_slot_free[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sm.bar_acc_full[a], 1);
-            mbar_init(&sm.bar_acc_free[a], 256);
+            mbar_init(&sm.bar_acc_free[a], kScanWorkers);
         }
         mbar_init(&sm.bar_drain, 1);
         sm.abort = 0;
@@ -758,29 +759,46 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mma_commit(&sm.bar_xh_free[xs]);
         }
     } else if (warp >= 4) {
-        // ---------------- workers: mask of head j (for T = 1 after scaling x_off and h_in),
-        // then the epilogue y = Y_diag + f_t Y_A of head j - 1, each for this warp's half
-        const int mt = threadIdx.x - 128;          // 0..255
+        // ---------------- workers, four per TMEM lane quarter.  Warp (qd, cq) owns rows
+        // t = 32 qd + lane of the tile and the 16-column slice [16 cq, 16 cq + 16) of every
+        // 64-column block: per head it builds that slice of both P blocks (mask; for T = 1 after
+        // its share of scaling x_off and h_in), then the epilogue y = Y_diag + f_t Y_A of the
+        // previous head for output columns [16 cq, 16 cq + 16).
+        const int wt = threadIdx.x - 128;          // 0 .. kScanWorkers - 1
         const int qd = warp & 3;
-        const int half = (warp - 4) >> 2;          // which 32 columns of each 64-column block
+        const int cq = (warp - 4) >> 2;
         const int t = qd * 32 + lane;             // row within the tile = TMEM lane
         const int tau = kTileRows * T + t;        // row within the chunk
         const int r = kTileRows * T + qd * 32 - 1;  // last row above this warp's 32-row slice
         const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
         float *vt = sm.vt[warp - 4];
+        // The slice of block qb is the 16-column unit u = 4 qb + cq of the diagonal block; its
+        // class relative to this row quarter: 0 below the 32 x 32 diagonal sub-block, 1 inside
+        // it, 2 above it (all zero).
+        const int u0 = cq, u1 = 4 + cq;
+        const int cls0 = u0 < 2 * qd ? 0 : (u0 <= 2 * qd + 1 ? 1 : 2);
+        const int cls1 = u1 < 2 * qd ? 0 : (u1 <= 2 * qd + 1 ? 1 : 2);
         bool ok = warp_wait(&sm.bar_g, 0, abort);
         tc_fence_after();
+        // this warp's part of the diagonal block of C B^T, kept in registers for every head
+        uint32_t g0[16], g1[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) g0[c] = g1[c] = 0u;
+        if (ok) {
+            if (cls0 < 2) tmem_ld16(lane_base + gdiag + 16 * u0, g0);
+            if (cls1 < 2) tmem_ld16(lane_base + gdiag + 16 * u1, g1);
+            tmem_ld_wait();
+        }
         if (ok && T) {
             // C B_off^T (TMEM columns [0, 128)) -> bf16, K-major swizzled tile in R; this warp
-            // converts its 32 rows x 64 columns [64 half, 64 half + 64)
-            uint8_t *dst = sm.R + half * kBoxBytes + t * kRowBytes;
-            uint32_t gv[64];
-            tmem_ld32(lane_base + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(gv));
-            tmem_ld32(lane_base + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(gv + 32));
+            // converts its 32 rows x columns [32 cq, 32 cq + 32)
+            uint32_t gv[32];
+            tmem_ld32(lane_base + 32 * cq, gv);
             tmem_ld_wait();
+            uint8_t *dst = sm.R + (cq >> 1) * kBoxBytes + t * kRowBytes;
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int pos = m ^ (t & 7);
+            for (int m = 0; m < 4; ++m) {
+                const int pos = ((cq & 1) * 4 + m) ^ (t & 7);
                 *reinterpret_cast<uint4 *>(dst + pos * 16) = make_uint4(
                     pack_bf16x2(__uint_as_float(gv[8 * m]), __uint_as_float(gv[8 * m + 1])),
                     pack_bf16x2(__uint_as_float(gv[8 * m + 2]), __uint_as_float(gv[8 * m + 3])),
@@ -801,59 +819,54 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 if (!warp_wait(&sm.bar_vec_full[vs], (j / kVecStages) & 1, abort)) break;
                 const float *cs_s = sm.cs_v[vs];
                 const float *dt_s = sm.dt_v[vs];
-                // this warp's two 32-column sub-blocks of the diagonal block: sbl = 2 qb + half
-                const int sb0 = half, sb1 = 2 + half;
-                uint32_t g0[32], g1[32];
-                if (sb0 <= qd) tmem_ld32(lane_base + gdiag + 32 * sb0, g0);
-                if (sb1 <= qd) tmem_ld32(lane_base + gdiag + 32 * sb1, g1);
                 if (T) {
                     // x rows [0, 128) *= exp(cs_127 - cs_i) dt_i; h_in *= exp(cs_127)
                     const int xs = j % nst;
                     if (!warp_wait(&sm.bar_xh_full[xs], (j / nst) & 1, abort)) break;
                     uint8_t *stg = scan_stage(sm, xs);
                     const float c127 = cs_s[127];
-                    scale_pieces<4>(stg, mt, 256, [&](int c) {
+                    scale_pieces<1024 / kScanWorkers>(stg, wt, kScanWorkers, [&](int c) {
                         const int i = c >> 3;
                         return __expf(c127 - cs_s[i]) * dt_s[i];
                     });
                     const float sh = __expf(c127);
-                    scale_pieces<4>(stg + kHOff, mt, 256, [&](int) { return sh; });
+                    scale_pieces<1024 / kScanWorkers>(stg + kHOff, wt, kScanWorkers,
+                                                      [&](int) { return sh; });
                     fence_async_smem();
                     mbar_arrive(&sm.bar_xv_ready[xs]);
                 }
                 const float Dh = sm.Dv[j];
                 const float ct = cs_s[tau];
-                // Column factors over this warp's sub-blocks (local column lc = 32 sbl + lane):
-                // below the 32 x 32 diagonal sub-block (sbl < qd) relative to row r, both
-                // factors <= 1; inside it (sbl == qd) relative to m = r + 1, the slice's first
-                // row: exp(cs_m - cs_i) <= exp(32 max|dt A|) and exp(cs_t - cs_m) <= 1, so
-                // neither over- nor underflows, and no element needs an exponential of its own.
+                // Row and column factors: below the 32 x 32 diagonal sub-block relative to row r,
+                // both <= 1; inside it relative to m = r + 1, the slice's first row:
+                // exp(cs_m - cs_i) <= exp(32 max|dt A|) and exp(cs_t - cs_m) <= 1, so neither
+                // over- nor underflows, and no element needs an exponential of its own.
                 const float cm = cs_s[r + 1];
+                const float crf = cs_s[r < 0 ? 0 : r];
                 const float um = __expf(ct - cm);
-                __syncwarp();
-#pragma unroll
-                for (int qb = 0; qb < 2; ++qb) {
-                    const int sbl = qb * 2 + half;
-                    const int lc = sbl * 32 + lane;
-                    const int i = kTileRows * T + lc;
-                    if (sbl < qd) vt[lc] = __expf(cs_s[r] - cs_s[i]) * dt_s[i];
-                    else if (sbl == qd) vt[lc] = __expf(cm - cs_s[i]) * dt_s[i];
+                const float uf = qd > 0 ? __expf(ct - crf) : 0.f;
+                {
+                    // lane l: column 16 (4 (l >> 4) + cq) + (l & 15) of the diagonal block
+                    const int uu = 4 * (lane >> 4) + cq;
+                    const int cl = uu < 2 * qd ? 0 : (uu <= 2 * qd + 1 ? 1 : 2);
+                    const int i = kTileRows * T + 16 * uu + (lane & 15);
+                    const float ref = cl == 0 ? crf : cm;
+                    const float v = __expf(ref - cs_s[i]) * dt_s[i];
+                    vt[lane] = cl < 2 ? v : 0.f;
                 }
-                const float uf = qd > 0 ? __expf(ct - cs_s[r]) : 0.f;
                 __syncwarp();
-                tmem_ld_wait();
 #pragma unroll
                 for (int qb = 0; qb < 2; ++qb, ++blk) {
                     const uint32_t slot = blk % kRing, su = blk / kRing;
-                    const int sbl = qb * 2 + half;
-                    const int lc0 = 32 * sbl;
+                    const int cl = qb ? cls1 : cls0;
                     const uint32_t *gv = qb ? g1 : g0;
-                    uint32_t pk[16];
-                    if (sbl < qd) {
+                    const float *vq = vt + 16 * qb;
+                    uint32_t pk[8];
+                    if (cl == 0) {
                         const float2 uu = make_float2(uf, uf);
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const float4 vv = *reinterpret_cast<const float4 *>(vt + lc0 + 4 * c);
+                        for (int c = 0; c < 4; ++c) {
+                            const float4 vv = *reinterpret_cast<const float4 *>(vq + 4 * c);
                             const float2 p0 = fmul2(
                                 fmul2(make_float2(__uint_as_float(gv[4 * c]),
                                                   __uint_as_float(gv[4 * c + 1])),
@@ -865,28 +878,33 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                             pk[2 * c] = pack_bf16x2(p0.x, p0.y);
                             pk[2 * c + 1] = pack_bf16x2(p1.x, p1.y);
                         }
-                    } else if (sbl == qd) {
-                        // causal 32 x 32 block: column c <= lane kept, + D at c = lane
+                    } else if (cl == 1) {
+                        // inside the causal 32 x 32 sub-block: local column lc kept for
+                        // lc <= lane, + D at lc = lane
+                        const int lc0 = 16 * (qb ? u1 : u0) - 32 * qd;   // 0 or 16
+                        const float2 uu = make_float2(um, um);
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const float2 ww = *reinterpret_cast<const float2 *>(vt + lc0 + 2 * c);
-                            float p0 = __uint_as_float(gv[2 * c]) * ww.x * um;
-                            float p1 = __uint_as_float(gv[2 * c + 1]) * ww.y * um;
-                            p0 = (2 * c <= lane) ? p0 : 0.f;
-                            p1 = (2 * c + 1 <= lane) ? p1 : 0.f;
-                            p0 += (2 * c == lane) ? Dh : 0.f;
-                            p1 += (2 * c + 1 == lane) ? Dh : 0.f;
-                            pk[c] = pack_bf16x2(p0, p1);
+                        for (int c = 0; c < 8; ++c) {
+                            const float2 ww = *reinterpret_cast<const float2 *>(vq + 2 * c);
+                            float2 pp = fmul2(fmul2(make_float2(__uint_as_float(gv[2 * c]),
+                                                                __uint_as_float(gv[2 * c + 1])),
+                                                    ww), uu);
+                            const int lc = lc0 + 2 * c;
+                            pp.x = (lc <= lane) ? pp.x : 0.f;
+                            pp.y = (lc + 1 <= lane) ? pp.y : 0.f;
+                            pp.x += (lc == lane) ? Dh : 0.f;
+                            pp.y += (lc + 1 == lane) ? Dh : 0.f;
+                            pk[c] = pack_bf16x2(pp.x, pp.y);
                         }
                     } else {
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) pk[c] = 0u;
+                        for (int c = 0; c < 8; ++c) pk[c] = 0u;
                     }
                     if (su >= 1 && !warp_wait(&sm.bar_slot_free[slot], (su - 1) & 1, abort)) {
                         ok = false;
                         break;
                     }
-                    tmem_st16(lane_base + pcol + 32 * slot + 16 * half, pk);
+                    tmem_st8(lane_base + pcol + 32 * slot + 8 * cq, pk);
                     tmem_st_wait();
                     tc_fence_before();
                     mbar_arrive(&sm.bar_slot_full[slot]);
@@ -894,38 +912,36 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 if (!ok) break;
             }
             if (j >= 1) {
-                // epilogue of head jj = j - 1 for output columns [32 half, 32 half + 32)
+                // epilogue of head jj = j - 1 for output columns [16 cq, 16 cq + 16)
                 const int jj = j - 1;
                 const int a = jj & 1;
                 const int vs = jj % kVecStages;
                 if (!warp_wait(&sm.bar_acc_full[a], (jj >> 1) & 1, abort)) break;
                 tc_fence_after();
-                const uint32_t col = lane_base + kAccCol + 128 * a + 32 * half;
-                uint32_t d0[32], a0[32];
-                tmem_ld32(col, d0);
-                tmem_ld32(col + 64, a0);
+                const uint32_t col = lane_base + kAccCol + 128 * a + 16 * cq;
+                uint32_t d0[16], a0[16];
+                tmem_ld16(col, d0);
+                tmem_ld16(col + 64, a0);
                 const float f = __expf(sm.cs_v[vs][tau] - (T ? sm.cs_v[vs][127] : 0.f));
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&sm.bar_acc_free[a]);
                 mbar_arrive(&sm.bar_vec_free[vs]);   // done with this head's cs / dt
-                uint32_t pk[16];
+                uint32_t pk[8];
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
+                for (int c = 0; c < 8; ++c)
                     pk[c] = pack_bf16x2(
                         fmaf(f, __uint_as_float(a0[2 * c]), __uint_as_float(d0[2 * c])),
                         fmaf(f, __uint_as_float(a0[2 * c + 1]), __uint_as_float(d0[2 * c + 1])));
                 if (tau < len) {
                     uint4 *yrow = reinterpret_cast<uint4 *>(
-                        y + ((b * seqlen + t0 + tau) * H + h0 + jj) * (int64_t)kP + 32 * half);
-#pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        yrow[m] = make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+                        y + ((b * seqlen + t0 + tau) * H + h0 + jj) * (int64_t)kP + 16 * cq);
+                    yrow[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    yrow[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             }
         }
     }
-
     __syncthreads();
     if (sm.abort) {
         if (warp == 1 && lane == 0) {
