@@ -98,7 +98,6 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int h0 = g * hpg + hb * hpc;
     const int nh = min(hpc, hpg - hb * hpc);
     const int64_t t0 = k * Q;
-    const int nrb = Q / kTileRows;
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_b, 1);
@@ -132,10 +131,8 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
             mbar_arrive_expect_tx(&sm.bar_b, 2u * Q * kRowBytes);
-            for (int a = 0; a < 2; ++a)
-                for (int r = 0; r < nrb; ++r)
-                    tma_load_4d(&sm.Bs[a][r * kTileRows * 64], &tm_b, &sm.bar_b, 64 * a, g,
-                                (int)(t0 + kTileRows * r), (int)b);
+            for (int a = 0; a < 2; ++a)   // boxes of Q rows
+                tma_load_4d(&sm.Bs[a][0], &tm_b, &sm.bar_b, 64 * a, g, (int)t0, (int)b);
             for (int j = 0; j < nh; ++j) {
                 const int s = j % kStateStages;
                 const uint32_t use = j / kStateStages;
@@ -143,9 +140,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     break;
                 const int64_t vrow = ((b * nchunks + k) * H + h0 + j) * (int64_t)Q;
                 mbar_arrive_expect_tx(&sm.bar_x_full[s], (uint32_t)Q * (kRowBytes + 8));
-                for (int r = 0; r < nrb; ++r)
-                    tma_load_4d(&sm.Xs[s][r * kTileRows * 64], &tm_x, &sm.bar_x_full[s], 0,
-                                h0 + j, (int)(t0 + kTileRows * r), (int)b);
+                tma_load_4d(&sm.Xs[s][0], &tm_x, &sm.bar_x_full[s], 0, h0 + j, (int)t0, (int)b);
                 bulk_load(sm.cs_v[s], cs + vrow, Q * 4, &sm.bar_x_full[s]);
                 bulk_load(sm.dt_v[s], dtc + vrow, Q * 4, &sm.bar_x_full[s]);
             }
@@ -167,11 +162,18 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 if (j >= 2 && !mbar_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + a * kP;
-                const uint32_t a0 = smem_u32(&sm.Bs[0][0]), b0 = smem_u32(&sm.Xs[s][0]);
-                for (int kk = 0; kk < Q / 16; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(a0 + kk * 2048, atom_bytes, 1024);
-                    const uint64_t bd = smem_desc_sw128(b0 + kk * 2048, atom_bytes, 1024);
-                    mma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                // base descriptors + constant K steps (16 rows = 2048 bytes) in fully unrolled
+                // loops: the issuing thread's own instruction chain sets the MMA issue rate
+                const uint64_t ad = smem_desc_sw128(smem_u32(&sm.Bs[0][0]), atom_bytes, 1024);
+                const uint64_t bd = smem_desc_sw128(smem_u32(&sm.Xs[s][0]), atom_bytes, 1024);
+                if (Q == 256) {
+#pragma unroll
+                    for (int kk = 0; kk < 16; ++kk)
+                        mma_bf16(d, ad + kk * 128, bd + kk * 128, idesc, kk > 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(d, ad + kk * 128, bd + kk * 128, idesc, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&sm.bar_x_free[s]);
                 mma_commit(&sm.bar_acc_full[a]);
@@ -376,12 +378,11 @@ chunk_state_pass_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     !mbar_wait(&sm.bar_acc_free[j], (uint32_t)(k - 1) & 1, abort))
                     break;
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(&sm.Bs[s][0][0]);
-                const uint32_t b0 = smem_u32(&sm.Xs[s][j][0]);
+                const uint64_t ad = smem_desc_sw128(smem_u32(&sm.Bs[s][0][0]), kBoxBytes, 1024);
+                const uint64_t bd = smem_desc_sw128(smem_u32(&sm.Xs[s][j][0]), kBoxBytes, 1024);
+#pragma unroll
                 for (int kk = 0; kk < kTileRows / 16; ++kk)
-                    mma_bf16(d, smem_desc_sw128(a0 + kk * 2048, kBoxBytes, 1024),
-                             smem_desc_sw128(b0 + kk * 2048, kBoxBytes, 1024), idesc,
-                             (r > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16(d, ad + kk * 128, bd + kk * 128, idesc, (r > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&sm.bar_free[s]);
                 if (r == nrb - 1) mma_commit(&sm.bar_acc_full[j]);
             }
@@ -454,10 +455,12 @@ chunk_state_pass_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 tc_fence_before();
                 mbar_arrive(&sm.bar_acc_free[j]);
                 const float a = __expf(sm.cs_v[vs][j][Q - 1]);
-                // the state entering chunk k, bf16, [p][n]: 64 contiguous bytes per warp store
-                bf16 *out = hin + (((b * nchunks + k) * H + h0 + j) * kP + p0) * (int64_t)kN + n;
+                // the state entering chunk k, bf16, in the swizzled block layout: 64 bytes of
+                // one 128-byte row per warp store
+                bf16 *out = hin + ((b * nchunks + k) * H + h0 + j) * (int64_t)(kP * kN);
 #pragma unroll
-                for (int c = 0; c < 32; ++c) out[c * kN] = __float2bfloat16_rn(__uint_as_float(hv[c]));
+                for (int c = 0; c < 32; ++c)
+                    out[hin_swizzled_offset(p0 + c, n)] = __float2bfloat16_rn(__uint_as_float(hv[c]));
                 uint32_t nv[16];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -517,7 +520,7 @@ chunk_state_pass_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
 // So y = Y_diag + f_t Y_A with f_t = exp(cs_t) (T = 0) or u_t (T = 1).
 constexpr int kXStagesMax = 3;   // x / h_in stages (T = 0: 3, the third in the B tile's space;
                                  // T = 1: 2, that space holds the bf16 off-diagonal block)
-constexpr int kVecStages = 4;    // cs / dt row stages
+constexpr int kScanMaxHeads = 8; // heads per CTA
 constexpr int kRing = 4;         // 64-column blocks of P in TMEM (two heads)
 constexpr int kStageBytes = 256 * kRowBytes + 2 * kP * kRowBytes;  // x (<= 256 rows) + h_in
 constexpr int kHOff = 256 * kRowBytes;                              // h_in inside a stage
@@ -528,13 +531,13 @@ struct alignas(1024) ScanSmem {
                                     // (K-major [i atom][128 rows t][64 i])
     uint8_t S01[2][kStageBytes];    // x / h_in stages 0 and 1: [KI rows i][64 p] then
                                     // [n atom][64 rows p][64 n]
-    float cs_v[kVecStages][256];    // per stage: the head's chunk-local cumsum row
-    float dt_v[kVecStages][256];    // per stage: the head's dt row (0 past the end)
+    float cs_v[kScanMaxHeads * 256];  // the CTA's heads' chunk-local cumsum rows (stride Q)
+    float dt_v[kScanMaxHeads * 256];  // and dt rows (0 past the end), loaded once
     float vt[16][32];               // per worker warp: column factors of its two slices
     float Dv[kMaxHeadsPerCta];      // D of the CTA's heads
     uint64_t bar_cb, bar_g, bar_goff;
     uint64_t bar_xh_full[kXStagesMax], bar_xh_free[kXStagesMax], bar_xv_ready[kXStagesMax];
-    uint64_t bar_vec_full[kVecStages], bar_vec_free[kVecStages];
+    uint64_t bar_vec;
     uint64_t bar_slot_full[kRing], bar_slot_free[kRing];
     uint64_t bar_acc_full[2], bar_acc_free[2];
     uint64_t bar_drain;
@@ -586,7 +589,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c,
-                     const __grid_constant__ CUtensorMap tm_h, const float *__restrict__ dtc,
+                     const __grid_constant__ CUtensorMap tm_x2, const bf16 *__restrict__ hin,
+                     const float *__restrict__ dtc,
                      const float *__restrict__ cs, const float *__restrict__ D,
                      bf16 *__restrict__ y, int *__restrict__ status, int64_t seqlen, int H,
                      int G, int Q, int64_t nchunks, int nhb, int hpc)
@@ -623,10 +627,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_init(&sm.bar_xh_free[s], 1);
             mbar_init(&sm.bar_xv_ready[s], kScanWorkers);
         }
-        for (int s = 0; s < kVecStages; ++s) {
-            mbar_init(&sm.bar_vec_full[s], 1);
-            mbar_init(&sm.bar_vec_free[s], kScanWorkers);
-        }
+        mbar_init(&sm.bar_vec, 1);
         for (int s = 0; s < kRing; ++s) {
             mbar_init(&sm.bar_slot_full[s], kScanWorkers);
             mbar_init(&sm.bar_slot_free[s], 1);
@@ -656,7 +657,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
             tma_prefetch_desc(&tm_c);
-            tma_prefetch_desc(&tm_h);
+            tma_prefetch_desc(&tm_x2);
             mbar_arrive_expect_tx(&sm.bar_cb, (uint32_t)(2 * kBoxBytes + 2 * KI * kRowBytes));
             for (int a = 0; a < 2; ++a)
                 tma_load_4d(&sm.Cs[a][0], &tm_c, &sm.bar_cb, 64 * a, g,
@@ -665,16 +666,14 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 for (int r = 0; r <= T; ++r)
                     tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
                                 64 * a, g, (int)(t0 + kTileRows * r), (int)b);
+            // cs and dt rows of all the CTA's heads (contiguous in the workspace): two copies
+            const int64_t vrow = ((b * nchunks + k) * H + h0) * (int64_t)Q;
+            mbar_arrive_expect_tx(&sm.bar_vec, (uint32_t)(8 * Q * nh));
+            bulk_load(sm.cs_v, cs + vrow, (uint32_t)(4 * Q * nh), &sm.bar_vec);
+            bulk_load(sm.dt_v, dtc + vrow, (uint32_t)(4 * Q * nh), &sm.bar_vec);
         }
         for (int j = 0; lane == 0 && j < nh; ++j) {   // lane 0 alone runs the loop
             const int h = h0 + j;
-            const int vs = j % kVecStages;
-            const uint32_t vu = j / kVecStages;
-            if (j >= kVecStages && !mbar_wait(&sm.bar_vec_free[vs], (vu - 1) & 1, abort)) break;
-            const int64_t vrow = ((b * nchunks + k) * H + h) * (int64_t)Q;
-            mbar_arrive_expect_tx(&sm.bar_vec_full[vs], (uint32_t)(8 * Q));
-            bulk_load(sm.cs_v[vs], cs + vrow, Q * 4, &sm.bar_vec_full[vs]);
-            bulk_load(sm.dt_v[vs], dtc + vrow, Q * 4, &sm.bar_vec_full[vs]);
             const int xs = j % nst;
             const uint32_t xu = j / nst;
             if (j >= nst && !mbar_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) break;
@@ -682,13 +681,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             uint8_t *stg = scan_stage(sm, xs);
             mbar_arrive_expect_tx(&sm.bar_xh_full[xs],
                                   (uint32_t)(KI * kRowBytes + 2 * kP * kRowBytes));
-            for (int r = 0; r <= T; ++r)
-                tma_load_4d(stg + r * kBoxBytes, &tm_x, &sm.bar_xh_full[xs], 0, h,
-                            (int)(t0 + kTileRows * r), (int)b);
-            const int hrow = (int)(((b * nchunks + k) * H + h) * kP);
-            for (int a = 0; a < 2; ++a)
-                tma_load_2d(stg + kHOff + a * kP * kRowBytes, &tm_h, &sm.bar_xh_full[xs],
-                            64 * a, hrow);
+            // x rows [0, KI) of the chunk as one box (fewer, larger TMA boxes stream faster);
+            // h_in is stored in its shared-memory layout, so one contiguous copy suffices
+            tma_load_4d(stg, T ? &tm_x2 : &tm_x, &sm.bar_xh_full[xs], 0, h, (int)t0, (int)b);
+            bulk_load(stg + kHOff, hin + ((b * nchunks + k) * H + h) * (int64_t)(kP * kN),
+                      kP * kN * 2, &sm.bar_xh_full[xs]);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (lane 0 alone runs the loop: a lane that issued
@@ -696,17 +693,19 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         const uint32_t id_g = idesc_bf16_f32(128, KI, false, false);
         const uint32_t id_kk = idesc_bf16_f32(128, kP, false, false);   // K-major A and B
         const uint32_t id_kmn = idesc_bf16_f32(128, kP, false, true);   // B (x) MN-major
-        const uint32_t c0 = smem_u32(&sm.Cs[0][0]);
-        const uint32_t rg = smem_u32(sm.R);
+        // base descriptors; K steps are constant offsets added in fully unrolled loops (the
+        // issuing thread's own instruction chain sets the MMA issue rate)
+        const uint64_t cd = smem_desc_sw128(smem_u32(&sm.Cs[0][0]), 16, 1024);
+        const uint64_t rd = smem_desc_sw128(smem_u32(sm.R), 16, 1024);
         bool ok = lane == 0 && mbar_wait(&sm.bar_cb, 0, abort);
         if (ok) {
             tc_fence_after();
             // G = C B^T: M = 128 rows t, N = KI columns i, K = 128 (n)
+#pragma unroll
             for (int kk = 0; kk < kN / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
                 const uint32_t boff = (kk >> 2) * KI * kRowBytes + (kk & 3) * 32;
-                mma_bf16(tmem, smem_desc_sw128(c0 + off, 16, 1024),
-                         smem_desc_sw128(rg + boff, 16, 1024), id_g, kk > 0 ? 1u : 0u);
+                mma_bf16(tmem, cd + (off >> 4), rd + (boff >> 4), id_g, kk > 0 ? 1u : 0u);
             }
             mma_commit(&sm.bar_g);
         }
@@ -721,24 +720,22 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             tc_fence_after();
             const uint32_t stg = smem_u32(scan_stage(sm, xs));
             const uint32_t dD = tmem + kAccCol + 128 * a, dA = dD + 64;
-            uint32_t acc = 0;
+            const uint64_t xd = smem_desc_sw128(stg, 256 * kRowBytes, 1024);   // x, MN-major
+            const uint64_t hd = smem_desc_sw128(stg + kHOff, 16, 1024);        // h_in, K-major
             if (T) {
                 // Y_A = (C B_off^T) (v dt o X_off): A = bf16 block in R, K = 128 (i)
+#pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t aoff = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    mma_bf16(dA, smem_desc_sw128(rg + aoff, 16, 1024),
-                             smem_desc_sw128(stg + kk * 2048, 256 * kRowBytes, 1024), id_kmn,
-                             acc);
-                    acc = 1;
+                    mma_bf16(dA, rd + (aoff >> 4), xd + kk * 128, id_kmn, kk > 0 ? 1u : 0u);
                 }
             }
             // Y_A (+)= C h^T: K = 128 (n); h = h_in (T = 0) or exp(cs_127) h_in (T = 1)
+#pragma unroll
             for (int kk = 0; kk < kN / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                const uint32_t hoff = kHOff + (kk >> 2) * (kP * kRowBytes) + (kk & 3) * 32;
-                mma_bf16(dA, smem_desc_sw128(c0 + off, 16, 1024),
-                         smem_desc_sw128(stg + hoff, 16, 1024), id_kk, acc);
-                acc = 1;
+                const uint32_t hoff = (kk >> 2) * (kP * kRowBytes) + (kk & 3) * 32;
+                mma_bf16(dA, cd + (off >> 4), hd + (hoff >> 4), id_kk, (T || kk > 0) ? 1u : 0u);
             }
             for (int qb = 0; qb < 2; ++qb) {
                 const uint32_t blk = 2 * j + qb;           // P blocks are numbered per head
@@ -747,11 +744,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 tc_fence_after();
                 // Y_diag += P[:, 64qb : +64] X[xdiag + 64qb : +64, :], P read from TMEM
                 const uint32_t pa = tmem + pcol + 32 * slot;
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(
-                        stg + (xdiag / 16 + qb * 4 + kk) * 2048, 256 * kRowBytes, 1024);
-                    mma_bf16_ts(dD, pa + 8 * kk, bd, id_kmn, (qb | kk) != 0 ? 1u : 0u);
-                }
+                const uint64_t bd = xd + (uint64_t)((xdiag / 16 + qb * 4) * 128);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ts(dD, pa + 8 * kk, bd + kk * 128, id_kmn, (qb | kk) != 0 ? 1u : 0u);
                 mma_commit(&sm.bar_slot_free[slot]);
             }
             if (!ok) break;
@@ -778,7 +774,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         const int u0 = cq, u1 = 4 + cq;
         const int cls0 = u0 < 2 * qd ? 0 : (u0 <= 2 * qd + 1 ? 1 : 2);
         const int cls1 = u1 < 2 * qd ? 0 : (u1 <= 2 * qd + 1 ? 1 : 2);
-        bool ok = warp_wait(&sm.bar_g, 0, abort);
+        bool ok = warp_wait(&sm.bar_g, 0, abort) && warp_wait(&sm.bar_vec, 0, abort);
         tc_fence_after();
         // this warp's part of the diagonal block of C B^T, kept in registers for every head
         uint32_t g0[16], g1[16];
@@ -815,10 +811,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         uint32_t blk = 0;
         for (int j = 0; ok && j <= nh; ++j) {
             if (j < nh) {
-                const int vs = j % kVecStages;
-                if (!warp_wait(&sm.bar_vec_full[vs], (j / kVecStages) & 1, abort)) break;
-                const float *cs_s = sm.cs_v[vs];
-                const float *dt_s = sm.dt_v[vs];
+                const float *cs_s = sm.cs_v + j * Q;
+                const float *dt_s = sm.dt_v + j * Q;
                 if (T) {
                     // x rows [0, 128) *= exp(cs_127 - cs_i) dt_i; h_in *= exp(cs_127)
                     const int xs = j % nst;
@@ -915,18 +909,17 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 // epilogue of head jj = j - 1 for output columns [16 cq, 16 cq + 16)
                 const int jj = j - 1;
                 const int a = jj & 1;
-                const int vs = jj % kVecStages;
                 if (!warp_wait(&sm.bar_acc_full[a], (jj >> 1) & 1, abort)) break;
                 tc_fence_after();
                 const uint32_t col = lane_base + kAccCol + 128 * a + 16 * cq;
                 uint32_t d0[16], a0[16];
                 tmem_ld16(col, d0);
                 tmem_ld16(col + 64, a0);
-                const float f = __expf(sm.cs_v[vs][tau] - (T ? sm.cs_v[vs][127] : 0.f));
+                const float *cs_j = sm.cs_v + jj * Q;
+                const float f = __expf(cs_j[tau] - (T ? cs_j[127] : 0.f));
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&sm.bar_acc_free[a]);
-                mbar_arrive(&sm.bar_vec_free[vs]);   // done with this head's cs / dt
                 uint32_t pk[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
@@ -993,13 +986,13 @@ bool make_map(CUtensorMap *m, const void *ptr, int rank, const cuuint64_t *dims,
 // (batch, seqlen, heads_or_groups, 64 * m) bf16 -> 4-D map {inner, heads, seqlen, batch} with
 // a 64 x 1 x 128 x 1 box.
 bool make_seq_map(CUtensorMap *m, const void *ptr, int64_t batch, int64_t seqlen, int64_t mid,
-                  int64_t inner)
+                  int64_t inner, int box_rows = kTileRows)
 {
     const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)mid, (cuuint64_t)seqlen,
                                 (cuuint64_t)batch};
     const cuuint64_t strides[3] = {(cuuint64_t)(inner * 2), (cuuint64_t)(mid * inner * 2),
                                    (cuuint64_t)(seqlen * mid * inner * 2)};
-    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kTileRows, 1};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     return make_map(m, ptr, 4, dims, strides, box);
 }
 
@@ -1038,8 +1031,9 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
                                   cudaStream_t st, const char **why)
 {
-    CUtensorMap mx, mb;
-    if (!make_seq_map(&mx, x, batch, seqlen, H, kP) || !make_seq_map(&mb, B, batch, seqlen, G, kN)) {
+    CUtensorMap mx, mb;   // boxes of a whole chunk (Q rows)
+    if (!make_seq_map(&mx, x, batch, seqlen, H, kP, Q) ||
+        !make_seq_map(&mb, B, batch, seqlen, G, kN, Q)) {
         *why = "chunk state: cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
@@ -1092,29 +1086,27 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
                                  int Q, int64_t nchunks, cudaStream_t st, const char **why)
 {
-    CUtensorMap mx, mb, mc, mh;
-    const int64_t hrows = batch * nchunks * H * kP;
-    const cuuint64_t hdims[2] = {(cuuint64_t)kN, (cuuint64_t)hrows};
-    const cuuint64_t hstr[1] = {(cuuint64_t)(kN * 2)};
-    const cuuint32_t hbox[2] = {64, (cuuint32_t)kP};
-    if (hrows > 0x7fffffffLL || !make_seq_map(&mx, x, batch, seqlen, H, kP) ||
+    CUtensorMap mx, mx2, mb, mc;
+    if (!make_seq_map(&mx, x, batch, seqlen, H, kP) ||
+        !make_seq_map(&mx2, x, batch, seqlen, H, kP, 2 * kTileRows) ||
         !make_seq_map(&mb, B, batch, seqlen, G, kN) ||
-        !make_seq_map(&mc, C, batch, seqlen, G, kN) || !make_map(&mh, hin, 2, hdims, hstr, hbox)) {
+        !make_seq_map(&mc, C, batch, seqlen, G, kN)) {
         *why = "chunk scan: cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
     const int hpg = H / G;
     // The scan's per-head cost (mask, three MMA chains, epilogue) dominates its per-CTA ramp, and
     // its two tiles differ in cost, so many small CTAs balance better than one CTA per group.
-    const int hpc = std::min(hpg, 8);
+    const int hpc = std::min(hpg, kScanMaxHeads);
     const int nhb = (hpg + hpc - 1) / hpc;
     const size_t smem = sizeof(ScanSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(chunk_scan_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk scan: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb * (Q / kTileRows));
-    chunk_scan_tc_kernel<<<grid, kScanThreads, smem, st>>>(mx, mb, mc, mh, dtc, cs, D, y, status,
-                                                           seqlen, H, G, Q, nchunks, nhb, hpc);
+    chunk_scan_tc_kernel<<<grid, kScanThreads, smem, st>>>(mx, mb, mc, mx2, hin, dtc, cs, D, y,
+                                                           status, seqlen, H, G, Q, nchunks, nhb,
+                                                           hpc);
     *why = "chunk scan (tcgen05) launch";
     return cudaGetLastError();
 }

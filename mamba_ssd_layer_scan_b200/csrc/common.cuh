@@ -24,7 +24,8 @@ struct WsLayout {
     size_t cs;          // float [b][c][H][Q]: chunk-local inclusive cumsum of dt*A
     size_t dtc;         // float [b][c][H][Q]: dt per chunk row, 0 past the end (tensor-core path)
     size_t states;      // float [b][c][H][P][N]: per-chunk state, then (in place) state entering
-    size_t hin_bf16;    // bf16  [b][c][H][P][N]: state entering each chunk (tensor-core path)
+    size_t hin_bf16;    // bf16  [b][c][H] blocks of P x N (hin_swizzled_offset): state entering
+                        // each chunk (tensor-core path)
     size_t total;
 };
 
@@ -69,6 +70,17 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
                                   cudaStream_t st, const char **why);
+// Offset (in elements), inside one (batch, chunk, head) block of the bf16 entering states, of
+// state element (p, n) for P = 64, N = 128.  The block is stored exactly as the tensor cores
+// read it from shared memory: two halves of 64 n, each 64 rows p of 128 bytes, with the 16-byte
+// pieces of row p permuted by p mod 8 (the 128-byte swizzle), so that one contiguous 16 KB copy
+// brings a block into shared memory ready for use.
+__host__ __device__ __forceinline__ int hin_swizzled_offset(int p, int n)
+{
+    const int a = n >> 6, nl = n & 63;
+    return a * 4096 + p * 64 + ((((nl >> 3) ^ (p & 7)) << 3) | (nl & 7));
+}
+
 // Chunk state and state passing in one kernel (chunks walked in order per block of heads):
 // writes the bf16 entering states and the float32 final state; no float32 chunk states.
 bool fused_state_pass_ok(int64_t batch, int H, int G);

@@ -52,12 +52,16 @@ state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
             if (k < nchunks) {
                 const int64_t off = ((b * nchunks + k) * H + h) * PN + v * 4;
                 if (kBf16Out) {
+                    // tensor-core path (P = 64, N = 128): the swizzled block layout
+                    const int e = (int)(v * 4);
+                    const int64_t hoff =
+                        ((b * nchunks + k) * H + h) * PN + hin_swizzled_offset(e >> 7, e & 127);
                     __nv_bfloat162 lo = __floats2bfloat162_rn(hs.x, hs.y);
                     __nv_bfloat162 hi = __floats2bfloat162_rn(hs.z, hs.w);
                     uint2 packed;
                     packed.x = *reinterpret_cast<uint32_t *>(&lo);
                     packed.y = *reinterpret_cast<uint32_t *>(&hi);
-                    __stcs(reinterpret_cast<uint2 *>(hin + off), packed);
+                    __stcs(reinterpret_cast<uint2 *>(hin + hoff), packed);
                 } else {
                     __stcs(reinterpret_cast<float4 *>(states + off), hs);
                 }
