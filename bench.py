@@ -399,6 +399,45 @@ def main():
     torch.cuda.synchronize()
     dec_ms = d0.elapsed_time(d1) / Kd
 
+    # ---- packed variable-length sequences: the 2.7B layer's tokens as 12 uneven sequences
+    wv = configs.SSD_VARLEN
+    vin = inputs.make_inputs(wv)
+    vt = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in
+          dict(x=vin.x, dt=vin.dt, A=vin.A, B=vin.B, C=vin.C, D=vin.D, init=vin.init).items()}
+    for k in ("x", "B", "C"):
+        vt[k] = vt[k].to(xdt)
+    vcu = torch.from_numpy(vin.cu_seqlens).to(dev)
+    vshape = ssd.make_shape(1, wv.seqlen, wv.nheads, wv.headdim, wv.dstate, wv.ngroups,
+                            ssd.SSD_BF16)
+    vws = torch.empty(ssd.varlen_workspace_size(vshape, wv.nseq, wv.chunk), dtype=torch.uint8,
+                      device=dev)
+    vy = torch.empty_like(vt["x"])
+    vfin = torch.empty((wv.nseq, wv.nheads, wv.headdim, wv.dstate), dtype=torch.float32,
+                       device=dev)
+
+    def vfwd():
+        ssd.chunk_scan_varlen_fwd(vt["x"], vt["dt"], vt["A"], vt["B"], vt["C"], vt["D"], vcu,
+                                  wv.chunk, init_states=vt["init"], y=vy, final_states=vfin,
+                                  workspace=vws)
+
+    for _ in range(3):
+        flush.fill_(1.0)
+        vfwd()
+    torch.cuda.synchronize()
+    Kv = max(10, min(K, 50))
+    v_ms = []
+    for _ in range(Kv):
+        flush.fill_(1.0)
+        v0 = torch.cuda.Event(enable_timing=True)
+        v1 = torch.cuda.Event(enable_timing=True)
+        v0.record(stream)
+        vfwd()
+        v1.record(stream)
+        torch.cuda.synchronize()
+        v_ms.append(v0.elapsed_time(v1))
+    assert ssd.workspace_status(vws) == ssd.SSD_OK, "varlen scan status"
+    varlen_ms = statistics.mean(v_ms)
+
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
@@ -462,6 +501,12 @@ def main():
                         "gbs_compulsory": total["bytes"] / (ms_per_step / 1e3) / 1e9,
                         "tflops_dense": total["flops"] / (ms_per_step / 1e3) / 1e12},
         "kernels": kernels,
+        "varlen": {"workload": wv.name, "metric": "ssd_chunk_scan_varlen_fwd_tokens_per_s",
+                   "value": wv.seqlen / (varlen_ms / 1e3), "unit": "tokens/s",
+                   "ms_per_step": varlen_ms, "steps": Kv,
+                   "sequence_lengths": np.diff(vin.cu_seqlens).tolist(),
+                   "kernels_per_step": 5,
+                   "l2": "256 MB buffer written before each timed call (outside the events)"},
         "decode": {"workload": wd.name, "metric": "ssd_state_update_GBps", "value":
                    dbytes / (dec_ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": dec_ms,
                    "frac_hbm": dbytes / (dec_ms / 1e3) / 1e9 / hbm, "bytes_per_step": dbytes,

@@ -122,6 +122,37 @@ ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, cons
                                      void *const *stage_events);
 
 /*
+ * Variable-length packed sequences: nseq sequences stored back to back along the token axis of
+ * a batch-1 tensor, each with its own state.  Sequence s covers tokens
+ * [cu_seqlens[s], cu_seqlens[s + 1]); its recurrence starts from init_states[s] (or zeros) at
+ * its first token and ends in final_states[s]; no state crosses a boundary, so the result for
+ * every sequence equals ssd_chunk_scan_fwd on that sequence alone (the state is carried between
+ * blocks of one sequence only: mohakchugh.is-a.dev "Mamba-2", Block Decomposition; packed
+ * sequences need no padding).  Sequences of any length, including 0, are allowed; a chunk never
+ * spans two sequences (each sequence's last chunk may be partial).
+ *
+ *   shape          batch must be 1; seqlen = total tokens = cu_seqlens[nseq].
+ *   x, y, dt, B, C (1, seqlen, ...) as for ssd_chunk_scan_fwd.
+ *   cu_seqlens     device int32[nseq + 1], cu_seqlens[0] = 0, non-decreasing, last = seqlen.
+ *                  Checked on the device: if inconsistent nothing is computed and
+ *                  ssd_workspace_status() returns SSD_ERR_INVALID_ARG.
+ *   init_states    nullable, float32 (nseq, nheads, headdim, dstate).
+ *   final_states   nullable, float32 (nseq, nheads, headdim, dstate).
+ *   workspace      ssd_chunk_scan_varlen_workspace_size() bytes, 256-byte aligned.
+ *
+ * Runs on the tensor-core path only (bf16, headdim 64, dstate 128, chunk_size 128 or 256);
+ * other shapes return SSD_ERR_UNSUPPORTED.  Returns 0 from the size query when the arguments
+ * are invalid.
+ */
+size_t ssd_chunk_scan_varlen_workspace_size(const ssd_shape *shape, int nseq, int chunk_size);
+ssd_status ssd_chunk_scan_varlen_fwd(const ssd_shape *shape, const void *x, const float *dt,
+                                     const float *A, const void *B, const void *C,
+                                     const float *D, int chunk_size, const int32_t *cu_seqlens,
+                                     int nseq, const float *init_states, void *y,
+                                     float *final_states, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
+/*
  * One recurrent (decode) step for one new token per sequence, O(1) in the length of the past
  * (crackai.dev "Transformers are SSMs", Why It Matters; mohakchugh.is-a.dev "Mamba-2", Why
  * This Matters for Hardware, linear mode):
@@ -137,10 +168,12 @@ ssd_status ssd_state_update(const ssd_shape *shape, float *state, const void *x,
                             const float *D, void *y, void *stream);
 
 /*
- * Synchronises `stream` and reads the device status word the last ssd_chunk_scan_fwd call on
- * this workspace left behind: SSD_OK, or SSD_ERR_TIMEOUT when an in-kernel wait on a
- * shared-memory barrier exceeded its bound and the kernel returned early (its outputs are
- * then incomplete).  Returns SSD_ERR_CUDA if the synchronisation itself reports an error.
+ * Synchronises `stream` and reads the device status word the last ssd_chunk_scan_fwd (or
+ * ssd_chunk_scan_varlen_fwd) call on this workspace left behind: SSD_OK; SSD_ERR_TIMEOUT when
+ * an in-kernel wait on a shared-memory barrier exceeded its bound and the kernel returned early
+ * (its outputs are then incomplete); SSD_ERR_INVALID_ARG when a variable-length call's
+ * cu_seqlens was inconsistent (nothing was computed).  Returns SSD_ERR_CUDA if the
+ * synchronisation itself reports an error.
  */
 ssd_status ssd_workspace_status(const void *workspace, size_t workspace_bytes, void *stream);
 

@@ -29,6 +29,7 @@ class Workload:
     init_state: bool      # nonzero fp32 initial state ~ N(0, 0.1^2)
     seed: int
     decode: bool = False  # consumed one token per call by the decode update
+    nseq: int = 0         # > 0: batch 1 holds nseq packed sequences of uneven length
 
     @property
     def tokens(self) -> int:
@@ -54,5 +55,10 @@ SSD_LONG = Workload("ssd_fwd_bf16_b1_L65536_H32_P64_N128_G8_Q256_init", 1, 65536
 SSD_DECODE = Workload("ssd_decode_bf16_b128_H80_P64_N128_1000steps", 128, 1000, 80, 64, 128, 1,
                       256, "bf16", True, 1004, decode=True)
 
-ALL = (SSD_F32_SMALL, SSD_370M, SSD_2P7B, SSD_LONG, SSD_DECODE)
+# Packed variable-length sequences: the 2.7B layer's 16384 tokens as 12 sequences of uneven
+# length in one row, each with its own nonzero initial state and final state.
+SSD_VARLEN = Workload("ssd_varlen_bf16_T16384_seq12_H80_P64_N128_Q256_init", 1, 16384, 80, 64,
+                      128, 1, 256, "bf16", True, 1005, nseq=12)
+
+ALL = (SSD_F32_SMALL, SSD_370M, SSD_2P7B, SSD_LONG, SSD_DECODE, SSD_VARLEN)
 BY_NAME = {w.name: w for w in ALL}

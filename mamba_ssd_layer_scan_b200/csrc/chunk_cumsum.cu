@@ -24,7 +24,7 @@ constexpr int kMaxSeg = 8;       // Q <= 256 = 8 segments of 32 tokens
 __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(const float *__restrict__ dt, const float *__restrict__ A,
                     float *__restrict__ cs, float *__restrict__ dtc, int *__restrict__ status,
-                    int64_t seqlen, int H, int Q, int64_t nchunks)
+                    int64_t seqlen, int H, int Q, int64_t nchunks, const int2 *__restrict__ tab)
 {
     // First kernel of every scan: clears the workspace status word the later kernels may set.
     if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
@@ -34,8 +34,10 @@ chunk_cumsum_kernel(const float *__restrict__ dt, const float *__restrict__ A,
     const int64_t k = (blockIdx.x / nht) % nchunks;
     const int64_t b = blockIdx.x / nht / nchunks;
     const int nh = min(kHeadTile, H - h0);
-    const int64_t t0 = k * Q;
-    const int len = (int)min((int64_t)Q, seqlen - t0);
+    int64_t t0;
+    int len;
+    chunk_span(tab, k, Q, seqlen, t0, len);
+    if (len <= 0) return;   // unused slot of a chunk table
 
     for (int idx = threadIdx.x; idx < Q * kHeadTile; idx += kThreads) {
         const int tau = idx / kHeadTile, j = idx % kHeadTile;
@@ -90,12 +92,12 @@ __global__ void fill_final_kernel(const float *__restrict__ init, float *__restr
 
 cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, float *dtc,
                                 int *status, int64_t batch, int64_t seqlen, int nheads, int Q,
-                                int64_t nchunks, cudaStream_t st)
+                                int64_t nchunks, cudaStream_t st, const int2 *tab)
 {
     const unsigned grid = (unsigned)(((nheads + kHeadTile - 1) / kHeadTile) * nchunks * batch);
     const size_t smem = (size_t)Q * (kHeadTile + 1) * sizeof(float);
     chunk_cumsum_kernel<<<grid, kThreads, smem, st>>>(dt, A, cs, dtc, status, seqlen, nheads,
-                                                      Q, nchunks);
+                                                      Q, nchunks, tab);
     return cudaGetLastError();
 }
 

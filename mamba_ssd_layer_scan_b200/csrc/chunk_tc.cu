@@ -83,7 +83,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                       const __grid_constant__ CUtensorMap tm_b, const float *__restrict__ dtc,
                       const float *__restrict__ cs, float *__restrict__ states,
                       int *__restrict__ status, int H, int G, int Q, int64_t nchunks, int nhb,
-                      int hpc)
+                      int hpc, int64_t seqlen, const int2 *__restrict__ tab)
 {
     extern __shared__ uint8_t smem_raw[];
     StateSmem &sm = *reinterpret_cast<StateSmem *>(
@@ -97,7 +97,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int hpg = H / G;
     const int h0 = g * hpg + hb * hpc;
     const int nh = min(hpc, hpg - hb * hpc);
-    const int64_t t0 = k * Q;
+    int64_t t0;
+    int len;
+    chunk_span(tab, k, Q, seqlen, t0, len);
+    if (len <= 0) return;   // unused slot of a chunk table (before any barrier or TMEM use)
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_b, 1);
@@ -593,7 +596,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const float *__restrict__ dtc,
                      const float *__restrict__ cs, const float *__restrict__ D,
                      bf16 *__restrict__ y, int *__restrict__ status, int64_t seqlen, int H,
-                     int G, int Q, int64_t nchunks, int nhb, int hpc)
+                     int G, int Q, int64_t nchunks, int nhb, int hpc, const int2 *__restrict__ tab)
 {
     extern __shared__ uint8_t smem_raw[];
     ScanSmem &sm = *reinterpret_cast<ScanSmem *>(
@@ -609,9 +612,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int hpg = H / G;
     const int h0 = g * hpg + hb * hpc;
     const int nh = min(hpc, hpg - hb * hpc);
-    const int64_t t0 = k * Q;
-    const int len = (int)min((int64_t)Q, seqlen - t0);
-    if (T * kTileRows >= len) return;  // tile entirely past the end of the sequence
+    int64_t t0;
+    int len;
+    chunk_span(tab, k, Q, seqlen, t0, len);
+    if (T * kTileRows >= len) return;  // tile past the end of the sequence, or unused slot
     const int KI = kTileRows * (T + 1);  // causal source columns of this tile
     const int nst = T ? 2 : 3;           // x / h_in stages
     const uint32_t gdiag = T ? 128u : 0u;  // TMEM column of the diagonal block of C B^T
@@ -1029,7 +1033,7 @@ bool tc_supported(bool is_bf16, int P, int N, int Q)
 cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
-                                  cudaStream_t st, const char **why)
+                                  cudaStream_t st, const char **why, const int2 *tab)
 {
     CUtensorMap mx, mb;   // boxes of a whole chunk (Q rows)
     if (!make_seq_map(&mx, x, batch, seqlen, H, kP, Q) ||
@@ -1046,7 +1050,8 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
     if (e != cudaSuccess) { *why = "chunk state: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb);
     chunk_state_tc_kernel<<<grid, kStateThreads, smem, st>>>(mx, mb, dtc, cs, states, status,
-                                                             H, G, Q, nchunks, nhb, hpc);
+                                                             H, G, Q, nchunks, nhb, hpc, seqlen,
+                                                             tab);
     *why = "chunk state (tcgen05) launch";
     return cudaGetLastError();
 }
@@ -1084,7 +1089,8 @@ cudaError_t launch_chunk_state_pass_tc(const bf16 *x, const float *dtc, const bf
 cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
-                                 int Q, int64_t nchunks, cudaStream_t st, const char **why)
+                                 int Q, int64_t nchunks, cudaStream_t st, const char **why,
+                                 const int2 *tab)
 {
     CUtensorMap mx, mx2, mb, mc;
     if (!make_seq_map(&mx, x, batch, seqlen, H, kP) ||
@@ -1106,7 +1112,7 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb * (Q / kTileRows));
     chunk_scan_tc_kernel<<<grid, kScanThreads, smem, st>>>(mx, mb, mc, mx2, hin, dtc, cs, D, y,
                                                            status, seqlen, H, G, Q, nchunks, nhb,
-                                                           hpc);
+                                                           hpc, tab);
     *why = "chunk scan (tcgen05) launch";
     return cudaGetLastError();
 }

@@ -29,6 +29,28 @@ struct WsLayout {
     size_t total;
 };
 
+// Where chunk k of the workspace sits in the token sequence.  Without a table (fixed-length
+// input) chunk k of batch row b starts at token k Q of that row and holds min(Q, L - k Q)
+// tokens.  With a table (packed variable-length input, batch 1) entry k holds the chunk's first
+// token and its length, 0 for an unused slot; a chunk never spans two sequences, so every
+// kernel treats a table chunk like the partial last chunk of a fixed-length sequence.
+__device__ __forceinline__ void chunk_span(const int2 *tab, int64_t k, int Q, int64_t seqlen,
+                                           int64_t &t0, int &len)
+{
+    if (tab) {
+        const int2 e = tab[k];
+        t0 = e.x;
+        len = e.y;
+    } else {
+        t0 = k * Q;
+        len = (int)(seqlen - t0 < Q ? seqlen - t0 : Q);
+    }
+}
+
+// Workspace status word bits: 1, 2, 4 = a bounded wait timed out (chunk scan, chunk state, fused
+// state); kStatusBadSeqlens = the cu_seqlens of a variable-length call are inconsistent.
+constexpr int kStatusBadSeqlens = 0x10000;
+
 // Sets the calling thread's message returned by ssd_last_error().
 void set_last_error(const char *msg);
 
@@ -37,7 +59,14 @@ void set_last_error(const char *msg);
 // non-null, writes dt re-laid out as (b, c, H, Q) with zeros past the end of the sequence.
 cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, float *dtc,
                                 int *status, int64_t batch, int64_t seqlen, int nheads, int Q,
-                                int64_t nchunks, cudaStream_t st);
+                                int64_t nchunks, cudaStream_t st, const int2 *tab = nullptr);
+
+// Packed variable-length input: the chunk table (tab, nchunks entries) and the first chunk of
+// every sequence (cstart, nseq + 1 entries) from cu_seqlens; clears *status and sets
+// kStatusBadSeqlens (and an empty table) when cu_seqlens is inconsistent.
+cudaError_t launch_build_chunk_table(const int32_t *cu_seqlens, int nseq, int64_t seqlen, int Q,
+                                     int64_t nchunks, int2 *tab, int32_t *cstart, int *status,
+                                     cudaStream_t st);
 
 cudaError_t launch_chunk_state_simt(bool is_bf16, const void *x, const float *dt,
                                     const void *B, const float *cs, float *states,
@@ -49,6 +78,12 @@ cudaError_t launch_chunk_state_simt(bool is_bf16, const void *x, const float *dt
 cudaError_t launch_state_passing(float *states, const float *cs, const float *init,
                                  float *final_state, bf16 *hin_bf16, int64_t batch, int H,
                                  int P, int N, int Q, int64_t nchunks, cudaStream_t st);
+// The same per packed sequence: sequence s owns chunks [cstart[s], cstart[s + 1]) and its own
+// initial and final state (init / final_state indexed [s][h][p][n]).
+cudaError_t launch_state_passing_varlen(float *states, const float *cs, const float *init,
+                                        float *final_state, bf16 *hin_bf16,
+                                        const int32_t *cstart, int nseq, int H, int P, int N,
+                                        int Q, int64_t nchunks, cudaStream_t st);
 
 cudaError_t launch_chunk_scan_simt(bool is_bf16, const void *x, const float *dt,
                                    const void *B, const void *C, const float *cs,
@@ -69,7 +104,7 @@ bool tc_supported(bool is_bf16, int P, int N, int Q);
 cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
-                                  cudaStream_t st, const char **why);
+                                  cudaStream_t st, const char **why, const int2 *tab = nullptr);
 // Offset (in elements), inside one (batch, chunk, head) block of the bf16 entering states, of
 // state element (p, n) for P = 64, N = 128.  The block is stored exactly as the tensor cores
 // read it from shared memory: two halves of 64 n, each 64 rows p of 128 bytes, with the 16-byte
@@ -92,6 +127,7 @@ cudaError_t launch_chunk_state_pass_tc(const bf16 *x, const float *dtc, const bf
 cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
-                                 int Q, int64_t nchunks, cudaStream_t st, const char **why);
+                                 int Q, int64_t nchunks, cudaStream_t st, const char **why,
+                                 const int2 *tab = nullptr);
 
 }  // namespace ssd

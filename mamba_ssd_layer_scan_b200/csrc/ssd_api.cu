@@ -97,6 +97,50 @@ ssd::WsLayout layout(const ssd_shape *s, int Q)
     return w;
 }
 
+// Workspace of a variable-length call: the status word, the chunk table (one slot per possible
+// chunk: L / Q + nseq bounds the chunks of any split of L tokens into nseq sequences), the
+// first chunk of each sequence, then the tensor-core path's per-chunk regions.
+struct VarlenLayout {
+    size_t status, tab, cstart, cs, dtc, states, hin, total;
+    int64_t slots;
+};
+
+VarlenLayout varlen_layout(const ssd_shape *s, int nseq, int Q)
+{
+    VarlenLayout w;
+    w.slots = s->seqlen / Q + nseq;
+    const size_t rows = (size_t)w.slots * s->nheads;
+    const size_t pn = (size_t)s->headdim * s->dstate;
+    w.status = 0;
+    w.tab = 256;
+    w.cstart = w.tab + round256((size_t)w.slots * 8);
+    w.cs = w.cstart + round256((size_t)(nseq + 1) * 4);
+    w.dtc = w.cs + round256(rows * Q * 4);
+    w.states = w.dtc + round256(rows * Q * 4);
+    w.hin = w.states + round256(rows * pn * 4);
+    w.total = w.hin + round256(rows * pn * 2);
+    return w;
+}
+
+ssd_status check_varlen(const ssd_shape *s, int nseq, int Q)
+{
+    ssd_status st = check_shape(s, true);
+    if (st != SSD_OK) return st;
+    if (s->batch != 1)
+        return fail(SSD_ERR_INVALID_ARG, "variable-length input is packed: batch must be 1 (got %lld)",
+                    (long long)s->batch);
+    if (nseq < 1) return fail(SSD_ERR_INVALID_ARG, "nseq must be >= 1 (got %d)", nseq);
+    if (s->seqlen > 0x7fffffffLL - 256)
+        return fail(SSD_ERR_UNSUPPORTED, "packed token count must fit int32 cu_seqlens");
+    if (!valid_chunk(Q))
+        return fail(SSD_ERR_UNSUPPORTED, "chunk_size must be 16, 32, 64, 128 or 256 (got %d)", Q);
+    if (!ssd::tc_supported(s->dtype == SSD_BF16, (int)s->headdim, (int)s->dstate, Q))
+        return fail(SSD_ERR_UNSUPPORTED,
+                    "variable-length scan runs on the tensor-core path only: bf16, headdim 64, "
+                    "dstate 128, chunk_size 128 or 256");
+    return SSD_OK;
+}
+
 }  // namespace
 
 void ssd::set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
@@ -240,6 +284,78 @@ ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, cons
     return SSD_OK;
 }
 
+size_t ssd_chunk_scan_varlen_workspace_size(const ssd_shape *shape, int nseq, int chunk_size)
+{
+    if (check_varlen(shape, nseq, chunk_size) != SSD_OK) return 0;
+    return varlen_layout(shape, nseq, chunk_size).total;
+}
+
+ssd_status ssd_chunk_scan_varlen_fwd(const ssd_shape *shape, const void *x, const float *dt,
+                                     const float *A, const void *B, const void *C,
+                                     const float *D, int chunk_size, const int32_t *cu_seqlens,
+                                     int nseq, const float *init_states, void *y,
+                                     float *final_states, void *workspace,
+                                     size_t workspace_bytes, void *stream)
+{
+    ssd_status st = check_varlen(shape, nseq, chunk_size);
+    if (st != SSD_OK) return st;
+    const ssd_shape s = *shape;
+    const int H = (int)s.nheads, G = (int)s.ngroups, P = (int)s.headdim, N = (int)s.dstate;
+    const int Q = chunk_size;
+    cudaStream_t cst = static_cast<cudaStream_t>(stream);
+    if (final_states && !aligned16(final_states))
+        return fail(SSD_ERR_INVALID_ARG, "final_states must be 16-byte aligned");
+    if (init_states && !aligned16(init_states))
+        return fail(SSD_ERR_INVALID_ARG, "init_states must be 16-byte aligned");
+    if (s.seqlen == 0) {   // every sequence is empty: final = init
+        if (final_states) {
+            cudaError_t e = ssd::launch_fill_final(init_states, final_states,
+                                                   (int64_t)nseq * H * P * N, cst);
+            if (e != cudaSuccess) return cuda_fail(e, "fill final states");
+        }
+        return SSD_OK;
+    }
+    if (!x || !dt || !A || !B || !C || !D || !y || !cu_seqlens || !workspace)
+        return fail(SSD_ERR_INVALID_ARG,
+                    "x, dt, A, B, C, D, y, cu_seqlens and workspace must be non-NULL");
+    if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(y))
+        return fail(SSD_ERR_INVALID_ARG, "x, B, C and y must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(SSD_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const VarlenLayout wl = varlen_layout(&s, nseq, Q);
+    if (workspace_bytes < wl.total)
+        return fail(SSD_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu",
+                    wl.total, workspace_bytes);
+    if (wl.slots * H * ((Q + 31) / 32) > 0x7fffffffLL)
+        return fail(SSD_ERR_UNSUPPORTED, "problem too large for one launch grid");
+
+    char *ws = static_cast<char *>(workspace);
+    int *status = reinterpret_cast<int *>(ws + wl.status);
+    int2 *tab = reinterpret_cast<int2 *>(ws + wl.tab);
+    int32_t *cstart = reinterpret_cast<int32_t *>(ws + wl.cstart);
+    float *cs = reinterpret_cast<float *>(ws + wl.cs);
+    float *dtc = reinterpret_cast<float *>(ws + wl.dtc);
+    float *states = reinterpret_cast<float *>(ws + wl.states);
+    ssd::bf16 *hin = reinterpret_cast<ssd::bf16 *>(ws + wl.hin);
+    const char *why = "";
+    cudaError_t e = ssd::launch_build_chunk_table(cu_seqlens, nseq, s.seqlen, Q, wl.slots, tab,
+                                                  cstart, status, cst);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk table launch");
+    e = ssd::launch_chunk_cumsum(dt, A, cs, dtc, nullptr, 1, s.seqlen, H, Q, wl.slots, cst, tab);
+    if (e != cudaSuccess) return cuda_fail(e, "dA cumsum launch");
+    e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs, states,
+                                   status, 1, s.seqlen, H, G, Q, wl.slots, cst, &why, tab);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+    e = ssd::launch_state_passing_varlen(states, cs, init_states, final_states, hin, cstart,
+                                         nseq, H, P, N, Q, wl.slots, cst);
+    if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
+    e = ssd::launch_chunk_scan_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B,
+                                  (const ssd::bf16 *)C, cs, hin, D, (ssd::bf16 *)y, status, 1,
+                                  s.seqlen, H, G, Q, wl.slots, cst, &why, tab);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+    return SSD_OK;
+}
+
 ssd_status ssd_state_update(const ssd_shape *shape, float *state, const void *x,
                             const float *dt, const float *A, const void *B, const void *C,
                             const float *D, void *y, void *stream)
@@ -269,6 +385,9 @@ ssd_status ssd_workspace_status(const void *workspace, size_t workspace_bytes, v
                                     static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "read workspace status");
+    if (word & ssd::kStatusBadSeqlens)
+        return fail(SSD_ERR_INVALID_ARG,
+                    "cu_seqlens must start at 0, never decrease and end at the token count");
     if (word != 0)
         return fail(SSD_ERR_TIMEOUT, "an in-kernel barrier wait exceeded its bound (code %d)",
                     word);

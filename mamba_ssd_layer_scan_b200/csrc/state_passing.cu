@@ -24,24 +24,30 @@ template <bool kBf16Out>
 __global__ void __launch_bounds__(kThreads)
 state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
                      const float *__restrict__ init, float *__restrict__ final_state,
-                     bf16 *__restrict__ hin, int H, int PN, int Q, int64_t nchunks)
+                     bf16 *__restrict__ hin, int H, int PN, int Q, int64_t nchunks,
+                     const int32_t *__restrict__ cstart)
 {
     const int nblk = (PN / 4 + kThreads - 1) / kThreads;
     const int64_t v = (blockIdx.x % nblk) * (int64_t)kThreads + threadIdx.x;  // float4 index
+    // b: batch row, or the packed sequence when cstart is given (its chunks are
+    // [cstart[b], cstart[b + 1]) of the single workspace row)
     const int64_t h = (blockIdx.x / nblk) % H, b = blockIdx.x / nblk / H;
     if (v * 4 >= PN) return;
+    const int64_t kbeg = cstart ? cstart[b] : 0;
+    const int64_t kend = cstart ? cstart[b + 1] : nchunks;
+    const int64_t rb = cstart ? 0 : b;   // workspace batch row
 
     float4 hs = make_float4(0.f, 0.f, 0.f, 0.f);
     if (init) hs = *reinterpret_cast<const float4 *>(init + (b * H + h) * PN + v * 4);
 
-    for (int64_t k0 = 0; k0 < nchunks; k0 += kGroup) {
+    for (int64_t k0 = kbeg; k0 < kend; k0 += kGroup) {
         float4 s[kGroup];
         float decay[kGroup];
 #pragma unroll
         for (int j = 0; j < kGroup; ++j) {
             const int64_t k = k0 + j;
-            if (k < nchunks) {
-                const int64_t row = (b * nchunks + k) * H + h;
+            if (k < kend) {
+                const int64_t row = (rb * nchunks + k) * H + h;
                 s[j] = __ldcs(reinterpret_cast<const float4 *>(states + row * PN + v * 4));
                 decay[j] = cs[row * Q + Q - 1];
             }
@@ -49,13 +55,13 @@ state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
 #pragma unroll
         for (int j = 0; j < kGroup; ++j) {
             const int64_t k = k0 + j;
-            if (k < nchunks) {
-                const int64_t off = ((b * nchunks + k) * H + h) * PN + v * 4;
+            if (k < kend) {
+                const int64_t off = ((rb * nchunks + k) * H + h) * PN + v * 4;
                 if (kBf16Out) {
                     // tensor-core path (P = 64, N = 128): the swizzled block layout
                     const int e = (int)(v * 4);
                     const int64_t hoff =
-                        ((b * nchunks + k) * H + h) * PN + hin_swizzled_offset(e >> 7, e & 127);
+                        ((rb * nchunks + k) * H + h) * PN + hin_swizzled_offset(e >> 7, e & 127);
                     __nv_bfloat162 lo = __floats2bfloat162_rn(hs.x, hs.y);
                     __nv_bfloat162 hi = __floats2bfloat162_rn(hs.z, hs.w);
                     uint2 packed;
@@ -87,10 +93,30 @@ cudaError_t launch_state_passing(float *states, const float *cs, const float *in
     const unsigned grid = (unsigned)(((PN / 4 + kThreads - 1) / kThreads) * H * batch);
     if (hin_bf16)
         state_passing_kernel<true><<<grid, kThreads, 0, st>>>(states, cs, init, final_state,
-                                                              hin_bf16, H, PN, Q, nchunks);
+                                                              hin_bf16, H, PN, Q, nchunks,
+                                                              nullptr);
     else
         state_passing_kernel<false><<<grid, kThreads, 0, st>>>(states, cs, init, final_state,
-                                                               nullptr, H, PN, Q, nchunks);
+                                                               nullptr, H, PN, Q, nchunks,
+                                                               nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_state_passing_varlen(float *states, const float *cs, const float *init,
+                                        float *final_state, bf16 *hin_bf16,
+                                        const int32_t *cstart, int nseq, int H, int P, int N,
+                                        int Q, int64_t nchunks, cudaStream_t st)
+{
+    const int PN = P * N;
+    const unsigned grid = (unsigned)(((PN / 4 + kThreads - 1) / kThreads) * H * (int64_t)nseq);
+    if (hin_bf16)
+        state_passing_kernel<true><<<grid, kThreads, 0, st>>>(states, cs, init, final_state,
+                                                              hin_bf16, H, PN, Q, nchunks,
+                                                              cstart);
+    else
+        state_passing_kernel<false><<<grid, kThreads, 0, st>>>(states, cs, init, final_state,
+                                                               nullptr, H, PN, Q, nchunks,
+                                                               cstart);
     return cudaGetLastError();
 }
 

@@ -11,6 +11,9 @@ workload's seed:
     B, C ~ N(0, 1) / sqrt(N)                      (b, L, G, N)
     D  ~ N(0, 1)                                  (H,)
     h0 ~ N(0, 0.1^2)                              (b, H, P, N)   only when the workload has one
+                                                  ((nseq, H, P, N) for packed sequences)
+    cu_seqlens: nseq - 1 distinct cut points drawn uniformly from 1 .. L-1, sorted, with 0 and
+                L added (packed variable-length workloads only; drawn last)
 
 Values are drawn in float32; x, B and C are then rounded to bfloat16 (round to nearest even) for
 bf16 workloads, and every consumer reads the rounded values, so the oracle sees exactly what the
@@ -55,6 +58,7 @@ class SSDInputs:
     C: np.ndarray
     D: np.ndarray
     init: Optional[np.ndarray]
+    cu_seqlens: Optional[np.ndarray] = None   # int32 (nseq + 1,) for packed sequences
 
 
 def make_inputs(w: Workload, seed: Optional[int] = None) -> SSDInputs:
@@ -69,10 +73,17 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> SSDInputs:
     C = rng.standard_normal((b, L, G, N), dtype=np.float32) * inv
     D = rng.standard_normal(H, dtype=np.float32)
     init = None
+    ns = w.nseq if w.nseq > 0 else b
     if w.init_state:
-        init = rng.standard_normal((b, H, P, N), dtype=np.float32) * np.float32(0.1)
+        init = rng.standard_normal((ns, H, P, N), dtype=np.float32) * np.float32(0.1)
+    cu = None
+    if w.nseq > 0:
+        if b != 1 or w.nseq > L:
+            raise ValueError("packed sequences need batch 1 and at most one sequence per token")
+        cuts = np.sort(rng.choice(np.arange(1, L), size=w.nseq - 1, replace=False))
+        cu = np.concatenate([[0], cuts, [L]]).astype(np.int32)
     if w.dtype == "bf16":
         x, B, C = round_bf16(x), round_bf16(B), round_bf16(C)
     elif w.dtype != "f32":
         raise ValueError(f"unknown dtype {w.dtype!r}")
-    return SSDInputs(w, x, dt, A, B, C, D, init)
+    return SSDInputs(w, x, dt, A, B, C, D, init, cu)

@@ -5,6 +5,7 @@ streams and dtypes.  There is no fallback: if the shared library is missing or w
 without the CUDA kernels, loading it raises.
 
     y, final = chunk_scan_fwd(x, dt, A, B, C, D, chunk_size=256, init_state=None)
+    y, finals = chunk_scan_varlen_fwd(x, dt, A, B, C, D, cu_seqlens)   # packed sequences
     y = state_update(state, x, dt, A, B, C, D)          # state updated in place
 """
 from __future__ import annotations
@@ -63,6 +64,13 @@ def lib():
     L.ssd_chunk_scan_fwd_staged.restype = ctypes.c_int
     L.ssd_chunk_scan_fwd_staged.argtypes = L.ssd_chunk_scan_fwd.argtypes + [
         ctypes.POINTER(ctypes.c_void_p)]
+    L.ssd_chunk_scan_varlen_workspace_size.restype = ctypes.c_size_t
+    L.ssd_chunk_scan_varlen_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int,
+                                                       ctypes.c_int]
+    L.ssd_chunk_scan_varlen_fwd.restype = ctypes.c_int
+    L.ssd_chunk_scan_varlen_fwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
+                                            ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp, _vp,
+                                            ctypes.c_size_t, _vp]
     L.ssd_state_update.restype = ctypes.c_int
     L.ssd_state_update.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _vp]
@@ -171,6 +179,48 @@ def chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int = 256, init_state=None,
         handles = (ctypes.c_void_p * 5)(*[ev.cuda_event for ev in stage_events])
         _check(lib().ssd_chunk_scan_fwd_staged(*args, handles))
     return y, final_state
+
+
+def varlen_workspace_size(shape: Shape, nseq: int, chunk_size: int) -> int:
+    n = lib().ssd_chunk_scan_varlen_workspace_size(ctypes.byref(shape), nseq, chunk_size)
+    if n == 0:
+        raise SSDError(SSD_ERR_INVALID_ARG, last_error())
+    return n
+
+
+def chunk_scan_varlen_fwd(x, dt, A, B, C, D, cu_seqlens, chunk_size: int = 256,
+                          init_states=None, return_final_states: bool = True, y=None,
+                          final_states=None, workspace=None, stream=None):
+    """Packed variable-length scan.  x (1, T, H, P), dt (1, T, H) f32, B/C (1, T, G, N),
+    cu_seqlens (nseq + 1,) int32 on the device, init_states (nseq, H, P, N) f32 or None.
+    Returns (y, final_states or None); sequence s is tokens cu_seqlens[s] .. cu_seqlens[s+1]-1
+    and carries its own state."""
+    torch = _torch()
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = x.device
+    code = _dtype_code(x)
+    for t, n in ((x, "x"), (B, "B"), (C, "C")):
+        _require(t, n, x.dtype, dev)
+    for t, n in ((dt, "dt"), (A, "A"), (D, "D")):
+        _require(t, n, torch.float32, dev)
+    _require(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    nseq = cu_seqlens.numel() - 1
+    if init_states is not None:
+        _require(init_states, "init_states", torch.float32, dev)
+    shape = make_shape(b, L, H, P, N, G, code)
+    if y is None:
+        y = torch.empty_like(x)
+    if final_states is None and return_final_states:
+        final_states = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(varlen_workspace_size(shape, nseq, chunk_size),
+                                dtype=torch.uint8, device=dev)
+    _check(lib().ssd_chunk_scan_varlen_fwd(
+        ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), chunk_size,
+        _ptr(cu_seqlens), nseq, _ptr(init_states), _ptr(y), _ptr(final_states), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream)))
+    return y, final_states
 
 
 def state_update(state, x, dt, A, B, C, D, y=None, stream=None):

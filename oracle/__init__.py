@@ -121,6 +121,32 @@ def ssd_scan_pairs(inp, pairs: Sequence[Tuple[int, int]], every: int = 0,
     return y, final[0], (None if boundary is None else boundary[0])
 
 
+def ssd_scan_varlen(x, dt, A, B, C, D, cu_seqlens, init=None):
+    """Packed variable-length sequences: sequence s (tokens cu_seqlens[s] .. cu_seqlens[s+1]-1
+    of the single batch row) is its own recurrence, started from init[s] (or zeros), so this is
+    the token-by-token oracle applied to each sequence separately.
+
+    x (1, T, H, P) etc., cu_seqlens (nseq + 1,), init (nseq, H, P, N) or None.
+    Returns (y (1, T, H, P), final (nseq, H, P, N)).
+    """
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    nseq = len(cu) - 1
+    _, T, H, P = x.shape
+    N = B.shape[3]
+    y = np.zeros((1, T, H, P))
+    final = np.zeros((nseq, H, P, N))
+    for s in range(nseq):
+        a, e = int(cu[s]), int(cu[s + 1])
+        h0 = None if init is None else init[s:s + 1]
+        if e == a:
+            final[s] = 0.0 if h0 is None else h0[0]
+            continue
+        ys, fs, _ = ssd_scan(x[:, a:e], dt[:, a:e], A, B[:, a:e], C[:, a:e], D, h0)
+        y[:, a:e] = ys
+        final[s] = fs[0]
+    return y, final
+
+
 def ssd_state_update(state, x, dt, A, B, C, D):
     """One decode step: the recurrence over a single token, state (b, H, P, N) updated and returned.
 

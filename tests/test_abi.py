@@ -17,6 +17,7 @@ def L():
 def test_exports_every_declared_function(L):
     declared = ssd.declared_functions()
     assert {"ssd_chunk_scan_fwd", "ssd_state_update", "ssd_chunk_scan_workspace_size",
+            "ssd_chunk_scan_varlen_fwd", "ssd_chunk_scan_varlen_workspace_size",
             "ssd_last_error"} <= set(declared)
     out = subprocess.run(["nm", "-D", "--defined-only", ssd.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -122,3 +123,29 @@ def test_product_path_has_no_cpu_fallback(tmp_path, monkeypatch):
     monkeypatch.setattr(ssd, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         ssd.lib()
+
+
+def test_varlen_workspace_size_layout():
+    T, H, P, N, Q, nseq = 16384, 80, 64, 128, 256, 12
+    slots = T // Q + nseq                  # chunks of any split of T tokens into nseq sequences
+    r = lambda v: (v + 255) // 256 * 256
+    rows = slots * H
+    expect = (256 + r(slots * 8) + r((nseq + 1) * 4) + 2 * r(rows * Q * 4) + r(rows * P * N * 4)
+              + r(rows * P * N * 2))
+    assert ssd.varlen_workspace_size(_shape(batch=1, seqlen=T), nseq, Q) == expect
+
+
+@pytest.mark.parametrize("kw,nseq,chunk,code", [
+    (dict(batch=2), 3, 256, ssd.SSD_ERR_INVALID_ARG),         # packed input is one row
+    (dict(batch=1), 0, 256, ssd.SSD_ERR_INVALID_ARG),         # no sequence
+    (dict(batch=1, dtype=ssd.SSD_F32), 3, 256, ssd.SSD_ERR_UNSUPPORTED),
+    (dict(batch=1), 3, 64, ssd.SSD_ERR_UNSUPPORTED),          # tensor-core chunk sizes only
+])
+def test_varlen_rejects_bad_arguments(L, kw, nseq, chunk, code):
+    sh = _shape(**kw)
+    assert L.ssd_chunk_scan_varlen_workspace_size(ctypes.byref(sh), nseq, chunk) == 0
+    p = ctypes.c_void_p(1 << 20)
+    rc = L.ssd_chunk_scan_varlen_fwd(ctypes.byref(sh), p, p, p, p, p, p, chunk, p, nseq, None, p,
+                                     None, p, 1 << 40, None)
+    assert rc == code
+    assert ssd.last_error()

@@ -257,3 +257,86 @@ def test_input_recipe_ranges():
     assert np.all(inp.A < 0) and np.all(inp.A >= -16.0) and np.all(inp.A <= -1.0)
     np.testing.assert_array_equal(inputs.round_bf16(inp.x), inp.x)
     assert abs(inp.B.std() * np.sqrt(128) - 1.0) < 0.05
+
+
+# ------------------------------------------------------------------ packed variable-length input
+def _packed_matrix_form(x, dt, A, B, C, D, cu, h0):
+    """Brute force for packed sequences from the matrix form: one T x T mixing matrix per head
+    that is block diagonal over the sequences (M[t, i] = 0 when t and i lie in different
+    sequences), each block the semiseparable matrix of _matrix_form, and each sequence's initial
+    state decayed from its own first token."""
+    _, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    nseq = len(cu) - 1
+    seq = np.zeros(T, dtype=int)
+    for s in range(nseq):
+        seq[cu[s]:cu[s + 1]] = s
+    y = np.zeros_like(x)
+    final = np.zeros((nseq, H, P, N))
+    for h in range(H):
+        g = h // (H // G)
+        a = np.exp(dt[0, :, h] * A[h])
+        M = np.zeros((T, T))
+        for t in range(T):
+            for i in range(t + 1):
+                if seq[i] == seq[t]:
+                    M[t, i] = C[0, t, g] @ B[0, i, g] * dt[0, i, h] * np.prod(a[i + 1:t + 1])
+        y[0, :, h] = M @ x[0, :, h] + D[h] * x[0, :, h]
+        for s in range(nseq):
+            lo, hi = cu[s], cu[s + 1]
+            for i in range(lo, hi):
+                final[s, h] += np.prod(a[i + 1:hi]) * dt[0, i, h] * np.outer(x[0, i, h], B[0, i, g])
+            if h0 is not None:
+                for t in range(lo, hi):
+                    y[0, t, h] += np.prod(a[lo:t + 1]) * (h0[s, h] @ C[0, t, g])
+                final[s, h] += np.prod(a[lo:hi]) * h0[s, h]
+    return y, final
+
+
+def _packed_case(seed, T=37, H=4, G=2, P=3, N=5):
+    x, dt, A, B, C, D, _ = _rand_case(seed, b=1, L=T, H=H, G=G, P=P, N=N, init=False)
+    cu = np.array([0, 6, 6, 7, 22, T], dtype=np.int32)   # an empty and a one-token sequence
+    rng = np.random.default_rng(seed + 7)
+    h0 = 0.3 * rng.standard_normal((len(cu) - 1, H, P, N))
+    return x, dt, A, B, C, D, cu, h0
+
+
+@pytest.mark.parametrize("seed", [3, 4])
+def test_packed_sequences_equal_block_diagonal_matrix(seed):
+    x, dt, A, B, C, D, cu, h0 = _packed_case(seed)
+    y, final = oracle.ssd_scan_varlen(x, dt, A, B, C, D, cu, h0)
+    y_ref, f_ref = _packed_matrix_form(x, dt, A, B, C, D, cu, h0)
+    assert _rel(y, y_ref) < 1e-12
+    assert _rel(final, f_ref) < 1e-12
+    assert np.array_equal(final[1], h0[1])   # the empty sequence hands its initial state back
+
+
+def test_packed_single_sequence_is_the_plain_scan():
+    x, dt, A, B, C, D, _, h0 = _packed_case(5)
+    cu = np.array([0, x.shape[1]], dtype=np.int32)
+    y, final = oracle.ssd_scan_varlen(x, dt, A, B, C, D, cu, h0[:1])
+    y_ref, f_ref, _ = oracle.ssd_scan(x, dt, A, B, C, D, h0[:1])
+    assert np.array_equal(y, y_ref) and np.array_equal(final, f_ref)
+
+
+def test_packed_sequences_do_not_see_each_other():
+    x, dt, A, B, C, D, cu, h0 = _packed_case(6)
+    y, final = oracle.ssd_scan_varlen(x, dt, A, B, C, D, cu, h0)
+    x2, B2 = x.copy(), B.copy()
+    x2[0, cu[3]:cu[4]] *= -3.0          # change only the fourth sequence's inputs
+    B2[0, cu[3]:cu[4]] += 1.0
+    y2, final2 = oracle.ssd_scan_varlen(x2, dt, A, B2, C, D, cu, h0)
+    outside = np.ones(x.shape[1], dtype=bool)
+    outside[cu[3]:cu[4]] = False
+    assert np.array_equal(y[0, outside], y2[0, outside])
+    assert np.array_equal(np.delete(final, 3, 0), np.delete(final2, 3, 0))
+    assert not np.allclose(y[0, ~outside], y2[0, ~outside])
+
+
+def test_packed_input_recipe():
+    w = configs.SSD_VARLEN.with_(seqlen=300, nheads=2, seed=77)
+    inp = inputs.make_inputs(w)
+    cu = inp.cu_seqlens
+    assert cu.dtype == np.int32 and len(cu) == w.nseq + 1
+    assert cu[0] == 0 and cu[-1] == w.seqlen and np.all(np.diff(cu) > 0)
+    assert inp.init.shape == (w.nseq, w.nheads, w.headdim, w.dstate)
