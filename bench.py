@@ -19,6 +19,7 @@ the float64 CPU oracle on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -399,6 +400,41 @@ def main():
     torch.cuda.synchronize()
     dec_ms = d0.elapsed_time(d1) / Kd
 
+    # ---- the same step with the block's fused steps: dt <- clamp(softplus(dt_raw + bias)) and
+    # the output gated by SiLU(z)
+    blk = inputs.make_block_inputs(w)
+    bz = torch.from_numpy(blk.z).to(dev).to(xdt)
+    bdt = torch.from_numpy(blk.dt_raw).to(dev)
+    bbias = torch.from_numpy(blk.dt_bias).to(dev)
+
+    def bfwd():
+        ssd.chunk_scan_fwd(t["x"], bdt, t["A"], t["B"], t["C"], t["D"], w.chunk, y=y,
+                           final_state=final, workspace=bws, z=bz, dt_bias=bbias,
+                           dt_softplus=True, dt_limit=blk.dt_limit)
+
+    bshape = ssd.make_shape(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                            ssd.SSD_BF16)
+    bopts = ssd.FwdOptions(bz.data_ptr(), bbias.data_ptr(), 1, *blk.dt_limit)
+    bws = torch.empty(ssd.lib().ssd_chunk_scan_fwd_ex_workspace_size(
+        ctypes.byref(bshape), w.chunk, ctypes.byref(bopts)), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        flush.fill_(1.0)
+        bfwd()
+    torch.cuda.synchronize()
+    Kb = max(10, min(K, 50))
+    b_ms = []
+    for _ in range(Kb):
+        flush.fill_(1.0)
+        b0 = torch.cuda.Event(enable_timing=True)
+        b1 = torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        bfwd()
+        b1.record(stream)
+        torch.cuda.synchronize()
+        b_ms.append(b0.elapsed_time(b1))
+    assert ssd.workspace_status(bws) == ssd.SSD_OK, "fused block scan status"
+    block_ms = statistics.mean(b_ms)
+
     # ---- packed variable-length sequences: the 2.7B layer's tokens as 12 uneven sequences
     wv = configs.SSD_VARLEN
     vin = inputs.make_inputs(wv)
@@ -501,6 +537,12 @@ def main():
                         "gbs_compulsory": total["bytes"] / (ms_per_step / 1e3) / 1e9,
                         "tflops_dense": total["flops"] / (ms_per_step / 1e3) / 1e12},
         "kernels": kernels,
+        "fused_block": {"workload": w.name + "_gated_softplus_dt",
+                        "metric": "ssd_chunk_scan_fwd_ex_tokens_per_s",
+                        "value": tokens_per_step / (block_ms / 1e3), "unit": "tokens/s",
+                        "ms_per_step": block_ms, "steps": Kb, "kernels_per_step": 5,
+                        "extra_bytes_per_step": int(blk.z.size * 2 + blk.dt_raw.size * 8),
+                        "l2": "256 MB buffer written before each timed call (outside the events)"},
         "varlen": {"workload": wv.name, "metric": "ssd_chunk_scan_varlen_fwd_tokens_per_s",
                    "value": wv.seqlen / (varlen_ms / 1e3), "unit": "tokens/s",
                    "ms_per_step": varlen_ms, "steps": Kv,

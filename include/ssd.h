@@ -122,6 +122,39 @@ ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, cons
                                      void *const *stage_events);
 
 /*
+ * Options of ssd_chunk_scan_fwd_ex: the Mamba-2 block's elementwise steps around the scan, fused
+ * into it (mohakchugh.is-a.dev "Mamba-2", Architecture: the SSM output is gated by SiLU of a
+ * second projection z; the discretisation step dt is the softplus of a projection plus a
+ * per-head bias).  Every field is optional; a zeroed struct (or NULL options) is the plain scan.
+ *
+ *   z            nullable; (batch, seqlen, nheads, headdim), element type `dtype`, 16-byte
+ *                aligned.  The output becomes y * z * sigmoid(z) (y as defined above).
+ *   dt_bias      nullable; (nheads,) float32, added to dt before the softplus.
+ *   dt_softplus  nonzero: the dt actually used is softplus(dt + dt_bias) = log(1 + exp(.)).
+ *   dt_min, dt_max
+ *                when dt_max > 0, that dt is then clamped to [dt_min, dt_max].
+ * With any of dt_bias, dt_softplus or the clamp active, `dt` is the raw projection (any sign).
+ */
+typedef struct {
+    const void *z;
+    const float *dt_bias;
+    int32_t dt_softplus;
+    float dt_min;
+    float dt_max;
+} ssd_fwd_options;
+
+/* Workspace bytes of ssd_chunk_scan_fwd_ex (0 when the arguments are invalid). */
+size_t ssd_chunk_scan_fwd_ex_workspace_size(const ssd_shape *shape, int chunk_size,
+                                            const ssd_fwd_options *options);
+
+/* ssd_chunk_scan_fwd with the fused prologue / epilogue of `options` (nullable). */
+ssd_status ssd_chunk_scan_fwd_ex(const ssd_shape *shape, const void *x, const float *dt,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 int chunk_size, const float *init_state, void *y,
+                                 float *final_state, void *workspace, size_t workspace_bytes,
+                                 void *stream, const ssd_fwd_options *options);
+
+/*
  * Variable-length packed sequences: nseq sequences stored back to back along the token axis of
  * a batch-1 tensor, each with its own state.  Sequence s covers tokens
  * [cu_seqlens[s], cu_seqlens[s + 1]); its recurrence starts from init_states[s] (or zeros) at

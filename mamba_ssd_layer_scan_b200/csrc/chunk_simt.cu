@@ -97,7 +97,7 @@ chunk_scan_simt_kernel(const T *__restrict__ x, const float *__restrict__ dt,
                        const T *__restrict__ B, const T *__restrict__ C,
                        const float *__restrict__ cs, const float *__restrict__ hin,
                        const float *__restrict__ D, T *__restrict__ y, int64_t seqlen, int H,
-                       int G, int P, int N, int Q, int64_t nchunks)
+                       int G, int P, int N, int Q, int64_t nchunks, const T *__restrict__ z)
 {
     extern __shared__ float sm[];
     float *cts = sm;                   // [kRows][N]   C rows of this tile
@@ -202,7 +202,8 @@ chunk_scan_simt_kernel(const T *__restrict__ x, const float *__restrict__ dt,
             const int t = o / P, p = o % P;
             if (t < rows) {
                 const int64_t off = ((b * seqlen + t0 + r0 + t) * H + h) * P + p;
-                y[off] = from_f32<T>(acc[j] + Dh * to_f32(x[off]));
+                const float v = acc[j] + Dh * to_f32(x[off]);
+                y[off] = from_f32<T>(z ? v * silu(to_f32(z[off])) : v);
             }
         }
     }
@@ -238,7 +239,7 @@ cudaError_t launch_chunk_scan_simt(bool is_bf16, const void *x, const float *dt,
                                    const void *B, const void *C, const float *cs,
                                    const float *hin, const float *D, void *y, int64_t batch,
                                    int64_t seqlen, int H, int G, int P, int N, int Q,
-                                   int64_t nchunks, cudaStream_t st)
+                                   int64_t nchunks, cudaStream_t st, const void *z)
 {
     const unsigned grid = (unsigned)(((Q + kRows - 1) / kRows) * H * batch * nchunks);
     const size_t smem = (size_t)(2 * kRows * N + kRows * P + kRows * (kRows + 1) +
@@ -250,14 +251,14 @@ cudaError_t launch_chunk_scan_simt(bool is_bf16, const void *x, const float *dt,
         if (e != cudaSuccess) return e;
         kern<<<grid, kThreads, smem, st>>>((const bf16 *)x, dt, (const bf16 *)B,
                                            (const bf16 *)C, cs, hin, D, (bf16 *)y, seqlen, H, G,
-                                           P, N, Q, nchunks);
+                                           P, N, Q, nchunks, (const bf16 *)z);
     } else {
         auto kern = chunk_scan_simt_kernel<float>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         kern<<<grid, kThreads, smem, st>>>((const float *)x, dt, (const float *)B,
                                            (const float *)C, cs, hin, D, (float *)y, seqlen, H,
-                                           G, P, N, Q, nchunks);
+                                           G, P, N, Q, nchunks, (const float *)z);
     }
     return cudaGetLastError();
 }

@@ -588,15 +588,18 @@ __device__ __forceinline__ void scale_pieces(uint8_t *base, int first, int strid
     }
 }
 
+template <bool kGate>   // kGate: the output is y * z * sigmoid(z)
 __global__ void __launch_bounds__(kScanThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c,
-                     const __grid_constant__ CUtensorMap tm_x2, const bf16 *__restrict__ hin,
+                     const __grid_constant__ CUtensorMap tm_x2,
+                     const __grid_constant__ CUtensorMap tm_z, const bf16 *__restrict__ hin,
                      const float *__restrict__ dtc,
                      const float *__restrict__ cs, const float *__restrict__ D,
                      bf16 *__restrict__ y, int *__restrict__ status, int64_t seqlen, int H,
-                     int G, int Q, int64_t nchunks, int nhb, int hpc, const int2 *__restrict__ tab)
+                     int G, int Q, int64_t nchunks, int nhb, int hpc, const int2 *__restrict__ tab,
+                     const bf16 *__restrict__ z)
 {
     extern __shared__ uint8_t smem_raw[];
     ScanSmem &sm = *reinterpret_cast<ScanSmem *>(
@@ -690,6 +693,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             tma_load_4d(stg, T ? &tm_x2 : &tm_x, &sm.bar_xh_full[xs], 0, h, (int)t0, (int)b);
             bulk_load(stg + kHOff, hin + ((b * nchunks + k) * H + h) * (int64_t)(kP * kN),
                       kP * kN * 2, &sm.bar_xh_full[xs]);
+            // the gate rows this tile's epilogue will read: into L2 now, a few heads ahead
+            if (kGate) tma_prefetch_l2_4d(&tm_z, 0, h, (int)(t0 + kTileRows * T), (int)b);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (lane 0 alone runs the loop: a lane that issued
@@ -924,15 +929,32 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&sm.bar_acc_free[a]);
+                const int64_t yoff = ((b * seqlen + t0 + tau) * H + h0 + jj) * (int64_t)kP + 16 * cq;
+                // gated output (z given): y * z * sigmoid(z); z kept as 8 packed bf16 pairs
+                const bool gz = kGate && tau < len;
+                uint4 z0 = make_uint4(0u, 0u, 0u, 0u), z1 = z0;
+                if (gz) {
+                    const uint4 *zrow = reinterpret_cast<const uint4 *>(z + yoff);
+                    z0 = zrow[0];
+                    z1 = zrow[1];
+                }
+                const uint32_t zw[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
                 uint32_t pk[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    pk[c] = pack_bf16x2(
-                        fmaf(f, __uint_as_float(a0[2 * c]), __uint_as_float(d0[2 * c])),
-                        fmaf(f, __uint_as_float(a0[2 * c + 1]), __uint_as_float(d0[2 * c + 1])));
+                for (int c = 0; c < 8; ++c) {
+                    float v0 = fmaf(f, __uint_as_float(a0[2 * c]), __uint_as_float(d0[2 * c]));
+                    float v1 =
+                        fmaf(f, __uint_as_float(a0[2 * c + 1]), __uint_as_float(d0[2 * c + 1]));
+                    if (gz) {
+                        const float2 zf = __bfloat1622float2(
+                            *reinterpret_cast<const __nv_bfloat162 *>(&zw[c]));
+                        v0 *= silu(zf.x);
+                        v1 *= silu(zf.y);
+                    }
+                    pk[c] = pack_bf16x2(v0, v1);
+                }
                 if (tau < len) {
-                    uint4 *yrow = reinterpret_cast<uint4 *>(
-                        y + ((b * seqlen + t0 + tau) * H + h0 + jj) * (int64_t)kP + 16 * cq);
+                    uint4 *yrow = reinterpret_cast<uint4 *>(y + yoff);
                     yrow[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     yrow[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
@@ -1090,9 +1112,17 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
                                  int Q, int64_t nchunks, cudaStream_t st, const char **why,
-                                 const int2 *tab)
+                                 const int2 *tab, const bf16 *z)
 {
-    CUtensorMap mx, mx2, mb, mc;
+    CUtensorMap mx, mx2, mb, mc, mz;
+    if (z) {
+        if (!make_seq_map(&mz, z, batch, seqlen, H, kP)) {
+            *why = "chunk scan: cuTensorMapEncodeTiled failed (z)";
+            return cudaErrorInvalidValue;
+        }
+    } else {
+        mz = {};
+    }
     if (!make_seq_map(&mx, x, batch, seqlen, H, kP) ||
         !make_seq_map(&mx2, x, batch, seqlen, H, kP, 2 * kTileRows) ||
         !make_seq_map(&mb, B, batch, seqlen, G, kN) ||
@@ -1106,13 +1136,13 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     const int hpc = std::min(hpg, kScanMaxHeads);
     const int nhb = (hpg + hpc - 1) / hpc;
     const size_t smem = sizeof(ScanSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(chunk_scan_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = z ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk scan: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb * (Q / kTileRows));
-    chunk_scan_tc_kernel<<<grid, kScanThreads, smem, st>>>(mx, mb, mc, mx2, hin, dtc, cs, D, y,
-                                                           status, seqlen, H, G, Q, nchunks, nhb,
-                                                           hpc, tab);
+    kern<<<grid, kScanThreads, smem, st>>>(mx, mb, mc, mx2, mz, hin, dtc, cs, D, y, status, seqlen,
+                                           H, G, Q, nchunks, nhb, hpc, tab, z);
     *why = "chunk scan (tcgen05) launch";
     return cudaGetLastError();
 }

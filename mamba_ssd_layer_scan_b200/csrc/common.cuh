@@ -18,6 +18,11 @@ template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __f
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// The SiLU gate z * sigmoid(z) of the block's output.  Fast exponential and division (about
+// 2 ulp; the gated output is stored in bf16 or compared at 1e-4): for z -> -inf the divisor
+// overflows to inf and the result is -0, the limit.
+__device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.f + __expf(-z)); }
+
 // Workspace regions of one ssd_chunk_scan_fwd call (byte offsets from the workspace base).
 struct WsLayout {
     size_t status;      // 256 bytes: device status word (nonzero after an in-kernel timeout)
@@ -85,11 +90,18 @@ cudaError_t launch_state_passing_varlen(float *states, const float *cs, const fl
                                         const int32_t *cstart, int nseq, int H, int P, int N,
                                         int Q, int64_t nchunks, cudaStream_t st);
 
+// z (nullable, x's element type and layout): the output is gated, y * z * sigmoid(z).
 cudaError_t launch_chunk_scan_simt(bool is_bf16, const void *x, const float *dt,
                                    const void *B, const void *C, const float *cs,
                                    const float *hin, const float *D, void *y, int64_t batch,
                                    int64_t seqlen, int H, int G, int P, int N, int Q,
-                                   int64_t nchunks, cudaStream_t st);
+                                   int64_t nchunks, cudaStream_t st, const void *z = nullptr);
+
+// dt_out[r][h] = clamp(softplus(dt[r][h] + bias[h])) over rows r < nrows (bias nullable; the
+// softplus and the clamp to [lo, hi] each optional).
+cudaError_t launch_dt_prologue(const float *dt, const float *bias, float *dt_out, int64_t nrows,
+                               int H, bool softplus, bool clamp, float lo, float hi,
+                               cudaStream_t st);
 
 cudaError_t launch_state_update(bool is_bf16, float *state, const void *x, const float *dt,
                                 const float *A, const void *B, const void *C, const float *D,
@@ -128,6 +140,6 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
                                  int Q, int64_t nchunks, cudaStream_t st, const char **why,
-                                 const int2 *tab = nullptr);
+                                 const int2 *tab = nullptr, const bf16 *z = nullptr);
 
 }  // namespace ssd

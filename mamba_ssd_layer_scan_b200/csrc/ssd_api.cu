@@ -172,12 +172,21 @@ ssd_status ssd_chunk_scan_fwd(const ssd_shape *shape, const void *x, const float
                                      final_state, workspace, workspace_bytes, stream, nullptr);
 }
 
-ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, const float *dt,
-                                     const float *A, const void *B, const void *C,
-                                     const float *D, int chunk_size, const float *init_state,
-                                     void *y, float *final_state, void *workspace,
-                                     size_t workspace_bytes, void *stream,
-                                     void *const *stage_events)
+}  // extern "C"
+
+namespace {
+
+bool prologue_active(const ssd_fwd_options *o)
+{
+    return o && (o->dt_bias || o->dt_softplus || o->dt_max > 0.f);
+}
+
+// The whole chunked scan; stage_events and options are both nullable.
+ssd_status scan_impl(const ssd_shape *shape, const void *x, const float *dt, const float *A,
+                     const void *B, const void *C, const float *D, int chunk_size,
+                     const float *init_state, void *y, float *final_state, void *workspace,
+                     size_t workspace_bytes, void *stream, void *const *stage_events,
+                     const ssd_fwd_options *opts)
 {
     ssd_status st = check_shape(shape, true);
     if (st != SSD_OK) return st;
@@ -209,13 +218,19 @@ ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, cons
         return fail(SSD_ERR_INVALID_ARG, "x, B, C and y must be 16-byte aligned");
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(SSD_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const void *z = opts ? opts->z : nullptr;
+    if (z && !aligned16(z)) return fail(SSD_ERR_INVALID_ARG, "z must be 16-byte aligned");
+    const bool pro = prologue_active(opts);
+    if (pro && opts->dt_max > 0.f && !(opts->dt_min <= opts->dt_max))
+        return fail(SSD_ERR_INVALID_ARG, "dt_min must not exceed dt_max");
     const int64_t nchunks = (s.seqlen + Q - 1) / Q;
     if (s.batch * nchunks * s.nheads * ((Q + 31) / 32) > 0x7fffffffLL)
         return fail(SSD_ERR_UNSUPPORTED, "problem too large for one launch grid");
     const ssd::WsLayout wl = layout(&s, Q);
-    if (workspace_bytes < wl.total)
-        return fail(SSD_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu",
-                    wl.total, workspace_bytes);
+    const size_t need = wl.total + (pro ? round256((size_t)s.batch * s.seqlen * H * 4) : 0);
+    if (workspace_bytes < need)
+        return fail(SSD_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", need,
+                    workspace_bytes);
 
     char *ws = static_cast<char *>(workspace);
     int *status = reinterpret_cast<int *>(ws + wl.status);
@@ -223,6 +238,14 @@ ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, cons
     float *states = reinterpret_cast<float *>(ws + wl.states);
     cudaError_t e = record(stage_events, 0, cs_stream);
     if (e != cudaSuccess) return cuda_fail(e, "record stage event");
+    if (pro) {   // dt <- clamp(softplus(dt + dt_bias)) into the workspace; the scan reads that
+        float *dt_eff = reinterpret_cast<float *>(ws + wl.total);
+        e = ssd::launch_dt_prologue(dt, opts->dt_bias, dt_eff, s.batch * s.seqlen, H,
+                                    opts->dt_softplus != 0, opts->dt_max > 0.f, opts->dt_min,
+                                    opts->dt_max, cs_stream);
+        if (e != cudaSuccess) return cuda_fail(e, "dt prologue launch");
+        dt = dt_eff;
+    }
     const bool tc = ssd::tc_supported(bf, P, N, Q);
     float *dtc = tc ? reinterpret_cast<float *>(ws + wl.dtc) : nullptr;
     e = ssd::launch_chunk_cumsum(dt, A, cs, dtc, status, s.batch, s.seqlen, H, Q, nchunks,
@@ -259,7 +282,8 @@ ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, cons
         }
         e = ssd::launch_chunk_scan_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B,
                                       (const ssd::bf16 *)C, cs, hin, D, (ssd::bf16 *)y, status,
-                                      s.batch, s.seqlen, H, G, Q, nchunks, cs_stream, &why);
+                                      s.batch, s.seqlen, H, G, Q, nchunks, cs_stream, &why,
+                                      nullptr, (const ssd::bf16 *)z);
         if (e != cudaSuccess) return cuda_fail(e, why);
         if ((e = record(stage_events, 4, cs_stream)) != cudaSuccess)
             return cuda_fail(e, "record stage event");
@@ -277,11 +301,44 @@ ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, cons
     if ((e = record(stage_events, 3, cs_stream)) != cudaSuccess)
         return cuda_fail(e, "record stage event");
     e = ssd::launch_chunk_scan_simt(bf, x, dt, B, C, cs, states, D, y, s.batch, s.seqlen, H, G,
-                                    P, N, Q, nchunks, cs_stream);
+                                    P, N, Q, nchunks, cs_stream, z);
     if (e != cudaSuccess) return cuda_fail(e, "chunk scan launch");
     if ((e = record(stage_events, 4, cs_stream)) != cudaSuccess)
         return cuda_fail(e, "record stage event");
     return SSD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ssd_status ssd_chunk_scan_fwd_staged(const ssd_shape *shape, const void *x, const float *dt,
+                                     const float *A, const void *B, const void *C,
+                                     const float *D, int chunk_size, const float *init_state,
+                                     void *y, float *final_state, void *workspace,
+                                     size_t workspace_bytes, void *stream,
+                                     void *const *stage_events)
+{
+    return scan_impl(shape, x, dt, A, B, C, D, chunk_size, init_state, y, final_state,
+                     workspace, workspace_bytes, stream, stage_events, nullptr);
+}
+
+size_t ssd_chunk_scan_fwd_ex_workspace_size(const ssd_shape *shape, int chunk_size,
+                                            const ssd_fwd_options *options)
+{
+    const size_t base = ssd_chunk_scan_workspace_size(shape, chunk_size);
+    if (base == 0 || !prologue_active(options)) return base;
+    return base + round256((size_t)shape->batch * shape->seqlen * shape->nheads * 4);
+}
+
+ssd_status ssd_chunk_scan_fwd_ex(const ssd_shape *shape, const void *x, const float *dt,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 int chunk_size, const float *init_state, void *y,
+                                 float *final_state, void *workspace, size_t workspace_bytes,
+                                 void *stream, const ssd_fwd_options *options)
+{
+    return scan_impl(shape, x, dt, A, B, C, D, chunk_size, init_state, y, final_state,
+                     workspace, workspace_bytes, stream, nullptr, options);
 }
 
 size_t ssd_chunk_scan_varlen_workspace_size(const ssd_shape *shape, int nseq, int chunk_size)

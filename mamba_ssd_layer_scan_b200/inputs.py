@@ -61,6 +61,29 @@ class SSDInputs:
     cu_seqlens: Optional[np.ndarray] = None   # int32 (nseq + 1,) for packed sequences
 
 
+@dataclass
+class BlockInputs:
+    """The Mamba-2 block's raw projections around the scan (float32, exact stored values)."""
+    z: np.ndarray          # gate, (b, L, H, P), rounded to bf16 for bf16 workloads
+    dt_raw: np.ndarray     # dt projection before bias / softplus / clamp, (b, L, H)
+    dt_bias: np.ndarray    # (H,)
+    dt_limit: tuple        # clamp after the softplus
+
+
+def make_block_inputs(w: Workload, seed: Optional[int] = None) -> BlockInputs:
+    """z ~ N(0, 1); dt_raw ~ N(0, 1); dt_bias_h = -4 + U(-0.5, 0.5); clamp (1e-3, 0.1), so that
+    softplus(dt_raw + dt_bias) matches the dt recipe above.  Drawn from its own PCG64 stream
+    (seed + 500) so the scan inputs of the same workload are unchanged."""
+    rng = np.random.Generator(np.random.PCG64((w.seed if seed is None else seed) + 500))
+    b, L, H, P = w.batch, w.seqlen, w.nheads, w.headdim
+    z = rng.standard_normal((b, L, H, P), dtype=np.float32)
+    dt_raw = rng.standard_normal((b, L, H), dtype=np.float32)
+    dt_bias = (-4.0 + rng.uniform(-0.5, 0.5, H)).astype(np.float32)
+    if w.dtype == "bf16":
+        z = round_bf16(z)
+    return BlockInputs(z, dt_raw, dt_bias, (1e-3, 0.1))
+
+
 def make_inputs(w: Workload, seed: Optional[int] = None) -> SSDInputs:
     rng = np.random.Generator(np.random.PCG64(w.seed if seed is None else seed))
     b, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups

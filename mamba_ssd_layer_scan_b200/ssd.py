@@ -36,6 +36,12 @@ class Shape(ctypes.Structure):
                 ("dtype", ctypes.c_int32)]
 
 
+class FwdOptions(ctypes.Structure):
+    _fields_ = [("z", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+                ("dt_softplus", ctypes.c_int32), ("dt_min", ctypes.c_float),
+                ("dt_max", ctypes.c_float)]
+
+
 _lib = None
 _vp = ctypes.c_void_p
 
@@ -64,6 +70,12 @@ def lib():
     L.ssd_chunk_scan_fwd_staged.restype = ctypes.c_int
     L.ssd_chunk_scan_fwd_staged.argtypes = L.ssd_chunk_scan_fwd.argtypes + [
         ctypes.POINTER(ctypes.c_void_p)]
+    L.ssd_chunk_scan_fwd_ex_workspace_size.restype = ctypes.c_size_t
+    L.ssd_chunk_scan_fwd_ex_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int,
+                                                       ctypes.POINTER(FwdOptions)]
+    L.ssd_chunk_scan_fwd_ex.restype = ctypes.c_int
+    L.ssd_chunk_scan_fwd_ex.argtypes = L.ssd_chunk_scan_fwd.argtypes + [
+        ctypes.POINTER(FwdOptions)]
     L.ssd_chunk_scan_varlen_workspace_size.restype = ctypes.c_size_t
     L.ssd_chunk_scan_varlen_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int,
                                                        ctypes.c_int]
@@ -146,12 +158,15 @@ def new_workspace(shape: Shape, chunk_size: int, device):
 
 def chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int = 256, init_state=None,
                    return_final_state: bool = True, y=None, final_state=None, workspace=None,
-                   stream=None, stage_events=None):
+                   stream=None, stage_events=None, z=None, dt_bias=None,
+                   dt_softplus: bool = False, dt_limit=None):
     """Chunked SSD scan.  x (b, L, H, P), dt (b, L, H) f32, A/D (H,) f32, B/C (b, L, G, N),
     init_state (b, H, P, N) f32 or None.  Returns (y, final_state or None).
 
     stage_events: optional list of 5 recorded-once torch.cuda.Event objects, recorded on the
-    stream around the four kernels (see ssd_chunk_scan_fwd_staged)."""
+    stream around the four kernels (see ssd_chunk_scan_fwd_staged).
+    z, dt_bias, dt_softplus, dt_limit=(lo, hi): the fused block steps of
+    ssd_chunk_scan_fwd_ex (gated output y * silu(z); dt <- clamp(softplus(dt + dt_bias)))."""
     torch = _torch()
     b, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
@@ -164,16 +179,35 @@ def chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int = 256, init_state=None,
     if init_state is not None:
         _require(init_state, "init_state", torch.float32, dev)
     shape = make_shape(b, L, H, P, N, G, code)
+    opts = None
+    if z is not None or dt_bias is not None or dt_softplus or dt_limit is not None:
+        if stage_events is not None:
+            raise ValueError("stage_events and the fused block options cannot be combined")
+        if z is not None:
+            _require(z, "z", x.dtype, dev)
+        if dt_bias is not None:
+            _require(dt_bias, "dt_bias", torch.float32, dev)
+        lo, hi = dt_limit if dt_limit is not None else (0.0, 0.0)
+        opts = FwdOptions(_ptr(z), _ptr(dt_bias), 1 if dt_softplus else 0, lo, hi)
     if y is None:
         y = torch.empty_like(x)
     if final_state is None and return_final_state:
         final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
     if workspace is None:
-        workspace = new_workspace(shape, chunk_size, dev)
+        if opts is None:
+            workspace = new_workspace(shape, chunk_size, dev)
+        else:
+            n = lib().ssd_chunk_scan_fwd_ex_workspace_size(ctypes.byref(shape), chunk_size,
+                                                          ctypes.byref(opts))
+            if n == 0:
+                raise SSDError(SSD_ERR_INVALID_ARG, last_error())
+            workspace = torch.empty(n, dtype=torch.uint8, device=dev)
     args = (ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
             chunk_size, _ptr(init_state), _ptr(y), _ptr(final_state), _ptr(workspace),
             workspace.numel(), _stream_handle(stream))
-    if stage_events is None:
+    if opts is not None:
+        _check(lib().ssd_chunk_scan_fwd_ex(*args, ctypes.byref(opts)))
+    elif stage_events is None:
         _check(lib().ssd_chunk_scan_fwd(*args))
     else:
         handles = (ctypes.c_void_p * 5)(*[ev.cuda_event for ev in stage_events])

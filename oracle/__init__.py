@@ -121,6 +121,33 @@ def ssd_scan_pairs(inp, pairs: Sequence[Tuple[int, int]], every: int = 0,
     return y, final[0], (None if boundary is None else boundary[0])
 
 
+def dt_prologue(dt, dt_bias=None, softplus: bool = False, dt_limit=None):
+    """The dt the scan uses when the block's raw projection is passed: dt + dt_bias, then
+    softplus(v) = log(1 + exp(v)) when asked, then clamped to dt_limit = (lo, hi) when given
+    (mohakchugh.is-a.dev "Mamba-2", Architecture: Multi-Head SSM).  float64."""
+    v = np.asarray(dt, dtype=np.float64)
+    if dt_bias is not None:
+        v = v + np.asarray(dt_bias, dtype=np.float64)
+    if softplus:
+        v = np.logaddexp(0.0, v)
+    if dt_limit is not None:
+        v = np.clip(v, dt_limit[0], dt_limit[1])
+    return v
+
+
+def ssd_scan_block(x, dt, A, B, C, D, init=None, z=None, dt_bias=None, softplus: bool = False,
+                   dt_limit=None):
+    """The scan with the Mamba-2 block's elementwise steps around it: the dt prologue above,
+    then the recurrence, then the output gated by SiLU(z) = z / (1 + exp(-z)) (same page, the
+    gated output of the block).  Returns (y, final_state)."""
+    dt_eff = dt_prologue(dt, dt_bias, softplus, dt_limit)
+    y, final, _ = ssd_scan(x, dt_eff, A, B, C, D, init)
+    if z is not None:
+        zf = np.asarray(z, dtype=np.float64)
+        y = y * (zf / (1.0 + np.exp(-zf)))
+    return y, final
+
+
 def ssd_scan_varlen(x, dt, A, B, C, D, cu_seqlens, init=None):
     """Packed variable-length sequences: sequence s (tokens cu_seqlens[s] .. cu_seqlens[s+1]-1
     of the single batch row) is its own recurrence, started from init[s] (or zeros), so this is

@@ -149,3 +149,24 @@ def test_varlen_rejects_bad_arguments(L, kw, nseq, chunk, code):
                                      None, p, 1 << 40, None)
     assert rc == code
     assert ssd.last_error()
+
+
+def test_fused_options_workspace_and_validation(L):
+    sh = _shape()
+    base = ssd.workspace_size(sh, 256)
+    gate_only = ssd.FwdOptions(1 << 20, None, 0, 0.0, 0.0)
+    assert L.ssd_chunk_scan_fwd_ex_workspace_size(ctypes.byref(sh), 256,
+                                                  ctypes.byref(gate_only)) == base
+    pro = ssd.FwdOptions(None, None, 1, 1e-3, 0.1)   # the prologue needs one dt per token-head
+    r = lambda v: (v + 255) // 256 * 256
+    assert L.ssd_chunk_scan_fwd_ex_workspace_size(ctypes.byref(sh), 256, ctypes.byref(pro)) == \
+        base + r(4 * 4096 * 80 * 4)
+    p = ctypes.c_void_p(1 << 20)
+    bad = ssd.FwdOptions(ctypes.c_void_p((1 << 20) + 2), None, 0, 0.0, 0.0)   # misaligned z
+    rc = L.ssd_chunk_scan_fwd_ex(ctypes.byref(sh), p, p, p, p, p, p, 256, None, p, None, p,
+                                 1 << 40, None, ctypes.byref(bad))
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "z must" in ssd.last_error()
+    inv = ssd.FwdOptions(None, None, 1, 0.5, 0.1)   # dt_min > dt_max
+    rc = L.ssd_chunk_scan_fwd_ex(ctypes.byref(sh), p, p, p, p, p, p, 256, None, p, None, p,
+                                 1 << 40, None, ctypes.byref(inv))
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "dt_min" in ssd.last_error()

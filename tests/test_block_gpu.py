@@ -1,0 +1,118 @@
+"""GPU parity of the fused block steps (ssd_chunk_scan_fwd_ex) against the float64 oracle.
+
+The dt the scan uses is softplus(dt_raw + dt_bias) clamped to (1e-3, 0.1) -- the same
+distribution as the plain workloads' dt -- and the output is gated by SiLU(z).  Both are fused:
+the prologue runs before the cumsum, the gate in the chunk-scan epilogue, on the tensor-core and
+on the CUDA-core paths.  Tolerances as for the plain scan (max over (batch, head) slices of the
+relative L2 error of y and of the final state).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from mamba_ssd_layer_scan_b200 import configs, inputs, ssd
+
+from _util import TOL, max_rel_per_pair, spread_pairs, to_np, torch_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(torch, inp, blk, chunk, device, gate=True, prologue=True):
+    t = torch_inputs(inp, device)
+    xdt = t["x"].dtype
+    z = torch.from_numpy(blk.z).to(device).to(xdt) if gate else None
+    if prologue:
+        dt = torch.from_numpy(blk.dt_raw).to(device)
+        bias = torch.from_numpy(blk.dt_bias).to(device)
+        y, final = ssd.chunk_scan_fwd(t["x"], dt, t["A"], t["B"], t["C"], t["D"], chunk,
+                                      init_state=t["init_state"], z=z, dt_bias=bias,
+                                      dt_softplus=True, dt_limit=blk.dt_limit)
+    else:
+        y, final = ssd.chunk_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk,
+                                      init_state=t["init_state"], z=z)
+    torch.cuda.synchronize()
+    return y, final
+
+
+def _reference(inp, blk, gate=True, prologue=True):
+    if prologue:
+        return oracle.ssd_scan_block(inp.x, blk.dt_raw, inp.A, inp.B, inp.C, inp.D, inp.init,
+                                     z=blk.z if gate else None, dt_bias=blk.dt_bias,
+                                     softplus=True, dt_limit=blk.dt_limit)
+    return oracle.ssd_scan_block(inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, inp.init,
+                                 z=blk.z if gate else None)
+
+
+def _compare(w, y, final, y_ref, f_ref):
+    yn, fn = to_np(y), to_np(final)
+    pairs = [(b, h) for b in range(w.batch) for h in range(w.nheads)]
+    ey = max_rel_per_pair([yn[b, :, h] for b, h in pairs], [y_ref[b, :, h] for b, h in pairs])
+    ef = max_rel_per_pair([fn[b, h] for b, h in pairs], [f_ref[b, h] for b, h in pairs])
+    assert np.isfinite(yn).all()
+    assert ey <= TOL[w.dtype], f"y relative L2 error {ey:.3e}"
+    assert ef <= TOL[w.dtype], f"final state relative L2 error {ef:.3e}"
+
+
+CASES = [
+    # (name, workload, chunk, gate, prologue)
+    ("tc_q256_both", configs.SSD_370M.with_(batch=2, seqlen=700, nheads=10, init_state=True), 256,
+     True, True),
+    ("tc_q128_gate", configs.SSD_370M.with_(batch=1, seqlen=600, nheads=8, ngroups=2), 128,
+     True, False),
+    ("tc_q256_prologue", configs.SSD_370M.with_(batch=1, seqlen=300, nheads=6), 256, False,
+     True),
+    ("f32_simt_both", configs.SSD_F32_SMALL.with_(batch=2, seqlen=333, nheads=4, ngroups=2,
+                                                  init_state=True), 64, True, True),
+    ("bf16_simt_both", configs.SSD_370M.with_(batch=1, seqlen=300, nheads=4), 64, True, True),
+]
+
+
+@pytest.mark.parametrize("name,w,chunk,gate,prologue", CASES, ids=[c[0] for c in CASES])
+def test_fused_block_parity(cuda_device, name, w, chunk, gate, prologue):
+    import torch
+    inp = inputs.make_inputs(w)
+    blk = inputs.make_block_inputs(w)
+    y, final = _run(torch, inp, blk, chunk, cuda_device, gate, prologue)
+    y_ref, f_ref = _reference(inp, blk, gate, prologue)
+    _compare(w, y, final, y_ref, f_ref)
+
+
+def test_fused_block_full_size_sampled(cuda_device):
+    """The 2.7B-layer shape in the benchmark's launch configuration, gated and with the dt
+    prologue; sampled (batch, head) slices against the oracle."""
+    import torch
+    w = configs.SSD_2P7B
+    inp = inputs.make_inputs(w)
+    blk = inputs.make_block_inputs(w)
+    y, final = _run(torch, inp, blk, w.chunk, cuda_device)
+    yn, fn = to_np(y), to_np(final)
+    dt_eff = oracle.dt_prologue(blk.dt_raw, blk.dt_bias, True, blk.dt_limit)
+    inp.dt = dt_eff
+    pairs = spread_pairs(w.batch, w.nheads, 8, seed=w.seed + 3)
+    ys, fs, _ = oracle.ssd_scan_pairs(inp, pairs)
+    zs = [blk.z[b, :, h].astype(np.float64) for b, h in pairs]
+    ys_ref = [ys[i] * (zs[i] / (1.0 + np.exp(-zs[i]))) for i in range(len(pairs))]
+    assert max_rel_per_pair([yn[b, :, h] for b, h in pairs], ys_ref) <= TOL["bf16"]
+    assert max_rel_per_pair([fn[b, h] for b, h in pairs], list(fs)) <= TOL["bf16"]
+
+
+def test_plain_options_equal_plain_scan(cuda_device):
+    """A zeroed options struct is the plain scan, bit for bit."""
+    import ctypes
+    import torch
+    w = configs.SSD_370M.with_(batch=1, seqlen=512, nheads=8)
+    t = torch_inputs(inputs.make_inputs(w), cuda_device)
+    y0, f0 = ssd.chunk_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], 256)
+    shape = ssd.make_shape(1, 512, 8, 64, 128, 1, ssd.SSD_BF16)
+    opts = ssd.FwdOptions(None, None, 0, 0.0, 0.0)
+    ws = ssd.new_workspace(shape, 256, cuda_device)
+    y1 = torch.empty_like(y0)
+    f1 = torch.empty_like(f0)
+    rc = ssd.lib().ssd_chunk_scan_fwd_ex(
+        ctypes.byref(shape), t["x"].data_ptr(), t["dt"].data_ptr(), t["A"].data_ptr(),
+        t["B"].data_ptr(), t["C"].data_ptr(), t["D"].data_ptr(), 256, None, y1.data_ptr(),
+        f1.data_ptr(), ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream,
+        ctypes.byref(opts))
+    assert rc == ssd.SSD_OK, ssd.last_error()
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1) and torch.equal(f0, f1)

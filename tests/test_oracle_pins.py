@@ -340,3 +340,49 @@ def test_packed_input_recipe():
     assert cu.dtype == np.int32 and len(cu) == w.nseq + 1
     assert cu[0] == 0 and cu[-1] == w.seqlen and np.all(np.diff(cu) > 0)
     assert inp.init.shape == (w.nseq, w.nheads, w.headdim, w.dstate)
+
+
+# ------------------------------------------------------------------ fused block steps
+def test_gate_closed_forms():
+    """SiLU(0) = 0 and SiLU(z) = z (1 - 1/(1+e^z)) -> z for large z: a zero gate silences the
+    output, a large gate scales it by z, and the state never sees the gate."""
+    x, dt, A, B, C, D, h0 = _rand_case(8)
+    y, f, _ = oracle.ssd_scan(x, dt, A, B, C, D, h0)
+    y0, f0 = oracle.ssd_scan_block(x, dt, A, B, C, D, h0, z=np.zeros_like(x))
+    assert np.all(y0 == 0.0) and np.array_equal(f0, f)
+    y50, _ = oracle.ssd_scan_block(x, dt, A, B, C, D, h0, z=np.full_like(x, 50.0))
+    assert _rel(y50, 50.0 * y) < 1e-14
+    ym, _ = oracle.ssd_scan_block(x, dt, A, B, C, D, h0, z=np.full_like(x, -50.0))
+    assert np.max(np.abs(ym)) <= 50.0 * np.exp(-50.0) * np.max(np.abs(y)) * 1.01
+
+
+def test_softplus_prologue_closed_form():
+    """softplus(log(e^v - 1)) = v: a raw dt of log(expm1(v)) reproduces the scan at dt = v."""
+    x, dt, A, B, C, D, h0 = _rand_case(9)
+    raw = np.log(np.expm1(dt))
+    y, f, _ = oracle.ssd_scan(x, dt, A, B, C, D, h0)
+    y2, f2 = oracle.ssd_scan_block(x, raw, A, B, C, D, h0, softplus=True)
+    assert _rel(y2, y) < 1e-12 and _rel(f2, f) < 1e-12
+    bias = np.linspace(-0.3, 0.4, A.shape[0])
+    y3, f3 = oracle.ssd_scan_block(x, raw - bias, A, B, C, D, h0, dt_bias=bias, softplus=True)
+    assert _rel(y3, y) < 1e-12 and _rel(f3, f) < 1e-12
+
+
+def test_clamp_prologue_equals_clipped_dt():
+    x, dt, A, B, C, D, h0 = _rand_case(10)
+    lo, hi = 0.05, 0.3
+    y, f, _ = oracle.ssd_scan(x, np.clip(dt, lo, hi), A, B, C, D, h0)
+    y2, f2 = oracle.ssd_scan_block(x, dt, A, B, C, D, h0, dt_limit=(lo, hi))
+    assert np.array_equal(y2, y) and np.array_equal(f2, f)
+    assert np.any(dt < lo) and np.any(dt > hi)   # the clamp is exercised on both sides
+
+
+def test_block_input_recipe():
+    w = configs.SSD_370M.with_(seqlen=512, nheads=8)
+    blk = inputs.make_block_inputs(w)
+    dt = oracle.dt_prologue(blk.dt_raw, blk.dt_bias, True, blk.dt_limit)
+    assert dt.min() >= 1e-3 and dt.max() <= 0.1
+    base = inputs.make_inputs(w)          # the scan inputs are not disturbed by the extra draw
+    again = inputs.make_inputs(w)
+    assert np.array_equal(base.x, again.x)
+    assert blk.z.shape == base.x.shape and np.array_equal(inputs.round_bf16(blk.z), blk.z)
