@@ -186,6 +186,42 @@ ssd_status ssd_chunk_scan_varlen_fwd(const ssd_shape *shape, const void *x, cons
                                      size_t workspace_bytes, void *stream);
 
 /*
+ * Sequence parallelism: one long sequence split into contiguous segments, one per rank (GPU),
+ * with one exchange of states between the two phases (the state is carried across segments
+ * exactly as across chunks: mohakchugh.is-a.dev "Mamba-2", Block Decomposition).  Every rank r
+ * holds its segment's x, dt, B, C as a (batch, seqlen_r, ...) tensor and calls
+ *
+ *   1. ssd_seqpar_local: chunk states of the segment and, from a zero initial state, its local
+ *      final state h_loc (batch, nheads, headdim, dstate) float32 and its total log-decay
+ *      log_decay (batch, nheads) float32 = sum of dt * A_h over the segment's tokens;
+ *   2. (the caller) all-gathers h_loc and log_decay of all ranks in rank order, e.g. with
+ *      torch.distributed.all_gather_into_tensor over NCCL: h_loc_all [nranks][batch][H][P][N],
+ *      log_decay_all [nranks][batch][H];
+ *   3. ssd_seqpar_finish: the segment's initial state
+ *          h_in(r) = sum_{q<r} exp(sum_{q<s<r} log_decay_s) h_loc(q)
+ *                    + exp(sum_{s<r} log_decay_s) init_state
+ *      (init_state: the whole sequence's initial state, nullable; every rank passes the same),
+ *      then y of the segment and, in final_state (nullable), the state after the segment's
+ *      last token -- the sequence's final state on the last rank.
+ *
+ * Both phases take the same workspace (ssd_seqpar_workspace_size bytes, 256-byte aligned),
+ * which carries the chunk states from phase 1 to phase 3.  On one rank (nranks = 1) the result
+ * equals ssd_chunk_scan_fwd.  Tensor-core path only (bf16, headdim 64, dstate 128, chunk_size
+ * 128 or 256); other shapes return SSD_ERR_UNSUPPORTED.  log_decay_all and h_loc_all may be
+ * NULL on rank 0 (nothing precedes it).
+ */
+size_t ssd_seqpar_workspace_size(const ssd_shape *shape, int chunk_size);
+ssd_status ssd_seqpar_local(const ssd_shape *shape, const void *x, const float *dt,
+                            const float *A, const void *B, int chunk_size, float *h_loc,
+                            float *log_decay, void *workspace, size_t workspace_bytes,
+                            void *stream);
+ssd_status ssd_seqpar_finish(const ssd_shape *shape, const void *x, const void *B, const void *C,
+                             const float *D, int chunk_size, const float *h_loc_all,
+                             const float *log_decay_all, int nranks, int rank,
+                             const float *init_state, void *y, float *final_state,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * One recurrent (decode) step for one new token per sequence, O(1) in the length of the past
  * (crackai.dev "Transformers are SSMs", Why It Matters; mohakchugh.is-a.dev "Mamba-2", Why
  * This Matters for Hardware, linear mode):

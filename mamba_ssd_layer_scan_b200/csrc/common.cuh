@@ -128,6 +128,15 @@ __host__ __device__ __forceinline__ int hin_swizzled_offset(int p, int n)
     return a * 4096 + p * 64 + ((((nl >> 3) ^ (p & 7)) << 3) | (nl & 7));
 }
 
+// Sequence parallelism (one contiguous segment per rank): the segment's total log-decay per
+// (batch, head), and the combine of the all-gathered local final states into the segment's
+// initial state (h_loc_all [nranks][BH][PN], logdec_all [nranks][BH]; init nullable).
+cudaError_t launch_segment_log_decay(const float *cs, float *out, int64_t batch, int H, int Q,
+                                     int64_t nchunks, cudaStream_t st);
+cudaError_t launch_seqpar_combine(const float *h_loc_all, const float *logdec_all,
+                                  const float *init, float *h_in, int nranks, int rank,
+                                  int64_t BH, int PN, cudaStream_t st);
+
 // Chunk state and state passing in one kernel (chunks walked in order per block of heads):
 // writes the bf16 entering states and the float32 final state; no float32 chunk states.
 bool fused_state_pass_ok(int64_t batch, int H, int G);

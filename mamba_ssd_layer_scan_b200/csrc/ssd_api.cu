@@ -413,6 +413,137 @@ ssd_status ssd_chunk_scan_varlen_fwd(const ssd_shape *shape, const void *x, cons
     return SSD_OK;
 }
 
+// ---- sequence parallelism (one contiguous segment of the sequence per rank)
+namespace {
+ssd_status check_seqpar(const ssd_shape *s, int Q)
+{
+    ssd_status st = check_shape(s, true);
+    if (st != SSD_OK) return st;
+    if (!valid_chunk(Q))
+        return fail(SSD_ERR_UNSUPPORTED, "chunk_size must be 16, 32, 64, 128 or 256 (got %d)", Q);
+    if (!ssd::tc_supported(s->dtype == SSD_BF16, (int)s->headdim, (int)s->dstate, Q))
+        return fail(SSD_ERR_UNSUPPORTED,
+                    "sequence-parallel scan runs on the tensor-core path only: bf16, headdim 64, "
+                    "dstate 128, chunk_size 128 or 256");
+    return SSD_OK;
+}
+size_t seqpar_hseg_offset(const ssd_shape *s, int Q) { return layout(s, Q).total; }
+}  // namespace
+
+size_t ssd_seqpar_workspace_size(const ssd_shape *shape, int chunk_size)
+{
+    if (check_seqpar(shape, chunk_size) != SSD_OK) return 0;
+    return seqpar_hseg_offset(shape, chunk_size) +
+           round256((size_t)shape->batch * shape->nheads * shape->headdim * shape->dstate * 4);
+}
+
+ssd_status ssd_seqpar_local(const ssd_shape *shape, const void *x, const float *dt,
+                            const float *A, const void *B, int chunk_size, float *h_loc,
+                            float *log_decay, void *workspace, size_t workspace_bytes,
+                            void *stream)
+{
+    ssd_status st = check_seqpar(shape, chunk_size);
+    if (st != SSD_OK) return st;
+    const ssd_shape s = *shape;
+    const int H = (int)s.nheads, G = (int)s.ngroups, P = (int)s.headdim, N = (int)s.dstate;
+    const int Q = chunk_size;
+    cudaStream_t cst = static_cast<cudaStream_t>(stream);
+    if (!h_loc || !log_decay || !aligned16(h_loc))
+        return fail(SSD_ERR_INVALID_ARG, "h_loc (16-byte aligned) and log_decay must be non-NULL");
+    if (s.batch == 0) return SSD_OK;
+    cudaError_t e;
+    if (s.seqlen == 0) {   // an empty segment: no state of its own, no decay
+        e = cudaMemsetAsync(h_loc, 0, (size_t)s.batch * H * P * N * 4, cst);
+        if (e == cudaSuccess) e = cudaMemsetAsync(log_decay, 0, (size_t)s.batch * H * 4, cst);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "clear empty segment");
+    }
+    if (!x || !dt || !A || !B || !workspace)
+        return fail(SSD_ERR_INVALID_ARG, "x, dt, A, B and workspace must be non-NULL");
+    if (!aligned16(x) || !aligned16(B) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(SSD_ERR_INVALID_ARG, "x, B must be 16-byte and workspace 256-byte aligned");
+    if (workspace_bytes < ssd_seqpar_workspace_size(shape, Q))
+        return fail(SSD_ERR_INVALID_ARG, "workspace too small");
+    const int64_t nchunks = (s.seqlen + Q - 1) / Q;
+    const ssd::WsLayout wl = layout(&s, Q);
+    char *ws = static_cast<char *>(workspace);
+    int *status = reinterpret_cast<int *>(ws + wl.status);
+    float *cs = reinterpret_cast<float *>(ws + wl.cs);
+    float *dtc = reinterpret_cast<float *>(ws + wl.dtc);
+    float *states = reinterpret_cast<float *>(ws + wl.states);
+    ssd::bf16 *hin = reinterpret_cast<ssd::bf16 *>(ws + wl.hin_bf16);
+    const char *why = "";
+    e = ssd::launch_chunk_cumsum(dt, A, cs, dtc, status, s.batch, s.seqlen, H, Q, nchunks, cst);
+    if (e != cudaSuccess) return cuda_fail(e, "dA cumsum launch");
+    e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs, states,
+                                   status, s.batch, s.seqlen, H, G, Q, nchunks, cst, &why);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+    // from a zero initial state: the final state is the segment's own contribution h_loc (the
+    // entering states it also writes are replaced in the finish phase; chunk states are kept)
+    e = ssd::launch_state_passing(states, cs, nullptr, h_loc, hin, s.batch, H, P, N, Q, nchunks,
+                                  cst);
+    if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
+    e = ssd::launch_segment_log_decay(cs, log_decay, s.batch, H, Q, nchunks, cst);
+    if (e != cudaSuccess) return cuda_fail(e, "segment decay launch");
+    return SSD_OK;
+}
+
+ssd_status ssd_seqpar_finish(const ssd_shape *shape, const void *x, const void *B, const void *C,
+                             const float *D, int chunk_size, const float *h_loc_all,
+                             const float *log_decay_all, int nranks, int rank,
+                             const float *init_state, void *y, float *final_state,
+                             void *workspace, size_t workspace_bytes, void *stream)
+{
+    ssd_status st = check_seqpar(shape, chunk_size);
+    if (st != SSD_OK) return st;
+    if (nranks < 1 || rank < 0 || rank >= nranks)
+        return fail(SSD_ERR_INVALID_ARG, "rank %d out of range for %d ranks", rank, nranks);
+    const ssd_shape s = *shape;
+    const int H = (int)s.nheads, G = (int)s.ngroups, P = (int)s.headdim, N = (int)s.dstate;
+    const int Q = chunk_size;
+    cudaStream_t cst = static_cast<cudaStream_t>(stream);
+    if ((rank > 0 && (!h_loc_all || !log_decay_all)) || !workspace)
+        return fail(SSD_ERR_INVALID_ARG, "h_loc_all, log_decay_all and workspace must be non-NULL");
+    if ((h_loc_all && !aligned16(h_loc_all)) || (init_state && !aligned16(init_state)) ||
+        (final_state && !aligned16(final_state)) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(SSD_ERR_INVALID_ARG, "state pointers must be 16-byte aligned, workspace 256");
+    if (workspace_bytes < ssd_seqpar_workspace_size(shape, Q))
+        return fail(SSD_ERR_INVALID_ARG, "workspace too small");
+    if (s.batch == 0) return SSD_OK;
+    char *ws = static_cast<char *>(workspace);
+    float *hseg = reinterpret_cast<float *>(ws + seqpar_hseg_offset(&s, Q));
+    const int64_t BH = s.batch * H;
+    cudaError_t e = ssd::launch_seqpar_combine(h_loc_all, log_decay_all, init_state, hseg, nranks,
+                                               rank, BH, P * N, cst);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    if (s.seqlen == 0) {
+        if (final_state) {
+            e = ssd::launch_fill_final(hseg, final_state, BH * P * N, cst);
+            if (e != cudaSuccess) return cuda_fail(e, "fill final state");
+        }
+        return SSD_OK;
+    }
+    if (!x || !B || !C || !D || !y) return fail(SSD_ERR_INVALID_ARG, "x, B, C, D, y must be non-NULL");
+    if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(y))
+        return fail(SSD_ERR_INVALID_ARG, "x, B, C and y must be 16-byte aligned");
+    const int64_t nchunks = (s.seqlen + Q - 1) / Q;
+    const ssd::WsLayout wl = layout(&s, Q);
+    int *status = reinterpret_cast<int *>(ws + wl.status);
+    float *cs = reinterpret_cast<float *>(ws + wl.cs);
+    float *dtc = reinterpret_cast<float *>(ws + wl.dtc);
+    float *states = reinterpret_cast<float *>(ws + wl.states);
+    ssd::bf16 *hin = reinterpret_cast<ssd::bf16 *>(ws + wl.hin_bf16);
+    const char *why = "";
+    e = ssd::launch_state_passing(states, cs, hseg, final_state, hin, s.batch, H, P, N, Q,
+                                  nchunks, cst);
+    if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
+    e = ssd::launch_chunk_scan_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B,
+                                  (const ssd::bf16 *)C, cs, hin, D, (ssd::bf16 *)y, status,
+                                  s.batch, s.seqlen, H, G, Q, nchunks, cst, &why);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+    return SSD_OK;
+}
+
 ssd_status ssd_state_update(const ssd_shape *shape, float *state, const void *x,
                             const float *dt, const float *A, const void *B, const void *C,
                             const float *D, void *y, void *stream)

@@ -76,6 +76,15 @@ def lib():
     L.ssd_chunk_scan_fwd_ex.restype = ctypes.c_int
     L.ssd_chunk_scan_fwd_ex.argtypes = L.ssd_chunk_scan_fwd.argtypes + [
         ctypes.POINTER(FwdOptions)]
+    L.ssd_seqpar_workspace_size.restype = ctypes.c_size_t
+    L.ssd_seqpar_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int]
+    L.ssd_seqpar_local.restype = ctypes.c_int
+    L.ssd_seqpar_local.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, ctypes.c_int, _vp,
+                                   _vp, _vp, ctypes.c_size_t, _vp]
+    L.ssd_seqpar_finish.restype = ctypes.c_int
+    L.ssd_seqpar_finish.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, ctypes.c_int, _vp,
+                                    _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp,
+                                    ctypes.c_size_t, _vp]
     L.ssd_chunk_scan_varlen_workspace_size.restype = ctypes.c_size_t
     L.ssd_chunk_scan_varlen_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int,
                                                        ctypes.c_int]
@@ -255,6 +264,75 @@ def chunk_scan_varlen_fwd(x, dt, A, B, C, D, cu_seqlens, chunk_size: int = 256,
         _ptr(cu_seqlens), nseq, _ptr(init_states), _ptr(y), _ptr(final_states), _ptr(workspace),
         workspace.numel(), _stream_handle(stream)))
     return y, final_states
+
+
+# ---------------------------------------------------------------- sequence parallelism
+def seqpar_local(x, dt, A, B, chunk_size: int = 256, workspace=None, stream=None):
+    """Phase 1 on this rank's segment: (h_loc (b, H, P, N) f32, log_decay (b, H) f32,
+    workspace to pass on to seqpar_finish)."""
+    torch = _torch()
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = x.device
+    shape = make_shape(b, L, H, P, N, G, _dtype_code(x))
+    if workspace is None:
+        n = lib().ssd_seqpar_workspace_size(ctypes.byref(shape), chunk_size)
+        if n == 0:
+            raise SSDError(SSD_ERR_INVALID_ARG, last_error())
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    h_loc = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    log_decay = torch.empty((b, H), dtype=torch.float32, device=dev)
+    _check(lib().ssd_seqpar_local(ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                                  chunk_size, _ptr(h_loc), _ptr(log_decay), _ptr(workspace),
+                                  workspace.numel(), _stream_handle(stream)))
+    return h_loc, log_decay, workspace
+
+
+def seqpar_finish(x, B, C, D, workspace, h_loc_all, log_decay_all, rank: int,
+                  chunk_size: int = 256, init_state=None, y=None, final_state=None,
+                  return_final_state: bool = True, stream=None):
+    """Phase 3 on this rank's segment, after the exchange: (y, final_state or None)."""
+    torch = _torch()
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = x.device
+    shape = make_shape(b, L, H, P, N, G, _dtype_code(x))
+    nranks = h_loc_all.shape[0]
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    _check(lib().ssd_seqpar_finish(ctypes.byref(shape), _ptr(x), _ptr(B), _ptr(C), _ptr(D),
+                                   chunk_size, _ptr(h_loc_all), _ptr(log_decay_all), nranks,
+                                   rank, _ptr(init_state), _ptr(y), _ptr(final_state),
+                                   _ptr(workspace), workspace.numel(), _stream_handle(stream)))
+    return y, final_state
+
+
+def exchange_states(h_loc, log_decay, group=None):
+    """The one exchange of the sequence-parallel scan: every rank's local final state and
+    segment log-decay, gathered in rank order (torch.distributed all_gather; NCCL over NVLink on
+    GPUs, gloo on CPU).  Returns (h_loc_all [nranks, ...], log_decay_all [nranks, ...])."""
+    torch = _torch()
+    import torch.distributed as dist
+    n = dist.get_world_size(group)
+    hs = [torch.empty_like(h_loc) for _ in range(n)]
+    ls = [torch.empty_like(log_decay) for _ in range(n)]
+    dist.all_gather(hs, h_loc.contiguous(), group=group)
+    dist.all_gather(ls, log_decay.contiguous(), group=group)
+    return torch.stack(hs), torch.stack(ls)
+
+
+def seqpar_scan(x, dt, A, B, C, D, chunk_size: int = 256, init_state=None, group=None,
+                stream=None):
+    """Sequence-parallel scan of this rank's contiguous segment (ranks hold the segments in
+    order): local phase, one all-gather of states, finish.  Returns (y, final_state); the final
+    state of the whole sequence is the last rank's."""
+    import torch.distributed as dist
+    h_loc, log_decay, ws = seqpar_local(x, dt, A, B, chunk_size, stream=stream)
+    h_all, l_all = exchange_states(h_loc, log_decay, group)
+    return seqpar_finish(x, B, C, D, ws, h_all, l_all, dist.get_rank(group), chunk_size,
+                         init_state=init_state, stream=stream)
 
 
 def state_update(state, x, dt, A, B, C, D, y=None, stream=None):

@@ -170,3 +170,15 @@ def test_fused_options_workspace_and_validation(L):
     rc = L.ssd_chunk_scan_fwd_ex(ctypes.byref(sh), p, p, p, p, p, p, 256, None, p, None, p,
                                  1 << 40, None, ctypes.byref(inv))
     assert rc == ssd.SSD_ERR_INVALID_ARG and "dt_min" in ssd.last_error()
+
+
+def test_seqpar_workspace_and_rejections(L):
+    sh = _shape()
+    assert ssd.lib().ssd_seqpar_workspace_size(ctypes.byref(sh), 256) == \
+        ssd.workspace_size(sh, 256) + 4 * 80 * 64 * 128 * 4
+    f32 = _shape(dtype=ssd.SSD_F32)
+    assert L.ssd_seqpar_workspace_size(ctypes.byref(f32), 256) == 0   # tensor-core path only
+    p = ctypes.c_void_p(1 << 20)
+    rc = L.ssd_seqpar_finish(ctypes.byref(sh), p, p, p, p, 256, p, p, 2, 2, None, p, None, p,
+                             1 << 40, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "rank" in ssd.last_error()
