@@ -523,7 +523,10 @@ chunk_state_pass_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
 // So y = Y_diag + f_t Y_A with f_t = exp(cs_t) (T = 0) or u_t (T = 1).
 constexpr int kXStagesMax = 3;   // x / h_in stages (T = 0: 3, the third in the B tile's space;
                                  // T = 1: 2, that space holds the bf16 off-diagonal block)
-constexpr int kScanMaxHeads = 8; // heads per CTA
+constexpr int kScanHeadsMin = 8;  // heads per CTA: chosen per launch in [8, 20] (fewer when a
+constexpr int kScanHeadsMax = 20; // group has fewer), see scan_heads_per_cta
+constexpr int kScanVecStages = 4; // cs / dt row stages (one head each)
+static_assert(kScanHeadsMax <= kMaxHeadsPerCta, "D of every head of a CTA is staged in smem");
 constexpr int kRing = 4;         // 64-column blocks of P in TMEM (two heads)
 constexpr int kStageBytes = 256 * kRowBytes + 2 * kP * kRowBytes;  // x (<= 256 rows) + h_in
 constexpr int kHOff = 256 * kRowBytes;                              // h_in inside a stage
@@ -534,13 +537,13 @@ struct alignas(1024) ScanSmem {
                                     // (K-major [i atom][128 rows t][64 i])
     uint8_t S01[2][kStageBytes];    // x / h_in stages 0 and 1: [KI rows i][64 p] then
                                     // [n atom][64 rows p][64 n]
-    float cs_v[kScanMaxHeads * 256];  // the CTA's heads' chunk-local cumsum rows (stride Q)
-    float dt_v[kScanMaxHeads * 256];  // and dt rows (0 past the end), loaded once
+    float cs_v[kScanVecStages][256];  // per stage: one head's chunk-local cumsum row
+    float dt_v[kScanVecStages][256];  // per stage: its dt row (0 past the end)
     float vt[16][32];               // per worker warp: column factors of its two slices
     float Dv[kMaxHeadsPerCta];      // D of the CTA's heads
     uint64_t bar_cb, bar_g, bar_goff;
     uint64_t bar_xh_full[kXStagesMax], bar_xh_free[kXStagesMax], bar_xv_ready[kXStagesMax];
-    uint64_t bar_vec;
+    uint64_t bar_vec_full[kScanVecStages], bar_vec_free[kScanVecStages];
     uint64_t bar_slot_full[kRing], bar_slot_free[kRing];
     uint64_t bar_acc_full[2], bar_acc_free[2];
     uint64_t bar_drain;
@@ -634,7 +637,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_init(&sm.bar_xh_free[s], 1);
             mbar_init(&sm.bar_xv_ready[s], kScanWorkers);
         }
-        mbar_init(&sm.bar_vec, 1);
+        for (int s = 0; s < kScanVecStages; ++s) {
+            mbar_init(&sm.bar_vec_full[s], 1);
+            mbar_init(&sm.bar_vec_free[s], kScanWorkers);
+        }
         for (int s = 0; s < kRing; ++s) {
             mbar_init(&sm.bar_slot_full[s], kScanWorkers);
             mbar_init(&sm.bar_slot_free[s], 1);
@@ -673,14 +679,17 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 for (int r = 0; r <= T; ++r)
                     tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
                                 64 * a, g, (int)(t0 + kTileRows * r), (int)b);
-            // cs and dt rows of all the CTA's heads (contiguous in the workspace): two copies
-            const int64_t vrow = ((b * nchunks + k) * H + h0) * (int64_t)Q;
-            mbar_arrive_expect_tx(&sm.bar_vec, (uint32_t)(8 * Q * nh));
-            bulk_load(sm.cs_v, cs + vrow, (uint32_t)(4 * Q * nh), &sm.bar_vec);
-            bulk_load(sm.dt_v, dtc + vrow, (uint32_t)(4 * Q * nh), &sm.bar_vec);
         }
         for (int j = 0; lane == 0 && j < nh; ++j) {   // lane 0 alone runs the loop
             const int h = h0 + j;
+            const int vs = j % kScanVecStages;
+            const uint32_t vu = j / kScanVecStages;
+            if (j >= kScanVecStages && !mbar_wait(&sm.bar_vec_free[vs], (vu - 1) & 1, abort))
+                break;
+            const int64_t vrow = ((b * nchunks + k) * H + h) * (int64_t)Q;
+            mbar_arrive_expect_tx(&sm.bar_vec_full[vs], (uint32_t)(8 * Q));
+            bulk_load(sm.cs_v[vs], cs + vrow, Q * 4, &sm.bar_vec_full[vs]);
+            bulk_load(sm.dt_v[vs], dtc + vrow, Q * 4, &sm.bar_vec_full[vs]);
             const int xs = j % nst;
             const uint32_t xu = j / nst;
             if (j >= nst && !mbar_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) break;
@@ -783,7 +792,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         const int u0 = cq, u1 = 4 + cq;
         const int cls0 = u0 < 2 * qd ? 0 : (u0 <= 2 * qd + 1 ? 1 : 2);
         const int cls1 = u1 < 2 * qd ? 0 : (u1 <= 2 * qd + 1 ? 1 : 2);
-        bool ok = warp_wait(&sm.bar_g, 0, abort) && warp_wait(&sm.bar_vec, 0, abort);
+        bool ok = warp_wait(&sm.bar_g, 0, abort);
         tc_fence_after();
         // this warp's part of the diagonal block of C B^T, kept in registers for every head
         uint32_t g0[16], g1[16];
@@ -820,8 +829,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         uint32_t blk = 0;
         for (int j = 0; ok && j <= nh; ++j) {
             if (j < nh) {
-                const float *cs_s = sm.cs_v + j * Q;
-                const float *dt_s = sm.dt_v + j * Q;
+                const int vs = j % kScanVecStages;
+                if (!warp_wait(&sm.bar_vec_full[vs], (j / kScanVecStages) & 1, abort)) break;
+                const float *cs_s = sm.cs_v[vs];
+                const float *dt_s = sm.dt_v[vs];
                 if (T) {
                     // x rows [0, 128) *= exp(cs_127 - cs_i) dt_i; h_in *= exp(cs_127)
                     const int xs = j % nst;
@@ -924,11 +935,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 uint32_t d0[16], a0[16];
                 tmem_ld16(col, d0);
                 tmem_ld16(col + 64, a0);
-                const float *cs_j = sm.cs_v + jj * Q;
+                const int vs = jj % kScanVecStages;
+                const float *cs_j = sm.cs_v[vs];
                 const float f = __expf(cs_j[tau] - (T ? cs_j[127] : 0.f));
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&sm.bar_acc_free[a]);
+                mbar_arrive(&sm.bar_vec_free[vs]);   // done with this head's cs / dt
                 const int64_t yoff = ((b * seqlen + t0 + tau) * H + h0 + jj) * (int64_t)kP + 16 * cq;
                 // gated output (z given): y * z * sigmoid(z); z kept as 8 packed bf16 pairs
                 const bool gz = kGate && tau < len;
@@ -1020,6 +1033,24 @@ bool make_seq_map(CUtensorMap *m, const void *ptr, int64_t batch, int64_t seqlen
                                    (cuuint64_t)(seqlen * mid * inner * 2)};
     const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     return make_map(m, ptr, 4, dims, strides, box);
+}
+
+// Heads per chunk-scan CTA.  Each CTA pays a ramp (C and B tiles, C B^T, the first loads) that
+// more heads amortise, but the two 128-row tiles of a chunk differ in cost and a CTA walks its
+// heads in sequence, so too few CTAs leave the last wave ragged.  Aim at about 3.5 waves of CTAs
+// over the SMs, within [kScanHeadsMin, kScanHeadsMax], then balance the head blocks (measured at
+// b=4, L=4096, H=80: 8 heads 207 us, 14 heads 195 us, 20 heads 195 us, 40 heads 210 us).
+int scan_heads_per_cta(int64_t tiles, int hpg)
+{
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const double target_ctas = 3.5 * sms;
+    int hpc = (int)std::ceil((double)hpg * (double)tiles / target_ctas);
+    hpc = std::max(kScanHeadsMin, std::min(kScanHeadsMax, hpc));
+    hpc = std::min(hpc, hpg);
+    const int nhb = (hpg + hpc - 1) / hpc;
+    return (hpg + nhb - 1) / nhb;   // the same number of head blocks, evenly filled
 }
 
 // Heads per CTA.  Every CTA pays a fixed ramp-up (its B / C tiles, C B^T, the first TMA round
@@ -1133,7 +1164,7 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     const int hpg = H / G;
     // The scan's per-head cost (mask, three MMA chains, epilogue) dominates its per-CTA ramp, and
     // its two tiles differ in cost, so many small CTAs balance better than one CTA per group.
-    const int hpc = std::min(hpg, kScanMaxHeads);
+    const int hpc = scan_heads_per_cta(batch * nchunks * G * (Q / kTileRows), hpg);
     const int nhb = (hpg + hpc - 1) / hpc;
     const size_t smem = sizeof(ScanSmem) + 1024;
     auto kern = z ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
