@@ -237,6 +237,16 @@ ssd_status ssd_state_update(const ssd_shape *shape, float *state, const void *x,
                             const float *D, void *y, void *stream);
 
 /*
+ * ssd_state_update with the block's fused steps of `options` (nullable; see ssd_fwd_options):
+ * z (batch, nheads, headdim) gates the output, y * z * sigmoid(z); dt_bias, dt_softplus and the
+ * clamp turn the raw dt projection into the step used, as for ssd_chunk_scan_fwd_ex.
+ */
+ssd_status ssd_state_update_ex(const ssd_shape *shape, float *state, const void *x,
+                               const float *dt, const float *A, const void *B, const void *C,
+                               const float *D, void *y, void *stream,
+                               const ssd_fwd_options *options);
+
+/*
  * Synchronises `stream` and reads the device status word the last ssd_chunk_scan_fwd (or
  * ssd_chunk_scan_varlen_fwd) call on this workspace left behind: SSD_OK; SSD_ERR_TIMEOUT when
  * an in-kernel wait on a shared-memory barrier exceeded its bound and the kernel returned early

@@ -18,6 +18,17 @@ template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __f
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// The dt the recurrence uses when the block's raw projection is passed: + bias, then softplus
+// log(1 + exp(v)) (equal to v in float32 for v > 20), then the clamp to [lo, hi]; each optional.
+__device__ __forceinline__ float dt_transform(float v, const float *bias, int h, bool softplus,
+                                              bool clamp, float lo, float hi)
+{
+    if (bias) v += bias[h];
+    if (softplus) v = v > 20.f ? v : log1pf(__expf(v));
+    if (clamp) v = fminf(fmaxf(v, lo), hi);
+    return v;
+}
+
 // The SiLU gate z * sigmoid(z) of the block's output.  Fast exponential and division (about
 // 2 ulp; the gated output is stored in bf16 or compared at 1e-4): for z -> -inf the divisor
 // overflows to inf and the result is -0, the limit.
@@ -103,10 +114,18 @@ cudaError_t launch_dt_prologue(const float *dt, const float *bias, float *dt_out
                                int H, bool softplus, bool clamp, float lo, float hi,
                                cudaStream_t st);
 
+// Options of the decode update (all nullable / off): the gate z (x's type and layout) and the
+// dt prologue, as for the fused scan.
+struct DecodeOptions {
+    const void *z = nullptr;
+    const float *dt_bias = nullptr;
+    bool softplus = false, clamp = false;
+    float lo = 0.f, hi = 0.f;
+};
 cudaError_t launch_state_update(bool is_bf16, float *state, const void *x, const float *dt,
                                 const float *A, const void *B, const void *C, const float *D,
                                 void *y, int64_t batch, int H, int G, int P, int N,
-                                cudaStream_t st);
+                                cudaStream_t st, const DecodeOptions &opt = DecodeOptions());
 
 cudaError_t launch_fill_final(const float *init, float *final_state, int64_t n,
                               cudaStream_t st);

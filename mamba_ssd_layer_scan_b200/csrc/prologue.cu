@@ -16,12 +16,7 @@ __global__ void dt_prologue_kernel(const float *__restrict__ dt, const float *__
 {
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= n) return;
-    float v = dt[i];
-    if (bias) v += bias[i % H];
-    // softplus(v) = log(1 + exp(v)); for v > 20 it equals v to float32 precision
-    if (softplus) v = v > 20.f ? v : log1pf(__expf(v));
-    if (clamp) v = fminf(fmaxf(v, lo), hi);
-    out[i] = v;
+    out[i] = dt_transform(dt[i], bias, (int)(i % H), softplus, clamp, lo, hi);
 }
 
 }  // namespace

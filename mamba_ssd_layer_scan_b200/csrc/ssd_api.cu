@@ -544,9 +544,10 @@ ssd_status ssd_seqpar_finish(const ssd_shape *shape, const void *x, const void *
     return SSD_OK;
 }
 
-ssd_status ssd_state_update(const ssd_shape *shape, float *state, const void *x,
-                            const float *dt, const float *A, const void *B, const void *C,
-                            const float *D, void *y, void *stream)
+ssd_status ssd_state_update_ex(const ssd_shape *shape, float *state, const void *x,
+                               const float *dt, const float *A, const void *B, const void *C,
+                               const float *D, void *y, void *stream,
+                               const ssd_fwd_options *options)
 {
     ssd_status st = check_shape(shape, false);
     if (st != SSD_OK) return st;
@@ -556,12 +557,30 @@ ssd_status ssd_state_update(const ssd_shape *shape, float *state, const void *x,
         return fail(SSD_ERR_INVALID_ARG, "state, x, dt, A, B, C, D and y must be non-NULL");
     if (!aligned16(state) || !aligned16(B) || !aligned16(C))
         return fail(SSD_ERR_INVALID_ARG, "state, B and C must be 16-byte aligned");
+    ssd::DecodeOptions opt;
+    if (options) {
+        if (options->dt_max > 0.f && !(options->dt_min <= options->dt_max))
+            return fail(SSD_ERR_INVALID_ARG, "dt_min must not exceed dt_max");
+        opt.z = options->z;
+        opt.dt_bias = options->dt_bias;
+        opt.softplus = options->dt_softplus != 0;
+        opt.clamp = options->dt_max > 0.f;
+        opt.lo = options->dt_min;
+        opt.hi = options->dt_max;
+    }
     cudaError_t e = ssd::launch_state_update(s.dtype == SSD_BF16, state, x, dt, A, B, C, D, y,
                                              s.batch, (int)s.nheads, (int)s.ngroups,
                                              (int)s.headdim, (int)s.dstate,
-                                             static_cast<cudaStream_t>(stream));
+                                             static_cast<cudaStream_t>(stream), opt);
     if (e != cudaSuccess) return cuda_fail(e, "state update launch");
     return SSD_OK;
+}
+
+ssd_status ssd_state_update(const ssd_shape *shape, float *state, const void *x,
+                            const float *dt, const float *A, const void *B, const void *C,
+                            const float *D, void *y, void *stream)
+{
+    return ssd_state_update_ex(shape, state, x, dt, A, B, C, D, y, stream, nullptr);
 }
 
 ssd_status ssd_workspace_status(const void *workspace, size_t workspace_bytes, void *stream)

@@ -56,12 +56,14 @@ template <> struct Vec<8> {
 };
 
 // grid.x = ceil(P / kRowsPerCta) * H * batch
-template <typename T, int V>
+template <typename T, int V, bool kOpts>   // kOpts: gate and dt prologue (else plain)
 __global__ void __launch_bounds__(kWarps * 32)
 state_update_kernel(float *__restrict__ state, const T *__restrict__ x,
                     const float *__restrict__ dt, const float *__restrict__ A,
                     const T *__restrict__ B, const T *__restrict__ C,
-                    const float *__restrict__ D, T *__restrict__ y, int H, int G, int P)
+                    const float *__restrict__ D, T *__restrict__ y, int H, int G, int P,
+                    const T *__restrict__ z, const float *__restrict__ dt_bias, bool softplus,
+                    bool clamp, float lo, float hi)
 {
     constexpr int N = 32 * V;
     const int pblocks = (P + kRowsPerCta - 1) / kRowsPerCta;
@@ -74,7 +76,8 @@ state_update_kernel(float *__restrict__ state, const T *__restrict__ x,
     const int p_end = min(P, p_begin + kRowsPerWarp);
     if (p_begin >= p_end) return;
 
-    const float dth = dt[b * H + h];
+    const float dth = kOpts ? dt_transform(dt[b * H + h], dt_bias, h, softplus, clamp, lo, hi)
+                            : dt[b * H + h];
     const float a = __expf(dth * A[h]);
     const float Dh = D[h];
     float bv[V], cv[V];
@@ -86,6 +89,7 @@ state_update_kernel(float *__restrict__ state, const T *__restrict__ x,
     float *srow = state + ((b * H + h) * (int64_t)P) * N + lane * V;
     const T *xrow = x + (b * H + h) * (int64_t)P;
     T *yrow = y + (b * H + h) * (int64_t)P;
+    const T *zrow = (kOpts && z) ? z + (b * H + h) * (int64_t)P : nullptr;
 
     for (int p0 = p_begin; p0 < p_end; p0 += kRowsInFlight) {
         float s[kRowsInFlight][V];
@@ -110,7 +114,11 @@ state_update_kernel(float *__restrict__ state, const T *__restrict__ x,
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-            if (lane == 0 && p0 + r < p_end) yrow[p0 + r] = from_f32<T>(fmaf(Dh, xv[r], dot));
+            if (lane == 0 && p0 + r < p_end) {
+                const float out = fmaf(Dh, xv[r], dot);
+                yrow[p0 + r] =
+                    from_f32<T>(kOpts && zrow ? out * silu(to_f32(zrow[p0 + r])) : out);
+            }
         }
     }
 }
@@ -118,18 +126,28 @@ state_update_kernel(float *__restrict__ state, const T *__restrict__ x,
 template <typename T>
 cudaError_t launch_typed(float *state, const void *x, const float *dt, const float *A,
                          const void *B, const void *C, const float *D, void *y, int64_t batch,
-                         int H, int G, int P, int N, cudaStream_t st)
+                         int H, int G, int P, int N, cudaStream_t st, const DecodeOptions &o)
 {
+    const T *zp = (const T *)o.z;
     const unsigned grid = (unsigned)(((P + kRowsPerCta - 1) / kRowsPerCta) * H * batch);
     const T *xp = (const T *)x, *Bp = (const T *)B, *Cp = (const T *)C;
     T *yp = (T *)y;
+    const bool opts = o.z || o.dt_bias || o.softplus || o.clamp;
+#define SSD_DECODE_LAUNCH(VV)                                                                   \
+    (opts ? state_update_kernel<T, VV, true><<<grid, kWarps * 32, 0, st>>>(                      \
+                state, xp, dt, A, Bp, Cp, D, yp, H, G, P, zp, o.dt_bias, o.softplus, o.clamp,     \
+                o.lo, o.hi)                                                                     \
+          : state_update_kernel<T, VV, false><<<grid, kWarps * 32, 0, st>>>(                     \
+                state, xp, dt, A, Bp, Cp, D, yp, H, G, P, nullptr, nullptr, false, false, 0.f,   \
+                0.f))
     switch (N) {
-    case 32: state_update_kernel<T, 1><<<grid, kWarps * 32, 0, st>>>(state, xp, dt, A, Bp, Cp, D, yp, H, G, P); break;
-    case 64: state_update_kernel<T, 2><<<grid, kWarps * 32, 0, st>>>(state, xp, dt, A, Bp, Cp, D, yp, H, G, P); break;
-    case 128: state_update_kernel<T, 4><<<grid, kWarps * 32, 0, st>>>(state, xp, dt, A, Bp, Cp, D, yp, H, G, P); break;
-    case 256: state_update_kernel<T, 8><<<grid, kWarps * 32, 0, st>>>(state, xp, dt, A, Bp, Cp, D, yp, H, G, P); break;
+    case 32: SSD_DECODE_LAUNCH(1); break;
+    case 64: SSD_DECODE_LAUNCH(2); break;
+    case 128: SSD_DECODE_LAUNCH(4); break;
+    case 256: SSD_DECODE_LAUNCH(8); break;
     default: return cudaErrorInvalidValue;
     }
+#undef SSD_DECODE_LAUNCH
     return cudaGetLastError();
 }
 
@@ -138,10 +156,11 @@ cudaError_t launch_typed(float *state, const void *x, const float *dt, const flo
 cudaError_t launch_state_update(bool is_bf16, float *state, const void *x, const float *dt,
                                 const float *A, const void *B, const void *C, const float *D,
                                 void *y, int64_t batch, int H, int G, int P, int N,
-                                cudaStream_t st)
+                                cudaStream_t st, const DecodeOptions &opt)
 {
-    if (is_bf16) return launch_typed<bf16>(state, x, dt, A, B, C, D, y, batch, H, G, P, N, st);
-    return launch_typed<float>(state, x, dt, A, B, C, D, y, batch, H, G, P, N, st);
+    if (is_bf16)
+        return launch_typed<bf16>(state, x, dt, A, B, C, D, y, batch, H, G, P, N, st, opt);
+    return launch_typed<float>(state, x, dt, A, B, C, D, y, batch, H, G, P, N, st, opt);
 }
 
 }  // namespace ssd

@@ -95,6 +95,8 @@ def lib():
     L.ssd_state_update.restype = ctypes.c_int
     L.ssd_state_update.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _vp]
+    L.ssd_state_update_ex.restype = ctypes.c_int
+    L.ssd_state_update_ex.argtypes = L.ssd_state_update.argtypes + [ctypes.POINTER(FwdOptions)]
     L.ssd_workspace_status.restype = ctypes.c_int
     L.ssd_workspace_status.argtypes = [_vp, ctypes.c_size_t, _vp]
     L.ssd_last_error.restype = ctypes.c_char_p
@@ -335,9 +337,11 @@ def seqpar_scan(x, dt, A, B, C, D, chunk_size: int = 256, init_state=None, group
                          init_state=init_state, stream=stream)
 
 
-def state_update(state, x, dt, A, B, C, D, y=None, stream=None):
+def state_update(state, x, dt, A, B, C, D, y=None, stream=None, z=None, dt_bias=None,
+                 dt_softplus: bool = False, dt_limit=None):
     """One decode step.  state (b, H, P, N) f32 (in place), x (b, H, P), dt (b, H) f32,
-    B/C (b, G, N).  Returns y (b, H, P)."""
+    B/C (b, G, N).  Returns y (b, H, P).  z, dt_bias, dt_softplus, dt_limit: the block's fused
+    steps (ssd_state_update_ex)."""
     torch = _torch()
     b, H, P = x.shape
     G, N = B.shape[1], B.shape[2]
@@ -350,8 +354,16 @@ def state_update(state, x, dt, A, B, C, D, y=None, stream=None):
     shape = make_shape(b, 1, H, P, N, G, code)
     if y is None:
         y = torch.empty_like(x)
-    _check(lib().ssd_state_update(ctypes.byref(shape), _ptr(state), _ptr(x), _ptr(dt), _ptr(A),
-                                  _ptr(B), _ptr(C), _ptr(D), _ptr(y), _stream_handle(stream)))
+    args = (ctypes.byref(shape), _ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+            _ptr(D), _ptr(y), _stream_handle(stream))
+    if z is None and dt_bias is None and not dt_softplus and dt_limit is None:
+        _check(lib().ssd_state_update(*args))
+    else:
+        if z is not None:
+            _require(z, "z", x.dtype, dev)
+        lo, hi = dt_limit if dt_limit is not None else (0.0, 0.0)
+        opts = FwdOptions(_ptr(z), _ptr(dt_bias), 1 if dt_softplus else 0, lo, hi)
+        _check(lib().ssd_state_update_ex(*args, ctypes.byref(opts)))
     return y
 
 

@@ -148,6 +148,18 @@ def ssd_scan_block(x, dt, A, B, C, D, init=None, z=None, dt_bias=None, softplus:
     return y, final
 
 
+def ssd_state_update_block(state, x, dt, A, B, C, D, z=None, dt_bias=None,
+                           softplus: bool = False, dt_limit=None):
+    """One decode step with the block's steps around it: the dt prologue, the recurrence over the
+    token, the SiLU(z) gate.  x, z (b, H, P), dt (b, H).  Returns (y, new_state)."""
+    dt_eff = dt_prologue(dt, dt_bias, softplus, dt_limit)
+    y, new_state = ssd_state_update(state, x, dt_eff, A, B, C, D)
+    if z is not None:
+        zf = np.asarray(z, dtype=np.float64)
+        y = y * (zf / (1.0 + np.exp(-zf)))
+    return y, new_state
+
+
 def ssd_scan_varlen(x, dt, A, B, C, D, cu_seqlens, init=None):
     """Packed variable-length sequences: sequence s (tokens cu_seqlens[s] .. cu_seqlens[s+1]-1
     of the single batch row) is its own recurrence, started from init[s] (or zeros), so this is

@@ -116,3 +116,39 @@ def test_plain_options_equal_plain_scan(cuda_device):
     assert rc == ssd.SSD_OK, ssd.last_error()
     torch.cuda.synchronize()
     assert torch.equal(y0, y1) and torch.equal(f0, f1)
+
+
+def test_decode_with_block_options(cuda_device):
+    """Gated decode steps with the dt prologue against the oracle, over 6 steps."""
+    import torch
+    rng = np.random.default_rng(77)
+    b, H, P, N, G = 8, 8, 64, 128, 2
+    state0 = (0.1 * rng.standard_normal((b, H, P, N))).astype(np.float32)
+    A = (-np.exp(rng.uniform(0.0, np.log(16.0), H))).astype(np.float32)
+    D = rng.standard_normal(H).astype(np.float32)
+    bias = (-4.0 + rng.uniform(-0.5, 0.5, H)).astype(np.float32)
+    dev = cuda_device
+    st = torch.from_numpy(state0).to(dev)
+    ref_state = state0.astype(np.float64)
+    errs = []
+    for step in range(6):
+        x = inputs.round_bf16(rng.standard_normal((b, H, P)).astype(np.float32))
+        z = inputs.round_bf16(rng.standard_normal((b, H, P)).astype(np.float32))
+        raw = rng.standard_normal((b, H)).astype(np.float32)
+        Bv = inputs.round_bf16((rng.standard_normal((b, G, N)) / np.sqrt(N)).astype(np.float32))
+        Cv = inputs.round_bf16((rng.standard_normal((b, G, N)) / np.sqrt(N)).astype(np.float32))
+        tt = lambda a, d=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(d)
+        y = ssd.state_update(st, tt(x, torch.bfloat16), tt(raw), tt(A), tt(Bv, torch.bfloat16),
+                             tt(Cv, torch.bfloat16), tt(D), z=tt(z, torch.bfloat16),
+                             dt_bias=tt(bias), dt_softplus=True, dt_limit=(1e-3, 0.1))
+        y_ref, ref_state = oracle.ssd_state_update_block(ref_state, x, raw, A, Bv, Cv, D, z=z,
+                                                         dt_bias=bias, softplus=True,
+                                                         dt_limit=(1e-3, 0.1))
+        torch.cuda.synchronize()
+        yn = to_np(y)
+        errs.append(max_rel_per_pair([yn[i, h] for i in range(b) for h in range(H)],
+                                     [y_ref[i, h] for i in range(b) for h in range(H)]))
+    sn = to_np(st)
+    es = max_rel_per_pair([sn[i, h] for i in range(b) for h in range(H)],
+                          [ref_state[i, h] for i in range(b) for h in range(H)])
+    assert max(errs) <= TOL["bf16"] and es <= 1e-5

@@ -386,3 +386,22 @@ def test_block_input_recipe():
     again = inputs.make_inputs(w)
     assert np.array_equal(base.x, again.x)
     assert blk.z.shape == base.x.shape and np.array_equal(inputs.round_bf16(blk.z), blk.z)
+
+
+def test_block_decode_steps_equal_block_scan():
+    """The gated decode step with the dt prologue, repeated over a sequence, is the gated scan
+    with the same prologue (both are the recurrence with the same per-token dt and gate)."""
+    x, dt, A, B, C, D, h0 = _rand_case(11, b=2, L=12)
+    rng = np.random.default_rng(12)
+    z = rng.standard_normal(x.shape)
+    raw = rng.standard_normal(dt.shape)
+    bias = -rng.uniform(0.5, 1.5, A.shape[0])
+    y_ref, f_ref = oracle.ssd_scan_block(x, raw, A, B, C, D, h0, z=z, dt_bias=bias,
+                                         softplus=True, dt_limit=(0.05, 0.4))
+    state = h0.copy()
+    for t in range(x.shape[1]):
+        y_t, state = oracle.ssd_state_update_block(state, x[:, t], raw[:, t], A, B[:, t],
+                                                   C[:, t], D, z=z[:, t], dt_bias=bias,
+                                                   softplus=True, dt_limit=(0.05, 0.4))
+        assert _rel(y_t, y_ref[:, t]) < 1e-12
+    assert _rel(state, f_ref) < 1e-12
