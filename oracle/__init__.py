@@ -160,6 +160,50 @@ def ssd_state_update_block(state, x, dt, A, B, C, D, z=None, dt_bias=None,
     return y, new_state
 
 
+def ssd_scan_bwd(x, dt, A, B, C, D, dy, init=None, dfinal=None):
+    """Gradients of L = sum_t <dy_t, y_t> + <dfinal, final_state> through the recurrence, by the
+    adjoint recurrence (reverse-mode differentiation of the token loop, float64):
+
+        g_t = dy_t (outer) C_t + a_{t+1} g_{t+1}           (g_{L-1} also gets dfinal)
+        dx_t = D_h dy_t + dt_t g_t B_t                      dB_t += dt_t g_t^T x_t  (per group)
+        dC_t += h_t^T dy_t  (per group)                     dD_h = sum_t <dy_t, x_t>
+        dl_t = a_t <g_t, h_{t-1}>   (l_t = dt_t A_h)        ddt_t = <g_t B_t, x_t> + A_h dl_t
+        dA_h = sum_t dt_t dl_t                              dinit = a_0 g_0
+
+    x (b, L, H, P), dt (b, L, H), B/C (b, L, G, N), dy like x, init/dfinal (b, H, P, N) or None.
+    Returns dict dx, ddt, dA, dB, dC, dD, dinit.  The forward states are kept per (b, h), so this
+    is for oracle-sized inputs."""
+    x, dt, A, B, C, D, dy = (np.asarray(v, dtype=np.float64) for v in (x, dt, A, B, C, D, dy))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    out = dict(dx=np.zeros_like(x), ddt=np.zeros_like(dt), dA=np.zeros(H), dB=np.zeros_like(B),
+               dC=np.zeros_like(C), dD=np.zeros(H), dinit=np.zeros((b, H, P, N)))
+    for bi in range(b):
+        for h in range(H):
+            g_ = h // (H // G)
+            a = np.exp(dt[bi, :, h] * A[h])
+            hs = np.zeros((L + 1, P, N))                     # hs[t + 1] = state after token t
+            if init is not None:
+                hs[0] = init[bi, h]
+            for t in range(L):
+                hs[t + 1] = a[t] * hs[t] + dt[bi, t, h] * np.outer(x[bi, t, h], B[bi, t, g_])
+                out["dC"][bi, t, g_] += hs[t + 1].T @ dy[bi, t, h]
+            gnext = np.zeros((P, N)) if dfinal is None else np.asarray(dfinal[bi, h], np.float64)
+            anext = 1.0
+            for t in range(L - 1, -1, -1):
+                g = np.outer(dy[bi, t, h], C[bi, t, g_]) + anext * gnext
+                gB = g @ B[bi, t, g_]
+                out["dx"][bi, t, h] = D[h] * dy[bi, t, h] + dt[bi, t, h] * gB
+                out["dB"][bi, t, g_] += dt[bi, t, h] * (g.T @ x[bi, t, h])
+                dl = a[t] * np.sum(g * hs[t])
+                out["ddt"][bi, t, h] = gB @ x[bi, t, h] + A[h] * dl
+                out["dA"][h] += dt[bi, t, h] * dl
+                out["dD"][h] += dy[bi, t, h] @ x[bi, t, h]
+                gnext, anext = g, a[t]
+            out["dinit"][bi, h] = anext * gnext
+    return out
+
+
 def ssd_scan_varlen(x, dt, A, B, C, D, cu_seqlens, init=None):
     """Packed variable-length sequences: sequence s (tokens cu_seqlens[s] .. cu_seqlens[s+1]-1
     of the single batch row) is its own recurrence, started from init[s] (or zeros), so this is

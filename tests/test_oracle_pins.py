@@ -405,3 +405,50 @@ def test_block_decode_steps_equal_block_scan():
                                                    softplus=True, dt_limit=(0.05, 0.4))
         assert _rel(y_t, y_ref[:, t]) < 1e-12
     assert _rel(state, f_ref) < 1e-12
+
+
+# ------------------------------------------------------------------ backward
+def _loss(x, dt, A, B, C, D, h0, dy, dfin):
+    y, f, _ = oracle.ssd_scan(x, dt, A, B, C, D, h0)
+    return float(np.sum(dy * y) + np.sum(dfin * f))
+
+
+@pytest.mark.parametrize("seed", [21, 22])
+def test_backward_equals_finite_differences(seed):
+    """Every gradient of the adjoint oracle against central differences of the (pinned) forward
+    oracle, element by element, on a tiny input with two groups and an initial state."""
+    x, dt, A, B, C, D, h0 = _rand_case(seed, b=1, L=7, H=4, G=2, P=2, N=3)
+    rng = np.random.default_rng(seed + 1)
+    dy = rng.standard_normal(x.shape)
+    dfin = rng.standard_normal(h0.shape)
+    g = oracle.ssd_scan_bwd(x, dt, A, B, C, D, dy, h0, dfin)
+    args = dict(x=x, dt=dt, A=A, B=B, C=C, D=D, init=h0)
+    key = dict(x="dx", dt="ddt", A="dA", B="dB", C="dC", D="dD", init="dinit")
+    eps = 1e-6
+    for name, arr in args.items():
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            saved = arr[idx]
+            arr[idx] = saved + eps
+            lp = _loss(*(args[k] for k in ("x", "dt", "A", "B", "C", "D", "init")), dy, dfin)
+            arr[idx] = saved - eps
+            lm = _loss(*(args[k] for k in ("x", "dt", "A", "B", "C", "D", "init")), dy, dfin)
+            arr[idx] = saved
+            num[idx] = (lp - lm) / (2 * eps)
+        assert _rel(g[key[name]], num) < 1e-7, name
+
+
+def test_backward_closed_form_scalar():
+    """N = P = 1, one token: y = (a h0 + dt x B) C + D x, so every gradient is a product."""
+    x, dt, A, B, C, D, h0 = 0.7, 0.3, -1.2, 0.5, -0.8, 0.4, 0.9
+    a = np.exp(dt * A)
+    g = oracle.ssd_scan_bwd(np.full((1, 1, 1, 1), x), np.full((1, 1, 1), dt), np.array([A]),
+                            np.full((1, 1, 1, 1), B), np.full((1, 1, 1, 1), C), np.array([D]),
+                            np.ones((1, 1, 1, 1)), np.full((1, 1, 1, 1), h0))
+    assert np.isclose(g["dx"].item(), D + dt * B * C)
+    assert np.isclose(g["dB"].item(), dt * x * C)
+    assert np.isclose(g["dC"].item(), a * h0 + dt * x * B)
+    assert np.isclose(g["ddt"].item(), x * B * C + A * a * h0 * C)
+    assert np.isclose(g["dA"].item(), dt * a * h0 * C)
+    assert np.isclose(g["dD"].item(), x)
+    assert np.isclose(g["dinit"].item(), a * C)
