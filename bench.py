@@ -36,6 +36,11 @@ sys.path.insert(0, ROOT)
 from mamba_ssd_layer_scan_b200 import configs, inputs  # noqa: E402
 
 KERNELS = ("chunk_cumsum", "chunk_state", "state_passing", "chunk_scan")
+# Kernels of one ssd_chunk_scan_bwd call with dfinal and dinit, no initial state: a zero fill;
+# the reversed tensor-core scan (3 gathers, dt shift, 4 scan kernels) and dinit; a fill of ones;
+# the dB scan (3 gathers, dfinal transpose, 4 scan kernels, group sum, head dot) and the dC scan
+# (the same without a transpose); the token and decay kernels.
+BWD_KERNELS = 1 + 8 + 1 + 1 + 10 + 9 + 2
 KERNEL_SOURCES = {
     "chunk_cumsum": ["chunk_cumsum.cu"],
     "chunk_state": ["chunk_tc.cu", "sm100.cuh"],
@@ -506,6 +511,35 @@ def main():
     assert ssd.workspace_status(vws) == ssd.SSD_OK, "varlen scan status"
     varlen_ms = statistics.mean(v_ms)
 
+    # ---- backward pass of the same scan (all seven gradients, forward recomputed inside)
+    gin = inputs.make_grad_inputs(w)
+    gdy = torch.from_numpy(gin.dy).to(dev).to(xdt)
+    gdf = torch.from_numpy(gin.dfinal).to(dev)
+    gws = torch.empty(ssd.bwd_workspace_size(bshape, w.chunk), dtype=torch.uint8, device=dev)
+
+    def bwd():
+        return ssd.chunk_scan_bwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], gdy, w.chunk,
+                                  dfinal=gdf, workspace=gws)
+
+    for _ in range(3):
+        flush.fill_(1.0)
+        bwd()
+    torch.cuda.synchronize()
+    Kg = max(5, min(K, 20))
+    g_ms = []
+    for _ in range(Kg):
+        flush.fill_(1.0)
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        bwd()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        g_ms.append(g0.elapsed_time(g1))
+    assert ssd.workspace_status(gws) == ssd.SSD_OK, "backward status"
+    bwd_ms = statistics.mean(g_ms)
+    del gws
+
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
@@ -581,6 +615,12 @@ def main():
                    "sequence_lengths": np.diff(vin.cu_seqlens).tolist(),
                    "kernels_per_step": 5,
                    "l2": "256 MB buffer written before each timed call (outside the events)"},
+        "backward": {"workload": w.name + "_bwd_dfinal",
+                     "metric": "ssd_chunk_scan_bwd_tokens_per_s",
+                     "value": tokens_per_step / (bwd_ms / 1e3), "unit": "tokens/s",
+                     "ms_per_step": bwd_ms, "steps": Kg, "kernels_per_step": BWD_KERNELS,
+                     "gradients": ["dx", "ddt", "dA", "dB", "dC", "dD", "dinit"],
+                     "l2": "256 MB buffer written before each timed call (outside the events)"},
         "decode": {"workload": wd.name, "metric": "ssd_state_update_GBps", "value":
                    dbytes / (dec_ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": dec_ms,
                    "frac_hbm": dbytes / (dec_ms / 1e3) / 1e9 / hbm, "bytes_per_step": dbytes,

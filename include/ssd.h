@@ -222,6 +222,45 @@ ssd_status ssd_seqpar_finish(const ssd_shape *shape, const void *x, const void *
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Backward pass of the chunked scan: the gradients of a scalar loss with respect to every input,
+ * given its gradients dy (with respect to y) and dfinal (with respect to the final state).
+ * The pages give no backward; it is the reverse-mode derivative of the forward definition.  The
+ * scan is a multiplication by a semiseparable matrix (mohakchugh.is-a.dev "Mamba-2", The
+ * Duality), whose transpose is semiseparable too, so the adjoint state g_t = dL/dh_t obeys a
+ * recurrence of the same form run backwards in time, g_t = exp(dt_{t+1} A_h) g_{t+1} + dy_t C_t^T with g_{L-1} = dy_{L-1} C_{L-1}^T + dfinal,
+ * and the three contractions of the backward are scans of the forward's kind:
+ *     dx_t = D_h dy_t + dt_t g_t B_t                  (tensor cores, time-reversed scan)
+ *     dB_t = sum over the group's heads of dt_t g_t^T x_t     (CUDA cores, float32)
+ *     dC_t = sum over the group's heads of h_t^T dy_t         (CUDA cores, float32)
+ *     ddt_t = <x_t, g_t B_t> + A_h sum_{k>=t} q_k,
+ *         q_k = <dy_k, y_k - D_h x_k> - dt_k <x_k, g_k B_k> (+ <dfinal, h_{L-1}> at k = L-1)
+ *     dA_h = sum_{b,t} dt_t sum_{k>=t} q_k,   dD_h = sum_{b,t} <dy_t, x_t>,
+ *     dinit = exp(dt_0 A_h) g_0.
+ * Nothing needs to be kept from the forward call: the dC scan runs the forward recurrence
+ * again (float32).  The decay gradient is a reverse cumulative sum that telescopes, so its two
+ * dot products are taken from the float32 scans (<dy_k, y_k - D x_k> = <h_k^T dy_k, C_k>,
+ * <x_k, g_k B_k> = <g_k^T x_k, B_k>), not from bf16 intermediates.
+ *
+ *   x, B, C, dy, dt, A, D, init_state: as for ssd_chunk_scan_fwd (dy has y's layout and dtype).
+ *   dfinal   (batch, nheads, headdim, dstate) float32, nullable (= zero).
+ *   dx (batch, seqlen, nheads, headdim), ddt (batch, seqlen, nheads), dA (nheads),
+ *   dB, dC (batch, seqlen, ngroups, dstate), dD (nheads): float32 outputs, all required;
+ *   dinit (batch, nheads, headdim, dstate) float32, nullable (skipped).  dA and dD are summed
+ *   over the batch.  No output may alias an input.
+ *   workspace: ssd_chunk_scan_bwd_workspace_size bytes, 256-byte aligned, caller-owned; its
+ *   status word (ssd_workspace_status) reports an in-kernel timeout as for the forward.
+ * Tensor-core shapes only (bf16, headdim 64, dstate 128, chunk_size 128 or 256); others return
+ * SSD_ERR_UNSUPPORTED, and the size query returns 0 for them.  Launches only on `stream`.
+ */
+size_t ssd_chunk_scan_bwd_workspace_size(const ssd_shape *shape, int chunk_size);
+ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float *dt,
+                              const float *A, const void *B, const void *C, const float *D,
+                              int chunk_size, const float *init_state, const void *dy,
+                              const float *dfinal, float *dx, float *ddt, float *dA, float *dB,
+                              float *dC, float *dD, float *dinit, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+/*
  * One recurrent (decode) step for one new token per sequence, O(1) in the length of the past
  * (crackai.dev "Transformers are SSMs", Why It Matters; mohakchugh.is-a.dev "Mamba-2", Why
  * This Matters for Hardware, linear mode):

@@ -24,7 +24,8 @@ constexpr int kMaxSeg = 8;       // Q <= 256 = 8 segments of 32 tokens
 __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(const float *__restrict__ dt, const float *__restrict__ A,
                     float *__restrict__ cs, float *__restrict__ dtc, int *__restrict__ status,
-                    int64_t seqlen, int H, int Q, int64_t nchunks, const int2 *__restrict__ tab)
+                    int64_t seqlen, int H, int Q, int64_t nchunks, const int2 *__restrict__ tab,
+                    bool unit_weights)
 {
     // First kernel of every scan: clears the workspace status word the later kernels may set.
     if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
@@ -60,7 +61,8 @@ chunk_cumsum_kernel(const float *__restrict__ dt, const float *__restrict__ A,
     for (int sg = 0; sg < kMaxSeg; ++sg) {
         const int tau = sg * 32 + lane;
         const float d = (sg < nseg && tau < Q) ? tile[tau * (kHeadTile + 1) + j] : 0.f;
-        if (dtc && sg < nseg && tau < Q) dtc[row + tau] = d;
+        // unit_weights: the input weight of every token is 1 (decay still from dt); 0 past the end
+        if (dtc && sg < nseg && tau < Q) dtc[row + tau] = unit_weights ? (tau < len ? 1.f : 0.f) : d;
         v[sg] = d * Ah;
     }
 #pragma unroll
@@ -92,12 +94,13 @@ __global__ void fill_final_kernel(const float *__restrict__ init, float *__restr
 
 cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, float *dtc,
                                 int *status, int64_t batch, int64_t seqlen, int nheads, int Q,
-                                int64_t nchunks, cudaStream_t st, const int2 *tab)
+                                int64_t nchunks, cudaStream_t st, const int2 *tab,
+                                bool unit_weights)
 {
     const unsigned grid = (unsigned)(((nheads + kHeadTile - 1) / kHeadTile) * nchunks * batch);
     const size_t smem = (size_t)Q * (kHeadTile + 1) * sizeof(float);
     chunk_cumsum_kernel<<<grid, kThreads, smem, st>>>(dt, A, cs, dtc, status, seqlen, nheads,
-                                                      Q, nchunks, tab);
+                                                      Q, nchunks, tab, unit_weights);
     return cudaGetLastError();
 }
 

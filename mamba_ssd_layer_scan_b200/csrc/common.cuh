@@ -75,7 +75,8 @@ void set_last_error(const char *msg);
 // non-null, writes dt re-laid out as (b, c, H, Q) with zeros past the end of the sequence.
 cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, float *dtc,
                                 int *status, int64_t batch, int64_t seqlen, int nheads, int Q,
-                                int64_t nchunks, cudaStream_t st, const int2 *tab = nullptr);
+                                int64_t nchunks, cudaStream_t st, const int2 *tab = nullptr,
+                                bool unit_weights = false);
 
 // Packed variable-length input: the chunk table (tab, nchunks entries) and the first chunk of
 // every sequence (cstart, nseq + 1 entries) from cu_seqlens; clears *status and sets
@@ -155,6 +156,41 @@ cudaError_t launch_segment_log_decay(const float *cs, float *out, int64_t batch,
 cudaError_t launch_seqpar_combine(const float *h_loc_all, const float *logdec_all,
                                   const float *init, float *h_in, int nranks, int rank,
                                   int64_t BH, int PN, cudaStream_t st);
+
+// ---- backward helpers (backward.cu)
+// out[b][t][r][e] = in[b][src][r_in][e]: src = L-1-t when `reverse`, r_in = r / (rows_out /
+// rows_in) (heads reading their group's row); converts the element type.
+cudaError_t launch_gather(const void *in, bool in_bf16, void *out, bool out_bf16, int64_t batch,
+                          int64_t L, int rows_in, int rows_out, int E, bool reverse,
+                          cudaStream_t st);
+// dt' for the time-reversed adjoint scan: dt'[b][t][h] = dt[b][L-t][h] for t >= 1, 0 for t = 0.
+cudaError_t launch_reverse_shift_dt(const float *dt, float *out, int64_t batch, int64_t L, int H,
+                                   cudaStream_t st);
+cudaError_t launch_fill(float *out, float value, int64_t n, cudaStream_t st);
+// per (b, h) matrix of rows x cols: out = in^T (in [.][rows][cols] -> out [.][cols][rows])
+cudaError_t launch_transpose(const float *in, float *out, int64_t mats, int rows, int cols,
+                             cudaStream_t st);
+// dx[b][t][h][p] = D_h dy + dt[b][t][h] gb[b][L-1-t][h][p];
+// q[b][t][h] = ydot - dt ddt_in (+ <dfinal, final> at t = L-1; fin_t is the final state (n, p))
+cudaError_t launch_bwd_tokens(const bf16 *dy, const float *dt, const float *D,
+                              const bf16 *gb_rev, const float *ydot, const float *ddt_in,
+                              const float *dfinal, const float *fin_t, float *dx, float *q,
+                              int64_t batch, int64_t L, int H, int P, int N, cudaStream_t st);
+// out[b][t][h] = sum_n in[b][src(t)][h][n] v[b][t][g(h)][n], src(t) = L-1-t when `reverse`
+cudaError_t launch_head_dot(const float *in, const bf16 *v, float *out, int64_t batch, int64_t L,
+                            int H, int G, int N, bool reverse, cudaStream_t st);
+// dl = reverse cumsum of q over t per (b, h); ddt = ddt_in + A_h dl; dA_h = sum dt dl;
+// dD_h = sum <dy, x>
+cudaError_t launch_bwd_decay(const float *q, const float *ddt_in, const float *dt,
+                             const float *A, const bf16 *x, const bf16 *dy, float *ddt,
+                             float *dA, float *dD, int64_t batch, int64_t L, int H, int P,
+                             cudaStream_t st);
+// out[b][t][g][n] = sum_{h in g} w[b][t][h] in[b][src(t)][h][n] (w = dt, or 1 when null)
+cudaError_t launch_group_sum(const float *in, const float *w, float *out, int64_t batch,
+                             int64_t L, int H, int G, int N, bool reverse, cudaStream_t st);
+// dinit[b][h] = exp(dt[b][0][h] A_h) F[b][h]
+cudaError_t launch_scale_init_grad(const float *F, const float *dt, const float *A, float *out,
+                                   int64_t batch, int64_t L, int H, int PN, cudaStream_t st);
 
 // Chunk state and state passing in one kernel (chunks walked in order per block of heads):
 // writes the bf16 entering states and the float32 final state; no float32 chunk states.

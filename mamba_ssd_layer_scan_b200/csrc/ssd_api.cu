@@ -413,6 +413,210 @@ ssd_status ssd_chunk_scan_varlen_fwd(const ssd_shape *shape, const void *x, cons
     return SSD_OK;
 }
 
+// ---- backward pass (the gradients of the chunked scan)
+namespace {
+constexpr int kBwdSimtChunk = 64;   // chunk of the two CUDA-core scans (head dim N, state P)
+
+struct BwdLayout {
+    size_t r_ws, s_ws;                          // tensor-core and CUDA-core scan workspaces
+    size_t dyr, Cr, Br, dtr, zerosD, gb, Fr, ones;
+    size_t xs, Bs, Cs, inits, ys, fin_t;        // the CUDA-core scans' operands (reused)
+    size_t ydot, ddt_in, q, total;
+    size_t r_bytes, s_bytes;
+};
+
+ssd_shape simt_shape(const ssd_shape &s)
+{
+    ssd_shape t = s;          // head dimension N, state dimension P, one group per head, f32
+    t.headdim = s.dstate;
+    t.dstate = s.headdim;
+    t.ngroups = s.nheads;
+    t.dtype = SSD_F32;
+    return t;
+}
+
+BwdLayout bwd_layout(const ssd_shape *s, int Q)
+{
+    BwdLayout w;
+    const size_t b = s->batch, L = s->seqlen, H = s->nheads, P = s->headdim, N = s->dstate,
+                 G = s->ngroups;
+    const ssd_shape t = simt_shape(*s);
+    w.r_bytes = layout(s, Q).total;
+    w.s_bytes = layout(&t, kBwdSimtChunk).total;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { const size_t at = o; o += round256(bytes); return at; };
+    w.r_ws = take(w.r_bytes);   // first: its status word is the workspace's
+    w.s_ws = take(w.s_bytes);
+    w.dyr = take(b * L * H * P * 2);
+    w.Cr = take(b * L * G * N * 2);
+    w.Br = take(b * L * G * N * 2);
+    w.dtr = take(b * L * H * 4);
+    w.zerosD = take(H * 4);
+    w.gb = take(b * L * H * P * 2);
+    w.Fr = take(b * H * P * N * 4);
+    w.ones = take(b * L * H * 4);
+    w.xs = take(b * L * H * N * 4);
+    w.Bs = take(b * L * H * P * 4);
+    w.Cs = take(b * L * H * P * 4);
+    w.inits = take(b * H * N * P * 4);
+    w.ys = take(b * L * H * N * 4);
+    w.fin_t = take(b * H * N * P * 4);
+    w.ydot = take(b * L * H * 4);
+    w.ddt_in = take(b * L * H * 4);
+    w.q = take(b * L * H * 4);
+    w.total = o;
+    return w;
+}
+
+ssd_status check_bwd(const ssd_shape *s, int Q)
+{
+    ssd_status st = check_shape(s, true);
+    if (st != SSD_OK) return st;
+    if (!valid_chunk(Q) || !ssd::tc_supported(s->dtype == SSD_BF16, (int)s->headdim,
+                                              (int)s->dstate, Q))
+        return fail(SSD_ERR_UNSUPPORTED,
+                    "the backward pass runs for the tensor-core shapes: bf16, headdim 64, "
+                    "dstate 128, chunk_size 128 or 256");
+    return SSD_OK;
+}
+}  // namespace
+
+size_t ssd_chunk_scan_bwd_workspace_size(const ssd_shape *shape, int chunk_size)
+{
+    if (check_bwd(shape, chunk_size) != SSD_OK) return 0;
+    return bwd_layout(shape, chunk_size).total;
+}
+
+ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float *dt,
+                              const float *A, const void *B, const void *C, const float *D,
+                              int chunk_size, const float *init_state, const void *dy,
+                              const float *dfinal, float *dx, float *ddt, float *dA, float *dB,
+                              float *dC, float *dD, float *dinit, void *workspace,
+                              size_t workspace_bytes, void *stream)
+{
+    ssd_status st = check_bwd(shape, chunk_size);
+    if (st != SSD_OK) return st;
+    const ssd_shape s = *shape;
+    const int H = (int)s.nheads, G = (int)s.ngroups, P = (int)s.headdim, N = (int)s.dstate;
+    const int Q = chunk_size;
+    const int64_t b = s.batch, L = s.seqlen;
+    cudaStream_t cst = static_cast<cudaStream_t>(stream);
+    if (!dA || !dD) return fail(SSD_ERR_INVALID_ARG, "dA and dD must be non-NULL");
+    if (b == 0 || L == 0) {   // no token: only dinit (= dfinal) and the zero dA, dD
+        cudaError_t e = cudaMemsetAsync(dA, 0, H * 4, cst);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dD, 0, H * 4, cst);
+        if (e == cudaSuccess && dinit)
+            e = ssd::launch_fill_final(dfinal, dinit, b * H * P * N, cst);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "empty backward");
+    }
+    if (!x || !dt || !A || !B || !C || !D || !dy || !dx || !ddt || !dB || !dC || !workspace)
+        return fail(SSD_ERR_INVALID_ARG, "inputs, dy and the gradient buffers must be non-NULL");
+    if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(dy) ||
+        (init_state && !aligned16(init_state)) || (dfinal && !aligned16(dfinal)) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(SSD_ERR_INVALID_ARG,
+                    "x, B, C, dy and the states must be 16-byte, the workspace 256-byte aligned");
+    const BwdLayout wl = bwd_layout(&s, Q);
+    if (workspace_bytes < wl.total)
+        return fail(SSD_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu",
+                    wl.total, workspace_bytes);
+    char *ws = static_cast<char *>(workspace);
+    auto F = [&](size_t off) { return reinterpret_cast<float *>(ws + off); };
+    auto Hh = [&](size_t off) { return reinterpret_cast<ssd::bf16 *>(ws + off); };
+    float *zerosD = F(wl.zerosD);
+    cudaError_t e = ssd::launch_fill(zerosD, 0.f, H, cst);
+    if (e != cudaSuccess) return cuda_fail(e, "fill");
+
+    // 1. g_t B_t: the forward scan of the reversed sequence (x' = dy, B' = C, C' = B), unit
+    // input weights, decays shifted by one token, started from dfinal; its final state is g_0.
+    // Its cumsum clears the workspace status word (offset 0) that the tensor-core kernels set.
+    const int64_t nch = (L + Q - 1) / Q;
+    const ssd::WsLayout rl = layout(&s, Q);
+    char *rw = ws + wl.r_ws;
+    int *status = reinterpret_cast<int *>(rw + rl.status);
+    float *cs_r = reinterpret_cast<float *>(rw + rl.cs);
+    float *dtc_r = reinterpret_cast<float *>(rw + rl.dtc);
+    float *states_r = reinterpret_cast<float *>(rw + rl.states);
+    ssd::bf16 *hin_r = reinterpret_cast<ssd::bf16 *>(rw + rl.hin_bf16);
+    const char *why = "";
+    if ((e = ssd::launch_gather(dy, true, Hh(wl.dyr), true, b, L, H, H, P, true, cst)) ||
+        (e = ssd::launch_gather(C, true, Hh(wl.Cr), true, b, L, G, G, N, true, cst)) ||
+        (e = ssd::launch_gather(B, true, Hh(wl.Br), true, b, L, G, G, N, true, cst)) ||
+        (e = ssd::launch_reverse_shift_dt(dt, F(wl.dtr), b, L, H, cst)))
+        return cuda_fail(e, "reverse inputs");
+    e = ssd::launch_chunk_cumsum(F(wl.dtr), A, cs_r, dtc_r, status, b, L, H, Q, nch, cst,
+                                 nullptr, true);
+    if (e != cudaSuccess) return cuda_fail(e, "reversed cumsum");
+    e = ssd::launch_chunk_state_tc(Hh(wl.dyr), dtc_r, Hh(wl.Cr), cs_r, states_r, status, b, L, H,
+                                   G, Q, nch, cst, &why);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+    e = ssd::launch_state_passing(states_r, cs_r, dfinal, F(wl.Fr), hin_r, b, H, P, N, Q, nch,
+                                  cst);
+    if (e != cudaSuccess) return cuda_fail(e, "reversed state passing");
+    e = ssd::launch_chunk_scan_tc(Hh(wl.dyr), dtc_r, Hh(wl.Cr), Hh(wl.Br), cs_r, hin_r, zerosD,
+                                  Hh(wl.gb), status, b, L, H, G, Q, nch, cst, &why);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+    if (dinit && (e = ssd::launch_scale_init_grad(F(wl.Fr), dt, A, dinit, b, L, H, P * N, cst)))
+        return cuda_fail(e, "dinit");
+
+    // 2. dB and dC: scans with head dimension N and state dimension P on CUDA cores (float32),
+    // summed over the heads of each group.  Their per-head outputs also give, contracted with
+    // B (resp. C), the two float32 dot products of the decay gradient: <x_t, g_t B_t> and
+    // <dy_t, y_t - D x_t>.
+    const ssd_shape t = simt_shape(s);
+    const int Qs = kBwdSimtChunk;
+    const int64_t nchs = (L + Qs - 1) / Qs;
+    const ssd::WsLayout sl = layout(&t, Qs);
+    char *sw = ws + wl.s_ws;
+    float *cs_s = reinterpret_cast<float *>(sw + sl.cs);
+    float *states_s = reinterpret_cast<float *>(sw + sl.states);
+    if ((e = ssd::launch_fill(F(wl.ones), 1.f, b * L * H, cst)))
+        return cuda_fail(e, "fill");
+    for (int pass = 0; pass < 2; ++pass) {   // 0: dB (reversed), 1: dC (forward)
+        const bool rev = pass == 0;
+        const float *init_s = rev ? dfinal : init_state;
+        if ((e = ssd::launch_gather(rev ? C : B, true, F(wl.xs), false, b, L, G, H, N, rev,
+                                    cst)) ||
+            (e = ssd::launch_gather(rev ? dy : x, true, F(wl.Bs), false, b, L, H, H, P, rev,
+                                    cst)) ||
+            (e = ssd::launch_gather(rev ? x : dy, true, F(wl.Cs), false, b, L, H, H, P, rev,
+                                    cst)))
+            return cuda_fail(e, "scan operands");
+        if (init_s && (e = ssd::launch_transpose(init_s, F(wl.inits), b * H, P, N, cst)))
+            return cuda_fail(e, "transpose");
+        const float *w_s = rev ? F(wl.ones) : dt;
+        e = ssd::launch_chunk_cumsum(rev ? F(wl.dtr) : dt, A, cs_s, nullptr, nullptr, b, L, H,
+                                     Qs, nchs, cst);
+        if (e == cudaSuccess)
+            e = ssd::launch_chunk_state_simt(false, F(wl.xs), w_s, F(wl.Bs), cs_s, states_s, b, L,
+                                             H, H, N, P, Qs, nchs, cst);
+        if (e == cudaSuccess)
+            e = ssd::launch_state_passing(states_s, cs_s, init_s ? F(wl.inits) : nullptr,
+                                          rev ? nullptr : F(wl.fin_t), nullptr, b, H, N, P, Qs,
+                                          nchs, cst);
+        if (e == cudaSuccess)
+            e = ssd::launch_chunk_scan_simt(false, F(wl.xs), w_s, F(wl.Bs), F(wl.Cs), cs_s,
+                                            states_s, zerosD, F(wl.ys), b, L, H, H, N, P, Qs,
+                                            nchs, cst);
+        if (e == cudaSuccess)
+            e = ssd::launch_group_sum(F(wl.ys), rev ? dt : nullptr, rev ? dB : dC, b, L, H, G, N,
+                                      rev, cst);
+        if (e == cudaSuccess)
+            e = ssd::launch_head_dot(F(wl.ys), (const ssd::bf16 *)(rev ? B : C),
+                                     F(rev ? wl.ddt_in : wl.ydot), b, L, H, G, N, rev, cst);
+        if (e != cudaSuccess) return cuda_fail(e, rev ? "dB scan" : "dC scan");
+    }
+
+    // 3. dx, the decay-gradient terms and their reverse cumsum: ddt, dA, dD
+    if ((e = ssd::launch_bwd_tokens((const ssd::bf16 *)dy, dt, D, Hh(wl.gb), F(wl.ydot),
+                                    F(wl.ddt_in), dfinal, F(wl.fin_t), dx, F(wl.q), b, L, H, P,
+                                    N, cst)) ||
+        (e = ssd::launch_bwd_decay(F(wl.q), F(wl.ddt_in), dt, A, (const ssd::bf16 *)x,
+                                   (const ssd::bf16 *)dy, ddt, dA, dD, b, L, H, P, cst)))
+        return cuda_fail(e, "token gradients");
+    return SSD_OK;
+}
+
 // ---- sequence parallelism (one contiguous segment of the sequence per rank)
 namespace {
 ssd_status check_seqpar(const ssd_shape *s, int Q)

@@ -84,6 +84,24 @@ def make_block_inputs(w: Workload, seed: Optional[int] = None) -> BlockInputs:
     return BlockInputs(z, dt_raw, dt_bias, (1e-3, 0.1))
 
 
+@dataclass
+class GradInputs:
+    """Upstream gradients for the backward pass (float32, exact stored values)."""
+    dy: np.ndarray         # like y, (b, L, H, P), rounded to bf16 for bf16 workloads
+    dfinal: np.ndarray     # like the final state, (b, H, P, N)
+
+
+def make_grad_inputs(w: Workload, seed: Optional[int] = None) -> GradInputs:
+    """dy ~ N(0, 1) and dfinal ~ 0.1 N(0, 1), from their own PCG64 stream (seed + 700)."""
+    rng = np.random.Generator(np.random.PCG64((w.seed if seed is None else seed) + 700))
+    b, L, H, P, N = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate
+    dy = rng.standard_normal((b, L, H, P), dtype=np.float32)
+    dfinal = (0.1 * rng.standard_normal((b, H, P, N), dtype=np.float32)).astype(np.float32)
+    if w.dtype == "bf16":
+        dy = round_bf16(dy)
+    return GradInputs(dy, dfinal)
+
+
 def make_inputs(w: Workload, seed: Optional[int] = None) -> SSDInputs:
     rng = np.random.Generator(np.random.PCG64(w.seed if seed is None else seed))
     b, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups

@@ -92,6 +92,12 @@ def lib():
     L.ssd_chunk_scan_varlen_fwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
                                             ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp, _vp,
                                             ctypes.c_size_t, _vp]
+    L.ssd_chunk_scan_bwd_workspace_size.restype = ctypes.c_size_t
+    L.ssd_chunk_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int]
+    L.ssd_chunk_scan_bwd.restype = ctypes.c_int
+    L.ssd_chunk_scan_bwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
+                                     ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, ctypes.c_size_t, _vp]
     L.ssd_state_update.restype = ctypes.c_int
     L.ssd_state_update.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _vp]
@@ -269,6 +275,49 @@ def chunk_scan_varlen_fwd(x, dt, A, B, C, D, cu_seqlens, chunk_size: int = 256,
 
 
 # ---------------------------------------------------------------- sequence parallelism
+def bwd_workspace_size(shape: Shape, chunk_size: int) -> int:
+    n = lib().ssd_chunk_scan_bwd_workspace_size(ctypes.byref(shape), chunk_size)
+    if n == 0:
+        raise SSDError(SSD_ERR_UNSUPPORTED, last_error())
+    return n
+
+
+def chunk_scan_bwd(x, dt, A, B, C, D, dy, chunk_size: int = 256, init_state=None, dfinal=None,
+                   return_dinit: bool = True, workspace=None, stream=None):
+    """Gradients of the chunked scan (ssd_chunk_scan_bwd): given dy (like y) and dfinal
+    (b, H, P, N) f32 or None, returns a dict of float32 tensors dx (b, L, H, P), ddt (b, L, H),
+    dA (H,), dB and dC (b, L, G, N), dD (H,) and dinit (b, H, P, N) (None unless
+    return_dinit).  bf16 tensor-core shapes only."""
+    torch = _torch()
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = x.device
+    for t, n in ((x, "x"), (B, "B"), (C, "C"), (dy, "dy")):
+        _require(t, n, x.dtype, dev)
+    for t, n in ((dt, "dt"), (A, "A"), (D, "D")):
+        _require(t, n, torch.float32, dev)
+    for t, n in ((init_state, "init_state"), (dfinal, "dfinal")):
+        if t is not None:
+            _require(t, n, torch.float32, dev)
+    if tuple(dy.shape) != tuple(x.shape):
+        raise ValueError(f"dy must have x's shape {tuple(x.shape)}, got {tuple(dy.shape)}")
+    shape = make_shape(b, L, H, P, N, G, _dtype_code(x))
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_size(shape, chunk_size), dtype=torch.uint8,
+                                device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = dict(dx=torch.empty((b, L, H, P), **f32), ddt=torch.empty((b, L, H), **f32),
+             dA=torch.empty((H,), **f32), dB=torch.empty((b, L, G, N), **f32),
+             dC=torch.empty((b, L, G, N), **f32), dD=torch.empty((H,), **f32),
+             dinit=torch.empty((b, H, P, N), **f32) if return_dinit else None)
+    _check(lib().ssd_chunk_scan_bwd(
+        ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), chunk_size,
+        _ptr(init_state), _ptr(dy), _ptr(dfinal), _ptr(g["dx"]), _ptr(g["ddt"]), _ptr(g["dA"]),
+        _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["dinit"]), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream)))
+    return g
+
+
 def seqpar_local(x, dt, A, B, chunk_size: int = 256, workspace=None, stream=None):
     """Phase 1 on this rank's segment: (h_loc (b, H, P, N) f32, log_decay (b, H) f32,
     workspace to pass on to seqpar_finish)."""

@@ -182,3 +182,30 @@ def test_seqpar_workspace_and_rejections(L):
     rc = L.ssd_seqpar_finish(ctypes.byref(sh), p, p, p, p, 256, p, p, 2, 2, None, p, None, p,
                              1 << 40, None)
     assert rc == ssd.SSD_ERR_INVALID_ARG and "rank" in ssd.last_error()
+
+
+def test_backward_workspace_and_rejections(L):
+    sh = _shape()
+    n = L.ssd_chunk_scan_bwd_workspace_size(ctypes.byref(sh), 256)
+    # two tensor-core scans' workspaces at least, plus the reversed operands
+    assert n >= 2 * ssd.workspace_size(sh, 256) + 4 * 4096 * 80 * 64 * 2
+    assert n % 256 == 0
+    f32 = _shape(dtype=ssd.SSD_F32)
+    assert L.ssd_chunk_scan_bwd_workspace_size(ctypes.byref(f32), 256) == 0
+    assert L.ssd_chunk_scan_bwd_workspace_size(ctypes.byref(sh), 64) == 0
+    p = ctypes.c_void_p(1 << 20)
+    args = lambda **kw: [kw.get(k, p) for k in ("x", "dt", "A", "B", "C", "D")] + [256, None] + \
+        [kw.get(k, p) for k in ("dy",)] + [None] + \
+        [kw.get(k, p) for k in ("dx", "ddt", "dA", "dB", "dC", "dD")] + [None, p,
+                                                                          kw.get("ws_bytes", n),
+                                                                          None]
+    rc = L.ssd_chunk_scan_bwd(ctypes.byref(f32), *args())
+    assert rc == ssd.SSD_ERR_UNSUPPORTED
+    rc = L.ssd_chunk_scan_bwd(ctypes.byref(sh), *args(dA=None))
+    assert rc == ssd.SSD_ERR_INVALID_ARG
+    rc = L.ssd_chunk_scan_bwd(ctypes.byref(sh), *args(dy=None))
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "dy" in ssd.last_error()
+    rc = L.ssd_chunk_scan_bwd(ctypes.byref(sh), *args(dy=ctypes.c_void_p((1 << 20) + 2)))
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "aligned" in ssd.last_error()
+    rc = L.ssd_chunk_scan_bwd(ctypes.byref(sh), *args(ws_bytes=n - 256))
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "workspace" in ssd.last_error()

@@ -1,0 +1,128 @@
+"""GPU parity of the backward pass (ssd_chunk_scan_bwd) against the float64 adjoint oracle.
+
+Every gradient is compared with oracle.ssd_scan_bwd on the same seeded inputs and upstream
+gradients (dy rounded to bf16 like y, dfinal float32).  The bar is the bf16 bound of the forward,
+max over slices of the relative L2 error: per (batch, head) for dx, ddt and dinit, per
+(batch, group) for dB and dC, over the head vector for dA and dD (those are sums over the batch
+and the sequence).  The cases span several chunks with a ragged tail, both tensor-core chunk
+sizes, several groups, with and without an initial state and dfinal, one token, and the
+2.7B-layer shape on sampled heads (dx, ddt, dA, dD and dinit of a head depend only on that head;
+dB and dC, sums over the group's heads, are checked at the smaller sizes).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from mamba_ssd_layer_scan_b200 import configs, inputs, ssd
+
+from _util import TOL, max_rel_per_pair, rel_l2, to_np, torch_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(torch, inp, gin, chunk, device, with_init=True, with_dfinal=True):
+    t = torch_inputs(inp, device)
+    dy = torch.from_numpy(gin.dy).to(device).to(t["x"].dtype)
+    dfinal = torch.from_numpy(gin.dfinal).to(device) if with_dfinal else None
+    init = t["init_state"] if with_init else None
+    g = ssd.chunk_scan_bwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], dy, chunk,
+                           init_state=init, dfinal=dfinal)
+    torch.cuda.synchronize()
+    return {k: (None if v is None else to_np(v)) for k, v in g.items()}
+
+
+def _check(w, g, ref, names=("dx", "ddt", "dB", "dC", "dA", "dD", "dinit")):
+    b, H, G = w.batch, w.nheads, w.ngroups
+    errs = {}
+    for k in names:
+        if k in ("dx", "ddt"):
+            errs[k] = max_rel_per_pair([g[k][i, :, h] for i in range(b) for h in range(H)],
+                                       [ref[k][i, :, h] for i in range(b) for h in range(H)])
+        elif k in ("dB", "dC"):
+            errs[k] = max_rel_per_pair([g[k][i, :, j] for i in range(b) for j in range(G)],
+                                       [ref[k][i, :, j] for i in range(b) for j in range(G)])
+        elif k == "dinit":
+            errs[k] = max_rel_per_pair([g[k][i, h] for i in range(b) for h in range(H)],
+                                       [ref[k][i, h] for i in range(b) for h in range(H)])
+        else:
+            errs[k] = rel_l2(g[k], ref[k])
+        assert np.isfinite(g[k]).all(), k
+    bad = {k: e for k, e in errs.items() if not e <= TOL["bf16"]}
+    assert not bad, f"relative L2 errors above {TOL['bf16']}: {bad} (all: {errs})"
+
+
+CASES = [
+    # (name, workload, chunk, with init_state, with dfinal)
+    ("q256_ragged_init", configs.SSD_370M.with_(batch=2, seqlen=600, nheads=8, ngroups=2,
+                                                 init_state=True), 256, True, True),
+    ("q128_ragged", configs.SSD_370M.with_(batch=1, seqlen=333, nheads=6, seed=77), 128, False,
+     True),
+    ("q256_no_dfinal", configs.SSD_370M.with_(batch=1, seqlen=512, nheads=4, init_state=True,
+                                               seed=78), 256, True, False),
+    ("q256_groups4", configs.SSD_370M.with_(batch=1, seqlen=700, nheads=8, ngroups=4,
+                                             init_state=True, seed=79), 256, True, True),
+    ("one_token", configs.SSD_370M.with_(batch=2, seqlen=1, nheads=4, init_state=True, seed=80),
+     256, True, True),
+]
+
+
+@pytest.mark.parametrize("name,w,chunk,with_init,with_dfinal", CASES, ids=[c[0] for c in CASES])
+def test_backward_parity_every_gradient(cuda_device, name, w, chunk, with_init, with_dfinal):
+    import torch
+    inp = inputs.make_inputs(w)
+    gin = inputs.make_grad_inputs(w)
+    g = _run(torch, inp, gin, chunk, cuda_device, with_init, with_dfinal)
+    ref = oracle.ssd_scan_bwd(inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, gin.dy,
+                              init=inp.init if with_init else None,
+                              dfinal=gin.dfinal if with_dfinal else None)
+    _check(w, g, ref)
+
+
+def test_backward_full_size_sampled_heads(cuda_device):
+    """The 2.7B-layer shape (batch 4, 4096 tokens, 80 heads) in one call; for sampled heads the
+    oracle runs on that head alone (first and last batch rows), which fixes its dx, ddt, dinit."""
+    import torch
+    w = configs.SSD_2P7B.with_(init_state=True)
+    inp = inputs.make_inputs(w)
+    gin = inputs.make_grad_inputs(w)
+    g = _run(torch, inp, gin, w.chunk, cuda_device)
+    heads = [0, 37, w.nheads - 1]
+    batches = [0, w.batch - 1]
+    for h in heads:
+        sl = slice(h, h + 1)
+        ref = oracle.ssd_scan_bwd(inp.x[batches][:, :, sl], inp.dt[batches][:, :, sl], inp.A[sl],
+                                  inp.B[batches], inp.C[batches], inp.D[sl],
+                                  gin.dy[batches][:, :, sl], init=inp.init[batches][:, sl],
+                                  dfinal=gin.dfinal[batches][:, sl])
+        for k in ("dx", "ddt"):
+            assert max_rel_per_pair([g[k][bi, :, h] for bi in batches],
+                                    [ref[k][i, :, 0] for i in range(len(batches))]) <= TOL["bf16"]
+        assert max_rel_per_pair([g["dinit"][bi, h] for bi in batches],
+                                [ref["dinit"][i, 0] for i in range(len(batches))]) <= TOL["bf16"]
+
+
+def test_backward_dD_and_linearity_in_D(cuda_device):
+    """dD_h is sum <dy, x> over the batch and the sequence, and D enters the gradients only
+    through dx = D dy + (a term independent of D): properties that hold at any size."""
+    import torch
+    w = configs.SSD_370M.with_(batch=1, seqlen=1024, nheads=8, seed=81)
+    inp = inputs.make_inputs(w)
+    gin = inputs.make_grad_inputs(w)
+    g1 = _run(torch, inp, gin, 256, cuda_device, False, True)
+    inp.D = inp.D + 0.5
+    g2 = _run(torch, inp, gin, 256, cuda_device, False, True)
+    dD = np.einsum("blhp,blhp->h", gin.dy.astype(np.float64), inp.x.astype(np.float64))
+    assert rel_l2(g1["dD"], dD) <= 1e-5
+    diff = (g2["dx"] - g1["dx"]) - 0.5 * gin.dy
+    assert np.abs(diff).max() <= 1e-5 * max(1.0, np.abs(g1["dx"]).max())
+    for k in ("ddt", "dB", "dC", "dA", "dinit"):
+        assert np.array_equal(g1[k], g2[k]), k
+
+
+def test_backward_unsupported_shape_rejected(cuda_device):
+    import torch
+    w = configs.SSD_F32_SMALL.with_(batch=1, seqlen=64, nheads=2)
+    inp = inputs.make_inputs(w)
+    t = torch_inputs(inp, cuda_device)
+    with pytest.raises(ssd.SSDError):
+        ssd.chunk_scan_bwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], t["x"].clone(), 64)
