@@ -37,10 +37,10 @@ from mamba_ssd_layer_scan_b200 import configs, inputs  # noqa: E402
 
 KERNELS = ("chunk_cumsum", "chunk_state", "state_passing", "chunk_scan")
 # Kernels of one ssd_chunk_scan_bwd call with dfinal and dinit, no initial state: a zero fill;
-# the reversed tensor-core scan (3 gathers, dt shift, 4 scan kernels) and dinit; a fill of ones;
-# the dB scan (3 gathers, dfinal transpose, 4 scan kernels, group sum, head dot) and the dC scan
+# the reversed tensor-core scan (3 gathers, dt shift, 4 scan kernels) and dinit; the dB scan
+# (dfinal transpose, cumsum, chunk state, state passing, chunk scan, group sum) and the dC scan
 # (the same without a transpose); the token and decay kernels.
-BWD_KERNELS = 1 + 8 + 1 + 1 + 10 + 9 + 2
+BWD_KERNELS = 1 + 8 + 1 + 6 + 5 + 2
 KERNEL_SOURCES = {
     "chunk_cumsum": ["chunk_cumsum.cu"],
     "chunk_state": ["chunk_tc.cu", "sm100.cuh"],

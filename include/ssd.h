@@ -246,7 +246,8 @@ ssd_status ssd_seqpar_finish(const ssd_shape *shape, const void *x, const void *
  *   dx (batch, seqlen, nheads, headdim), ddt (batch, seqlen, nheads), dA (nheads),
  *   dB, dC (batch, seqlen, ngroups, dstate), dD (nheads): float32 outputs, all required;
  *   dinit (batch, nheads, headdim, dstate) float32, nullable (skipped).  dA and dD are summed
- *   over the batch.  No output may alias an input.
+ *   over the batch.  No output may alias an input.  x, B, C, dy, dx and the states must be
+ *   16-byte aligned.
  *   workspace: ssd_chunk_scan_bwd_workspace_size bytes, 256-byte aligned, caller-owned; its
  *   status word (ssd_workspace_status) reports an in-kernel timeout as for the forward.
  * Tensor-core shapes only (bf16, headdim 64, dstate 128, chunk_size 128 or 256); others return

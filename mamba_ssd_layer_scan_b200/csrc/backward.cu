@@ -28,21 +28,23 @@
 namespace ssd {
 namespace {
 
-template <typename TI, typename TO>
-__global__ void gather_kernel(const TI *__restrict__ in, TO *__restrict__ out, int64_t batch,
-                              int64_t L, int rows_in, int rows_out, int E, bool reverse)
+// out[b][t][r][:] = in[b][src][r / (rows_out / rows_in)][:] (src = L-1-t when `reverse`), rows of
+// E8 16-byte vectors, one vector per thread.
+__global__ void gather8_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out,
+                               int64_t batch, int64_t L, int rows_in, int rows_out, int E8,
+                               bool reverse)
 {
-    const int64_t n = batch * L * rows_out * E;
+    const int64_t n = batch * L * rows_out * E8;
     const int rep = rows_out / rows_in;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
-        const int e = (int)(i % E);
-        int64_t r = i / E;
+        const int e = (int)(i % E8);
+        int64_t r = i / E8;
         const int ro = (int)(r % rows_out);
         r /= rows_out;
         const int64_t t = r % L, b = r / L;
         const int64_t src = reverse ? L - 1 - t : t;
-        out[i] = from_f32<TO>(to_f32(in[((b * L + src) * rows_in + ro / rep) * E + e]));
+        out[i] = in[((b * L + src) * rows_in + ro / rep) * E8 + e];
     }
 }
 
@@ -78,96 +80,110 @@ __global__ void transpose_kernel(const float *__restrict__ in, float *__restrict
     }
 }
 
-// One warp per (b, t, h): dx over the P channels, and the decay-gradient term q.
-__global__ void bwd_tokens_kernel(const bf16 *__restrict__ dy, const float *__restrict__ dt,
-                                  const float *__restrict__ D, const bf16 *__restrict__ gb_rev,
+// Eight lanes per (b, t, h) row of P = 64 channels, 16 bytes of each bf16 input per lane: dx,
+// <x, dy>, and the decay-gradient term q.
+constexpr int kTokLanes = 8;
+
+__global__ void bwd_tokens_kernel(const bf16 *__restrict__ x, const bf16 *__restrict__ dy,
+                                  const float *__restrict__ dt, const float *__restrict__ D,
+                                  const bf16 *__restrict__ gb_rev,
                                   const float *__restrict__ ydot,
                                   const float *__restrict__ ddt_in,
                                   const float *__restrict__ dfinal,
                                   const float *__restrict__ fin_t, float *__restrict__ dx,
-                                  float *__restrict__ q, int64_t batch, int64_t L, int H, int P,
-                                  int N)
+                                  float *__restrict__ q, float *__restrict__ xdy, int64_t batch,
+                                  int64_t L, int H, int N)
 {
-    const int lane = threadIdx.x % 32;
-    const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / 32;
-    if (w >= batch * L * H) return;
+    constexpr int P = kTokLanes * 8;
+    const int64_t gid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t w = gid / kTokLanes;   // (b, t, h) row
+    const int part = (int)(gid % kTokLanes);
+    const bool ok = w < batch * L * H;
     const int h = (int)(w % H);
     const int64_t t = (w / H) % L, b = w / H / L;
-    const int64_t row = w * P;                                   // (b, t, h) row of dy / dx
-    const int64_t rrow = ((b * L + (L - 1 - t)) * H + h) * P;    // reversed row of gb
-    const float dth = dt[w];
-    for (int p = lane; p < P; p += 32)
-        dx[row + p] = D[h] * to_f32(dy[row + p]) + dth * to_f32(gb_rev[rrow + p]);
-    float sf = 0.f;
-    if (dfinal && t == L - 1) {   // the final state also depends on the last log-decay cumsum
-        // fin_t is the final state transposed, (n, p)
-        const int64_t base = (b * H + h) * (int64_t)P * N;
-        for (int i = lane; i < P * N; i += 32)
-            sf = fmaf(dfinal[base + i], fin_t[base + (int64_t)(i % N) * P + i / N], sf);
+    float sd = 0.f, sf = 0.f, dth = 0.f;
+    if (ok) {
+        dth = dt[w];
+        const int64_t row = w * P + part * 8;
+        const int64_t rrow = ((b * L + (L - 1 - t)) * H + h) * P + part * 8;
+        float xv[8], dyv[8], gv[8];
+        const uint4 rx = *reinterpret_cast<const uint4 *>(x + row);
+        const uint4 rd = *reinterpret_cast<const uint4 *>(dy + row);
+        const uint4 rg = *reinterpret_cast<const uint4 *>(gb_rev + rrow);
+        const bf16 *px = reinterpret_cast<const bf16 *>(&rx);
+        const bf16 *pd = reinterpret_cast<const bf16 *>(&rd);
+        const bf16 *pg = reinterpret_cast<const bf16 *>(&rg);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sf += __shfl_xor_sync(0xffffffffu, sf, o);
+        for (int i = 0; i < 8; ++i) {
+            xv[i] = __bfloat162float(px[i]);
+            dyv[i] = __bfloat162float(pd[i]);
+            gv[i] = __bfloat162float(pg[i]);
+            sd = fmaf(dyv[i], xv[i], sd);
+        }
+        const float Dh = D[h];
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = fmaf(Dh, dyv[i], dth * gv[i]);
+        *reinterpret_cast<float4 *>(dx + row) = make_float4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<float4 *>(dx + row + 4) = make_float4(o[4], o[5], o[6], o[7]);
+        if (dfinal && t == L - 1) {   // the final state also depends on the last log-decay cumsum
+            // fin_t is the final state transposed, (n, p)
+            const int64_t base = (b * H + h) * (int64_t)P * N;
+            for (int i = part; i < P * N; i += kTokLanes)
+                sf = fmaf(dfinal[base + i], fin_t[base + (int64_t)(i % N) * P + i / N], sf);
+        }
     }
-    if (lane == 0) q[w] = ydot[w] - dth * ddt_in[w] + sf;
-}
-
-// One warp per (b, t, h): out = <in[b][src(t)][h][:], v[b][t][g(h)][:]> over N (src = L-1-t
-// when `reverse`).
-__global__ void head_dot_kernel(const float *__restrict__ in, const bf16 *__restrict__ v,
-                                float *__restrict__ out, int64_t batch, int64_t L, int H, int G,
-                                int N, bool reverse)
-{
-    const int lane = threadIdx.x % 32;
-    const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / 32;
-    if (w >= batch * L * H) return;
-    const int h = (int)(w % H);
-    const int64_t t = (w / H) % L, b = w / H / L;
-    const int64_t src = reverse ? L - 1 - t : t;
-    const float *a = in + ((b * L + src) * H + h) * (int64_t)N;
-    const bf16 *c = v + ((b * L + t) * G + h / (H / G)) * (int64_t)N;
-    float s = 0.f;
-    for (int n = lane; n < N; n += 32) s = fmaf(a[n], to_f32(c[n]), s);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) out[w] = s;
+    for (int o = 1; o < kTokLanes; o <<= 1) {
+        sd += __shfl_xor_sync(0xffffffffu, sd, o);
+        sf += __shfl_xor_sync(0xffffffffu, sf, o);
+    }
+    if (ok && part == 0) {
+        q[w] = ydot[w] - dth * ddt_in[w] + sf;
+        xdy[w] = sd;
+    }
 }
 
-// One warp per (b, h): reverse cumsum of q over t in tiles of 32; ddt and the per-(b, h)
-// partial sums of dA and dD (atomically added per head).
-__global__ void bwd_decay_kernel(const float *__restrict__ q, const float *__restrict__ ddt_in,
-                                 const float *__restrict__ dt, const float *__restrict__ A,
-                                 const bf16 *__restrict__ x, const bf16 *__restrict__ dy,
-                                 float *__restrict__ ddt, float *__restrict__ dA,
-                                 float *__restrict__ dD, int64_t batch, int64_t L, int H, int P)
+// One block per (b, h): the reverse cumsum of q over t (each thread a contiguous segment, the
+// segments' totals combined by a block-wide suffix scan), ddt, and the (b, h) partial sums of dA
+// and dD (atomically added per head).
+constexpr int kDecayThreads = 256;
+
+__global__ void __launch_bounds__(kDecayThreads)
+bwd_decay_kernel(const float *__restrict__ q, const float *__restrict__ ddt_in,
+                 const float *__restrict__ dt, const float *__restrict__ A,
+                 const float *__restrict__ xdy, float *__restrict__ ddt, float *__restrict__ dA,
+                 float *__restrict__ dD, int64_t L, int H)
 {
-    const int lane = threadIdx.x % 32;
-    const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / 32;
-    if (w >= batch * H) return;
-    const int h = (int)(w % H);
-    const int64_t b = w / H;
+    __shared__ float wsum[kDecayThreads / 32];
+    __shared__ float red[2][kDecayThreads / 32];
+    const int h = (int)(blockIdx.x % H);
+    const int64_t b = blockIdx.x / H;
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    const int64_t per = (L + kDecayThreads - 1) / kDecayThreads;
+    const int64_t ta = min(L, threadIdx.x * per), te = min(L, ta + per);
+    const int64_t base = b * L * H + h;
+    float tot = 0.f;
+    for (int64_t t = ta; t < te; ++t) tot += q[base + t * H];
+    // exclusive suffix sum of the threads' totals: within the warp, then over the warps
+    float v = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_down_sync(0xffffffffu, v, o);
+        if (lane + o < 32) v += u;
+    }
+    if (lane == 0) wsum[warp] = v;   // the warp's total
+    __syncthreads();
+    float carry = v - tot;           // later threads of this warp
+    for (int j = warp + 1; j < kDecayThreads / 32; ++j) carry += wsum[j];
     const float Ah = A[h];
-    float carry = 0.f, sa = 0.f, sd = 0.f;
-    for (int64_t t0 = ((L - 1) / 32) * 32; t0 >= 0; t0 -= 32) {
-        const int64_t t = t0 + lane;
-        const int64_t i = (b * L + t) * H + h;
-        const float qv = t < L ? q[i] : 0.f;
-        // inclusive suffix sum within the tile (lane l sums lanes l..31), then the carry
-        float v = qv;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float u = __shfl_down_sync(0xffffffffu, v, o);
-            if (lane + o < 32) v += u;
-        }
-        const float dl = v + carry;
-        carry += __shfl_sync(0xffffffffu, v, 0);
-        if (t < L) {
-            ddt[i] = ddt_in[i] + Ah * dl;
-            sa = fmaf(dt[i], dl, sa);
-        }
-    }
-    for (int64_t i = lane; i < L * P; i += 32) {   // dD_h = sum_t <dy_t, x_t>
-        const int64_t t = i / P, p = i % P;
-        const int64_t off = ((b * L + t) * H + h) * P + p;
-        sd = fmaf(to_f32(dy[off]), to_f32(x[off]), sd);
+    float sa = 0.f, sd = 0.f;
+    for (int64_t t = te - 1; t >= ta; --t) {
+        const int64_t i = base + t * H;
+        carry += q[i];
+        ddt[i] = ddt_in[i] + Ah * carry;
+        sa = fmaf(dt[i], carry, sa);
+        sd += xdy[i];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -175,8 +191,18 @@ __global__ void bwd_decay_kernel(const float *__restrict__ q, const float *__res
         sd += __shfl_xor_sync(0xffffffffu, sd, o);
     }
     if (lane == 0) {
-        atomicAdd(&dA[h], sa);
-        atomicAdd(&dD[h], sd);
+        red[0][warp] = sa;
+        red[1][warp] = sd;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float a = 0.f, d = 0.f;
+        for (int j = 0; j < kDecayThreads / 32; ++j) {
+            a += red[0][j];
+            d += red[1][j];
+        }
+        atomicAdd(&dA[h], a);
+        atomicAdd(&dD[h], d);
     }
 }
 
@@ -220,25 +246,15 @@ unsigned grid_for(int64_t n) { return (unsigned)std::min<int64_t>((n + 255) / 25
 
 }  // namespace
 
-cudaError_t launch_gather(const void *in, bool in_bf16, void *out, bool out_bf16, int64_t batch,
-                          int64_t L, int rows_in, int rows_out, int E, bool reverse,
-                          cudaStream_t st)
+cudaError_t launch_gather(const bf16 *in, bf16 *out, int64_t batch, int64_t L, int rows_in,
+                          int rows_out, int E, bool reverse, cudaStream_t st)
 {
-    const int64_t n = batch * L * rows_out * E;
+    if (E % 8 != 0 || rows_in <= 0 || rows_out % rows_in != 0) return cudaErrorInvalidValue;
+    const int64_t n = batch * L * rows_out * (E / 8);
     if (n == 0) return cudaSuccess;
-    const unsigned g = grid_for(n);
-    if (in_bf16 && out_bf16)
-        gather_kernel<bf16, bf16><<<g, 256, 0, st>>>((const bf16 *)in, (bf16 *)out, batch, L,
-                                                     rows_in, rows_out, E, reverse);
-    else if (in_bf16)
-        gather_kernel<bf16, float><<<g, 256, 0, st>>>((const bf16 *)in, (float *)out, batch, L,
-                                                      rows_in, rows_out, E, reverse);
-    else if (out_bf16)
-        gather_kernel<float, bf16><<<g, 256, 0, st>>>((const float *)in, (bf16 *)out, batch, L,
-                                                      rows_in, rows_out, E, reverse);
-    else
-        gather_kernel<float, float><<<g, 256, 0, st>>>((const float *)in, (float *)out, batch, L,
-                                                       rows_in, rows_out, E, reverse);
+    gather8_kernel<<<grid_for(n), 256, 0, st>>>(reinterpret_cast<const uint4 *>(in),
+                                               reinterpret_cast<uint4 *>(out), batch, L, rows_in,
+                                               rows_out, E / 8, reverse);
     return cudaGetLastError();
 }
 
@@ -267,40 +283,31 @@ cudaError_t launch_transpose(const float *in, float *out, int64_t mats, int rows
     return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_tokens(const bf16 *dy, const float *dt, const float *D,
+cudaError_t launch_bwd_tokens(const bf16 *x, const bf16 *dy, const float *dt, const float *D,
                               const bf16 *gb_rev, const float *ydot, const float *ddt_in,
                               const float *dfinal, const float *fin_t, float *dx, float *q,
-                              int64_t batch, int64_t L, int H, int P, int N, cudaStream_t st)
+                              float *xdy, int64_t batch, int64_t L, int H, int P, int N,
+                              cudaStream_t st)
 {
-    const int64_t warps = batch * L * H;
-    if (warps == 0) return cudaSuccess;
-    bwd_tokens_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
-        dy, dt, D, gb_rev, ydot, ddt_in, dfinal, fin_t, dx, q, batch, L, H, P, N);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_head_dot(const float *in, const bf16 *v, float *out, int64_t batch, int64_t L,
-                            int H, int G, int N, bool reverse, cudaStream_t st)
-{
-    const int64_t warps = batch * L * H;
-    if (warps == 0) return cudaSuccess;
-    head_dot_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(in, v, out, batch, L,
-                                                                       H, G, N, reverse);
+    if (P != kTokLanes * 8) return cudaErrorInvalidValue;
+    const int64_t threads = batch * L * H * kTokLanes;
+    if (threads == 0) return cudaSuccess;
+    bwd_tokens_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+        x, dy, dt, D, gb_rev, ydot, ddt_in, dfinal, fin_t, dx, q, xdy, batch, L, H, N);
     return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_decay(const float *q, const float *ddt_in, const float *dt,
-                             const float *A, const bf16 *x, const bf16 *dy, float *ddt,
-                             float *dA, float *dD, int64_t batch, int64_t L, int H, int P,
-                             cudaStream_t st)
+                             const float *A, const float *xdy, float *ddt, float *dA, float *dD,
+                             int64_t batch, int64_t L, int H, cudaStream_t st)
 {
     cudaError_t e = cudaMemsetAsync(dA, 0, H * sizeof(float), st);
     if (e == cudaSuccess) e = cudaMemsetAsync(dD, 0, H * sizeof(float), st);
     if (e != cudaSuccess) return e;
-    const int64_t warps = batch * H;
-    if (warps == 0) return cudaSuccess;
-    bwd_decay_kernel<<<(unsigned)((warps * 32 + 127) / 128), 128, 0, st>>>(
-        q, ddt_in, dt, A, x, dy, ddt, dA, dD, batch, L, H, P);
+    const int64_t n = batch * H;
+    if (n == 0 || L == 0) return cudaSuccess;
+    bwd_decay_kernel<<<(unsigned)n, kDecayThreads, 0, st>>>(q, ddt_in, dt, A, xdy, ddt, dA, dD,
+                                                           L, H);
     return cudaGetLastError();
 }
 

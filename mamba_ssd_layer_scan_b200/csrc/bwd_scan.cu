@@ -1,0 +1,322 @@
+// The two float32 scans of the backward pass (dB and dC), specialised for their shape.
+//
+// Both are scans of the forward's kind with the head and state dimensions swapped: the state
+// is E x K = N x P (128 x 64) per (batch, head), the "x" operand x'' has E = N = 128 channels and
+// is shared by the heads of a group (it is B or C), the "B" and "C" operands B'', C'' have
+// K = P = 64 channels per head (x or dy):
+//
+//   chunk state   S_k[e][j] = sum_{r in k} exp(cs_last - cs_r) w_r x''_r[e] B''_r[j]
+//   chunk output  y_t[e]    = sum_{s <= t, s in k} exp(cs_t - cs_s) w_s (C''_t . B''_s) x''_s[e]
+//                           + exp(cs_t) sum_j S_in[e][j] C''_t[j]
+//
+// (the same chunked form as the forward: mohakchugh.is-a.dev "Mamba-2", Block Decomposition).
+// dB runs it on the time-reversed sequence (x'' = C, B'' = dy, C'' = x, unit weights, decays
+// shifted by one token), dC forward (x'' = B, B'' = x, C'' = dy, weights dt).  The operands are
+// read in place from the bf16 inputs (reversed rows, the group's row for x''); everything is
+// float32 from there on, because the decay gradient needs the outputs' dot products with B and C
+// to float32 accuracy (see backward.cu).  Each output row's dot product with the group's B or C
+// row is formed in the epilogue.
+//
+// Register tiling: the chunk-state kernel gives each of its 256 threads a 4 x 8 block of the
+// 128 x 64 state; the chunk-output kernel gives each thread 4 rows x 8 channels of the 64 x 128
+// output tile, and 4 x 4 of the 64 x 64 masked Gram matrix before that.  The channels of a
+// thread are two runs of 4 at e0 and 64 + e0, so that each 16-byte shared-memory load of a half
+// warp reads 256 contiguous bytes (two wavefronts, no bank conflict).
+#include "common.cuh"
+
+namespace ssd {
+namespace {
+
+constexpr int kQs = 64;     // chunk
+constexpr int kE = 128;     // x'' channels (dstate of the forward)
+constexpr int kK = 64;      // B'' / C'' channels (headdim of the forward)
+constexpr int kThreads = 256;
+constexpr int kTS = kQs + 4;   // row stride of the transposed [channel][token] tiles
+
+__device__ __forceinline__ void unpack8(const uint4 raw, float *v)
+{
+    const bf16 *p = reinterpret_cast<const bf16 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(p[i]);
+}
+
+__device__ __forceinline__ int64_t src_row(int64_t tau, int64_t L, bool rev)
+{
+    return rev ? L - 1 - tau : tau;
+}
+
+__global__ void __launch_bounds__(kThreads)
+bwd_chunk_state_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
+                       const float *__restrict__ w, const float *__restrict__ cs,
+                       float *__restrict__ states, int64_t L, int H, int G, int64_t nch, bool rev)
+{
+    __shared__ __align__(16) float xs[kQs][kE];
+    __shared__ __align__(16) float bs[kQs][kK];
+    const int h = (int)(blockIdx.x % H);
+    const int64_t k = (blockIdx.x / H) % nch, b = blockIdx.x / H / nch;
+    const int g = h / (H / G);
+    const int64_t t0 = k * kQs;
+    const int len = (int)min((int64_t)kQs, L - t0);
+    const float *csk = cs + ((b * nch + k) * H + h) * (int64_t)kQs;
+    const float cl = csk[len - 1];
+
+    for (int i = threadIdx.x; i < kQs * kE / 8; i += kThreads) {
+        const int r = i / (kE / 8), c8 = i % (kE / 8);
+        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (r < len) {
+            const int64_t s = src_row(t0 + r, L, rev);
+            unpack8(*reinterpret_cast<const uint4 *>(xg + ((b * L + s) * G + g) * kE + c8 * 8), v);
+        }
+        *reinterpret_cast<float4 *>(&xs[r][c8 * 8]) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4 *>(&xs[r][c8 * 8 + 4]) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+    for (int i = threadIdx.x; i < kQs * kK / 8; i += kThreads) {
+        const int r = i / (kK / 8), c8 = i % (kK / 8);
+        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (r < len) {
+            const int64_t tau = t0 + r, s = src_row(tau, L, rev);
+            const float f = __expf(cl - csk[r]) * (w ? w[(b * L + tau) * H + h] : 1.f);
+            unpack8(*reinterpret_cast<const uint4 *>(bh + ((b * L + s) * H + h) * kK + c8 * 8), v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] *= f;
+        }
+        *reinterpret_cast<float4 *>(&bs[r][c8 * 8]) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4 *>(&bs[r][c8 * 8 + 4]) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+    __syncthreads();
+
+    // thread: state rows e0..e0+3, columns kg*4..+3 and 32+kg*4..+3 (conflict-free float4s)
+    const int e0 = (threadIdx.x / 8) * 4, kg = threadIdx.x % 8;
+    float acc[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int r = 0; r < len; ++r) {
+        const float4 xv = *reinterpret_cast<const float4 *>(&xs[r][e0]);
+        const float4 b0 = *reinterpret_cast<const float4 *>(&bs[r][kg * 4]);
+        const float4 b1 = *reinterpret_cast<const float4 *>(&bs[r][32 + kg * 4]);
+        const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+        const float ba[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xa[i], ba[j], acc[i][j]);
+    }
+    float *out = states + ((b * nch + k) * H + h) * (int64_t)(kE * kK);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float *row = out + (e0 + i) * kK;
+        *reinterpret_cast<float4 *>(row + kg * 4) =
+            make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        *reinterpret_cast<float4 *>(row + 32 + kg * 4) =
+            make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+    }
+}
+
+struct ScanSmem {
+    float xs[kQs][kE];        // x'' rows
+    union {
+        float bT[kK][kTS];    // B'' * w transposed: bT[j][s] (until the Gram matrix is formed)
+        float pT[kQs][kTS];   // masked, decayed Gram matrix, transposed: pT[s][t]
+    };
+    float cT[kK][kTS];        // C'' transposed: cT[j][t]
+    float hT[kK][kE];         // entering state transposed: hT[j][e]
+    float css[kQs];           // chunk-local cumsum
+};
+static_assert(kK == kQs, "bT and pT share their storage");
+
+__global__ void __launch_bounds__(kThreads, 2)
+bwd_chunk_scan_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
+                      const bf16 *__restrict__ ch, const float *__restrict__ w,
+                      const float *__restrict__ cs, const float *__restrict__ hin,
+                      const bf16 *__restrict__ vg, float *__restrict__ ys,
+                      float *__restrict__ dot, int64_t L, int H, int G, int64_t nch, bool rev)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    ScanSmem &sm = *reinterpret_cast<ScanSmem *>(smem_raw);
+    const int h = (int)(blockIdx.x % H);
+    const int64_t k = (blockIdx.x / H) % nch, b = blockIdx.x / H / nch;
+    const int g = h / (H / G);
+    const int64_t t0 = k * kQs;
+    const int len = (int)min((int64_t)kQs, L - t0);
+    const float *csk = cs + ((b * nch + k) * H + h) * (int64_t)kQs;
+    const float *hk = hin + ((b * nch + k) * H + h) * (int64_t)(kE * kK);
+
+    if (threadIdx.x < kQs) sm.css[threadIdx.x] = threadIdx.x < len ? csk[threadIdx.x] : 0.f;
+    for (int i = threadIdx.x; i < kQs * kE / 8; i += kThreads) {
+        const int r = i / (kE / 8), c8 = i % (kE / 8);
+        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (r < len) {
+            const int64_t s = src_row(t0 + r, L, rev);
+            unpack8(*reinterpret_cast<const uint4 *>(xg + ((b * L + s) * G + g) * kE + c8 * 8), v);
+        }
+        *reinterpret_cast<float4 *>(&sm.xs[r][c8 * 8]) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4 *>(&sm.xs[r][c8 * 8 + 4]) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+    for (int i = threadIdx.x; i < kQs * kK / 8; i += kThreads) {
+        const int r = i % kQs, c8 = i / kQs;   // consecutive threads: consecutive tokens, so the
+                                               // transposed stores below hit distinct banks
+        float vb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float vc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (r < len) {
+            const int64_t tau = t0 + r, s = src_row(tau, L, rev);
+            const int64_t off = ((b * L + s) * H + h) * kK + c8 * 8;
+            unpack8(*reinterpret_cast<const uint4 *>(bh + off), vb);
+            unpack8(*reinterpret_cast<const uint4 *>(ch + off), vc);
+            const float f = w ? w[(b * L + tau) * H + h] : 1.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) vb[j] *= f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            sm.bT[c8 * 8 + j][r] = vb[j];
+            sm.cT[c8 * 8 + j][r] = vc[j];
+        }
+    }
+    for (int i = threadIdx.x; i < kE * kK / 4; i += kThreads) {
+        const int e = i % kE, j4 = i / kE;   // consecutive threads: consecutive e (no conflicts)
+        const float4 v = *reinterpret_cast<const float4 *>(hk + e * kK + j4 * 4);
+        sm.hT[j4 * 4 + 0][e] = v.x;
+        sm.hT[j4 * 4 + 1][e] = v.y;
+        sm.hT[j4 * 4 + 2][e] = v.z;
+        sm.hT[j4 * 4 + 3][e] = v.w;
+    }
+    __syncthreads();
+
+    // masked, decayed Gram matrix P[t][s] = (C''_t . w_s B''_s) exp(cs_t - cs_s), s <= t < len
+    {
+        const int ta = (threadIdx.x / 16) * 4, sa = (threadIdx.x % 16) * 4;
+        float gm[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) gm[i][j] = 0.f;
+        if (sa <= ta + 3) {
+            for (int j = 0; j < kK; ++j) {
+                const float4 c = *reinterpret_cast<const float4 *>(&sm.cT[j][ta]);
+                const float4 bb = *reinterpret_cast<const float4 *>(&sm.bT[j][sa]);
+                const float ca[4] = {c.x, c.y, c.z, c.w};
+                const float ba[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) gm[i][q] = fmaf(ca[i], ba[q], gm[i][q]);
+            }
+        }
+        __syncthreads();   // every read of bT is done before pT overwrites it
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int s = sa + q;
+            float o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = ta + i;
+                o[i] = (s <= t && t < len) ? gm[i][q] * __expf(sm.css[t] - sm.css[s]) : 0.f;
+            }
+            *reinterpret_cast<float4 *>(&sm.pT[s][ta]) = make_float4(o[0], o[1], o[2], o[3]);
+        }
+    }
+    __syncthreads();
+
+    // output rows tg..tg+3, channels e0..e0+3 and 64+e0..64+e0+3 (each 16-byte shared-memory load
+    // of a half warp covers 256 contiguous bytes): first the entering state's term
+    // exp(cs_t) sum_j C''_t[j] S_in[e][j], scaled in registers, then the masked P X on top
+    const int tg = (threadIdx.x / 16) * 4, e0 = (threadIdx.x % 16) * 4;
+    float acc[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int m = 0; m < 8; ++m) acc[i][m] = 0.f;
+    for (int j = 0; j < kK; ++j) {
+        const float4 c = *reinterpret_cast<const float4 *>(&sm.cT[j][tg]);
+        const float4 h0 = *reinterpret_cast<const float4 *>(&sm.hT[j][e0]);
+        const float4 h1 = *reinterpret_cast<const float4 *>(&sm.hT[j][64 + e0]);
+        const float ca[4] = {c.x, c.y, c.z, c.w};
+        const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc[i][m] = fmaf(ca[i], hv[m], acc[i][m]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float dec = __expf(sm.css[tg + i]);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) acc[i][m] *= dec;
+    }
+    const int smax = min(len, tg + 4);
+    for (int s = 0; s < smax; ++s) {
+        const float4 p = *reinterpret_cast<const float4 *>(&sm.pT[s][tg]);
+        const float4 x0 = *reinterpret_cast<const float4 *>(&sm.xs[s][e0]);
+        const float4 x1 = *reinterpret_cast<const float4 *>(&sm.xs[s][64 + e0]);
+        const float pa[4] = {p.x, p.y, p.z, p.w};
+        const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc[i][m] = fmaf(pa[i], xv[m], acc[i][m]);
+    }
+
+    // epilogue: rows written at their source token (forward time), dot with the group's V row
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = tg + i;
+        const bool valid = t < len;
+        const int64_t s = valid ? src_row(t0 + t, L, rev) : 0;
+        float d = 0.f;
+        if (valid) {
+            float *yrow = ys + ((b * L + s) * H + h) * (int64_t)kE + e0;
+            *reinterpret_cast<float4 *>(yrow) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+            *reinterpret_cast<float4 *>(yrow + 64) =
+                make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+            const bf16 *vrow = vg + ((b * L + s) * G + g) * (int64_t)kE + e0;
+            const uint2 r0 = *reinterpret_cast<const uint2 *>(vrow);
+            const uint2 r1 = *reinterpret_cast<const uint2 *>(vrow + 64);
+            // bf16 -> float32 is exact: the bf16 bits are the float's upper half
+            const float v[8] = {__uint_as_float(r0.x << 16), __uint_as_float(r0.x & 0xffff0000u),
+                                __uint_as_float(r0.y << 16), __uint_as_float(r0.y & 0xffff0000u),
+                                __uint_as_float(r1.x << 16), __uint_as_float(r1.x & 0xffff0000u),
+                                __uint_as_float(r1.y << 16), __uint_as_float(r1.y & 0xffff0000u)};
+#pragma unroll
+            for (int m = 0; m < 8; ++m) d = fmaf(acc[i][m], v[m], d);
+        }
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        if (valid && e0 == 0) dot[(b * L + s) * H + h] = d;
+    }
+}
+
+}  // namespace
+
+bool bwd_scan_supported(int P, int N) { return P == kK && N == kE; }
+
+cudaError_t launch_bwd_chunk_state(const bf16 *xg, const bf16 *bh, const float *w,
+                                   const float *cs, float *states, int64_t batch, int64_t L,
+                                   int H, int G, int64_t nch, bool rev, cudaStream_t st)
+{
+    const int64_t n = batch * nch * H;
+    if (n == 0) return cudaSuccess;
+    bwd_chunk_state_kernel<<<(unsigned)n, kThreads, 0, st>>>(xg, bh, w, cs, states, L, H, G, nch,
+                                                             rev);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_chunk_scan(const bf16 *xg, const bf16 *bh, const bf16 *ch, const float *w,
+                                  const float *cs, const float *hin, const bf16 *vg, float *ys,
+                                  float *dot, int64_t batch, int64_t L, int H, int G,
+                                  int64_t nch, bool rev, cudaStream_t st)
+{
+    const int64_t n = batch * nch * H;
+    if (n == 0) return cudaSuccess;
+    const int smem = (int)sizeof(ScanSmem);
+    cudaError_t e = cudaFuncSetAttribute(bwd_chunk_scan_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    bwd_chunk_scan_kernel<<<(unsigned)n, kThreads, smem, st>>>(xg, bh, ch, w, cs, hin, vg, ys,
+                                                                dot, L, H, G, nch, rev);
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

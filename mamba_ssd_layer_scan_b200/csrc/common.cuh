@@ -158,11 +158,10 @@ cudaError_t launch_seqpar_combine(const float *h_loc_all, const float *logdec_al
                                   int64_t BH, int PN, cudaStream_t st);
 
 // ---- backward helpers (backward.cu)
-// out[b][t][r][e] = in[b][src][r_in][e]: src = L-1-t when `reverse`, r_in = r / (rows_out /
-// rows_in) (heads reading their group's row); converts the element type.
-cudaError_t launch_gather(const void *in, bool in_bf16, void *out, bool out_bf16, int64_t batch,
-                          int64_t L, int rows_in, int rows_out, int E, bool reverse,
-                          cudaStream_t st);
+// bf16 rows of E (a multiple of 8): out[b][t][r][:] = in[b][src][r_in][:], src = L-1-t when
+// `reverse`, r_in = r / (rows_out / rows_in) (heads reading their group's row).
+cudaError_t launch_gather(const bf16 *in, bf16 *out, int64_t batch, int64_t L, int rows_in,
+                          int rows_out, int E, bool reverse, cudaStream_t st);
 // dt' for the time-reversed adjoint scan: dt'[b][t][h] = dt[b][L-t][h] for t >= 1, 0 for t = 0.
 cudaError_t launch_reverse_shift_dt(const float *dt, float *out, int64_t batch, int64_t L, int H,
                                    cudaStream_t st);
@@ -170,21 +169,31 @@ cudaError_t launch_fill(float *out, float value, int64_t n, cudaStream_t st);
 // per (b, h) matrix of rows x cols: out = in^T (in [.][rows][cols] -> out [.][cols][rows])
 cudaError_t launch_transpose(const float *in, float *out, int64_t mats, int rows, int cols,
                              cudaStream_t st);
-// dx[b][t][h][p] = D_h dy + dt[b][t][h] gb[b][L-1-t][h][p];
+// dx[b][t][h][p] = D_h dy + dt[b][t][h] gb[b][L-1-t][h][p];  xdy[b][t][h] = <x, dy>;
 // q[b][t][h] = ydot - dt ddt_in (+ <dfinal, final> at t = L-1; fin_t is the final state (n, p))
-cudaError_t launch_bwd_tokens(const bf16 *dy, const float *dt, const float *D,
+cudaError_t launch_bwd_tokens(const bf16 *x, const bf16 *dy, const float *dt, const float *D,
                               const bf16 *gb_rev, const float *ydot, const float *ddt_in,
                               const float *dfinal, const float *fin_t, float *dx, float *q,
-                              int64_t batch, int64_t L, int H, int P, int N, cudaStream_t st);
-// out[b][t][h] = sum_n in[b][src(t)][h][n] v[b][t][g(h)][n], src(t) = L-1-t when `reverse`
-cudaError_t launch_head_dot(const float *in, const bf16 *v, float *out, int64_t batch, int64_t L,
-                            int H, int G, int N, bool reverse, cudaStream_t st);
+                              float *xdy, int64_t batch, int64_t L, int H, int P, int N,
+                              cudaStream_t st);
 // dl = reverse cumsum of q over t per (b, h); ddt = ddt_in + A_h dl; dA_h = sum dt dl;
-// dD_h = sum <dy, x>
+// dD_h = sum xdy (both summed over the batch)
 cudaError_t launch_bwd_decay(const float *q, const float *ddt_in, const float *dt,
-                             const float *A, const bf16 *x, const bf16 *dy, float *ddt,
-                             float *dA, float *dD, int64_t batch, int64_t L, int H, int P,
-                             cudaStream_t st);
+                             const float *A, const float *xdy, float *ddt, float *dA, float *dD,
+                             int64_t batch, int64_t L, int H, cudaStream_t st);
+// The backward's two float32 scans for P = 64, N = 128 (bwd_scan.cu): x'' (batch, L, G, 128)
+// bf16, B'' and C'' (batch, L, H, 64) bf16, all read at row L-1-tau for scan step tau when
+// `rev`; w (batch, L, H) in scan order, null = 1; cs (batch, nch, H, 64) chunk-local cumsum in
+// scan order; states / hin (batch, nch, H, 128, 64).  The scan writes its output row tau at
+// ys[b][src(tau)][h][:] and its dot product with vg[b][src(tau)][g(h)][:] at dot[b][src(tau)][h].
+bool bwd_scan_supported(int P, int N);
+cudaError_t launch_bwd_chunk_state(const bf16 *xg, const bf16 *bh, const float *w,
+                                   const float *cs, float *states, int64_t batch, int64_t L,
+                                   int H, int G, int64_t nch, bool rev, cudaStream_t st);
+cudaError_t launch_bwd_chunk_scan(const bf16 *xg, const bf16 *bh, const bf16 *ch, const float *w,
+                                  const float *cs, const float *hin, const bf16 *vg, float *ys,
+                                  float *dot, int64_t batch, int64_t L, int H, int G,
+                                  int64_t nch, bool rev, cudaStream_t st);
 // out[b][t][g][n] = sum_{h in g} w[b][t][h] in[b][src(t)][h][n] (w = dt, or 1 when null)
 cudaError_t launch_group_sum(const float *in, const float *w, float *out, int64_t batch,
                              int64_t L, int H, int G, int N, bool reverse, cudaStream_t st);

@@ -419,9 +419,9 @@ constexpr int kBwdSimtChunk = 64;   // chunk of the two CUDA-core scans (head di
 
 struct BwdLayout {
     size_t r_ws, s_ws;                          // tensor-core and CUDA-core scan workspaces
-    size_t dyr, Cr, Br, dtr, zerosD, gb, Fr, ones;
-    size_t xs, Bs, Cs, inits, ys, fin_t;        // the CUDA-core scans' operands (reused)
-    size_t ydot, ddt_in, q, total;
+    size_t dyr, Cr, Br, dtr, zerosD, gb, Fr;
+    size_t inits, ys, fin_t;                    // the CUDA-core scans' state and output (reused)
+    size_t ydot, ddt_in, q, xdy, total;
     size_t r_bytes, s_bytes;
 };
 
@@ -454,16 +454,13 @@ BwdLayout bwd_layout(const ssd_shape *s, int Q)
     w.zerosD = take(H * 4);
     w.gb = take(b * L * H * P * 2);
     w.Fr = take(b * H * P * N * 4);
-    w.ones = take(b * L * H * 4);
-    w.xs = take(b * L * H * N * 4);
-    w.Bs = take(b * L * H * P * 4);
-    w.Cs = take(b * L * H * P * 4);
     w.inits = take(b * H * N * P * 4);
     w.ys = take(b * L * H * N * 4);
     w.fin_t = take(b * H * N * P * 4);
     w.ydot = take(b * L * H * 4);
     w.ddt_in = take(b * L * H * 4);
     w.q = take(b * L * H * 4);
+    w.xdy = take(b * L * H * 4);
     w.total = o;
     return w;
 }
@@ -511,11 +508,11 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
     }
     if (!x || !dt || !A || !B || !C || !D || !dy || !dx || !ddt || !dB || !dC || !workspace)
         return fail(SSD_ERR_INVALID_ARG, "inputs, dy and the gradient buffers must be non-NULL");
-    if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(dy) ||
+    if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(dy) || !aligned16(dx) ||
         (init_state && !aligned16(init_state)) || (dfinal && !aligned16(dfinal)) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-        return fail(SSD_ERR_INVALID_ARG,
-                    "x, B, C, dy and the states must be 16-byte, the workspace 256-byte aligned");
+        return fail(SSD_ERR_INVALID_ARG, "x, B, C, dy, dx and the states must be 16-byte, the "
+                                         "workspace 256-byte aligned");
     const BwdLayout wl = bwd_layout(&s, Q);
     if (workspace_bytes < wl.total)
         return fail(SSD_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu",
@@ -539,9 +536,12 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
     float *states_r = reinterpret_cast<float *>(rw + rl.states);
     ssd::bf16 *hin_r = reinterpret_cast<ssd::bf16 *>(rw + rl.hin_bf16);
     const char *why = "";
-    if ((e = ssd::launch_gather(dy, true, Hh(wl.dyr), true, b, L, H, H, P, true, cst)) ||
-        (e = ssd::launch_gather(C, true, Hh(wl.Cr), true, b, L, G, G, N, true, cst)) ||
-        (e = ssd::launch_gather(B, true, Hh(wl.Br), true, b, L, G, G, N, true, cst)) ||
+    using ssd::bf16;
+    const bf16 *xb = static_cast<const bf16 *>(x), *dyb = static_cast<const bf16 *>(dy);
+    const bf16 *Bb = static_cast<const bf16 *>(B), *Cb = static_cast<const bf16 *>(C);
+    if ((e = ssd::launch_gather(dyb, Hh(wl.dyr), b, L, H, H, P, true, cst)) ||
+        (e = ssd::launch_gather(Cb, Hh(wl.Cr), b, L, G, G, N, true, cst)) ||
+        (e = ssd::launch_gather(Bb, Hh(wl.Br), b, L, G, G, N, true, cst)) ||
         (e = ssd::launch_reverse_shift_dt(dt, F(wl.dtr), b, L, H, cst)))
         return cuda_fail(e, "reverse inputs");
     e = ssd::launch_chunk_cumsum(F(wl.dtr), A, cs_r, dtc_r, status, b, L, H, Q, nch, cst,
@@ -560,9 +560,9 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
         return cuda_fail(e, "dinit");
 
     // 2. dB and dC: scans with head dimension N and state dimension P on CUDA cores (float32),
-    // summed over the heads of each group.  Their per-head outputs also give, contracted with
-    // B (resp. C), the two float32 dot products of the decay gradient: <x_t, g_t B_t> and
-    // <dy_t, y_t - D x_t>.
+    // reading the bf16 operands in place, summed over the heads of each group.  Their per-head
+    // outputs also give, contracted with B (resp. C), the two float32 dot products of the decay
+    // gradient: <x_t, g_t B_t> and <dy_t, y_t - D x_t>.
     const ssd_shape t = simt_shape(s);
     const int Qs = kBwdSimtChunk;
     const int64_t nchs = (L + Qs - 1) / Qs;
@@ -570,49 +570,37 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
     char *sw = ws + wl.s_ws;
     float *cs_s = reinterpret_cast<float *>(sw + sl.cs);
     float *states_s = reinterpret_cast<float *>(sw + sl.states);
-    if ((e = ssd::launch_fill(F(wl.ones), 1.f, b * L * H, cst)))
-        return cuda_fail(e, "fill");
     for (int pass = 0; pass < 2; ++pass) {   // 0: dB (reversed), 1: dC (forward)
         const bool rev = pass == 0;
         const float *init_s = rev ? dfinal : init_state;
-        if ((e = ssd::launch_gather(rev ? C : B, true, F(wl.xs), false, b, L, G, H, N, rev,
-                                    cst)) ||
-            (e = ssd::launch_gather(rev ? dy : x, true, F(wl.Bs), false, b, L, H, H, P, rev,
-                                    cst)) ||
-            (e = ssd::launch_gather(rev ? x : dy, true, F(wl.Cs), false, b, L, H, H, P, rev,
-                                    cst)))
-            return cuda_fail(e, "scan operands");
+        const float *w_s = rev ? nullptr : dt;
         if (init_s && (e = ssd::launch_transpose(init_s, F(wl.inits), b * H, P, N, cst)))
             return cuda_fail(e, "transpose");
-        const float *w_s = rev ? F(wl.ones) : dt;
         e = ssd::launch_chunk_cumsum(rev ? F(wl.dtr) : dt, A, cs_s, nullptr, nullptr, b, L, H,
                                      Qs, nchs, cst);
         if (e == cudaSuccess)
-            e = ssd::launch_chunk_state_simt(false, F(wl.xs), w_s, F(wl.Bs), cs_s, states_s, b, L,
-                                             H, H, N, P, Qs, nchs, cst);
+            e = ssd::launch_bwd_chunk_state(rev ? Cb : Bb, rev ? dyb : xb, w_s, cs_s, states_s, b,
+                                            L, H, G, nchs, rev, cst);
         if (e == cudaSuccess)
             e = ssd::launch_state_passing(states_s, cs_s, init_s ? F(wl.inits) : nullptr,
                                           rev ? nullptr : F(wl.fin_t), nullptr, b, H, N, P, Qs,
                                           nchs, cst);
         if (e == cudaSuccess)
-            e = ssd::launch_chunk_scan_simt(false, F(wl.xs), w_s, F(wl.Bs), F(wl.Cs), cs_s,
-                                            states_s, zerosD, F(wl.ys), b, L, H, H, N, P, Qs,
-                                            nchs, cst);
+            e = ssd::launch_bwd_chunk_scan(rev ? Cb : Bb, rev ? dyb : xb, rev ? xb : dyb, w_s,
+                                           cs_s, states_s, rev ? Bb : Cb, F(wl.ys),
+                                           F(rev ? wl.ddt_in : wl.ydot), b, L, H, G, nchs, rev,
+                                           cst);
         if (e == cudaSuccess)
             e = ssd::launch_group_sum(F(wl.ys), rev ? dt : nullptr, rev ? dB : dC, b, L, H, G, N,
-                                      rev, cst);
-        if (e == cudaSuccess)
-            e = ssd::launch_head_dot(F(wl.ys), (const ssd::bf16 *)(rev ? B : C),
-                                     F(rev ? wl.ddt_in : wl.ydot), b, L, H, G, N, rev, cst);
+                                      false, cst);
         if (e != cudaSuccess) return cuda_fail(e, rev ? "dB scan" : "dC scan");
     }
 
     // 3. dx, the decay-gradient terms and their reverse cumsum: ddt, dA, dD
-    if ((e = ssd::launch_bwd_tokens((const ssd::bf16 *)dy, dt, D, Hh(wl.gb), F(wl.ydot),
-                                    F(wl.ddt_in), dfinal, F(wl.fin_t), dx, F(wl.q), b, L, H, P,
-                                    N, cst)) ||
-        (e = ssd::launch_bwd_decay(F(wl.q), F(wl.ddt_in), dt, A, (const ssd::bf16 *)x,
-                                   (const ssd::bf16 *)dy, ddt, dA, dD, b, L, H, P, cst)))
+    if ((e = ssd::launch_bwd_tokens(xb, dyb, dt, D, Hh(wl.gb), F(wl.ydot), F(wl.ddt_in), dfinal,
+                                    F(wl.fin_t), dx, F(wl.q), F(wl.xdy), b, L, H, P, N, cst)) ||
+        (e = ssd::launch_bwd_decay(F(wl.q), F(wl.ddt_in), dt, A, F(wl.xdy), ddt, dA, dD, b, L, H,
+                                   cst)))
         return cuda_fail(e, "token gradients");
     return SSD_OK;
 }
