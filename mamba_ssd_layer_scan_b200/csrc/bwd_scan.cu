@@ -114,19 +114,30 @@ bwd_chunk_state_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
     }
 }
 
+// x'' and C'' are bf16 inputs and stay bf16 here (exact); B'' * w, the Gram matrix and the
+// entering state are float32.  74 KB: three CTAs per SM.
 struct ScanSmem {
-    float xs[kQs][kE];        // x'' rows
+    bf16 xs[kQs][kE];         // x'' rows
     union {
         float bT[kK][kTS];    // B'' * w transposed: bT[j][s] (until the Gram matrix is formed)
         float pT[kQs][kTS];   // masked, decayed Gram matrix, transposed: pT[s][t]
     };
-    float cT[kK][kTS];        // C'' transposed: cT[j][t]
+    bf16 cT[kK][kTS];         // C'' transposed: cT[j][t]
     float hT[kK][kE];         // entering state transposed: hT[j][e]
     float css[kQs];           // chunk-local cumsum
 };
+
+// four bf16 (8 bytes) -> float32, exactly: the bf16 bits are the float's upper half
+__device__ __forceinline__ void bf16x4_to_f32(const uint2 r, float *v)
+{
+    v[0] = __uint_as_float(r.x << 16);
+    v[1] = __uint_as_float(r.x & 0xffff0000u);
+    v[2] = __uint_as_float(r.y << 16);
+    v[3] = __uint_as_float(r.y & 0xffff0000u);
+}
 static_assert(kK == kQs, "bT and pT share their storage");
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 3)
 bwd_chunk_scan_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
                       const bf16 *__restrict__ ch, const float *__restrict__ w,
                       const float *__restrict__ cs, const float *__restrict__ hin,
@@ -146,32 +157,32 @@ bwd_chunk_scan_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
     if (threadIdx.x < kQs) sm.css[threadIdx.x] = threadIdx.x < len ? csk[threadIdx.x] : 0.f;
     for (int i = threadIdx.x; i < kQs * kE / 8; i += kThreads) {
         const int r = i / (kE / 8), c8 = i % (kE / 8);
-        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (r < len) {
             const int64_t s = src_row(t0 + r, L, rev);
-            unpack8(*reinterpret_cast<const uint4 *>(xg + ((b * L + s) * G + g) * kE + c8 * 8), v);
+            v = *reinterpret_cast<const uint4 *>(xg + ((b * L + s) * G + g) * kE + c8 * 8);
         }
-        *reinterpret_cast<float4 *>(&sm.xs[r][c8 * 8]) = make_float4(v[0], v[1], v[2], v[3]);
-        *reinterpret_cast<float4 *>(&sm.xs[r][c8 * 8 + 4]) = make_float4(v[4], v[5], v[6], v[7]);
+        *reinterpret_cast<uint4 *>(&sm.xs[r][c8 * 8]) = v;
     }
     for (int i = threadIdx.x; i < kQs * kK / 8; i += kThreads) {
         const int r = i % kQs, c8 = i / kQs;   // consecutive threads: consecutive tokens, so the
                                                // transposed stores below hit distinct banks
         float vb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        float vc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        uint4 rc = make_uint4(0u, 0u, 0u, 0u);
         if (r < len) {
             const int64_t tau = t0 + r, s = src_row(tau, L, rev);
             const int64_t off = ((b * L + s) * H + h) * kK + c8 * 8;
             unpack8(*reinterpret_cast<const uint4 *>(bh + off), vb);
-            unpack8(*reinterpret_cast<const uint4 *>(ch + off), vc);
+            rc = *reinterpret_cast<const uint4 *>(ch + off);
             const float f = w ? w[(b * L + tau) * H + h] : 1.f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) vb[j] *= f;
         }
+        const bf16 *pc = reinterpret_cast<const bf16 *>(&rc);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             sm.bT[c8 * 8 + j][r] = vb[j];
-            sm.cT[c8 * 8 + j][r] = vc[j];
+            sm.cT[c8 * 8 + j][r] = pc[j];
         }
     }
     for (int i = threadIdx.x; i < kE * kK / 4; i += kThreads) {
@@ -194,9 +205,9 @@ bwd_chunk_scan_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
             for (int j = 0; j < 4; ++j) gm[i][j] = 0.f;
         if (sa <= ta + 3) {
             for (int j = 0; j < kK; ++j) {
-                const float4 c = *reinterpret_cast<const float4 *>(&sm.cT[j][ta]);
+                float ca[4];
+                bf16x4_to_f32(*reinterpret_cast<const uint2 *>(&sm.cT[j][ta]), ca);
                 const float4 bb = *reinterpret_cast<const float4 *>(&sm.bT[j][sa]);
-                const float ca[4] = {c.x, c.y, c.z, c.w};
                 const float ba[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
@@ -229,10 +240,10 @@ bwd_chunk_scan_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
 #pragma unroll
         for (int m = 0; m < 8; ++m) acc[i][m] = 0.f;
     for (int j = 0; j < kK; ++j) {
-        const float4 c = *reinterpret_cast<const float4 *>(&sm.cT[j][tg]);
+        float ca[4];
+        bf16x4_to_f32(*reinterpret_cast<const uint2 *>(&sm.cT[j][tg]), ca);
         const float4 h0 = *reinterpret_cast<const float4 *>(&sm.hT[j][e0]);
         const float4 h1 = *reinterpret_cast<const float4 *>(&sm.hT[j][64 + e0]);
-        const float ca[4] = {c.x, c.y, c.z, c.w};
         const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -248,10 +259,10 @@ bwd_chunk_scan_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
     const int smax = min(len, tg + 4);
     for (int s = 0; s < smax; ++s) {
         const float4 p = *reinterpret_cast<const float4 *>(&sm.pT[s][tg]);
-        const float4 x0 = *reinterpret_cast<const float4 *>(&sm.xs[s][e0]);
-        const float4 x1 = *reinterpret_cast<const float4 *>(&sm.xs[s][64 + e0]);
         const float pa[4] = {p.x, p.y, p.z, p.w};
-        const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        float xv[8];
+        bf16x4_to_f32(*reinterpret_cast<const uint2 *>(&sm.xs[s][e0]), xv);
+        bf16x4_to_f32(*reinterpret_cast<const uint2 *>(&sm.xs[s][64 + e0]), xv + 4);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
