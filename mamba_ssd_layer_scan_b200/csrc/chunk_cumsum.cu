@@ -27,6 +27,8 @@ chunk_cumsum_kernel(const float *__restrict__ dt, const float *__restrict__ A,
                     int64_t seqlen, int H, int Q, int64_t nchunks, const int2 *__restrict__ tab,
                     bool unit_weights)
 {
+    griddep_wait();               // nothing of an earlier kernel is touched before this
+    griddep_launch_dependents();
     // First kernel of every scan: clears the workspace status word the later kernels may set.
     if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
     extern __shared__ float tile[];  // [Q][kHeadTile + 1]
@@ -99,9 +101,8 @@ cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, floa
 {
     const unsigned grid = (unsigned)(((nheads + kHeadTile - 1) / kHeadTile) * nchunks * batch);
     const size_t smem = (size_t)Q * (kHeadTile + 1) * sizeof(float);
-    chunk_cumsum_kernel<<<grid, kThreads, smem, st>>>(dt, A, cs, dtc, status, seqlen, nheads,
-                                                      Q, nchunks, tab, unit_weights);
-    return cudaGetLastError();
+    return launch_pdl(chunk_cumsum_kernel, grid, kThreads, smem, st, dt, A, cs, dtc, status,
+                      seqlen, nheads, Q, nchunks, tab, unit_weights);
 }
 
 cudaError_t launch_fill_final(const float *init, float *final_state, int64_t n,

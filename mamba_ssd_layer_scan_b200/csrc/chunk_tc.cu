@@ -124,6 +124,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (threadIdx.x == 0) griddep_launch_dependents();
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort = &sm.abort;
 
@@ -136,6 +137,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_arrive_expect_tx(&sm.bar_b, 2u * Q * kRowBytes);
             for (int a = 0; a < 2; ++a)   // boxes of Q rows
                 tma_load_4d(&sm.Bs[a][0], &tm_b, &sm.bar_b, 64 * a, g, (int)t0, (int)b);
+            griddep_wait();   // cs / dt come from the cumsum kernel
             for (int j = 0; j < nh; ++j) {
                 const int s = j % kStateStages;
                 const uint32_t use = j / kStateStages;
@@ -661,6 +663,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (threadIdx.x == 0) griddep_launch_dependents();
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort = &sm.abort;
 
@@ -679,6 +682,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 for (int r = 0; r <= T; ++r)
                     tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
                                 64 * a, g, (int)(t0 + kTileRows * r), (int)b);
+            griddep_wait();   // cs / dt and the entering states come from earlier kernels
         }
         for (int j = 0; lane == 0 && j < nh; ++j) {   // lane 0 alone runs the loop
             const int h = h0 + j;
@@ -1102,11 +1106,9 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk state: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb);
-    chunk_state_tc_kernel<<<grid, kStateThreads, smem, st>>>(mx, mb, dtc, cs, states, status,
-                                                             H, G, Q, nchunks, nhb, hpc, seqlen,
-                                                             tab);
     *why = "chunk state (tcgen05) launch";
-    return cudaGetLastError();
+    return launch_pdl(chunk_state_tc_kernel, grid, kStateThreads, smem, st, mx, mb, dtc, cs,
+                      states, status, H, G, Q, nchunks, nhb, hpc, seqlen, tab);
 }
 
 // The fused chunk state + state passing kernel walks the chunks of a (batch, group, 3 heads)
@@ -1172,10 +1174,9 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk scan: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb * (Q / kTileRows));
-    kern<<<grid, kScanThreads, smem, st>>>(mx, mb, mc, mx2, mz, hin, dtc, cs, D, y, status, seqlen,
-                                           H, G, Q, nchunks, nhb, hpc, tab, z);
     *why = "chunk scan (tcgen05) launch";
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, kScanThreads, smem, st, mx, mb, mc, mx2, mz, hin, dtc, cs, D, y,
+                      status, seqlen, H, G, Q, nchunks, nhb, hpc, tab, z);
 }
 
 }  // namespace ssd

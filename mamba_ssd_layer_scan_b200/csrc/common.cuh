@@ -18,6 +18,39 @@ template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __f
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Programmatic dependent launch.  The four kernels of the chunked scan (cumsum, chunk state,
+// state passing, chunk scan) are launched so that each may start while its predecessor in the
+// stream is still running: a kernel calls griddep_launch_dependents() once its CTAs are resident,
+// and its successor calls griddep_wait() before its first access to anything an earlier kernel
+// of the stream writes (the wait returns when the predecessor grid has completed and its memory
+// is visible; without a programmatic predecessor it returns at once).  The scan's own inputs (x,
+// B, C, z, D) are never written by these kernels and may be read before the wait.  Since every
+// kernel of the chain waits before it writes anything, completion is transitive: when a wait
+// returns, every earlier kernel of the stream has completed.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch `kern` on `st` with programmatic stream serialisation (see above).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args &&...args)
+{
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // The dt the recurrence uses when the block's raw projection is passed: + bias, then softplus
 // log(1 + exp(v)) (equal to v in float32 for v > 20), then the clamp to [lo, hi]; each optional.
 __device__ __forceinline__ float dt_transform(float v, const float *bias, int h, bool softplus,

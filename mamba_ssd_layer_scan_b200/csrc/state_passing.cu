@@ -27,6 +27,8 @@ state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
                      bf16 *__restrict__ hin, int H, int PN, int Q, int64_t nchunks,
                      const int32_t *__restrict__ cstart)
 {
+    griddep_wait();   // the chunk states come from the previous kernel
+    griddep_launch_dependents();
     const int nblk = (PN / 4 + kThreads - 1) / kThreads;
     const int64_t v = (blockIdx.x % nblk) * (int64_t)kThreads + threadIdx.x;  // float4 index
     // b: batch row, or the packed sequence when cstart is given (its chunks are
@@ -91,15 +93,10 @@ cudaError_t launch_state_passing(float *states, const float *cs, const float *in
 {
     const int PN = P * N;  // multiple of 32 (N is)
     const unsigned grid = (unsigned)(((PN / 4 + kThreads - 1) / kThreads) * H * batch);
-    if (hin_bf16)
-        state_passing_kernel<true><<<grid, kThreads, 0, st>>>(states, cs, init, final_state,
-                                                              hin_bf16, H, PN, Q, nchunks,
-                                                              nullptr);
-    else
-        state_passing_kernel<false><<<grid, kThreads, 0, st>>>(states, cs, init, final_state,
-                                                               nullptr, H, PN, Q, nchunks,
-                                                               nullptr);
-    return cudaGetLastError();
+    const int32_t *none = nullptr;
+    return launch_pdl(hin_bf16 ? state_passing_kernel<true> : state_passing_kernel<false>, grid,
+                      kThreads, 0, st, states, cs, init, final_state, hin_bf16, H, PN, Q, nchunks,
+                      none);
 }
 
 cudaError_t launch_state_passing_varlen(float *states, const float *cs, const float *init,
@@ -109,15 +106,9 @@ cudaError_t launch_state_passing_varlen(float *states, const float *cs, const fl
 {
     const int PN = P * N;
     const unsigned grid = (unsigned)(((PN / 4 + kThreads - 1) / kThreads) * H * (int64_t)nseq);
-    if (hin_bf16)
-        state_passing_kernel<true><<<grid, kThreads, 0, st>>>(states, cs, init, final_state,
-                                                              hin_bf16, H, PN, Q, nchunks,
-                                                              cstart);
-    else
-        state_passing_kernel<false><<<grid, kThreads, 0, st>>>(states, cs, init, final_state,
-                                                               nullptr, H, PN, Q, nchunks,
-                                                               cstart);
-    return cudaGetLastError();
+    return launch_pdl(hin_bf16 ? state_passing_kernel<true> : state_passing_kernel<false>, grid,
+                      kThreads, 0, st, states, cs, init, final_state, hin_bf16, H, PN, Q, nchunks,
+                      cstart);
 }
 
 }  // namespace ssd

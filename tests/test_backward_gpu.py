@@ -126,3 +126,29 @@ def test_backward_unsupported_shape_rejected(cuda_device):
     t = torch_inputs(inp, cuda_device)
     with pytest.raises(ssd.SSDError):
         ssd.chunk_scan_bwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], t["x"].clone(), 64)
+
+
+def test_backward_empty_sequence(cuda_device):
+    """No token: the final state is the initial state, so dinit = dfinal exactly and every other
+    gradient is empty or zero."""
+    import torch
+    w = configs.SSD_370M.with_(batch=2, seqlen=0, nheads=4, init_state=True, seed=82)
+    inp = inputs.make_inputs(w)
+    gin = inputs.make_grad_inputs(w)
+    g = _run(torch, inp, gin, 256, cuda_device)
+    assert np.array_equal(g["dinit"], gin.dfinal)
+    assert not g["dA"].any() and not g["dD"].any()
+    for k in ("dx", "ddt", "dB", "dC"):
+        assert g[k].size == 0, k
+    g = _run(torch, inp, gin, 256, cuda_device, with_dfinal=False)
+    assert not g["dinit"].any()
+
+
+def test_backward_empty_batch(cuda_device):
+    import torch
+    w = configs.SSD_370M.with_(batch=0, seqlen=300, nheads=4, seed=83)
+    inp = inputs.make_inputs(w)
+    gin = inputs.make_grad_inputs(w)
+    g = _run(torch, inp, gin, 256, cuda_device, with_init=False)
+    assert not g["dA"].any() and not g["dD"].any()
+    assert g["dx"].size == 0 and g["dinit"].size == 0
