@@ -4,10 +4,17 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / r
 import this package.  It wraps ``ssd_oracle.c`` (the token-by-token recurrence, see that file for
 the definition and its sources) through ctypes and never touches the CUDA library.
 
-Parity status: pinned.  ``tests/test_oracle_pins.py`` checks it against the explicit
-semiseparable matrix form on tiny inputs, a hand-worked example, closed forms for N = P = 1, the
-low-rank property of off-diagonal blocks, and invariances (dt = 0 padding, split/resume,
-linearity).
+Parity status: pinned.  ``tests/test_oracle_pins.py`` checks it against:
+
+- the explicit semiseparable matrix form on tiny inputs;
+- a hand-worked example;
+- closed forms for N = P = 1;
+- the low-rank property of off-diagonal blocks;
+- invariances (dt = 0 padding, split/resume, linearity).
+
+The block, varlen and decode variants are pinned by closed forms and by equalities with the
+pinned scan.  The backward (``ssd_scan_bwd``) is pinned element by element against central
+differences of the forward, and against a one-token closed form.
 """
 from __future__ import annotations
 
