@@ -469,8 +469,9 @@ ssd_status check_bwd(const ssd_shape *s, int Q)
 {
     ssd_status st = check_shape(s, true);
     if (st != SSD_OK) return st;
-    if (!valid_chunk(Q) || !ssd::tc_supported(s->dtype == SSD_BF16, (int)s->headdim,
-                                              (int)s->dstate, Q))
+    if (!valid_chunk(Q) ||
+        !ssd::tc_supported(s->dtype == SSD_BF16, (int)s->headdim, (int)s->dstate, Q) ||
+        !ssd::bwd_scan_supported((int)s->headdim, (int)s->dstate))
         return fail(SSD_ERR_UNSUPPORTED,
                     "the backward pass runs for the tensor-core shapes: bf16, headdim 64, "
                     "dstate 128, chunk_size 128 or 256");
