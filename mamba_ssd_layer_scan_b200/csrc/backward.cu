@@ -89,10 +89,9 @@ __global__ void bwd_tokens_kernel(const bf16 *__restrict__ x, const bf16 *__rest
                                   const bf16 *__restrict__ gb_rev,
                                   const float *__restrict__ ydot,
                                   const float *__restrict__ ddt_in,
-                                  const float *__restrict__ dfinal,
-                                  const float *__restrict__ fin_t, float *__restrict__ dx,
+                                  const float *__restrict__ fdot, float *__restrict__ dx,
                                   float *__restrict__ q, float *__restrict__ xdy, int64_t batch,
-                                  int64_t L, int H, int N)
+                                  int64_t L, int H)
 {
     constexpr int P = kTokLanes * 8;
     const int64_t gid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
@@ -126,21 +125,38 @@ __global__ void bwd_tokens_kernel(const bf16 *__restrict__ x, const bf16 *__rest
         for (int i = 0; i < 8; ++i) o[i] = fmaf(Dh, dyv[i], dth * gv[i]);
         *reinterpret_cast<float4 *>(dx + row) = make_float4(o[0], o[1], o[2], o[3]);
         *reinterpret_cast<float4 *>(dx + row + 4) = make_float4(o[4], o[5], o[6], o[7]);
-        if (dfinal && t == L - 1) {   // the final state also depends on the last log-decay cumsum
-            // fin_t is the final state transposed, (n, p)
-            const int64_t base = (b * H + h) * (int64_t)P * N;
-            for (int i = part; i < P * N; i += kTokLanes)
-                sf = fmaf(dfinal[base + i], fin_t[base + (int64_t)(i % N) * P + i / N], sf);
-        }
+        // the final state also depends on the last log-decay cumsum: + <dfinal, final>
+        if (fdot && t == L - 1) sf = fdot[b * H + h];
     }
 #pragma unroll
-    for (int o = 1; o < kTokLanes; o <<= 1) {
-        sd += __shfl_xor_sync(0xffffffffu, sd, o);
-        sf += __shfl_xor_sync(0xffffffffu, sf, o);
-    }
+    for (int o = 1; o < kTokLanes; o <<= 1) sd += __shfl_xor_sync(0xffffffffu, sd, o);
     if (ok && part == 0) {
         q[w] = ydot[w] - dth * ddt_in[w] + sf;
         xdy[w] = sd;
+    }
+}
+
+// One block per (b, h): out[b][h] = <a, c> over the (b, h) state, both in the same layout.
+__global__ void __launch_bounds__(256)
+state_dot_kernel(const float *__restrict__ a, const float *__restrict__ c, float *__restrict__ out,
+                 int PN)
+{
+    __shared__ float red[8];
+    const float4 *a4 = reinterpret_cast<const float4 *>(a + blockIdx.x * (int64_t)PN);
+    const float4 *c4 = reinterpret_cast<const float4 *>(c + blockIdx.x * (int64_t)PN);
+    float s = 0.f;
+    for (int i = threadIdx.x; i < PN / 4; i += 256) {
+        const float4 u = a4[i], v = c4[i];
+        s = fmaf(u.x, v.x, fmaf(u.y, v.y, fmaf(u.z, v.z, fmaf(u.w, v.w, s))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.f;
+        for (int j = 0; j < 8; ++j) t += red[j];
+        out[blockIdx.x] = t;
     }
 }
 
@@ -283,17 +299,25 @@ cudaError_t launch_transpose(const float *in, float *out, int64_t mats, int rows
     return cudaGetLastError();
 }
 
+cudaError_t launch_state_dot(const float *a, const float *c, float *out, int64_t mats, int PN,
+                             cudaStream_t st)
+{
+    if (PN % 4 != 0) return cudaErrorInvalidValue;
+    if (mats == 0) return cudaSuccess;
+    state_dot_kernel<<<(unsigned)mats, 256, 0, st>>>(a, c, out, PN);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_bwd_tokens(const bf16 *x, const bf16 *dy, const float *dt, const float *D,
                               const bf16 *gb_rev, const float *ydot, const float *ddt_in,
-                              const float *dfinal, const float *fin_t, float *dx, float *q,
-                              float *xdy, int64_t batch, int64_t L, int H, int P, int N,
-                              cudaStream_t st)
+                              const float *fdot, float *dx, float *q, float *xdy, int64_t batch,
+                              int64_t L, int H, int P, cudaStream_t st)
 {
     if (P != kTokLanes * 8) return cudaErrorInvalidValue;
     const int64_t threads = batch * L * H * kTokLanes;
     if (threads == 0) return cudaSuccess;
     bwd_tokens_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-        x, dy, dt, D, gb_rev, ydot, ddt_in, dfinal, fin_t, dx, q, xdy, batch, L, H, N);
+        x, dy, dt, D, gb_rev, ydot, ddt_in, fdot, dx, q, xdy, batch, L, H);
     return cudaGetLastError();
 }
 

@@ -203,12 +203,14 @@ cudaError_t launch_fill(float *out, float value, int64_t n, cudaStream_t st);
 cudaError_t launch_transpose(const float *in, float *out, int64_t mats, int rows, int cols,
                              cudaStream_t st);
 // dx[b][t][h][p] = D_h dy + dt[b][t][h] gb[b][L-1-t][h][p];  xdy[b][t][h] = <x, dy>;
-// q[b][t][h] = ydot - dt ddt_in (+ <dfinal, final> at t = L-1; fin_t is the final state (n, p))
+// q[b][t][h] = ydot - dt ddt_in (+ fdot[b][h] = <dfinal, final> at t = L-1; fdot nullable)
 cudaError_t launch_bwd_tokens(const bf16 *x, const bf16 *dy, const float *dt, const float *D,
                               const bf16 *gb_rev, const float *ydot, const float *ddt_in,
-                              const float *dfinal, const float *fin_t, float *dx, float *q,
-                              float *xdy, int64_t batch, int64_t L, int H, int P, int N,
-                              cudaStream_t st);
+                              const float *fdot, float *dx, float *q, float *xdy, int64_t batch,
+                              int64_t L, int H, int P, cudaStream_t st);
+// out[m] = <a[m], c[m]> over PN contiguous floats (PN % 4 == 0, 16-byte aligned matrices)
+cudaError_t launch_state_dot(const float *a, const float *c, float *out, int64_t mats, int PN,
+                             cudaStream_t st);
 // dl = reverse cumsum of q over t per (b, h); ddt = ddt_in + A_h dl; dA_h = sum dt dl;
 // dD_h = sum xdy (both summed over the batch)
 cudaError_t launch_bwd_decay(const float *q, const float *ddt_in, const float *dt,

@@ -420,8 +420,8 @@ constexpr int kBwdSimtChunk = 64;   // chunk of the two CUDA-core scans (head di
 struct BwdLayout {
     size_t r_ws, s_ws;                          // tensor-core and CUDA-core scan workspaces
     size_t dyr, Cr, Br, dtr, zerosD, gb, Fr;
-    size_t inits, ys, fin_t;                    // the CUDA-core scans' state and output (reused)
-    size_t ydot, ddt_in, q, xdy, total;
+    size_t inits, dft, ys, fin_t;               // the CUDA-core scans' states and output
+    size_t ydot, ddt_in, q, xdy, fdot, total;
     size_t r_bytes, s_bytes;
 };
 
@@ -455,12 +455,14 @@ BwdLayout bwd_layout(const ssd_shape *s, int Q)
     w.gb = take(b * L * H * P * 2);
     w.Fr = take(b * H * P * N * 4);
     w.inits = take(b * H * N * P * 4);
+    w.dft = take(b * H * N * P * 4);
     w.ys = take(b * L * H * N * 4);
     w.fin_t = take(b * H * N * P * 4);
     w.ydot = take(b * L * H * 4);
     w.ddt_in = take(b * L * H * 4);
     w.q = take(b * L * H * 4);
     w.xdy = take(b * L * H * 4);
+    w.fdot = take(b * H * 4);
     w.total = o;
     return w;
 }
@@ -574,8 +576,9 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
     for (int pass = 0; pass < 2; ++pass) {   // 0: dB (reversed), 1: dC (forward)
         const bool rev = pass == 0;
         const float *init_s = rev ? dfinal : init_state;
+        float *init_t = F(rev ? wl.dft : wl.inits);   // dfinal^T is kept for <dfinal, final>
         const float *w_s = rev ? nullptr : dt;
-        if (init_s && (e = ssd::launch_transpose(init_s, F(wl.inits), b * H, P, N, cst)))
+        if (init_s && (e = ssd::launch_transpose(init_s, init_t, b * H, P, N, cst)))
             return cuda_fail(e, "transpose");
         e = ssd::launch_chunk_cumsum(rev ? F(wl.dtr) : dt, A, cs_s, nullptr, nullptr, b, L, H,
                                      Qs, nchs, cst);
@@ -583,7 +586,7 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
             e = ssd::launch_bwd_chunk_state(rev ? Cb : Bb, rev ? dyb : xb, w_s, cs_s, states_s, b,
                                             L, H, G, nchs, rev, cst);
         if (e == cudaSuccess)
-            e = ssd::launch_state_passing(states_s, cs_s, init_s ? F(wl.inits) : nullptr,
+            e = ssd::launch_state_passing(states_s, cs_s, init_s ? init_t : nullptr,
                                           rev ? nullptr : F(wl.fin_t), nullptr, b, H, N, P, Qs,
                                           nchs, cst);
         if (e == cudaSuccess)
@@ -598,8 +601,13 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
     }
 
     // 3. dx, the decay-gradient terms and their reverse cumsum: ddt, dA, dD
-    if ((e = ssd::launch_bwd_tokens(xb, dyb, dt, D, Hh(wl.gb), F(wl.ydot), F(wl.ddt_in), dfinal,
-                                    F(wl.fin_t), dx, F(wl.q), F(wl.xdy), b, L, H, P, N, cst)) ||
+    // <dfinal, final>, both transposed to (n, p): the final state's share of the decay gradient
+    if (dfinal && (e = ssd::launch_state_dot(F(wl.dft), F(wl.fin_t), F(wl.fdot), b * H, P * N,
+                                             cst)))
+        return cuda_fail(e, "final-state term");
+    if ((e = ssd::launch_bwd_tokens(xb, dyb, dt, D, Hh(wl.gb), F(wl.ydot), F(wl.ddt_in),
+                                    dfinal ? F(wl.fdot) : nullptr, dx, F(wl.q), F(wl.xdy), b, L,
+                                    H, P, cst)) ||
         (e = ssd::launch_bwd_decay(F(wl.q), F(wl.ddt_in), dt, A, F(wl.xdy), ddt, dA, dD, b, L, H,
                                    cst)))
         return cuda_fail(e, "token gradients");
