@@ -9,11 +9,13 @@
 //   g_t B_t          = the forward scan of the time-reversed sequence with x' = dy, B' = C,
 //                      C' = B, unit input weights and each decay shifted by one token, started
 //                      from dfinal (tensor cores);  dx_t = D dy_t + dt_t g_t B_t
-//   dB_t (per head)  = dt_t x (reversed scan with x' = C, B' = dy, C' = x, from dfinal^T)
-//   dC_t (per head)  = the forward scan with x' = B, B' = x, C' = dy, weights dt, from h0^T
+//   dB_t (per head)  = dt_t times the output of the reversed scan with x' = C, B' = dy, C' = x,
+//                      unit weights, started from dfinal^T
+//   dC_t (per head)  = the output of the forward scan with x' = B, B' = x, C' = dy, weights dt,
+//                      started from h0^T
 //
-// (the last two have head dimension N and state dimension P, run on CUDA cores in float32, and
-// are summed over the heads of a group).  The decay gradient uses the identity, for the global
+// (the last two have head dimension N and state dimension P, run on CUDA cores in float32 --
+// bwd_scan.cu -- and are summed over the heads of a group).  The decay gradient uses the identity, for the global
 // log-decay cumsum Lcs_k,
 //     dL/dLcs_k = <dy_k, y_k - D x_k> - dt_k <x_k, g_k B_k>  (+ <dfinal, final> at k = L-1)
 // followed by a reverse cumsum: dL/d(dt_k A_h) = sum_{j >= k} dL/dLcs_j (which equals
