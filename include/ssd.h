@@ -92,10 +92,6 @@ size_t ssd_chunk_scan_workspace_size(const ssd_shape *shape, int chunk_size);
  *
  * Concurrent calls must use distinct workspaces.  batch == 0 or seqlen == 0 is valid: y is
  * empty and final_state is set to init_state (or zeros).
- *
- * On the tensor-core path the per-chunk states and the carry across chunks run as two kernels
- * by default; setting the environment variable SSD_STATE_PASSING=fused runs them as one kernel
- * that walks the chunks in order (=split forces the two kernels).  Both give the same result.
  */
 ssd_status ssd_chunk_scan_fwd(const ssd_shape *shape, const void *x, const float *dt,
                               const float *A, const void *B, const void *C, const float *D,
@@ -319,12 +315,25 @@ ssd_status ssd_workspace_status(const void *workspace, size_t workspace_bytes, v
  *   - All calls on a device share the one array: calls whose kernels overlap on the GPU (other
  *     streams, other host threads) race and corrupt each other's results.  Issue them one after
  *     another on a single stream.
- *   - Results are the same as ssd_chunk_scan_fwd's for the same arguments.
+ *   - The address is cached per device for the device's primary context (the CUDA runtime's);
+ *     running the scan in another context, or after a device reset, is not supported.
+ *   - Results are bit-identical to ssd_chunk_scan_fwd's for the same arguments.
+ *   - An in-kernel timeout is recorded in the array's status word, which
+ *     ssd_chunk_scan_fwd_static_status() reads.
  */
 ssd_status ssd_chunk_scan_fwd_static(const ssd_shape *shape, const void *x, const float *dt,
                                      const float *A, const void *B, const void *C,
                                      const float *D, int chunk_size, const float *init_state,
                                      void *y, float *final_state, void *stream);
+
+/*
+ * The status word that the last ssd_chunk_scan_fwd_static call on the current device left in
+ * the built-in scratch array, as ssd_workspace_status() reports it for a caller workspace:
+ * synchronises `stream`, then SSD_OK, or SSD_ERR_TIMEOUT when a bounded in-kernel wait gave up
+ * (the outputs of that call are then incomplete).  SSD_ERR_CUDA if the array's address cannot
+ * be looked up or the synchronisation reports an error.  Allocates nothing.
+ */
+ssd_status ssd_chunk_scan_fwd_static_status(void *stream);
 
 /* Message for the calling thread's last non-OK status ("" if none). */
 const char *ssd_last_error(void);

@@ -83,7 +83,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                       const __grid_constant__ CUtensorMap tm_b, const float *__restrict__ dtc,
                       const float *__restrict__ cs, float *__restrict__ states,
                       int *__restrict__ status, int H, int G, int Q, int64_t nchunks, int nhb,
-                      int hpc, int64_t seqlen, const int2 *__restrict__ tab)
+                      int hpc, int64_t seqlen, const int2 *__restrict__ tab, int skip_cta)
 {
     extern __shared__ uint8_t smem_raw[];
     StateSmem &sm = *reinterpret_cast<StateSmem *>(
@@ -143,6 +143,8 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 const uint32_t use = j / kStateStages;
                 if (j >= kStateStages && !mbar_wait(&sm.bar_x_free[s], (use - 1) & 1, abort))
                     break;
+                // failure injection (tests only): this stage is left unissued
+                if (j == 0 && (int)blockIdx.x == skip_cta) continue;
                 const int64_t vrow = ((b * nchunks + k) * H + h0 + j) * (int64_t)Q;
                 mbar_arrive_expect_tx(&sm.bar_x_full[s], (uint32_t)Q * (kRowBytes + 8));
                 tma_load_4d(&sm.Xs[s][0], &tm_x, &sm.bar_x_full[s], 0, h0 + j, (int)t0, (int)b);
@@ -254,262 +256,6 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     }
 }
 
-// ============================================================ chunk state + state passing, fused
-//
-// One CTA per (batch, group, block of up to 3 heads) walks the chunks in order and carries the
-// recurrence across them itself (mohakchugh.is-a.dev "Mamba-2", Block Decomposition: across
-// blocks the state is propagated sequentially):
-//
-//     S_k     = B_k^T (w o X_k)              (tensor cores, TMEM)
-//     h_in[k] = h;   h <- exp(cs_k[Q-1]) h + S_k      (h in TMEM, fp32)
-//
-// so the float32 chunk states never go to HBM.  Each chunk is consumed in 128-row halves
-// through a 2-stage ring (the half's B rows, shared by the heads, and each head's x rows).
-// Three MMA issuer warps (one per head) keep three accumulation chains in flight; 8 epilogue
-// warps own the state: per chunk they store h (bf16) as the state entering the chunk and fold
-// S into it; after the last chunk they store it (float32) as the final state.
-constexpr int kFusedHeads = 3;
-struct alignas(1024) FusedSmem {
-    bf16 Bs[2][2][kTileRows * 64];                  // per stage: MN-major A, [n atom][128 tau][64 n]
-    bf16 Xs[2][kFusedHeads][kTileRows * 64];        // per stage and head: MN-major B [128 tau][64 p]
-    float cs_v[2][kFusedHeads][256];                // per chunk slot and head: cs row
-    float dt_v[2][kFusedHeads][256];                // per chunk slot and head: dt row
-    uint64_t bar_full[2], bar_ready[2], bar_free[2];
-    uint64_t bar_vec_full[2], bar_vec_free[2];
-    uint64_t bar_acc_full[kFusedHeads], bar_acc_free[kFusedHeads];
-    uint64_t bar_drain;
-    uint32_t tmem_base;
-    int abort;
-};
-// warp 0 TMA, warps 1-3 MMA (warp 1 + j issues head j; warp 2 also owns TMEM), warps 4-11 scale
-// x, warps 12-19 state epilogue (two per TMEM lane quarter, 32 columns p each)
-constexpr int kFusedThreads = 640;
-constexpr uint32_t kFusedTmemCols = 512;   // S of head j at 64 j, h of head j at 256 + 64 j
-static_assert(sizeof(FusedSmem) + 1024 <= 232448, "fused state smem exceeds 227 KB");
-
-__global__ void __launch_bounds__(kFusedThreads, 1)
-chunk_state_pass_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
-                           const __grid_constant__ CUtensorMap tm_b,
-                           const float *__restrict__ dtc, const float *__restrict__ cs,
-                           const float *__restrict__ init, float *__restrict__ final_state,
-                           bf16 *__restrict__ hin, int *__restrict__ status, int H, int G, int Q,
-                           int64_t nchunks, int nhb)
-{
-    extern __shared__ uint8_t smem_raw[];
-    FusedSmem &sm = *reinterpret_cast<FusedSmem *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-
-    int64_t u = blockIdx.x;
-    const int hb = (int)(u % nhb); u /= nhb;
-    const int g = (int)(u % G); u /= G;
-    const int64_t b = u;
-    const int hpg = H / G;
-    const int h0 = g * hpg + hb * kFusedHeads;
-    const int nh = min(kFusedHeads, hpg - hb * kFusedHeads);
-    const int nrb = Q / kTileRows;               // 128-row halves per chunk
-    const int64_t nunits = nchunks * nrb;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&sm.bar_full[s], 1);
-            mbar_init(&sm.bar_ready[s], 256);
-            mbar_init(&sm.bar_free[s], nh);
-            mbar_init(&sm.bar_vec_full[s], 1);
-            mbar_init(&sm.bar_vec_free[s], 256 + 256);
-        }
-        for (int j = 0; j < kFusedHeads; ++j) {
-            mbar_init(&sm.bar_acc_full[j], 1);
-            mbar_init(&sm.bar_acc_free[j], 256);
-        }
-        mbar_init(&sm.bar_drain, kFusedHeads);
-        sm.abort = 0;
-        fence_mbar_init();
-    }
-    if (warp == 2) {
-        tmem_alloc(&sm.tmem_base, kFusedTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = sm.tmem_base;
-    volatile int *abort = &sm.abort;
-
-    if (warp == 0) {
-        // ---------------- TMA producer (lane 0 alone)
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_x);
-            tma_prefetch_desc(&tm_b);
-            for (int64_t un = 0; un < nunits; ++un) {
-                const int64_t k = un / nrb;
-                const int r = (int)(un % nrb);
-                if (r == 0) {
-                    const int vs = (int)(k & 1);
-                    if (k >= 2 &&
-                        !mbar_wait(&sm.bar_vec_free[vs], (uint32_t)((k >> 1) - 1) & 1, abort))
-                        break;
-                    mbar_arrive_expect_tx(&sm.bar_vec_full[vs], (uint32_t)(8 * Q * nh));
-                    for (int j = 0; j < nh; ++j) {
-                        const int64_t vrow = ((b * nchunks + k) * H + h0 + j) * (int64_t)Q;
-                        bulk_load(sm.cs_v[vs][j], cs + vrow, Q * 4, &sm.bar_vec_full[vs]);
-                        bulk_load(sm.dt_v[vs][j], dtc + vrow, Q * 4, &sm.bar_vec_full[vs]);
-                    }
-                }
-                const int s = (int)(un & 1);
-                if (un >= 2 && !mbar_wait(&sm.bar_free[s], (uint32_t)((un >> 1) - 1) & 1, abort))
-                    break;
-                const int row = (int)(k * Q + kTileRows * r);
-                mbar_arrive_expect_tx(&sm.bar_full[s], (uint32_t)((2 + nh) * kBoxBytes));
-                for (int a = 0; a < 2; ++a)
-                    tma_load_4d(&sm.Bs[s][a][0], &tm_b, &sm.bar_full[s], 64 * a, g, row, (int)b);
-                for (int j = 0; j < nh; ++j)
-                    tma_load_4d(&sm.Xs[s][j][0], &tm_x, &sm.bar_full[s], 0, h0 + j, row, (int)b);
-            }
-        }
-    } else if (warp >= 1 && warp <= 3) {
-        // ---------------- MMA issuer for head j = warp - 1: S_j (+)= B^T (w o X_j); lane 0
-        // alone runs the loop (see the chunk state kernel)
-        const int j = warp - 1;
-        if (j < nh && lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, kP, true, true);
-            const uint32_t d = tmem + 64 * j;
-            for (int64_t un = 0; un < nunits; ++un) {
-                const int64_t k = un / nrb;
-                const int r = (int)(un % nrb);
-                const int s = (int)(un & 1);
-                if (!mbar_wait(&sm.bar_ready[s], (uint32_t)(un >> 1) & 1, abort)) break;
-                if (r == 0 && k >= 1 &&
-                    !mbar_wait(&sm.bar_acc_free[j], (uint32_t)(k - 1) & 1, abort))
-                    break;
-                tc_fence_after();
-                const uint64_t ad = smem_desc_sw128(smem_u32(&sm.Bs[s][0][0]), kBoxBytes, 1024);
-                const uint64_t bd = smem_desc_sw128(smem_u32(&sm.Xs[s][j][0]), kBoxBytes, 1024);
-#pragma unroll
-                for (int kk = 0; kk < kTileRows / 16; ++kk)
-                    mma_bf16(d, ad + kk * 128, bd + kk * 128, idesc, (r > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&sm.bar_free[s]);
-                if (r == nrb - 1) mma_commit(&sm.bar_acc_full[j]);
-            }
-        }
-    } else if (warp >= 4 && warp < 12) {
-        // ---------------- scale x rows of every head by w_tau = exp(cs_last - cs_tau) dt_tau
-        const int st = threadIdx.x - 128;             // 0..255
-        for (int64_t un = 0; un < nunits; ++un) {
-            const int64_t k = un / nrb;
-            const int r = (int)(un % nrb);
-            const int s = (int)(un & 1);
-            const int vs = (int)(k & 1);
-            if (!warp_wait(&sm.bar_full[s], (uint32_t)(un >> 1) & 1, abort)) break;
-            if (!warp_wait(&sm.bar_vec_full[vs], (uint32_t)(k >> 1) & 1, abort)) break;
-            for (int c = st; c < nh * kTileRows * 8; c += 256) {
-                const int j = c / (kTileRows * 8);
-                const int pc = c % (kTileRows * 8);
-                const int tau = kTileRows * r + (pc >> 3);
-                const float w = __expf(sm.cs_v[vs][j][Q - 1] - sm.cs_v[vs][j][tau]) *
-                                sm.dt_v[vs][j][tau];
-                uint4 *ptr = reinterpret_cast<uint4 *>(&sm.Xs[s][j][0]) + pc;
-                uint4 v = *ptr;
-                uint32_t *wv = &v.x;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162 *>(&wv[e]));
-                    const float2 sc = fmul2(f, make_float2(w, w));
-                    wv[e] = pack_bf16x2(sc.x, sc.y);
-                }
-                *ptr = v;
-            }
-            fence_async_smem();
-            mbar_arrive(&sm.bar_ready[s]);
-            if (r == nrb - 1) mbar_arrive(&sm.bar_vec_free[vs]);
-        }
-    } else {
-        // ---------------- state epilogue: lane n (TMEM lane), columns p in [32 half, +32)
-        const int qd = warp & 3;
-        const int half = (warp - 12) >> 2;
-        const int n = qd * 32 + lane;
-        const int p0 = 32 * half;
-        const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
-        // initial state (caller layout [p][n]) -> TMEM h
-        for (int j = 0; j < nh; ++j) {
-            uint32_t hv[16];
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const int p = p0 + 16 * hh + c;
-                    hv[c] = __float_as_uint(
-                        init ? init[((b * H + h0 + j) * kP + p) * (int64_t)kN + n] : 0.f);
-                }
-                tmem_st16(lane_base + 256 + 64 * j + p0 + 16 * hh, hv);
-            }
-        }
-        tmem_st_wait();
-        bool ok = true;
-        for (int64_t k = 0; ok && k < nchunks; ++k) {
-            const int vs = (int)(k & 1);
-            if (!warp_wait(&sm.bar_vec_full[vs], (uint32_t)(k >> 1) & 1, abort)) break;
-            for (int j = 0; j < nh; ++j) {
-                if (!warp_wait(&sm.bar_acc_full[j], (uint32_t)k & 1, abort)) { ok = false; break; }
-                tc_fence_after();
-                uint32_t sv[32], hv[32];
-                tmem_ld32(lane_base + 64 * j + p0, sv);
-                tmem_ld32(lane_base + 256 + 64 * j + p0, hv);
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(&sm.bar_acc_free[j]);
-                const float a = __expf(sm.cs_v[vs][j][Q - 1]);
-                // the state entering chunk k, bf16, in the swizzled block layout: 64 bytes of
-                // one 128-byte row per warp store
-                bf16 *out = hin + ((b * nchunks + k) * H + h0 + j) * (int64_t)(kP * kN);
-#pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    out[hin_swizzled_offset(p0 + c, n)] = __float2bfloat16_rn(__uint_as_float(hv[c]));
-                uint32_t nv[16];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        nv[c] = __float_as_uint(fmaf(a, __uint_as_float(hv[16 * hh + c]),
-                                                     __uint_as_float(sv[16 * hh + c])));
-                    tmem_st16(lane_base + 256 + 64 * j + p0 + 16 * hh, nv);
-                }
-                tmem_st_wait();
-            }
-            if (ok) mbar_arrive(&sm.bar_vec_free[vs]);
-        }
-        if (ok && final_state) {
-            for (int j = 0; j < nh; ++j) {
-                uint32_t hv[32];
-                tmem_ld32(lane_base + 256 + 64 * j + p0, hv);
-                tmem_ld_wait();
-                float *fo = final_state + ((b * H + h0 + j) * kP + p0) * (int64_t)kN + n;
-#pragma unroll
-                for (int c = 0; c < 32; ++c) fo[c * kN] = __uint_as_float(hv[c]);
-            }
-        }
-    }
-
-    __syncthreads();
-    if (sm.abort) {
-        if (warp >= 1 && warp <= 3 && lane == 0) {
-            mma_commit(&sm.bar_drain);
-            mbar_wait_drain(&sm.bar_drain, 0);
-        }
-        if (threadIdx.x == 0) {
-            drain_sleep();
-            atomicOr(status, 4);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 2) {
-        tc_fence_after();
-        tmem_dealloc(tmem, kFusedTmemCols);
-    }
-}
-
 // ============================================================ chunk scan (intra-chunk + off-chunk)
 //
 // Tile T of a chunk holds rows [128 T, 128 T + 128).  Its output splits into
@@ -604,7 +350,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const float *__restrict__ cs, const float *__restrict__ D,
                      bf16 *__restrict__ y, int *__restrict__ status, int64_t seqlen, int H,
                      int G, int Q, int64_t nchunks, int nhb, int hpc, const int2 *__restrict__ tab,
-                     const bf16 *__restrict__ z)
+                     const bf16 *__restrict__ z, int skip_cta)
 {
     extern __shared__ uint8_t smem_raw[];
     ScanSmem &sm = *reinterpret_cast<ScanSmem *>(
@@ -698,6 +444,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             const uint32_t xu = j / nst;
             if (j >= nst && !mbar_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) break;
             if (xs == 2 && xu == 0 && !mbar_wait(&sm.bar_g, 0, abort)) break;  // B tile in use
+            // failure injection (tests only): this stage is left unissued
+            if (j == 0 && (int)blockIdx.x == skip_cta) continue;
             uint8_t *stg = scan_stage(sm, xs);
             mbar_arrive_expect_tx(&sm.bar_xh_full[xs],
                                   (uint32_t)(KI * kRowBytes + 2 * kP * kRowBytes));
@@ -1108,37 +856,8 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb);
     *why = "chunk state (tcgen05) launch";
     return launch_pdl(chunk_state_tc_kernel, grid, kStateThreads, smem, st, mx, mb, dtc, cs,
-                      states, status, H, G, Q, nchunks, nhb, hpc, seqlen, tab);
-}
-
-// The fused chunk state + state passing kernel walks the chunks of a (batch, group, 3 heads)
-// block in order, one CTA per block, so it needs about one block per SM to keep the GPU busy; at
-// the shapes measured so far (b 4 x H 80, b 2 x H 24, b 1 x H 32 with 8 groups) the two-kernel
-// path was faster, so the fused form is used only on request.
-bool fused_state_pass_ok(int64_t, int, int) { return false; }
-
-cudaError_t launch_chunk_state_pass_tc(const bf16 *x, const float *dtc, const bf16 *B,
-                                       const float *cs, const float *init, float *final_state,
-                                       bf16 *hin, int *status, int64_t batch, int64_t seqlen,
-                                       int H, int G, int Q, int64_t nchunks, cudaStream_t st,
-                                       const char **why)
-{
-    CUtensorMap mx, mb;
-    if (!make_seq_map(&mx, x, batch, seqlen, H, kP) || !make_seq_map(&mb, B, batch, seqlen, G, kN)) {
-        *why = "fused chunk state: cuTensorMapEncodeTiled failed";
-        return cudaErrorInvalidValue;
-    }
-    const int hpg = H / G;
-    const int nhb = (hpg + kFusedHeads - 1) / kFusedHeads;
-    const size_t smem = sizeof(FusedSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(chunk_state_pass_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) { *why = "fused chunk state: set smem attribute"; return e; }
-    const unsigned grid = (unsigned)(batch * G * nhb);
-    chunk_state_pass_tc_kernel<<<grid, kFusedThreads, smem, st>>>(
-        mx, mb, dtc, cs, init, final_state, hin, status, H, G, Q, nchunks, nhb);
-    *why = "fused chunk state (tcgen05) launch";
-    return cudaGetLastError();
+                      states, status, H, G, Q, nchunks, nhb, hpc, seqlen, tab,
+                      take_test_skip(kTestChunkState));
 }
 
 cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
@@ -1176,7 +895,8 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb * (Q / kTileRows));
     *why = "chunk scan (tcgen05) launch";
     return launch_pdl(kern, grid, kScanThreads, smem, st, mx, mb, mc, mx2, mz, hin, dtc, cs, D, y,
-                      status, seqlen, H, G, Q, nchunks, nhb, hpc, tab, z);
+                      status, seqlen, H, G, Q, nchunks, nhb, hpc, tab, z,
+                      take_test_skip(kTestChunkScan));
 }
 
 }  // namespace ssd

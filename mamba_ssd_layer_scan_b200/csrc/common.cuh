@@ -96,12 +96,20 @@ __device__ __forceinline__ void chunk_span(const int2 *tab, int64_t k, int Q, in
     }
 }
 
-// Workspace status word bits: 1, 2, 4 = a bounded wait timed out (chunk scan, chunk state, fused
-// state); kStatusBadSeqlens = the cu_seqlens of a variable-length call are inconsistent.
+// Workspace status word bits: 1, 2 = a bounded wait timed out (chunk state, chunk scan);
+// kStatusBadSeqlens = the cu_seqlens of a variable-length call are inconsistent.
 constexpr int kStatusBadSeqlens = 0x10000;
 
 // Sets the calling thread's message returned by ssd_last_error().
 void set_last_error(const char *msg);
+
+// Failure injection for the tests of the bounded waits (include/ssd_testing.h): the CTA index of
+// the next launch of `kernel` (kTestChunkState or kTestChunkScan) whose TMA producer leaves its
+// first head's operand stage unissued, so the consumers' bounded waits on that stage run out;
+// -1 (the default) for none.  Reading the setting clears it.
+constexpr int kTestChunkState = 1;
+constexpr int kTestChunkScan = 2;
+int take_test_skip(int kernel);
 
 // ---- launchers (each returns the launch's cudaError_t) ----
 // Also zeroes *status (nullable) so each scan starts with a clean status word, and, when dtc is
@@ -212,10 +220,11 @@ cudaError_t launch_bwd_tokens(const bf16 *x, const bf16 *dy, const float *dt, co
 cudaError_t launch_state_dot(const float *a, const float *c, float *out, int64_t mats, int PN,
                              cudaStream_t st);
 // dl = reverse cumsum of q over t per (b, h); ddt = ddt_in + A_h dl; dA_h = sum dt dl;
-// dD_h = sum xdy (both summed over the batch)
+// dD_h = sum xdy (both summed over the batch in batch order, through the 2 * batch * H floats of
+// `part`, so repeated calls give bit-identical results)
 cudaError_t launch_bwd_decay(const float *q, const float *ddt_in, const float *dt,
                              const float *A, const float *xdy, float *ddt, float *dA, float *dD,
-                             int64_t batch, int64_t L, int H, cudaStream_t st);
+                             float *part, int64_t batch, int64_t L, int H, cudaStream_t st);
 // The backward's two float32 scans for P = 64, N = 128 (bwd_scan.cu): x'' (batch, L, G, 128)
 // bf16, B'' and C'' (batch, L, H, 64) bf16, all read at row L-1-tau for scan step tau when
 // `rev`; w (batch, L, H) in scan order, null = 1; cs (batch, nch, H, 64) chunk-local cumsum in
@@ -236,14 +245,6 @@ cudaError_t launch_group_sum(const float *in, const float *w, float *out, int64_
 cudaError_t launch_scale_init_grad(const float *F, const float *dt, const float *A, float *out,
                                    int64_t batch, int64_t L, int H, int PN, cudaStream_t st);
 
-// Chunk state and state passing in one kernel (chunks walked in order per block of heads):
-// writes the bf16 entering states and the float32 final state; no float32 chunk states.
-bool fused_state_pass_ok(int64_t batch, int H, int G);
-cudaError_t launch_chunk_state_pass_tc(const bf16 *x, const float *dtc, const bf16 *B,
-                                       const float *cs, const float *init, float *final_state,
-                                       bf16 *hin, int *status, int64_t batch, int64_t seqlen,
-                                       int H, int G, int Q, int64_t nchunks, cudaStream_t st,
-                                       const char **why);
 cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,

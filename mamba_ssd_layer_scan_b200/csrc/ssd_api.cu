@@ -12,10 +12,11 @@
 // nothing synchronises; errors are reported through the returned status.
 #include <cstdarg>
 #include <cstdio>
-#include <cstdlib>
-#include <cstring>
+
+#include <atomic>
 
 #include "../../include/ssd.h"
+#include "../../include/ssd_testing.h"
 #include "common.cuh"
 
 namespace {
@@ -66,18 +67,6 @@ ssd_status check_shape(const ssd_shape *s, bool need_seq)
     if (s->nheads > 65535 || s->batch > 65535)
         return fail(SSD_ERR_UNSUPPORTED, "batch and nheads must be <= 65535");
     return SSD_OK;
-}
-
-// Tensor-core path: chunk state and state passing run either as one fused kernel or as two
-// kernels; ssd::fused_state_pass_ok picks the form, and the environment variable
-// SSD_STATE_PASSING=fused|split forces one (both compute the same result; the switch exists to
-// test and time each).
-bool use_fused_state_pass(int64_t batch, int H, int G)
-{
-    const char *f = getenv("SSD_STATE_PASSING");
-    if (f && strcmp(f, "fused") == 0) return true;
-    if (f && strcmp(f, "split") == 0) return false;
-    return ssd::fused_state_pass_ok(batch, H, G);
 }
 
 bool valid_chunk(int q) { return q == 16 || q == 32 || q == 64 || q == 128 || q == 256; }
@@ -145,11 +134,35 @@ ssd_status check_varlen(const ssd_shape *s, int nseq, int Q)
 
 void ssd::set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
 
+namespace {
+std::atomic<int> g_test_kernel{0};
+std::atomic<int> g_test_cta{-1};
+}  // namespace
+
+int ssd::take_test_skip(int kernel)
+{
+    int k = kernel;
+    if (!g_test_kernel.compare_exchange_strong(k, 0)) return -1;
+    return g_test_cta.exchange(-1);
+}
+
 extern "C" {
 
 const char *ssd_last_error(void) { return g_err; }
 
 const char *ssd_version(void) { return "ssd-b200 0.1 (sm_100a)"; }
+
+ssd_status ssd_testing_skip_stage(int kernel, int cta)
+{
+    if (kernel != SSD_TESTING_CHUNK_STATE && kernel != SSD_TESTING_CHUNK_SCAN)
+        return fail(SSD_ERR_INVALID_ARG, "kernel must be SSD_TESTING_CHUNK_STATE or "
+                                         "SSD_TESTING_CHUNK_SCAN (got %d)", kernel);
+    if (cta < 0) return fail(SSD_ERR_INVALID_ARG, "cta must be >= 0 (got %d)", cta);
+    g_test_cta.store(cta);
+    g_test_kernel.store(kernel == SSD_TESTING_CHUNK_STATE ? ssd::kTestChunkState
+                                                          : ssd::kTestChunkScan);
+    return SSD_OK;
+}
 
 size_t ssd_chunk_scan_workspace_size(const ssd_shape *shape, int chunk_size)
 {
@@ -257,29 +270,17 @@ ssd_status scan_impl(const ssd_shape *shape, const void *x, const float *dt, con
     if (tc) {
         const char *why = "";
         ssd::bf16 *hin = reinterpret_cast<ssd::bf16 *>(ws + wl.hin_bf16);
-        if (use_fused_state_pass(s.batch, H, G)) {
-            // chunk state and state passing in one launch; the passing stage is then empty
-            e = ssd::launch_chunk_state_pass_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B,
-                                                cs, init_state, final_state, hin, status,
-                                                s.batch, s.seqlen, H, G, Q, nchunks, cs_stream,
-                                                &why);
-            if (e != cudaSuccess) return cuda_fail(e, why);
-            if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess ||
-                (e = record(stage_events, 3, cs_stream)) != cudaSuccess)
-                return cuda_fail(e, "record stage event");
-        } else {
-            e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs,
-                                           states, status, s.batch, s.seqlen, H, G, Q, nchunks,
-                                           cs_stream, &why);
-            if (e != cudaSuccess) return cuda_fail(e, why);
-            if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess)
-                return cuda_fail(e, "record stage event");
-            e = ssd::launch_state_passing(states, cs, init_state, final_state, hin, s.batch, H,
-                                          P, N, Q, nchunks, cs_stream);
-            if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
-            if ((e = record(stage_events, 3, cs_stream)) != cudaSuccess)
-                return cuda_fail(e, "record stage event");
-        }
+        e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs,
+                                       states, status, s.batch, s.seqlen, H, G, Q, nchunks,
+                                       cs_stream, &why);
+        if (e != cudaSuccess) return cuda_fail(e, why);
+        if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess)
+            return cuda_fail(e, "record stage event");
+        e = ssd::launch_state_passing(states, cs, init_state, final_state, hin, s.batch, H, P, N,
+                                      Q, nchunks, cs_stream);
+        if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
+        if ((e = record(stage_events, 3, cs_stream)) != cudaSuccess)
+            return cuda_fail(e, "record stage event");
         e = ssd::launch_chunk_scan_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B,
                                       (const ssd::bf16 *)C, cs, hin, D, (ssd::bf16 *)y, status,
                                       s.batch, s.seqlen, H, G, Q, nchunks, cs_stream, &why,
@@ -421,7 +422,7 @@ struct BwdLayout {
     size_t r_ws, s_ws;                          // tensor-core and CUDA-core scan workspaces
     size_t dyr, Cr, Br, dtr, zerosD, gb, Fr;
     size_t inits, dft, ys, fin_t;               // the CUDA-core scans' states and output
-    size_t ydot, ddt_in, q, xdy, fdot, total;
+    size_t ydot, ddt_in, q, xdy, fdot, part, total;
     size_t r_bytes, s_bytes;
 };
 
@@ -463,6 +464,7 @@ BwdLayout bwd_layout(const ssd_shape *s, int Q)
     w.q = take(b * L * H * 4);
     w.xdy = take(b * L * H * 4);
     w.fdot = take(b * H * 4);
+    w.part = take(2 * b * H * 4);
     w.total = o;
     return w;
 }
@@ -608,8 +610,8 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
     if ((e = ssd::launch_bwd_tokens(xb, dyb, dt, D, Hh(wl.gb), F(wl.ydot), F(wl.ddt_in),
                                     dfinal ? F(wl.fdot) : nullptr, dx, F(wl.q), F(wl.xdy), b, L,
                                     H, P, cst)) ||
-        (e = ssd::launch_bwd_decay(F(wl.q), F(wl.ddt_in), dt, A, F(wl.xdy), ddt, dA, dD, b, L, H,
-                                   cst)))
+        (e = ssd::launch_bwd_decay(F(wl.q), F(wl.ddt_in), dt, A, F(wl.xdy), ddt, dA, dD,
+                                   F(wl.part), b, L, H, cst)))
         return cuda_fail(e, "token gradients");
     return SSD_OK;
 }

@@ -27,6 +27,21 @@ def test_exports_every_declared_function(L):
         assert hasattr(L, name)
 
 
+def test_testing_header_exported_and_validated(L):
+    import re
+    text = open(ssd.HEADER.replace("ssd.h", "ssd_testing.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = sorted(set(re.findall(r"\b(ssd_[a-z0-9_]+)\s*\(", text)))
+    assert names == ["ssd_testing_skip_stage"]
+    for name in names:
+        assert hasattr(L, name)
+    f = L.ssd_testing_skip_stage
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int, ctypes.c_int]
+    assert f(7, 0) == ssd.SSD_ERR_INVALID_ARG
+    assert f(2, -1) == ssd.SSD_ERR_INVALID_ARG
+
+
 def test_version(L):
     assert b"sm_100a" in L.ssd_version()
 
