@@ -53,6 +53,8 @@ def _load():
         lib.oracle_ssd_scan.restype = ctypes.c_int
         lib.oracle_ssd_scan.argtypes = [_I64] * 6 + [_D] * 6 + [_D, _D, _D, _D, _I64, _I64,
                                                                  ctypes.POINTER(_I64), _I64]
+        lib.oracle_ssd_scan_bwd.restype = ctypes.c_int
+        lib.oracle_ssd_scan_bwd.argtypes = [_I64] * 6 + [_D] * 16
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -169,7 +171,8 @@ def ssd_state_update_block(state, x, dt, A, B, C, D, z=None, dt_bias=None,
 
 def ssd_scan_bwd(x, dt, A, B, C, D, dy, init=None, dfinal=None):
     """Gradients of L = sum_t <dy_t, y_t> + <dfinal, final_state> through the recurrence, by the
-    adjoint recurrence (reverse-mode differentiation of the token loop, float64):
+    adjoint recurrence (reverse-mode differentiation of the token loop, float64, in
+    ``ssd_oracle.c``, ``oracle_ssd_scan_bwd``):
 
         g_t = dy_t (outer) C_t + a_{t+1} g_{t+1}           (g_{L-1} also gets dfinal)
         dx_t = D_h dy_t + dt_t g_t B_t                      dB_t += dt_t g_t^T x_t  (per group)
@@ -177,38 +180,35 @@ def ssd_scan_bwd(x, dt, A, B, C, D, dy, init=None, dfinal=None):
         dl_t = a_t <g_t, h_{t-1}>   (l_t = dt_t A_h)        ddt_t = <g_t B_t, x_t> + A_h dl_t
         dA_h = sum_t dt_t dl_t                              dinit = a_0 g_0
 
+    The C loop gives each head's share of dB, dC, dA and dD; the group sums over heads and the
+    batch sums are numpy sums here.
+
     x (b, L, H, P), dt (b, L, H), B/C (b, L, G, N), dy like x, init/dfinal (b, H, P, N) or None.
-    Returns dict dx, ddt, dA, dB, dC, dD, dinit.  The forward states are kept per (b, h), so this
-    is for oracle-sized inputs."""
-    x, dt, A, B, C, D, dy = (np.asarray(v, dtype=np.float64) for v in (x, dt, A, B, C, D, dy))
+    Returns dict dx, ddt, dA, dB, dC, dD, dinit."""
+    x, dt, A, B, C, D, dy, init, dfinal = map(_f64, (x, dt, A, B, C, D, dy, init, dfinal))
     b, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
-    out = dict(dx=np.zeros_like(x), ddt=np.zeros_like(dt), dA=np.zeros(H), dB=np.zeros_like(B),
-               dC=np.zeros_like(C), dD=np.zeros(H), dinit=np.zeros((b, H, P, N)))
-    for bi in range(b):
-        for h in range(H):
-            g_ = h // (H // G)
-            a = np.exp(dt[bi, :, h] * A[h])
-            hs = np.zeros((L + 1, P, N))                     # hs[t + 1] = state after token t
-            if init is not None:
-                hs[0] = init[bi, h]
-            for t in range(L):
-                hs[t + 1] = a[t] * hs[t] + dt[bi, t, h] * np.outer(x[bi, t, h], B[bi, t, g_])
-                out["dC"][bi, t, g_] += hs[t + 1].T @ dy[bi, t, h]
-            gnext = np.zeros((P, N)) if dfinal is None else np.asarray(dfinal[bi, h], np.float64)
-            anext = 1.0
-            for t in range(L - 1, -1, -1):
-                g = np.outer(dy[bi, t, h], C[bi, t, g_]) + anext * gnext
-                gB = g @ B[bi, t, g_]
-                out["dx"][bi, t, h] = D[h] * dy[bi, t, h] + dt[bi, t, h] * gB
-                out["dB"][bi, t, g_] += dt[bi, t, h] * (g.T @ x[bi, t, h])
-                dl = a[t] * np.sum(g * hs[t])
-                out["ddt"][bi, t, h] = gB @ x[bi, t, h] + A[h] * dl
-                out["dA"][h] += dt[bi, t, h] * dl
-                out["dD"][h] += dy[bi, t, h] @ x[bi, t, h]
-                gnext, anext = g, a[t]
-            out["dinit"][bi, h] = anext * gnext
-    return out
+    assert dt.shape == (b, L, H) and A.shape == (H,) and D.shape == (H,) and dy.shape == x.shape
+    assert B.shape == (b, L, G, N) and C.shape == (b, L, G, N)
+    assert init is None or init.shape == (b, H, P, N)
+    assert dfinal is None or dfinal.shape == (b, H, P, N)
+    dx = np.zeros_like(x)
+    ddt = np.zeros_like(dt)
+    dB_h = np.zeros((b, L, H, N))
+    dC_h = np.zeros((b, L, H, N))
+    dA_bh = np.zeros((b, H))
+    dD_bh = np.zeros((b, H))
+    dinit = np.zeros((b, H, P, N))
+    rc = _load().oracle_ssd_scan_bwd(
+        b, L, H, P, N, G, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init),
+        _ptr(dy), _ptr(dfinal), _ptr(dx), _ptr(ddt), _ptr(dB_h), _ptr(dC_h), _ptr(dA_bh),
+        _ptr(dD_bh), _ptr(dinit))
+    if rc != 0:
+        raise RuntimeError("oracle_ssd_scan_bwd rejected its arguments")
+    hpg = H // G
+    return dict(dx=dx, ddt=ddt, dA=dA_bh.sum(0), dD=dD_bh.sum(0),
+                dB=dB_h.reshape(b, L, G, hpg, N).sum(3), dC=dC_h.reshape(b, L, G, hpg, N).sum(3),
+                dinit=dinit)
 
 
 def ssd_scan_varlen(x, dt, A, B, C, D, cu_seqlens, init=None):
