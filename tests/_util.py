@@ -40,3 +40,16 @@ def spread_pairs(batch, nheads, n, seed=0):
     while len(pairs) < min(n, batch * nheads):
         pairs.add((int(rng.integers(batch)), int(rng.integers(nheads))))
     return sorted(pairs)
+
+
+def max_rel_slices(gpu, ref, reduce_axes):
+    """Max relative L2 error over slices, vectorised: the norms are taken over `reduce_axes` of
+    the two equally shaped arrays and the worst slice is returned (with its index)."""
+    g = np.asarray(gpu, np.float64)
+    r = np.asarray(ref, np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    num = np.sqrt(np.sum((g - r) ** 2, axis=reduce_axes))
+    den = np.maximum(np.sqrt(np.sum(r ** 2, axis=reduce_axes)), 1e-30)
+    rel = num / den
+    i = int(np.argmax(rel))
+    return float(rel.flat[i]), np.unravel_index(i, rel.shape)

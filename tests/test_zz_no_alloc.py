@@ -5,8 +5,10 @@ inside a framework's planning or capture phase, a runtime that owns all device m
 with a fixed memory budget -- call ssd_chunk_scan_fwd_static.  It runs the same kernels but uses
 a scratch array built into the library instead of a caller-provided workspace.  These tests
 call it through the C ABI twice in a row (the second call must not be disturbed by what the
-first left in the shared array) and compare each result with the workspace entry point's, within
-the bf16 parity tolerance; they also check that problems larger than the array are refused.
+first left in the shared array), read the array's status word after each call, and require each
+result to equal the workspace entry point's bit for bit (the same kernels on the same inputs)
+and to match the float64 oracle within the bf16 parity tolerance; they also check that problems
+larger than the array are refused.
 
 The file is named so that pytest collects it last: if it fails, a run that stops at the first
 failure has already run every other test.
@@ -16,9 +18,10 @@ import ctypes
 import numpy as np
 import pytest
 
+import oracle
 from mamba_ssd_layer_scan_b200 import configs, inputs, ssd
 
-from _util import TOL, max_rel_per_pair, to_np, torch_inputs
+from _util import TOL, max_rel_slices, to_np, torch_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -28,6 +31,13 @@ def _static_entry():
     f.restype = ctypes.c_int
     f.argtypes = ([ctypes.POINTER(ssd.Shape)] + [ctypes.c_void_p] * 6 + [ctypes.c_int]
                   + [ctypes.c_void_p] * 4)
+    return f
+
+
+def _status_entry():
+    f = ssd.lib().ssd_chunk_scan_fwd_static_status
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p]
     return f
 
 
@@ -41,11 +51,14 @@ def _call_static(torch, t, w, chunk):
     final = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
                         device=t["x"].device)
     init = t["init_state"]
+    stream = torch.cuda.current_stream().cuda_stream
     rc = _static_entry()(ctypes.byref(_shape(w)), t["x"].data_ptr(), t["dt"].data_ptr(),
                          t["A"].data_ptr(), t["B"].data_ptr(), t["C"].data_ptr(),
                          t["D"].data_ptr(), chunk, None if init is None else init.data_ptr(),
-                         y.data_ptr(), final.data_ptr(), torch.cuda.current_stream().cuda_stream)
+                         y.data_ptr(), final.data_ptr(), stream)
     assert rc == ssd.SSD_OK, ssd.last_error()
+    st = _status_entry()(stream)
+    assert st == ssd.SSD_OK, ssd.last_error()
     return y, final
 
 
@@ -57,22 +70,24 @@ def test_static_scratch_matches_workspace_entry_point_on_two_calls(cuda_device):
     ]
     prepared = []
     for w, chunk in cases:
-        t = torch_inputs(inputs.make_inputs(w), cuda_device)
+        inp = inputs.make_inputs(w)
+        t = torch_inputs(inp, cuda_device)
         y_ref, f_ref = ssd.chunk_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk,
                                           init_state=t["init_state"])
-        prepared.append((w, chunk, t, y_ref, f_ref))
+        prepared.append((inp, chunk, t, y_ref, f_ref))
     torch.cuda.synchronize()
-    outs = [_call_static(torch, t, w, chunk) for w, chunk, t, _, _ in prepared]  # two in a row
+    outs = [_call_static(torch, t, inp.w, chunk) for inp, chunk, t, _, _ in prepared]
     torch.cuda.synchronize()
-    for (w, chunk, t, y_ref, f_ref), (y, f) in zip(prepared, outs):
-        yn, yr = to_np(y), to_np(y_ref)
-        fn, fr = to_np(f), to_np(f_ref)
-        pairs = [(b, h) for b in range(w.batch) for h in range(w.nheads)]
-        ey = max_rel_per_pair([yn[b, :, h] for b, h in pairs], [yr[b, :, h] for b, h in pairs])
-        ef = max_rel_per_pair([fn[b, h] for b, h in pairs], [fr[b, h] for b, h in pairs])
+    for (inp, chunk, t, y_ref, f_ref), (y, f) in zip(prepared, outs):
+        assert torch.equal(y, y_ref), "y differs from ssd_chunk_scan_fwd's"
+        assert torch.equal(f, f_ref), "final state differs from ssd_chunk_scan_fwd's"
+        yo, fo, _ = oracle.ssd_scan(inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, inp.init)
+        yn = to_np(y)
         assert np.isfinite(yn).all()
-        assert ey <= TOL[w.dtype], f"y differs from ssd_chunk_scan_fwd by {ey:.3e}"
-        assert ef <= TOL[w.dtype], f"final state differs from ssd_chunk_scan_fwd by {ef:.3e}"
+        ey = max_rel_slices(yn, yo, (1, 3))[0]
+        ef = max_rel_slices(to_np(f), fo, (2, 3))[0]
+        assert ey <= TOL[inp.w.dtype], f"y relative L2 error against the oracle {ey:.3e}"
+        assert ef <= TOL[inp.w.dtype], f"final state relative L2 error {ef:.3e}"
 
 
 def test_static_scratch_refuses_problems_larger_than_the_array(cuda_device):
