@@ -164,14 +164,15 @@ state_dot_kernel(const float *__restrict__ a, const float *__restrict__ c, float
 
 // One block per (b, h): the reverse cumsum of q over t (each thread a contiguous segment, the
 // segments' totals combined by a block-wide suffix scan), ddt, and the (b, h) partial sums of dA
-// and dD (atomically added per head).
+// and dD, written to part[0][b][h] and part[1][b][h] (summed over the batch in a fixed order by
+// batch_sum_kernel, so the result does not depend on the order the blocks run in).
 constexpr int kDecayThreads = 256;
 
 __global__ void __launch_bounds__(kDecayThreads)
 bwd_decay_kernel(const float *__restrict__ q, const float *__restrict__ ddt_in,
                  const float *__restrict__ dt, const float *__restrict__ A,
-                 const float *__restrict__ xdy, float *__restrict__ ddt, float *__restrict__ dA,
-                 float *__restrict__ dD, int64_t L, int H)
+                 const float *__restrict__ xdy, float *__restrict__ ddt, float *__restrict__ part,
+                 int64_t batch, int64_t L, int H)
 {
     __shared__ float wsum[kDecayThreads / 32];
     __shared__ float red[2][kDecayThreads / 32];
@@ -219,9 +220,21 @@ bwd_decay_kernel(const float *__restrict__ q, const float *__restrict__ ddt_in,
             a += red[0][j];
             d += red[1][j];
         }
-        atomicAdd(&dA[h], a);
-        atomicAdd(&dD[h], d);
+        part[b * H + h] = a;
+        part[(batch + b) * H + h] = d;
     }
+}
+
+// dA[h] = sum_b part[0][b][h], dD[h] = sum_b part[1][b][h], in batch order.
+__global__ void batch_sum_kernel(const float *__restrict__ part, float *__restrict__ dA,
+                                 float *__restrict__ dD, int64_t batch, int H)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= 2 * H) return;
+    const int h = i % H, which = i / H;
+    float s = 0.f;
+    for (int64_t b = 0; b < batch; ++b) s += part[(which * batch + b) * H + h];
+    (which ? dD : dA)[h] = s;
 }
 
 __global__ void group_sum_kernel(const float *__restrict__ in, const float *__restrict__ w,
@@ -325,15 +338,19 @@ cudaError_t launch_bwd_tokens(const bf16 *x, const bf16 *dy, const float *dt, co
 
 cudaError_t launch_bwd_decay(const float *q, const float *ddt_in, const float *dt,
                              const float *A, const float *xdy, float *ddt, float *dA, float *dD,
-                             int64_t batch, int64_t L, int H, cudaStream_t st)
+                             float *part, int64_t batch, int64_t L, int H, cudaStream_t st)
 {
-    cudaError_t e = cudaMemsetAsync(dA, 0, H * sizeof(float), st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dD, 0, H * sizeof(float), st);
-    if (e != cudaSuccess) return e;
     const int64_t n = batch * H;
-    if (n == 0 || L == 0) return cudaSuccess;
-    bwd_decay_kernel<<<(unsigned)n, kDecayThreads, 0, st>>>(q, ddt_in, dt, A, xdy, ddt, dA, dD,
-                                                           L, H);
+    if (n == 0 || L == 0) {
+        cudaError_t e = cudaMemsetAsync(dA, 0, H * sizeof(float), st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dD, 0, H * sizeof(float), st);
+        return e;
+    }
+    bwd_decay_kernel<<<(unsigned)n, kDecayThreads, 0, st>>>(q, ddt_in, dt, A, xdy, ddt, part,
+                                                           batch, L, H);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    batch_sum_kernel<<<(2 * H + 127) / 128, 128, 0, st>>>(part, dA, dD, batch, H);
     return cudaGetLastError();
 }
 

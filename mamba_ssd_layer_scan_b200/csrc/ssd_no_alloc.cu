@@ -15,6 +15,10 @@
 // call therefore does a little setup work and should happen before any stream capture.  The
 // address is then handed to the same kernels ssd_chunk_scan_fwd runs, as their workspace.
 //
+// The scratch address is cached per device ordinal, for the device's primary context (the one
+// the CUDA runtime uses); a caller that runs the scan in a context of its own making, or that
+// resets the device after the first call, is not supported.
+//
 // Nothing here allocates: no cudaMalloc, no cudaFree, no allocating library call.  Nothing in
 // the array needs to start at zero: the scan's first kernel clears the status word and every
 // other byte it reads was written earlier in the same call.  The array keeps whatever the last
@@ -95,6 +99,21 @@ ssd_status ssd_chunk_scan_fwd_static(const ssd_shape *shape, const void *x, cons
     }
     return ssd_chunk_scan_fwd(shape, x, dt, A, B, C, D, chunk_size, init_state, y, final_state,
                               scratch, kStaticScratchBytes, stream);
+}
+
+ssd_status ssd_chunk_scan_fwd_static_status(void *stream)
+{
+    void *scratch = nullptr;
+    const cudaError_t e = scratch_address(&scratch);
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof(msg),
+                 "ssd_chunk_scan_fwd_static_status: cannot get the scratch array's device "
+                 "address: %s", cudaGetErrorString(e));
+        ssd::set_last_error(msg);
+        return SSD_ERR_CUDA;
+    }
+    return ssd_workspace_status(scratch, kStaticScratchBytes, stream);
 }
 
 }  // extern "C"
