@@ -39,8 +39,9 @@ KERNELS = ("chunk_cumsum", "chunk_state", "state_passing", "chunk_scan")
 # Kernels of one ssd_chunk_scan_bwd call with dfinal and dinit, no initial state: a zero fill;
 # the reversed tensor-core scan (3 gathers, dt shift, 4 scan kernels) and dinit; the dB scan
 # (dfinal transpose, cumsum, chunk state, state passing, chunk scan, group sum) and the dC scan
-# (the same without a transpose); the final-state dot product, the token and decay kernels.
-BWD_KERNELS = 1 + 8 + 1 + 6 + 5 + 3
+# (the same without a transpose); the final-state dot product, the token and decay kernels and
+# the batch sum of dA and dD.
+BWD_KERNELS = 1 + 8 + 1 + 6 + 5 + 4
 KERNEL_SOURCES = {
     "chunk_cumsum": ["chunk_cumsum.cu"],
     "chunk_state": ["chunk_tc.cu", "sm100.cuh"],
@@ -55,30 +56,42 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def work_model(w):
     """Algorithmic bytes and flops per launch of each kernel, and for the whole step.
 
-    Bytes are what each kernel must move at minimum given its inputs and outputs (element size
-    e for x/B/C/y, 4 for fp32); flops count the dense Q x Q intra-chunk product as the method
-    materialises it, plus the chunk-state and off-chunk products (2NP each per token-head) and
-    C B^T once per group (2QN per token-group)."""
+    Algorithmic bytes are the compulsory traffic of the method: x, B, C and dt read, y written,
+    the initial state read and the final state written, each counted once (element size e for
+    x/B/C/y, 4 for float32).  Each kernel's share is the part of that traffic it must move:
+    the cumsum kernel reads dt; the chunk-state kernel reads x, B and dt; the state-passing
+    kernel reads the initial state and writes the final state; the chunk-scan kernel reads x, B,
+    C and dt and writes y.  What a
+    kernel moves beyond that is workspace traffic, reported separately as "ws_bytes": the
+    per-chunk float32 states (written by the chunk-state kernel, read by state passing), the
+    bf16 states entering each chunk (written by state passing, read by the chunk scan), and the
+    chunk-local cumsum rows (written by the cumsum kernel, read by the two tensor-core kernels;
+    the dt rows it re-lays out per chunk stand in for the dt those kernels count).  Flops count the dense Q x Q intra-chunk product as the method materialises it,
+    plus the chunk-state and off-chunk products (2NP each per token-head) and C B^T once per
+    group (2QN per token-group); "flops_causal" counts only the causal half of the Q x Q block."""
     b, L, H, P, N, G, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
     c = -(-L // Q)
     e = 2 if w.dtype == "bf16" else 4
     x = b * L * H * P * e
+    y = x
     bc = b * L * G * N * e
     dt = b * L * H * 4
-    cs = b * c * H * Q * 4
-    st = b * c * H * P * N
+    cs = b * c * H * Q * 4            # cs rows; the dt rows re-laid out per chunk are the same size
+    st = b * c * H * P * N            # elements of the per-chunk states
     fin = b * H * P * N * 4
     init = fin if w.init_state else 0
     k = {
-        "chunk_cumsum": {"bytes": dt + cs, "flops": 0},
-        "chunk_state": {"bytes": x + bc + dt + cs + st * 4, "flops": 2 * b * L * H * P * N},
-        "state_passing": {"bytes": st * 4 + st * 2 + fin + init, "flops": 0},
-        "chunk_scan": {"bytes": x + 2 * bc + dt + cs + st * 2 + x,
+        "chunk_cumsum": {"bytes": dt, "ws_bytes": 2 * cs, "flops": 0},
+        "chunk_state": {"bytes": x + bc + dt, "ws_bytes": cs + st * 4,
+                        "flops": 2 * b * L * H * P * N},
+        "state_passing": {"bytes": fin + init, "ws_bytes": cs // Q + st * 4 + st * 2,
+                          "flops": 0},
+        "chunk_scan": {"bytes": x + 2 * bc + dt + y, "ws_bytes": cs + st * 2,
                        "flops": b * L * H * (2 * Q * P + 2 * N * P) + b * L * G * 2 * Q * N,
                        "flops_causal": b * L * H * ((Q + 1) * P + 2 * N * P)
                        + b * L * G * (Q + 1) * N},
     }
-    total = {"bytes": x + 2 * bc + dt + x + fin + init,
+    total = {"bytes": x + 2 * bc + dt + y + fin + init,
              "flops": b * L * H * (2 * Q * P + 4 * N * P) + b * L * G * 2 * Q * N,
              "flops_causal": b * L * H * ((Q + 1) * P + 4 * N * P) + b * L * G * (Q + 1) * N}
     return k, total
@@ -261,6 +274,124 @@ def run_reference(args, w):
     return 0
 
 
+# ------------------------------------------------------------------ forward timing
+def device_inputs(torch, w, inp, dev):
+    xdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    host = {k: torch.from_numpy(np.ascontiguousarray(v)) for k, v in
+            dict(x=inp.x, dt=inp.dt, A=inp.A, B=inp.B, C=inp.C, D=inp.D).items()}
+    host["x"], host["B"], host["C"] = (host[k].to(xdt) for k in ("x", "B", "C"))
+    if inp.init is not None:
+        host["init"] = torch.from_numpy(np.ascontiguousarray(inp.init))
+    return host, {k: v.to(dev) for k, v in host.items()}
+
+
+def time_forward(ssd, torch, w, t, dev, stream, K, warmup, flush, barrier=lambda: None,
+                 before_timing=None):
+    """K plain ssd_chunk_scan_fwd calls, each bracketed by CUDA events on the launching stream
+    with the L2 flush written before it (outside the events), after `warmup` untimed calls;
+    then K staged calls (events between the kernels) for the per-kernel times.  Returns
+    (per-step ms, staged per-step ms, per-kernel ms lists, wall seconds of the timed loop)."""
+    shape = ssd.make_shape(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                           ssd.SSD_BF16 if w.dtype == "bf16" else ssd.SSD_F32)
+    ws = ssd.new_workspace(shape, w.chunk, dev)
+    y = torch.empty_like(t["x"])
+    final = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
+                        device=dev)
+    init = t.get("init")
+
+    def fwd(events=None):
+        ssd.chunk_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], w.chunk,
+                           init_state=init, y=y, final_state=final, workspace=ws,
+                           stage_events=events)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for row in ev:            # create the underlying CUDA events before handing them over
+        for e in row:
+            e.record(stream)
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        fwd()
+    torch.cuda.synchronize()
+    assert ssd.workspace_status(ws) == ssd.SSD_OK, "in-kernel timeout during warm-up"
+    if before_timing:
+        before_timing(fwd)
+    # The timed steps are plain calls: events recorded between the four kernels would keep each
+    # kernel from starting while its predecessor drains (programmatic dependent launch), so the
+    # per-kernel breakdown comes from a second, staged pass below.
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(K):
+        flush.fill_(1.0)
+        ev_step[i][0].record(stream)
+        fwd()
+        ev_step[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - wall0
+    assert ssd.workspace_status(ws) == ssd.SSD_OK, "in-kernel timeout during timing"
+    for i in range(K):
+        flush.fill_(1.0)
+        fwd(ev[i])
+    torch.cuda.synchronize()
+    assert ssd.workspace_status(ws) == ssd.SSD_OK, "in-kernel timeout during the staged pass"
+    step_ms = [a.elapsed_time(e) for a, e in ev_step]
+    staged_ms = [ev[i][0].elapsed_time(ev[i][4]) for i in range(K)]
+    kern_ms = {name: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)]
+               for j, name in enumerate(KERNELS)}
+    return step_ms, staged_ms, kern_ms, wall, (ws, y, final)
+
+
+def kernel_rooflines(w, staged_ms, kern_ms, hbm, tc_peak):
+    """Per kernel: mean time, share of the staged step, achieved GB/s on its algorithmic bytes
+    and on all the bytes it moves (algorithmic + workspace), TFLOP/s, the fractions of the
+    measured peaks, and which roof bounds it at its algorithmic intensity."""
+    kmodel, _ = work_model(w)
+    out = {}
+    for name in KERNELS:
+        ms = statistics.mean(kern_ms[name])
+        m = kmodel[name]
+        sec = ms / 1e3
+        gbs = m["bytes"] / sec / 1e9
+        gbs_moved = (m["bytes"] + m["ws_bytes"]) / sec / 1e9
+        tfs = m["flops"] / sec / 1e12
+        t_hbm = m["bytes"] / (hbm * 1e9)
+        t_tc = m["flops"] / (tc_peak * 1e12)
+        out[name] = {"ms": ms, "share": ms / statistics.mean(staged_ms), "gbs": gbs,
+                     "frac_hbm": gbs / hbm, "gbs_moved": gbs_moved,
+                     "frac_hbm_moved": gbs_moved / hbm, "tflops": tfs,
+                     "frac_tensor": tfs / tc_peak,
+                     "bound": "tensor" if t_tc > t_hbm else "hbm",
+                     "alg_bytes": m["bytes"], "ws_bytes": m["ws_bytes"], "alg_flops": m["flops"]}
+    return out
+
+
+def tensor_core_summary(w, kernels, tc_peak, hbm):
+    kmodel, _ = work_model(w)
+    tc_ms = kernels["chunk_state"]["ms"] + kernels["chunk_scan"]["ms"]
+    tc_flops = kmodel["chunk_state"]["flops"] + kmodel["chunk_scan"]["flops"]
+    tc_bytes = kmodel["chunk_state"]["bytes"] + kmodel["chunk_scan"]["bytes"]
+    tf = tc_flops / (tc_ms / 1e3) / 1e12
+    gb = tc_bytes / (tc_ms / 1e3) / 1e9
+    return {"tflops": tf, "frac_of_bf16_peak": tf / tc_peak, "gbs": gb, "frac_hbm": gb / hbm,
+            "ms": tc_ms, "flops": tc_flops, "alg_bytes": tc_bytes,
+            "kernels": ["chunk_state", "chunk_scan"]}
+
+
+def step_summary(w, ms_per_step, hbm, tc_peak):
+    _, total = work_model(w)
+    sec = ms_per_step / 1e3
+    return {"alg_bytes": total["bytes"], "alg_flops": total["flops"],
+            "alg_flops_causal": total["flops_causal"],
+            "gbs_compulsory": total["bytes"] / sec / 1e9,
+            "frac_hbm": total["bytes"] / sec / 1e9 / hbm,
+            "tflops_dense": total["flops"] / sec / 1e12,
+            "tflops_causal": total["flops_causal"] / sec / 1e12,
+            "frac_tensor_dense": total["flops"] / sec / 1e12 / tc_peak}
+
+
 # ------------------------------------------------------------------ our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -299,74 +430,38 @@ def main():
     # ---- inputs for the scan (same seeded draw on every rank: weak-scaling replicas)
     inp = inputs.make_inputs(w)
     xdt = torch.bfloat16
-    host = {k: torch.from_numpy(np.ascontiguousarray(v)) for k, v in
-            dict(x=inp.x, dt=inp.dt, A=inp.A, B=inp.B, C=inp.C, D=inp.D).items()}
-    host["x"], host["B"], host["C"] = (host[k].to(xdt) for k in ("x", "B", "C"))
+    host, t = device_inputs(torch, w, inp, dev)
     pinned = {k: v.pin_memory() for k, v in host.items()}
-    t = {k: v.to(dev) for k, v in host.items()}
-    shape = ssd.make_shape(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
-                           ssd.SSD_BF16)
-    ws = ssd.new_workspace(shape, w.chunk, dev)
-    y = torch.empty_like(t["x"])
-    final = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
-                        device=dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-
-    def fwd(events=None):
-        ssd.chunk_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], w.chunk, y=y,
-                           final_state=final, workspace=ws, stage_events=events)
-
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    for row in ev:            # create the underlying CUDA events before handing them over
-        for e in row:
-            e.record(stream)
-    for _ in range(args.warmup):
-        flush.fill_(1.0)
-        fwd()
-    torch.cuda.synchronize()
-    assert ssd.workspace_status(ws) == ssd.SSD_OK, "in-kernel timeout during warm-up"
 
     sampler = ClockSampler(nvml_index(torch, local)) if rank == 0 else None
-    if sampler:
-        sampler.start()
-        t_pre = time.perf_counter()
-        while time.perf_counter() - t_pre < 0.6:      # load the GPU while sampling starts
-            fwd()
-        torch.cuda.synchronize()
 
-    # The timed steps are plain calls: events recorded between the four kernels would keep each
-    # kernel from starting while its predecessor drains (programmatic dependent launch), so the
-    # per-kernel breakdown comes from a second, staged pass below.
-    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(K)]
-    barrier()
-    torch.cuda.synchronize()
-    wall0 = time.perf_counter()
-    for i in range(K):
-        flush.fill_(1.0)
-        ev_step[i][0].record(stream)
-        fwd()
-        ev_step[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    wall = time.perf_counter() - wall0
-    assert ssd.workspace_status(ws) == ssd.SSD_OK, "in-kernel timeout during timing"
-    for i in range(K):            # staged pass: per-kernel times for the rooflines
-        flush.fill_(1.0)
-        fwd(ev[i])
-    torch.cuda.synchronize()
+    def start_clocks(fwd):
+        if sampler:
+            sampler.start()
+            t_pre = time.perf_counter()
+            while time.perf_counter() - t_pre < 0.6:      # load the GPU while sampling starts
+                fwd()
+            torch.cuda.synchronize()
+
+    step_ms, staged_ms, kern_ms, wall, (ws, y, final) = time_forward(
+        ssd, torch, w, t, dev, stream, K, args.warmup, flush, barrier, start_clocks)
     clocks = sampler.stop() if sampler else None
-    assert ssd.workspace_status(ws) == ssd.SSD_OK, "in-kernel timeout during the staged pass"
-
-    step_ms = [a.elapsed_time(e) for a, e in ev_step]
-    staged_ms = [ev[i][0].elapsed_time(ev[i][4]) for i in range(K)]
-    kern_ms = {name: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)]
-               for j, name in enumerate(KERNELS)}
     total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / K
     tokens_per_step = w.batch * w.seqlen
     value = scaled_throughput(tokens_per_step * K, world, total_ms / 1e3)
+
+    # ---- the other forward workloads of the layer scan: the ~370M layer (batch 2 x 2048 x 24
+    # heads) and the long-context case (1 x 65536 tokens, 32 heads, 8 groups, initial state)
+    extra = {}
+    for wx in (configs.SSD_370M, configs.SSD_LONG):
+        _, tx = device_inputs(torch, wx, inputs.make_inputs(wx), dev)
+        Kx = max(10, min(K, 100))
+        sx, stx, kx, _, _ = time_forward(ssd, torch, wx, tx, dev, stream, Kx, args.warmup, flush)
+        extra[wx.name] = (wx, Kx, sx, stx, kx)
+        del tx
 
     # ---- end to end through the C ABI with host buffers: every step copies its inputs from
     # pinned host memory, runs the scan through the public API and copies y and the final state
@@ -562,19 +657,7 @@ def main():
     peaks, peak_src = load_peaks()
     hbm = peaks["hbm_gbs"]
     tc_peak = peaks["bf16_tflops"]
-    kmodel, total = work_model(w)
-    kernels = {}
-    for name in KERNELS:
-        ms = statistics.mean(kern_ms[name])
-        m = kmodel[name]
-        gbs = m["bytes"] / (ms / 1e3) / 1e9
-        tfs = m["flops"] / (ms / 1e3) / 1e12
-        t_hbm = m["bytes"] / (hbm * 1e9)
-        t_tc = m["flops"] / (tc_peak * 1e12)
-        kernels[name] = {"ms": ms, "share": ms / statistics.mean(staged_ms), "gbs": gbs,
-                         "frac_hbm": gbs / hbm, "tflops": tfs, "frac_tensor": tfs / tc_peak,
-                         "bound": "tensor" if t_tc > t_hbm else "hbm",
-                         "alg_bytes": m["bytes"], "alg_flops": m["flops"]}
+    kernels = kernel_rooflines(w, staged_ms, kern_ms, hbm, tc_peak)
     dom = max(KERNELS, key=lambda n: kernels[n]["ms"])
     kd = kernels[dom]
     if kd["bound"] == "tensor":
@@ -584,11 +667,27 @@ def main():
         roof = {"bound": "hbm", "achieved": kd["gbs"], "peak": hbm, "unit": "GB/s",
                 "frac": kd["gbs"] / hbm}
     roof.update({"kernel": dom, "traffic": profiled_traffic(dom, w.name),
-                 "alg_bytes_per_launch": kd["alg_bytes"], "alg_flops_per_launch": kd["alg_flops"],
-                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured"
-                 else "fallback"})
-    tc_ms = kernels["chunk_state"]["ms"] + kernels["chunk_scan"]["ms"]
-    tc_flops = kmodel["chunk_state"]["flops"] + kmodel["chunk_scan"]["flops"]
+                 "alg_bytes_per_launch": kd["alg_bytes"], "ws_bytes_per_launch": kd["ws_bytes"],
+                 "alg_flops_per_launch": kd["alg_flops"],
+                 "frac_hbm": kd["frac_hbm"], "frac_tensor": kd["frac_tensor"],
+                 "tensor_core_kernels": {n: {"frac_hbm": kernels[n]["frac_hbm"],
+                                             "frac_tensor": kernels[n]["frac_tensor"]}
+                                         for n in ("chunk_state", "chunk_scan")},
+                 "peak_source": (f"{peak_src} (MEASURED_PEAKS.json burst)"
+                                 if peak_src == "measured" else "fallback")})
+    config_lines = {}
+    for name, (wx, Kx, sx, stx, kx) in extra.items():
+        msx = max_over_ranks(sum(sx), dev) / Kx
+        kern_x = kernel_rooflines(wx, stx, kx, hbm, tc_peak)
+        config_lines[name] = {
+            "workload": name, "metric": "ssd_chunk_scan_fwd_tokens_per_s",
+            "value": scaled_throughput(wx.batch * wx.seqlen, world, msx / 1e3),
+            "unit": "tokens/s", "ms_per_step": msx, "steps": Kx,
+            "staged_ms_per_step": statistics.mean(stx),
+            "step_totals": step_summary(wx, msx, hbm, tc_peak),
+            "tensor_core_kernels": tensor_core_summary(wx, kern_x, tc_peak, hbm),
+            "kernels": kern_x,
+            "l2": "256 MB buffer written between timed steps (outside the events)"}
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -609,14 +708,10 @@ def main():
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
         "staged_ms_per_step": statistics.mean(staged_ms),
-        "tensor_core_kernels": {"tflops": tc_flops / (tc_ms / 1e3) / 1e12,
-                                "frac_of_bf16_peak": tc_flops / (tc_ms / 1e3) / 1e12 / tc_peak,
-                                "ms": tc_ms, "flops": tc_flops},
-        "step_totals": {"alg_bytes": total["bytes"], "alg_flops": total["flops"],
-                        "alg_flops_causal": total["flops_causal"],
-                        "gbs_compulsory": total["bytes"] / (ms_per_step / 1e3) / 1e9,
-                        "tflops_dense": total["flops"] / (ms_per_step / 1e3) / 1e12},
+        "tensor_core_kernels": tensor_core_summary(w, kernels, tc_peak, hbm),
+        "step_totals": step_summary(w, ms_per_step, hbm, tc_peak),
         "kernels": kernels,
+        "configs": config_lines,
         "fused_block": {"workload": w.name + "_gated_softplus_dt",
                         "metric": "ssd_chunk_scan_fwd_ex_tokens_per_s",
                         "value": tokens_per_step / (block_ms / 1e3), "unit": "tokens/s",
@@ -635,7 +730,8 @@ def main():
                      "ms_per_step": bwd_ms, "steps": Kg, "kernels_per_step": BWD_KERNELS,
                      "gradients": ["dx", "ddt", "dA", "dB", "dC", "dD", "dinit"],
                      "l2": "256 MB buffer written before each timed call (outside the events)"},
-        "decode": {"workload": wd.name, "metric": "ssd_state_update_GBps", "value":
+        "decode": {"workload": wd.name + " (one token's x, B, C and dt repeated every step)",
+                   "metric": "ssd_state_update_GBps", "value":
                    dbytes / (dec_ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": dec_ms,
                    "frac_hbm": dbytes / (dec_ms / 1e3) / 1e9 / hbm, "bytes_per_step": dbytes,
                    "tokens_per_s": wd.batch / (dec_ms / 1e3), "steps": Kd},
