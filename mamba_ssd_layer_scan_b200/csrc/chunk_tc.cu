@@ -65,25 +65,58 @@ struct alignas(1024) StateSmem {
     bf16 Xs[kStateStages][256 * 64];      // MN-major B operand per stage: [Q rows tau][64 p]
     float cs_v[kStateStages][256];        // per stage: the head's chunk-local cumsum row
     float dt_v[kStateStages][256];        // per stage: the head's dt row (0 past the end)
+    float cs_last[kMaxHeadsPerCta];       // chained form: each head's chunk log-decay
     uint64_t bar_b;
     uint64_t bar_x_full[kStateStages], bar_x_ready[kStateStages], bar_x_free[kStateStages];
     uint64_t bar_acc_full[2], bar_acc_free[2];
+    uint64_t bar_flag_ok, bar_pub;        // chained form: predecessor's state seen / ours stored
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort;
+    int ticket;
+    int published;                        // chained form: heads whose outgoing state is out
 };
 // warp 0 TMA, warps 1 and 3 MMA (alternate heads), warp 2 TMEM owner, warps 4-11 scale x,
 // warps 12-15 epilogue
 constexpr int kStateThreads = 512;
 constexpr int kStateScaleThreads = 256;
 constexpr uint32_t kStateTmemCols = 128;
+constexpr int kChainAbort = 0x40000000;   // flag value: the chain was broken by a timeout
 
+// The chained form of the chunk-state kernel carries the recurrence across chunks itself
+// (mohakchugh.is-a.dev "Mamba-2", Block Decomposition: across blocks the state is propagated
+// sequentially), so the float32 chunk states never go to HBM:
+//
+//     h_in[k+1] = exp(cs_k[Q-1]) h_in[k] + S_k          per (batch, head), chunk after chunk
+//
+// Work items (chunk, batch, group, head block) are handed out in chunk-major order by a ticket
+// counter, so an item only ever waits for an item with a smaller ticket, whose CTA has already
+// started: no wait can depend on a CTA that is not resident.  For each head the epilogue takes
+// S_k from TMEM, waits (bounded) until the item of chunk k-1 has published h_in[k] for that
+// head, writes h_in[k] as the chunk scan's bf16 operand, and publishes h_in[k+1] (float32, in a
+// two-slot ring per (batch, head) that stays in L2; the final state instead for the last chunk).
+// The ring is safe with two slots: the item of chunk k+1 overwrites slot k & 1 only after it has
+// read slot (k+1) & 1, which the item of chunk k wrote after it had read slot k & 1.
+__device__ __forceinline__ int ld_acquire_gpu(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int *p, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <bool kChain>
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                       const __grid_constant__ CUtensorMap tm_b, const float *__restrict__ dtc,
                       const float *__restrict__ cs, float *__restrict__ states,
                       int *__restrict__ status, int H, int G, int Q, int64_t nchunks, int nhb,
-                      int hpc, int64_t seqlen, const int2 *__restrict__ tab, int skip_cta)
+                      int hpc, int64_t seqlen, const int2 *__restrict__ tab, int skip_cta,
+                      StateChain chain)
 {
     extern __shared__ uint8_t smem_raw[];
     StateSmem &sm = *reinterpret_cast<StateSmem *>(
@@ -91,9 +124,23 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     int64_t u = blockIdx.x;
+    if (kChain) {
+        // the ticket counter is cleared by the cumsum kernel: wait for it first
+        griddep_wait();
+        if (threadIdx.x == 0) sm.ticket = atomicAdd(chain.counter, 1);
+        __syncthreads();
+        u = sm.ticket;   // chunk-major: u = ((k * batch + b) * G + g) * nhb + hb
+    }
     const int hb = (int)(u % nhb); u /= nhb;
     const int g = (int)(u % G); u /= G;
-    const int64_t k = u % nchunks, b = u / nchunks;
+    int64_t k, b;
+    if (kChain) {
+        b = u % chain.batch;
+        k = u / chain.batch;
+    } else {
+        k = u % nchunks;
+        b = u / nchunks;
+    }
     const int hpg = H / G;
     const int h0 = g * hpg + hb * hpc;
     const int nh = min(hpc, hpg - hb * hpc);
@@ -113,8 +160,11 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_init(&sm.bar_acc_full[s], 1);
             mbar_init(&sm.bar_acc_free[s], 128);
         }
+        mbar_init(&sm.bar_flag_ok, 1);
+        mbar_init(&sm.bar_pub, 128);
         mbar_init(&sm.bar_drain, 2);
         sm.abort = 0;
+        sm.published = 0;
         fence_mbar_init();
     }
     if (warp == 2) {
@@ -137,6 +187,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_arrive_expect_tx(&sm.bar_b, 2u * Q * kRowBytes);
             for (int a = 0; a < 2; ++a)   // boxes of Q rows
                 tma_load_4d(&sm.Bs[a][0], &tm_b, &sm.bar_b, 64 * a, g, (int)t0, (int)b);
+            // x is an input of the scan: start streaming the first heads' tiles into L2 while
+            // the cumsum kernel finishes
+            for (int j = 0; j < nh && j < kStateStages; ++j)
+                tma_prefetch_l2_4d(&tm_x, 0, h0 + j, (int)t0, (int)b);
             griddep_wait();   // cs / dt come from the cumsum kernel
             for (int j = 0; j < nh; ++j) {
                 const int s = j % kStateStages;
@@ -150,6 +204,9 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 tma_load_4d(&sm.Xs[s][0], &tm_x, &sm.bar_x_full[s], 0, h0 + j, (int)t0, (int)b);
                 bulk_load(sm.cs_v[s], cs + vrow, Q * 4, &sm.bar_x_full[s]);
                 bulk_load(sm.dt_v[s], dtc + vrow, Q * 4, &sm.bar_x_full[s]);
+                // the tile this stage will hold next: into L2 now, so its load is an L2 hit
+                if (j + kStateStages < nh)
+                    tma_prefetch_l2_4d(&tm_x, 0, h0 + j + kStateStages, (int)t0, (int)b);
             }
         }
     } else if (warp == 1 || warp == 3) {
@@ -195,6 +252,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             const uint32_t use = j / kStateStages;
             if (!warp_wait(&sm.bar_x_full[s], use & 1, abort)) break;
             const float cs_last = sm.cs_v[s][Q - 1];
+            if (kChain && st == 0) sm.cs_last[j] = cs_last;   // for the epilogue's carry
             for (int c = st; c < chunks; c += kStateScaleThreads) {
                 const int tau = c >> 3;
                 const float w = __expf(cs_last - sm.cs_v[s][tau]) * sm.dt_v[s][tau];
@@ -214,8 +272,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_arrive(&sm.bar_x_ready[s]);
         }
     } else if (warp >= 12) {
-        // ---------------- epilogue: TMEM (lane n, column p) -> states[b][k][h][p][n]
+        // ---------------- epilogue: TMEM (lane n, column p) -> S^T row n
         const int q = warp & 3;
+        const int n = q * 32 + lane;
+        const int et = threadIdx.x - 384;   // 0..127 within the epilogue warps
         for (int j = 0; j < nh; ++j) {
             const int a = j & 1;
             if (!warp_wait(&sm.bar_acc_full[a], (j >> 1) & 1, abort)) break;
@@ -227,12 +287,108 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(&sm.bar_acc_free[a]);
-            const int n = q * 32 + lane;
-            float *out = states + ((b * nchunks + k) * H + h0 + j) * (int64_t)(kP * kN) + n;
+            if (!kChain) {
+                // the chunk states are kept as [n][p]: 64 consecutive p per thread
+                float4 *out = reinterpret_cast<float4 *>(
+                    states + (((b * nchunks + k) * H + h0 + j) * (int64_t)kN + n) * kP);
 #pragma unroll
-            for (int p = 0; p < 32; ++p) out[p * kN] = __uint_as_float(r0[p]);
+                for (int c = 0; c < 8; ++c)
+                    __stcs(out + c,
+                           make_float4(__uint_as_float(r0[4 * c]), __uint_as_float(r0[4 * c + 1]),
+                                       __uint_as_float(r0[4 * c + 2]),
+                                       __uint_as_float(r0[4 * c + 3])));
 #pragma unroll
-            for (int p = 0; p < 32; ++p) out[(32 + p) * kN] = __uint_as_float(r1[p]);
+                for (int c = 0; c < 8; ++c)
+                    __stcs(out + 8 + c,
+                           make_float4(__uint_as_float(r1[4 * c]), __uint_as_float(r1[4 * c + 1]),
+                                       __uint_as_float(r1[4 * c + 2]),
+                                       __uint_as_float(r1[4 * c + 3])));
+                continue;
+            }
+            // ---- chained: the entering state h_in[k] of head h, then h_in[k+1].  Every
+            // hand-off between the four epilogue warps goes through an mbarrier with a bounded
+            // wait, so a timeout anywhere lets every thread leave the loop.
+            // Per head, thread 0 of the epilogue first completes bar_flag_ok (after seeing the
+            // previous chunk's state, for k > 0), and it completes it for head j + 1 only after
+            // bar_pub of head j, where all 128 threads have arrived: so no thread's wait or
+            // arrival on either barrier can fall a phase behind.
+            const int64_t bh = b * H + h0 + j;
+            int *flag = chain.flags + bh;
+            if (et == 0) {
+                if (k > 0) {
+                    // bounded wait for the item of chunk k-1 (a smaller ticket, already running)
+                    const unsigned long long tw = globaltimer();
+                    int f;
+                    while ((f = ld_acquire_gpu(flag)) < (int)k) {
+                        if (*abort || globaltimer() - tw > kWaitLimitNs) {
+                            *abort = 1;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    if (f >= kChainAbort) *abort = 1;
+                }
+                mbar_arrive(&sm.bar_flag_ok);
+            }
+            if (!warp_wait(&sm.bar_flag_ok, j & 1, abort)) break;
+            if (__shfl_sync(0xffffffffu, *abort, 0)) break;
+            const float dec = __expf(sm.cs_last[j]);
+            bf16 *hrow = chain.hin + ((b * nchunks + k) * H + h0 + j) * (int64_t)(kP * kN) + n * 64;
+            const float *ring_in = chain.ring + ((bh * 2 + (k & 1)) * kN + n) * (int64_t)kP;
+            float *ring_out = chain.ring + ((bh * 2 + ((k + 1) & 1)) * kN + n) * (int64_t)kP;
+            const float *ip = chain.init ? chain.init + bh * (int64_t)(kP * kN) + n : nullptr;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const uint32_t *sv = half ? r1 : r0;
+                float hv[32];
+                if (k == 0) {
+#pragma unroll
+                    for (int p = 0; p < 32; ++p) hv[p] = ip ? ip[(32 * half + p) * kN] : 0.f;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(ring_in) +
+                                                8 * half + c);
+                        hv[4 * c] = v.x;
+                        hv[4 * c + 1] = v.y;
+                        hv[4 * c + 2] = v.z;
+                        hv[4 * c + 3] = v.w;
+                    }
+                }
+                // h_in[k+1] = exp(cs_last) h_in[k] + S_k: the ring slot the next chunk reads, or
+                // the final state after the last chunk
+                if (k + 1 < nchunks) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        __stcg(reinterpret_cast<float4 *>(ring_out) + 8 * half + c,
+                               make_float4(fmaf(dec, hv[4 * c], __uint_as_float(sv[4 * c])),
+                                           fmaf(dec, hv[4 * c + 1], __uint_as_float(sv[4 * c + 1])),
+                                           fmaf(dec, hv[4 * c + 2], __uint_as_float(sv[4 * c + 2])),
+                                           fmaf(dec, hv[4 * c + 3], __uint_as_float(sv[4 * c + 3]))));
+                } else if (chain.final_state) {
+                    float *fo = chain.final_state + bh * (int64_t)(kP * kN) + n;
+#pragma unroll
+                    for (int p = 0; p < 32; ++p)
+                        fo[(32 * half + p) * kN] = fmaf(dec, hv[p], __uint_as_float(sv[p]));
+                }
+                // h_in[k] as the chunk scan's operand: row n of 64 p, 16-byte pieces swizzled
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int piece = 4 * half + c;
+                    *reinterpret_cast<uint4 *>(hrow + 8 * (piece ^ (n & 7))) =
+                        make_uint4(pack_bf16x2(hv[8 * c], hv[8 * c + 1]),
+                                   pack_bf16x2(hv[8 * c + 2], hv[8 * c + 3]),
+                                   pack_bf16x2(hv[8 * c + 4], hv[8 * c + 5]),
+                                   pack_bf16x2(hv[8 * c + 6], hv[8 * c + 7]));
+                }
+            }
+            // every thread's part of h_in[k+1] is visible GPU-wide before the flag
+            if (k + 1 < nchunks) __threadfence();
+            mbar_arrive(&sm.bar_pub);
+            if (et == 0 && mbar_wait(&sm.bar_pub, j & 1, abort) && k + 1 < nchunks) {
+                st_release_gpu(flag, (int)(k + 1));
+                sm.published = j + 1;
+            }
         }
     }
 
@@ -244,8 +400,13 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_wait_drain(&sm.bar_drain, 0);
         }
         if (threadIdx.x == 0) {
+            // chained form: heads whose outgoing state was not published break the chain on
+            // purpose, so that the later chunks' items stop waiting at once
+            if (kChain && k + 1 < nchunks)
+                for (int j = sm.published; j < nh; ++j)
+                    st_release_gpu(chain.flags + b * H + h0 + j, kChainAbort);
             drain_sleep();
-            atomicOr(status, 1);
+            atomicOr(status, kChain ? 4 : 1);
         }
     }
     tc_fence_before();
@@ -284,7 +445,7 @@ struct alignas(1024) ScanSmem {
                                     // that, T = 0: x / h_in stage 2; T = 1: bf16 C B_off^T
                                     // (K-major [i atom][128 rows t][64 i])
     uint8_t S01[2][kStageBytes];    // x / h_in stages 0 and 1: [KI rows i][64 p] then
-                                    // [n atom][64 rows p][64 n]
+                                    // [128 rows n][64 p]
     float cs_v[kScanVecStages][256];  // per stage: one head's chunk-local cumsum row
     float dt_v[kScanVecStages][256];  // per stage: its dt row (0 past the end)
     float vt[16][32];               // per worker warp: column factors of its two slices
@@ -428,6 +589,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 for (int r = 0; r <= T; ++r)
                     tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
                                 64 * a, g, (int)(t0 + kTileRows * r), (int)b);
+            // x is an input of the scan: start streaming the first heads' tiles into L2 while
+            // the state-passing kernel finishes
+            for (int j = 0; j < nh && j < nst; ++j)
+                tma_prefetch_l2_4d(T ? &tm_x2 : &tm_x, 0, h0 + j, (int)t0, (int)b);
             griddep_wait();   // cs / dt and the entering states come from earlier kernels
         }
         for (int j = 0; lane == 0 && j < nh; ++j) {   // lane 0 alone runs the loop
@@ -454,6 +619,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             tma_load_4d(stg, T ? &tm_x2 : &tm_x, &sm.bar_xh_full[xs], 0, h, (int)t0, (int)b);
             bulk_load(stg + kHOff, hin + ((b * nchunks + k) * H + h) * (int64_t)(kP * kN),
                       kP * kN * 2, &sm.bar_xh_full[xs]);
+            // the operands this stage will hold next: into L2 now, so their loads are L2 hits
+            if (j + nst < nh) {
+                tma_prefetch_l2_4d(T ? &tm_x2 : &tm_x, 0, h + nst, (int)t0, (int)b);
+                bulk_prefetch_l2(hin + ((b * nchunks + k) * H + h + nst) * (int64_t)(kP * kN),
+                                 kP * kN * 2);
+            }
             // the gate rows this tile's epilogue will read: into L2 now, a few heads ahead
             if (kGate) tma_prefetch_l2_4d(&tm_z, 0, h, (int)(t0 + kTileRows * T), (int)b);
         }
@@ -461,7 +632,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         // ---------------- MMA issuer (lane 0 alone runs the loop: a lane that issued
         // tcgen05.mma and then rejoins its warp stalls for the MMAs' issue latency)
         const uint32_t id_g = idesc_bf16_f32(128, KI, false, false);
-        const uint32_t id_kk = idesc_bf16_f32(128, kP, false, false);   // K-major A and B
         const uint32_t id_kmn = idesc_bf16_f32(128, kP, false, true);   // B (x) MN-major
         // base descriptors; K steps are constant offsets added in fully unrolled loops (the
         // issuing thread's own instruction chain sets the MMA issue rate)
@@ -491,7 +661,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             const uint32_t stg = smem_u32(scan_stage(sm, xs));
             const uint32_t dD = tmem + kAccCol + 128 * a, dA = dD + 64;
             const uint64_t xd = smem_desc_sw128(stg, 256 * kRowBytes, 1024);   // x, MN-major
-            const uint64_t hd = smem_desc_sw128(stg + kHOff, 16, 1024);        // h_in, K-major
+            const uint64_t hd = smem_desc_sw128(stg + kHOff, 16384, 1024);     // h_in, MN-major
             if (T) {
                 // Y_A = (C B_off^T) (v dt o X_off): A = bf16 block in R, K = 128 (i)
 #pragma unroll
@@ -500,12 +670,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     mma_bf16(dA, rd + (aoff >> 4), xd + kk * 128, id_kmn, kk > 0 ? 1u : 0u);
                 }
             }
-            // Y_A (+)= C h^T: K = 128 (n); h = h_in (T = 0) or exp(cs_127) h_in (T = 1)
+            // Y_A (+)= C h^T: K = 128 (n), h^T MN-major (rows n); h = h_in (T = 0) or
+            // exp(cs_127) h_in (T = 1)
 #pragma unroll
             for (int kk = 0; kk < kN / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                const uint32_t hoff = (kk >> 2) * (kP * kRowBytes) + (kk & 3) * 32;
-                mma_bf16(dA, cd + (off >> 4), hd + (hoff >> 4), id_kk, (T || kk > 0) ? 1u : 0u);
+                mma_bf16(dA, cd + (off >> 4), hd + kk * 128, id_kmn, (T || kk > 0) ? 1u : 0u);
             }
             for (int qb = 0; qb < 2; ++qb) {
                 const uint32_t blk = 2 * j + qb;           // P blocks are numbered per head
@@ -838,7 +1008,8 @@ bool tc_supported(bool is_bf16, int P, int N, int Q)
 cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
-                                  cudaStream_t st, const char **why, const int2 *tab)
+                                  cudaStream_t st, const char **why, const int2 *tab,
+                                  const StateChain *chain)
 {
     CUtensorMap mx, mb;   // boxes of a whole chunk (Q rows)
     if (!make_seq_map(&mx, x, batch, seqlen, H, kP, Q) ||
@@ -846,18 +1017,24 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
         *why = "chunk state: cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
+    if (chain && tab) {
+        *why = "chunk state: the chained form takes fixed-length input only";
+        return cudaErrorInvalidValue;
+    }
     const int hpg = H / G;
     const int hpc = heads_per_cta(batch * nchunks * G, hpg, 4.0, 2.0);
     const int nhb = (hpg + hpc - 1) / hpc;
     const size_t smem = sizeof(StateSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(chunk_state_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = chain ? chunk_state_tc_kernel<true> : chunk_state_tc_kernel<false>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk state: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb);
-    *why = "chunk state (tcgen05) launch";
-    return launch_pdl(chunk_state_tc_kernel, grid, kStateThreads, smem, st, mx, mb, dtc, cs,
-                      states, status, H, G, Q, nchunks, nhb, hpc, seqlen, tab,
-                      take_test_skip(kTestChunkState));
+    StateChain none = {};
+    *why = chain ? "chained chunk state (tcgen05) launch" : "chunk state (tcgen05) launch";
+    return launch_pdl(kern, grid, kStateThreads, smem, st, mx, mb, dtc, cs, states, status, H, G,
+                      Q, nchunks, nhb, hpc, seqlen, tab, take_test_skip(kTestChunkState),
+                      chain ? *chain : none);
 }
 
 cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,

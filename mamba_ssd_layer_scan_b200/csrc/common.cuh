@@ -72,11 +72,16 @@ struct WsLayout {
     size_t status;      // 256 bytes: device status word (nonzero after an in-kernel timeout)
     size_t cs;          // float [b][c][H][Q]: chunk-local inclusive cumsum of dt*A
     size_t dtc;         // float [b][c][H][Q]: dt per chunk row, 0 past the end (tensor-core path)
-    size_t states;      // float [b][c][H][P][N]: per-chunk state, then (in place) state entering
+    size_t states;      // float [b][c][H][P][N] (CUDA-core path) or [b][c][H][N][P] (tensor-core
+                        // path): per-chunk state, then (in place) state entering
     size_t hin_bf16;    // bf16  [b][c][H] blocks of P x N (hin_swizzled_offset): state entering
                         // each chunk (tensor-core path)
+    size_t sync;        // int [kSyncFlags + b * H]: the chained chunk state's ticket counter (at
+                        // 0) and per-(batch, head) flags (from kSyncFlags) (tensor-core path)
     size_t total;
 };
+
+constexpr int kSyncFlags = 64;   // the flags start one 256-byte line after the counter
 
 // Where chunk k of the workspace sits in the token sequence.  Without a table (fixed-length
 // input) chunk k of batch row b starts at token k Q of that row and holds min(Q, L - k Q)
@@ -96,7 +101,8 @@ __device__ __forceinline__ void chunk_span(const int2 *tab, int64_t k, int Q, in
     }
 }
 
-// Workspace status word bits: 1, 2 = a bounded wait timed out (chunk state, chunk scan);
+// Workspace status word bits: 1, 2, 4 = a bounded wait timed out (chunk state, chunk scan,
+// chained chunk state);
 // kStatusBadSeqlens = the cu_seqlens of a variable-length call are inconsistent.
 constexpr int kStatusBadSeqlens = 0x10000;
 
@@ -112,12 +118,14 @@ constexpr int kTestChunkScan = 2;
 int take_test_skip(int kernel);
 
 // ---- launchers (each returns the launch's cudaError_t) ----
-// Also zeroes *status (nullable) so each scan starts with a clean status word, and, when dtc is
-// non-null, writes dt re-laid out as (b, c, H, Q) with zeros past the end of the sequence.
+// Also zeroes *status (nullable) so each scan starts with a clean status word, and the nsync
+// ints at sync (nullable: the chained chunk state's counter and flags); when dtc is non-null,
+// writes dt re-laid out as (b, c, H, Q) with zeros past the end of the sequence.
 cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, float *dtc,
                                 int *status, int64_t batch, int64_t seqlen, int nheads, int Q,
                                 int64_t nchunks, cudaStream_t st, const int2 *tab = nullptr,
-                                bool unit_weights = false);
+                                bool unit_weights = false, int *sync = nullptr,
+                                int64_t nsync = 0);
 
 // Packed variable-length input: the chunk table (tab, nchunks entries) and the first chunk of
 // every sequence (cstart, nseq + 1 entries) from cu_seqlens; clears *status and sets
@@ -133,6 +141,8 @@ cudaError_t launch_chunk_state_simt(bool is_bf16, const void *x, const float *dt
 
 // Carries the state across chunks: states[k] (chunk-local contribution) is replaced in place by
 // the state entering chunk k (float32), or that state is written to hin_bf16 when non-null.
+// With hin_bf16 (the tensor-core path) the chunk states are stored transposed, [N][P] per
+// (batch, chunk, head); init and final_state are always in the caller's [P][N] layout.
 cudaError_t launch_state_passing(float *states, const float *cs, const float *init,
                                  float *final_state, bf16 *hin_bf16, int64_t batch, int H,
                                  int P, int N, int Q, int64_t nchunks, cudaStream_t st);
@@ -174,19 +184,34 @@ cudaError_t launch_fill_final(const float *init, float *final_state, int64_t n,
 
 // Tensor-core (tcgen05 + TMA) path: bf16, P = 64, N = 128, Q in {128, 256}.
 bool tc_supported(bool is_bf16, int P, int N, int Q);
+
+// The chained form of the chunk-state kernel (fixed-length input only): it also carries the
+// state across chunks, so no float32 chunk states go to HBM and no state-passing kernel runs.
+// ring: batch * H * 2 * P * N floats; flags: batch * H ints and counter: one int, all zero at
+// the launch (the cumsum kernel clears them).  hin receives the bf16 entering states,
+// final_state (nullable) the float32 state after the last chunk, from init (nullable).
+struct StateChain {
+    float *ring;
+    int *flags;
+    int *counter;
+    const float *init;
+    float *final_state;
+    bf16 *hin;
+    int64_t batch;
+};
 cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
-                                  cudaStream_t st, const char **why, const int2 *tab = nullptr);
+                                  cudaStream_t st, const char **why, const int2 *tab = nullptr,
+                                  const StateChain *chain = nullptr);
 // Offset (in elements), inside one (batch, chunk, head) block of the bf16 entering states, of
 // state element (p, n) for P = 64, N = 128.  The block is stored exactly as the tensor cores
-// read it from shared memory: two halves of 64 n, each 64 rows p of 128 bytes, with the 16-byte
-// pieces of row p permuted by p mod 8 (the 128-byte swizzle), so that one contiguous 16 KB copy
-// brings a block into shared memory ready for use.
+// read it from shared memory as the MN-major operand h^T (K = n, N = p): 128 rows n of 64 p
+// (128 bytes), the 16-byte pieces of row n permuted by n mod 8 (the 128-byte swizzle), so that
+// one contiguous 16 KB copy brings a block into shared memory ready for use.
 __host__ __device__ __forceinline__ int hin_swizzled_offset(int p, int n)
 {
-    const int a = n >> 6, nl = n & 63;
-    return a * 4096 + p * 64 + ((((nl >> 3) ^ (p & 7)) << 3) | (nl & 7));
+    return n * 64 + ((((p >> 3) ^ (n & 7)) << 3) | (p & 7));
 }
 
 // Sequence parallelism (one contiguous segment per rank): the segment's total log-decay per

@@ -165,6 +165,14 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
                  "r"(c2), "r"(c3), "r"(smem_u32(bar)) : "memory");
 }
 
+// Bring `bytes` of contiguous global memory (16-byte aligned, a multiple of 16 bytes) into L2
+// ahead of a later copy of it (no shared memory, no barrier).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                 ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes) : "memory");
+}
+
 // Contiguous global -> shared copy by the TMA unit (both addresses 16-byte aligned, size a
 // multiple of 16 bytes), completing `bytes` transactions on `bar`.  No cluster multicast.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,

@@ -14,7 +14,7 @@ import pytest
 import oracle
 from mamba_ssd_layer_scan_b200 import configs, inputs, ssd
 
-from _util import TOL, max_rel_per_pair, max_rel_slices, to_np, torch_inputs
+from _util import TOL, max_rel_per_pair, max_rel_slices, set_state_form, to_np, torch_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -105,17 +105,44 @@ def test_small_full_parity(cuda_device, name, w, chunk):
     check_against_oracle(inp, y, final)
 
 
-# The tensor-core cases again with a nonzero initial state and a fresh draw.
+# The tensor-core cases again with a nonzero initial state and a fresh draw, once with each way
+# of carrying the state across chunks: the chunk-state kernel followed by the state-passing
+# kernel (form 1), and the chained chunk-state kernel that carries it itself (form 2).
 TC_SMALL = [s for s in SMALL if s[0].startswith("bf16_tc")]
 
 
+@pytest.fixture
+def state_form():
+    yield set_state_form
+    set_state_form(0)
+
+
+@pytest.mark.parametrize("form", [1, 2], ids=["two_kernels", "chained"])
 @pytest.mark.parametrize("name,w,chunk", TC_SMALL, ids=[s[0] for s in TC_SMALL])
-def test_small_parity_with_initial_state(cuda_device, name, w, chunk):
+def test_small_parity_with_initial_state(cuda_device, state_form, form, name, w, chunk):
     import torch
+    state_form(form)
     inp = inputs.make_inputs(w.with_(init_state=True, seed=w.seed + 17))
     t = torch_inputs(inp, cuda_device)
     y, final = run_fwd(torch, t, inp.w, chunk, cuda_device)
     check_against_oracle(inp, y, final)
+
+
+@pytest.mark.parametrize("w", [configs.SSD_2P7B.with_(init_state=True),
+                               configs.SSD_LONG.with_(seqlen=16384)],
+                         ids=["ssd_2p7b_init", "long_g8_64_chunks"])
+def test_state_forms_are_bit_identical(cuda_device, state_form, w):
+    """Both forms run the same arithmetic (the same MMAs for the chunk states, the same
+    fused multiply-add and rounding for the carry), so y and the final state agree bit for bit."""
+    import torch
+    inp = inputs.make_inputs(w)
+    t = torch_inputs(inp, cuda_device)
+    outs = []
+    for form in (1, 2):
+        state_form(form)
+        outs.append(run_fwd(torch, t, w, w.chunk, cuda_device, guards=False))
+    assert torch.equal(outs[0][0], outs[1][0]), "y differs between the two forms"
+    assert torch.equal(outs[0][1], outs[1][1]), "final state differs between the two forms"
 
 
 # ------------------------------------------------------------------ full-size workloads
