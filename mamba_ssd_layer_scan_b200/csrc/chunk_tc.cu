@@ -66,6 +66,7 @@ struct alignas(1024) StateSmem {
     float cs_v[kStateStages][256];        // per stage: the head's chunk-local cumsum row
     float dt_v[kStateStages][256];        // per stage: the head's dt row (0 past the end)
     float cs_last[kMaxHeadsPerCta];       // chained form: each head's chunk log-decay
+    float cs_mid[kMaxHeadsPerCta];        // chained form, Q = 256: its log-decay to row 127
     uint64_t bar_b;
     uint64_t bar_x_full[kStateStages], bar_x_ready[kStateStages], bar_x_free[kStateStages];
     uint64_t bar_acc_full[2], bar_acc_free[2];
@@ -80,7 +81,7 @@ struct alignas(1024) StateSmem {
 // warps 12-15 epilogue
 constexpr int kStateThreads = 512;
 constexpr int kStateScaleThreads = 256;
-constexpr uint32_t kStateTmemCols = 128;
+constexpr uint32_t kStateTmemCols = 256;   // two buffers of (rows 0-127, rows 128-255) x 64 p
 constexpr int kChainAbort = 0x40000000;   // flag value: the chain was broken by a timeout
 
 // The chained form of the chunk-state kernel carries the recurrence across chunks itself
@@ -225,12 +226,21 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 if (!mbar_wait(&sm.bar_x_ready[s], use & 1, abort)) break;
                 if (j >= 2 && !mbar_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
                 tc_fence_after();
-                const uint32_t d = tmem + a * kP;
+                const uint32_t d = tmem + a * 128;
                 // base descriptors + constant K steps (16 rows = 2048 bytes) in fully unrolled
                 // loops: the issuing thread's own instruction chain sets the MMA issue rate
                 const uint64_t ad = smem_desc_sw128(smem_u32(&sm.Bs[0][0]), atom_bytes, 1024);
                 const uint64_t bd = smem_desc_sw128(smem_u32(&sm.Xs[s][0]), atom_bytes, 1024);
-                if (Q == 256) {
+                if (Q == 256 && kChain) {
+                    // chained form: rows 0-127 and rows 128-255 into separate accumulators (the
+                    // state at row 127 is the second half-chunk's entering state)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(d, ad + kk * 128, bd + kk * 128, idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 8; kk < 16; ++kk)
+                        mma_bf16(d + 64, ad + kk * 128, bd + kk * 128, idesc, kk > 8 ? 1u : 0u);
+                } else if (Q == 256) {
 #pragma unroll
                     for (int kk = 0; kk < 16; ++kk)
                         mma_bf16(d, ad + kk * 128, bd + kk * 128, idesc, kk > 0 ? 1u : 0u);
@@ -252,10 +262,18 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             const uint32_t use = j / kStateStages;
             if (!warp_wait(&sm.bar_x_full[s], use & 1, abort)) break;
             const float cs_last = sm.cs_v[s][Q - 1];
-            if (kChain && st == 0) sm.cs_last[j] = cs_last;   // for the epilogue's carry
+            // chained form, Q = 256: rows 0-127 are decayed to row 127 (their own accumulator),
+            // rows 128-255 to the chunk's last row; otherwise every row to the last row
+            const bool halves = kChain && Q == 256;
+            const float cs_ref0 = halves ? sm.cs_v[s][127] : cs_last;
+            if (kChain && st == 0) {   // for the epilogue's carry
+                sm.cs_last[j] = cs_last;
+                sm.cs_mid[j] = cs_ref0;
+            }
             for (int c = st; c < chunks; c += kStateScaleThreads) {
                 const int tau = c >> 3;
-                const float w = __expf(cs_last - sm.cs_v[s][tau]) * sm.dt_v[s][tau];
+                const float ref = tau < 128 ? cs_ref0 : cs_last;
+                const float w = __expf(ref - sm.cs_v[s][tau]) * sm.dt_v[s][tau];
                 uint4 *ptr = reinterpret_cast<uint4 *>(&sm.Xs[s][0]) + c;
                 uint4 v = *ptr;
                 uint32_t *wv = &v.x;
@@ -280,14 +298,14 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             const int a = j & 1;
             if (!warp_wait(&sm.bar_acc_full[a], (j >> 1) & 1, abort)) break;
             tc_fence_after();
-            uint32_t r0[32], r1[32];
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + a * kP;
-            tmem_ld32(taddr, r0);
-            tmem_ld32(taddr + 32, r1);
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(&sm.bar_acc_free[a]);
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + a * 128;
             if (!kChain) {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(taddr, r0);
+                tmem_ld32(taddr + 32, r1);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&sm.bar_acc_free[a]);
                 // the chunk states are kept as [n][p]: 64 consecutive p per thread
                 float4 *out = reinterpret_cast<float4 *>(
                     states + (((b * nchunks + k) * H + h0 + j) * (int64_t)kN + n) * kP);
@@ -332,56 +350,87 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             }
             if (!warp_wait(&sm.bar_flag_ok, j & 1, abort)) break;
             if (__shfl_sync(0xffffffffu, *abort, 0)) break;
+            // Q = 256: the accumulators hold S_lo (rows 0-127, decayed to row 127) and S_hi
+            // (rows 128-255, decayed to row 255); the chunk's own state is
+            // S = exp(cs_255 - cs_127) S_lo + S_hi, and the state entering rows 128-255 is
+            // h_mid = exp(cs_127) h_in[k] + S_lo.  Q = 128: one accumulator, S.
+            const bool halves = Q == 256;
             const float dec = __expf(sm.cs_last[j]);
-            bf16 *hrow = chain.hin + ((b * nchunks + k) * H + h0 + j) * (int64_t)(kP * kN) + n * 64;
+            const float dmid = __expf(sm.cs_mid[j]);
+            const float dhl = __expf(sm.cs_last[j] - sm.cs_mid[j]);
+            const int nsub = Q / kTileRows;
+            const int64_t sub0 = (b * nchunks + k) * nsub;   // sub-chunk index of rows 0-127
+            bf16 *hrow = chain.hin + (sub0 * H + h0 + j) * (int64_t)(kP * kN) + n * 64;
+            bf16 *mrow = chain.hin + ((sub0 + 1) * H + h0 + j) * (int64_t)(kP * kN) + n * 64;
             const float *ring_in = chain.ring + ((bh * 2 + (k & 1)) * kN + n) * (int64_t)kP;
             float *ring_out = chain.ring + ((bh * 2 + ((k + 1) & 1)) * kN + n) * (int64_t)kP;
             const float *ip = chain.init ? chain.init + bh * (int64_t)(kP * kN) + n : nullptr;
+            // 16 columns p at a time (registers: the accumulators, the entering state)
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const uint32_t *sv = half ? r1 : r0;
-                float hv[32];
+            for (int qq = 0; qq < 4; ++qq) {
+                uint32_t lo[16], hi[16];
+                tmem_ld16(taddr + 16 * qq, lo);
+                if (halves) tmem_ld16(taddr + 64 + 16 * qq, hi);
+                float hv[16];
                 if (k == 0) {
 #pragma unroll
-                    for (int p = 0; p < 32; ++p) hv[p] = ip ? ip[(32 * half + p) * kN] : 0.f;
+                    for (int p = 0; p < 16; ++p) hv[p] = ip ? ip[(16 * qq + p) * kN] : 0.f;
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
+                    for (int c = 0; c < 4; ++c) {
                         const float4 v = __ldcg(reinterpret_cast<const float4 *>(ring_in) +
-                                                8 * half + c);
+                                                4 * qq + c);
                         hv[4 * c] = v.x;
                         hv[4 * c + 1] = v.y;
                         hv[4 * c + 2] = v.z;
                         hv[4 * c + 3] = v.w;
                     }
                 }
-                // h_in[k+1] = exp(cs_last) h_in[k] + S_k: the ring slot the next chunk reads, or
-                // the final state after the last chunk
-                if (k + 1 < nchunks) {
+                tmem_ld_wait();
+                // the entering states of the two half-chunks as the chunk scan's operands:
+                // row n of 64 p, 16-byte pieces swizzled
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        __stcg(reinterpret_cast<float4 *>(ring_out) + 8 * half + c,
-                               make_float4(fmaf(dec, hv[4 * c], __uint_as_float(sv[4 * c])),
-                                           fmaf(dec, hv[4 * c + 1], __uint_as_float(sv[4 * c + 1])),
-                                           fmaf(dec, hv[4 * c + 2], __uint_as_float(sv[4 * c + 2])),
-                                           fmaf(dec, hv[4 * c + 3], __uint_as_float(sv[4 * c + 3]))));
-                } else if (chain.final_state) {
-                    float *fo = chain.final_state + bh * (int64_t)(kP * kN) + n;
-#pragma unroll
-                    for (int p = 0; p < 32; ++p)
-                        fo[(32 * half + p) * kN] = fmaf(dec, hv[p], __uint_as_float(sv[p]));
-                }
-                // h_in[k] as the chunk scan's operand: row n of 64 p, 16-byte pieces swizzled
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int piece = 4 * half + c;
+                for (int c = 0; c < 2; ++c) {
+                    const int piece = 2 * qq + c;
                     *reinterpret_cast<uint4 *>(hrow + 8 * (piece ^ (n & 7))) =
                         make_uint4(pack_bf16x2(hv[8 * c], hv[8 * c + 1]),
                                    pack_bf16x2(hv[8 * c + 2], hv[8 * c + 3]),
                                    pack_bf16x2(hv[8 * c + 4], hv[8 * c + 5]),
                                    pack_bf16x2(hv[8 * c + 6], hv[8 * c + 7]));
+                    if (halves) {
+                        float m[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            m[e] = fmaf(dmid, hv[8 * c + e], __uint_as_float(lo[8 * c + e]));
+                        *reinterpret_cast<uint4 *>(mrow + 8 * (piece ^ (n & 7))) =
+                            make_uint4(pack_bf16x2(m[0], m[1]), pack_bf16x2(m[2], m[3]),
+                                       pack_bf16x2(m[4], m[5]), pack_bf16x2(m[6], m[7]));
+                    }
+                }
+                float sf[16];   // the chunk's own state S, these 16 columns
+#pragma unroll
+                for (int p = 0; p < 16; ++p)
+                    sf[p] = halves ? fmaf(dhl, __uint_as_float(lo[p]), __uint_as_float(hi[p]))
+                                   : __uint_as_float(lo[p]);
+                // h_in[k+1] = exp(cs_last) h_in[k] + S: the ring slot the next chunk reads, or
+                // the final state after the last chunk
+                if (k + 1 < nchunks) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        __stcg(reinterpret_cast<float4 *>(ring_out) + 4 * qq + c,
+                               make_float4(fmaf(dec, hv[4 * c], sf[4 * c]),
+                                           fmaf(dec, hv[4 * c + 1], sf[4 * c + 1]),
+                                           fmaf(dec, hv[4 * c + 2], sf[4 * c + 2]),
+                                           fmaf(dec, hv[4 * c + 3], sf[4 * c + 3])));
+                } else if (chain.final_state) {
+                    float *fo = chain.final_state + bh * (int64_t)(kP * kN) + n;
+#pragma unroll
+                    for (int p = 0; p < 16; ++p)
+                        fo[(16 * qq + p) * kN] = fmaf(dec, hv[p], sf[p]);
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&sm.bar_acc_free[a]);
             // every thread's part of h_in[k+1] is visible GPU-wide before the flag
             if (k + 1 < nchunks) __threadfence();
             mbar_arrive(&sm.bar_pub);
@@ -500,7 +549,12 @@ __device__ __forceinline__ void scale_pieces(uint8_t *base, int first, int strid
     }
 }
 
-template <bool kGate>   // kGate: the output is y * z * sigmoid(z)
+// kGate: the output is y * z * sigmoid(z).
+// kSub: the state entering each 128-row tile is given (hin holds one block per tile: the
+// state entering the chunk, and for Q = 256 the state at its row 127), so the second tile of a
+// chunk is computed exactly like the first -- its diagonal block plus C h^T from its own
+// entering state -- with no off-diagonal block.
+template <bool kGate, bool kSub>
 __global__ void __launch_bounds__(kScanThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_b,
@@ -531,11 +585,16 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     int len;
     chunk_span(tab, k, Q, seqlen, t0, len);
     if (T * kTileRows >= len) return;  // tile past the end of the sequence, or unused slot
-    const int KI = kTileRows * (T + 1);  // causal source columns of this tile
-    const int nst = T ? 2 : 3;           // x / h_in stages
-    const uint32_t gdiag = T ? 128u : 0u;  // TMEM column of the diagonal block of C B^T
-    const uint32_t pcol = T ? 0u : 128u;   // TMEM columns of the P ring (T = 1: over C B_off^T)
-    const int xdiag = kTileRows * T;       // first x row of the diagonal block
+    const bool offd = T && !kSub;        // the tile has an off-diagonal block
+    const int KI = offd ? 2 * kTileRows : kTileRows;  // source columns (x rows) of the tile
+    const int xrow = kSub ? kTileRows * T : 0;        // first sequence row of those, in the chunk
+    const int nst = offd ? 2 : 3;        // x / h_in stages
+    const uint32_t gdiag = offd ? 128u : 0u;  // TMEM column of the diagonal block of C B^T
+    const uint32_t pcol = offd ? 0u : 128u;   // TMEM columns of the P ring (over C B_off^T)
+    const int xdiag = offd ? kTileRows : 0;   // first x row of the diagonal block in the stage
+    // this tile's entering-state block: one per chunk, or one per 128-row tile (kSub)
+    const bf16 *hblk = hin + (kSub ? (b * nchunks + k) * nT + T : b * nchunks + k) * (int64_t)H *
+                                 (kP * kN);
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_cb, 1);
@@ -586,13 +645,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 tma_load_4d(&sm.Cs[a][0], &tm_c, &sm.bar_cb, 64 * a, g,
                             (int)(t0 + kTileRows * T), (int)b);
             for (int a = 0; a < 2; ++a)
-                for (int r = 0; r <= T; ++r)
+                for (int r = 0; r < KI / kTileRows; ++r)
                     tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
-                                64 * a, g, (int)(t0 + kTileRows * r), (int)b);
+                                64 * a, g, (int)(t0 + xrow + kTileRows * r), (int)b);
             // x is an input of the scan: start streaming the first heads' tiles into L2 while
             // the state-passing kernel finishes
             for (int j = 0; j < nh && j < nst; ++j)
-                tma_prefetch_l2_4d(T ? &tm_x2 : &tm_x, 0, h0 + j, (int)t0, (int)b);
+                tma_prefetch_l2_4d(offd ? &tm_x2 : &tm_x, 0, h0 + j, (int)(t0 + xrow), (int)b);
             griddep_wait();   // cs / dt and the entering states come from earlier kernels
         }
         for (int j = 0; lane == 0 && j < nh; ++j) {   // lane 0 alone runs the loop
@@ -616,14 +675,14 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                                   (uint32_t)(KI * kRowBytes + 2 * kP * kRowBytes));
             // x rows [0, KI) of the chunk as one box (fewer, larger TMA boxes stream faster);
             // h_in is stored in its shared-memory layout, so one contiguous copy suffices
-            tma_load_4d(stg, T ? &tm_x2 : &tm_x, &sm.bar_xh_full[xs], 0, h, (int)t0, (int)b);
-            bulk_load(stg + kHOff, hin + ((b * nchunks + k) * H + h) * (int64_t)(kP * kN),
-                      kP * kN * 2, &sm.bar_xh_full[xs]);
+            tma_load_4d(stg, offd ? &tm_x2 : &tm_x, &sm.bar_xh_full[xs], 0, h,
+                        (int)(t0 + xrow), (int)b);
+            bulk_load(stg + kHOff, hblk + (int64_t)h * (kP * kN), kP * kN * 2,
+                      &sm.bar_xh_full[xs]);
             // the operands this stage will hold next: into L2 now, so their loads are L2 hits
             if (j + nst < nh) {
-                tma_prefetch_l2_4d(T ? &tm_x2 : &tm_x, 0, h + nst, (int)t0, (int)b);
-                bulk_prefetch_l2(hin + ((b * nchunks + k) * H + h + nst) * (int64_t)(kP * kN),
-                                 kP * kN * 2);
+                tma_prefetch_l2_4d(offd ? &tm_x2 : &tm_x, 0, h + nst, (int)(t0 + xrow), (int)b);
+                bulk_prefetch_l2(hblk + (int64_t)(h + nst) * (kP * kN), kP * kN * 2);
             }
             // the gate rows this tile's epilogue will read: into L2 now, a few heads ahead
             if (kGate) tma_prefetch_l2_4d(&tm_z, 0, h, (int)(t0 + kTileRows * T), (int)b);
@@ -649,20 +708,20 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             }
             mma_commit(&sm.bar_g);
         }
-        if (ok && T) ok = mbar_wait(&sm.bar_goff, 0, abort);   // bf16 C B_off^T in smem
+        if (ok && offd) ok = mbar_wait(&sm.bar_goff, 0, abort);   // bf16 C B_off^T in smem
         for (int j = 0; ok && j < nh; ++j) {
             const int xs = j % nst;
             const uint32_t xu = j / nst;
             const int a = j & 1;
             if (!mbar_wait(&sm.bar_xh_full[xs], xu & 1, abort)) break;
-            if (T && !mbar_wait(&sm.bar_xv_ready[xs], xu & 1, abort)) break;
+            if (offd && !mbar_wait(&sm.bar_xv_ready[xs], xu & 1, abort)) break;
             if (j >= 2 && !mbar_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
             tc_fence_after();
             const uint32_t stg = smem_u32(scan_stage(sm, xs));
             const uint32_t dD = tmem + kAccCol + 128 * a, dA = dD + 64;
             const uint64_t xd = smem_desc_sw128(stg, 256 * kRowBytes, 1024);   // x, MN-major
             const uint64_t hd = smem_desc_sw128(stg + kHOff, 16384, 1024);     // h_in, MN-major
-            if (T) {
+            if (offd) {
                 // Y_A = (C B_off^T) (v dt o X_off): A = bf16 block in R, K = 128 (i)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -675,7 +734,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
 #pragma unroll
             for (int kk = 0; kk < kN / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                mma_bf16(dA, cd + (off >> 4), hd + kk * 128, id_kmn, (T || kk > 0) ? 1u : 0u);
+                mma_bf16(dA, cd + (off >> 4), hd + kk * 128, id_kmn, (offd || kk > 0) ? 1u : 0u);
             }
             for (int qb = 0; qb < 2; ++qb) {
                 const uint32_t blk = 2 * j + qb;           // P blocks are numbered per head
@@ -725,7 +784,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             if (cls1 < 2) tmem_ld16(lane_base + gdiag + 16 * u1, g1);
             tmem_ld_wait();
         }
-        if (ok && T) {
+        if (ok && offd) {
             // C B_off^T (TMEM columns [0, 128)) -> bf16, K-major swizzled tile in R; this warp
             // converts its 32 rows x columns [32 cq, 32 cq + 32)
             uint32_t gv[32];
@@ -755,7 +814,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 if (!warp_wait(&sm.bar_vec_full[vs], (j / kScanVecStages) & 1, abort)) break;
                 const float *cs_s = sm.cs_v[vs];
                 const float *dt_s = sm.dt_v[vs];
-                if (T) {
+                if (offd) {
                     // x rows [0, 128) *= exp(cs_127 - cs_i) dt_i; h_in *= exp(cs_127)
                     const int xs = j % nst;
                     if (!warp_wait(&sm.bar_xh_full[xs], (j / nst) & 1, abort)) break;
@@ -1041,7 +1100,7 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
                                  int Q, int64_t nchunks, cudaStream_t st, const char **why,
-                                 const int2 *tab, const bf16 *z)
+                                 const int2 *tab, const bf16 *z, bool sub)
 {
     CUtensorMap mx, mx2, mb, mc, mz;
     if (z) {
@@ -1065,7 +1124,8 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     const int hpc = scan_heads_per_cta(batch * nchunks * G * (Q / kTileRows), hpg);
     const int nhb = (hpg + hpc - 1) / hpc;
     const size_t smem = sizeof(ScanSmem) + 1024;
-    auto kern = z ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
+    auto kern = z ? (sub ? chunk_scan_tc_kernel<true, true> : chunk_scan_tc_kernel<true, false>)
+                  : (sub ? chunk_scan_tc_kernel<false, true> : chunk_scan_tc_kernel<false, false>);
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk scan: set smem attribute"; return e; }

@@ -75,7 +75,8 @@ struct WsLayout {
     size_t states;      // float [b][c][H][P][N] (CUDA-core path) or [b][c][H][N][P] (tensor-core
                         // path): per-chunk state, then (in place) state entering
     size_t hin_bf16;    // bf16  [b][c][H] blocks of P x N (hin_swizzled_offset): state entering
-                        // each chunk (tensor-core path)
+                        // each chunk (tensor-core path); [b][c][Q / 128][H] blocks, the state
+                        // entering each 128-row tile, when the chained chunk state runs
     size_t sync;        // int [kSyncFlags + b * H]: the chained chunk state's ticket counter (at
                         // 0) and per-(batch, head) flags (from kSyncFlags) (tensor-core path)
     size_t total;
@@ -188,8 +189,10 @@ bool tc_supported(bool is_bf16, int P, int N, int Q);
 // The chained form of the chunk-state kernel (fixed-length input only): it also carries the
 // state across chunks, so no float32 chunk states go to HBM and no state-passing kernel runs.
 // ring: batch * H * 2 * P * N floats; flags: batch * H ints and counter: one int, all zero at
-// the launch (the cumsum kernel clears them).  hin receives the bf16 entering states,
-// final_state (nullable) the float32 state after the last chunk, from init (nullable).
+// the launch (the cumsum kernel clears them).  hin receives the bf16 state entering every
+// 128-row tile (Q / 128 blocks per chunk: the chunk's entering state, and for Q = 256 the state
+// at its row 127), final_state (nullable) the float32 state after the last chunk, from init
+// (nullable).
 struct StateChain {
     float *ring;
     int *flags;
@@ -270,10 +273,13 @@ cudaError_t launch_group_sum(const float *in, const float *w, float *out, int64_
 cudaError_t launch_scale_init_grad(const float *F, const float *dt, const float *A, float *out,
                                    int64_t batch, int64_t L, int H, int PN, cudaStream_t st);
 
+// sub: hin holds the entering state of every 128-row tile (Q / 128 blocks per chunk, as the
+// chained chunk-state kernel writes them), otherwise one block per chunk.
 cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
                                  int Q, int64_t nchunks, cudaStream_t st, const char **why,
-                                 const int2 *tab = nullptr, const bf16 *z = nullptr);
+                                 const int2 *tab = nullptr, const bf16 *z = nullptr,
+                                 bool sub = false);
 
 }  // namespace ssd

@@ -82,7 +82,10 @@ ssd::WsLayout layout(const ssd_shape *s, int Q)
     w.dtc = w.cs + round256(rows * Q * sizeof(float));
     w.states = w.dtc + (tc ? round256(rows * Q * sizeof(float)) : 0);
     w.hin_bf16 = w.states + round256(rows * s->headdim * s->dstate * sizeof(float));
-    w.sync = w.hin_bf16 + (tc ? round256(rows * s->headdim * s->dstate * sizeof(uint16_t)) : 0);
+    // the chained form keeps one entering state per 128-row tile (Q / 128 per chunk)
+    const size_t nsub = Q > 128 ? (size_t)(Q / 128) : 1;
+    w.sync = w.hin_bf16 +
+             (tc ? round256(nsub * rows * s->headdim * s->dstate * sizeof(uint16_t)) : 0);
     w.total = w.sync + (tc ? round256((ssd::kSyncFlags + (size_t)s->batch * s->nheads) * 4) : 0);
     return w;
 }
@@ -327,7 +330,7 @@ ssd_status scan_impl(const ssd_shape *shape, const void *x, const float *dt, con
         e = ssd::launch_chunk_scan_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B,
                                       (const ssd::bf16 *)C, cs, hin, D, (ssd::bf16 *)y, status,
                                       s.batch, s.seqlen, H, G, Q, nchunks, cs_stream, &why,
-                                      nullptr, (const ssd::bf16 *)z);
+                                      nullptr, (const ssd::bf16 *)z, chain);
         if (e != cudaSuccess) return cuda_fail(e, why);
         if ((e = record(stage_events, 4, cs_stream)) != cudaSuccess)
             return cuda_fail(e, "record stage event");

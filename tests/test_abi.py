@@ -63,10 +63,11 @@ def test_workspace_size_layout():
     c = L_ // Q
     ws = ssd.workspace_size(_shape(), Q)
     # status word + cs (f32) + per-chunk dt rows (f32) + chunk states (f32) + bf16 entering
-    # states + the chained chunk state's counter and per-(batch, head) flags, 256-byte rounded
-    # (the dt rows, bf16 states and flags only on the tensor-core path)
+    # states of every 128-row tile + the chained chunk state's counter and per-(batch, head)
+    # flags, 256-byte rounded (the dt rows, bf16 states and flags only on the tensor-core path)
     sync = -(-(64 + b * H) * 4 // 256) * 256
-    expect = 256 + 2 * b * c * H * Q * 4 + b * c * H * P * N * 4 + b * c * H * P * N * 2 + sync
+    expect = (256 + 2 * b * c * H * Q * 4 + b * c * H * P * N * 4 + (Q // 128) * b * c * H * P * N * 2
+              + sync)
     assert ws == expect
     # float32 inputs run the CUDA-core path, which keeps the entering state in place (no bf16 copy)
     ws32 = ssd.workspace_size(_shape(dtype=ssd.SSD_F32), Q)

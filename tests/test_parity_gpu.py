@@ -131,18 +131,21 @@ def test_small_parity_with_initial_state(cuda_device, state_form, form, name, w,
 @pytest.mark.parametrize("w", [configs.SSD_2P7B.with_(init_state=True),
                                configs.SSD_LONG.with_(seqlen=16384)],
                          ids=["ssd_2p7b_init", "long_g8_64_chunks"])
-def test_state_forms_are_bit_identical(cuda_device, state_form, w):
-    """Both forms run the same arithmetic (the same MMAs for the chunk states, the same
-    fused multiply-add and rounding for the carry), so y and the final state agree bit for bit."""
+def test_state_forms_full_size_every_output(cuda_device, state_form, w):
+    """Both forms at full size, every slice against the oracle.  They round differently (the
+    chained form decays the two 128-row halves of a chunk to their own last rows and hands the
+    second half its own bf16 entering state), so they agree with each other only to the bound."""
     import torch
     inp = inputs.make_inputs(w)
     t = torch_inputs(inp, cuda_device)
     outs = []
     for form in (1, 2):
         state_form(form)
-        outs.append(run_fwd(torch, t, w, w.chunk, cuda_device, guards=False))
-    assert torch.equal(outs[0][0], outs[1][0]), "y differs between the two forms"
-    assert torch.equal(outs[0][1], outs[1][1]), "final state differs between the two forms"
+        y, f = run_fwd(torch, t, w, w.chunk, cuda_device, guards=False)
+        check_against_oracle(inp, y, f, rows_per_block=1)
+        outs.append((y, f))
+    ey = max_rel_slices(to_np(outs[0][0]), to_np(outs[1][0]), (1, 3))[0]
+    assert ey <= TOL["bf16"], f"the two forms differ by {ey:.3e}"
 
 
 # ------------------------------------------------------------------ full-size workloads
