@@ -479,21 +479,23 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
 //   - the off-chunk term exp(cs_t) C h_in^T = u_t C (exp(cs_127) h_in)^T, which (scaled h_in)
 //     accumulates into the same TMEM accumulator as the off-diagonal block.
 // So y = Y_diag + f_t Y_A with f_t = exp(cs_t) (T = 0) or u_t (T = 1).
-constexpr int kXStagesMax = 3;   // x / h_in stages (T = 0: 3, the third in the B tile's space;
-                                 // T = 1: 2, that space holds the bf16 off-diagonal block)
+constexpr int kXStagesMax = 5;   // x / h_in stages: tiles without an off-diagonal block use 5
+                                 // of 32 KB (three in S01, two in the B tile's space once C B^T
+                                 // is done); the second tile of a chunk with one uses 2 of 48 KB
+                                 // (S01; the B tile's space then holds the bf16 block)
 constexpr int kScanHeadsMin = 8;  // heads per CTA: chosen per launch in [8, 20] (fewer when a
 constexpr int kScanHeadsMax = 20; // group has fewer), see scan_heads_per_cta
-constexpr int kScanVecStages = 4; // cs / dt row stages (one head each)
+constexpr int kScanVecStages = 6; // cs / dt row stages (one head each)
 static_assert(kScanHeadsMax <= kMaxHeadsPerCta, "D of every head of a CTA is staged in smem");
 constexpr int kRing = 4;         // 64-column blocks of P in TMEM (two heads)
-constexpr int kStageBytes = 256 * kRowBytes + 2 * kP * kRowBytes;  // x (<= 256 rows) + h_in
-constexpr int kHOff = 256 * kRowBytes;                              // h_in inside a stage
+constexpr int kStageBytes = 256 * kRowBytes + 2 * kP * kRowBytes;  // 48 KB: 256 x rows + h_in
+constexpr int kStage32 = 128 * kRowBytes + 2 * kP * kRowBytes;     // 32 KB: 128 x rows + h_in
 struct alignas(1024) ScanSmem {
     bf16 Cs[2][kTileRows * 64];     // K-major A (C tile): [n atom][128 rows t][64 n]
     uint8_t R[kStageBytes + 16384]; // B rows for C B^T (K-major [n atom][KI rows][64]); after
                                     // that, T = 0: x / h_in stage 2; T = 1: bf16 C B_off^T
                                     // (K-major [i atom][128 rows t][64 i])
-    uint8_t S01[2][kStageBytes];    // x / h_in stages 0 and 1: [KI rows i][64 p] then
+    uint8_t S01[2 * kStageBytes];   // x / h_in stages: [KI rows i][64 p] then h_in
                                     // [128 rows n][64 p]
     float cs_v[kScanVecStages][256];  // per stage: one head's chunk-local cumsum row
     float dt_v[kScanVecStages][256];  // per stage: its dt row (0 past the end)
@@ -519,10 +521,14 @@ constexpr uint32_t kAccCol = 256;   // accumulator buffer a: Y_diag at 256 + 128
 static_assert(sizeof(StateSmem) + 1024 <= 232448, "chunk state smem exceeds 227 KB");
 static_assert(sizeof(ScanSmem) + 1024 <= 232448, "chunk scan smem exceeds 227 KB");
 
-__device__ __forceinline__ uint8_t *scan_stage(ScanSmem &sm, int s)
+// Stage s: with an off-diagonal block (48 KB stages) s in {0, 1} in S01; otherwise (32 KB
+// stages) s in 0..2 in S01 and 3..4 in the B tile's space.  h_in follows the x rows.
+__device__ __forceinline__ uint8_t *scan_stage(ScanSmem &sm, int s, bool offd)
 {
-    return s < 2 ? sm.S01[s] : sm.R;
+    if (offd) return sm.S01 + s * kStageBytes;
+    return s < 3 ? sm.S01 + s * kStage32 : sm.R + (s - 3) * kStage32;
 }
+__device__ __forceinline__ int scan_hoff(bool offd) { return (offd ? 256 : 128) * kRowBytes; }
 
 // Scale the 16-byte pieces [first, first + count * stride) of a bf16 smem tile in place; the
 // factor of piece c is f(c).  Works on any swizzled layout whose rows are whole 128-byte lines.
@@ -588,7 +594,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const bool offd = T && !kSub;        // the tile has an off-diagonal block
     const int KI = offd ? 2 * kTileRows : kTileRows;  // source columns (x rows) of the tile
     const int xrow = kSub ? kTileRows * T : 0;        // first sequence row of those, in the chunk
-    const int nst = offd ? 2 : 3;        // x / h_in stages
+    const int nst = offd ? 2 : kXStagesMax;   // x / h_in stages
     const uint32_t gdiag = offd ? 128u : 0u;  // TMEM column of the diagonal block of C B^T
     const uint32_t pcol = offd ? 0u : 128u;   // TMEM columns of the P ring (over C B_off^T)
     const int xdiag = offd ? kTileRows : 0;   // first x row of the diagonal block in the stage
@@ -667,17 +673,18 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             const int xs = j % nst;
             const uint32_t xu = j / nst;
             if (j >= nst && !mbar_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) break;
-            if (xs == 2 && xu == 0 && !mbar_wait(&sm.bar_g, 0, abort)) break;  // B tile in use
+            if (!offd && xs >= 3 && xu == 0 && !mbar_wait(&sm.bar_g, 0, abort))
+                break;   // the B tile's space is in use until C B^T is done
             // failure injection (tests only): this stage is left unissued
             if (j == 0 && (int)blockIdx.x == skip_cta) continue;
-            uint8_t *stg = scan_stage(sm, xs);
+            uint8_t *stg = scan_stage(sm, xs, offd);
             mbar_arrive_expect_tx(&sm.bar_xh_full[xs],
                                   (uint32_t)(KI * kRowBytes + 2 * kP * kRowBytes));
             // x rows [0, KI) of the chunk as one box (fewer, larger TMA boxes stream faster);
             // h_in is stored in its shared-memory layout, so one contiguous copy suffices
             tma_load_4d(stg, offd ? &tm_x2 : &tm_x, &sm.bar_xh_full[xs], 0, h,
                         (int)(t0 + xrow), (int)b);
-            bulk_load(stg + kHOff, hblk + (int64_t)h * (kP * kN), kP * kN * 2,
+            bulk_load(stg + scan_hoff(offd), hblk + (int64_t)h * (kP * kN), kP * kN * 2,
                       &sm.bar_xh_full[xs]);
             // the operands this stage will hold next: into L2 now, so their loads are L2 hits
             if (j + nst < nh) {
@@ -717,10 +724,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             if (offd && !mbar_wait(&sm.bar_xv_ready[xs], xu & 1, abort)) break;
             if (j >= 2 && !mbar_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
             tc_fence_after();
-            const uint32_t stg = smem_u32(scan_stage(sm, xs));
+            const uint32_t stg = smem_u32(scan_stage(sm, xs, offd));
             const uint32_t dD = tmem + kAccCol + 128 * a, dA = dD + 64;
             const uint64_t xd = smem_desc_sw128(stg, 256 * kRowBytes, 1024);   // x, MN-major
-            const uint64_t hd = smem_desc_sw128(stg + kHOff, 16384, 1024);     // h_in, MN-major
+            const uint64_t hd = smem_desc_sw128(stg + scan_hoff(offd), 16384, 1024);  // h_in
             if (offd) {
                 // Y_A = (C B_off^T) (v dt o X_off): A = bf16 block in R, K = 128 (i)
 #pragma unroll
@@ -818,14 +825,14 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     // x rows [0, 128) *= exp(cs_127 - cs_i) dt_i; h_in *= exp(cs_127)
                     const int xs = j % nst;
                     if (!warp_wait(&sm.bar_xh_full[xs], (j / nst) & 1, abort)) break;
-                    uint8_t *stg = scan_stage(sm, xs);
+                    uint8_t *stg = scan_stage(sm, xs, offd);
                     const float c127 = cs_s[127];
                     scale_pieces<1024 / kScanWorkers>(stg, wt, kScanWorkers, [&](int c) {
                         const int i = c >> 3;
                         return __expf(c127 - cs_s[i]) * dt_s[i];
                     });
                     const float sh = __expf(c127);
-                    scale_pieces<1024 / kScanWorkers>(stg + kHOff, wt, kScanWorkers,
+                    scale_pieces<1024 / kScanWorkers>(stg + scan_hoff(offd), wt, kScanWorkers,
                                                       [&](int) { return sh; });
                     fence_async_smem();
                     mbar_arrive(&sm.bar_xv_ready[xs]);
