@@ -1,8 +1,7 @@
 /*
- * ssd_testing.h -- test controls: failure injection for the tests of the library's bounded
- * in-kernel waits, and the choice between the two equivalent ways of carrying the state across
- * chunks.  Not needed to use the library.  (No counterpart on the pages: this is how the
- * library's own failure handling and alternative kernel paths are exercised.)
+ * ssd_testing.h -- failure injection for the tests of the library's bounded in-kernel waits.
+ * Not needed to use the library.  (No counterpart on the pages: this is how the library's own
+ * failure handling is exercised.)
  *
  * Every wait of the tensor-core kernels on one of their shared-memory barriers is bounded: after
  * about 2 s the waiting thread records a timeout, the CTA lets its own in-flight tensor-core
@@ -33,16 +32,6 @@ enum { SSD_TESTING_CHUNK_STATE = 1, SSD_TESTING_CHUNK_SCAN = 2 };
  * affected call's outputs are incomplete; a later call on the same workspace starts clean.
  */
 ssd_status ssd_testing_skip_stage(int kernel, int cta);
-
-/*
- * Selects how the tensor-core path of ssd_chunk_scan_fwd carries the state across chunks, for
- * every later call of this process: 0 = automatic (the default: the chained chunk-state kernel
- * for sequences of at most 32 chunks, otherwise the chunk-state kernel followed by the
- * state-passing kernel), 1 = always the two kernels, 2 = always the chained kernel.  Both forms
- * compute the same result; the setting exists so that the tests can check each form at any
- * shape.  Returns SSD_ERR_INVALID_ARG for any other value.
- */
-ssd_status ssd_testing_state_form(int form);
 
 #ifdef __cplusplus
 }

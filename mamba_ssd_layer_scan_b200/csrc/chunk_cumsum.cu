@@ -25,16 +25,12 @@ __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(const float *__restrict__ dt, const float *__restrict__ A,
                     float *__restrict__ cs, float *__restrict__ dtc, int *__restrict__ status,
                     int64_t seqlen, int H, int Q, int64_t nchunks, const int2 *__restrict__ tab,
-                    bool unit_weights, int *__restrict__ sync, int64_t nsync)
+                    bool unit_weights)
 {
     griddep_wait();               // nothing of an earlier kernel is touched before this
     griddep_launch_dependents();
-    // First kernel of every scan: clears the workspace status word the later kernels may set,
-    // and the chained chunk state's counter and flags.
+    // First kernel of every scan: clears the workspace status word the later kernels may set.
     if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
-    for (int64_t i = blockIdx.x * (int64_t)kThreads + threadIdx.x; i < nsync;
-         i += (int64_t)gridDim.x * kThreads)
-        sync[i] = 0;
     extern __shared__ float tile[];  // [Q][kHeadTile + 1]
     const int nht = (H + kHeadTile - 1) / kHeadTile;
     const int h0 = (int)(blockIdx.x % nht) * kHeadTile;
@@ -101,12 +97,12 @@ __global__ void fill_final_kernel(const float *__restrict__ init, float *__restr
 cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, float *dtc,
                                 int *status, int64_t batch, int64_t seqlen, int nheads, int Q,
                                 int64_t nchunks, cudaStream_t st, const int2 *tab,
-                                bool unit_weights, int *sync, int64_t nsync)
+                                bool unit_weights)
 {
     const unsigned grid = (unsigned)(((nheads + kHeadTile - 1) / kHeadTile) * nchunks * batch);
     const size_t smem = (size_t)Q * (kHeadTile + 1) * sizeof(float);
     return launch_pdl(chunk_cumsum_kernel, grid, kThreads, smem, st, dt, A, cs, dtc, status,
-                      seqlen, nheads, Q, nchunks, tab, unit_weights, sync, nsync);
+                      seqlen, nheads, Q, nchunks, tab, unit_weights);
 }
 
 cudaError_t launch_fill_final(const float *init, float *final_state, int64_t n,

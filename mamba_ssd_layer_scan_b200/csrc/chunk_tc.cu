@@ -65,59 +65,25 @@ struct alignas(1024) StateSmem {
     bf16 Xs[kStateStages][256 * 64];      // MN-major B operand per stage: [Q rows tau][64 p]
     float cs_v[kStateStages][256];        // per stage: the head's chunk-local cumsum row
     float dt_v[kStateStages][256];        // per stage: the head's dt row (0 past the end)
-    float cs_last[kMaxHeadsPerCta];       // chained form: each head's chunk log-decay
-    float cs_mid[kMaxHeadsPerCta];        // chained form, Q = 256: its log-decay to row 127
     uint64_t bar_b;
     uint64_t bar_x_full[kStateStages], bar_x_ready[kStateStages], bar_x_free[kStateStages];
     uint64_t bar_acc_full[2], bar_acc_free[2];
-    uint64_t bar_flag_ok, bar_pub;        // chained form: predecessor's state seen / ours stored
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort;
-    int ticket;
-    int published;                        // chained form: heads whose outgoing state is out
 };
 // warp 0 TMA, warps 1 and 3 MMA (alternate heads), warp 2 TMEM owner, warps 4-11 scale x,
 // warps 12-15 epilogue
 constexpr int kStateThreads = 512;
 constexpr int kStateScaleThreads = 256;
-constexpr uint32_t kStateTmemCols = 256;   // two buffers of (rows 0-127, rows 128-255) x 64 p
-constexpr int kChainAbort = 0x40000000;   // flag value: the chain was broken by a timeout
+constexpr uint32_t kStateTmemCols = 128;   // two accumulator buffers of 64 p
 
-// The chained form of the chunk-state kernel carries the recurrence across chunks itself
-// (mohakchugh.is-a.dev "Mamba-2", Block Decomposition: across blocks the state is propagated
-// sequentially), so the float32 chunk states never go to HBM:
-//
-//     h_in[k+1] = exp(cs_k[Q-1]) h_in[k] + S_k          per (batch, head), chunk after chunk
-//
-// Work items (chunk, batch, group, head block) are handed out in chunk-major order by a ticket
-// counter, so an item only ever waits for an item with a smaller ticket, whose CTA has already
-// started: no wait can depend on a CTA that is not resident.  For each head the epilogue takes
-// S_k from TMEM, waits (bounded) until the item of chunk k-1 has published h_in[k] for that
-// head, writes h_in[k] as the chunk scan's bf16 operand, and publishes h_in[k+1] (float32, in a
-// two-slot ring per (batch, head) that stays in L2; the final state instead for the last chunk).
-// The ring is safe with two slots: the item of chunk k+1 overwrites slot k & 1 only after it has
-// read slot (k+1) & 1, which the item of chunk k wrote after it had read slot k & 1.
-__device__ __forceinline__ int ld_acquire_gpu(const int *p)
-{
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_gpu(int *p, int v)
-{
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-template <bool kChain>
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                       const __grid_constant__ CUtensorMap tm_b, const float *__restrict__ dtc,
                       const float *__restrict__ cs, float *__restrict__ states,
                       int *__restrict__ status, int H, int G, int Q, int64_t nchunks, int nhb,
-                      int hpc, int64_t seqlen, const int2 *__restrict__ tab, int skip_cta,
-                      StateChain chain)
+                      int hpc, int64_t seqlen, const int2 *__restrict__ tab, int skip_cta)
 {
     extern __shared__ uint8_t smem_raw[];
     StateSmem &sm = *reinterpret_cast<StateSmem *>(
@@ -125,23 +91,9 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     int64_t u = blockIdx.x;
-    if (kChain) {
-        // the ticket counter is cleared by the cumsum kernel: wait for it first
-        griddep_wait();
-        if (threadIdx.x == 0) sm.ticket = atomicAdd(chain.counter, 1);
-        __syncthreads();
-        u = sm.ticket;   // chunk-major: u = ((k * batch + b) * G + g) * nhb + hb
-    }
     const int hb = (int)(u % nhb); u /= nhb;
     const int g = (int)(u % G); u /= G;
-    int64_t k, b;
-    if (kChain) {
-        b = u % chain.batch;
-        k = u / chain.batch;
-    } else {
-        k = u % nchunks;
-        b = u / nchunks;
-    }
+    const int64_t k = u % nchunks, b = u / nchunks;
     const int hpg = H / G;
     const int h0 = g * hpg + hb * hpc;
     const int nh = min(hpc, hpg - hb * hpc);
@@ -161,11 +113,8 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_init(&sm.bar_acc_full[s], 1);
             mbar_init(&sm.bar_acc_free[s], 128);
         }
-        mbar_init(&sm.bar_flag_ok, 1);
-        mbar_init(&sm.bar_pub, 128);
         mbar_init(&sm.bar_drain, 2);
         sm.abort = 0;
-        sm.published = 0;
         fence_mbar_init();
     }
     if (warp == 2) {
@@ -226,21 +175,12 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 if (!mbar_wait(&sm.bar_x_ready[s], use & 1, abort)) break;
                 if (j >= 2 && !mbar_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
                 tc_fence_after();
-                const uint32_t d = tmem + a * 128;
+                const uint32_t d = tmem + a * kP;
                 // base descriptors + constant K steps (16 rows = 2048 bytes) in fully unrolled
                 // loops: the issuing thread's own instruction chain sets the MMA issue rate
                 const uint64_t ad = smem_desc_sw128(smem_u32(&sm.Bs[0][0]), atom_bytes, 1024);
                 const uint64_t bd = smem_desc_sw128(smem_u32(&sm.Xs[s][0]), atom_bytes, 1024);
-                if (Q == 256 && kChain) {
-                    // chained form: rows 0-127 and rows 128-255 into separate accumulators (the
-                    // state at row 127 is the second half-chunk's entering state)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(d, ad + kk * 128, bd + kk * 128, idesc, kk > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int kk = 8; kk < 16; ++kk)
-                        mma_bf16(d + 64, ad + kk * 128, bd + kk * 128, idesc, kk > 8 ? 1u : 0u);
-                } else if (Q == 256) {
+                if (Q == 256) {
 #pragma unroll
                     for (int kk = 0; kk < 16; ++kk)
                         mma_bf16(d, ad + kk * 128, bd + kk * 128, idesc, kk > 0 ? 1u : 0u);
@@ -262,18 +202,9 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             const uint32_t use = j / kStateStages;
             if (!warp_wait(&sm.bar_x_full[s], use & 1, abort)) break;
             const float cs_last = sm.cs_v[s][Q - 1];
-            // chained form, Q = 256: rows 0-127 are decayed to row 127 (their own accumulator),
-            // rows 128-255 to the chunk's last row; otherwise every row to the last row
-            const bool halves = kChain && Q == 256;
-            const float cs_ref0 = halves ? sm.cs_v[s][127] : cs_last;
-            if (kChain && st == 0) {   // for the epilogue's carry
-                sm.cs_last[j] = cs_last;
-                sm.cs_mid[j] = cs_ref0;
-            }
             for (int c = st; c < chunks; c += kStateScaleThreads) {
                 const int tau = c >> 3;
-                const float ref = tau < 128 ? cs_ref0 : cs_last;
-                const float w = __expf(ref - sm.cs_v[s][tau]) * sm.dt_v[s][tau];
+                const float w = __expf(cs_last - sm.cs_v[s][tau]) * sm.dt_v[s][tau];
                 uint4 *ptr = reinterpret_cast<uint4 *>(&sm.Xs[s][0]) + c;
                 uint4 v = *ptr;
                 uint32_t *wv = &v.x;
@@ -293,151 +224,30 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         // ---------------- epilogue: TMEM (lane n, column p) -> S^T row n
         const int q = warp & 3;
         const int n = q * 32 + lane;
-        const int et = threadIdx.x - 384;   // 0..127 within the epilogue warps
         for (int j = 0; j < nh; ++j) {
             const int a = j & 1;
             if (!warp_wait(&sm.bar_acc_full[a], (j >> 1) & 1, abort)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + a * 128;
-            if (!kChain) {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(taddr, r0);
-                tmem_ld32(taddr + 32, r1);
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(&sm.bar_acc_free[a]);
-                // the chunk states are kept as [n][p]: 64 consecutive p per thread
-                float4 *out = reinterpret_cast<float4 *>(
-                    states + (((b * nchunks + k) * H + h0 + j) * (int64_t)kN + n) * kP);
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    __stcs(out + c,
-                           make_float4(__uint_as_float(r0[4 * c]), __uint_as_float(r0[4 * c + 1]),
-                                       __uint_as_float(r0[4 * c + 2]),
-                                       __uint_as_float(r0[4 * c + 3])));
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    __stcs(out + 8 + c,
-                           make_float4(__uint_as_float(r1[4 * c]), __uint_as_float(r1[4 * c + 1]),
-                                       __uint_as_float(r1[4 * c + 2]),
-                                       __uint_as_float(r1[4 * c + 3])));
-                continue;
-            }
-            // ---- chained: the entering state h_in[k] of head h, then h_in[k+1].  Every
-            // hand-off between the four epilogue warps goes through an mbarrier with a bounded
-            // wait, so a timeout anywhere lets every thread leave the loop.
-            // Per head, thread 0 of the epilogue first completes bar_flag_ok (after seeing the
-            // previous chunk's state, for k > 0), and it completes it for head j + 1 only after
-            // bar_pub of head j, where all 128 threads have arrived: so no thread's wait or
-            // arrival on either barrier can fall a phase behind.
-            const int64_t bh = b * H + h0 + j;
-            int *flag = chain.flags + bh;
-            if (et == 0) {
-                if (k > 0) {
-                    // bounded wait for the item of chunk k-1 (a smaller ticket, already running)
-                    const unsigned long long tw = globaltimer();
-                    int f;
-                    while ((f = ld_acquire_gpu(flag)) < (int)k) {
-                        if (*abort || globaltimer() - tw > kWaitLimitNs) {
-                            *abort = 1;
-                            break;
-                        }
-                        __nanosleep(64);
-                    }
-                    if (f >= kChainAbort) *abort = 1;
-                }
-                mbar_arrive(&sm.bar_flag_ok);
-            }
-            if (!warp_wait(&sm.bar_flag_ok, j & 1, abort)) break;
-            if (__shfl_sync(0xffffffffu, *abort, 0)) break;
-            // Q = 256: the accumulators hold S_lo (rows 0-127, decayed to row 127) and S_hi
-            // (rows 128-255, decayed to row 255); the chunk's own state is
-            // S = exp(cs_255 - cs_127) S_lo + S_hi, and the state entering rows 128-255 is
-            // h_mid = exp(cs_127) h_in[k] + S_lo.  Q = 128: one accumulator, S.
-            const bool halves = Q == 256;
-            const float dec = __expf(sm.cs_last[j]);
-            const float dmid = __expf(sm.cs_mid[j]);
-            const float dhl = __expf(sm.cs_last[j] - sm.cs_mid[j]);
-            const int nsub = Q / kTileRows;
-            const int64_t sub0 = (b * nchunks + k) * nsub;   // sub-chunk index of rows 0-127
-            bf16 *hrow = chain.hin + (sub0 * H + h0 + j) * (int64_t)(kP * kN) + n * 64;
-            bf16 *mrow = chain.hin + ((sub0 + 1) * H + h0 + j) * (int64_t)(kP * kN) + n * 64;
-            const float *ring_in = chain.ring + ((bh * 2 + (k & 1)) * kN + n) * (int64_t)kP;
-            float *ring_out = chain.ring + ((bh * 2 + ((k + 1) & 1)) * kN + n) * (int64_t)kP;
-            const float *ip = chain.init ? chain.init + bh * (int64_t)(kP * kN) + n : nullptr;
-            // 16 columns p at a time (registers: the accumulators, the entering state)
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                uint32_t lo[16], hi[16];
-                tmem_ld16(taddr + 16 * qq, lo);
-                if (halves) tmem_ld16(taddr + 64 + 16 * qq, hi);
-                float hv[16];
-                if (k == 0) {
-#pragma unroll
-                    for (int p = 0; p < 16; ++p) hv[p] = ip ? ip[(16 * qq + p) * kN] : 0.f;
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(ring_in) +
-                                                4 * qq + c);
-                        hv[4 * c] = v.x;
-                        hv[4 * c + 1] = v.y;
-                        hv[4 * c + 2] = v.z;
-                        hv[4 * c + 3] = v.w;
-                    }
-                }
-                tmem_ld_wait();
-                // the entering states of the two half-chunks as the chunk scan's operands:
-                // row n of 64 p, 16-byte pieces swizzled
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int piece = 2 * qq + c;
-                    *reinterpret_cast<uint4 *>(hrow + 8 * (piece ^ (n & 7))) =
-                        make_uint4(pack_bf16x2(hv[8 * c], hv[8 * c + 1]),
-                                   pack_bf16x2(hv[8 * c + 2], hv[8 * c + 3]),
-                                   pack_bf16x2(hv[8 * c + 4], hv[8 * c + 5]),
-                                   pack_bf16x2(hv[8 * c + 6], hv[8 * c + 7]));
-                    if (halves) {
-                        float m[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            m[e] = fmaf(dmid, hv[8 * c + e], __uint_as_float(lo[8 * c + e]));
-                        *reinterpret_cast<uint4 *>(mrow + 8 * (piece ^ (n & 7))) =
-                            make_uint4(pack_bf16x2(m[0], m[1]), pack_bf16x2(m[2], m[3]),
-                                       pack_bf16x2(m[4], m[5]), pack_bf16x2(m[6], m[7]));
-                    }
-                }
-                float sf[16];   // the chunk's own state S, these 16 columns
-#pragma unroll
-                for (int p = 0; p < 16; ++p)
-                    sf[p] = halves ? fmaf(dhl, __uint_as_float(lo[p]), __uint_as_float(hi[p]))
-                                   : __uint_as_float(lo[p]);
-                // h_in[k+1] = exp(cs_last) h_in[k] + S: the ring slot the next chunk reads, or
-                // the final state after the last chunk
-                if (k + 1 < nchunks) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        __stcg(reinterpret_cast<float4 *>(ring_out) + 4 * qq + c,
-                               make_float4(fmaf(dec, hv[4 * c], sf[4 * c]),
-                                           fmaf(dec, hv[4 * c + 1], sf[4 * c + 1]),
-                                           fmaf(dec, hv[4 * c + 2], sf[4 * c + 2]),
-                                           fmaf(dec, hv[4 * c + 3], sf[4 * c + 3])));
-                } else if (chain.final_state) {
-                    float *fo = chain.final_state + bh * (int64_t)(kP * kN) + n;
-#pragma unroll
-                    for (int p = 0; p < 16; ++p)
-                        fo[(16 * qq + p) * kN] = fmaf(dec, hv[p], sf[p]);
-                }
-            }
+            uint32_t r0[32], r1[32];
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + a * kP;
+            tmem_ld32(taddr, r0);
+            tmem_ld32(taddr + 32, r1);
+            tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(&sm.bar_acc_free[a]);
-            // every thread's part of h_in[k+1] is visible GPU-wide before the flag
-            if (k + 1 < nchunks) __threadfence();
-            mbar_arrive(&sm.bar_pub);
-            if (et == 0 && mbar_wait(&sm.bar_pub, j & 1, abort) && k + 1 < nchunks) {
-                st_release_gpu(flag, (int)(k + 1));
-                sm.published = j + 1;
-            }
+            // the chunk states are kept as [n][p]: 64 consecutive p per thread
+            float4 *out = reinterpret_cast<float4 *>(
+                states + (((b * nchunks + k) * H + h0 + j) * (int64_t)kN + n) * kP);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                __stcs(out + c,
+                       make_float4(__uint_as_float(r0[4 * c]), __uint_as_float(r0[4 * c + 1]),
+                                   __uint_as_float(r0[4 * c + 2]), __uint_as_float(r0[4 * c + 3])));
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                __stcs(out + 8 + c,
+                       make_float4(__uint_as_float(r1[4 * c]), __uint_as_float(r1[4 * c + 1]),
+                                   __uint_as_float(r1[4 * c + 2]), __uint_as_float(r1[4 * c + 3])));
         }
     }
 
@@ -449,13 +259,8 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_wait_drain(&sm.bar_drain, 0);
         }
         if (threadIdx.x == 0) {
-            // chained form: heads whose outgoing state was not published break the chain on
-            // purpose, so that the later chunks' items stop waiting at once
-            if (kChain && k + 1 < nchunks)
-                for (int j = sm.published; j < nh; ++j)
-                    st_release_gpu(chain.flags + b * H + h0 + j, kChainAbort);
             drain_sleep();
-            atomicOr(status, kChain ? 4 : 1);
+            atomicOr(status, 1);
         }
     }
     tc_fence_before();
@@ -555,12 +360,7 @@ __device__ __forceinline__ void scale_pieces(uint8_t *base, int first, int strid
     }
 }
 
-// kGate: the output is y * z * sigmoid(z).
-// kSub: the state entering each 128-row tile is given (hin holds one block per tile: the
-// state entering the chunk, and for Q = 256 the state at its row 127), so the second tile of a
-// chunk is computed exactly like the first -- its diagonal block plus C h^T from its own
-// entering state -- with no off-diagonal block.
-template <bool kGate, bool kSub>
+template <bool kGate>   // kGate: the output is y * z * sigmoid(z)
 __global__ void __launch_bounds__(kScanThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_b,
@@ -591,16 +391,14 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     int len;
     chunk_span(tab, k, Q, seqlen, t0, len);
     if (T * kTileRows >= len) return;  // tile past the end of the sequence, or unused slot
-    const bool offd = T && !kSub;        // the tile has an off-diagonal block
+    const bool offd = T != 0;            // the second tile has an off-diagonal block
     const int KI = offd ? 2 * kTileRows : kTileRows;  // source columns (x rows) of the tile
-    const int xrow = kSub ? kTileRows * T : 0;        // first sequence row of those, in the chunk
     const int nst = offd ? 2 : kXStagesMax;   // x / h_in stages
     const uint32_t gdiag = offd ? 128u : 0u;  // TMEM column of the diagonal block of C B^T
     const uint32_t pcol = offd ? 0u : 128u;   // TMEM columns of the P ring (over C B_off^T)
     const int xdiag = offd ? kTileRows : 0;   // first x row of the diagonal block in the stage
-    // this tile's entering-state block: one per chunk, or one per 128-row tile (kSub)
-    const bf16 *hblk = hin + (kSub ? (b * nchunks + k) * nT + T : b * nchunks + k) * (int64_t)H *
-                                 (kP * kN);
+    // the chunk's entering-state blocks (one per head)
+    const bf16 *hblk = hin + (b * nchunks + k) * (int64_t)H * (kP * kN);
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_cb, 1);
@@ -653,11 +451,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             for (int a = 0; a < 2; ++a)
                 for (int r = 0; r < KI / kTileRows; ++r)
                     tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
-                                64 * a, g, (int)(t0 + xrow + kTileRows * r), (int)b);
+                                64 * a, g, (int)(t0 + kTileRows * r), (int)b);
             // x is an input of the scan: start streaming the first heads' tiles into L2 while
             // the state-passing kernel finishes
             for (int j = 0; j < nh && j < nst; ++j)
-                tma_prefetch_l2_4d(offd ? &tm_x2 : &tm_x, 0, h0 + j, (int)(t0 + xrow), (int)b);
+                tma_prefetch_l2_4d(offd ? &tm_x2 : &tm_x, 0, h0 + j, (int)t0, (int)b);
             griddep_wait();   // cs / dt and the entering states come from earlier kernels
         }
         for (int j = 0; lane == 0 && j < nh; ++j) {   // lane 0 alone runs the loop
@@ -682,13 +480,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                                   (uint32_t)(KI * kRowBytes + 2 * kP * kRowBytes));
             // x rows [0, KI) of the chunk as one box (fewer, larger TMA boxes stream faster);
             // h_in is stored in its shared-memory layout, so one contiguous copy suffices
-            tma_load_4d(stg, offd ? &tm_x2 : &tm_x, &sm.bar_xh_full[xs], 0, h,
-                        (int)(t0 + xrow), (int)b);
+            tma_load_4d(stg, offd ? &tm_x2 : &tm_x, &sm.bar_xh_full[xs], 0, h, (int)t0, (int)b);
             bulk_load(stg + scan_hoff(offd), hblk + (int64_t)h * (kP * kN), kP * kN * 2,
                       &sm.bar_xh_full[xs]);
             // the operands this stage will hold next: into L2 now, so their loads are L2 hits
             if (j + nst < nh) {
-                tma_prefetch_l2_4d(offd ? &tm_x2 : &tm_x, 0, h + nst, (int)(t0 + xrow), (int)b);
+                tma_prefetch_l2_4d(offd ? &tm_x2 : &tm_x, 0, h + nst, (int)t0, (int)b);
                 bulk_prefetch_l2(hblk + (int64_t)(h + nst) * (kP * kN), kP * kN * 2);
             }
             // the gate rows this tile's epilogue will read: into L2 now, a few heads ahead
@@ -1074,8 +871,7 @@ bool tc_supported(bool is_bf16, int P, int N, int Q)
 cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
-                                  cudaStream_t st, const char **why, const int2 *tab,
-                                  const StateChain *chain)
+                                  cudaStream_t st, const char **why, const int2 *tab)
 {
     CUtensorMap mx, mb;   // boxes of a whole chunk (Q rows)
     if (!make_seq_map(&mx, x, batch, seqlen, H, kP, Q) ||
@@ -1083,31 +879,25 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
         *why = "chunk state: cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
-    if (chain && tab) {
-        *why = "chunk state: the chained form takes fixed-length input only";
-        return cudaErrorInvalidValue;
-    }
     const int hpg = H / G;
     const int hpc = heads_per_cta(batch * nchunks * G, hpg, 4.0, 2.0);
     const int nhb = (hpg + hpc - 1) / hpc;
     const size_t smem = sizeof(StateSmem) + 1024;
-    auto kern = chain ? chunk_state_tc_kernel<true> : chunk_state_tc_kernel<false>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(chunk_state_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk state: set smem attribute"; return e; }
     const unsigned grid = (unsigned)(batch * nchunks * G * nhb);
-    StateChain none = {};
-    *why = chain ? "chained chunk state (tcgen05) launch" : "chunk state (tcgen05) launch";
-    return launch_pdl(kern, grid, kStateThreads, smem, st, mx, mb, dtc, cs, states, status, H, G,
-                      Q, nchunks, nhb, hpc, seqlen, tab, take_test_skip(kTestChunkState),
-                      chain ? *chain : none);
+    *why = "chunk state (tcgen05) launch";
+    return launch_pdl(chunk_state_tc_kernel, grid, kStateThreads, smem, st, mx, mb, dtc, cs,
+                      states, status, H, G, Q, nchunks, nhb, hpc, seqlen, tab,
+                      take_test_skip(kTestChunkState));
 }
 
 cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
                                  int Q, int64_t nchunks, cudaStream_t st, const char **why,
-                                 const int2 *tab, const bf16 *z, bool sub)
+                                 const int2 *tab, const bf16 *z)
 {
     CUtensorMap mx, mx2, mb, mc, mz;
     if (z) {
@@ -1131,8 +921,7 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     const int hpc = scan_heads_per_cta(batch * nchunks * G * (Q / kTileRows), hpg);
     const int nhb = (hpg + hpc - 1) / hpc;
     const size_t smem = sizeof(ScanSmem) + 1024;
-    auto kern = z ? (sub ? chunk_scan_tc_kernel<true, true> : chunk_scan_tc_kernel<true, false>)
-                  : (sub ? chunk_scan_tc_kernel<false, true> : chunk_scan_tc_kernel<false, false>);
+    auto kern = z ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk scan: set smem attribute"; return e; }

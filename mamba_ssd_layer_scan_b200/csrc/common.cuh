@@ -75,14 +75,9 @@ struct WsLayout {
     size_t states;      // float [b][c][H][P][N] (CUDA-core path) or [b][c][H][N][P] (tensor-core
                         // path): per-chunk state, then (in place) state entering
     size_t hin_bf16;    // bf16  [b][c][H] blocks of P x N (hin_swizzled_offset): state entering
-                        // each chunk (tensor-core path); [b][c][Q / 128][H] blocks, the state
-                        // entering each 128-row tile, when the chained chunk state runs
-    size_t sync;        // int [kSyncFlags + b * H]: the chained chunk state's ticket counter (at
-                        // 0) and per-(batch, head) flags (from kSyncFlags) (tensor-core path)
+                        // each chunk (tensor-core path)
     size_t total;
 };
-
-constexpr int kSyncFlags = 64;   // the flags start one 256-byte line after the counter
 
 // Where chunk k of the workspace sits in the token sequence.  Without a table (fixed-length
 // input) chunk k of batch row b starts at token k Q of that row and holds min(Q, L - k Q)
@@ -102,8 +97,7 @@ __device__ __forceinline__ void chunk_span(const int2 *tab, int64_t k, int Q, in
     }
 }
 
-// Workspace status word bits: 1, 2, 4 = a bounded wait timed out (chunk state, chunk scan,
-// chained chunk state);
+// Workspace status word bits: 1, 2 = a bounded wait timed out (chunk state, chunk scan);
 // kStatusBadSeqlens = the cu_seqlens of a variable-length call are inconsistent.
 constexpr int kStatusBadSeqlens = 0x10000;
 
@@ -119,14 +113,12 @@ constexpr int kTestChunkScan = 2;
 int take_test_skip(int kernel);
 
 // ---- launchers (each returns the launch's cudaError_t) ----
-// Also zeroes *status (nullable) so each scan starts with a clean status word, and the nsync
-// ints at sync (nullable: the chained chunk state's counter and flags); when dtc is non-null,
-// writes dt re-laid out as (b, c, H, Q) with zeros past the end of the sequence.
+// Also zeroes *status (nullable) so each scan starts with a clean status word, and, when dtc is
+// non-null, writes dt re-laid out as (b, c, H, Q) with zeros past the end of the sequence.
 cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *cs, float *dtc,
                                 int *status, int64_t batch, int64_t seqlen, int nheads, int Q,
                                 int64_t nchunks, cudaStream_t st, const int2 *tab = nullptr,
-                                bool unit_weights = false, int *sync = nullptr,
-                                int64_t nsync = 0);
+                                bool unit_weights = false);
 
 // Packed variable-length input: the chunk table (tab, nchunks entries) and the first chunk of
 // every sequence (cstart, nseq + 1 entries) from cu_seqlens; clears *status and sets
@@ -186,27 +178,10 @@ cudaError_t launch_fill_final(const float *init, float *final_state, int64_t n,
 // Tensor-core (tcgen05 + TMA) path: bf16, P = 64, N = 128, Q in {128, 256}.
 bool tc_supported(bool is_bf16, int P, int N, int Q);
 
-// The chained form of the chunk-state kernel (fixed-length input only): it also carries the
-// state across chunks, so no float32 chunk states go to HBM and no state-passing kernel runs.
-// ring: batch * H * 2 * P * N floats; flags: batch * H ints and counter: one int, all zero at
-// the launch (the cumsum kernel clears them).  hin receives the bf16 state entering every
-// 128-row tile (Q / 128 blocks per chunk: the chunk's entering state, and for Q = 256 the state
-// at its row 127), final_state (nullable) the float32 state after the last chunk, from init
-// (nullable).
-struct StateChain {
-    float *ring;
-    int *flags;
-    int *counter;
-    const float *init;
-    float *final_state;
-    bf16 *hin;
-    int64_t batch;
-};
 cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
-                                  cudaStream_t st, const char **why, const int2 *tab = nullptr,
-                                  const StateChain *chain = nullptr);
+                                  cudaStream_t st, const char **why, const int2 *tab = nullptr);
 // Offset (in elements), inside one (batch, chunk, head) block of the bf16 entering states, of
 // state element (p, n) for P = 64, N = 128.  The block is stored exactly as the tensor cores
 // read it from shared memory as the MN-major operand h^T (K = n, N = p): 128 rows n of 64 p
@@ -273,13 +248,10 @@ cudaError_t launch_group_sum(const float *in, const float *w, float *out, int64_
 cudaError_t launch_scale_init_grad(const float *F, const float *dt, const float *A, float *out,
                                    int64_t batch, int64_t L, int H, int PN, cudaStream_t st);
 
-// sub: hin holds the entering state of every 128-row tile (Q / 128 blocks per chunk, as the
-// chained chunk-state kernel writes them), otherwise one block per chunk.
 cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
                                  int Q, int64_t nchunks, cudaStream_t st, const char **why,
-                                 const int2 *tab = nullptr, const bf16 *z = nullptr,
-                                 bool sub = false);
+                                 const int2 *tab = nullptr, const bf16 *z = nullptr);
 
 }  // namespace ssd

@@ -82,28 +82,8 @@ ssd::WsLayout layout(const ssd_shape *s, int Q)
     w.dtc = w.cs + round256(rows * Q * sizeof(float));
     w.states = w.dtc + (tc ? round256(rows * Q * sizeof(float)) : 0);
     w.hin_bf16 = w.states + round256(rows * s->headdim * s->dstate * sizeof(float));
-    // the chained form keeps one entering state per 128-row tile (Q / 128 per chunk)
-    const size_t nsub = Q > 128 ? (size_t)(Q / 128) : 1;
-    w.sync = w.hin_bf16 +
-             (tc ? round256(nsub * rows * s->headdim * s->dstate * sizeof(uint16_t)) : 0);
-    w.total = w.sync + (tc ? round256((ssd::kSyncFlags + (size_t)s->batch * s->nheads) * 4) : 0);
+    w.total = w.hin_bf16 + (tc ? round256(rows * s->headdim * s->dstate * sizeof(uint16_t)) : 0);
     return w;
-}
-
-// How the tensor-core path carries the state across chunks: the chained chunk-state kernel
-// (chunk states stay on chip, one item per chunk waits for the previous chunk's) for short
-// sequences, or the chunk-state kernel followed by the state-passing kernel.  The chained form
-// is serial in the chunks (one hand-off of a few microseconds each), so long sequences take the
-// two-kernel form.
-constexpr int64_t kChainMaxChunks = 32;
-std::atomic<int> g_state_form{0};   // failure-injection / test override: 0 auto, 1 split, 2 chain
-
-bool use_state_chain(int64_t nchunks)
-{
-    const int f = g_state_form.load();
-    if (f == 1) return false;
-    if (f == 2) return true;
-    return nchunks <= kChainMaxChunks;
 }
 
 // Workspace of a variable-length call: the status word, the chunk table (one slot per possible
@@ -171,15 +151,6 @@ extern "C" {
 const char *ssd_last_error(void) { return g_err; }
 
 const char *ssd_version(void) { return "ssd-b200 0.1 (sm_100a)"; }
-
-ssd_status ssd_testing_state_form(int form)
-{
-    if (form < 0 || form > 2)
-        return fail(SSD_ERR_INVALID_ARG, "form must be 0 (automatic), 1 (two kernels) or 2 "
-                                         "(chained) (got %d)", form);
-    g_state_form.store(form);
-    return SSD_OK;
-}
 
 ssd_status ssd_testing_skip_stage(int kernel, int cta)
 {
@@ -289,12 +260,9 @@ ssd_status scan_impl(const ssd_shape *shape, const void *x, const float *dt, con
         dt = dt_eff;
     }
     const bool tc = ssd::tc_supported(bf, P, N, Q);
-    const bool chain = tc && use_state_chain(nchunks);
     float *dtc = tc ? reinterpret_cast<float *>(ws + wl.dtc) : nullptr;
-    int *sync = reinterpret_cast<int *>(ws + wl.sync);
     e = ssd::launch_chunk_cumsum(dt, A, cs, dtc, status, s.batch, s.seqlen, H, Q, nchunks,
-                                 cs_stream, nullptr, false, chain ? sync : nullptr,
-                                 chain ? ssd::kSyncFlags + s.batch * H : 0);
+                                 cs_stream);
     if (e != cudaSuccess) return cuda_fail(e, "dA cumsum launch");
     if ((e = record(stage_events, 1, cs_stream)) != cudaSuccess)
         return cuda_fail(e, "record stage event");
@@ -302,35 +270,21 @@ ssd_status scan_impl(const ssd_shape *shape, const void *x, const float *dt, con
     if (tc) {
         const char *why = "";
         ssd::bf16 *hin = reinterpret_cast<ssd::bf16 *>(ws + wl.hin_bf16);
-        if (chain) {
-            // chunk states and the carry across chunks in one kernel; the state-passing stage
-            // is then empty (its two stage events are recorded back to back)
-            const ssd::StateChain sc = {states, sync + ssd::kSyncFlags, sync, init_state,
-                                        final_state, hin, s.batch};
-            e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs,
-                                           states, status, s.batch, s.seqlen, H, G, Q, nchunks,
-                                           cs_stream, &why, nullptr, &sc);
-            if (e != cudaSuccess) return cuda_fail(e, why);
-            if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess ||
-                (e = record(stage_events, 3, cs_stream)) != cudaSuccess)
-                return cuda_fail(e, "record stage event");
-        } else {
-            e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs,
-                                           states, status, s.batch, s.seqlen, H, G, Q, nchunks,
-                                           cs_stream, &why);
-            if (e != cudaSuccess) return cuda_fail(e, why);
-            if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess)
-                return cuda_fail(e, "record stage event");
-            e = ssd::launch_state_passing(states, cs, init_state, final_state, hin, s.batch, H,
-                                          P, N, Q, nchunks, cs_stream);
-            if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
-            if ((e = record(stage_events, 3, cs_stream)) != cudaSuccess)
-                return cuda_fail(e, "record stage event");
-        }
+        e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs,
+                                       states, status, s.batch, s.seqlen, H, G, Q, nchunks,
+                                       cs_stream, &why);
+        if (e != cudaSuccess) return cuda_fail(e, why);
+        if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess)
+            return cuda_fail(e, "record stage event");
+        e = ssd::launch_state_passing(states, cs, init_state, final_state, hin, s.batch, H, P, N,
+                                      Q, nchunks, cs_stream);
+        if (e != cudaSuccess) return cuda_fail(e, "state passing launch");
+        if ((e = record(stage_events, 3, cs_stream)) != cudaSuccess)
+            return cuda_fail(e, "record stage event");
         e = ssd::launch_chunk_scan_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B,
                                       (const ssd::bf16 *)C, cs, hin, D, (ssd::bf16 *)y, status,
                                       s.batch, s.seqlen, H, G, Q, nchunks, cs_stream, &why,
-                                      nullptr, (const ssd::bf16 *)z, chain);
+                                      nullptr, (const ssd::bf16 *)z);
         if (e != cudaSuccess) return cuda_fail(e, why);
         if ((e = record(stage_events, 4, cs_stream)) != cudaSuccess)
             return cuda_fail(e, "record stage event");

@@ -54,13 +54,3 @@ def max_rel_slices(gpu, ref, reduce_axes):
     i = int(np.argmax(rel))
     return float(rel.flat[i]), np.unravel_index(i, rel.shape)
 
-
-def set_state_form(form):
-    """Selects how the tensor-core path carries the state across chunks (include/ssd_testing.h):
-    0 automatic, 1 chunk-state + state-passing kernels, 2 the chained chunk-state kernel."""
-    import ctypes
-    from mamba_ssd_layer_scan_b200 import ssd
-    f = ssd.lib().ssd_testing_state_form
-    f.restype = ctypes.c_int
-    f.argtypes = [ctypes.c_int]
-    assert f(form) == ssd.SSD_OK, ssd.last_error()

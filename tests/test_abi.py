@@ -32,7 +32,7 @@ def test_testing_header_exported_and_validated(L):
     text = open(ssd.HEADER.replace("ssd.h", "ssd_testing.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = sorted(set(re.findall(r"\b(ssd_[a-z0-9_]+)\s*\(", text)))
-    assert names == ["ssd_testing_skip_stage", "ssd_testing_state_form"]
+    assert names == ["ssd_testing_skip_stage"]
     for name in names:
         assert hasattr(L, name)
     f = L.ssd_testing_skip_stage
@@ -40,11 +40,6 @@ def test_testing_header_exported_and_validated(L):
     f.argtypes = [ctypes.c_int, ctypes.c_int]
     assert f(7, 0) == ssd.SSD_ERR_INVALID_ARG
     assert f(2, -1) == ssd.SSD_ERR_INVALID_ARG
-    g = L.ssd_testing_state_form
-    g.restype = ctypes.c_int
-    g.argtypes = [ctypes.c_int]
-    assert g(3) == ssd.SSD_ERR_INVALID_ARG
-    assert g(0) == ssd.SSD_OK
 
 
 def test_version(L):
@@ -63,11 +58,8 @@ def test_workspace_size_layout():
     c = L_ // Q
     ws = ssd.workspace_size(_shape(), Q)
     # status word + cs (f32) + per-chunk dt rows (f32) + chunk states (f32) + bf16 entering
-    # states of every 128-row tile + the chained chunk state's counter and per-(batch, head)
-    # flags, 256-byte rounded (the dt rows, bf16 states and flags only on the tensor-core path)
-    sync = -(-(64 + b * H) * 4 // 256) * 256
-    expect = (256 + 2 * b * c * H * Q * 4 + b * c * H * P * N * 4 + (Q // 128) * b * c * H * P * N * 2
-              + sync)
+    # states (the last two regions only on the tensor-core path)
+    expect = 256 + 2 * b * c * H * Q * 4 + b * c * H * P * N * 4 + b * c * H * P * N * 2
     assert ws == expect
     # float32 inputs run the CUDA-core path, which keeps the entering state in place (no bf16 copy)
     ws32 = ssd.workspace_size(_shape(dtype=ssd.SSD_F32), Q)

@@ -14,7 +14,7 @@ import pytest
 import oracle
 from mamba_ssd_layer_scan_b200 import configs, inputs, ssd
 
-from _util import TOL, max_rel_per_pair, max_rel_slices, set_state_form, to_np, torch_inputs
+from _util import TOL, max_rel_per_pair, max_rel_slices, to_np, torch_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -105,52 +105,23 @@ def test_small_full_parity(cuda_device, name, w, chunk):
     check_against_oracle(inp, y, final)
 
 
-# The tensor-core cases again with a nonzero initial state and a fresh draw, once with each way
-# of carrying the state across chunks: the chunk-state kernel followed by the state-passing
-# kernel (form 1), and the chained chunk-state kernel that carries it itself (form 2).
+# The tensor-core cases again with a nonzero initial state and a fresh draw.
 TC_SMALL = [s for s in SMALL if s[0].startswith("bf16_tc")]
 
 
-@pytest.fixture
-def state_form():
-    yield set_state_form
-    set_state_form(0)
-
-
-@pytest.mark.parametrize("form", [1, 2], ids=["two_kernels", "chained"])
 @pytest.mark.parametrize("name,w,chunk", TC_SMALL, ids=[s[0] for s in TC_SMALL])
-def test_small_parity_with_initial_state(cuda_device, state_form, form, name, w, chunk):
+def test_small_parity_with_initial_state(cuda_device, name, w, chunk):
     import torch
-    state_form(form)
     inp = inputs.make_inputs(w.with_(init_state=True, seed=w.seed + 17))
     t = torch_inputs(inp, cuda_device)
     y, final = run_fwd(torch, t, inp.w, chunk, cuda_device)
     check_against_oracle(inp, y, final)
 
 
-@pytest.mark.parametrize("w", [configs.SSD_2P7B.with_(init_state=True),
-                               configs.SSD_LONG.with_(seqlen=16384)],
-                         ids=["ssd_2p7b_init", "long_g8_64_chunks"])
-def test_state_forms_full_size_every_output(cuda_device, state_form, w):
-    """Both forms at full size, every slice against the oracle.  They round differently (the
-    chained form decays the two 128-row halves of a chunk to their own last rows and hands the
-    second half its own bf16 entering state), so they agree with each other only to the bound."""
-    import torch
-    inp = inputs.make_inputs(w)
-    t = torch_inputs(inp, cuda_device)
-    outs = []
-    for form in (1, 2):
-        state_form(form)
-        y, f = run_fwd(torch, t, w, w.chunk, cuda_device, guards=False)
-        check_against_oracle(inp, y, f, rows_per_block=1)
-        outs.append((y, f))
-    ey = max_rel_slices(to_np(outs[0][0]), to_np(outs[1][0]), (1, 3))[0]
-    assert ey <= TOL["bf16"], f"the two forms differ by {ey:.3e}"
-
-
 # ------------------------------------------------------------------ full-size workloads
 FULL = [("ssd_370m", configs.SSD_370M, None),
         ("ssd_2p7b", configs.SSD_2P7B, 1),
+        ("ssd_2p7b_init", configs.SSD_2P7B.with_(init_state=True), 1),
         ("ssd_long", configs.SSD_LONG, 1)]
 
 

@@ -80,6 +80,8 @@ def test_local_phase_outputs(cuda_device):
 
 
 def test_one_rank_equals_plain_scan(cuda_device):
+    """With one rank the two phases run the plain scan's kernels (chunk states, then state
+    passing, then the chunk scan), so they equal it bit for bit."""
     import torch
     w = configs.SSD_370M.with_(batch=2, seqlen=800, nheads=8, init_state=True)
     t = torch_inputs(inputs.make_inputs(w), cuda_device)
