@@ -9,11 +9,12 @@
 // block matrix multiplications).  Two kernels:
 //
 // chunk_state_tc_kernel   S_k^T = B_k^T (w o X_k),  w_tau = exp(cs_last - cs_tau) dt_tau
-//     One CTA per (batch, chunk, group, block of heads).  The chunk's B rows are loaded once
-//     and shared by the heads of the block; per head, the x tile and the head's cs / dt rows
-//     arrive by TMA (4 stages), 8 warps scale the x rows by w in shared memory, one
-//     M=128 (n) x N=64 (p) x K=Q MMA chain accumulates S^T in TMEM (double-buffered), and 4
-//     epilogue warps move it to global memory while the next head's MMAs run.
+//     One CTA per SM, each taking an equal run of the flat list of (batch, chunk, group, head)
+//     items.  A chunk's B rows are loaded once per run of its heads and shared by them; per
+//     head, the x tile and the head's cs / dt rows arrive by TMA (4 stages), 8 warps scale the x
+//     rows by w in shared memory, one M=128 (n) x N=64 (p) x K=Q MMA chain accumulates S^T in
+//     TMEM (double-buffered), and 4 epilogue warps move it to global memory while the next
+//     head's MMAs run.
 //
 // chunk_scan_tc_kernel    y = (C B^T o L o dt + diag(D)) X  +  exp(cs) o (C h_in^T)
 //     One CTA per (batch, chunk, 128-row tile of the chunk, group, block of heads).  C B^T is
@@ -26,8 +27,7 @@
 //     exponential of its own.  The same worker warps then run the previous head's epilogue.
 //
 // Roles (warp-specialised; every wait is on an mbarrier and bounded, see sm100.cuh):
-//   state kernel: warp 0 TMA, warps 1 and 3 MMA (alternate heads), warp 2 TMEM owner,
-//                 warps 4-11 scale, 12-15 epilogue
+//   state kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-11 scale, 12-15 epilogue
 //   scan  kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-19 mask + epilogue
 #include <cudaTypedefs.h>
 
@@ -59,51 +59,70 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // ============================================================ chunk state
+//
+// Work is the flat list of (batch, chunk, group, head) items, the heads of a group consecutive;
+// CTA c of a grid of one CTA per SM takes items [c n / grid, (c + 1) n / grid), so every SM gets
+// the same number of heads to within one.  A run of items of the same (batch, chunk, group) is a
+// segment: its heads share the chunk's B tile, which the CTA loads once per segment.
 constexpr int kStateStages = 4;
 struct alignas(1024) StateSmem {
     bf16 Bs[2][256 * 64];                 // MN-major A operand: [n atom][Q rows tau][64 n]
     bf16 Xs[kStateStages][256 * 64];      // MN-major B operand per stage: [Q rows tau][64 p]
     float cs_v[kStateStages][256];        // per stage: the head's chunk-local cumsum row
     float dt_v[kStateStages][256];        // per stage: the head's dt row (0 past the end)
-    uint64_t bar_b;
+    uint64_t bar_b, bar_b_free;
     uint64_t bar_x_full[kStateStages], bar_x_ready[kStateStages], bar_x_free[kStateStages];
     uint64_t bar_acc_full[2], bar_acc_free[2];
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort;
 };
-// warp 0 TMA, warps 1 and 3 MMA (alternate heads), warp 2 TMEM owner, warps 4-11 scale x,
-// warps 12-15 epilogue
+// warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-11 scale x, warps 12-15 epilogue
 constexpr int kStateThreads = 512;
 constexpr int kStateScaleThreads = 256;
 constexpr uint32_t kStateTmemCols = 128;   // two accumulator buffers of 64 p
+
+// Item f of the flat list: its batch row, chunk, group and head.
+struct StateItem {
+    int64_t b, k;
+    int g, h;
+    bool seg_start;   // first item of its (batch, chunk, group) within the CTA
+};
+__device__ __forceinline__ StateItem state_item(int64_t f, int64_t f0, int hpg, int G,
+                                                int64_t nchunks)
+{
+    StateItem it;
+    const int hl = (int)(f % hpg);
+    const int64_t seg = f / hpg;
+    it.g = (int)(seg % G);
+    const int64_t bk = seg / G;
+    it.k = bk % nchunks;
+    it.b = bk / nchunks;
+    it.h = it.g * hpg + hl;
+    it.seg_start = f == f0 || hl == 0;
+    return it;
+}
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                       const __grid_constant__ CUtensorMap tm_b, const float *__restrict__ dtc,
                       const float *__restrict__ cs, float *__restrict__ states,
-                      int *__restrict__ status, int H, int G, int Q, int64_t nchunks, int nhb,
-                      int hpc, int64_t seqlen, const int2 *__restrict__ tab, int skip_cta)
+                      int *__restrict__ status, int H, int G, int Q, int64_t nchunks,
+                      int64_t nitems, int64_t seqlen, const int2 *__restrict__ tab, int skip_cta)
 {
     extern __shared__ uint8_t smem_raw[];
     StateSmem &sm = *reinterpret_cast<StateSmem *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-
-    int64_t u = blockIdx.x;
-    const int hb = (int)(u % nhb); u /= nhb;
-    const int g = (int)(u % G); u /= G;
-    const int64_t k = u % nchunks, b = u / nchunks;
     const int hpg = H / G;
-    const int h0 = g * hpg + hb * hpc;
-    const int nh = min(hpc, hpg - hb * hpc);
-    int64_t t0;
-    int len;
-    chunk_span(tab, k, Q, seqlen, t0, len);
-    if (len <= 0) return;   // unused slot of a chunk table (before any barrier or TMEM use)
+    const int64_t f0 = (int64_t)blockIdx.x * nitems / gridDim.x;
+    const int64_t f1 = ((int64_t)blockIdx.x + 1) * nitems / gridDim.x;
+    const int nh = (int)(f1 - f0);
+    if (nh <= 0) return;
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_b, 1);
+        mbar_init(&sm.bar_b_free, 1);
         for (int s = 0; s < kStateStages; ++s) {
             mbar_init(&sm.bar_x_full[s], 1);
             mbar_init(&sm.bar_x_ready[s], kStateScaleThreads);
@@ -113,7 +132,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_init(&sm.bar_acc_full[s], 1);
             mbar_init(&sm.bar_acc_free[s], 128);
         }
-        mbar_init(&sm.bar_drain, 2);
+        mbar_init(&sm.bar_drain, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -129,46 +148,72 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     volatile int *abort = &sm.abort;
 
     if (warp == 0) {
-        // ---------------- TMA producer (lane 0 alone): B once, then per head its x tile and
-        // cs / dt rows
+        // ---------------- TMA producer (lane 0 alone): per segment the B tile, per head its x
+        // tile and cs / dt rows
         if (lane == 0) {
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
-            mbar_arrive_expect_tx(&sm.bar_b, 2u * Q * kRowBytes);
-            for (int a = 0; a < 2; ++a)   // boxes of Q rows
-                tma_load_4d(&sm.Bs[a][0], &tm_b, &sm.bar_b, 64 * a, g, (int)t0, (int)b);
-            // x is an input of the scan: start streaming the first heads' tiles into L2 while
-            // the cumsum kernel finishes
-            for (int j = 0; j < nh && j < kStateStages; ++j)
-                tma_prefetch_l2_4d(&tm_x, 0, h0 + j, (int)t0, (int)b);
-            griddep_wait();   // cs / dt come from the cumsum kernel
+            // x and B are inputs of the scan: start streaming the first heads' tiles into L2
+            // while the cumsum kernel finishes
+            for (int j = 0; j < nh && j < kStateStages; ++j) {
+                const StateItem it = state_item(f0 + j, f0, hpg, G, nchunks);
+                int64_t t0;
+                int len;
+                chunk_span(tab, it.k, Q, seqlen, t0, len);
+                tma_prefetch_l2_4d(&tm_x, 0, it.h, (int)t0, (int)it.b);
+            }
+            griddep_wait();   // cs / dt (and a chunk table) come from earlier kernels
+            int seg = -1;
             for (int j = 0; j < nh; ++j) {
+                const StateItem it = state_item(f0 + j, f0, hpg, G, nchunks);
+                int64_t t0;
+                int len;
+                chunk_span(tab, it.k, Q, seqlen, t0, len);
+                if (it.seg_start) {
+                    ++seg;
+                    // the previous segment's MMAs must be done with the B tile
+                    if (seg > 0 && !mbar_wait(&sm.bar_b_free, (seg - 1) & 1, abort)) break;
+                    mbar_arrive_expect_tx(&sm.bar_b, 2u * Q * kRowBytes);
+                    for (int a = 0; a < 2; ++a)   // boxes of Q rows
+                        tma_load_4d(&sm.Bs[a][0], &tm_b, &sm.bar_b, 64 * a, it.g, (int)t0,
+                                    (int)it.b);
+                }
                 const int s = j % kStateStages;
                 const uint32_t use = j / kStateStages;
                 if (j >= kStateStages && !mbar_wait(&sm.bar_x_free[s], (use - 1) & 1, abort))
                     break;
                 // failure injection (tests only): this stage is left unissued
                 if (j == 0 && (int)blockIdx.x == skip_cta) continue;
-                const int64_t vrow = ((b * nchunks + k) * H + h0 + j) * (int64_t)Q;
+                const int64_t vrow = ((it.b * nchunks + it.k) * H + it.h) * (int64_t)Q;
                 mbar_arrive_expect_tx(&sm.bar_x_full[s], (uint32_t)Q * (kRowBytes + 8));
-                tma_load_4d(&sm.Xs[s][0], &tm_x, &sm.bar_x_full[s], 0, h0 + j, (int)t0, (int)b);
+                tma_load_4d(&sm.Xs[s][0], &tm_x, &sm.bar_x_full[s], 0, it.h, (int)t0, (int)it.b);
                 bulk_load(sm.cs_v[s], cs + vrow, Q * 4, &sm.bar_x_full[s]);
                 bulk_load(sm.dt_v[s], dtc + vrow, Q * 4, &sm.bar_x_full[s]);
                 // the tile this stage will hold next: into L2 now, so its load is an L2 hit
-                if (j + kStateStages < nh)
-                    tma_prefetch_l2_4d(&tm_x, 0, h0 + j + kStateStages, (int)t0, (int)b);
+                if (j + kStateStages < nh) {
+                    const StateItem nx = state_item(f0 + j + kStateStages, f0, hpg, G, nchunks);
+                    int64_t nt0;
+                    int nlen;
+                    chunk_span(tab, nx.k, Q, seqlen, nt0, nlen);
+                    tma_prefetch_l2_4d(&tm_x, 0, nx.h, (int)nt0, (int)nx.b);
+                }
             }
         }
-    } else if (warp == 1 || warp == 3) {
-        // ---------------- MMA issuers: D[n][p] += sum_tau B[tau][n] * Xw[tau][p].  Two warps
-        // issue alternate heads (each into its own accumulator buffer).  In each, lane 0 alone
+    } else if (warp == 1) {
+        // ---------------- MMA issuer: D[n][p] += sum_tau B[tau][n] * Xw[tau][p].  Lane 0 alone
         // runs the whole loop, waits included: a lane that issued tcgen05.mma and then rejoins
         // its warp stalls for the MMAs' issue latency (hundreds of cycles) at every rejoin.
-        const int par = warp == 1 ? 0 : 1;
         const uint32_t idesc = idesc_bf16_f32(128, kP, true, true);
         const uint32_t atom_bytes = 256 * kRowBytes;  // distance between the two n atoms of Bs
-        if (lane == 0 && mbar_wait(&sm.bar_b, 0, abort)) {
-            for (int j = par; j < nh; j += 2) {
+        if (lane == 0) {
+            int seg = -1;
+            for (int j = 0; j < nh; ++j) {
+                const StateItem it = state_item(f0 + j, f0, hpg, G, nchunks);
+                const bool seg_end = j + 1 == nh || (f0 + j + 1) % hpg == 0;
+                if (it.seg_start) {
+                    ++seg;
+                    if (!mbar_wait(&sm.bar_b, seg & 1, abort)) break;
+                }
                 const int s = j % kStateStages;
                 const uint32_t use = j / kStateStages;
                 const int a = j & 1;
@@ -191,6 +236,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 }
                 mma_commit(&sm.bar_x_free[s]);
                 mma_commit(&sm.bar_acc_full[a]);
+                if (seg_end) mma_commit(&sm.bar_b_free);
             }
         }
     } else if (warp >= 4 && warp < 12) {
@@ -221,10 +267,11 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_arrive(&sm.bar_x_ready[s]);
         }
     } else if (warp >= 12) {
-        // ---------------- epilogue: TMEM (lane n, column p) -> S^T row n
+        // ---------------- epilogue: TMEM (lane n, column p) -> states[b][k][h][p][n]
         const int q = warp & 3;
         const int n = q * 32 + lane;
         for (int j = 0; j < nh; ++j) {
+            const StateItem it = state_item(f0 + j, f0, hpg, G, nchunks);
             const int a = j & 1;
             if (!warp_wait(&sm.bar_acc_full[a], (j >> 1) & 1, abort)) break;
             tc_fence_after();
@@ -235,26 +282,20 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(&sm.bar_acc_free[a]);
-            // the chunk states are kept as [n][p]: 64 consecutive p per thread
-            float4 *out = reinterpret_cast<float4 *>(
-                states + (((b * nchunks + k) * H + h0 + j) * (int64_t)kN + n) * kP);
+            // lane n writes column n of every row p: each store of the warp is 128 contiguous
+            // bytes
+            float *out = states + ((it.b * nchunks + it.k) * H + it.h) * (int64_t)(kP * kN) + n;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                __stcs(out + c,
-                       make_float4(__uint_as_float(r0[4 * c]), __uint_as_float(r0[4 * c + 1]),
-                                   __uint_as_float(r0[4 * c + 2]), __uint_as_float(r0[4 * c + 3])));
+            for (int p = 0; p < 32; ++p) out[p * kN] = __uint_as_float(r0[p]);
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                __stcs(out + 8 + c,
-                       make_float4(__uint_as_float(r1[4 * c]), __uint_as_float(r1[4 * c + 1]),
-                                   __uint_as_float(r1[4 * c + 2]), __uint_as_float(r1[4 * c + 3])));
+            for (int p = 0; p < 32; ++p) out[(32 + p) * kN] = __uint_as_float(r1[p]);
         }
     }
 
     __syncthreads();
     if (sm.abort) {
         // Let this CTA's own MMAs and TMA copies finish before TMEM and smem are released.
-        if ((warp == 1 || warp == 3) && lane == 0) {
+        if (warp == 1 && lane == 0) {
             mma_commit(&sm.bar_drain);
             mbar_wait_drain(&sm.bar_drain, 0);
         }
@@ -301,7 +342,7 @@ struct alignas(1024) ScanSmem {
                                     // that, T = 0: x / h_in stage 2; T = 1: bf16 C B_off^T
                                     // (K-major [i atom][128 rows t][64 i])
     uint8_t S01[2 * kStageBytes];   // x / h_in stages: [KI rows i][64 p] then h_in
-                                    // [128 rows n][64 p]
+                                    // [n atom][64 rows p][64 n]
     float cs_v[kScanVecStages][256];  // per stage: one head's chunk-local cumsum row
     float dt_v[kScanVecStages][256];  // per stage: its dt row (0 past the end)
     float vt[16][32];               // per worker warp: column factors of its two slices
@@ -495,6 +536,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         // ---------------- MMA issuer (lane 0 alone runs the loop: a lane that issued
         // tcgen05.mma and then rejoins its warp stalls for the MMAs' issue latency)
         const uint32_t id_g = idesc_bf16_f32(128, KI, false, false);
+        const uint32_t id_kk = idesc_bf16_f32(128, kP, false, false);   // K-major A and B
         const uint32_t id_kmn = idesc_bf16_f32(128, kP, false, true);   // B (x) MN-major
         // base descriptors; K steps are constant offsets added in fully unrolled loops (the
         // issuing thread's own instruction chain sets the MMA issue rate)
@@ -524,7 +566,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             const uint32_t stg = smem_u32(scan_stage(sm, xs, offd));
             const uint32_t dD = tmem + kAccCol + 128 * a, dA = dD + 64;
             const uint64_t xd = smem_desc_sw128(stg, 256 * kRowBytes, 1024);   // x, MN-major
-            const uint64_t hd = smem_desc_sw128(stg + scan_hoff(offd), 16384, 1024);  // h_in
+            const uint64_t hd = smem_desc_sw128(stg + scan_hoff(offd), 16, 1024);  // h_in, K-major
             if (offd) {
                 // Y_A = (C B_off^T) (v dt o X_off): A = bf16 block in R, K = 128 (i)
 #pragma unroll
@@ -533,12 +575,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     mma_bf16(dA, rd + (aoff >> 4), xd + kk * 128, id_kmn, kk > 0 ? 1u : 0u);
                 }
             }
-            // Y_A (+)= C h^T: K = 128 (n), h^T MN-major (rows n); h = h_in (T = 0) or
-            // exp(cs_127) h_in (T = 1)
+            // Y_A (+)= C h^T: K = 128 (n), h K-major (rows p, two halves of 64 n); h = h_in
+            // (T = 0) or exp(cs_127) h_in (T = 1)
 #pragma unroll
             for (int kk = 0; kk < kN / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                mma_bf16(dA, cd + (off >> 4), hd + kk * 128, id_kmn, (offd || kk > 0) ? 1u : 0u);
+                const uint32_t hoff = (kk >> 2) * (kP * kRowBytes) + (kk & 3) * 32;
+                mma_bf16(dA, cd + (off >> 4), hd + (hoff >> 4), id_kk, (offd || kk > 0) ? 1u : 0u);
             }
             for (int qb = 0; qb < 2; ++qb) {
                 const uint32_t blk = 2 * j + qb;           // P blocks are numbered per head
@@ -838,29 +881,6 @@ int scan_heads_per_cta(int64_t tiles, int hpg)
     return (hpg + nhb - 1) / nhb;   // the same number of head blocks, evenly filled
 }
 
-// Heads per CTA.  Every CTA pays a fixed ramp-up (its B / C tiles, C B^T, the first TMA round
-// trips) and drain, which only a long run of heads amortises, while too few CTAs leave SMs idle.
-// Pick the count that minimises waves x (ramp + heads x per-head time), with the waves counted
-// over the SMs of the device.
-int heads_per_cta(int64_t groups_work, int hpg, double ramp_us, double head_us)
-{
-    int sms = 148;
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int best = 1;
-    double best_t = 1e30;
-    for (int hpc = 1; hpc <= std::min(hpg, kMaxHeadsPerCta); ++hpc) {
-        const int nhb = (hpg + hpc - 1) / hpc;
-        if (hpc > 1 && (hpg + hpc - 2) / (hpc - 1) == nhb) continue;   // same split, fewer heads
-        const double ctas = (double)groups_work * nhb;
-        const double waves = std::ceil(ctas / sms);
-        const double t = waves * (ramp_us + hpc * head_us);
-        if (t < best_t - 1e-9) { best_t = t; best = hpc; }
-    }
-    return best;
-}
-
 }  // namespace
 
 bool tc_supported(bool is_bf16, int P, int N, int Q)
@@ -879,17 +899,19 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
         *why = "chunk state: cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
-    const int hpg = H / G;
-    const int hpc = heads_per_cta(batch * nchunks * G, hpg, 4.0, 2.0);
-    const int nhb = (hpg + hpc - 1) / hpc;
+    const int64_t nitems = batch * nchunks * H;   // (batch, chunk, group, head) items
+    if (nitems == 0) return cudaSuccess;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t smem = sizeof(StateSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(chunk_state_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk state: set smem attribute"; return e; }
-    const unsigned grid = (unsigned)(batch * nchunks * G * nhb);
+    const unsigned grid = (unsigned)std::min<int64_t>(sms, nitems);
     *why = "chunk state (tcgen05) launch";
     return launch_pdl(chunk_state_tc_kernel, grid, kStateThreads, smem, st, mx, mb, dtc, cs,
-                      states, status, H, G, Q, nchunks, nhb, hpc, seqlen, tab,
+                      states, status, H, G, Q, nchunks, nitems, seqlen, tab,
                       take_test_skip(kTestChunkState));
 }
 

@@ -72,8 +72,7 @@ struct WsLayout {
     size_t status;      // 256 bytes: device status word (nonzero after an in-kernel timeout)
     size_t cs;          // float [b][c][H][Q]: chunk-local inclusive cumsum of dt*A
     size_t dtc;         // float [b][c][H][Q]: dt per chunk row, 0 past the end (tensor-core path)
-    size_t states;      // float [b][c][H][P][N] (CUDA-core path) or [b][c][H][N][P] (tensor-core
-                        // path): per-chunk state, then (in place) state entering
+    size_t states;      // float [b][c][H][P][N]: per-chunk state, then (in place) state entering
     size_t hin_bf16;    // bf16  [b][c][H] blocks of P x N (hin_swizzled_offset): state entering
                         // each chunk (tensor-core path)
     size_t total;
@@ -134,8 +133,6 @@ cudaError_t launch_chunk_state_simt(bool is_bf16, const void *x, const float *dt
 
 // Carries the state across chunks: states[k] (chunk-local contribution) is replaced in place by
 // the state entering chunk k (float32), or that state is written to hin_bf16 when non-null.
-// With hin_bf16 (the tensor-core path) the chunk states are stored transposed, [N][P] per
-// (batch, chunk, head); init and final_state are always in the caller's [P][N] layout.
 cudaError_t launch_state_passing(float *states, const float *cs, const float *init,
                                  float *final_state, bf16 *hin_bf16, int64_t batch, int H,
                                  int P, int N, int Q, int64_t nchunks, cudaStream_t st);
@@ -184,12 +181,13 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
                                   cudaStream_t st, const char **why, const int2 *tab = nullptr);
 // Offset (in elements), inside one (batch, chunk, head) block of the bf16 entering states, of
 // state element (p, n) for P = 64, N = 128.  The block is stored exactly as the tensor cores
-// read it from shared memory as the MN-major operand h^T (K = n, N = p): 128 rows n of 64 p
-// (128 bytes), the 16-byte pieces of row n permuted by n mod 8 (the 128-byte swizzle), so that
-// one contiguous 16 KB copy brings a block into shared memory ready for use.
+// read it from shared memory: two halves of 64 n, each 64 rows p of 128 bytes, with the 16-byte
+// pieces of row p permuted by p mod 8 (the 128-byte swizzle), so that one contiguous 16 KB copy
+// brings a block into shared memory ready for use.
 __host__ __device__ __forceinline__ int hin_swizzled_offset(int p, int n)
 {
-    return n * 64 + ((((p >> 3) ^ (n & 7)) << 3) | (p & 7));
+    const int a = n >> 6, nl = n & 63;
+    return a * 4096 + p * 64 + ((((nl >> 3) ^ (p & 7)) << 3) | (nl & 7));
 }
 
 // Sequence parallelism (one contiguous segment per rank): the segment's total log-decay per

@@ -20,19 +20,15 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int kGroup = 8;  // chunks whose loads are issued together
 
-// kBf16Out (tensor-core path): the chunk states are [N][P] per (batch, chunk, head) and the
-// entering states go to hin in the chunk scan's operand layout; otherwise the states are [P][N]
-// and are overwritten in place by the entering states.  init and final_state are [P][N].
 template <bool kBf16Out>
 __global__ void __launch_bounds__(kThreads)
 state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
                      const float *__restrict__ init, float *__restrict__ final_state,
-                     bf16 *__restrict__ hin, int H, int P, int N, int Q, int64_t nchunks,
+                     bf16 *__restrict__ hin, int H, int PN, int Q, int64_t nchunks,
                      const int32_t *__restrict__ cstart)
 {
     griddep_wait();   // the chunk states come from the previous kernel
     griddep_launch_dependents();
-    const int PN = P * N;
     const int nblk = (PN / 4 + kThreads - 1) / kThreads;
     const int64_t v = (blockIdx.x % nblk) * (int64_t)kThreads + threadIdx.x;  // float4 index
     // b: batch row, or the packed sequence when cstart is given (its chunks are
@@ -42,21 +38,9 @@ state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
     const int64_t kbeg = cstart ? cstart[b] : 0;
     const int64_t kend = cstart ? cstart[b + 1] : nchunks;
     const int64_t rb = cstart ? 0 : b;   // workspace batch row
-    // the four elements of this thread in the caller's [P][N] layout: (p0 + i, n) for the
-    // transposed tensor-core states, (p0, n + i) otherwise
-    const int e = (int)(v * 4);
-    const int n_t = e / P, p_t = e % P;
-    const int64_t ubase = (b * H + h) * (int64_t)PN;
 
     float4 hs = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (init) {
-        if (kBf16Out) {
-            const float *ip = init + ubase + (int64_t)p_t * N + n_t;
-            hs = make_float4(ip[0], ip[N], ip[2 * N], ip[3 * N]);
-        } else {
-            hs = *reinterpret_cast<const float4 *>(init + ubase + e);
-        }
-    }
+    if (init) hs = *reinterpret_cast<const float4 *>(init + (b * H + h) * PN + v * 4);
 
     for (int64_t k0 = kbeg; k0 < kend; k0 += kGroup) {
         float4 s[kGroup];
@@ -66,7 +50,7 @@ state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
             const int64_t k = k0 + j;
             if (k < kend) {
                 const int64_t row = (rb * nchunks + k) * H + h;
-                s[j] = __ldcs(reinterpret_cast<const float4 *>(states + row * PN + e));
+                s[j] = __ldcs(reinterpret_cast<const float4 *>(states + row * PN + v * 4));
                 decay[j] = cs[row * Q + Q - 1];
             }
         }
@@ -74,19 +58,20 @@ state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
         for (int j = 0; j < kGroup; ++j) {
             const int64_t k = k0 + j;
             if (k < kend) {
-                const int64_t off = ((rb * nchunks + k) * H + h) * PN;
+                const int64_t off = ((rb * nchunks + k) * H + h) * PN + v * 4;
                 if (kBf16Out) {
-                    // tensor-core path (P = 64, N = 128): four consecutive p of row n of the
-                    // swizzled operand block, one 8-byte store
+                    // tensor-core path (P = 64, N = 128): the swizzled block layout
+                    const int e = (int)(v * 4);
+                    const int64_t hoff =
+                        ((rb * nchunks + k) * H + h) * PN + hin_swizzled_offset(e >> 7, e & 127);
                     __nv_bfloat162 lo = __floats2bfloat162_rn(hs.x, hs.y);
                     __nv_bfloat162 hi = __floats2bfloat162_rn(hs.z, hs.w);
                     uint2 packed;
                     packed.x = *reinterpret_cast<uint32_t *>(&lo);
                     packed.y = *reinterpret_cast<uint32_t *>(&hi);
-                    __stcs(reinterpret_cast<uint2 *>(hin + off + hin_swizzled_offset(p_t, n_t)),
-                           packed);
+                    __stcs(reinterpret_cast<uint2 *>(hin + hoff), packed);
                 } else {
-                    __stcs(reinterpret_cast<float4 *>(states + off + e), hs);
+                    __stcs(reinterpret_cast<float4 *>(states + off), hs);
                 }
                 const float a = __expf(decay[j]);
                 hs.x = fmaf(a, hs.x, s[j].x);
@@ -96,17 +81,8 @@ state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
             }
         }
     }
-    if (final_state) {
-        if (kBf16Out) {
-            float *fp = final_state + ubase + (int64_t)p_t * N + n_t;
-            fp[0] = hs.x;
-            fp[N] = hs.y;
-            fp[2 * N] = hs.z;
-            fp[3 * N] = hs.w;
-        } else {
-            *reinterpret_cast<float4 *>(final_state + ubase + e) = hs;
-        }
-    }
+    if (final_state)
+        *reinterpret_cast<float4 *>(final_state + (b * H + h) * PN + v * 4) = hs;
 }
 
 }  // namespace
@@ -119,7 +95,7 @@ cudaError_t launch_state_passing(float *states, const float *cs, const float *in
     const unsigned grid = (unsigned)(((PN / 4 + kThreads - 1) / kThreads) * H * batch);
     const int32_t *none = nullptr;
     return launch_pdl(hin_bf16 ? state_passing_kernel<true> : state_passing_kernel<false>, grid,
-                      kThreads, 0, st, states, cs, init, final_state, hin_bf16, H, P, N, Q, nchunks,
+                      kThreads, 0, st, states, cs, init, final_state, hin_bf16, H, PN, Q, nchunks,
                       none);
 }
 
@@ -131,7 +107,7 @@ cudaError_t launch_state_passing_varlen(float *states, const float *cs, const fl
     const int PN = P * N;
     const unsigned grid = (unsigned)(((PN / 4 + kThreads - 1) / kThreads) * H * (int64_t)nseq);
     return launch_pdl(hin_bf16 ? state_passing_kernel<true> : state_passing_kernel<false>, grid,
-                      kThreads, 0, st, states, cs, init, final_state, hin_bf16, H, P, N, Q, nchunks,
+                      kThreads, 0, st, states, cs, init, final_state, hin_bf16, H, PN, Q, nchunks,
                       cstart);
 }
 
