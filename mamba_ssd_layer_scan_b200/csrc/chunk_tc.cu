@@ -28,7 +28,7 @@
 //
 // Roles (warp-specialised; every wait is on an mbarrier and bounded, see sm100.cuh):
 //   state kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-11 scale, 12-15 epilogue
-//   scan  kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-19 mask + epilogue
+//   scan  kernel: warp 0 TMA, warp 1 MMA and TMEM owner, warps 2-17 mask + epilogue
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -45,7 +45,6 @@ using namespace sm100;
 
 constexpr int kP = 64;
 constexpr int kN = 128;
-constexpr int kMaxHeadsPerCta = 128;   // heads one CTA walks through (chosen per launch)
 constexpr int kRowBytes = 128;                  // one swizzled smem row: 64 bf16
 constexpr int kTileRows = 128;                  // rows of one TMA box / one MMA M tile
 constexpr int kBoxBytes = kTileRows * kRowBytes;  // 16 KB
@@ -329,10 +328,8 @@ constexpr int kXStagesMax = 5;   // x / h_in stages: tiles without an off-diagon
                                  // of 32 KB (three in S01, two in the B tile's space once C B^T
                                  // is done); the second tile of a chunk with one uses 2 of 48 KB
                                  // (S01; the B tile's space then holds the bf16 block)
-constexpr int kScanHeadsMin = 8;  // heads per CTA: chosen per launch in [8, 20] (fewer when a
-constexpr int kScanHeadsMax = 20; // group has fewer), see scan_heads_per_cta
+constexpr double kOffdCost = 1.35; // cost of a second-tile head relative to a first-tile head
 constexpr int kScanVecStages = 6; // cs / dt row stages (one head each)
-static_assert(kScanHeadsMax <= kMaxHeadsPerCta, "D of every head of a CTA is staged in smem");
 constexpr int kRing = 4;         // 64-column blocks of P in TMEM (two heads)
 constexpr int kStageBytes = 256 * kRowBytes + 2 * kP * kRowBytes;  // 48 KB: 256 x rows + h_in
 constexpr int kStage32 = 128 * kRowBytes + 2 * kP * kRowBytes;     // 32 KB: 128 x rows + h_in
@@ -346,8 +343,7 @@ struct alignas(1024) ScanSmem {
     float cs_v[kScanVecStages][256];  // per stage: one head's chunk-local cumsum row
     float dt_v[kScanVecStages][256];  // per stage: its dt row (0 past the end)
     float vt[16][32];               // per worker warp: column factors of its two slices
-    float Dv[kMaxHeadsPerCta];      // D of the CTA's heads
-    uint64_t bar_cb, bar_g, bar_goff;
+    uint64_t bar_cb, bar_g, bar_goff, bar_seg_done;
     uint64_t bar_xh_full[kXStagesMax], bar_xh_free[kXStagesMax], bar_xv_ready[kXStagesMax];
     uint64_t bar_vec_full[kScanVecStages], bar_vec_free[kScanVecStages];
     uint64_t bar_slot_full[kRing], bar_slot_free[kRing];
@@ -356,11 +352,11 @@ struct alignas(1024) ScanSmem {
     uint32_t tmem_base;
     int abort;
 };
-// warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warp 3 idle, warps 4-19 workers: four per TMEM
+// warp 0 TMA, warp 1 MMA and TMEM owner, warps 2-17 workers: four per TMEM
 // lane quarter, each owning a 16-column slice of every 64-column block; per head they build
 // their slice of P (mask) and then run the epilogue of the previous head for their slice of y
 constexpr int kScanWorkers = 512;
-constexpr int kScanThreads = 128 + kScanWorkers;
+constexpr int kScanThreads = 64 + kScanWorkers;   // 576 threads: up to 112 registers each
 constexpr uint32_t kScanTmemCols = 512;
 constexpr uint32_t kAccCol = 256;   // accumulator buffer a: Y_diag at 256 + 128 a, Y_A at +64
 
@@ -401,8 +397,65 @@ __device__ __forceinline__ void scale_pieces(uint8_t *base, int first, int strid
     }
 }
 
+// Work of one launch: for each 128-row tile class T of the chunks (T = 1, the tiles with an
+// off-diagonal block, exists for Q = 256), the flat list of (batch, chunk, group, head) items,
+// heads of a group consecutive.  One CTA per SM: CTAs [0, ncta1) take the T = 1 items, the rest
+// the T = 0 items, each an equal run of its class's list (the host splits the SMs between the
+// classes in proportion to their cost).  A run of items of the same (batch, chunk, group) is a
+// segment: its heads share the C and B tiles and C B^T, which the CTA computes once per
+// segment; the per-head pipeline runs on across segments, its barrier phases counted by a
+// head counter that does not restart.
+struct ScanWork {
+    int T;               // tile class of this CTA
+    int64_t f0, f1;      // its run of items
+};
+__device__ __forceinline__ ScanWork scan_work(int nT, int ncta1, int64_t nitems)
+{
+    ScanWork w;
+    int idx = blockIdx.x, m = gridDim.x;
+    if (nT == 2 && (int)blockIdx.x < ncta1) {
+        w.T = 1;
+        m = ncta1;
+    } else {
+        w.T = 0;
+        if (nT == 2) {
+            idx -= ncta1;
+            m -= ncta1;
+        }
+    }
+    w.f0 = (int64_t)idx * nitems / m;
+    w.f1 = ((int64_t)idx + 1) * nitems / m;
+    return w;
+}
+
+// The segment that starts at item f of a CTA's run [.., f1): its (batch, chunk, group), first
+// head and head count, and its chunk's span.  A segment whose tile lies past the end of its
+// chunk (a short last chunk, an unused slot of a chunk table) is skipped by every role alike.
+struct Seg {
+    int64_t b, k, t0;
+    int g, h0, nh, len;
+    bool skip;
+};
+__device__ __forceinline__ Seg scan_segment(int64_t f, int64_t f1, int hpg, int G,
+                                            int64_t nchunks, int Q, int64_t seqlen, int T,
+                                            const int2 *tab)
+{
+    Seg sg;
+    const int64_t id = f / hpg;
+    const int64_t hi = min(f1, (id + 1) * hpg);
+    sg.g = (int)(id % G);
+    const int64_t bk = id / G;
+    sg.k = bk % nchunks;
+    sg.b = bk / nchunks;
+    sg.h0 = sg.g * hpg + (int)(f % hpg);
+    sg.nh = (int)(hi - f);
+    chunk_span(tab, sg.k, Q, seqlen, sg.t0, sg.len);
+    sg.skip = T * kTileRows >= sg.len;
+    return sg;
+}
+
 template <bool kGate>   // kGate: the output is y * z * sigmoid(z)
-__global__ void __launch_bounds__(kScanThreads, 1)
+__global__ void __maxnreg__(112)   // one CTA of kScanThreads per SM: 65536 / 576 registers
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c,
@@ -411,8 +464,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const float *__restrict__ dtc,
                      const float *__restrict__ cs, const float *__restrict__ D,
                      bf16 *__restrict__ y, int *__restrict__ status, int64_t seqlen, int H,
-                     int G, int Q, int64_t nchunks, int nhb, int hpc, const int2 *__restrict__ tab,
-                     const bf16 *__restrict__ z, int skip_cta)
+                     int G, int Q, int64_t nchunks, int64_t nitems, int ncta1,
+                     const int2 *__restrict__ tab, const bf16 *__restrict__ z, int skip_cta)
 {
     extern __shared__ uint8_t smem_raw[];
     ScanSmem &sm = *reinterpret_cast<ScanSmem *>(
@@ -420,31 +473,24 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     const int nT = Q / kTileRows;
-    int64_t u = blockIdx.x;
-    const int T = nT - 1 - (int)(u % nT); u /= nT;       // heavier (later) tiles first
-    const int hb = (int)(u % nhb); u /= nhb;
-    const int g = (int)(u % G); u /= G;
-    const int64_t k = u % nchunks, b = u / nchunks;
+    const ScanWork wk = scan_work(nT, ncta1, nitems);
+    const int T = wk.T;
     const int hpg = H / G;
-    const int h0 = g * hpg + hb * hpc;
-    const int nh = min(hpc, hpg - hb * hpc);
-    int64_t t0;
-    int len;
-    chunk_span(tab, k, Q, seqlen, t0, len);
-    if (T * kTileRows >= len) return;  // tile past the end of the sequence, or unused slot
+    if (wk.f1 <= wk.f0) return;
     const bool offd = T != 0;            // the second tile has an off-diagonal block
     const int KI = offd ? 2 * kTileRows : kTileRows;  // source columns (x rows) of the tile
     const int nst = offd ? 2 : kXStagesMax;   // x / h_in stages
     const uint32_t gdiag = offd ? 128u : 0u;  // TMEM column of the diagonal block of C B^T
     const uint32_t pcol = offd ? 0u : 128u;   // TMEM columns of the P ring (over C B_off^T)
     const int xdiag = offd ? kTileRows : 0;   // first x row of the diagonal block in the stage
-    // the chunk's entering-state blocks (one per head)
-    const bf16 *hblk = hin + (b * nchunks + k) * (int64_t)H * (kP * kN);
+
+#define segment(f) scan_segment((f), wk.f1, hpg, G, nchunks, Q, seqlen, T, tab)
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_cb, 1);
         mbar_init(&sm.bar_g, 1);
         mbar_init(&sm.bar_goff, kScanWorkers);
+        mbar_init(&sm.bar_seg_done, 1);
         for (int s = 0; s < kXStagesMax; ++s) {
             mbar_init(&sm.bar_xh_full[s], 1);
             mbar_init(&sm.bar_xh_free[s], 1);
@@ -466,8 +512,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         sm.abort = 0;
         fence_mbar_init();
     }
-    for (int i = threadIdx.x; i < nh; i += blockDim.x) sm.Dv[i] = D[h0 + i];
-    if (warp == 2) {
+    if (warp == 1) {
         tmem_alloc(&sm.tmem_base, kScanTmemCols);
         tmem_relinquish();
     }
@@ -479,58 +524,92 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     volatile int *abort = &sm.abort;
 
     if (warp == 0) {
-        // ---------------- TMA producer
+        // ---------------- TMA producer (lane 0 alone): per segment the C and B tiles, per
+        // head its cs / dt rows and its x / h_in stage
         if (lane == 0) {
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
             tma_prefetch_desc(&tm_c);
             tma_prefetch_desc(&tm_x2);
-            mbar_arrive_expect_tx(&sm.bar_cb, (uint32_t)(2 * kBoxBytes + 2 * KI * kRowBytes));
-            for (int a = 0; a < 2; ++a)
-                tma_load_4d(&sm.Cs[a][0], &tm_c, &sm.bar_cb, 64 * a, g,
-                            (int)(t0 + kTileRows * T), (int)b);
-            for (int a = 0; a < 2; ++a)
-                for (int r = 0; r < KI / kTileRows; ++r)
-                    tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
-                                64 * a, g, (int)(t0 + kTileRows * r), (int)b);
-            // x is an input of the scan: start streaming the first heads' tiles into L2 while
-            // the state-passing kernel finishes
-            for (int j = 0; j < nh && j < nst; ++j)
-                tma_prefetch_l2_4d(offd ? &tm_x2 : &tm_x, 0, h0 + j, (int)t0, (int)b);
-            griddep_wait();   // cs / dt and the entering states come from earlier kernels
-        }
-        for (int j = 0; lane == 0 && j < nh; ++j) {   // lane 0 alone runs the loop
-            const int h = h0 + j;
-            const int vs = j % kScanVecStages;
-            const uint32_t vu = j / kScanVecStages;
-            if (j >= kScanVecStages && !mbar_wait(&sm.bar_vec_free[vs], (vu - 1) & 1, abort))
-                break;
-            const int64_t vrow = ((b * nchunks + k) * H + h) * (int64_t)Q;
-            mbar_arrive_expect_tx(&sm.bar_vec_full[vs], (uint32_t)(8 * Q));
-            bulk_load(sm.cs_v[vs], cs + vrow, Q * 4, &sm.bar_vec_full[vs]);
-            bulk_load(sm.dt_v[vs], dtc + vrow, Q * 4, &sm.bar_vec_full[vs]);
-            const int xs = j % nst;
-            const uint32_t xu = j / nst;
-            if (j >= nst && !mbar_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) break;
-            if (!offd && xs >= 3 && xu == 0 && !mbar_wait(&sm.bar_g, 0, abort))
-                break;   // the B tile's space is in use until C B^T is done
-            // failure injection (tests only): this stage is left unissued
-            if (j == 0 && (int)blockIdx.x == skip_cta) continue;
-            uint8_t *stg = scan_stage(sm, xs, offd);
-            mbar_arrive_expect_tx(&sm.bar_xh_full[xs],
-                                  (uint32_t)(KI * kRowBytes + 2 * kP * kRowBytes));
-            // x rows [0, KI) of the chunk as one box (fewer, larger TMA boxes stream faster);
-            // h_in is stored in its shared-memory layout, so one contiguous copy suffices
-            tma_load_4d(stg, offd ? &tm_x2 : &tm_x, &sm.bar_xh_full[xs], 0, h, (int)t0, (int)b);
-            bulk_load(stg + scan_hoff(offd), hblk + (int64_t)h * (kP * kN), kP * kN * 2,
-                      &sm.bar_xh_full[xs]);
-            // the operands this stage will hold next: into L2 now, so their loads are L2 hits
-            if (j + nst < nh) {
-                tma_prefetch_l2_4d(offd ? &tm_x2 : &tm_x, 0, h + nst, (int)t0, (int)b);
-                bulk_prefetch_l2(hblk + (int64_t)(h + nst) * (kP * kN), kP * kN * 2);
+            uint32_t J = 0;   // heads issued so far (all segments)
+            int si = 0;       // segments whose tiles were loaded
+            bool ok = true;
+            for (int64_t f = wk.f0; ok && f < wk.f1;) {
+                const Seg sg = segment(f);
+                f += sg.nh;
+                if (sg.skip) continue;
+                // the previous segment's MMAs must be done with the C tile and the B space
+                if (si > 0 && !mbar_wait(&sm.bar_seg_done, (si - 1) & 1, abort)) break;
+                mbar_arrive_expect_tx(&sm.bar_cb, (uint32_t)(2 * kBoxBytes + 2 * KI * kRowBytes));
+                for (int a = 0; a < 2; ++a)
+                    tma_load_4d(&sm.Cs[a][0], &tm_c, &sm.bar_cb, 64 * a, sg.g,
+                                (int)(sg.t0 + kTileRows * T), (int)sg.b);
+                for (int a = 0; a < 2; ++a)
+                    for (int r = 0; r < KI / kTileRows; ++r)
+                        tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
+                                    64 * a, sg.g, (int)(sg.t0 + kTileRows * r), (int)sg.b);
+                if (si == 0) {
+                    // x is an input of the scan: start streaming the first heads' tiles into
+                    // L2 while the state-passing kernel finishes
+                    for (int j = 0; j < sg.nh && j < nst; ++j)
+                        tma_prefetch_l2_4d(offd ? &tm_x2 : &tm_x, 0, sg.h0 + j, (int)sg.t0,
+                                           (int)sg.b);
+                    griddep_wait();   // cs / dt and the entering states come from earlier kernels
+                }
+                const bf16 *hblk = hin + (sg.b * nchunks + sg.k) * (int64_t)H * (kP * kN);
+                bool waited_g = false;
+                for (int j = 0; j < sg.nh; ++j, ++J) {
+                    const int h = sg.h0 + j;
+                    const int vs = J % kScanVecStages;
+                    const uint32_t vu = J / kScanVecStages;
+                    if (J >= kScanVecStages &&
+                        !mbar_wait(&sm.bar_vec_free[vs], (vu - 1) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    const int64_t vrow = ((sg.b * nchunks + sg.k) * H + h) * (int64_t)Q;
+                    mbar_arrive_expect_tx(&sm.bar_vec_full[vs], (uint32_t)(8 * Q));
+                    bulk_load(sm.cs_v[vs], cs + vrow, Q * 4, &sm.bar_vec_full[vs]);
+                    bulk_load(sm.dt_v[vs], dtc + vrow, Q * 4, &sm.bar_vec_full[vs]);
+                    const int xs = J % nst;
+                    const uint32_t xu = J / nst;
+                    if (J >= (uint32_t)nst &&
+                        !mbar_wait(&sm.bar_xh_free[xs], (xu - 1) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!offd && xs >= 3 && !waited_g) {
+                        // the B tile's space is in use until this segment's C B^T is done
+                        if (!mbar_wait(&sm.bar_g, si & 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        waited_g = true;
+                    }
+                    // failure injection (tests only): this stage is left unissued
+                    if (J == 0 && (int)blockIdx.x == skip_cta) continue;
+                    uint8_t *stg = scan_stage(sm, xs, offd);
+                    mbar_arrive_expect_tx(&sm.bar_xh_full[xs],
+                                          (uint32_t)(KI * kRowBytes + 2 * kP * kRowBytes));
+                    // x rows [0, KI) of the chunk as one box (fewer, larger TMA boxes stream
+                    // faster); h_in is stored in its shared-memory layout, so one contiguous copy
+                    tma_load_4d(stg, offd ? &tm_x2 : &tm_x, &sm.bar_xh_full[xs], 0, h,
+                                (int)sg.t0, (int)sg.b);
+                    bulk_load(stg + scan_hoff(offd), hblk + (int64_t)h * (kP * kN), kP * kN * 2,
+                              &sm.bar_xh_full[xs]);
+                    // the operands this stage will hold next: into L2 now (the same segment's
+                    // heads only), so their loads are L2 hits
+                    if (j + nst < sg.nh) {
+                        tma_prefetch_l2_4d(offd ? &tm_x2 : &tm_x, 0, h + nst, (int)sg.t0,
+                                           (int)sg.b);
+                        bulk_prefetch_l2(hblk + (int64_t)(h + nst) * (kP * kN), kP * kN * 2);
+                    }
+                    // the gate rows this tile's epilogue will read: into L2 now
+                    if (kGate)
+                        tma_prefetch_l2_4d(&tm_z, 0, h, (int)(sg.t0 + kTileRows * T), (int)sg.b);
+                }
+                ++si;
             }
-            // the gate rows this tile's epilogue will read: into L2 now, a few heads ahead
-            if (kGate) tma_prefetch_l2_4d(&tm_z, 0, h, (int)(t0 + kTileRows * T), (int)b);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (lane 0 alone runs the loop: a lane that issued
@@ -542,10 +621,18 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         // issuing thread's own instruction chain sets the MMA issue rate)
         const uint64_t cd = smem_desc_sw128(smem_u32(&sm.Cs[0][0]), 16, 1024);
         const uint64_t rd = smem_desc_sw128(smem_u32(sm.R), 16, 1024);
-        bool ok = lane == 0 && mbar_wait(&sm.bar_cb, 0, abort);
-        if (ok) {
+        bool ok = lane == 0;
+        uint32_t J = 0;
+        int si = 0;
+        for (int64_t f = wk.f0; ok && f < wk.f1;) {
+            const Seg sg = segment(f);
+            f += sg.nh;
+            if (sg.skip) continue;
+            if (!mbar_wait(&sm.bar_cb, si & 1, abort)) break;
             tc_fence_after();
-            // G = C B^T: M = 128 rows t, N = KI columns i, K = 128 (n)
+            // G = C B^T: M = 128 rows t, N = KI columns i, K = 128 (n).  It overwrites the P
+            // ring and C B_off^T of the previous segment only after this thread's earlier MMAs,
+            // which read them, were issued (in order).
 #pragma unroll
             for (int kk = 0; kk < kN / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
@@ -553,253 +640,297 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 mma_bf16(tmem, cd + (off >> 4), rd + (boff >> 4), id_g, kk > 0 ? 1u : 0u);
             }
             mma_commit(&sm.bar_g);
-        }
-        if (ok && offd) ok = mbar_wait(&sm.bar_goff, 0, abort);   // bf16 C B_off^T in smem
-        for (int j = 0; ok && j < nh; ++j) {
-            const int xs = j % nst;
-            const uint32_t xu = j / nst;
-            const int a = j & 1;
-            if (!mbar_wait(&sm.bar_xh_full[xs], xu & 1, abort)) break;
-            if (offd && !mbar_wait(&sm.bar_xv_ready[xs], xu & 1, abort)) break;
-            if (j >= 2 && !mbar_wait(&sm.bar_acc_free[a], ((j >> 1) - 1) & 1, abort)) break;
-            tc_fence_after();
-            const uint32_t stg = smem_u32(scan_stage(sm, xs, offd));
-            const uint32_t dD = tmem + kAccCol + 128 * a, dA = dD + 64;
-            const uint64_t xd = smem_desc_sw128(stg, 256 * kRowBytes, 1024);   // x, MN-major
-            const uint64_t hd = smem_desc_sw128(stg + scan_hoff(offd), 16, 1024);  // h_in, K-major
-            if (offd) {
-                // Y_A = (C B_off^T) (v dt o X_off): A = bf16 block in R, K = 128 (i)
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    mma_bf16(dA, rd + (aoff >> 4), xd + kk * 128, id_kmn, kk > 0 ? 1u : 0u);
+            if (offd && !mbar_wait(&sm.bar_goff, si & 1, abort)) break;   // bf16 C B_off^T
+            for (int j = 0; ok && j < sg.nh; ++j, ++J) {
+                const int xs = J % nst;
+                const uint32_t xu = J / nst;
+                const int a = J & 1;
+                if (!mbar_wait(&sm.bar_xh_full[xs], xu & 1, abort)) { ok = false; break; }
+                if (offd && !mbar_wait(&sm.bar_xv_ready[xs], xu & 1, abort)) { ok = false; break; }
+                if (J >= 2 && !mbar_wait(&sm.bar_acc_free[a], ((J >> 1) - 1) & 1, abort)) {
+                    ok = false;
+                    break;
                 }
-            }
-            // Y_A (+)= C h^T: K = 128 (n), h K-major (rows p, two halves of 64 n); h = h_in
-            // (T = 0) or exp(cs_127) h_in (T = 1)
-#pragma unroll
-            for (int kk = 0; kk < kN / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                const uint32_t hoff = (kk >> 2) * (kP * kRowBytes) + (kk & 3) * 32;
-                mma_bf16(dA, cd + (off >> 4), hd + (hoff >> 4), id_kk, (offd || kk > 0) ? 1u : 0u);
-            }
-            for (int qb = 0; qb < 2; ++qb) {
-                const uint32_t blk = 2 * j + qb;           // P blocks are numbered per head
-                const uint32_t slot = blk % kRing, su = blk / kRing;
-                if (!mbar_wait(&sm.bar_slot_full[slot], su & 1, abort)) { ok = false; break; }
                 tc_fence_after();
-                // Y_diag += P[:, 64qb : +64] X[xdiag + 64qb : +64, :], P read from TMEM
-                const uint32_t pa = tmem + pcol + 32 * slot;
-                const uint64_t bd = xd + (uint64_t)((xdiag / 16 + qb * 4) * 128);
+                const uint32_t stg = smem_u32(scan_stage(sm, xs, offd));
+                const uint32_t dD = tmem + kAccCol + 128 * a, dA = dD + 64;
+                const uint64_t xd = smem_desc_sw128(stg, 256 * kRowBytes, 1024);   // x, MN-major
+                const uint64_t hd = smem_desc_sw128(stg + scan_hoff(offd), 16, 1024);  // h_in
+                if (offd) {
+                    // Y_A = (C B_off^T) (v dt o X_off): A = bf16 block in R, K = 128 (i)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ts(dD, pa + 8 * kk, bd + kk * 128, id_kmn, (qb | kk) != 0 ? 1u : 0u);
-                mma_commit(&sm.bar_slot_free[slot]);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t aoff = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                        mma_bf16(dA, rd + (aoff >> 4), xd + kk * 128, id_kmn, kk > 0 ? 1u : 0u);
+                    }
+                }
+                // Y_A (+)= C h^T: K = 128 (n), h K-major (rows p, two halves of 64 n);
+                // h = h_in (T = 0) or exp(cs_127) h_in (T = 1)
+#pragma unroll
+                for (int kk = 0; kk < kN / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                    const uint32_t hoff = (kk >> 2) * (kP * kRowBytes) + (kk & 3) * 32;
+                    mma_bf16(dA, cd + (off >> 4), hd + (hoff >> 4), id_kk,
+                             (offd || kk > 0) ? 1u : 0u);
+                }
+                for (int qb = 0; qb < 2; ++qb) {
+                    const uint32_t blk = 2 * J + qb;           // P blocks are numbered per head
+                    const uint32_t slot = blk % kRing, su = blk / kRing;
+                    if (!mbar_wait(&sm.bar_slot_full[slot], su & 1, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    // Y_diag += P[:, 64qb : +64] X[xdiag + 64qb : +64, :], P read from TMEM
+                    const uint32_t pa = tmem + pcol + 32 * slot;
+                    const uint64_t bd = xd + (uint64_t)((xdiag / 16 + qb * 4) * 128);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(dD, pa + 8 * kk, bd + kk * 128, id_kmn,
+                                    (qb | kk) != 0 ? 1u : 0u);
+                    mma_commit(&sm.bar_slot_free[slot]);
+                }
+                if (!ok) break;
+                mma_commit(&sm.bar_acc_full[a]);
+                mma_commit(&sm.bar_xh_free[xs]);
             }
             if (!ok) break;
-            mma_commit(&sm.bar_acc_full[a]);
-            mma_commit(&sm.bar_xh_free[xs]);
+            mma_commit(&sm.bar_seg_done);   // this segment's MMAs are done with C and R
+            ++si;
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 2) {
         // ---------------- workers, four per TMEM lane quarter.  Warp (qd, cq) owns rows
         // t = 32 qd + lane of the tile and the 16-column slice [16 cq, 16 cq + 16) of every
         // 64-column block: per head it builds that slice of both P blocks (mask; for T = 1 after
         // its share of scaling x_off and h_in), then the epilogue y = Y_diag + f_t Y_A of the
         // previous head for output columns [16 cq, 16 cq + 16).
-        const int wt = threadIdx.x - 128;          // 0 .. kScanWorkers - 1
+        const int wt = threadIdx.x - 64;           // 0 .. kScanWorkers - 1
         const int qd = warp & 3;
-        const int cq = (warp - 4) >> 2;
+        const int cq = (warp - 2) >> 2;
         const int t = qd * 32 + lane;             // row within the tile = TMEM lane
         const int tau = kTileRows * T + t;        // row within the chunk
         const int r = kTileRows * T + qd * 32 - 1;  // last row above this warp's 32-row slice
         const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
-        float *vt = sm.vt[warp - 4];
+        float *vt = sm.vt[warp - 2];
         // The slice of block qb is the 16-column unit u = 4 qb + cq of the diagonal block; its
         // class relative to this row quarter: 0 below the 32 x 32 diagonal sub-block, 1 inside
         // it, 2 above it (all zero).
         const int u0 = cq, u1 = 4 + cq;
         const int cls0 = u0 < 2 * qd ? 0 : (u0 <= 2 * qd + 1 ? 1 : 2);
         const int cls1 = u1 < 2 * qd ? 0 : (u1 <= 2 * qd + 1 ? 1 : 2);
-        bool ok = warp_wait(&sm.bar_g, 0, abort);
-        tc_fence_after();
-        // this warp's part of the diagonal block of C B^T, kept in registers for every head
-        uint32_t g0[16], g1[16];
+        bool ok = true;
+        uint32_t J = 0;
+        int si = 0;
+        for (int64_t f = wk.f0; ok && f < wk.f1;) {
+            const Seg sg = segment(f);
+            f += sg.nh;
+            if (sg.skip) continue;
+            ok = warp_wait(&sm.bar_g, si & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+            // this warp's part of the diagonal block of C B^T, kept in registers for every head
+            // of the segment
+            uint32_t g0[16], g1[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) g0[c] = g1[c] = 0u;
-        if (ok) {
+            for (int c = 0; c < 16; ++c) g0[c] = g1[c] = 0u;
             if (cls0 < 2) tmem_ld16(lane_base + gdiag + 16 * u0, g0);
             if (cls1 < 2) tmem_ld16(lane_base + gdiag + 16 * u1, g1);
             tmem_ld_wait();
-        }
-        if (ok && offd) {
-            // C B_off^T (TMEM columns [0, 128)) -> bf16, K-major swizzled tile in R; this warp
-            // converts its 32 rows x columns [32 cq, 32 cq + 32)
-            uint32_t gv[32];
-            tmem_ld32(lane_base + 32 * cq, gv);
-            tmem_ld_wait();
-            uint8_t *dst = sm.R + (cq >> 1) * kBoxBytes + t * kRowBytes;
+            if (offd) {
+                // C B_off^T (TMEM columns [0, 128)) -> bf16, K-major swizzled tile in R; this
+                // warp converts its 32 rows x columns [32 cq, 32 cq + 32)
+                uint32_t gv[32];
+                tmem_ld32(lane_base + 32 * cq, gv);
+                tmem_ld_wait();
+                uint8_t *dst = sm.R + (cq >> 1) * kBoxBytes + t * kRowBytes;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int pos = ((cq & 1) * 4 + m) ^ (t & 7);
-                *reinterpret_cast<uint4 *>(dst + pos * 16) = make_uint4(
-                    pack_bf16x2(__uint_as_float(gv[8 * m]), __uint_as_float(gv[8 * m + 1])),
-                    pack_bf16x2(__uint_as_float(gv[8 * m + 2]), __uint_as_float(gv[8 * m + 3])),
-                    pack_bf16x2(__uint_as_float(gv[8 * m + 4]), __uint_as_float(gv[8 * m + 5])),
-                    pack_bf16x2(__uint_as_float(gv[8 * m + 6]), __uint_as_float(gv[8 * m + 7])));
+                for (int m = 0; m < 4; ++m) {
+                    const int pos = ((cq & 1) * 4 + m) ^ (t & 7);
+                    *reinterpret_cast<uint4 *>(dst + pos * 16) = make_uint4(
+                        pack_bf16x2(__uint_as_float(gv[8 * m]), __uint_as_float(gv[8 * m + 1])),
+                        pack_bf16x2(__uint_as_float(gv[8 * m + 2]), __uint_as_float(gv[8 * m + 3])),
+                        pack_bf16x2(__uint_as_float(gv[8 * m + 4]), __uint_as_float(gv[8 * m + 5])),
+                        pack_bf16x2(__uint_as_float(gv[8 * m + 6]), __uint_as_float(gv[8 * m + 7])));
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(&sm.bar_goff);
+                // the P ring reuses these TMEM columns: wait until every warp has read them
+                ok = warp_wait(&sm.bar_goff, si & 1, abort);
+                if (!ok) break;
+                tc_fence_after();
             }
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(&sm.bar_goff);
-            // the P ring reuses these TMEM columns: wait until every warp has read them
-            ok = warp_wait(&sm.bar_goff, 0, abort);
-            tc_fence_after();
-        }
-        uint32_t blk = 0;
-        for (int j = 0; ok && j <= nh; ++j) {
-            if (j < nh) {
-                const int vs = j % kScanVecStages;
-                if (!warp_wait(&sm.bar_vec_full[vs], (j / kScanVecStages) & 1, abort)) break;
-                const float *cs_s = sm.cs_v[vs];
-                const float *dt_s = sm.dt_v[vs];
-                if (offd) {
-                    // x rows [0, 128) *= exp(cs_127 - cs_i) dt_i; h_in *= exp(cs_127)
-                    const int xs = j % nst;
-                    if (!warp_wait(&sm.bar_xh_full[xs], (j / nst) & 1, abort)) break;
-                    uint8_t *stg = scan_stage(sm, xs, offd);
-                    const float c127 = cs_s[127];
-                    scale_pieces<1024 / kScanWorkers>(stg, wt, kScanWorkers, [&](int c) {
-                        const int i = c >> 3;
-                        return __expf(c127 - cs_s[i]) * dt_s[i];
-                    });
-                    const float sh = __expf(c127);
-                    scale_pieces<1024 / kScanWorkers>(stg + scan_hoff(offd), wt, kScanWorkers,
-                                                      [&](int) { return sh; });
-                    fence_async_smem();
-                    mbar_arrive(&sm.bar_xv_ready[xs]);
-                }
-                const float Dh = sm.Dv[j];
-                const float ct = cs_s[tau];
-                // Row and column factors: below the 32 x 32 diagonal sub-block relative to row r,
-                // both <= 1; inside it relative to m = r + 1, the slice's first row:
-                // exp(cs_m - cs_i) <= exp(32 max|dt A|) and exp(cs_t - cs_m) <= 1, so neither
-                // over- nor underflows, and no element needs an exponential of its own.
-                const float cm = cs_s[r + 1];
-                const float crf = cs_s[r < 0 ? 0 : r];
-                const float um = __expf(ct - cm);
-                const float uf = qd > 0 ? __expf(ct - crf) : 0.f;
-                {
-                    // lane l: column 16 (4 (l >> 4) + cq) + (l & 15) of the diagonal block
-                    const int uu = 4 * (lane >> 4) + cq;
-                    const int cl = uu < 2 * qd ? 0 : (uu <= 2 * qd + 1 ? 1 : 2);
-                    const int i = kTileRows * T + 16 * uu + (lane & 15);
-                    const float ref = cl == 0 ? crf : cm;
-                    const float v = __expf(ref - cs_s[i]) * dt_s[i];
-                    vt[lane] = cl < 2 ? v : 0.f;
-                }
-                __syncwarp();
-#pragma unroll
-                for (int qb = 0; qb < 2; ++qb, ++blk) {
-                    const uint32_t slot = blk % kRing, su = blk / kRing;
-                    const int cl = qb ? cls1 : cls0;
-                    const uint32_t *gv = qb ? g1 : g0;
-                    const float *vq = vt + 16 * qb;
-                    uint32_t pk[8];
-                    if (cl == 0) {
-                        const float2 uu = make_float2(uf, uf);
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const float4 vv = *reinterpret_cast<const float4 *>(vq + 4 * c);
-                            const float2 p0 = fmul2(
-                                fmul2(make_float2(__uint_as_float(gv[4 * c]),
-                                                  __uint_as_float(gv[4 * c + 1])),
-                                      make_float2(vv.x, vv.y)), uu);
-                            const float2 p1 = fmul2(
-                                fmul2(make_float2(__uint_as_float(gv[4 * c + 2]),
-                                                  __uint_as_float(gv[4 * c + 3])),
-                                      make_float2(vv.z, vv.w)), uu);
-                            pk[2 * c] = pack_bf16x2(p0.x, p0.y);
-                            pk[2 * c + 1] = pack_bf16x2(p1.x, p1.y);
-                        }
-                    } else if (cl == 1) {
-                        // inside the causal 32 x 32 sub-block: local column lc kept for
-                        // lc <= lane, + D at lc = lane
-                        const int lc0 = 16 * (qb ? u1 : u0) - 32 * qd;   // 0 or 16
-                        const float2 uu = make_float2(um, um);
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const float2 ww = *reinterpret_cast<const float2 *>(vq + 2 * c);
-                            float2 pp = fmul2(fmul2(make_float2(__uint_as_float(gv[2 * c]),
-                                                                __uint_as_float(gv[2 * c + 1])),
-                                                    ww), uu);
-                            const int lc = lc0 + 2 * c;
-                            pp.x = (lc <= lane) ? pp.x : 0.f;
-                            pp.y = (lc + 1 <= lane) ? pp.y : 0.f;
-                            pp.x += (lc == lane) ? Dh : 0.f;
-                            pp.y += (lc + 1 == lane) ? Dh : 0.f;
-                            pk[c] = pack_bf16x2(pp.x, pp.y);
-                        }
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) pk[c] = 0u;
-                    }
-                    if (su >= 1 && !warp_wait(&sm.bar_slot_free[slot], (su - 1) & 1, abort)) {
+            const uint32_t J0 = J;   // first head of the segment
+            const int snh = sg.nh;
+            const float *Dseg = D + sg.h0;
+            const bool row_in = tau < sg.len;   // this thread's row exists in the chunk
+            // output row tau of the segment's first head, this warp's 16 columns
+            bf16 *yseg = y + ((sg.b * seqlen + sg.t0 + tau) * H + sg.h0) * (int64_t)kP + 16 * cq;
+            const bf16 *zseg = kGate ? z + (yseg - y) : nullptr;
+            for (int j = 0; ok && j <= snh; ++j) {
+                if (j < snh) {
+                    const uint32_t Jj = J0 + j;
+                    const int vs = Jj % kScanVecStages;
+                    if (!warp_wait(&sm.bar_vec_full[vs], (Jj / kScanVecStages) & 1, abort)) {
                         ok = false;
                         break;
                     }
-                    tmem_st8(lane_base + pcol + 32 * slot + 8 * cq, pk);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(&sm.bar_slot_full[slot]);
-                }
-                if (!ok) break;
-            }
-            if (j >= 1) {
-                // epilogue of head jj = j - 1 for output columns [16 cq, 16 cq + 16)
-                const int jj = j - 1;
-                const int a = jj & 1;
-                if (!warp_wait(&sm.bar_acc_full[a], (jj >> 1) & 1, abort)) break;
-                tc_fence_after();
-                const uint32_t col = lane_base + kAccCol + 128 * a + 16 * cq;
-                uint32_t d0[16], a0[16];
-                tmem_ld16(col, d0);
-                tmem_ld16(col + 64, a0);
-                const int vs = jj % kScanVecStages;
-                const float *cs_j = sm.cs_v[vs];
-                const float f = __expf(cs_j[tau] - (T ? cs_j[127] : 0.f));
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(&sm.bar_acc_free[a]);
-                mbar_arrive(&sm.bar_vec_free[vs]);   // done with this head's cs / dt
-                const int64_t yoff = ((b * seqlen + t0 + tau) * H + h0 + jj) * (int64_t)kP + 16 * cq;
-                // gated output (z given): y * z * sigmoid(z); z kept as 8 packed bf16 pairs
-                const bool gz = kGate && tau < len;
-                uint4 z0 = make_uint4(0u, 0u, 0u, 0u), z1 = z0;
-                if (gz) {
-                    const uint4 *zrow = reinterpret_cast<const uint4 *>(z + yoff);
-                    z0 = zrow[0];
-                    z1 = zrow[1];
-                }
-                const uint32_t zw[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-                uint32_t pk[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float v0 = fmaf(f, __uint_as_float(a0[2 * c]), __uint_as_float(d0[2 * c]));
-                    float v1 =
-                        fmaf(f, __uint_as_float(a0[2 * c + 1]), __uint_as_float(d0[2 * c + 1]));
-                    if (gz) {
-                        const float2 zf = __bfloat1622float2(
-                            *reinterpret_cast<const __nv_bfloat162 *>(&zw[c]));
-                        v0 *= silu(zf.x);
-                        v1 *= silu(zf.y);
+                    const float *cs_s = sm.cs_v[vs];
+                    const float *dt_s = sm.dt_v[vs];
+                    if (offd) {
+                        // x rows [0, 128) *= exp(cs_127 - cs_i) dt_i; h_in *= exp(cs_127)
+                        const int xs = Jj % nst;
+                        if (!warp_wait(&sm.bar_xh_full[xs], (Jj / nst) & 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *stg = scan_stage(sm, xs, offd);
+                        const float c127 = cs_s[127];
+                        scale_pieces<1024 / kScanWorkers>(stg, wt, kScanWorkers, [&](int c) {
+                            const int i = c >> 3;
+                            return __expf(c127 - cs_s[i]) * dt_s[i];
+                        });
+                        const float sh = __expf(c127);
+                        scale_pieces<1024 / kScanWorkers>(stg + scan_hoff(offd), wt, kScanWorkers,
+                                                          [&](int) { return sh; });
+                        fence_async_smem();
+                        mbar_arrive(&sm.bar_xv_ready[xs]);
                     }
-                    pk[c] = pack_bf16x2(v0, v1);
+                    const float Dh = Dseg[j];
+                    const float ct = cs_s[tau];
+                    // Row and column factors: below the 32 x 32 diagonal sub-block relative to
+                    // row r, both <= 1; inside it relative to m = r + 1, the slice's first row:
+                    // exp(cs_m - cs_i) <= exp(32 max|dt A|) and exp(cs_t - cs_m) <= 1, so
+                    // neither over- nor underflows, and no element needs an exponential of its
+                    // own.
+                    const float cm = cs_s[r + 1];
+                    const float crf = cs_s[r < 0 ? 0 : r];
+                    const float um = __expf(ct - cm);
+                    const float uf = qd > 0 ? __expf(ct - crf) : 0.f;
+                    {
+                        // lane l: column 16 (4 (l >> 4) + cq) + (l & 15) of the diagonal block
+                        const int uu = 4 * (lane >> 4) + cq;
+                        const int cl = uu < 2 * qd ? 0 : (uu <= 2 * qd + 1 ? 1 : 2);
+                        const int i = kTileRows * T + 16 * uu + (lane & 15);
+                        const float ref = cl == 0 ? crf : cm;
+                        const float v = __expf(ref - cs_s[i]) * dt_s[i];
+                        vt[lane] = cl < 2 ? v : 0.f;
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int qb = 0; qb < 2; ++qb) {
+                        const uint32_t blk = 2 * Jj + qb;
+                        const uint32_t slot = blk % kRing, su = blk / kRing;
+                        const int cl = qb ? cls1 : cls0;
+                        const uint32_t *gv = qb ? g1 : g0;
+                        const float *vq = vt + 16 * qb;
+                        uint32_t pk[8];
+                        if (cl == 0) {
+                            const float2 uu = make_float2(uf, uf);
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const float4 vv = *reinterpret_cast<const float4 *>(vq + 4 * c);
+                                const float2 p0 = fmul2(
+                                    fmul2(make_float2(__uint_as_float(gv[4 * c]),
+                                                      __uint_as_float(gv[4 * c + 1])),
+                                          make_float2(vv.x, vv.y)), uu);
+                                const float2 p1 = fmul2(
+                                    fmul2(make_float2(__uint_as_float(gv[4 * c + 2]),
+                                                      __uint_as_float(gv[4 * c + 3])),
+                                          make_float2(vv.z, vv.w)), uu);
+                                pk[2 * c] = pack_bf16x2(p0.x, p0.y);
+                                pk[2 * c + 1] = pack_bf16x2(p1.x, p1.y);
+                            }
+                        } else if (cl == 1) {
+                            // inside the causal 32 x 32 sub-block: local column lc kept for
+                            // lc <= lane, + D at lc = lane
+                            const int lc0 = 16 * (qb ? u1 : u0) - 32 * qd;   // 0 or 16
+                            const float2 uu = make_float2(um, um);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const float2 ww = *reinterpret_cast<const float2 *>(vq + 2 * c);
+                                float2 pp = fmul2(fmul2(make_float2(__uint_as_float(gv[2 * c]),
+                                                                    __uint_as_float(gv[2 * c + 1])),
+                                                        ww), uu);
+                                const int lc = lc0 + 2 * c;
+                                pp.x = (lc <= lane) ? pp.x : 0.f;
+                                pp.y = (lc + 1 <= lane) ? pp.y : 0.f;
+                                pp.x += (lc == lane) ? Dh : 0.f;
+                                pp.y += (lc + 1 == lane) ? Dh : 0.f;
+                                pk[c] = pack_bf16x2(pp.x, pp.y);
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) pk[c] = 0u;
+                        }
+                        if (su >= 1 &&
+                            !warp_wait(&sm.bar_slot_free[slot], (su - 1) & 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        // a slice above the diagonal is all zero; a slot always holds the same
+                        // block qb and so the same slices, so once its zeros are written (by
+                        // the segment's first two heads: C B^T of a tile with an off-diagonal
+                        // block overwrites the ring at every segment) they stay
+                        if (cl != 2 || j < 2) {
+                            tmem_st8(lane_base + pcol + 32 * slot + 8 * cq, pk);
+                            tmem_st_wait();
+                        }
+                        tc_fence_before();
+                        mbar_arrive(&sm.bar_slot_full[slot]);
+                    }
+                    if (!ok) break;
                 }
-                if (tau < len) {
-                    uint4 *yrow = reinterpret_cast<uint4 *>(y + yoff);
-                    yrow[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    yrow[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                if (j >= 1) {
+                    // epilogue of head jj = j - 1 for output columns [16 cq, 16 cq + 16)
+                    const uint32_t Jj = J0 + j - 1;
+                    const int a = Jj & 1;
+                    if (!warp_wait(&sm.bar_acc_full[a], (Jj >> 1) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t col = lane_base + kAccCol + 128 * a + 16 * cq;
+                    uint32_t d0[16], a0[16];
+                    tmem_ld16(col, d0);
+                    tmem_ld16(col + 64, a0);
+                    const int vs = Jj % kScanVecStages;
+                    const float *cs_j = sm.cs_v[vs];
+                    const float fct = __expf(cs_j[tau] - (T ? cs_j[127] : 0.f));
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    mbar_arrive(&sm.bar_acc_free[a]);
+                    mbar_arrive(&sm.bar_vec_free[vs]);   // done with this head's cs / dt
+                    const int64_t yoff = (int64_t)(j - 1) * kP;
+                    // gated output (z given): y * z * sigmoid(z); z kept as 8 packed bf16 pairs
+                    const bool gz = kGate && row_in;
+                    uint4 z0 = make_uint4(0u, 0u, 0u, 0u), z1 = z0;
+                    if (gz) {
+                        const uint4 *zrow = reinterpret_cast<const uint4 *>(zseg + yoff);
+                        z0 = zrow[0];
+                        z1 = zrow[1];
+                    }
+                    const uint32_t zw[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        float v0 = fmaf(fct, __uint_as_float(a0[2 * c]), __uint_as_float(d0[2 * c]));
+                        float v1 = fmaf(fct, __uint_as_float(a0[2 * c + 1]),
+                                        __uint_as_float(d0[2 * c + 1]));
+                        if (gz) {
+                            const float2 zf = __bfloat1622float2(
+                                *reinterpret_cast<const __nv_bfloat162 *>(&zw[c]));
+                            v0 *= silu(zf.x);
+                            v1 *= silu(zf.y);
+                        }
+                        pk[c] = pack_bf16x2(v0, v1);
+                    }
+                    if (row_in) {
+                        uint4 *yrow = reinterpret_cast<uint4 *>(yseg + yoff);
+                        yrow[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        yrow[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    }
                 }
             }
+            J = J0 + snh;
+            ++si;
         }
     }
     __syncthreads();
@@ -815,11 +946,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kScanTmemCols);
     }
 }
+#undef segment
 
 // ============================================================ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
@@ -861,24 +993,6 @@ bool make_seq_map(CUtensorMap *m, const void *ptr, int64_t batch, int64_t seqlen
                                    (cuuint64_t)(seqlen * mid * inner * 2)};
     const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     return make_map(m, ptr, 4, dims, strides, box);
-}
-
-// Heads per chunk-scan CTA.  Each CTA pays a ramp (C and B tiles, C B^T, the first loads) that
-// more heads amortise, but the two 128-row tiles of a chunk differ in cost and a CTA walks its
-// heads in sequence, so too few CTAs leave the last wave ragged.  Aim at about 3.5 waves of CTAs
-// over the SMs, within [kScanHeadsMin, kScanHeadsMax], then balance the head blocks (measured at
-// b=4, L=4096, H=80: 8 heads 207 us, 14 heads 195 us, 20 heads 195 us, 40 heads 210 us).
-int scan_heads_per_cta(int64_t tiles, int hpg)
-{
-    int sms = 148, dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const double target_ctas = 3.5 * sms;
-    int hpc = (int)std::ceil((double)hpg * (double)tiles / target_ctas);
-    hpc = std::max(kScanHeadsMin, std::min(kScanHeadsMax, hpc));
-    hpc = std::min(hpc, hpg);
-    const int nhb = (hpg + hpc - 1) / hpc;
-    return (hpg + nhb - 1) / nhb;   // the same number of head blocks, evenly filled
 }
 
 }  // namespace
@@ -937,20 +1051,28 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
         *why = "chunk scan: cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
-    const int hpg = H / G;
-    // The scan's per-head cost (mask, three MMA chains, epilogue) dominates its per-CTA ramp, and
-    // its two tiles differ in cost, so many small CTAs balance better than one CTA per group.
-    const int hpc = scan_heads_per_cta(batch * nchunks * G * (Q / kTileRows), hpg);
-    const int nhb = (hpg + hpc - 1) / hpc;
+    const int64_t nitems = batch * nchunks * H;   // (batch, chunk, group, head) items per class
+    if (nitems == 0) return cudaSuccess;
+    const int nT = Q / kTileRows;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = (int)std::min<int64_t>(sms, nT * nitems);
+    // SMs for the second-tile class (off-diagonal block, 24 MMAs and two scaling passes per
+    // head against 16 MMAs for the first tile): in proportion to kOffdCost : 1
+    int ncta1 = 0;
+    if (nT == 2) {
+        ncta1 = (int)std::lround(grid * kOffdCost / (1.0 + kOffdCost));
+        ncta1 = std::max(1, std::min(grid - 1, ncta1));
+    }
     const size_t smem = sizeof(ScanSmem) + 1024;
     auto kern = z ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk scan: set smem attribute"; return e; }
-    const unsigned grid = (unsigned)(batch * nchunks * G * nhb * (Q / kTileRows));
     *why = "chunk scan (tcgen05) launch";
-    return launch_pdl(kern, grid, kScanThreads, smem, st, mx, mb, mc, mx2, mz, hin, dtc, cs, D, y,
-                      status, seqlen, H, G, Q, nchunks, nhb, hpc, tab, z,
+    return launch_pdl(kern, (unsigned)grid, kScanThreads, smem, st, mx, mb, mc, mx2, mz, hin,
+                      dtc, cs, D, y, status, seqlen, H, G, Q, nchunks, nitems, ncta1, tab, z,
                       take_test_skip(kTestChunkScan));
 }
 
