@@ -356,7 +356,8 @@ struct alignas(1024) ScanSmem {
 // lane quarter, each owning a 16-column slice of every 64-column block; per head they build
 // their slice of P (mask) and then run the epilogue of the previous head for their slice of y
 constexpr int kScanWorkers = 512;
-constexpr int kScanThreads = 64 + kScanWorkers;   // 576 threads: up to 112 registers each
+constexpr int kScanThreads = 64 + kScanWorkers;   // 576 threads (five warps on some SMSPs: 96
+                                                  // registers each)
 constexpr uint32_t kScanTmemCols = 512;
 constexpr uint32_t kAccCol = 256;   // accumulator buffer a: Y_diag at 256 + 128 a, Y_A at +64
 
@@ -455,7 +456,7 @@ __device__ __forceinline__ Seg scan_segment(int64_t f, int64_t f1, int hpg, int 
 }
 
 template <bool kGate>   // kGate: the output is y * z * sigmoid(z)
-__global__ void __maxnreg__(112)   // one CTA of kScanThreads per SM: 65536 / 576 registers
+__global__ void __launch_bounds__(kScanThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c,
@@ -725,14 +726,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             ok = warp_wait(&sm.bar_g, si & 1, abort);
             if (!ok) break;
             tc_fence_after();
-            // this warp's part of the diagonal block of C B^T, kept in registers for every head
-            // of the segment
-            uint32_t g0[16], g1[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) g0[c] = g1[c] = 0u;
-            if (cls0 < 2) tmem_ld16(lane_base + gdiag + 16 * u0, g0);
-            if (cls1 < 2) tmem_ld16(lane_base + gdiag + 16 * u1, g1);
-            tmem_ld_wait();
             if (offd) {
                 // C B_off^T (TMEM columns [0, 128)) -> bf16, K-major swizzled tile in R; this
                 // warp converts its 32 rows x columns [32 cq, 32 cq + 32)
@@ -759,11 +752,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             }
             const uint32_t J0 = J;   // first head of the segment
             const int snh = sg.nh;
-            const float *Dseg = D + sg.h0;
+            const int sh0 = sg.h0;
             const bool row_in = tau < sg.len;   // this thread's row exists in the chunk
             // output row tau of the segment's first head, this warp's 16 columns
-            bf16 *yseg = y + ((sg.b * seqlen + sg.t0 + tau) * H + sg.h0) * (int64_t)kP + 16 * cq;
-            const bf16 *zseg = kGate ? z + (yseg - y) : nullptr;
+            const int64_t yseg = ((sg.b * seqlen + sg.t0 + tau) * H + sh0) * (int64_t)kP + 16 * cq;
             for (int j = 0; ok && j <= snh; ++j) {
                 if (j < snh) {
                     const uint32_t Jj = J0 + j;
@@ -774,6 +766,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     }
                     const float *cs_s = sm.cs_v[vs];
                     const float *dt_s = sm.dt_v[vs];
+                    // this warp's part of the diagonal block of C B^T: it stays in TMEM for the
+                    // whole segment (the P ring and the accumulators use other columns), so it
+                    // is read again per head instead of held in registers
+                    uint32_t g0[16], g1[16];
+                    if (cls0 < 2) tmem_ld16(lane_base + gdiag + 16 * u0, g0);
+                    if (cls1 < 2) tmem_ld16(lane_base + gdiag + 16 * u1, g1);
                     if (offd) {
                         // x rows [0, 128) *= exp(cs_127 - cs_i) dt_i; h_in *= exp(cs_127)
                         const int xs = Jj % nst;
@@ -793,7 +791,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                         fence_async_smem();
                         mbar_arrive(&sm.bar_xv_ready[xs]);
                     }
-                    const float Dh = Dseg[j];
+                    const float Dh = D[sh0 + j];
                     const float ct = cs_s[tau];
                     // Row and column factors: below the 32 x 32 diagonal sub-block relative to
                     // row r, both <= 1; inside it relative to m = r + 1, the slice's first row:
@@ -814,6 +812,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                         vt[lane] = cl < 2 ? v : 0.f;
                     }
                     __syncwarp();
+                    tmem_ld_wait();
 #pragma unroll
                     for (int qb = 0; qb < 2; ++qb) {
                         const uint32_t blk = 2 * Jj + qb;
@@ -898,12 +897,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     tc_fence_before();
                     mbar_arrive(&sm.bar_acc_free[a]);
                     mbar_arrive(&sm.bar_vec_free[vs]);   // done with this head's cs / dt
-                    const int64_t yoff = (int64_t)(j - 1) * kP;
+                    const int64_t yoff = yseg + (int64_t)(j - 1) * kP;
                     // gated output (z given): y * z * sigmoid(z); z kept as 8 packed bf16 pairs
                     const bool gz = kGate && row_in;
                     uint4 z0 = make_uint4(0u, 0u, 0u, 0u), z1 = z0;
                     if (gz) {
-                        const uint4 *zrow = reinterpret_cast<const uint4 *>(zseg + yoff);
+                        const uint4 *zrow = reinterpret_cast<const uint4 *>(z + yoff);
                         z0 = zrow[0];
                         z1 = zrow[1];
                     }
@@ -923,7 +922,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                         pk[c] = pack_bf16x2(v0, v1);
                     }
                     if (row_in) {
-                        uint4 *yrow = reinterpret_cast<uint4 *>(yseg + yoff);
+                        uint4 *yrow = reinterpret_cast<uint4 *>(y + yoff);
                         yrow[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         yrow[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     }
