@@ -328,7 +328,6 @@ constexpr int kXStagesMax = 5;   // x / h_in stages: tiles without an off-diagon
                                  // of 32 KB (three in S01, two in the B tile's space once C B^T
                                  // is done); the second tile of a chunk with one uses 2 of 48 KB
                                  // (S01; the B tile's space then holds the bf16 block)
-constexpr double kOffdCost = 1.35; // cost of a second-tile head relative to a first-tile head
 constexpr int kScanVecStages = 6; // cs / dt row stages (one head each)
 constexpr int kRing = 4;         // 64-column blocks of P in TMEM (two heads)
 constexpr int kStageBytes = 256 * kRowBytes + 2 * kP * kRowBytes;  // 48 KB: 256 x rows + h_in
@@ -401,11 +400,14 @@ __device__ __forceinline__ void scale_pieces(uint8_t *base, int first, int strid
 // Work of one launch: for each 128-row tile class T of the chunks (T = 1, the tiles with an
 // off-diagonal block, exists for Q = 256), the flat list of (batch, chunk, group, head) items,
 // heads of a group consecutive.  One CTA per SM: CTAs [0, ncta1) take the T = 1 items, the rest
-// the T = 0 items, each an equal run of its class's list (the host splits the SMs between the
-// classes in proportion to their cost).  A run of items of the same (batch, chunk, group) is a
-// segment: its heads share the C and B tiles and C B^T, which the CTA computes once per
-// segment; the per-head pipeline runs on across segments, its barrier phases counted by a
-// head counter that does not restart.
+// the T = 0 items, each an equal run of its class's list.  For Q = 256 the two classes get the
+// same number of CTAs and the same runs, so CTA i of each class walks the same heads in the same
+// order at about the same time: both tiles of a head read x rows 0-127 and the head's entering
+// state, and the second read is then an L2 hit (with the classes split unevenly it was not:
+// 415 MB of DRAM reads per launch at the 2.7B shape instead of 271 MB).  A run of items of the
+// same (batch, chunk, group) is a segment: its heads share the C and B tiles and C B^T, which
+// the CTA computes once per segment; the per-head pipeline runs on across segments, its barrier
+// phases counted by a head counter that does not restart.
 struct ScanWork {
     int T;               // tile class of this CTA
     int64_t f0, f1;      // its run of items
@@ -1056,14 +1058,10 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = (int)std::min<int64_t>(sms, nT * nitems);
-    // SMs for the second-tile class (off-diagonal block, 24 MMAs and two scaling passes per
-    // head against 16 MMAs for the first tile): in proportion to kOffdCost : 1
-    int ncta1 = 0;
-    if (nT == 2) {
-        ncta1 = (int)std::lround(grid * kOffdCost / (1.0 + kOffdCost));
-        ncta1 = std::max(1, std::min(grid - 1, ncta1));
-    }
+    // Q = 256: half the SMs per tile class, with identical runs (see scan_work)
+    const int per = (int)std::min<int64_t>(nT == 2 ? sms / 2 : sms, nitems);
+    const int grid = nT * per;
+    const int ncta1 = nT == 2 ? per : 0;
     const size_t smem = sizeof(ScanSmem) + 1024;
     auto kern = z ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
     cudaError_t e =
