@@ -176,6 +176,17 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     for (int a = 0; a < 2; ++a)   // boxes of Q rows
                         tma_load_4d(&sm.Bs[a][0], &tm_b, &sm.bar_b, 64 * a, it.g, (int)t0,
                                     (int)it.b);
+                    // the next segment's B tile into L2 now, so that its load after this
+                    // segment's last MMA is short
+                    const int64_t fn = (f0 + j) - (f0 + j) % hpg + hpg;
+                    if (fn < f1) {
+                        const StateItem nx = state_item(fn, f0, hpg, G, nchunks);
+                        int64_t nt0;
+                        int nlen;
+                        chunk_span(tab, nx.k, Q, seqlen, nt0, nlen);
+                        for (int a = 0; a < 2; ++a)
+                            tma_prefetch_l2_4d(&tm_b, 64 * a, nx.g, (int)nt0, (int)nx.b);
+                    }
                 }
                 const int s = j % kStateStages;
                 const uint32_t use = j / kStateStages;
@@ -551,6 +562,19 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     for (int r = 0; r < KI / kTileRows; ++r)
                         tma_load_4d(sm.R + a * KI * kRowBytes + r * kBoxBytes, &tm_b, &sm.bar_cb,
                                     64 * a, sg.g, (int)(sg.t0 + kTileRows * r), (int)sg.b);
+                // the next segment's C and B tiles into L2 now, so that their loads after this
+                // segment's last MMA are short
+                if (f < wk.f1) {
+                    const Seg nx = segment(f);
+                    if (!nx.skip)
+                        for (int a = 0; a < 2; ++a) {
+                            tma_prefetch_l2_4d(&tm_c, 64 * a, nx.g,
+                                               (int)(nx.t0 + kTileRows * T), (int)nx.b);
+                            for (int r = 0; r < KI / kTileRows; ++r)
+                                tma_prefetch_l2_4d(&tm_b, 64 * a, nx.g,
+                                                   (int)(nx.t0 + kTileRows * r), (int)nx.b);
+                        }
+                }
                 if (si == 0) {
                     // x is an input of the scan: start streaming the first heads' tiles into
                     // L2 while the state-passing kernel finishes
