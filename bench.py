@@ -53,14 +53,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ------------------------------------------------------------------ work model
-def fuses_cumsum(w):
-    """True where the tensor-core chunk-state kernel computes the dA cumsum itself (bf16,
-    P = 64, N = 128, Q of 128 or 256, heads a multiple of 4): the cumsum kernel then does not
-    run and its work and bytes belong to the chunk-state kernel."""
-    return (w.dtype == "bf16" and w.headdim == 64 and w.dstate == 128 and w.chunk in (128, 256)
-            and w.nheads % 4 == 0)
-
-
 def work_model(w):
     """Algorithmic bytes and flops per launch of each kernel, and for the whole step.
 
@@ -74,10 +66,7 @@ def work_model(w):
     per-chunk float32 states (written by the chunk-state kernel, read by state passing), the
     bf16 states entering each chunk (written by state passing, read by the chunk scan), and the
     chunk-local cumsum rows (written by the cumsum kernel, read by the two tensor-core kernels;
-    the dt rows it re-lays out per chunk stand in for the dt those kernels count).  Where the
-    chunk-state kernel computes the cumsum itself (fuses_cumsum), the cumsum kernel has no
-    entry and the chunk-state kernel writes those rows.  Flops count the dense Q x Q intra-chunk
-    product as the method materialises it,
+    the dt rows it re-lays out per chunk stand in for the dt those kernels count).  Flops count the dense Q x Q intra-chunk product as the method materialises it,
     plus the chunk-state and off-chunk products (2NP each per token-head) and C B^T once per
     group (2QN per token-group); "flops_causal" counts only the causal half of the Q x Q block."""
     b, L, H, P, N, G, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk
@@ -93,8 +82,7 @@ def work_model(w):
     init = fin if w.init_state else 0
     k = {
         "chunk_cumsum": {"bytes": dt, "ws_bytes": 2 * cs, "flops": 0},
-        "chunk_state": {"bytes": x + bc + dt,
-                        "ws_bytes": (2 * cs if fuses_cumsum(w) else cs) + st * 4,
+        "chunk_state": {"bytes": x + bc + dt, "ws_bytes": cs + st * 4,
                         "flops": 2 * b * L * H * P * N},
         "state_passing": {"bytes": fin + init, "ws_bytes": cs // Q + st * 4 + st * 2,
                           "flops": 0},
@@ -103,8 +91,6 @@ def work_model(w):
                        "flops_causal": b * L * H * ((Q + 1) * P + 2 * N * P)
                        + b * L * G * (Q + 1) * N},
     }
-    if fuses_cumsum(w):
-        del k["chunk_cumsum"]
     total = {"bytes": x + 2 * bc + dt + y + fin + init,
              "flops": b * L * H * (2 * Q * P + 4 * N * P) + b * L * G * 2 * Q * N,
              "flops_causal": b * L * H * ((Q + 1) * P + 4 * N * P) + b * L * G * (Q + 1) * N}
@@ -365,9 +351,6 @@ def kernel_rooflines(w, staged_ms, kern_ms, hbm, tc_peak):
     kmodel, _ = work_model(w)
     out = {}
     for name in KERNELS:
-        if name not in kmodel:   # work done inside another kernel (its stage is empty)
-            out[name] = {"ms": statistics.mean(kern_ms[name]), "fused_into": "chunk_state"}
-            continue
         ms = statistics.mean(kern_ms[name])
         m = kmodel[name]
         sec = ms / 1e3
@@ -732,8 +715,7 @@ def main():
         "fused_block": {"workload": w.name + "_gated_softplus_dt",
                         "metric": "ssd_chunk_scan_fwd_ex_tokens_per_s",
                         "value": tokens_per_step / (block_ms / 1e3), "unit": "tokens/s",
-                        "ms_per_step": block_ms, "steps": Kb,
-                        "kernels_per_step": 4 if fuses_cumsum(w) else 5,
+                        "ms_per_step": block_ms, "steps": Kb, "kernels_per_step": 5,
                         "extra_bytes_per_step": int(blk.z.size * 2 + blk.dt_raw.size * 8),
                         "l2": "256 MB buffer written before each timed call (outside the events)"},
         "varlen": {"workload": wv.name, "metric": "ssd_chunk_scan_varlen_fwd_tokens_per_s",
@@ -759,7 +741,7 @@ def main():
                              "(3 streams, 2 buffer sets)"},
         "cpu_baseline": cpu,
         "clocks": clocks,
-        "gpu_launches": (3 if fuses_cumsum(w) else 4) * K,
+        "gpu_launches": 4 * K,
         "wall_s_timed_region": wall,
         "peaks": {"hbm_gbs": hbm, "bf16_tflops": tc_peak, "source": peak_src},
     }

@@ -69,9 +69,7 @@ struct alignas(1024) StateSmem {
     bf16 Xs[kStateStages][256 * 64];      // MN-major B operand per stage: [Q rows tau][64 p]
     float cs_v[kStateStages][256];        // per stage: the head's chunk-local cumsum row
     float dt_v[kStateStages][256];        // per stage: the head's dt row (0 past the end)
-    float dtbox[kStateStages][256][4];    // kCs: per stage, dt of 4 heads (from h & ~3) by row
-    float scan_tot[2][8];                 // kCs: per head (two alternating), each scale warp's sum
-    uint64_t bar_b, bar_b_free, bar_scan;
+    uint64_t bar_b, bar_b_free;
     uint64_t bar_x_full[kStateStages], bar_x_ready[kStateStages], bar_x_free[kStateStages];
     uint64_t bar_acc_full[2], bar_acc_free[2];
     uint64_t bar_drain;
@@ -104,20 +102,12 @@ __device__ __forceinline__ StateItem state_item(int64_t f, int64_t f0, int hpg, 
     return it;
 }
 
-// kCs: the kernel also computes the chunk-local cumsum of dt A (no separate cumsum kernel):
-// per head the producer loads the dt rows of 4 heads with one TMA box, the scale warps scan
-// their head's 256 (or 128) values -- a warp scan, then the warps' totals through shared memory
-// -- write the cs and dt rows to the workspace for the later kernels (cs and dtc are then
-// outputs), and scale each its own row of x.  CTA 0 also clears the workspace status word.
-template <bool kCs>
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
-                      const __grid_constant__ CUtensorMap tm_b,
-                      const __grid_constant__ CUtensorMap tm_dt, float *__restrict__ dtc,
-                      float *__restrict__ cs, const float *__restrict__ A,
-                      float *__restrict__ states, int *__restrict__ status, int H, int G, int Q,
-                      int64_t nchunks, int64_t nitems, int64_t seqlen,
-                      const int2 *__restrict__ tab, int skip_cta)
+                      const __grid_constant__ CUtensorMap tm_b, const float *__restrict__ dtc,
+                      const float *__restrict__ cs, float *__restrict__ states,
+                      int *__restrict__ status, int H, int G, int Q, int64_t nchunks,
+                      int64_t nitems, int64_t seqlen, const int2 *__restrict__ tab, int skip_cta)
 {
     extern __shared__ uint8_t smem_raw[];
     StateSmem &sm = *reinterpret_cast<StateSmem *>(
@@ -132,7 +122,6 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_b, 1);
         mbar_init(&sm.bar_b_free, 1);
-        mbar_init(&sm.bar_scan, kStateScaleThreads);
         for (int s = 0; s < kStateStages; ++s) {
             mbar_init(&sm.bar_x_full[s], 1);
             mbar_init(&sm.bar_x_ready[s], kStateScaleThreads);
@@ -156,20 +145,13 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     if (threadIdx.x == 0) griddep_launch_dependents();
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort = &sm.abort;
-    if (kCs && blockIdx.x == 0 && threadIdx.x == 32) {
-        // first kernel of the scan: clear the status word once the previous kernel of the
-        // stream (which may use the same workspace) is done
-        griddep_wait();
-        *status = 0;
-    }
 
     if (warp == 0) {
         // ---------------- TMA producer (lane 0 alone): per segment the B tile, per head its x
-        // tile and cs / dt rows (kCs: its dt rows)
+        // tile and cs / dt rows
         if (lane == 0) {
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
-            if (kCs) tma_prefetch_desc(&tm_dt);
             // x and B are inputs of the scan: start streaming the first heads' tiles into L2
             // while the cumsum kernel finishes
             for (int j = 0; j < nh && j < kStateStages; ++j) {
@@ -179,9 +161,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 chunk_span(tab, it.k, Q, seqlen, t0, len);
                 tma_prefetch_l2_4d(&tm_x, 0, it.h, (int)t0, (int)it.b);
             }
-            // cs / dt (and a chunk table) come from earlier kernels; with kCs, the workspace this
-            // kernel writes may still be read by the previous kernel of the stream
-            griddep_wait();
+            griddep_wait();   // cs / dt (and a chunk table) come from earlier kernels
             int seg = -1;
             for (int j = 0; j < nh; ++j) {
                 const StateItem it = state_item(f0 + j, f0, hpg, G, nchunks);
@@ -215,21 +195,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 // failure injection (tests only): this stage is left unissued
                 if (j == 0 && (int)blockIdx.x == skip_cta) continue;
                 const int64_t vrow = ((it.b * nchunks + it.k) * H + it.h) * (int64_t)Q;
-                if (kCs) {
-                    // x rows and the dt rows of heads (h & ~3) .. + 3 (rows past the end of the
-                    // sequence read as zero)
-                    mbar_arrive_expect_tx(&sm.bar_x_full[s], (uint32_t)Q * (kRowBytes + 16));
-                    tma_load_4d(&sm.Xs[s][0], &tm_x, &sm.bar_x_full[s], 0, it.h, (int)t0,
-                                (int)it.b);
-                    tma_load_3d(&sm.dtbox[s][0][0], &tm_dt, &sm.bar_x_full[s], it.h & ~3,
-                                (int)t0, (int)it.b);
-                } else {
-                    mbar_arrive_expect_tx(&sm.bar_x_full[s], (uint32_t)Q * (kRowBytes + 8));
-                    tma_load_4d(&sm.Xs[s][0], &tm_x, &sm.bar_x_full[s], 0, it.h, (int)t0,
-                                (int)it.b);
-                    bulk_load(sm.cs_v[s], cs + vrow, Q * 4, &sm.bar_x_full[s]);
-                    bulk_load(sm.dt_v[s], dtc + vrow, Q * 4, &sm.bar_x_full[s]);
-                }
+                mbar_arrive_expect_tx(&sm.bar_x_full[s], (uint32_t)Q * (kRowBytes + 8));
+                tma_load_4d(&sm.Xs[s][0], &tm_x, &sm.bar_x_full[s], 0, it.h, (int)t0, (int)it.b);
+                bulk_load(sm.cs_v[s], cs + vrow, Q * 4, &sm.bar_x_full[s]);
+                bulk_load(sm.dt_v[s], dtc + vrow, Q * 4, &sm.bar_x_full[s]);
                 // the tile this stage will hold next: into L2 now, so its load is an L2 hit
                 if (j + kStateStages < nh) {
                     const StateItem nx = state_item(f0 + j + kStateStages, f0, hpg, G, nchunks);
@@ -279,58 +248,6 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 mma_commit(&sm.bar_acc_full[a]);
                 if (seg_end) mma_commit(&sm.bar_b_free);
             }
-        }
-    } else if (warp >= 4 && warp < 12 && kCs) {
-        // ---------------- cumsum of dt A, then scale x row tau by
-        // w_tau = exp(cs_last - cs_tau) dt_tau (in place); thread st owns row tau = st
-        const int st = threadIdx.x - 128;             // 0..255
-        const int sw = st >> 5;                       // scale warp 0..7
-        for (int j = 0; j < nh; ++j) {
-            const StateItem it = state_item(f0 + j, f0, hpg, G, nchunks);
-            const int s = j % kStateStages;
-            const uint32_t use = j / kStateStages;
-            if (!warp_wait(&sm.bar_x_full[s], use & 1, abort)) break;
-            const float d = st < Q ? sm.dtbox[s][st][it.h & 3] : 0.f;
-            float v = d * A[it.h];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
-            }
-            float *tot = sm.scan_tot[j & 1];
-            if (lane == 31) tot[sw] = v;
-            mbar_arrive(&sm.bar_scan);
-            if (!warp_wait(&sm.bar_scan, j & 1, abort)) break;
-            float off = 0.f, all = 0.f;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                const float tw = tot[w];
-                off += w < sw ? tw : 0.f;
-                all += tw;
-            }
-            const float c = v + off;
-            if (st < Q) {
-                const int64_t vrow = ((it.b * nchunks + it.k) * H + it.h) * (int64_t)Q;
-                cs[vrow + st] = c;
-                dtc[vrow + st] = d;
-                const float wgt = __expf(all - c) * d;
-                uint4 *row = reinterpret_cast<uint4 *>(&sm.Xs[s][0]) + st * 8;
-#pragma unroll
-                for (int pc = 0; pc < 8; ++pc) {
-                    uint4 xv = row[pc];
-                    uint32_t *wv = &xv.x;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(
-                            *reinterpret_cast<const __nv_bfloat162 *>(&wv[e]));
-                        const float2 sc = fmul2(f, make_float2(wgt, wgt));
-                        wv[e] = pack_bf16x2(sc.x, sc.y);
-                    }
-                    row[pc] = xv;
-                }
-            }
-            fence_async_smem();
-            mbar_arrive(&sm.bar_x_ready[s]);
         }
     } else if (warp >= 4 && warp < 12) {
         // ---------------- scale x rows by w_tau = exp(cs_last - cs_tau) dt_tau (in place)
@@ -1090,23 +1007,6 @@ bool make_map(CUtensorMap *m, const void *ptr, int rank, const cuuint64_t *dims,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// dt (batch, seqlen, heads) float32 -> 3-D map {heads, seqlen, batch} with a 4 x rows x 1 box
-// (16 bytes of heads: the dt rows of four consecutive heads), no swizzle.  Needs heads % 4 == 0
-// (the row stride must be a multiple of 16 bytes).
-bool make_dt_map(CUtensorMap *m, const float *dt, int64_t batch, int64_t seqlen, int64_t heads,
-                 int rows)
-{
-    auto fn = encode_fn();
-    if (!fn || heads % 4 != 0) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)heads, (cuuint64_t)seqlen, (cuuint64_t)batch};
-    const cuuint64_t strides[2] = {(cuuint64_t)(heads * 4), (cuuint64_t)(seqlen * heads * 4)};
-    const cuuint32_t box[3] = {4, (cuuint32_t)rows, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(dt), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // (batch, seqlen, heads_or_groups, 64 * m) bf16 -> 4-D map {inner, heads, seqlen, batch} with
 // a 64 x 1 x 128 x 1 box.
 bool make_seq_map(CUtensorMap *m, const void *ptr, int64_t batch, int64_t seqlen, int64_t mid,
@@ -1127,32 +1027,16 @@ bool tc_supported(bool is_bf16, int P, int N, int Q)
     return is_bf16 && P == kP && N == kN && (Q == 128 || Q == 256);
 }
 
-bool state_fuses_cumsum(int H, const float *dt)
+cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
+                                  const float *cs, float *states, int *status, int64_t batch,
+                                  int64_t seqlen, int H, int G, int Q, int64_t nchunks,
+                                  cudaStream_t st, const char **why, const int2 *tab)
 {
-    return H % 4 == 0 && (reinterpret_cast<uintptr_t>(dt) & 15u) == 0;
-}
-
-cudaError_t launch_chunk_state_tc(const bf16 *x, float *dtc, const bf16 *B, float *cs,
-                                  float *states, int *status, int64_t batch, int64_t seqlen,
-                                  int H, int G, int Q, int64_t nchunks, cudaStream_t st,
-                                  const char **why, const int2 *tab, const float *dt,
-                                  const float *A)
-{
-    CUtensorMap mx, mb, mdt;   // boxes of a whole chunk (Q rows)
+    CUtensorMap mx, mb;   // boxes of a whole chunk (Q rows)
     if (!make_seq_map(&mx, x, batch, seqlen, H, kP, Q) ||
         !make_seq_map(&mb, B, batch, seqlen, G, kN, Q)) {
         *why = "chunk state: cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
-    }
-    const bool fuse = dt != nullptr;
-    if (fuse) {
-        if (tab || !A || !state_fuses_cumsum(H, dt) || !make_dt_map(&mdt, dt, batch, seqlen, H, Q)) {
-            *why = "chunk state: the fused cumsum needs fixed-length input, heads % 4 == 0 and a "
-                   "16-byte aligned dt";
-            return cudaErrorInvalidValue;
-        }
-    } else {
-        mdt = {};
     }
     const int64_t nitems = batch * nchunks * H;   // (batch, chunk, group, head) items
     if (nitems == 0) return cudaSuccess;
@@ -1160,14 +1044,13 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, float *dtc, const bf16 *B, floa
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t smem = sizeof(StateSmem) + 1024;
-    auto kern = fuse ? chunk_state_tc_kernel<true> : chunk_state_tc_kernel<false>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(chunk_state_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk state: set smem attribute"; return e; }
     const unsigned grid = (unsigned)std::min<int64_t>(sms, nitems);
     *why = "chunk state (tcgen05) launch";
-    return launch_pdl(kern, grid, kStateThreads, smem, st, mx, mb, mdt, dtc, cs, A, states,
-                      status, H, G, Q, nchunks, nitems, seqlen, tab,
+    return launch_pdl(chunk_state_tc_kernel, grid, kStateThreads, smem, st, mx, mb, dtc, cs,
+                      states, status, H, G, Q, nchunks, nitems, seqlen, tab,
                       take_test_skip(kTestChunkState));
 }
 

@@ -175,16 +175,10 @@ cudaError_t launch_fill_final(const float *init, float *final_state, int64_t n,
 // Tensor-core (tcgen05 + TMA) path: bf16, P = 64, N = 128, Q in {128, 256}.
 bool tc_supported(bool is_bf16, int P, int N, int Q);
 
-// With dt (and A) given, the kernel also computes the chunk-local cumsum of dt A itself and
-// writes the cs and dtc rows (no cumsum kernel runs before it) and clears *status; this needs
-// fixed-length input and state_fuses_cumsum(H, dt).  Otherwise cs and dtc are inputs from the
-// cumsum kernel.
-bool state_fuses_cumsum(int H, const float *dt);
-cudaError_t launch_chunk_state_tc(const bf16 *x, float *dtc, const bf16 *B, float *cs,
-                                  float *states, int *status, int64_t batch, int64_t seqlen,
-                                  int H, int G, int Q, int64_t nchunks, cudaStream_t st,
-                                  const char **why, const int2 *tab = nullptr,
-                                  const float *dt = nullptr, const float *A = nullptr);
+cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
+                                  const float *cs, float *states, int *status, int64_t batch,
+                                  int64_t seqlen, int H, int G, int Q, int64_t nchunks,
+                                  cudaStream_t st, const char **why, const int2 *tab = nullptr);
 // Offset (in elements), inside one (batch, chunk, head) block of the bf16 entering states, of
 // state element (p, n) for P = 64, N = 128.  The block is stored exactly as the tensor cores
 // read it from shared memory: two halves of 64 n, each 64 rows p of 128 bytes, with the 16-byte

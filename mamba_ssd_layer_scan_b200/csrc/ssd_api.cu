@@ -261,14 +261,9 @@ ssd_status scan_impl(const ssd_shape *shape, const void *x, const float *dt, con
     }
     const bool tc = ssd::tc_supported(bf, P, N, Q);
     float *dtc = tc ? reinterpret_cast<float *>(ws + wl.dtc) : nullptr;
-    // the tensor-core chunk-state kernel computes the cumsum itself where it can (heads % 4 == 0,
-    // aligned dt); stage 1 then ends where it starts
-    const bool fuse_cs = tc && ssd::state_fuses_cumsum(H, dt);
-    if (!fuse_cs) {
-        e = ssd::launch_chunk_cumsum(dt, A, cs, dtc, status, s.batch, s.seqlen, H, Q, nchunks,
-                                     cs_stream);
-        if (e != cudaSuccess) return cuda_fail(e, "dA cumsum launch");
-    }
+    e = ssd::launch_chunk_cumsum(dt, A, cs, dtc, status, s.batch, s.seqlen, H, Q, nchunks,
+                                 cs_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "dA cumsum launch");
     if ((e = record(stage_events, 1, cs_stream)) != cudaSuccess)
         return cuda_fail(e, "record stage event");
 
@@ -277,7 +272,7 @@ ssd_status scan_impl(const ssd_shape *shape, const void *x, const float *dt, con
         ssd::bf16 *hin = reinterpret_cast<ssd::bf16 *>(ws + wl.hin_bf16);
         e = ssd::launch_chunk_state_tc((const ssd::bf16 *)x, dtc, (const ssd::bf16 *)B, cs,
                                        states, status, s.batch, s.seqlen, H, G, Q, nchunks,
-                                       cs_stream, &why, nullptr, fuse_cs ? dt : nullptr, A);
+                                       cs_stream, &why);
         if (e != cudaSuccess) return cuda_fail(e, why);
         if ((e = record(stage_events, 2, cs_stream)) != cudaSuccess)
             return cuda_fail(e, "record stage event");
