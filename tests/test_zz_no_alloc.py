@@ -97,3 +97,33 @@ def test_static_scratch_refuses_problems_larger_than_the_array(cuda_device):
     rc = _static_entry()(ctypes.byref(_shape(w)), p, p, p, p, p, p, w.chunk, None, p, None, None)
     assert rc == ssd.SSD_ERR_UNSUPPORTED
     assert "ssd_chunk_scan_fwd_static" in ssd.last_error()
+
+
+def test_static_scratch_status_is_cleared_by_the_next_call(cuda_device):
+    """A call whose chunk scan is made to time out (the test control of include/ssd_testing.h:
+    one CTA's producer leaves its first stage unissued) leaves the scratch array's status word at
+    SSD_ERR_TIMEOUT; the next call clears it and matches the oracle."""
+    import torch
+    arm = ssd.lib().ssd_testing_skip_stage
+    arm.restype = ctypes.c_int
+    arm.argtypes = [ctypes.c_int, ctypes.c_int]
+    w = configs.SSD_370M.with_(batch=1, seqlen=1024, nheads=8, init_state=True, seed=608)
+    inp = inputs.make_inputs(w)
+    t = torch_inputs(inp, cuda_device)
+    torch.cuda.synchronize()
+    assert arm(2, 1) == ssd.SSD_OK, ssd.last_error()   # the chunk scan, CTA 1
+    stream = torch.cuda.current_stream().cuda_stream
+    y = torch.empty_like(t["x"])
+    final = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
+                        device=t["x"].device)
+    rc = _static_entry()(ctypes.byref(_shape(w)), t["x"].data_ptr(), t["dt"].data_ptr(),
+                         t["A"].data_ptr(), t["B"].data_ptr(), t["C"].data_ptr(),
+                         t["D"].data_ptr(), w.chunk, t["init_state"].data_ptr(), y.data_ptr(),
+                         final.data_ptr(), stream)
+    assert rc == ssd.SSD_OK, ssd.last_error()
+    assert _status_entry()(stream) == ssd.SSD_ERR_TIMEOUT
+    y, final = _call_static(torch, t, w, w.chunk)   # asserts SSD_OK from the status word
+    torch.cuda.synchronize()
+    yo, fo, _ = oracle.ssd_scan(inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, inp.init)
+    assert max_rel_slices(to_np(y), yo, (1, 3))[0] <= TOL["bf16"]
+    assert max_rel_slices(to_np(final), fo, (2, 3))[0] <= TOL["bf16"]
