@@ -334,7 +334,13 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
 //     shared by all heads, X_off is scaled row-wise per head, and u is applied in the epilogue;
 //   - the off-chunk term exp(cs_t) C h_in^T = u_t C (exp(cs_127) h_in)^T, which (scaled h_in)
 //     accumulates into the same TMEM accumulator as the off-diagonal block.
-// So y = Y_diag + f_t Y_A with f_t = exp(cs_t) (T = 0) or u_t (T = 1).
+// So y = Y_diag + f_t Y_A with f_t = exp(cs_t) (T = 0) or u_t (T = 1).  Where the whole chunk
+// decays by at most exp(kRef0Floor) (cs_{Q-1} >= kRef0Floor), T = 1 instead takes the reference
+// "row -1" (cs = 0): x_off scaled by exp(-cs_i) dt_i <= exp(-kRef0Floor) dt_i, h_in unscaled,
+// f_t = exp(cs_t) >= exp(kRef0Floor), which saves scaling h_in; the factors stay well inside the
+// float32 and bf16 range (e^60 ~ 1e26).
+constexpr float kRef0Floor = -60.f;
+__device__ __forceinline__ bool scan_ref0(float cs_last) { return cs_last >= kRef0Floor; }
 constexpr int kXStagesMax = 5;   // x / h_in stages: tiles without an off-diagonal block use 5
                                  // of 32 KB (three in S01, two in the B tile's space once C B^T
                                  // is done); the second tile of a chunk with one uses 2 of 48 KB
@@ -352,7 +358,7 @@ struct alignas(1024) ScanSmem {
                                     // [n atom][64 rows p][64 n]
     float cs_v[kScanVecStages][256];  // per stage: one head's chunk-local cumsum row
     float dt_v[kScanVecStages][256];  // per stage: its dt row (0 past the end)
-    float vt[16][32];               // per worker warp: column factors of its two slices
+    float vt[8][64];                // per worker warp: column factors of its two slices
     uint64_t bar_cb, bar_g, bar_goff, bar_seg_done;
     uint64_t bar_xh_full[kXStagesMax], bar_xh_free[kXStagesMax], bar_xv_ready[kXStagesMax];
     uint64_t bar_vec_full[kScanVecStages], bar_vec_free[kScanVecStages];
@@ -362,12 +368,11 @@ struct alignas(1024) ScanSmem {
     uint32_t tmem_base;
     int abort;
 };
-// warp 0 TMA, warp 1 MMA and TMEM owner, warps 2-17 workers: four per TMEM
-// lane quarter, each owning a 16-column slice of every 64-column block; per head they build
+// warp 0 TMA, warp 1 MMA and TMEM owner, warps 2-9 workers: two per TMEM
+// lane quarter, each owning a 32-column slice of every 64-column block; per head they build
 // their slice of P (mask) and then run the epilogue of the previous head for their slice of y
-constexpr int kScanWorkers = 512;
-constexpr int kScanThreads = 64 + kScanWorkers;   // 576 threads (five warps on some SMSPs: 96
-                                                  // registers each)
+constexpr int kScanWorkers = 256;
+constexpr int kScanThreads = 64 + kScanWorkers;   // 320 threads
 constexpr uint32_t kScanTmemCols = 512;
 constexpr uint32_t kAccCol = 256;   // accumulator buffer a: Y_diag at 256 + 128 a, Y_A at +64
 
@@ -723,11 +728,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             ++si;
         }
     } else if (warp >= 2) {
-        // ---------------- workers, four per TMEM lane quarter.  Warp (qd, cq) owns rows
-        // t = 32 qd + lane of the tile and the 16-column slice [16 cq, 16 cq + 16) of every
+        // ---------------- workers, two per TMEM lane quarter.  Warp (qd, cq) owns rows
+        // t = 32 qd + lane of the tile and the 32-column slice [32 cq, 32 cq + 32) of every
         // 64-column block: per head it builds that slice of both P blocks (mask; for T = 1 after
         // its share of scaling x_off and h_in), then the epilogue y = Y_diag + f_t Y_A of the
-        // previous head for output columns [16 cq, 16 cq + 16).
+        // previous head for output columns [32 cq, 32 cq + 32).
         const int wt = threadIdx.x - 64;           // 0 .. kScanWorkers - 1
         const int qd = warp & 3;
         const int cq = (warp - 2) >> 2;
@@ -736,12 +741,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
         const int r = kTileRows * T + qd * 32 - 1;  // last row above this warp's 32-row slice
         const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
         float *vt = sm.vt[warp - 2];
-        // The slice of block qb is the 16-column unit u = 4 qb + cq of the diagonal block; its
-        // class relative to this row quarter: 0 below the 32 x 32 diagonal sub-block, 1 inside
-        // it, 2 above it (all zero).
-        const int u0 = cq, u1 = 4 + cq;
-        const int cls0 = u0 < 2 * qd ? 0 : (u0 <= 2 * qd + 1 ? 1 : 2);
-        const int cls1 = u1 < 2 * qd ? 0 : (u1 <= 2 * qd + 1 ? 1 : 2);
+        // The slice of block qb is the 32-column unit u = 2 qb + cq of the diagonal block; its
+        // class relative to this row quarter: 0 below the 32 x 32 diagonal sub-block, 1 the
+        // sub-block itself, 2 above it (all zero).
+        const int u0 = cq, u1 = 2 + cq;
+        const int cls0 = u0 < qd ? 0 : (u0 == qd ? 1 : 2);
+        const int cls1 = u1 < qd ? 0 : (u1 == qd ? 1 : 2);
         bool ok = true;
         uint32_t J = 0;
         int si = 0;
@@ -754,19 +759,22 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             tc_fence_after();
             if (offd) {
                 // C B_off^T (TMEM columns [0, 128)) -> bf16, K-major swizzled tile in R; this
-                // warp converts its 32 rows x columns [32 cq, 32 cq + 32)
-                uint32_t gv[32];
-                tmem_ld32(lane_base + 32 * cq, gv);
-                tmem_ld_wait();
-                uint8_t *dst = sm.R + (cq >> 1) * kBoxBytes + t * kRowBytes;
+                // warp converts its 32 rows x columns [64 cq, 64 cq + 64) (one 64-column atom)
+                uint8_t *dst = sm.R + cq * kBoxBytes + t * kRowBytes;
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int pos = ((cq & 1) * 4 + m) ^ (t & 7);
-                    *reinterpret_cast<uint4 *>(dst + pos * 16) = make_uint4(
-                        pack_bf16x2(__uint_as_float(gv[8 * m]), __uint_as_float(gv[8 * m + 1])),
-                        pack_bf16x2(__uint_as_float(gv[8 * m + 2]), __uint_as_float(gv[8 * m + 3])),
-                        pack_bf16x2(__uint_as_float(gv[8 * m + 4]), __uint_as_float(gv[8 * m + 5])),
-                        pack_bf16x2(__uint_as_float(gv[8 * m + 6]), __uint_as_float(gv[8 * m + 7])));
+                for (int e = 0; e < 2; ++e) {
+                    uint32_t gv[32];
+                    tmem_ld32(lane_base + 64 * cq + 32 * e, gv);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const int pos = (e * 4 + m) ^ (t & 7);
+                        *reinterpret_cast<uint4 *>(dst + pos * 16) = make_uint4(
+                            pack_bf16x2(__uint_as_float(gv[8 * m]), __uint_as_float(gv[8 * m + 1])),
+                            pack_bf16x2(__uint_as_float(gv[8 * m + 2]), __uint_as_float(gv[8 * m + 3])),
+                            pack_bf16x2(__uint_as_float(gv[8 * m + 4]), __uint_as_float(gv[8 * m + 5])),
+                            pack_bf16x2(__uint_as_float(gv[8 * m + 6]), __uint_as_float(gv[8 * m + 7])));
+                    }
                 }
                 fence_async_smem();
                 tc_fence_before();
@@ -780,8 +788,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             const int snh = sg.nh;
             const int sh0 = sg.h0;
             const bool row_in = tau < sg.len;   // this thread's row exists in the chunk
-            // output row tau of the segment's first head, this warp's 16 columns
-            const int64_t yseg = ((sg.b * seqlen + sg.t0 + tau) * H + sh0) * (int64_t)kP + 16 * cq;
+            // output row tau of the segment's first head, this warp's 32 columns
+            const int64_t yseg = ((sg.b * seqlen + sg.t0 + tau) * H + sh0) * (int64_t)kP + 32 * cq;
             for (int j = 0; ok && j <= snh; ++j) {
                 if (j < snh) {
                     const uint32_t Jj = J0 + j;
@@ -792,12 +800,6 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     }
                     const float *cs_s = sm.cs_v[vs];
                     const float *dt_s = sm.dt_v[vs];
-                    // this warp's part of the diagonal block of C B^T: it stays in TMEM for the
-                    // whole segment (the P ring and the accumulators use other columns), so it
-                    // is read again per head instead of held in registers
-                    uint32_t g0[16], g1[16];
-                    if (cls0 < 2) tmem_ld16(lane_base + gdiag + 16 * u0, g0);
-                    if (cls1 < 2) tmem_ld16(lane_base + gdiag + 16 * u1, g1);
                     if (offd) {
                         // x rows [0, 128) *= exp(cs_127 - cs_i) dt_i; h_in *= exp(cs_127)
                         const int xs = Jj % nst;
@@ -806,14 +808,22 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                             break;
                         }
                         uint8_t *stg = scan_stage(sm, xs, offd);
-                        const float c127 = cs_s[127];
+                        // reference row 127 (x rows * exp(cs_127 - cs_i) dt_i, h_in *
+                        // exp(cs_127)), or, where the chunk decays by at most exp(kRef0Floor),
+                        // reference "row -1" (x rows * exp(-cs_i) dt_i, h_in as it is): all
+                        // factors then lie in [exp(kRef0Floor), exp(-kRef0Floor)], and the h_in
+                        // pass is saved
+                        const float ref = scan_ref0(cs_s[Q - 1]) ? 0.f : cs_s[127];
                         scale_pieces<1024 / kScanWorkers>(stg, wt, kScanWorkers, [&](int c) {
                             const int i = c >> 3;
-                            return __expf(c127 - cs_s[i]) * dt_s[i];
+                            return __expf(ref - cs_s[i]) * dt_s[i];
                         });
-                        const float sh = __expf(c127);
-                        scale_pieces<1024 / kScanWorkers>(stg + scan_hoff(offd), wt, kScanWorkers,
-                                                          [&](int) { return sh; });
+                        if (ref != 0.f) {
+                            const float sh = __expf(ref);
+                            scale_pieces<1024 / kScanWorkers>(stg + scan_hoff(offd), wt,
+                                                              kScanWorkers,
+                                                              [&](int) { return sh; });
+                        }
                         fence_async_smem();
                         mbar_arrive(&sm.bar_xv_ready[xs]);
                     }
@@ -828,29 +838,36 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     const float crf = cs_s[r < 0 ? 0 : r];
                     const float um = __expf(ct - cm);
                     const float uf = qd > 0 ? __expf(ct - crf) : 0.f;
-                    {
-                        // lane l: column 16 (4 (l >> 4) + cq) + (l & 15) of the diagonal block
-                        const int uu = 4 * (lane >> 4) + cq;
-                        const int cl = uu < 2 * qd ? 0 : (uu <= 2 * qd + 1 ? 1 : 2);
-                        const int i = kTileRows * T + 16 * uu + (lane & 15);
+#pragma unroll
+                    for (int qb = 0; qb < 2; ++qb) {
+                        // lane l: column 32 u + l of the diagonal block, u = 2 qb + cq
+                        const int uu = 2 * qb + cq;
+                        const int cl = uu < qd ? 0 : (uu == qd ? 1 : 2);
+                        const int i = kTileRows * T + 32 * uu + lane;
                         const float ref = cl == 0 ? crf : cm;
                         const float v = __expf(ref - cs_s[i]) * dt_s[i];
-                        vt[lane] = cl < 2 ? v : 0.f;
+                        vt[32 * qb + lane] = cl < 2 ? v : 0.f;
                     }
                     __syncwarp();
-                    tmem_ld_wait();
 #pragma unroll
                     for (int qb = 0; qb < 2; ++qb) {
                         const uint32_t blk = 2 * Jj + qb;
                         const uint32_t slot = blk % kRing, su = blk / kRing;
                         const int cl = qb ? cls1 : cls0;
-                        const uint32_t *gv = qb ? g1 : g0;
-                        const float *vq = vt + 16 * qb;
-                        uint32_t pk[8];
+                        const float *vq = vt + 32 * qb;
+                        // this warp's part of the diagonal block of C B^T: it stays in TMEM for
+                        // the whole segment (the P ring and the accumulators use other
+                        // columns), so it is read again per head instead of held in registers
+                        uint32_t gv[32];
+                        if (cl < 2) {
+                            tmem_ld32(lane_base + gdiag + 32 * (qb ? u1 : u0), gv);
+                            tmem_ld_wait();
+                        }
+                        uint32_t pk[16];
                         if (cl == 0) {
                             const float2 uu = make_float2(uf, uf);
 #pragma unroll
-                            for (int c = 0; c < 4; ++c) {
+                            for (int c = 0; c < 8; ++c) {
                                 const float4 vv = *reinterpret_cast<const float4 *>(vq + 4 * c);
                                 const float2 p0 = fmul2(
                                     fmul2(make_float2(__uint_as_float(gv[4 * c]),
@@ -864,17 +881,16 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                                 pk[2 * c + 1] = pack_bf16x2(p1.x, p1.y);
                             }
                         } else if (cl == 1) {
-                            // inside the causal 32 x 32 sub-block: local column lc kept for
-                            // lc <= lane, + D at lc = lane
-                            const int lc0 = 16 * (qb ? u1 : u0) - 32 * qd;   // 0 or 16
+                            // the causal 32 x 32 sub-block: local column lc kept for lc <= lane,
+                            // + D at lc = lane
                             const float2 uu = make_float2(um, um);
 #pragma unroll
-                            for (int c = 0; c < 8; ++c) {
+                            for (int c = 0; c < 16; ++c) {
                                 const float2 ww = *reinterpret_cast<const float2 *>(vq + 2 * c);
                                 float2 pp = fmul2(fmul2(make_float2(__uint_as_float(gv[2 * c]),
                                                                     __uint_as_float(gv[2 * c + 1])),
                                                         ww), uu);
-                                const int lc = lc0 + 2 * c;
+                                const int lc = 2 * c;
                                 pp.x = (lc <= lane) ? pp.x : 0.f;
                                 pp.y = (lc + 1 <= lane) ? pp.y : 0.f;
                                 pp.x += (lc == lane) ? Dh : 0.f;
@@ -883,7 +899,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                             }
                         } else {
 #pragma unroll
-                            for (int c = 0; c < 8; ++c) pk[c] = 0u;
+                            for (int c = 0; c < 16; ++c) pk[c] = 0u;
                         }
                         if (su >= 1 &&
                             !warp_wait(&sm.bar_slot_free[slot], (su - 1) & 1, abort)) {
@@ -895,7 +911,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                         // the segment's first two heads: C B^T of a tile with an off-diagonal
                         // block overwrites the ring at every segment) they stay
                         if (cl != 2 || j < 2) {
-                            tmem_st8(lane_base + pcol + 32 * slot + 8 * cq, pk);
+                            tmem_st16(lane_base + pcol + 32 * slot + 16 * cq, pk);
                             tmem_st_wait();
                         }
                         tc_fence_before();
@@ -904,7 +920,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     if (!ok) break;
                 }
                 if (j >= 1) {
-                    // epilogue of head jj = j - 1 for output columns [16 cq, 16 cq + 16)
+                    // epilogue of head jj = j - 1 for output columns [32 cq, 32 cq + 32)
                     const uint32_t Jj = J0 + j - 1;
                     const int a = Jj & 1;
                     if (!warp_wait(&sm.bar_acc_full[a], (Jj >> 1) & 1, abort)) {
@@ -912,45 +928,44 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t col = lane_base + kAccCol + 128 * a + 16 * cq;
-                    uint32_t d0[16], a0[16];
-                    tmem_ld16(col, d0);
-                    tmem_ld16(col + 64, a0);
+                    const uint32_t col = lane_base + kAccCol + 128 * a + 32 * cq;
+                    uint32_t d0[32], a0[32];
+                    tmem_ld32(col, d0);
+                    tmem_ld32(col + 64, a0);
                     const int vs = Jj % kScanVecStages;
                     const float *cs_j = sm.cs_v[vs];
-                    const float fct = __expf(cs_j[tau] - (T ? cs_j[127] : 0.f));
+                    const float fct =
+                        __expf(cs_j[tau] - (T && !scan_ref0(cs_j[Q - 1]) ? cs_j[127] : 0.f));
                     tmem_ld_wait();
                     tc_fence_before();
                     mbar_arrive(&sm.bar_acc_free[a]);
                     mbar_arrive(&sm.bar_vec_free[vs]);   // done with this head's cs / dt
                     const int64_t yoff = yseg + (int64_t)(j - 1) * kP;
-                    // gated output (z given): y * z * sigmoid(z); z kept as 8 packed bf16 pairs
+                    // gated output (z given): y * z * sigmoid(z), z as packed bf16 pairs
                     const bool gz = kGate && row_in;
-                    uint4 z0 = make_uint4(0u, 0u, 0u, 0u), z1 = z0;
-                    if (gz) {
-                        const uint4 *zrow = reinterpret_cast<const uint4 *>(z + yoff);
-                        z0 = zrow[0];
-                        z1 = zrow[1];
-                    }
-                    const uint32_t zw[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-                    uint32_t pk[8];
+                    uint4 *yrow = reinterpret_cast<uint4 *>(y + yoff);
+                    const uint4 *zrow = reinterpret_cast<const uint4 *>(z + yoff);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float v0 = fmaf(fct, __uint_as_float(a0[2 * c]), __uint_as_float(d0[2 * c]));
-                        float v1 = fmaf(fct, __uint_as_float(a0[2 * c + 1]),
-                                        __uint_as_float(d0[2 * c + 1]));
-                        if (gz) {
-                            const float2 zf = __bfloat1622float2(
-                                *reinterpret_cast<const __nv_bfloat162 *>(&zw[c]));
-                            v0 *= silu(zf.x);
-                            v1 *= silu(zf.y);
+                    for (int q = 0; q < 4; ++q) {   // 8 columns per 16-byte store
+                        uint4 zq = make_uint4(0u, 0u, 0u, 0u);
+                        if (gz) zq = zrow[q];
+                        const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int e = 8 * q + 2 * c;
+                            float v0 = fmaf(fct, __uint_as_float(a0[e]), __uint_as_float(d0[e]));
+                            float v1 = fmaf(fct, __uint_as_float(a0[e + 1]),
+                                            __uint_as_float(d0[e + 1]));
+                            if (gz) {
+                                const float2 zf = __bfloat1622float2(
+                                    *reinterpret_cast<const __nv_bfloat162 *>(&zw[c]));
+                                v0 *= silu(zf.x);
+                                v1 *= silu(zf.y);
+                            }
+                            pk[c] = pack_bf16x2(v0, v1);
                         }
-                        pk[c] = pack_bf16x2(v0, v1);
-                    }
-                    if (row_in) {
-                        uint4 *yrow = reinterpret_cast<uint4 *>(y + yoff);
-                        yrow[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        yrow[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        if (row_in) yrow[q] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     }
                 }
             }

@@ -19,16 +19,21 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kGroup = 8;  // chunks whose loads are issued together
+// Programmatic dependent launch: over chains of at most this many chunks the kernel lets the
+// chunk scan launch at its start, so that the scan's set-up (barriers, TMEM, its first C and B
+// tiles and C B^T) overlaps the recurrence; over longer chains only at its end, because the
+// scan's early CTAs then slowed the recurrence itself (256 chunks at L = 65536: 25 us).
+constexpr int64_t kEarlyTriggerChunks = 64;
 
 template <bool kBf16Out>
 __global__ void __launch_bounds__(kThreads)
 state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
                      const float *__restrict__ init, float *__restrict__ final_state,
                      bf16 *__restrict__ hin, int H, int PN, int Q, int64_t nchunks,
-                     const int32_t *__restrict__ cstart)
+                     const int32_t *__restrict__ cstart, bool trigger_early)
 {
     griddep_wait();   // the chunk states come from the previous kernel
-    griddep_launch_dependents();
+    if (trigger_early) griddep_launch_dependents();
     const int nblk = (PN / 4 + kThreads - 1) / kThreads;
     const int64_t v = (blockIdx.x % nblk) * (int64_t)kThreads + threadIdx.x;  // float4 index
     // b: batch row, or the packed sequence when cstart is given (its chunks are
@@ -83,6 +88,7 @@ state_passing_kernel(float *__restrict__ states, const float *__restrict__ cs,
     }
     if (final_state)
         *reinterpret_cast<float4 *>(final_state + (b * H + h) * PN + v * 4) = hs;
+    if (!trigger_early) griddep_launch_dependents();
 }
 
 }  // namespace
@@ -96,7 +102,7 @@ cudaError_t launch_state_passing(float *states, const float *cs, const float *in
     const int32_t *none = nullptr;
     return launch_pdl(hin_bf16 ? state_passing_kernel<true> : state_passing_kernel<false>, grid,
                       kThreads, 0, st, states, cs, init, final_state, hin_bf16, H, PN, Q, nchunks,
-                      none);
+                      none, nchunks <= kEarlyTriggerChunks);
 }
 
 cudaError_t launch_state_passing_varlen(float *states, const float *cs, const float *init,
@@ -106,9 +112,10 @@ cudaError_t launch_state_passing_varlen(float *states, const float *cs, const fl
 {
     const int PN = P * N;
     const unsigned grid = (unsigned)(((PN / 4 + kThreads - 1) / kThreads) * H * (int64_t)nseq);
+    // packed sequences: chains of one sequence each, short next to the packed total
     return launch_pdl(hin_bf16 ? state_passing_kernel<true> : state_passing_kernel<false>, grid,
                       kThreads, 0, st, states, cs, init, final_state, hin_bf16, H, PN, Q, nchunks,
-                      cstart);
+                      cstart, true);
 }
 
 }  // namespace ssd
