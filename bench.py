@@ -344,6 +344,27 @@ def time_forward(ssd, torch, w, t, dev, stream, K, warmup, flush, barrier=lambda
     return step_ms, staged_ms, kern_ms, wall, (ws, y, final)
 
 
+def time_graph(ssd, torch, w, t, stream, K, flush):
+    """The same step captured once into a CUDA graph (ssd.CapturedScan) and replayed: K
+    replays, each bracketed by CUDA events with the L2 flush written before it (outside the
+    events).  Returns the mean ms per replay."""
+    cap = ssd.CapturedScan(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], w.chunk,
+                           init_state=t.get("init"))
+    for _ in range(3):
+        flush.fill_(1.0)
+        cap.replay()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for a, b in ev:
+        flush.fill_(1.0)
+        a.record(stream)
+        cap.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    assert ssd.workspace_status(cap.workspace) == ssd.SSD_OK, "graph replay status"
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+
 def kernel_rooflines(w, staged_ms, kern_ms, hbm, tc_peak):
     """Per kernel: mean time, share of the staged step, achieved GB/s on its algorithmic bytes
     and on all the bytes it moves (algorithmic + workspace), TFLOP/s, the fractions of the
@@ -460,8 +481,10 @@ def main():
         _, tx = device_inputs(torch, wx, inputs.make_inputs(wx), dev)
         Kx = max(10, min(K, 100))
         sx, stx, kx, _, _ = time_forward(ssd, torch, wx, tx, dev, stream, Kx, args.warmup, flush)
-        extra[wx.name] = (wx, Kx, sx, stx, kx)
+        gx = time_graph(ssd, torch, wx, tx, stream, Kx, flush)
+        extra[wx.name] = (wx, Kx, sx, stx, kx, gx)
         del tx
+    graph_ms = time_graph(ssd, torch, w, t, stream, max(10, min(K, 100)), flush)
 
     # ---- end to end through the C ABI with host buffers: every step copies its inputs from
     # pinned host memory, runs the scan through the public API and copies y and the final state
@@ -676,7 +699,7 @@ def main():
                  "peak_source": (f"{peak_src} (MEASURED_PEAKS.json burst)"
                                  if peak_src == "measured" else "fallback")})
     config_lines = {}
-    for name, (wx, Kx, sx, stx, kx) in extra.items():
+    for name, (wx, Kx, sx, stx, kx, gx) in extra.items():
         msx = max_over_ranks(sum(sx), dev) / Kx
         kern_x = kernel_rooflines(wx, stx, kx, hbm, tc_peak)
         config_lines[name] = {
@@ -687,6 +710,8 @@ def main():
             "step_totals": step_summary(wx, msx, hbm, tc_peak),
             "tensor_core_kernels": tensor_core_summary(wx, kern_x, tc_peak, hbm),
             "kernels": kern_x,
+            "graph": {"ms_per_step": gx, "value": wx.batch * wx.seqlen / (gx / 1e3),
+                      "how": "the step captured once into a CUDA graph (ssd.CapturedScan), replayed"},
             "l2": "256 MB buffer written between timed steps (outside the events)"}
 
     cpu = None
@@ -712,6 +737,10 @@ def main():
         "step_totals": step_summary(w, ms_per_step, hbm, tc_peak),
         "kernels": kernels,
         "configs": config_lines,
+        "graph": {"ms_per_step": graph_ms, "value": tokens_per_step / (graph_ms / 1e3),
+                  "unit": "tokens/s",
+                  "how": "the step captured once into a CUDA graph (ssd.CapturedScan), replayed; "
+                         "L2 flushed between replays (outside the events)"},
         "fused_block": {"workload": w.name + "_gated_softplus_dt",
                         "metric": "ssd_chunk_scan_fwd_ex_tokens_per_s",
                         "value": tokens_per_step / (block_ms / 1e3), "unit": "tokens/s",

@@ -232,6 +232,75 @@ def chunk_scan_fwd(x, dt, A, B, C, D, chunk_size: int = 256, init_state=None,
     return y, final_state
 
 
+class CapturedScan:
+    """One chunk_scan_fwd call captured into a CUDA graph, replayed as a whole.
+
+    For steps short enough that launching the scan's kernels is a visible share of the step (at
+    2 x 2048 tokens x 24 heads the replay takes about 42 us against 48 us for the launched call;
+    at 4 x 4096 x 80 the two are equal).  The graph holds the call's kernels with their
+    programmatic dependent launches, bound to the tensors given here: refill x, dt, A, B, C, D
+    (and init_state) in place between replays; the outputs land in ``y`` and ``final_state``
+    each time.  Keyword arguments are those of chunk_scan_fwd (the fused block options
+    included; stage_events excluded)."""
+
+    def __init__(self, x, dt, A, B, C, D, chunk_size: int = 256, init_state=None, **kw):
+        torch = _torch()
+        if "stage_events" in kw or "stream" in kw:
+            raise ValueError("CapturedScan takes no stage_events or stream")
+        dev = x.device
+        b, L, H, P = x.shape
+        N = B.shape[3]
+        self.y = kw.pop("y", None)
+        if self.y is None:
+            self.y = torch.empty_like(x)
+        self.final_state = kw.pop("final_state", None)
+        if self.final_state is None and kw.pop("return_final_state", True):
+            self.final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+        self.workspace = kw.pop("workspace", None)
+        args = (x, dt, A, B, C, D, chunk_size)
+
+        def call(stream):
+            chunk_scan_fwd(*args, init_state=init_state, y=self.y,
+                           final_state=self.final_state,
+                           return_final_state=self.final_state is not None,
+                           workspace=self.workspace, stream=stream, **kw)
+
+        if self.workspace is None:   # allocated once, outside the capture
+            self.workspace = _workspace_for(x, B, chunk_size, kw)
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            call(side)   # first launch outside the capture (module load, kernel attributes)
+        side.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=side):
+            call(side)
+        torch.cuda.current_stream(dev).wait_stream(side)
+
+    def replay(self):
+        """Run the captured call on the current stream; returns (y, final_state)."""
+        self.graph.replay()
+        return self.y, self.final_state
+
+
+def _workspace_for(x, B, chunk_size, kw):
+    """The workspace chunk_scan_fwd would allocate for this call."""
+    torch = _torch()
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    shape = make_shape(b, L, H, P, N, G, _dtype_code(x))
+    z, dt_bias = kw.get("z"), kw.get("dt_bias")
+    if z is None and dt_bias is None and not kw.get("dt_softplus") and kw.get("dt_limit") is None:
+        return new_workspace(shape, chunk_size, x.device)
+    lo, hi = kw.get("dt_limit") or (0.0, 0.0)
+    opts = FwdOptions(_ptr(z), _ptr(dt_bias), 1 if kw.get("dt_softplus") else 0, lo, hi)
+    n = lib().ssd_chunk_scan_fwd_ex_workspace_size(ctypes.byref(shape), chunk_size,
+                                                  ctypes.byref(opts))
+    if n == 0:
+        raise SSDError(SSD_ERR_INVALID_ARG, last_error())
+    return torch.empty(n, dtype=torch.uint8, device=x.device)
+
+
 def varlen_workspace_size(shape: Shape, nseq: int, chunk_size: int) -> int:
     n = lib().ssd_chunk_scan_varlen_workspace_size(ctypes.byref(shape), nseq, chunk_size)
     if n == 0:
