@@ -37,11 +37,10 @@ from mamba_ssd_layer_scan_b200 import configs, inputs  # noqa: E402
 
 KERNELS = ("chunk_cumsum", "chunk_state", "state_passing", "chunk_scan")
 # Kernels of one ssd_chunk_scan_bwd call with dfinal and dinit, no initial state: a zero fill;
-# the reversed tensor-core scan (3 gathers, dt shift, 4 scan kernels) and dinit; the dB scan
-# (dfinal transpose, cumsum, chunk state, state passing, chunk scan, group sum) and the dC scan
-# (the same without a transpose); the final-state dot product, the token and decay kernels and
-# the batch sum of dA and dD.
-BWD_KERNELS = 1 + 8 + 1 + 6 + 5 + 4
+# the reversed tensor-core scan (3 gathers, dt shift, 4 scan kernels) and dinit; the dB scan and
+# the dC scan (cumsum, tensor-core chunk state, state passing, chunk scan, group sum each); the
+# final-state dot product, the token and decay kernels and the batch sum of dA and dD.
+BWD_KERNELS = 1 + 8 + 1 + 5 + 5 + 4
 KERNEL_SOURCES = {
     "chunk_cumsum": ["chunk_cumsum.cu"],
     "chunk_state": ["chunk_tc.cu", "sm100.cuh"],

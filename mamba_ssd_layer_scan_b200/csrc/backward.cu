@@ -69,19 +69,6 @@ __global__ void fill_kernel(float *__restrict__ out, float v, int64_t n)
         out[i] = v;
 }
 
-__global__ void transpose_kernel(const float *__restrict__ in, float *__restrict__ out,
-                                 int64_t mats, int rows, int cols)
-{
-    const int64_t n = mats * rows * cols;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int c = (int)(i % cols);
-        const int r = (int)((i / cols) % rows);
-        const int64_t m = i / cols / rows;
-        out[(m * cols + c) * rows + r] = in[i];
-    }
-}
-
 // Eight lanes per (b, t, h) row of P = 64 channels, 16 bytes of each bf16 input per lane: dx,
 // <x, dy>, and the decay-gradient term q.
 constexpr int kTokLanes = 8;
@@ -302,15 +289,6 @@ cudaError_t launch_fill(float *out, float value, int64_t n, cudaStream_t st)
 {
     if (n == 0) return cudaSuccess;
     fill_kernel<<<grid_for(n), 256, 0, st>>>(out, value, n);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_transpose(const float *in, float *out, int64_t mats, int rows, int cols,
-                             cudaStream_t st)
-{
-    const int64_t n = mats * rows * cols;
-    if (n == 0) return cudaSuccess;
-    transpose_kernel<<<grid_for(n), 256, 0, st>>>(in, out, mats, rows, cols);
     return cudaGetLastError();
 }
 

@@ -1,27 +1,29 @@
-// The two float32 scans of the backward pass (dB and dC), specialised for their shape.
+// The chunk-output kernel of the backward pass's two scans (dB and dC), in float32,
+// specialised for their shape.
 //
-// Both are scans of the forward's kind with the head and state dimensions swapped: the state
-// is E x K = N x P (128 x 64) per (batch, head), the "x" operand x'' has E = N = 128 channels and
-// is shared by the heads of a group (it is B or C), the "B" and "C" operands B'', C'' have
-// K = P = 64 channels per head (x or dy):
+// Both scans are of the forward's kind with the head and state dimensions swapped: the state
+// is K x E = P x N (64 x 128) per (batch, head), stored [j][e] like the forward's [p][n]; the
+// "x" operand x'' has E = N = 128 channels and is shared by the heads of a group (it is B or C),
+// the "B" and "C" operands B'', C'' have K = P = 64 channels per head (x or dy):
 //
-//   chunk state   S_k[e][j] = sum_{r in k} exp(cs_last - cs_r) w_r x''_r[e] B''_r[j]
+//   chunk state   S_k[j][e] = sum_{r in k} exp(cs_last - cs_r) w_r B''_r[j] x''_r[e]
 //   chunk output  y_t[e]    = sum_{s <= t, s in k} exp(cs_t - cs_s) w_s (C''_t . B''_s) x''_s[e]
-//                           + exp(cs_t) sum_j S_in[e][j] C''_t[j]
+//                           + exp(cs_t) sum_j S_in[j][e] C''_t[j]
 //
 // (the same chunked form as the forward: mohakchugh.is-a.dev "Mamba-2", Block Decomposition).
 // dB runs it on the time-reversed sequence (x'' = C, B'' = dy, C'' = x, unit weights, decays
-// shifted by one token), dC forward (x'' = B, B'' = x, C'' = dy, weights dt).  The operands are
-// read in place from the bf16 inputs (reversed rows, the group's row for x''); everything is
-// float32 from there on, because the decay gradient needs the outputs' dot products with B and C
-// to float32 accuracy (see backward.cu).  Each output row's dot product with the group's B or C
-// row is formed in the epilogue.
+// shifted by one token), dC forward (x'' = B, B'' = x, C'' = dy, weights dt).  The chunk states
+// come from the tensor-core chunk-state kernel (chunk_tc.cu) with split bf16 operands; this
+// kernel forms the chunk outputs.  It reads the operands in place from the bf16 inputs
+// (reversed rows, the group's row for x''); everything is float32 from there on, because the
+// decay gradient needs the outputs' dot products with B and C to float32 accuracy (see
+// backward.cu).  Each output row's dot product with the group's B or C row is formed in the
+// epilogue.
 //
-// Register tiling: the chunk-state kernel gives each of its 256 threads a 4 x 8 block of the
-// 128 x 64 state; the chunk-output kernel gives each thread 4 rows x 8 channels of the 64 x 128
-// output tile, and 4 x 4 of the 64 x 64 masked Gram matrix before that.  The channels of a
-// thread are two runs of 4 at e0 and 64 + e0, so that each 16-byte shared-memory load of a half
-// warp reads 256 contiguous bytes (two wavefronts, no bank conflict).
+// Register tiling: each thread holds 4 rows x 8 channels of the 64 x 128 output tile, and 4 x 4
+// of the 64 x 64 masked Gram matrix before that.  The channels of a thread are two runs of 4 at
+// e0 and 64 + e0, so that each 16-byte shared-memory load of a half warp reads 256 contiguous
+// bytes (two wavefronts, no bank conflict).
 #include "common.cuh"
 
 namespace ssd {
@@ -43,75 +45,6 @@ __device__ __forceinline__ void unpack8(const uint4 raw, float *v)
 __device__ __forceinline__ int64_t src_row(int64_t tau, int64_t L, bool rev)
 {
     return rev ? L - 1 - tau : tau;
-}
-
-__global__ void __launch_bounds__(kThreads)
-bwd_chunk_state_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
-                       const float *__restrict__ w, const float *__restrict__ cs,
-                       float *__restrict__ states, int64_t L, int H, int G, int64_t nch, bool rev)
-{
-    __shared__ __align__(16) float xs[kQs][kE];
-    __shared__ __align__(16) float bs[kQs][kK];
-    const int h = (int)(blockIdx.x % H);
-    const int64_t k = (blockIdx.x / H) % nch, b = blockIdx.x / H / nch;
-    const int g = h / (H / G);
-    const int64_t t0 = k * kQs;
-    const int len = (int)min((int64_t)kQs, L - t0);
-    const float *csk = cs + ((b * nch + k) * H + h) * (int64_t)kQs;
-    const float cl = csk[len - 1];
-
-    for (int i = threadIdx.x; i < kQs * kE / 8; i += kThreads) {
-        const int r = i / (kE / 8), c8 = i % (kE / 8);
-        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (r < len) {
-            const int64_t s = src_row(t0 + r, L, rev);
-            unpack8(*reinterpret_cast<const uint4 *>(xg + ((b * L + s) * G + g) * kE + c8 * 8), v);
-        }
-        *reinterpret_cast<float4 *>(&xs[r][c8 * 8]) = make_float4(v[0], v[1], v[2], v[3]);
-        *reinterpret_cast<float4 *>(&xs[r][c8 * 8 + 4]) = make_float4(v[4], v[5], v[6], v[7]);
-    }
-    for (int i = threadIdx.x; i < kQs * kK / 8; i += kThreads) {
-        const int r = i / (kK / 8), c8 = i % (kK / 8);
-        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (r < len) {
-            const int64_t tau = t0 + r, s = src_row(tau, L, rev);
-            const float f = __expf(cl - csk[r]) * (w ? w[(b * L + tau) * H + h] : 1.f);
-            unpack8(*reinterpret_cast<const uint4 *>(bh + ((b * L + s) * H + h) * kK + c8 * 8), v);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] *= f;
-        }
-        *reinterpret_cast<float4 *>(&bs[r][c8 * 8]) = make_float4(v[0], v[1], v[2], v[3]);
-        *reinterpret_cast<float4 *>(&bs[r][c8 * 8 + 4]) = make_float4(v[4], v[5], v[6], v[7]);
-    }
-    __syncthreads();
-
-    // thread: state rows e0..e0+3, columns kg*4..+3 and 32+kg*4..+3 (conflict-free float4s)
-    const int e0 = (threadIdx.x / 8) * 4, kg = threadIdx.x % 8;
-    float acc[4][8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-    for (int r = 0; r < len; ++r) {
-        const float4 xv = *reinterpret_cast<const float4 *>(&xs[r][e0]);
-        const float4 b0 = *reinterpret_cast<const float4 *>(&bs[r][kg * 4]);
-        const float4 b1 = *reinterpret_cast<const float4 *>(&bs[r][32 + kg * 4]);
-        const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
-        const float ba[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xa[i], ba[j], acc[i][j]);
-    }
-    float *out = states + ((b * nch + k) * H + h) * (int64_t)(kE * kK);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float *row = out + (e0 + i) * kK;
-        *reinterpret_cast<float4 *>(row + kg * 4) =
-            make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-        *reinterpret_cast<float4 *>(row + 32 + kg * 4) =
-            make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
-    }
 }
 
 // x'' and C'' are bf16 inputs and stay bf16 here (exact); B'' * w, the Gram matrix and the
@@ -185,13 +118,10 @@ bwd_chunk_scan_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
             sm.cT[c8 * 8 + j][r] = pc[j];
         }
     }
-    for (int i = threadIdx.x; i < kE * kK / 4; i += kThreads) {
-        const int e = i % kE, j4 = i / kE;   // consecutive threads: consecutive e (no conflicts)
-        const float4 v = *reinterpret_cast<const float4 *>(hk + e * kK + j4 * 4);
-        sm.hT[j4 * 4 + 0][e] = v.x;
-        sm.hT[j4 * 4 + 1][e] = v.y;
-        sm.hT[j4 * 4 + 2][e] = v.z;
-        sm.hT[j4 * 4 + 3][e] = v.w;
+    for (int i = threadIdx.x; i < kE * kK / 4; i += kThreads) {   // [j][e]: a plain copy
+        const int j = i / (kE / 4), e4 = i % (kE / 4);
+        *reinterpret_cast<float4 *>(&sm.hT[j][e4 * 4]) =
+            *reinterpret_cast<const float4 *>(hk + j * kE + e4 * 4);
     }
     __syncthreads();
 
@@ -302,17 +232,6 @@ bwd_chunk_scan_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
 }  // namespace
 
 bool bwd_scan_supported(int P, int N) { return P == kK && N == kE; }
-
-cudaError_t launch_bwd_chunk_state(const bf16 *xg, const bf16 *bh, const float *w,
-                                   const float *cs, float *states, int64_t batch, int64_t L,
-                                   int H, int G, int64_t nch, bool rev, cudaStream_t st)
-{
-    const int64_t n = batch * nch * H;
-    if (n == 0) return cudaSuccess;
-    bwd_chunk_state_kernel<<<(unsigned)n, kThreads, 0, st>>>(xg, bh, w, cs, states, L, H, G, nch,
-                                                             rev);
-    return cudaGetLastError();
-}
 
 cudaError_t launch_bwd_chunk_scan(const bf16 *xg, const bf16 *bh, const bf16 *ch, const float *w,
                                   const float *cs, const float *hin, const bf16 *vg, float *ys,

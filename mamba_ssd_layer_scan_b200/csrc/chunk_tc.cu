@@ -113,6 +113,13 @@ __device__ __forceinline__ StateItem state_item(int64_t f, int64_t f0, int hpg, 
     return it;
 }
 
+// kSplit (Q = 64 only): the scaled rows w_tau x_tau go to the MMA as two bf16 tiles, the rounded
+// value and the rounding remainder (the second in the upper part of the stage), accumulated by
+// two MMA chains: the state to about float32 accuracy (the backward's decay gradient needs it).
+// kRev: the chunks run over the time-reversed sequence: chunk k covers the reversed tokens
+// [kQ, kQ + Q), i.e. the memory rows [L - kQ - Q, L - kQ) in descending order; the rows are
+// loaded in memory order and row i of the tile is reversed token Q - 1 - i.
+template <bool kSplit, bool kRev>
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                       const __grid_constant__ CUtensorMap tm_b, const float *__restrict__ dtc,
@@ -129,6 +136,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int64_t f1 = ((int64_t)blockIdx.x + 1) * nitems / gridDim.x;
     const int nh = (int)(f1 - f0);
     if (nh <= 0) return;
+    // first memory row of the tile of the chunk that starts at (reversed) token t0
+    auto row0 = [&](int64_t t0) { return (int)(kRev ? seqlen - t0 - Q : t0); };
+    // L2 prefetches are hints: a tile that starts before row 0 is not prefetched
+    auto pf_row = [&](int64_t t0) { return row0(t0) < 0 ? 0 : row0(t0); };
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_b, 1);
@@ -170,7 +181,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 int64_t t0;
                 int len;
                 chunk_span(tab, it.k, Q, seqlen, t0, len);
-                tma_prefetch_l2_4d(&tm_x, 0, it.h, (int)t0, (int)it.b);
+                tma_prefetch_l2_4d(&tm_x, 0, it.h, pf_row(t0), (int)it.b);
             }
             griddep_wait();   // cs / dt (and a chunk table) come from earlier kernels
             int seg = -1;
@@ -185,7 +196,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     if (seg > 0 && !mbar_wait(&sm.bar_b_free, (seg - 1) & 1, abort)) break;
                     mbar_arrive_expect_tx(&sm.bar_b, 2u * Q * kRowBytes);
                     for (int a = 0; a < 2; ++a)   // boxes of Q rows
-                        tma_load_4d(&sm.Bs[a][0], &tm_b, &sm.bar_b, 64 * a, it.g, (int)t0,
+                        tma_load_4d(&sm.Bs[a][0], &tm_b, &sm.bar_b, 64 * a, it.g, row0(t0),
                                     (int)it.b);
                     // the next segment's B tile into L2 now, so that its load after this
                     // segment's last MMA is short
@@ -196,7 +207,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                         int nlen;
                         chunk_span(tab, nx.k, Q, seqlen, nt0, nlen);
                         for (int a = 0; a < 2; ++a)
-                            tma_prefetch_l2_4d(&tm_b, 64 * a, nx.g, (int)nt0, (int)nx.b);
+                            tma_prefetch_l2_4d(&tm_b, 64 * a, nx.g, pf_row(nt0), (int)nx.b);
                     }
                 }
                 const int s = j % kStateStages;
@@ -207,7 +218,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 if (j == 0 && (int)blockIdx.x == skip_cta) continue;
                 const int64_t vrow = ((it.b * nchunks + it.k) * H + it.h) * (int64_t)Q;
                 mbar_arrive_expect_tx(&sm.bar_x_full[s], (uint32_t)Q * (kRowBytes + 8));
-                tma_load_4d(&sm.Xs[s][0], &tm_x, &sm.bar_x_full[s], 0, it.h, (int)t0, (int)it.b);
+                tma_load_4d(&sm.Xs[s][0], &tm_x, &sm.bar_x_full[s], 0, it.h, row0(t0), (int)it.b);
                 bulk_load(sm.cs_v[s], cs + vrow, Q * 4, &sm.bar_x_full[s]);
                 bulk_load(sm.dt_v[s], dtc + vrow, Q * 4, &sm.bar_x_full[s]);
                 // the tile this stage will hold next: into L2 now, so its load is an L2 hit
@@ -216,7 +227,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     int64_t nt0;
                     int nlen;
                     chunk_span(tab, nx.k, Q, seqlen, nt0, nlen);
-                    tma_prefetch_l2_4d(&tm_x, 0, nx.h, (int)nt0, (int)nx.b);
+                    tma_prefetch_l2_4d(&tm_x, 0, nx.h, pf_row(nt0), (int)nx.b);
                 }
             }
         }
@@ -246,7 +257,15 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                 // loops: the issuing thread's own instruction chain sets the MMA issue rate
                 const uint64_t ad = smem_desc_sw128(smem_u32(&sm.Bs[0][0]), atom_bytes, 1024);
                 const uint64_t bd = smem_desc_sw128(smem_u32(&sm.Xs[s][0]), atom_bytes, 1024);
-                if (Q == 256) {
+                if (kSplit) {   // Q = 64: the rounded rows, then their remainders (8 KB on)
+                    const uint64_t bl = bd + ((64 * kRowBytes) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(d, ad + kk * 128, bd + kk * 128, idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(d, ad + kk * 128, bl + kk * 128, idesc, 1u);
+                } else if (Q == 256) {
 #pragma unroll
                     for (int kk = 0; kk < 16; ++kk)
                         mma_bf16(d, ad + kk * 128, bd + kk * 128, idesc, kk > 0 ? 1u : 0u);
@@ -270,19 +289,27 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             if (!warp_wait(&sm.bar_x_full[s], use & 1, abort)) break;
             const float cs_last = sm.cs_v[s][Q - 1];
             for (int c = st; c < chunks; c += kStateScaleThreads) {
-                const int tau = c >> 3;
+                const int tau = kRev ? Q - 1 - (c >> 3) : c >> 3;   // (reversed) token of the row
                 const float w = __expf(cs_last - sm.cs_v[s][tau]) * sm.dt_v[s][tau];
                 uint4 *ptr = reinterpret_cast<uint4 *>(&sm.Xs[s][0]) + c;
                 uint4 v = *ptr;
                 uint32_t *wv = &v.x;
+                uint4 lo = make_uint4(0u, 0u, 0u, 0u);
+                uint32_t *lv = &lo.x;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 f = __bfloat1622float2(
                         *reinterpret_cast<const __nv_bfloat162 *>(&wv[e]));
                     const float2 sc = fmul2(f, make_float2(w, w));
                     wv[e] = pack_bf16x2(sc.x, sc.y);
+                    if (kSplit) {   // the remainder sc - bf16(sc), rounded to bf16 in turn
+                        const float2 hi = __bfloat1622float2(
+                            *reinterpret_cast<const __nv_bfloat162 *>(&wv[e]));
+                        lv[e] = pack_bf16x2(sc.x - hi.x, sc.y - hi.y);
+                    }
                 }
                 *ptr = v;
+                if (kSplit) ptr[64 * 8] = lo;   // Q = 64: the remainder tile 8 KB on
             }
             fence_async_smem();
             mbar_arrive(&sm.bar_x_ready[s]);
@@ -1060,8 +1087,13 @@ bool tc_supported(bool is_bf16, int P, int N, int Q)
 cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
-                                  cudaStream_t st, const char **why, const int2 *tab)
+                                  cudaStream_t st, const char **why, const int2 *tab, bool split,
+                                  bool rev)
 {
+    if ((split && Q != 64) || (!split && Q != 128 && Q != 256) || (rev && (tab || !split))) {
+        *why = "chunk state: unsupported chunk / split / reversal combination";
+        return cudaErrorInvalidValue;
+    }
     CUtensorMap mx, mb;   // boxes of a whole chunk (Q rows)
     if (!make_seq_map(&mx, x, batch, seqlen, H, kP, Q) ||
         !make_seq_map(&mb, B, batch, seqlen, G, kN, Q)) {
@@ -1074,12 +1106,15 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t smem = sizeof(StateSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(chunk_state_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = !split ? chunk_state_tc_kernel<false, false>
+                       : (rev ? chunk_state_tc_kernel<true, true>
+                              : chunk_state_tc_kernel<true, false>);
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk state: set smem attribute"; return e; }
     const unsigned grid = (unsigned)std::min<int64_t>(sms, nitems);
     *why = "chunk state (tcgen05) launch";
-    return launch_pdl(chunk_state_tc_kernel, grid, kStateThreads, smem, st, mx, mb, dtc, cs,
+    return launch_pdl(kern, grid, kStateThreads, smem, st, mx, mb, dtc, cs,
                       states, status, H, G, Q, nchunks, nitems, seqlen, tab,
                       take_test_skip(kTestChunkState));
 }

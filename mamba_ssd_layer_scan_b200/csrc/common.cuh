@@ -175,10 +175,13 @@ cudaError_t launch_fill_final(const float *init, float *final_state, int64_t n,
 // Tensor-core (tcgen05 + TMA) path: bf16, P = 64, N = 128, Q in {128, 256}.
 bool tc_supported(bool is_bf16, int P, int N, int Q);
 
+// split (Q = 64): the scaled rows as rounded bf16 plus their bf16 remainder, two MMA chains
+// (float32-accurate states); rev: over the time-reversed sequence (rows read backwards).
 cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B,
                                   const float *cs, float *states, int *status, int64_t batch,
                                   int64_t seqlen, int H, int G, int Q, int64_t nchunks,
-                                  cudaStream_t st, const char **why, const int2 *tab = nullptr);
+                                  cudaStream_t st, const char **why, const int2 *tab = nullptr,
+                                  bool split = false, bool rev = false);
 // Offset (in elements), inside one (batch, chunk, head) block of the bf16 entering states, of
 // state element (p, n) for P = 64, N = 128.  The block is stored exactly as the tensor cores
 // read it from shared memory: two halves of 64 n, each 64 rows p of 128 bytes, with the 16-byte
@@ -208,9 +211,6 @@ cudaError_t launch_gather(const bf16 *in, bf16 *out, int64_t batch, int64_t L, i
 cudaError_t launch_reverse_shift_dt(const float *dt, float *out, int64_t batch, int64_t L, int H,
                                    cudaStream_t st);
 cudaError_t launch_fill(float *out, float value, int64_t n, cudaStream_t st);
-// per (b, h) matrix of rows x cols: out = in^T (in [.][rows][cols] -> out [.][cols][rows])
-cudaError_t launch_transpose(const float *in, float *out, int64_t mats, int rows, int cols,
-                             cudaStream_t st);
 // dx[b][t][h][p] = D_h dy + dt[b][t][h] gb[b][L-1-t][h][p];  xdy[b][t][h] = <x, dy>;
 // q[b][t][h] = ydot - dt ddt_in (+ fdot[b][h] = <dfinal, final> at t = L-1; fdot nullable)
 cudaError_t launch_bwd_tokens(const bf16 *x, const bf16 *dy, const float *dt, const float *D,
@@ -226,15 +226,13 @@ cudaError_t launch_state_dot(const float *a, const float *c, float *out, int64_t
 cudaError_t launch_bwd_decay(const float *q, const float *ddt_in, const float *dt,
                              const float *A, const float *xdy, float *ddt, float *dA, float *dD,
                              float *part, int64_t batch, int64_t L, int H, cudaStream_t st);
-// The backward's two float32 scans for P = 64, N = 128 (bwd_scan.cu): x'' (batch, L, G, 128)
-// bf16, B'' and C'' (batch, L, H, 64) bf16, all read at row L-1-tau for scan step tau when
-// `rev`; w (batch, L, H) in scan order, null = 1; cs (batch, nch, H, 64) chunk-local cumsum in
-// scan order; states / hin (batch, nch, H, 128, 64).  The scan writes its output row tau at
-// ys[b][src(tau)][h][:] and its dot product with vg[b][src(tau)][g(h)][:] at dot[b][src(tau)][h].
+// The backward's float32 chunk-output kernel for P = 64, N = 128 (bwd_scan.cu): x''
+// (batch, L, G, 128) bf16, B'' and C'' (batch, L, H, 64) bf16, all read at row L-1-tau for scan
+// step tau when `rev`; w (batch, L, H) in scan order, null = 1; cs (batch, nch, H, 64)
+// chunk-local cumsum in scan order; hin (batch, nch, H, 64, 128), the entering states [p][n].
+// It writes its output row tau at ys[b][src(tau)][h][:] and its dot product with
+// vg[b][src(tau)][g(h)][:] at dot[b][src(tau)][h].
 bool bwd_scan_supported(int P, int N);
-cudaError_t launch_bwd_chunk_state(const bf16 *xg, const bf16 *bh, const float *w,
-                                   const float *cs, float *states, int64_t batch, int64_t L,
-                                   int H, int G, int64_t nch, bool rev, cudaStream_t st);
 cudaError_t launch_bwd_chunk_scan(const bf16 *xg, const bf16 *bh, const bf16 *ch, const float *w,
                                   const float *cs, const float *hin, const bf16 *vg, float *ys,
                                   float *dot, int64_t batch, int64_t L, int H, int G,

@@ -419,9 +419,10 @@ namespace {
 constexpr int kBwdSimtChunk = 64;   // chunk of the two CUDA-core scans (head dim N, state P)
 
 struct BwdLayout {
-    size_t r_ws, s_ws;                          // tensor-core and CUDA-core scan workspaces
+    size_t r_ws, s_ws;                          // the reversed scan's and the dB / dC scans'
+    size_t dtc_s;                               // the dB / dC scans' per-chunk weight rows
     size_t dyr, Cr, Br, dtr, zerosD, gb, Fr;
-    size_t inits, dft, ys, fin_t;               // the CUDA-core scans' states and output
+    size_t ys, fin_s;                           // the dB / dC scans' output and final state
     size_t ydot, ddt_in, q, xdy, fdot, part, total;
     size_t r_bytes, s_bytes;
 };
@@ -448,6 +449,7 @@ BwdLayout bwd_layout(const ssd_shape *s, int Q)
     auto take = [&](size_t bytes) { const size_t at = o; o += round256(bytes); return at; };
     w.r_ws = take(w.r_bytes);   // first: its status word is the workspace's
     w.s_ws = take(w.s_bytes);
+    w.dtc_s = take(b * ((L + kBwdSimtChunk - 1) / kBwdSimtChunk) * H * kBwdSimtChunk * 4);
     w.dyr = take(b * L * H * P * 2);
     w.Cr = take(b * L * G * N * 2);
     w.Br = take(b * L * G * N * 2);
@@ -455,10 +457,8 @@ BwdLayout bwd_layout(const ssd_shape *s, int Q)
     w.zerosD = take(H * 4);
     w.gb = take(b * L * H * P * 2);
     w.Fr = take(b * H * P * N * 4);
-    w.inits = take(b * H * N * P * 4);
-    w.dft = take(b * H * N * P * 4);
     w.ys = take(b * L * H * N * 4);
-    w.fin_t = take(b * H * N * P * 4);
+    w.fin_s = take(b * H * N * P * 4);
     w.ydot = take(b * L * H * 4);
     w.ddt_in = take(b * L * H * 4);
     w.q = take(b * L * H * 4);
@@ -564,9 +564,12 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
     if (dinit && (e = ssd::launch_scale_init_grad(F(wl.Fr), dt, A, dinit, b, L, H, P * N, cst)))
         return cuda_fail(e, "dinit");
 
-    // 2. dB and dC: scans with head dimension N and state dimension P on CUDA cores (float32),
-    // reading the bf16 operands in place, summed over the heads of each group.  Their per-head
-    // outputs also give, contracted with B (resp. C), the two float32 dot products of the decay
+    // 2. dB and dC: scans with head dimension N and state dimension P, summed over the heads of
+    // each group.  Their chunk states come from the tensor-core chunk-state kernel with its
+    // operands swapped (x'' in the place of B, B'' in the place of x) and split into bf16 pairs
+    // (float32-accurate states, stored [p][n] like the forward's); the chunk outputs from the
+    // float32 CUDA-core kernel, which reads the bf16 operands in place.  Their per-head outputs
+    // also give, contracted with B (resp. C), the two float32 dot products of the decay
     // gradient: <x_t, g_t B_t> and <dy_t, y_t - D x_t>.
     const ssd_shape t = simt_shape(s);
     const int Qs = kBwdSimtChunk;
@@ -575,22 +578,22 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
     char *sw = ws + wl.s_ws;
     float *cs_s = reinterpret_cast<float *>(sw + sl.cs);
     float *states_s = reinterpret_cast<float *>(sw + sl.states);
+    float *dtc_s = F(wl.dtc_s);
     for (int pass = 0; pass < 2; ++pass) {   // 0: dB (reversed), 1: dC (forward)
         const bool rev = pass == 0;
-        const float *init_s = rev ? dfinal : init_state;
-        float *init_t = F(rev ? wl.dft : wl.inits);   // dfinal^T is kept for <dfinal, final>
+        const float *init_s = rev ? dfinal : init_state;   // (p, n), as the states
         const float *w_s = rev ? nullptr : dt;
-        if (init_s && (e = ssd::launch_transpose(init_s, init_t, b * H, P, N, cst)))
-            return cuda_fail(e, "transpose");
-        e = ssd::launch_chunk_cumsum(rev ? F(wl.dtr) : dt, A, cs_s, nullptr, nullptr, b, L, H,
-                                     Qs, nchs, cst);
+        // decays from the (reversed, shifted) dt; weights dt (dC) or 1 (dB) as the dt rows
+        e = ssd::launch_chunk_cumsum(rev ? F(wl.dtr) : dt, A, cs_s, dtc_s, nullptr, b, L, H, Qs,
+                                     nchs, cst, nullptr, rev);
+        const char *why = "dB / dC chunk state";
         if (e == cudaSuccess)
-            e = ssd::launch_bwd_chunk_state(rev ? Cb : Bb, rev ? dyb : xb, w_s, cs_s, states_s, b,
-                                            L, H, G, nchs, rev, cst);
+            e = ssd::launch_chunk_state_tc(rev ? dyb : xb, dtc_s, rev ? Cb : Bb, cs_s, states_s,
+                                           status, b, L, H, G, Qs, nchs, cst, &why, nullptr,
+                                           true, rev);
         if (e == cudaSuccess)
-            e = ssd::launch_state_passing(states_s, cs_s, init_s ? init_t : nullptr,
-                                          rev ? nullptr : F(wl.fin_t), nullptr, b, H, N, P, Qs,
-                                          nchs, cst);
+            e = ssd::launch_state_passing(states_s, cs_s, init_s, rev ? nullptr : F(wl.fin_s),
+                                          nullptr, b, H, P, N, Qs, nchs, cst);
         if (e == cudaSuccess)
             e = ssd::launch_bwd_chunk_scan(rev ? Cb : Bb, rev ? dyb : xb, rev ? xb : dyb, w_s,
                                            cs_s, states_s, rev ? Bb : Cb, F(wl.ys),
@@ -604,7 +607,7 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
 
     // 3. dx, the decay-gradient terms and their reverse cumsum: ddt, dA, dD
     // <dfinal, final>, both transposed to (n, p): the final state's share of the decay gradient
-    if (dfinal && (e = ssd::launch_state_dot(F(wl.dft), F(wl.fin_t), F(wl.fdot), b * H, P * N,
+    if (dfinal && (e = ssd::launch_state_dot(dfinal, F(wl.fin_s), F(wl.fdot), b * H, P * N,
                                              cst)))
         return cuda_fail(e, "final-state term");
     if ((e = ssd::launch_bwd_tokens(xb, dyb, dt, D, Hh(wl.gb), F(wl.ydot), F(wl.ddt_in),
