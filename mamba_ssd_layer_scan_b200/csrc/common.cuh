@@ -230,13 +230,17 @@ cudaError_t launch_bwd_decay(const float *q, const float *ddt_in, const float *d
 // (batch, L, G, 128) bf16, B'' and C'' (batch, L, H, 64) bf16, all read at row L-1-tau for scan
 // step tau when `rev`; w (batch, L, H) in scan order, null = 1; cs (batch, nch, H, 64)
 // chunk-local cumsum in scan order; hin (batch, nch, H, 64, 128), the entering states [p][n].
-// It writes its output row tau at ys[b][src(tau)][h][:] and its dot product with
-// vg[b][src(tau)][g(h)][:] at dot[b][src(tau)][h].
+// It writes each head's output row tau's dot product with vg[b][src(tau)][g(h)][:] at
+// dot[b][src(tau)][h].
+// Each CTA takes a run of bwd_scan_heads_per_cta(H, G) heads of one group and writes the sum
+// of their output rows, each weighted by ow[b][src][h] (null = 1), to ys[b][src][run][:]
+// (batch, L, H / heads_per_cta, 128).
 bool bwd_scan_supported(int P, int N);
+int bwd_scan_heads_per_cta(int H, int G);
 cudaError_t launch_bwd_chunk_scan(const bf16 *xg, const bf16 *bh, const bf16 *ch, const float *w,
-                                  const float *cs, const float *hin, const bf16 *vg, float *ys,
-                                  float *dot, int64_t batch, int64_t L, int H, int G,
-                                  int64_t nch, bool rev, cudaStream_t st);
+                                  const float *cs, const float *hin, const bf16 *vg,
+                                  const float *ow, float *ys, float *dot, int64_t batch,
+                                  int64_t L, int H, int G, int64_t nch, bool rev, cudaStream_t st);
 // out[b][t][g][n] = sum_{h in g} w[b][t][h] in[b][src(t)][h][n] (w = dt, or 1 when null)
 cudaError_t launch_group_sum(const float *in, const float *w, float *out, int64_t batch,
                              int64_t L, int H, int G, int N, bool reverse, cudaStream_t st);

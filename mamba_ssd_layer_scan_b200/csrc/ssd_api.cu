@@ -594,13 +594,16 @@ ssd_status ssd_chunk_scan_bwd(const ssd_shape *shape, const void *x, const float
         if (e == cudaSuccess)
             e = ssd::launch_state_passing(states_s, cs_s, init_s, rev ? nullptr : F(wl.fin_s),
                                           nullptr, b, H, P, N, Qs, nchs, cst);
+        // the chunk outputs, summed over runs of heads (weighted by dt for dB), then the runs'
+        // partial sums over each group
+        const int hpc = ssd::bwd_scan_heads_per_cta(H, G);
         if (e == cudaSuccess)
             e = ssd::launch_bwd_chunk_scan(rev ? Cb : Bb, rev ? dyb : xb, rev ? xb : dyb, w_s,
-                                           cs_s, states_s, rev ? Bb : Cb, F(wl.ys),
-                                           F(rev ? wl.ddt_in : wl.ydot), b, L, H, G, nchs, rev,
-                                           cst);
+                                           cs_s, states_s, rev ? Bb : Cb, rev ? dt : nullptr,
+                                           F(wl.ys), F(rev ? wl.ddt_in : wl.ydot), b, L, H, G,
+                                           nchs, rev, cst);
         if (e == cudaSuccess)
-            e = ssd::launch_group_sum(F(wl.ys), rev ? dt : nullptr, rev ? dB : dC, b, L, H, G, N,
+            e = ssd::launch_group_sum(F(wl.ys), nullptr, rev ? dB : dC, b, L, H / hpc, G, N,
                                       false, cst);
         if (e != cudaSuccess) return cuda_fail(e, rev ? "dB scan" : "dC scan");
     }
