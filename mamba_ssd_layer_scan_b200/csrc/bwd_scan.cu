@@ -1,5 +1,5 @@
-// The chunk-output kernel of the backward pass's two scans (dB and dC), in float32,
-// specialised for their shape.
+// The chunk-output kernel of the backward pass's two scans (dB and dC), specialised for their
+// shape.
 //
 // Both scans are of the forward's kind with the head and state dimensions swapped: the state
 // is K x E = P x N (64 x 128) per (batch, head), stored [j][e] like the forward's [p][n]; the
@@ -14,16 +14,11 @@
 // dB runs it on the time-reversed sequence (x'' = C, B'' = dy, C'' = x, unit weights, decays
 // shifted by one token), dC forward (x'' = B, B'' = x, C'' = dy, weights dt).  The chunk states
 // come from the tensor-core chunk-state kernel (chunk_tc.cu) with split bf16 operands; this
-// kernel forms the chunk outputs.  It reads the operands in place from the bf16 inputs
-// (reversed rows, the group's row for x''); everything is float32 from there on, because the
-// decay gradient needs the outputs' dot products with B and C to float32 accuracy (see
-// backward.cu).  Each output row's dot product with the group's B or C row is formed in the
-// epilogue.
-//
-// Register tiling: each thread holds 4 rows x 8 channels of the 64 x 128 output tile, and 4 x 4
-// of the 64 x 64 masked Gram matrix before that.  The channels of a thread are two runs of 4 at
-// e0 and 64 + e0, so that each 16-byte shared-memory load of a half warp reads 256 contiguous
-// bytes (two wavefronts, no bank conflict).
+// kernel forms the chunk outputs, reading the operands in place from the bf16 inputs (reversed
+// rows, the group's row for x'').  The decay gradient needs the outputs' dot products with B
+// and C to float32 accuracy (see backward.cu), so every operand that is not bf16 already is
+// split into two bf16 parts, and every product accumulates in float32.  Each output row's dot
+// product with the group's B or C row is formed in the epilogue.
 #include "common.cuh"
 
 namespace ssd {
@@ -33,7 +28,6 @@ constexpr int kQs = 64;     // chunk
 constexpr int kE = 128;     // x'' channels (dstate of the forward)
 constexpr int kK = 64;      // B'' / C'' channels (headdim of the forward)
 constexpr int kThreads = 256;
-constexpr int kTS = kQs + 4;   // row stride of the transposed [channel][token] tiles
 
 __device__ __forceinline__ void unpack8(const uint4 raw, float *v)
 {
@@ -47,214 +41,274 @@ __device__ __forceinline__ int64_t src_row(int64_t tau, int64_t L, bool rev)
     return rev ? L - 1 - tau : tau;
 }
 
-// x'' and C'' are bf16 inputs and stay bf16 here (exact); B'' * w, the Gram matrix and the
-// entering state are float32.  74 KB: three CTAs per SM.
-struct ScanSmem {
-    bf16 xs[kQs][kE];         // x'' rows
-    union {
-        float bT[kK][kTS];    // B'' * w transposed: bT[j][s] (until the Gram matrix is formed)
-        float pT[kQs][kTS];   // masked, decayed Gram matrix, transposed: pT[s][t]
-    };
-    bf16 cT[kK][kTS];         // C'' transposed: cT[j][t]
-    float hT[kK][kE];         // entering state transposed: hT[j][e]
+// The chunk outputs on warp-level bf16 tensor-core products (mma.sync m16n8k16, float32
+// accumulate).  The operands that are not bf16 already -- w B'' (the Gram matrix's right
+// factor), the masked Gram matrix P and the entering state S -- are split into their bf16
+// rounding and the bf16 rounding of the remainder, and each product with them runs as two
+// chains into the same float32 accumulator, which keeps the outputs to about float32 accuracy.
+// Per head, with 8 warps:
+//   G = C'' (w B'')^T       64 x 64, K = 64: warp (mt, nh) the rows 16 mt.., columns 32 nh..
+//   P = G o decay o causal  masked in registers, split, stored [t][s]
+//   Y = exp(cs_t) C'' S + P x''   64 x 128: warp (mt, nh) the rows 16 mt.., columns 64 nh..
+// Fragment layouts are those of the PTX ISA for mma.m16n8k16 (row-major A, column-major B);
+// ldmatrix loads them from shared-memory tiles whose row pitches (144 and 272 bytes) put the 8
+// rows of each 8 x 8 matrix in distinct bank groups.
+constexpr int kPA = 72;    // row pitch (elements) of the 64-column bf16 tiles
+constexpr int kPB = 136;   // row pitch of the 128-column bf16 tiles
+struct MmaSmem {
+    bf16 xm[kQs][kPB];        // x'' rows [s][e], the group's (once per CTA)
+    bf16 cm[kQs][kPA];        // C'' rows [t][j]
+    bf16 bw[2][kQs][kPA];     // w B'' rows [s][j], split; then P [t][s], split
+    bf16 st[2][kK][kPB];      // entering state [j][e], split
     float css[kQs];           // chunk-local cumsum
+    float dotp[2][kQs];       // per column half: the rows' partial dot products with V
 };
 
-// four bf16 (8 bytes) -> float32, exactly: the bf16 bits are the float's upper half
-__device__ __forceinline__ void bf16x4_to_f32(const uint2 r, float *v)
+__device__ __forceinline__ uint32_t sh_addr(const void *p)
 {
-    v[0] = __uint_as_float(r.x << 16);
-    v[1] = __uint_as_float(r.x & 0xffff0000u);
-    v[2] = __uint_as_float(r.y << 16);
-    v[3] = __uint_as_float(r.y & 0xffff0000u);
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-static_assert(kK == kQs, "bT and pT share their storage");
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(sh_addr(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void *p)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(sh_addr(p)));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+                 "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// two floats -> their bf16 roundings (hi) and the bf16 roundings of the remainders (lo), each
+// pair packed with the first value in the low half
+__device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x - hf.x, y - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
 
-// One CTA per (batch, chunk, run of kHPC heads of one group): the group's x'' rows are loaded
-// once, the heads are taken in turn, and their output rows -- weighted by ow (dt for dB, 1 for
-// dC) -- are summed in registers, so the CTA writes one partial sum of the group's output per
-// run of heads (the group sum then adds H / G / kHPC partials instead of H / G outputs).
 template <int kHPC>
-__global__ void __launch_bounds__(kThreads, kHPC > 1 ? 2 : 3)
-bwd_chunk_scan_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
-                      const bf16 *__restrict__ ch, const float *__restrict__ w,
-                      const float *__restrict__ cs, const float *__restrict__ hin,
-                      const bf16 *__restrict__ vg, const float *__restrict__ ow,
-                      float *__restrict__ ys, float *__restrict__ dot, int64_t L, int H, int G,
-                      int64_t nch, bool rev)
+__global__ void __launch_bounds__(kThreads, 2)
+bwd_chunk_scan_mma_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ bh,
+                          const bf16 *__restrict__ ch, const float *__restrict__ w,
+                          const float *__restrict__ cs, const float *__restrict__ hin,
+                          const bf16 *__restrict__ vg, const float *__restrict__ ow,
+                          float *__restrict__ ys, float *__restrict__ dot, int64_t L, int H,
+                          int G, int64_t nch, bool rev)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    ScanSmem &sm = *reinterpret_cast<ScanSmem *>(smem_raw);
-    const int nhb = H / kHPC;                      // runs of heads
+    MmaSmem &sm = *reinterpret_cast<MmaSmem *>(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g8 = lane >> 2, c4 = lane & 3;   // fragment row and column pair
+    const int mt = warp & 3, nh = warp >> 2;   // this warp's row tile and column half
+    const int nhb = H / kHPC;
     const int hb = (int)(blockIdx.x % nhb);
     const int64_t k = (blockIdx.x / nhb) % nch, b = blockIdx.x / nhb / nch;
     const int g = hb * kHPC / (H / G);
     const int64_t t0 = k * kQs;
     const int len = (int)min((int64_t)kQs, L - t0);
 
-    for (int i = threadIdx.x; i < kQs * kE / 8; i += kThreads) {
+    for (int i = threadIdx.x; i < kQs * kE / 8; i += kThreads) {   // x'' rows, once
         const int r = i / (kE / 8), c8 = i % (kE / 8);
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (r < len) {
             const int64_t s = src_row(t0 + r, L, rev);
             v = *reinterpret_cast<const uint4 *>(xg + ((b * L + s) * G + g) * kE + c8 * 8);
         }
-        *reinterpret_cast<uint4 *>(&sm.xs[r][c8 * 8]) = v;
+        *reinterpret_cast<uint4 *>(&sm.xm[r][c8 * 8]) = v;
     }
 
-    // output rows tg..tg+3, channels e0..e0+3 and 64+e0..64+e0+3 (each 16-byte shared-memory load
-    // of a half warp covers 256 contiguous bytes)
-    const int tg = (threadIdx.x / 16) * 4, e0 = (threadIdx.x % 16) * 4;
-    float tot[4][8];
+    float tot[8][4];   // the run's weighted sum of output fragments (8 column tiles of 8)
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int n = 0; n < 8; ++n)
 #pragma unroll
-        for (int m = 0; m < 8; ++m) tot[i][m] = 0.f;
+        for (int q = 0; q < 4; ++q) tot[n][q] = 0.f;
 
     for (int hh = 0; hh < kHPC; ++hh) {
         const int h = hb * kHPC + hh;
         const float *csk = cs + ((b * nch + k) * H + h) * (int64_t)kQs;
         const float *hk = hin + ((b * nch + k) * H + h) * (int64_t)(kE * kK);
-        if (hh > 0) __syncthreads();   // the previous head is done with css, bT / pT, cT, hT
+        if (hh > 0) __syncthreads();   // the previous head is done with css, cm, bw, st, dotp
         if (threadIdx.x < kQs) sm.css[threadIdx.x] = threadIdx.x < len ? csk[threadIdx.x] : 0.f;
-        for (int i = threadIdx.x; i < kQs * kK / 8; i += kThreads) {
-            const int r = i % kQs, c8 = i / kQs;   // consecutive threads: consecutive tokens, so
-                                                   // the transposed stores below hit distinct banks
-            float vb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            uint4 rc = make_uint4(0u, 0u, 0u, 0u);
+        for (int i = threadIdx.x; i < kQs * kK / 8; i += kThreads) {   // C'' and w B'' rows
+            const int r = i / (kK / 8), c8 = i % (kK / 8);
+            uint4 cv = make_uint4(0u, 0u, 0u, 0u), bhi = cv, blo = cv;
             if (r < len) {
                 const int64_t tau = t0 + r, s = src_row(tau, L, rev);
                 const int64_t off = ((b * L + s) * H + h) * kK + c8 * 8;
+                cv = *reinterpret_cast<const uint4 *>(ch + off);
+                float vb[8];
                 unpack8(*reinterpret_cast<const uint4 *>(bh + off), vb);
-                rc = *reinterpret_cast<const uint4 *>(ch + off);
                 const float f = w ? w[(b * L + tau) * H + h] : 1.f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) vb[j] *= f;
+                split2(vb[0] * f, vb[1] * f, bhi.x, blo.x);
+                split2(vb[2] * f, vb[3] * f, bhi.y, blo.y);
+                split2(vb[4] * f, vb[5] * f, bhi.z, blo.z);
+                split2(vb[6] * f, vb[7] * f, bhi.w, blo.w);
             }
-            const bf16 *pc = reinterpret_cast<const bf16 *>(&rc);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                sm.bT[c8 * 8 + j][r] = vb[j];
-                sm.cT[c8 * 8 + j][r] = pc[j];
-            }
+            *reinterpret_cast<uint4 *>(&sm.cm[r][c8 * 8]) = cv;
+            *reinterpret_cast<uint4 *>(&sm.bw[0][r][c8 * 8]) = bhi;
+            *reinterpret_cast<uint4 *>(&sm.bw[1][r][c8 * 8]) = blo;
         }
-        for (int i = threadIdx.x; i < kE * kK / 4; i += kThreads) {   // [j][e]: a plain copy
+        for (int i = threadIdx.x; i < kK * kE / 4; i += kThreads) {   // entering state, split
             const int j = i / (kE / 4), e4 = i % (kE / 4);
-            *reinterpret_cast<float4 *>(&sm.hT[j][e4 * 4]) =
-                *reinterpret_cast<const float4 *>(hk + j * kE + e4 * 4);
+            const float4 v = *reinterpret_cast<const float4 *>(hk + j * kE + e4 * 4);
+            uint2 hi, lo;
+            split2(v.x, v.y, hi.x, lo.x);
+            split2(v.z, v.w, hi.y, lo.y);
+            *reinterpret_cast<uint2 *>(&sm.st[0][j][e4 * 4]) = hi;
+            *reinterpret_cast<uint2 *>(&sm.st[1][j][e4 * 4]) = lo;
         }
         __syncthreads();
 
-        // masked, decayed Gram matrix P[t][s] = (C''_t . w_s B''_s) exp(cs_t - cs_s), s <= t < len
+        // G = C'' (w B'')^T for rows 16 mt.., columns 32 nh.. (none above the diagonal)
+        const bool gram_on = 16 * mt + 15 >= 32 * nh;
+        float gacc[4][4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) gacc[n][q] = 0.f;
+        if (gram_on) {
+#pragma unroll
+            for (int kk = 0; kk < kK / 16; ++kk) {
+                uint32_t a[4];
+                ldsm_x4(a, &sm.cm[16 * mt + (lane & 15)][16 * kk + (lane >> 4) * 8]);
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int np = 0; np < 2; ++np) {
+                        uint32_t bb[4];
+                        const int n0 = 32 * nh + 16 * np;
+                        ldsm_x4(bb, &sm.bw[part][n0 + (lane & 7) + ((lane >> 4) << 3)]
+                                              [16 * kk + ((lane >> 3) & 1) * 8]);
+                        mma16816(gacc[2 * np], a, bb[0], bb[1]);
+                        mma16816(gacc[2 * np + 1], a, bb[2], bb[3]);
+                    }
+            }
+        }
+        __syncthreads();   // every read of w B'' is done before P overwrites it
+        if (gram_on) {     // P = G exp(cs_t - cs_s) for s <= t < len, else 0; split, [t][s]
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int t = 16 * mt + g8 + 8 * half;
+                    const int s0 = 32 * nh + 8 * n + 2 * c4;
+                    const float ct = sm.css[t];
+                    const float p0 = (s0 <= t && t < len)
+                                         ? gacc[n][2 * half] * __expf(ct - sm.css[s0]) : 0.f;
+                    const float p1 = (s0 + 1 <= t && t < len)
+                                         ? gacc[n][2 * half + 1] * __expf(ct - sm.css[s0 + 1])
+                                         : 0.f;
+                    uint32_t hi, lo;
+                    split2(p0, p1, hi, lo);
+                    *reinterpret_cast<uint32_t *>(&sm.bw[0][t][s0]) = hi;
+                    *reinterpret_cast<uint32_t *>(&sm.bw[1][t][s0]) = lo;
+                }
+        }
+        __syncthreads();
+
+        // Y for rows 16 mt.., columns 64 nh..: the entering state's term, scaled by exp(cs_t),
+        // then P x'' (source columns s <= 16 mt + 15 only)
+        float acc[8][4];
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[n][q] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < kK / 16; ++kk) {
+            uint32_t a[4];
+            ldsm_x4(a, &sm.cm[16 * mt + (lane & 15)][16 * kk + (lane >> 4) * 8]);
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int np = 0; np < 4; ++np) {
+                    uint32_t bb[4];
+                    const int n0 = 64 * nh + 16 * np;
+                    ldsm_x4_t(bb, &sm.st[part][16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8]
+                                             [n0 + (lane >> 4) * 8]);
+                    mma16816(acc[2 * np], a, bb[0], bb[1]);
+                    mma16816(acc[2 * np + 1], a, bb[2], bb[3]);
+                }
+        }
         {
-            const int ta = (threadIdx.x / 16) * 4, sa = (threadIdx.x % 16) * 4;
-            float gm[4][4];
+            const float d0 = __expf(sm.css[16 * mt + g8]), d1 = __expf(sm.css[16 * mt + g8 + 8]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) gm[i][j] = 0.f;
-            if (sa <= ta + 3) {
-                for (int j = 0; j < kK; ++j) {
-                    float ca[4];
-                    bf16x4_to_f32(*reinterpret_cast<const uint2 *>(&sm.cT[j][ta]), ca);
-                    const float4 bb = *reinterpret_cast<const float4 *>(&sm.bT[j][sa]);
-                    const float ba[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) gm[i][q] = fmaf(ca[i], ba[q], gm[i][q]);
-                }
-            }
-            __syncthreads();   // every read of bT is done before pT overwrites it
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int s = sa + q;
-                float o[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int t = ta + i;
-                    o[i] = (s <= t && t < len) ? gm[i][q] * __expf(sm.css[t] - sm.css[s]) : 0.f;
-                }
-                *reinterpret_cast<float4 *>(&sm.pT[s][ta]) = make_float4(o[0], o[1], o[2], o[3]);
+            for (int n = 0; n < 8; ++n) {
+                acc[n][0] *= d0;
+                acc[n][1] *= d0;
+                acc[n][2] *= d1;
+                acc[n][3] *= d1;
             }
         }
-        __syncthreads();
-
-        // first the entering state's term exp(cs_t) sum_j C''_t[j] S_in[j][e], scaled in
-        // registers, then the masked P X on top
-        float acc[4][8];
+        for (int kk = 0; kk <= mt; ++kk) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+            for (int part = 0; part < 2; ++part) {
+                uint32_t a[4];
+                ldsm_x4(a, &sm.bw[part][16 * mt + (lane & 15)][16 * kk + (lane >> 4) * 8]);
 #pragma unroll
-            for (int m = 0; m < 8; ++m) acc[i][m] = 0.f;
-        for (int j = 0; j < kK; ++j) {
-            float ca[4];
-            bf16x4_to_f32(*reinterpret_cast<const uint2 *>(&sm.cT[j][tg]), ca);
-            const float4 h0 = *reinterpret_cast<const float4 *>(&sm.hT[j][e0]);
-            const float4 h1 = *reinterpret_cast<const float4 *>(&sm.hT[j][64 + e0]);
-            const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int m = 0; m < 8; ++m) acc[i][m] = fmaf(ca[i], hv[m], acc[i][m]);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float dec = __expf(sm.css[tg + i]);
-#pragma unroll
-            for (int m = 0; m < 8; ++m) acc[i][m] *= dec;
-        }
-        const int smax = min(len, tg + 4);
-        for (int s = 0; s < smax; ++s) {
-            const float4 p = *reinterpret_cast<const float4 *>(&sm.pT[s][tg]);
-            const float pa[4] = {p.x, p.y, p.z, p.w};
-            float xv[8];
-            bf16x4_to_f32(*reinterpret_cast<const uint2 *>(&sm.xs[s][e0]), xv);
-            bf16x4_to_f32(*reinterpret_cast<const uint2 *>(&sm.xs[s][64 + e0]), xv + 4);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int m = 0; m < 8; ++m) acc[i][m] = fmaf(pa[i], xv[m], acc[i][m]);
+                for (int np = 0; np < 4; ++np) {
+                    uint32_t bb[4];
+                    const int n0 = 64 * nh + 16 * np;
+                    ldsm_x4_t(bb, &sm.xm[16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8]
+                                        [n0 + (lane >> 4) * 8]);
+                    mma16816(acc[2 * np], a, bb[0], bb[1]);
+                    mma16816(acc[2 * np + 1], a, bb[2], bb[3]);
+                }
+            }
         }
 
-        // this head's rows: the dot with the group's V row (at the row's source token), and
-        // the weighted sum over the run of heads
+        // this head's rows: the dot with the group's V row (at the row's source token), and the
+        // weighted sum over the run of heads
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = tg + i;
+        for (int half = 0; half < 2; ++half) {
+            const int t = 16 * mt + g8 + 8 * half;
             const bool valid = t < len;
             const int64_t s = valid ? src_row(t0 + t, L, rev) : 0;
             float d = 0.f;
             if (valid) {
-                const bf16 *vrow = vg + ((b * L + s) * G + g) * (int64_t)kE + e0;
-                const uint2 r0 = *reinterpret_cast<const uint2 *>(vrow);
-                const uint2 r1 = *reinterpret_cast<const uint2 *>(vrow + 64);
-                float v[8];
-                bf16x4_to_f32(r0, v);
-                bf16x4_to_f32(r1, v + 4);
-#pragma unroll
-                for (int m = 0; m < 8; ++m) d = fmaf(acc[i][m], v[m], d);
+                const bf16 *vrow = vg + ((b * L + s) * G + g) * (int64_t)kE + 64 * nh + 2 * c4;
                 const float wo = ow ? ow[(b * L + s) * H + h] : 1.f;
 #pragma unroll
-                for (int m = 0; m < 8; ++m) tot[i][m] = fmaf(wo, acc[i][m], tot[i][m]);
+                for (int n = 0; n < 8; ++n) {
+                    const float2 v = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162 *>(vrow + 8 * n));
+                    d = fmaf(acc[n][2 * half], v.x, d);
+                    d = fmaf(acc[n][2 * half + 1], v.y, d);
+                    tot[n][2 * half] = fmaf(wo, acc[n][2 * half], tot[n][2 * half]);
+                    tot[n][2 * half + 1] = fmaf(wo, acc[n][2 * half + 1], tot[n][2 * half + 1]);
+                }
             }
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-            if (valid && e0 == 0) dot[(b * L + s) * H + h] = d;
+            d += __shfl_xor_sync(0xffffffffu, d, 1);
+            d += __shfl_xor_sync(0xffffffffu, d, 2);
+            if (c4 == 0) sm.dotp[nh][t] = d;
         }
+        __syncthreads();
+        if (threadIdx.x < len)
+            dot[(b * L + src_row(t0 + threadIdx.x, L, rev)) * H + h] =
+                sm.dotp[0][threadIdx.x] + sm.dotp[1][threadIdx.x];
     }
 
     // the run's partial sum of the group's output, at the rows' source tokens (forward time)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int t = tg + i;
+    for (int half = 0; half < 2; ++half) {
+        const int t = 16 * mt + g8 + 8 * half;
         if (t >= len) continue;
         const int64_t s = src_row(t0 + t, L, rev);
-        float *yrow = ys + ((b * L + s) * nhb + hb) * (int64_t)kE + e0;
-        *reinterpret_cast<float4 *>(yrow) =
-            make_float4(tot[i][0], tot[i][1], tot[i][2], tot[i][3]);
-        *reinterpret_cast<float4 *>(yrow + 64) =
-            make_float4(tot[i][4], tot[i][5], tot[i][6], tot[i][7]);
+        float *yrow = ys + ((b * L + s) * nhb + hb) * (int64_t)kE + 64 * nh + 2 * c4;
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+            *reinterpret_cast<float2 *>(yrow + 8 * n) =
+                make_float2(tot[n][2 * half], tot[n][2 * half + 1]);
     }
 }
 
@@ -276,9 +330,9 @@ cudaError_t launch_bwd_chunk_scan(const bf16 *xg, const bf16 *bh, const bf16 *ch
     const int hpc = bwd_scan_heads_per_cta(H, G);
     const int64_t n = batch * nch * (H / hpc);
     if (n == 0) return cudaSuccess;
-    const int smem = (int)sizeof(ScanSmem);
-    auto kern = hpc == 4 ? bwd_chunk_scan_kernel<4>
-                         : (hpc == 2 ? bwd_chunk_scan_kernel<2> : bwd_chunk_scan_kernel<1>);
+    const int smem = (int)sizeof(MmaSmem);
+    auto kern = hpc == 4 ? bwd_chunk_scan_mma_kernel<4>
+                         : (hpc == 2 ? bwd_chunk_scan_mma_kernel<2> : bwd_chunk_scan_mma_kernel<1>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)n, kThreads, smem, st>>>(xg, bh, ch, w, cs, hin, vg, ow, ys, dot, L, H, G,
