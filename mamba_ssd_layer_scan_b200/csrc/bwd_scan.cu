@@ -60,6 +60,7 @@ struct MmaSmem {
     bf16 cm[kQs][kPA];        // C'' rows [t][j]
     bf16 bw[2][kQs][kPA];     // w B'' rows [s][j], split; then P [t][s], split
     bf16 st[2][kK][kPB];      // entering state [j][e], split
+    float sf[kK][kE];         // the entering state as loaded (float32), fetched one head ahead
     float css[kQs];           // chunk-local cumsum
     float dotp[2][kQs];       // per column half: the rows' partial dot products with V
 };
@@ -78,6 +79,15 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void *p)
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(sh_addr(p)));
 }
+// 16-byte global -> shared copies that complete asynchronously (cp.async), in one group
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sh_addr(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1)
 {
@@ -117,6 +127,15 @@ bwd_chunk_scan_mma_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ 
     const int g = hb * kHPC / (H / G);
     const int64_t t0 = k * kQs;
     const int len = (int)min((int64_t)kQs, L - t0);
+    // the entering state of the run's head hh into sf, asynchronously
+    auto fetch_state = [&](int hh) {
+        const float *hk =
+            hin + ((b * nch + k) * H + hb * kHPC + hh) * (int64_t)(kE * kK);
+        for (int i = threadIdx.x; i < kK * kE / 4; i += kThreads)
+            cp_async16(&sm.sf[0][0] + 4 * i, hk + 4 * i);
+        cp_async_commit();
+    };
+    fetch_state(0);
 
     for (int i = threadIdx.x; i < kQs * kE / 8; i += kThreads) {   // x'' rows, once
         const int r = i / (kE / 8), c8 = i % (kE / 8);
@@ -137,8 +156,9 @@ bwd_chunk_scan_mma_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ 
     for (int hh = 0; hh < kHPC; ++hh) {
         const int h = hb * kHPC + hh;
         const float *csk = cs + ((b * nch + k) * H + h) * (int64_t)kQs;
-        const float *hk = hin + ((b * nch + k) * H + h) * (int64_t)(kE * kK);
         if (hh > 0) __syncthreads();   // the previous head is done with css, cm, bw, st, dotp
+        cp_async_wait_all();           // this head's entering state (every thread's part) ...
+        __syncthreads();               // ... is in sf
         if (threadIdx.x < kQs) sm.css[threadIdx.x] = threadIdx.x < len ? csk[threadIdx.x] : 0.f;
         for (int i = threadIdx.x; i < kQs * kK / 8; i += kThreads) {   // C'' and w B'' rows
             const int r = i / (kK / 8), c8 = i % (kK / 8);
@@ -161,7 +181,7 @@ bwd_chunk_scan_mma_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ 
         }
         for (int i = threadIdx.x; i < kK * kE / 4; i += kThreads) {   // entering state, split
             const int j = i / (kE / 4), e4 = i % (kE / 4);
-            const float4 v = *reinterpret_cast<const float4 *>(hk + j * kE + e4 * 4);
+            const float4 v = *reinterpret_cast<const float4 *>(&sm.sf[j][e4 * 4]);
             uint2 hi, lo;
             split2(v.x, v.y, hi.x, lo.x);
             split2(v.z, v.w, hi.y, lo.y);
@@ -169,6 +189,7 @@ bwd_chunk_scan_mma_kernel(const bf16 *__restrict__ xg, const bf16 *__restrict__ 
             *reinterpret_cast<uint2 *>(&sm.st[1][j][e4 * 4]) = lo;
         }
         __syncthreads();
+        if (hh + 1 < kHPC) fetch_state(hh + 1);   // sf is free: lands while this head computes
 
         // G = C'' (w B'')^T for rows 16 mt.., columns 32 nh.. (none above the diagonal)
         const bool gram_on = 16 * mt + 15 >= 32 * nh;
