@@ -340,7 +340,7 @@ bool bwd_scan_supported(int P, int N) { return P == kK && N == kE; }
 int bwd_scan_heads_per_cta(int H, int G)
 {
     const int hpg = H / G;
-    return hpg % 4 == 0 ? 4 : (hpg % 2 == 0 ? 2 : 1);
+    return hpg % 8 == 0 ? 8 : (hpg % 4 == 0 ? 4 : (hpg % 2 == 0 ? 2 : 1));
 }
 
 cudaError_t launch_bwd_chunk_scan(const bf16 *xg, const bf16 *bh, const bf16 *ch, const float *w,
@@ -352,7 +352,8 @@ cudaError_t launch_bwd_chunk_scan(const bf16 *xg, const bf16 *bh, const bf16 *ch
     const int64_t n = batch * nch * (H / hpc);
     if (n == 0) return cudaSuccess;
     const int smem = (int)sizeof(MmaSmem);
-    auto kern = hpc == 4 ? bwd_chunk_scan_mma_kernel<4>
+    auto kern = hpc == 8 ? bwd_chunk_scan_mma_kernel<8>
+                : hpc == 4 ? bwd_chunk_scan_mma_kernel<4>
                          : (hpc == 2 ? bwd_chunk_scan_mma_kernel<2> : bwd_chunk_scan_mma_kernel<1>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

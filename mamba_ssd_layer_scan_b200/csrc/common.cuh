@@ -232,9 +232,9 @@ cudaError_t launch_bwd_decay(const float *q, const float *ddt_in, const float *d
 // chunk-local cumsum in scan order; hin (batch, nch, H, 64, 128), the entering states [p][n].
 // It writes each head's output row tau's dot product with vg[b][src(tau)][g(h)][:] at
 // dot[b][src(tau)][h].
-// Each CTA takes a run of bwd_scan_heads_per_cta(H, G) heads of one group and writes the sum
-// of their output rows, each weighted by ow[b][src][h] (null = 1), to ys[b][src][run][:]
-// (batch, L, H / heads_per_cta, 128).
+// Each CTA takes a run of bwd_scan_heads_per_cta(H, G) (8, 4, 2 or 1) heads of one group and
+// writes the sum of their output rows, each weighted by ow[b][src][h] (null = 1), to
+// ys[b][src][run][:] (batch, L, H / heads_per_cta, 128).
 bool bwd_scan_supported(int P, int N);
 int bwd_scan_heads_per_cta(int H, int G);
 cudaError_t launch_bwd_chunk_scan(const bf16 *xg, const bf16 *bh, const bf16 *ch, const float *w,

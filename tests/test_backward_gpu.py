@@ -62,6 +62,10 @@ CASES = [
                                              init_state=True, seed=79), 256, True, True),
     ("one_token", configs.SSD_370M.with_(batch=2, seqlen=1, nheads=4, init_state=True, seed=80),
      256, True, True),
+    # three heads per group: the dB / dC chunk outputs take one head per CTA
+    ("q256_three_heads_per_group", configs.SSD_370M.with_(batch=2, seqlen=300, nheads=6,
+                                                          ngroups=2, init_state=True, seed=81),
+     256, True, True),
 ]
 
 
