@@ -50,6 +50,11 @@ __device__ __forceinline__ int64_t src_row(int64_t tau, int64_t L, bool rev)
 //   G = C'' (w B'')^T       64 x 64, K = 64: warp (mt, nh) the rows 16 mt.., columns 32 nh..
 //   P = G o decay o causal  masked in registers, split, stored [t][s]
 //   Y = exp(cs_t) C'' S + P x''   64 x 128: warp (mt, nh) the rows 16 mt.., columns 64 nh..
+// One CTA per (batch, chunk, run of kHPC heads of one group): the group's x'' rows are loaded
+// once, the heads are taken in turn (the next head's entering state fetched with cp.async while
+// the current one computes), and their output rows, weighted by ow (dt for dB, 1 for dC), are
+// summed in registers, so the CTA writes one partial sum of the group's output per run (the
+// group sum then adds H / G / kHPC partials).
 // Fragment layouts are those of the PTX ISA for mma.m16n8k16 (row-major A, column-major B);
 // ldmatrix loads them from shared-memory tiles whose row pitches (144 and 272 bytes) put the 8
 // rows of each 8 x 8 matrix in distinct bank groups.
