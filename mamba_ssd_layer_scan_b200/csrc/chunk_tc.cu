@@ -453,20 +453,25 @@ __device__ __forceinline__ void scale_pieces(uint8_t *base, int first, int strid
 
 // Work of one launch: for each 128-row tile class T of the chunks (T = 1, the tiles with an
 // off-diagonal block, exists for Q = 256), the flat list of (batch, chunk, group, head) items,
-// heads of a group consecutive.  One CTA per SM: CTAs [0, ncta1) take the T = 1 items, the rest
-// the T = 0 items, each an equal run of its class's list.  For Q = 256 the two classes get the
-// same number of CTAs and the same runs, so CTA i of each class walks the same heads in the same
-// order at about the same time: both tiles of a head read x rows 0-127 and the head's entering
-// state, and the second read is then an L2 hit (with the classes split unevenly it was not:
-// 415 MB of DRAM reads per launch at the 2.7B shape instead of 271 MB).  A run of items of the
-// same (batch, chunk, group) is a segment: its heads share the C and B tiles and C B^T, which
+// heads of a group consecutive.  One CTA per SM: CTAs [0, ncta1) take the T = 1 items, the next
+// ones the T = 0 items, each an equal run of its class's list.  For Q = 256 the two classes get
+// the same number of CTAs and the same runs, so CTA i of each class walks the same heads in the
+// same order at about the same time: both tiles of a head read x rows 0-127 and the head's
+// entering state, and the second read is then an L2 hit (with the classes split unevenly it was
+// not: 415 MB of DRAM reads per launch at the 2.7B shape instead of 271 MB).  A second tile
+// costs more than a first (twice the mask and P x work, and the scaling of x_off), so the last
+// tail_q / 1024 of each second-tile run goes to a third group of CTAs, [2 ncta1, 3 ncta1).
+// With one CTA per SM these start only as SMs free up, which the first-tile CTAs do first, when
+// the second-tile CTAs are nearly at their tails: both classes then end together, and the
+// tails' x rows are still in L2.  No CTA waits for another, so the order in which the CTAs
+// start matters for time only.  A run of items of the same (batch, chunk, group) is a segment: its heads share the C and B tiles and C B^T, which
 // the CTA computes once per segment; the per-head pipeline runs on across segments, its barrier
 // phases counted by a head counter that does not restart.
 struct ScanWork {
     int T;               // tile class of this CTA
     int64_t f0, f1;      // its run of items
 };
-__device__ __forceinline__ ScanWork scan_work(int nT, int ncta1, int64_t nitems)
+__device__ __forceinline__ ScanWork scan_work(int nT, int ncta1, int64_t nitems, int tail_q)
 {
     ScanWork w;
     int idx = blockIdx.x, m = gridDim.x;
@@ -477,11 +482,18 @@ __device__ __forceinline__ ScanWork scan_work(int nT, int ncta1, int64_t nitems)
         w.T = 0;
         if (nT == 2) {
             idx -= ncta1;
-            m -= ncta1;
+            m = ncta1;
         }
     }
-    w.f0 = (int64_t)idx * nitems / m;
-    w.f1 = ((int64_t)idx + 1) * nitems / m;
+    const int tail = nT == 2 && idx >= m;   // the tails of the second-tile runs
+    if (tail) {
+        w.T = 1;
+        idx -= m;
+    }
+    const int64_t f0 = (int64_t)idx * nitems / m, f1 = ((int64_t)idx + 1) * nitems / m;
+    const int64_t nt = w.T ? (f1 - f0) * tail_q / 1024 : 0;
+    w.f0 = tail ? f1 - nt : f0;
+    w.f1 = tail ? f1 : f1 - nt;
     return w;
 }
 
@@ -522,7 +534,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const float *__restrict__ cs, const float *__restrict__ D,
                      bf16 *__restrict__ y, int *__restrict__ status, int64_t seqlen, int H,
                      int G, int Q, int64_t nchunks, int64_t nitems, int ncta1,
-                     const int2 *__restrict__ tab, const bf16 *__restrict__ z, int skip_cta)
+                     const int2 *__restrict__ tab, const bf16 *__restrict__ z, int tail_q,
+                     int skip_cta)
 {
     extern __shared__ uint8_t smem_raw[];
     ScanSmem &sm = *reinterpret_cast<ScanSmem *>(
@@ -530,7 +543,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     const int nT = Q / kTileRows;
-    const ScanWork wk = scan_work(nT, ncta1, nitems);
+    const ScanWork wk = scan_work(nT, ncta1, nitems, tail_q);
     const int T = wk.T;
     const int hpg = H / G;
     if (wk.f1 <= wk.f0) return;
@@ -1119,6 +1132,16 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
                       take_test_skip(kTestChunkState));
 }
 
+// The share (per 1024) of each second-tile run that a third group of CTAs takes (see scan_work).
+// Measured at the 2.7B-layer shape (80 heads per group: the C and B tiles and C B^T computed
+// once per 80 heads) and at b = 1, L = 65536, 32 heads in 8 groups (4 heads per group, where
+// the second tile's per-segment work, C B^T over 256 columns and its bf16 copy, weighs more).
+constexpr int kTailLongSeg = 64, kTailShortSeg = 128;
+static int scan_tail(int heads_per_group)
+{
+    return heads_per_group >= 16 ? kTailLongSeg : kTailShortSeg;
+}
+
 cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B, const bf16 *C,
                                  const float *cs, const bf16 *hin, const float *D, bf16 *y,
                                  int *status, int64_t batch, int64_t seqlen, int H, int G,
@@ -1147,9 +1170,10 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // Q = 256: half the SMs per tile class, with identical runs (see scan_work)
+    // Q = 256: half the SMs per tile class, with identical runs, and a third group of CTAs for
+    // the tails of the second-tile runs (see scan_work)
     const int per = (int)std::min<int64_t>(nT == 2 ? sms / 2 : sms, nitems);
-    const int grid = nT * per;
+    const int grid = nT == 2 ? 3 * per : per;
     const int ncta1 = nT == 2 ? per : 0;
     const size_t smem = sizeof(ScanSmem) + 1024;
     auto kern = z ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
@@ -1159,7 +1183,7 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     *why = "chunk scan (tcgen05) launch";
     return launch_pdl(kern, (unsigned)grid, kScanThreads, smem, st, mx, mb, mc, mx2, mz, hin,
                       dtc, cs, D, y, status, seqlen, H, G, Q, nchunks, nitems, ncta1, tab, z,
-                      take_test_skip(kTestChunkScan));
+                      scan_tail(H / G), take_test_skip(kTestChunkScan));
 }
 
 }  // namespace ssd
