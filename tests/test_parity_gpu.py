@@ -93,6 +93,13 @@ SMALL = [
     ("bf16_tc_groups_init", configs.SSD_LONG.with_(seqlen=1000, nheads=16, ngroups=4), 256),
     ("bf16_tc_groups_q128", configs.SSD_LONG.with_(seqlen=640, nheads=24, ngroups=8), 128),
     ("bf16_tc_many_heads", configs.SSD_2P7B.with_(batch=1, seqlen=384), 256),
+    # runs long enough that the last share of each second-tile run goes to the third group of
+    # CTAs (80 heads in one group: 1360 items, runs of 18-19, tails of 1; 4 groups of 10 heads:
+    # 720 items, runs of 9-10, tails of 1), with a 100-token last chunk whose second tiles are
+    # skipped, also inside tails, and tails that start inside a segment
+    ("bf16_tc_tails_many_heads", configs.SSD_2P7B.with_(batch=1, seqlen=4196), 256),
+    ("bf16_tc_tails_groups", configs.SSD_LONG.with_(batch=2, seqlen=2148, nheads=40,
+                                                     ngroups=4), 256),
 ]
 
 
