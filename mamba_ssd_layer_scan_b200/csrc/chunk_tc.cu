@@ -56,6 +56,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort);
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
+// The same with every lane observing the phase itself: for data that a TMA copy writes just
+// before the lanes read it (one lane's observation does not make the copy's bytes visible to
+// the others).  The result is the same for the whole warp.
+__device__ __forceinline__ bool warp_wait_each(uint64_t *bar, uint32_t parity,
+                                               volatile int *abort)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort) ? 1 : 0) != 0;
+}
 
 // z * sigmoid(z) = z (1 + tanh(z / 2)) / 2 with the hardware tanh approximation: one
 // special-function operation per element instead of an exponential and a reciprocal (relative
@@ -402,20 +410,25 @@ struct alignas(1024) ScanSmem {
     uint64_t bar_vec_full[kScanVecStages], bar_vec_free[kScanVecStages];
     uint64_t bar_slot_full[kRing], bar_slot_free[kRing];
     uint64_t bar_acc_full[2], bar_acc_free[2];
+    uint64_t bar_z_full, bar_z_free;   // the gate rows' stage (gated output only)
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort;
 };
+// Gated output: one head's gate rows (128 rows x 64 columns bf16, 128-byte swizzle) in a stage
+// after ScanSmem, loaded by TMA one P build ahead of the epilogue that reads them.
+constexpr int kZStageBytes = kTileRows * kRowBytes;
 // warp 0 TMA, warp 1 MMA and TMEM owner, warps 2-9 workers: two per TMEM
 // lane quarter, each owning a 32-column slice of every 64-column block; per head they build
 // their slice of P (mask) and then run the epilogue of the previous head for their slice of y
 constexpr int kScanWorkers = 256;
 constexpr int kScanThreads = 64 + kScanWorkers;   // 320 threads
+constexpr int kZWarp = kScanThreads / 32;          // gated output: warp 10 loads the gate rows
 constexpr uint32_t kScanTmemCols = 512;
 constexpr uint32_t kAccCol = 256;   // accumulator buffer a: Y_diag at 256 + 128 a, Y_A at +64
 
 static_assert(sizeof(StateSmem) + 1024 <= 232448, "chunk state smem exceeds 227 KB");
-static_assert(sizeof(ScanSmem) + 1024 <= 232448, "chunk scan smem exceeds 227 KB");
+static_assert(sizeof(ScanSmem) + 1024 + kZStageBytes <= 232448, "chunk scan smem exceeds 227 KB");
 
 // Stage s: with an off-diagonal block (48 KB stages) s in {0, 1} in S01; otherwise (32 KB
 // stages) s in 0..2 in S01 and 3..4 in the B tile's space.  h_in follows the x rows.
@@ -524,7 +537,7 @@ __device__ __forceinline__ Seg scan_segment(int64_t f, int64_t f1, int hpg, int 
 }
 
 template <bool kGate>   // kGate: the output is y * z * sigmoid(z)
-__global__ void __launch_bounds__(kScanThreads, 1)
+__global__ void __launch_bounds__(kGate ? kScanThreads + 32 : kScanThreads, 1)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_c,
@@ -540,6 +553,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
     extern __shared__ uint8_t smem_raw[];
     ScanSmem &sm = *reinterpret_cast<ScanSmem *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *zst = reinterpret_cast<uint8_t *>(&sm) + sizeof(ScanSmem);   // gate rows (kGate)
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     const int nT = Q / kTileRows;
@@ -578,6 +592,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             mbar_init(&sm.bar_acc_full[a], 1);
             mbar_init(&sm.bar_acc_free[a], kScanWorkers);
         }
+        mbar_init(&sm.bar_z_full, 1);
+        mbar_init(&sm.bar_z_free, kScanWorkers);
         mbar_init(&sm.bar_drain, 1);
         sm.abort = 0;
         fence_mbar_init();
@@ -601,6 +617,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             tma_prefetch_desc(&tm_b);
             tma_prefetch_desc(&tm_c);
             tma_prefetch_desc(&tm_x2);
+            if (kGate) tma_prefetch_desc(&tm_z);
             uint32_t J = 0;   // heads issued so far (all segments)
             int si = 0;       // segments whose tiles were loaded
             bool ok = true;
@@ -777,6 +794,27 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
             if (!ok) break;
             mma_commit(&sm.bar_seg_done);   // this segment's MMAs are done with C and R
             ++si;
+        }
+    } else if (kGate && warp == kZWarp) {
+        // ---------------- gate rows (lane 0 alone): each head's into the z stage, in the
+        // workers' order, as soon as the epilogue of the previous head has read the stage
+        if (lane == 0) {
+            uint32_t Jz = 0;
+            bool ok = true;
+            for (int64_t f = wk.f0; ok && f < wk.f1;) {
+                const Seg sg = segment(f);
+                f += sg.nh;
+                if (sg.skip) continue;
+                for (int j = 0; j < sg.nh; ++j, ++Jz) {
+                    if (Jz >= 1 && !mbar_wait(&sm.bar_z_free, (Jz - 1) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sm.bar_z_full, (uint32_t)kZStageBytes);
+                    tma_load_4d(zst, &tm_z, &sm.bar_z_full, 0, sg.h0 + j,
+                                (int)(sg.t0 + kTileRows * T), (int)sg.b);
+                }
+            }
         }
     } else if (warp >= 2) {
         // ---------------- workers, two per TMEM lane quarter.  Warp (qd, cq) owns rows
@@ -975,14 +1013,28 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     const uint32_t Jj = J0 + j - 1;
                     const int a = Jj & 1;
                     const int64_t yoff = yseg + (int64_t)(j - 1) * kP;
-                    // gated output (z given): y * z * sigmoid(z), z as packed bf16 pairs, its
-                    // four 16-byte pieces loaded before the accumulator wait
+                    // gated output (z given): y * z * sigmoid(z), z as packed bf16 pairs, this
+                    // thread's four 16-byte pieces of row t read from the z stage (swizzled)
+                    // before the accumulator wait
                     const bool gz = kGate && row_in;
                     uint4 zq[4];
+                    if (kGate) {
+                        if (!warp_wait_each(&sm.bar_z_full, Jj & 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint8_t *zrow = zst + t * kRowBytes;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        zq[q] = make_uint4(0u, 0u, 0u, 0u);
-                        if (gz) zq[q] = reinterpret_cast<const uint4 *>(z + yoff)[q];
+                        for (int q = 0; q < 4; ++q)
+                            zq[q] = *reinterpret_cast<const uint4 *>(
+                                zrow + (((4 * cq + q) ^ (t & 7)) << 4));
+                        // the next head's rows arrive by TMA (the async proxy): order these
+                        // reads before it
+                        fence_async_smem();
+                        mbar_arrive(&sm.bar_z_free);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) zq[q] = make_uint4(0u, 0u, 0u, 0u);
                     }
                     if (!warp_wait(&sm.bar_acc_full[a], (Jj >> 1) & 1, abort)) {
                         ok = false;
@@ -1000,7 +1052,10 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                     tmem_ld_wait();
                     tc_fence_before();
                     mbar_arrive(&sm.bar_acc_free[a]);
-                    mbar_arrive(&sm.bar_vec_free[vs]);   // done with this head's cs / dt
+                    // done with this head's cs / dt rows, which the producer's next bulk copy
+                    // (the async proxy) overwrites: order these reads before it
+                    fence_async_smem();
+                    mbar_arrive(&sm.bar_vec_free[vs]);
                     uint4 *yrow = reinterpret_cast<uint4 *>(y + yoff);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {   // 8 columns per 16-byte store
@@ -1175,13 +1230,14 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     const int per = (int)std::min<int64_t>(nT == 2 ? sms / 2 : sms, nitems);
     const int grid = nT == 2 ? 3 * per : per;
     const int ncta1 = nT == 2 ? per : 0;
-    const size_t smem = sizeof(ScanSmem) + 1024;
+    const size_t smem = sizeof(ScanSmem) + 1024 + (z ? kZStageBytes : 0);
     auto kern = z ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) { *why = "chunk scan: set smem attribute"; return e; }
     *why = "chunk scan (tcgen05) launch";
-    return launch_pdl(kern, (unsigned)grid, kScanThreads, smem, st, mx, mb, mc, mx2, mz, hin,
+    return launch_pdl(kern, (unsigned)grid, z ? kScanThreads + 32 : kScanThreads, smem, st, mx,
+                      mb, mc, mx2, mz, hin,
                       dtc, cs, D, y, status, seqlen, H, G, Q, nchunks, nitems, ncta1, tab, z,
                       scan_tail(H / G), take_test_skip(kTestChunkScan));
 }
