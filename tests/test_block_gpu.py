@@ -61,6 +61,11 @@ CASES = [
      True, False),
     ("tc_q256_prologue", configs.SSD_370M.with_(batch=1, seqlen=300, nheads=6), 256, False,
      True),
+    # runs long enough for the chunk scan's third group of CTAs (4 groups of 10 heads: the last
+    # 128/1024 of each second-tile run), a 100-token last chunk (its second tiles skipped, also
+    # by the warp that stages the gate rows), segments that end inside runs
+    ("tc_q256_both_tails_groups", configs.SSD_LONG.with_(batch=2, seqlen=2148, nheads=40,
+                                                          ngroups=4), 256, True, True),
     ("f32_simt_both", configs.SSD_F32_SMALL.with_(batch=2, seqlen=333, nheads=4, ngroups=2,
                                                   init_state=True), 64, True, True),
     ("bf16_simt_both", configs.SSD_370M.with_(batch=1, seqlen=300, nheads=4), 64, True, True),
