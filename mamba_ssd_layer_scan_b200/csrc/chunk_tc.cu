@@ -1190,10 +1190,13 @@ cudaError_t launch_chunk_state_tc(const bf16 *x, const float *dtc, const bf16 *B
 // The share (per 1024) of each second-tile run that a third group of CTAs takes (see scan_work).
 // Measured at the 2.7B-layer shape (80 heads per group: the C and B tiles and C B^T computed
 // once per 80 heads) and at b = 1, L = 65536, 32 heads in 8 groups (4 heads per group, where
-// the second tile's per-segment work, C B^T over 256 columns and its bf16 copy, weighs more).
+// the second tile's per-segment work, C B^T over 256 columns and its bf16 copy, weighs more);
+// the gated output (a longer epilogue in both tile classes) at the 2.7B-layer shape.
 constexpr int kTailLongSeg = 64, kTailShortSeg = 128;
-static int scan_tail(int heads_per_group)
+constexpr int kTailLongSegGated = 96;
+static int scan_tail(int heads_per_group, bool gated)
 {
+    if (gated && heads_per_group >= 16) return kTailLongSegGated;
     return heads_per_group >= 16 ? kTailLongSeg : kTailShortSeg;
 }
 
@@ -1239,7 +1242,7 @@ cudaError_t launch_chunk_scan_tc(const bf16 *x, const float *dtc, const bf16 *B,
     return launch_pdl(kern, (unsigned)grid, z ? kScanThreads + 32 : kScanThreads, smem, st, mx,
                       mb, mc, mx2, mz, hin,
                       dtc, cs, D, y, status, seqlen, H, G, Q, nchunks, nitems, ncta1, tab, z,
-                      scan_tail(H / G), take_test_skip(kTestChunkScan));
+                      scan_tail(H / G, z != nullptr), take_test_skip(kTestChunkScan));
 }
 
 }  // namespace ssd
