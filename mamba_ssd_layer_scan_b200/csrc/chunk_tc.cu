@@ -17,18 +17,25 @@
 //     head's MMAs run.
 //
 // chunk_scan_tc_kernel    y = (C B^T o L o dt + diag(D)) X  +  exp(cs) o (C h_in^T)
-//     One CTA per (batch, chunk, 128-row tile of the chunk, group, block of heads).  C B^T is
-//     computed once per CTA and shared by the heads (all heads of a group see the same B, C).
+//     One CTA per SM per 128-row tile class of the chunks, each taking an equal run of the flat
+//     (batch, chunk, group, head) list, and for 256-token chunks a third group of CTAs that takes
+//     the tails of the second-tile runs (see scan_work).  C B^T is computed once per segment (a
+//     run of one chunk's heads of a group, which see the same B and C) and shared by its heads.
 //     The diagonal 128 x 128 block of the masked matrix is built per head by 8 worker warps from
 //     TMEM and written back to TMEM as bf16 (a ring of 64-column blocks), where the MMAs read it
 //     as their A operand; for the second tile of a 256-token chunk the off-diagonal block is
-//     rank-1 in its decay and runs as a plain product with C B_off^T converted to bf16 once
-//     (see the section comment below).  The decay is factorised so that no element needs an
-//     exponential of its own.  The same worker warps then run the previous head's epilogue.
+//     rank-1 in its decay and runs as a plain product with C B_off^T converted to bf16 once per
+//     segment (see the section comment below).  The decay is factorised so that no element
+//     needs an exponential of its own.  The same worker warps then run the previous head's
+//     epilogue.
 //
 // Roles (warp-specialised; every wait is on an mbarrier and bounded, see sm100.cuh):
 //   state kernel: warp 0 TMA, warp 1 MMA, warp 2 TMEM owner, warps 4-11 scale, 12-15 epilogue
-//   scan  kernel: warp 0 TMA, warp 1 MMA and TMEM owner, warps 2-17 mask + epilogue
+//   scan  kernel: warp 0 TMA, warp 1 MMA and TMEM owner, warps 2-9 mask + epilogue, and for a
+//                 gated output warp 10, which stages each head's gate rows by TMA
+// A buffer that a TMA or bulk copy fills and that threads then read (or write) with plain
+// loads is released to the next copy only after those threads' fence.proxy.async: the copy
+// runs in the async proxy, which the generic proxy's release and acquire alone do not order.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
